@@ -1,0 +1,417 @@
+"""Pins of the fp64 oracle against things other than itself: figures the pages
+print, library conversions, closed forms, special cases and brute force."""
+import json
+import math
+import os
+
+import numpy as np
+import pytest
+import torch
+
+from oracle import lmoe_oracle as orc
+from latent_mixture_experts_softmax_b200 import synth
+
+GOLD = os.path.join(os.path.dirname(__file__), "golden")
+
+
+def _gold(name):
+    with open(os.path.join(GOLD, name)) as f:
+        return json.load(f)
+
+
+# ----------------------------------------------------------------------------
+# storage formats: byte totals the pages print
+# ----------------------------------------------------------------------------
+
+def test_record_and_build_sizes_match_pages():
+    g = _gold("page_figures.json")
+    H, E, G, F, NL = (g[k]["value"] for k in ("hidden", "experts_per_layer", "groups", "swiglu_width", "layers"))
+    L145, L120 = g["latent_145b"]["value"], g["latent_120b"]["value"]
+    assert 3 * L145 * F == g["expert_weights_latent1792"]["value"]
+    assert 3 * H * F == g["expert_weights_base"]["value"]
+    assert orc.expert_record_bytes(L145, F) == g["nvfp4_record_bytes_latent1792"]["value"]
+    # 145B NVFP4 build = experts + Q8_0 D and U (8 groups each), 48 layers
+    per_layer = E * orc.expert_record_bytes(L145, F) + G * (orc.du_matrix_bytes(orc.Q8_0, L145, H)
+                                                            + orc.du_matrix_bytes(orc.Q8_0, H, L145))
+    assert NL * per_layer == g["weights_145b_nvfp4_bytes"]["value"]
+    # the model page prints 47.79 GiB for the same byte total (47.785 GiB; it rounds up)
+    assert abs(NL * per_layer / 2 ** 30 - g["weights_145b_nvfp4_gib"]["value"]) < 0.01
+    # 120B NVFP4 build with Q4_0 D/U
+    per_layer = E * orc.expert_record_bytes(L120, F) + G * (orc.du_matrix_bytes(orc.Q4_0, L120, H)
+                                                            + orc.du_matrix_bytes(orc.Q4_0, H, L120))
+    assert round(NL * per_layer / 2 ** 30, 2) == g["weights_120b_nvfp4_gib"]["value"]
+    # with Q8_0 D/U the 120B would not match the printed build size
+    per_layer_q8 = E * orc.expert_record_bytes(L120, F) + 2 * G * orc.du_matrix_bytes(orc.Q8_0, L120, H)
+    assert round(NL * per_layer_q8 / 2 ** 30, 2) != g["weights_120b_nvfp4_gib"]["value"]
+    # D+U parameters per layer and routed parameters per layer
+    assert round(2 * H * L145 * G / 1e6, 1) == g["du_params_per_layer_145b"]["value"] / 1e6
+    assert round(NL * 2 * H * L145 * G / 1e9, 2) == g["du_params_48_layers_145b"]["value"] / 1e9
+    assert round(g["top_k"]["value"] * 3 * L145 * F / 1e6, 1) == g["routed_params_per_layer_145b"]["value"] / 1e6
+
+
+# ----------------------------------------------------------------------------
+# scalar formats against library conversions and the spec table
+# ----------------------------------------------------------------------------
+
+def test_e2m1_all_codes_match_spec_table():
+    want = np.array(_gold("e2m1_values.json")["values"])
+    got = orc.e2m1_to_f64(np.arange(16))
+    np.testing.assert_array_equal(got, want)
+    assert np.all(np.signbit(got[8:]))
+
+
+def test_e4m3fn_all_codes_match_torch():
+    codes = torch.arange(256, dtype=torch.int32).to(torch.uint8)
+    ref = codes.view(torch.float8_e4m3fn).to(torch.float64).numpy()
+    got = orc.e4m3fn_to_f64(np.arange(256))
+    nan = np.isnan(ref)
+    assert np.array_equal(nan, np.isnan(got))
+    assert nan.sum() == 2                               # 0x7F and 0xFF
+    np.testing.assert_array_equal(got[~nan], ref[~nan])
+    assert got[0x7E] == 448.0 and got[0x01] == 2.0 ** -9 and got[0x08] == 2.0 ** -6
+
+
+def test_fp16_all_codes_match_numpy():
+    codes = np.arange(65536, dtype=np.uint32).astype(np.uint16)
+    ref = codes.view(np.float16).astype(np.float64)
+    got = orc.fp16_to_f64(codes)
+    nan = np.isnan(ref)
+    assert np.array_equal(nan, np.isnan(got))
+    np.testing.assert_array_equal(got[~nan], ref[~nan])
+
+
+def test_bf16_matches_torch():
+    rng = np.random.default_rng(3)
+    codes = rng.integers(0, 65536, size=20000).astype(np.uint16)
+    codes = codes[((codes >> 7) & 0xFF) != 0xFF]        # finite values only
+    ref = torch.from_numpy(codes.view(np.int16)).view(torch.bfloat16).to(torch.float64).numpy()
+    np.testing.assert_array_equal(orc.bf16_to_f64(codes), ref)
+
+
+# ----------------------------------------------------------------------------
+# matrix formats: blobs packed element by element here, independently
+# ----------------------------------------------------------------------------
+
+def _fp16_bits(v):
+    return int(np.array([v], np.float16).view(np.uint16)[0])
+
+
+def test_decode_q8_0_hand_packed():
+    R, C = 3, 96
+    rng = np.random.default_rng(1)
+    q = rng.integers(-127, 128, size=(R, C))
+    d = rng.choice([0.5, 0.25, 0.015625, 3.0, 0.0078125], size=(R, C // 32))
+    blob = bytearray(R * C + R * C // 16)
+    want = np.zeros((R, C))
+    for r in range(R):
+        for c in range(C):
+            b, j = divmod(c, 32)
+            blob[(b * R + r) * 32 + j] = int(q[r, c]) & 0xFF
+            want[r, c] = q[r, c] * d[r, b]
+        for b in range(C // 32):
+            bits = _fp16_bits(d[r, b])
+            off = R * C + 2 * (b * R + r)
+            blob[off], blob[off + 1] = bits & 0xFF, bits >> 8
+    got = orc.decode_q8_0(np.frombuffer(bytes(blob), np.uint8), R, C)
+    np.testing.assert_array_equal(got, want)
+
+
+def test_decode_q4_0_hand_packed():
+    R, C = 2, 64
+    rng = np.random.default_rng(2)
+    q = rng.integers(0, 16, size=(R, C))
+    d = rng.choice([0.5, -0.25, 2.0, 0.125], size=(R, C // 32))
+    blob = bytearray(R * C // 2 + R * C // 16)
+    want = np.zeros((R, C))
+    for r in range(R):
+        for c in range(C):
+            b, j = divmod(c, 32)
+            pos = (b * R + r) * 16 + (j % 16)
+            if j < 16:
+                blob[pos] |= int(q[r, c])
+            else:
+                blob[pos] |= int(q[r, c]) << 4
+            want[r, c] = (q[r, c] - 8) * d[r, b]
+        for b in range(C // 32):
+            bits = _fp16_bits(d[r, b])
+            off = R * C // 2 + 2 * (b * R + r)
+            blob[off], blob[off + 1] = bits & 0xFF, bits >> 8
+    got = orc.decode_q4_0(np.frombuffer(bytes(blob), np.uint8), R, C)
+    np.testing.assert_array_equal(got, want)
+
+
+def test_decode_nvfp4_hand_packed():
+    R, C = 3, 128
+    rng = np.random.default_rng(4)
+    codes = rng.integers(0, 16, size=(R, C))
+    scodes = rng.integers(0x08, 0x7E, size=(R, C // 16))
+    ts = np.float32(0.0123)
+    table = _gold("e2m1_values.json")["values"]
+    s_val = torch.tensor(scodes.reshape(-1), dtype=torch.int32).to(torch.uint8).view(torch.float8_e4m3fn) \
+        .to(torch.float64).numpy().reshape(R, C // 16)
+    qb = bytearray(R * C // 2)
+    sb = bytearray(R * C // 16)
+    want = np.zeros((R, C))
+    for r in range(R):
+        for c in range(C):
+            pos = ((c // 32) * R + r) * 16 + (c % 32) // 2
+            qb[pos] |= int(codes[r, c]) << (4 * (c % 2))
+            want[r, c] = table[codes[r, c]] * s_val[r, c // 16] * float(ts)
+        for b in range(C // 16):
+            sb[((b // 4) * R + r) * 4 + b % 4] = int(scodes[r, b])
+    got = orc.decode_nvfp4(np.frombuffer(bytes(qb), np.uint8), np.frombuffer(bytes(sb), np.uint8), ts, R, C)
+    np.testing.assert_array_equal(got, want)
+
+
+def test_generator_round_trip_within_quantisation_error():
+    """Bytes from the generator decode to the matrix it was asked to encode,
+    within each format's rounding step."""
+    rng = np.random.default_rng(5)
+    w = rng.normal(0, 0.02, size=(64, 128))
+    for fmt, steps in ((orc.Q8_0, 127.0), (orc.Q4_0, 8.0)):
+        back = orc.decode_du(fmt, synth.qmatrix_encode(fmt, w), 64, 128)
+        amax = np.abs(w).reshape(64, 4, 32).max(axis=2)
+        bound = np.repeat(amax / steps, 32, axis=1) * 0.5 * 1.01 + 1e-12
+        if fmt == orc.Q4_0:
+            bound = np.repeat(amax / 8.0, 32, axis=1) * 1.01 + 1e-12   # asymmetric range: up to one step
+        assert np.all(np.abs(back - w) <= bound)
+    wg, wu, wd = rng.normal(0, 0.02, (64, 128)), rng.normal(0, 0.02, (64, 128)), rng.normal(0, 0.02, (128, 64))
+    rec = synth.expert_record_encode(wg, wu, wd)
+    g2, u2, d2 = orc.decode_expert(rec, 128, 64)
+    for a, b in ((wg, g2), (wu, u2), (wd, d2)):
+        # E2M1 keeps values to within 1/4 of a grid step relative to the block max (6 levels)
+        assert orc.rel_l2(b, a) < 0.15
+        assert np.corrcoef(a.ravel(), b.ravel())[0, 1] > 0.99
+
+
+# ----------------------------------------------------------------------------
+# router
+# ----------------------------------------------------------------------------
+
+def _brute_route(logits_row, K):
+    order = sorted(range(len(logits_row)), key=lambda e: (-logits_row[e], e))
+    sel = order[:K]
+    mx = max(logits_row[e] for e in sel)
+    ex = [math.exp(logits_row[e] - mx) for e in sel]
+    tot = sum(ex)
+    return sel, [v / tot for v in ex]
+
+
+def test_route_matches_full_sort_and_closed_form_weights():
+    rng = np.random.default_rng(7)
+    T, E, H, K = 6, 40, 32, 10
+    x = rng.normal(size=(T, H))
+    Wr = rng.normal(0, 0.3, size=(E, H))
+    b = rng.normal(0, 1.0, size=E)
+    idx, w, gap, logits = orc.route(x, Wr, b, K)
+    for t in range(T):
+        lt = [float(sum(x[t, i] * Wr[e, i] for i in range(H)) + b[e]) for e in range(E)]
+        sel, ws = _brute_route(lt, K)
+        assert list(idx[t]) == sel
+        np.testing.assert_allclose(w[t], ws, rtol=1e-12)
+        assert abs(w[t].sum() - 1.0) < 1e-12
+        srt = sorted(lt, reverse=True)
+        assert abs(gap[t] - (srt[K - 1] - srt[K])) < 1e-12
+
+
+def test_route_ties_lowest_index_and_bias_moves_selection():
+    E, K = 8, 3
+    x = np.zeros((1, 4))
+    Wr = np.zeros((E, 4))
+    b = np.array([0.0, 1.0, 1.0, 1.0, 1.0, 0.5, 0.0, 2.0])
+    idx, w, gap, _ = orc.route(x, Wr, b, K)
+    assert list(idx[0]) == [7, 1, 2]          # 2.0 first, then the lowest indices among the tie at 1.0
+    assert gap[0] == 0.0
+    e2, e1 = math.exp(2.0), math.exp(1.0)
+    np.testing.assert_allclose(w[0], [e2 / (e2 + 2 * e1), e1 / (e2 + 2 * e1), e1 / (e2 + 2 * e1)], rtol=1e-14)
+
+
+def test_route_permutation_invariance():
+    rng = np.random.default_rng(8)
+    T, E, H, K = 5, 32, 16, 4
+    x = rng.normal(size=(T, H))
+    Wr = rng.normal(size=(E, H))
+    perm = rng.permutation(E)
+    idx, w, _, _ = orc.route(x, Wr, None, K)
+    idx_p, w_p, _, _ = orc.route(x, Wr[perm], None, K)
+    for t in range(T):
+        assert sorted(perm[idx_p[t]]) == sorted(idx[t])
+        np.testing.assert_allclose(sorted(w_p[t]), sorted(w[t]), rtol=1e-12)
+
+
+# ----------------------------------------------------------------------------
+# block: brute force and special cases on tiny shapes
+# ----------------------------------------------------------------------------
+
+TINY = synth.LayerShape(hidden=128, latent=64, n_experts=12, top_k=3, n_groups=3, ffn=64, shared_ffn=64,
+                        du_fmt=synth.Q8_0, router_dtype="f32")
+
+
+def _tiny_layer(shape=TINY, seed=11, fmt=None):
+    wl = synth.Workload("t", shape if fmt is None else synth.replace(shape, du_fmt=fmt), T=5, seed=seed,
+                        groups="uniform", bias_sigma=0.5, weight_sigma=0.1)
+    return wl, synth.make_layer(wl), synth.make_x(wl)
+
+
+def _t(a):
+    return torch.from_numpy(np.asarray(a, np.float64))
+
+
+@pytest.mark.parametrize("fmt", [synth.Q8_0, synth.Q4_0])
+def test_block_equals_dense_masked_brute_force(fmt):
+    wl, layer, xb = _tiny_layer(fmt=fmt)
+    s = wl.shape
+    y, idx, w, _ = orc.latent_moe_forward(s, layer, xb)
+    # independent arrangement: every expert on every token, then a [T, E] mask of weights
+    x = _t(orc.bf16_to_f64(xb))
+    Wr = _t(layer["router_w"].astype(np.float64))
+    logits = x @ Wr.T + _t(layer["router_b"].astype(np.float64))
+    T = x.shape[0]
+    M = torch.zeros(T, s.n_experts, dtype=torch.float64)
+    for t in range(T):
+        sel, ws = _brute_route(logits[t].tolist(), s.top_k)
+        for e, v in zip(sel, ws):
+            M[t, e] = v
+    grp = layer["expert_group"].astype(np.int64)
+    D = [_t(orc.decode_du(fmt, orc.du_slice(layer["D"], fmt, g, s.latent, s.hidden), s.latent, s.hidden))
+         for g in range(s.n_groups)]
+    U = [_t(orc.decode_du(fmt, orc.du_slice(layer["U"], fmt, g, s.hidden, s.latent), s.hidden, s.latent))
+         for g in range(s.n_groups)]
+    out_all = torch.zeros(T, s.n_experts, s.latent, dtype=torch.float64)
+    for e in range(s.n_experts):
+        Wg, Wu, Wd = (_t(m) for m in orc.decode_expert(orc.expert_slice(layer["experts"], e, s.latent, s.ffn),
+                                                       s.latent, s.ffn))
+        h = x @ D[grp[e]].T                                              # [T, latent]
+        out_all[:, e] = (torch.nn.functional.silu(h @ Wg.T) * (h @ Wu.T)) @ Wd.T
+    Wsg, Wsu = _t(orc.bf16_to_f64(layer["shared_gate"])), _t(orc.bf16_to_f64(layer["shared_up"]))
+    Wsd = _t(orc.bf16_to_f64(layer["shared_down"]))
+    y_bf = (torch.nn.functional.silu(x @ Wsg.T) * (x @ Wsu.T)) @ Wsd.T
+    for g in range(s.n_groups):
+        mask_g = M * torch.tensor(grp == g, dtype=torch.float64)[None, :]
+        s_g = torch.einsum("te,tel->tl", mask_g, out_all)
+        y_bf = y_bf + s_g @ U[g].T
+    np.testing.assert_allclose(y, y_bf.numpy(), rtol=1e-10, atol=1e-12)
+    np.testing.assert_allclose(M.numpy()[np.arange(T)[:, None], idx], w, rtol=1e-12)
+
+
+def test_block_linearity_of_U():
+    """U_g applied to the per-group sum equals the sum of U_g applied to each weighted expert output."""
+    wl, layer, xb = _tiny_layer()
+    s = wl.shape
+    y, idx, w, _ = orc.latent_moe_forward(s, layer, xb)
+    W = orc.Weights(s, layer)
+    x = orc.bf16_to_f64(xb)
+    y2 = orc.shared_expert(x, W.Wsg, W.Wsu, W.Wsd)
+    for t in range(x.shape[0]):
+        for k in range(s.top_k):
+            e = int(idx[t, k])
+            g = int(W.group[e])
+            o = orc.expert_apply(*W.expert(e), W.D(g) @ x[t])
+            y2[t] += W.U(g) @ (w[t, k] * o)
+    np.testing.assert_allclose(y, y2, rtol=1e-10, atol=1e-13)
+
+
+def test_block_single_expert_single_group_is_textbook_chain():
+    s = synth.replace(TINY, n_experts=1, top_k=1, n_groups=1)
+    wl, layer, xb = _tiny_layer(shape=s)
+    y, idx, w, _ = orc.latent_moe_forward(s, layer, xb)
+    assert np.all(idx == 0) and np.all(w == 1.0)
+    x = _t(orc.bf16_to_f64(xb))
+    D = _t(orc.decode_q8_0(layer["D"], s.latent, s.hidden))
+    U = _t(orc.decode_q8_0(layer["U"], s.hidden, s.latent))
+    Wg, Wu, Wd = (_t(m) for m in orc.decode_expert(layer["experts"], s.latent, s.ffn))
+    Wsg, Wsu = _t(orc.bf16_to_f64(layer["shared_gate"])), _t(orc.bf16_to_f64(layer["shared_up"]))
+    Wsd = _t(orc.bf16_to_f64(layer["shared_down"]))
+    F = torch.nn.functional
+    h = x @ D.T
+    want = (F.silu(h @ Wg.T) * (h @ Wu.T)) @ Wd.T @ U.T + (F.silu(x @ Wsg.T) * (x @ Wsu.T)) @ Wsd.T
+    np.testing.assert_allclose(y, want.numpy(), rtol=1e-11, atol=1e-14)
+
+
+def test_block_zero_input_gives_zero():
+    wl, layer, xb = _tiny_layer()
+    y, _, _, _ = orc.latent_moe_forward(wl.shape, layer, np.zeros_like(xb))
+    assert np.all(y == 0.0)
+
+
+def test_block_zero_experts_gives_shared_only():
+    wl, layer, xb = _tiny_layer()
+    layer = dict(layer)
+    layer["experts"] = np.zeros_like(layer["experts"])
+    y, _, _, _ = orc.latent_moe_forward(wl.shape, layer, xb)
+    W = orc.Weights(wl.shape, layer)
+    x = orc.bf16_to_f64(xb)
+    np.testing.assert_allclose(y, orc.shared_expert(x, W.Wsg, W.Wsu, W.Wsd), rtol=1e-13, atol=0)
+
+
+def _identity_q8_0(n):
+    """Q8_0 identity matrix [n, n] packed by hand: q = 1 on the diagonal, d = 1.0."""
+    blob = bytearray(n * n + n * n // 16)
+    for r in range(n):
+        blob[((r // 32) * n + r) * 32 + r % 32] = 1
+        for b in range(n // 32):
+            off = n * n + 2 * (b * n + r)
+            blob[off], blob[off + 1] = 0x00, 0x3C                  # fp16 1.0
+    return np.frombuffer(bytes(blob), np.uint8)
+
+
+def test_block_identity_latent_reduces_to_standard_moe():
+    s = synth.replace(TINY, latent=TINY.hidden)
+    wl, layer, xb = _tiny_layer(shape=s)
+    layer = dict(layer)
+    I = _identity_q8_0(s.hidden)
+    layer["D"] = np.concatenate([I] * s.n_groups)
+    layer["U"] = np.concatenate([I] * s.n_groups)
+    y, idx, w, _ = orc.latent_moe_forward(s, layer, xb)
+    F = torch.nn.functional
+    x = _t(orc.bf16_to_f64(xb))
+    want = (F.silu(x @ _t(orc.bf16_to_f64(layer["shared_gate"])).T) * (x @ _t(orc.bf16_to_f64(layer["shared_up"])).T)) \
+        @ _t(orc.bf16_to_f64(layer["shared_down"])).T
+    for t in range(x.shape[0]):
+        for k in range(s.top_k):
+            Wg, Wu, Wd = (_t(m) for m in orc.decode_expert(orc.expert_slice(layer["experts"], int(idx[t, k]),
+                                                                             s.latent, s.ffn), s.latent, s.ffn))
+            want[t] += w[t, k] * (Wd @ (F.silu(Wg @ x[t]) * (Wu @ x[t])))
+    np.testing.assert_allclose(y, want.numpy(), rtol=1e-11, atol=1e-14)
+
+
+def test_block_injection_overrides_routing():
+    wl, layer, xb = _tiny_layer()
+    s = wl.shape
+    T = xb.shape[0]
+    inj_idx = np.tile(np.arange(s.top_k), (T, 1))
+    inj_w = np.full((T, s.top_k), 1.0 / s.top_k)
+    y, idx, w, _ = orc.latent_moe_forward(s, layer, xb, inject_idx=inj_idx, inject_w=inj_w)
+    assert np.array_equal(idx, inj_idx) and np.array_equal(w, inj_w)
+    y_ref, _, _, _ = orc.latent_moe_forward(s, layer, xb)
+    assert orc.rel_l2(y, y_ref) > 1e-3
+
+
+def test_residual_adds():
+    wl, layer, xb = _tiny_layer()
+    r = synth.bf16_normal(123, 1.0, xb.shape)
+    y0, _, _, _ = orc.latent_moe_forward(wl.shape, layer, xb)
+    y1, _, _, _ = orc.latent_moe_forward(wl.shape, layer, xb, residual_bits=r)
+    np.testing.assert_allclose(y1 - y0, orc.bf16_to_f64(r), rtol=0, atol=1e-12)
+
+
+def test_rmsnorm_closed_form():
+    v = np.array([[3.0, -4.0], [0.0, 0.0]])
+    g = np.array([2.0, 0.5])
+    out = orc.rmsnorm(v, g, 0.0 + 1e-30)
+    r = math.sqrt((9 + 16) / 2)
+    np.testing.assert_allclose(out[0], [2 * 3 / r, 0.5 * -4 / r], rtol=1e-15)
+    assert np.all(out[1] == 0)
+    np.testing.assert_allclose(orc.rmsnorm(np.array([[1.0, 1.0]]), np.ones(2), 1.0), [[1 / math.sqrt(2)] * 2])
+
+
+def test_stack_layer_is_residual_plus_block_of_norm():
+    wl, layer, xb = _tiny_layer()
+    s = wl.shape
+    gamma = np.linspace(0.5, 1.5, s.hidden)
+    y, _, _, _ = orc.stack_layer_forward(s, layer, xb, gamma, 1e-6)
+    x = orc.bf16_to_f64(xb)
+    ms = (x * x).mean(axis=1, keepdims=True)
+    xn = gamma[None, :] * x / np.sqrt(ms + 1e-6)
+    blk, _, _, _ = orc.latent_moe_forward(s, layer, None, x_f64=xn)
+    np.testing.assert_allclose(y, x + blk, rtol=1e-13, atol=1e-14)
