@@ -1,0 +1,382 @@
+#!/usr/bin/env python
+"""Throughput of the latent mixture-of-experts FFN block on B200.
+
+One step = one pass of the whole block (router, bucketing, D_g, experts,
+U_g + shared + combine) over one batch of T tokens of one layer.  The default
+workload is the Edge0-120B-shaped layer at T=4 (an MTP verify window).
+
+Timing: W untimed warm-up steps, then K steps between CUDA events on the
+launching stream, barrier + synchronize on both sides, max over ranks.  Each
+step runs on one of R device copies of the layer's weights (R x the bytes a
+step touches > 2 x the 126 MB L2), so no step finds its weights in L2, and on
+its own seeded token batch.  Multi-GPU: every rank is an independent replica
+(the block shards by tokens and needs no collective): weak scaling.
+
+`--impl reference` times the fp64 CPU oracle on the host cores instead (a
+bounded sample of the same workload per step)."""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "latent-MoE layer tokens/s (T=4 decode, T=4096 prefill); % HBM/FP4 roofline"
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=500)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default="edge0_120b_decode")
+    ap.add_argument("--T", type=int, default=None, help="override the workload's token count")
+    ap.add_argument("--copies", type=int, default=0, help="weight copies to rotate (0: enough to defeat L2)")
+    ap.add_argument("--cpu-seconds", type=float, default=15.0, help="CPU-oracle sample budget")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    return ap.parse_args()
+
+
+# ----------------------------------------------------------------------------
+# clocks during the timed region (NVML, read only)
+# ----------------------------------------------------------------------------
+
+class ClockSampler:
+    REASONS = {0x0000000000000002: "applications_clocks_setting", 0x0000000000000004: "sw_power_cap",
+               0x0000000000000008: "hw_slowdown", 0x0000000000000020: "sw_thermal_slowdown",
+               0x0000000000000040: "hw_thermal_slowdown", 0x0000000000000080: "hw_power_brake_slowdown",
+               0x0000000000000100: "display_clock_setting"}
+
+    def __init__(self, device_index: int, period_s: float = 0.001):
+        self.period = period_s
+        self.samples = []
+        self.ok = False
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self.nv = pynvml
+            self.h = pynvml.nvmlDeviceGetHandleByIndex(device_index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
+            self.ok = True
+        except Exception as e:  # no NVML: report that
+            self.err = str(e)
+        self._stop = threading.Event()
+
+    def _run(self):
+        while not self._stop.is_set():
+            try:
+                mhz = self.nv.nvmlDeviceGetClockInfo(self.h, self.nv.NVML_CLOCK_SM)
+                rs = self.nv.nvmlDeviceGetCurrentClocksEventReasons(self.h)
+                self.samples.append((mhz, rs))
+            except Exception:
+                pass
+            time.sleep(self.period)
+
+    def __enter__(self):
+        if self.ok:
+            self.t = threading.Thread(target=self._run, daemon=True)
+            self.t.start()
+        return self
+
+    def __exit__(self, *a):
+        if self.ok:
+            self._stop.set()
+            self.t.join()
+
+    def summary(self):
+        if not self.ok:
+            return {"error": getattr(self, "err", "nvml unavailable")}
+        if not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": [], "samples": 0}
+        reasons = set()
+        for _, rs in self.samples:
+            for bit, name in self.REASONS.items():
+                if rs & bit:
+                    reasons.add(name)
+        return {"sm_mhz": statistics.median(m for m, _ in self.samples), "sm_max_mhz": self.max_mhz,
+                "reasons": sorted(reasons), "samples": len(self.samples)}
+
+
+# ----------------------------------------------------------------------------
+# algorithmic bytes of one step (from the routing actually taken)
+# ----------------------------------------------------------------------------
+
+def step_bytes(shape, idx: np.ndarray, groups: np.ndarray, T: int) -> dict:
+    """Bytes each kernel must move at least once: weights it reads plus its
+    activations in and out."""
+    H, L, E, K, G, F, Fs = (shape.hidden, shape.latent, shape.n_experts, shape.top_k, shape.n_groups, shape.ffn,
+                            shape.shared_ffn)
+    du = L * H // 32 * (34 if shape.du_fmt == 8 else 18)
+    rec_gu = 2 * (F * L // 2 + F * L // 16)
+    rec_d = F * L // 2 + F * L // 16
+    rw = E * H * (2 if shape.router_dtype == "bf16" else 4)
+    hit = {int(groups[e]) for e in idx.reshape(-1)}
+    n_distinct = len(set(idx.reshape(-1).tolist()))
+    b = {
+        "k_router_shared": rw + 2 * Fs * H * 2 + T * H * 2,
+        "k_dproj": len(hit) * du + T * H * 2,
+        "k_expert_gateup": n_distinct * rec_gu,
+        "k_expert_down": n_distinct * rec_d,
+        "k_uproj": len(hit) * du + H * Fs * 2 + 2 * T * H * 2,
+    }
+    b["n_distinct"] = n_distinct
+    b["n_groups_hit"] = len(hit)
+    return b
+
+
+STAGES = ["k_router_shared", "k_dproj", "k_expert_gateup", "k_expert_down", "k_uproj"]
+
+
+def workload_desc(wl, T):
+    s = wl.shape
+    fmt = "Q8_0" if s.du_fmt == 8 else "Q4_0"
+    bias = "none" if wl.bias_sigma is None else f"N(0,{wl.bias_sigma:g})"
+    return (f"{wl.name}: T={T}, hidden {s.hidden}, latent {s.latent}, {s.n_experts} experts top-{s.top_k}, "
+            f"{s.n_groups} {fmt} D/U groups, NVFP4 experts ffn {s.ffn}, bf16 shared ffn {s.shared_ffn}, "
+            f"{s.router_dtype} router, bias {bias}, expert_group {wl.groups}, x bf16 N(0,1), weights N(0,0.02)")
+
+
+# ----------------------------------------------------------------------------
+# the oracle as a CPU baseline / reference arm
+# ----------------------------------------------------------------------------
+
+def cpu_oracle_rate(wl, layer, T, budget_s, max_steps=None, tokens_per_step=None):
+    """Runs the fp64 oracle on successive token samples of the workload until
+    the budget (or max_steps) is used; returns (tokens/s, tokens, seconds,
+    threads, steps, decode_seconds)."""
+    from oracle import lmoe_oracle as orc
+    from latent_mixture_experts_softmax_b200 import synth
+    try:
+        from threadpoolctl import threadpool_info
+        threads = max([i.get("num_threads", 1) for i in threadpool_info()] + [1])
+    except Exception:
+        threads = os.cpu_count() or 1
+    t0 = time.perf_counter()
+    W = orc.Weights(wl.shape, layer, max_cached_experts=128)
+    for g in range(wl.shape.n_groups):
+        W.D(g), W.U(g)
+    t_decode = time.perf_counter() - t0
+    ntok = tokens_per_step or T
+    done = 0
+    steps = 0
+    t0 = time.perf_counter()
+    while True:
+        xb = synth.make_x(wl, T=T, draw=10_000 + steps)[:ntok]
+        orc.latent_moe_forward(wl.shape, layer, xb, weights=W)
+        done += ntok
+        steps += 1
+        el = time.perf_counter() - t0
+        if (max_steps is not None and steps >= max_steps) or (max_steps is None and el >= budget_s):
+            break
+    return done / el, done, el, threads, steps, t_decode
+
+
+def run_reference(args, wl, T, rank, world):
+    """The reference arm: the oracle timed on the host cores (rank 0 only)."""
+    if rank != 0:
+        return
+    from latent_mixture_experts_softmax_b200 import synth
+    layer = synth.make_layer(wl)
+    # a bounded sample per step: one token of the batch per step, so the whole
+    # run stays within a few minutes
+    _, _, _, _, _, _ = cpu_oracle_rate(wl, layer, T, 0, max_steps=args.warmup, tokens_per_step=1)
+    rate, done, el, threads, steps, t_dec = cpu_oracle_rate(wl, layer, T, 0, max_steps=args.steps,
+                                                            tokens_per_step=1)
+    line = {"impl": "reference", "metric": METRIC, "value": rate, "unit": "tokens/s", "n_gpus": world,
+            "steps": steps, "warmup": args.warmup, "ms_per_step": 1000 * el / steps, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": workload_desc(wl, T), "T": T},
+            "cpu_baseline": {"value": rate, "unit": "tokens/s", "cores": threads, "kind": "oracle",
+                             "sample": f"one token of the T={T} batch per step, {steps} steps, fresh seeded x per "
+                                       f"step; weight decode ({t_dec:.1f} s) outside the timed steps"},
+            "e2e": {"value": rate, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+# ----------------------------------------------------------------------------
+# our arm
+# ----------------------------------------------------------------------------
+
+def main():
+    args = parse()
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+
+    from latent_mixture_experts_softmax_b200 import synth
+    wl = synth.WORKLOADS[args.workload]
+    T = args.T or wl.T
+
+    if args.impl == "reference":
+        run_reference(args, wl, T, rank, world)
+        return
+
+    import torch
+    import torch.distributed as dist
+    from latent_mixture_experts_softmax_b200 import binding as B
+    from latent_mixture_experts_softmax_b200 import build
+    from latent_mixture_experts_softmax_b200.layer import DeviceLayer, to_device
+
+    torch.cuda.set_device(local)
+    dev_name = torch.device("cuda", local)
+    if world > 1:
+        from datetime import timedelta
+        dist.init_process_group("nccl", timeout=timedelta(seconds=120), device_id=dev_name)
+    build.build_all()
+
+    layer = synth.make_layer(wl)
+    base = DeviceLayer(wl.shape, layer, device=dev_name)
+    # bytes a step can touch: every weight except the experts not routed
+    s = wl.shape
+    per_step_max = base.weight_bytes() - base.experts.numel() + 2 * T * s.top_k * \
+        B.lmoe_expert_record_bytes(base.cfg)
+    R = args.copies or max(2, int(np.ceil(2 * 126e6 / per_step_max)) + 1)
+    devs = [base]
+    for _ in range(R - 1):
+        d = DeviceLayer.__new__(DeviceLayer)
+        d.__dict__.update(base.__dict__)
+        for name in ("router_w", "router_b", "expert_group", "D", "U", "experts", "shared_gate", "shared_up",
+                     "shared_down"):
+            t = getattr(base, name)
+            setattr(d, name, None if t is None else t.clone())
+        d.shared = B.make_shared(d.shared_gate, d.shared_up, d.shared_down)
+        devs.append(d)
+    ws = base.workspace(T)
+    K, W = args.steps, args.warmup
+    n_steps = K + W
+    xs_host = [synth.make_x(wl, T=T, draw=rank * 100_003 + i) for i in range(n_steps)]
+    xs = [to_device(x, dev_name) for x in xs_host]
+    ys = [torch.empty_like(x) for x in xs]
+    idx_all = torch.empty((n_steps, T, s.top_k), dtype=torch.int32, device=dev_name)
+    w_all = torch.empty((n_steps, T, s.top_k), dtype=torch.float32, device=dev_name)
+    stream = torch.cuda.current_stream()
+
+    def step(i):
+        d = devs[i % R]
+        B.lmoe_forward_ex(d.cfg, xs[i], d.router_w, d.router_b, d.expert_group, d.D, d.U, d.experts, d.shared,
+                          None, None, None, idx_all[i], w_all[i], ys[i], T, ws, stream)
+
+    for i in range(W):
+        step(i)
+    torch.cuda.synchronize()
+
+    # per-kernel events inside the timed region
+    n_ev = len(STAGES) + 1
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(n_ev)] for _ in range(K)]
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    with ClockSampler(local) as clk:
+        start.record()
+        for k in range(K):
+            B.lmoe_profile_stage_events(evs[k])
+            step(W + k)
+        end.record()
+        torch.cuda.synchronize()
+    B.lmoe_profile_stage_events([])
+    if world > 1:
+        dist.barrier()
+    ms = start.elapsed_time(end)
+    ms_t = torch.tensor([ms], dtype=torch.float64, device=dev_name)
+    if world > 1:
+        dist.all_reduce(ms_t, op=dist.ReduceOp.MAX)
+    ms_max = float(ms_t.item())
+    status = B.lmoe_last_device_status(ws)
+
+    # per-kernel times and algorithmic bytes
+    stage_ms = np.zeros(len(STAGES))
+    for k in range(K):
+        for j in range(len(STAGES)):
+            stage_ms[j] += evs[k][j].elapsed_time(evs[k][j + 1])
+    idx_np = idx_all.cpu().numpy()
+    groups = layer["expert_group"]
+    tot = {st: 0 for st in STAGES}
+    nd = []
+    for k in range(K):
+        b = step_bytes(s, idx_np[W + k], groups, T)
+        nd.append(b["n_distinct"])
+        for st in STAGES:
+            tot[st] += b[st]
+    step_alg_bytes = sum(tot.values()) / K
+    peaks = {}
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            peaks = json.load(f)
+        hbm_peak, peak_src = float(peaks["hbm_gbs"]), "measured"
+    except Exception:
+        hbm_peak, peak_src = 6650.0, "fallback"
+    dom = int(np.argmax(stage_ms))
+    dom_name = STAGES[dom]
+    dom_avg_s = stage_ms[dom] / K / 1e3
+    dom_gbs = tot[dom_name] / K / dom_avg_s / 1e9
+
+    # e2e through the host-buffer entry point (copies inside the timed region)
+    x_pin = [torch.from_numpy(x.view(np.int16)).pin_memory() for x in xs_host[:K]]
+    y_pin = torch.empty((T, s.hidden), dtype=torch.int16).pin_memory()
+    for i in range(min(W, K)):
+        d = devs[i % R]
+        B.lmoe_forward_host(d.cfg, x_pin[i], d.router_w, d.router_b, d.expert_group, d.D, d.U, d.experts, d.shared,
+                            y_pin, T, ws, stream)
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for i in range(K):
+        d = devs[i % R]
+        B.lmoe_forward_host(d.cfg, x_pin[i], d.router_w, d.router_b, d.expert_group, d.D, d.U, d.experts, d.shared,
+                            y_pin, T, ws, stream)
+    e1.record()
+    torch.cuda.synchronize()
+    e2e_ms = torch.tensor([e0.elapsed_time(e1)], dtype=torch.float64, device=dev_name)
+    if world > 1:
+        dist.all_reduce(e2e_ms, op=dist.ReduceOp.MAX)
+    e2e_rate = world * T * K / (float(e2e_ms.item()) / 1e3)
+
+    value = world * T * K / (ms_max / 1e3)
+    line = {
+        "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": K, "warmup": W,
+        "ms_per_step": ms_max / K, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "f32", "data": "synthetic",
+        "config": {"workload": workload_desc(wl, T), "T": T, "parallelism": f"replicas x{world}",
+                   "l2": f"inputs larger than L2: {R} weight copies rotated, "
+                         f"{R * per_step_max / 1e6:.0f} MB touched between reuses",
+                   "weights": "NVFP4 experts, Q8_0/Q4_0 D/U, bf16 router and shared expert; "
+                              "bf16 activations in and out, fp32 accumulation"},
+        "roofline": {"bound": "hbm", "kernel": dom_name, "achieved": dom_gbs, "peak": hbm_peak, "unit": "GB/s",
+                     "frac": dom_gbs / hbm_peak, "peak_source": peak_src, "traffic": None},
+        "layer_gbs": step_alg_bytes / (ms_max / K / 1e3) / 1e9,
+        "layer_frac_hbm": step_alg_bytes / (ms_max / K / 1e3) / 1e9 / hbm_peak,
+        "algorithmic_bytes_per_step": step_alg_bytes,
+        "distinct_experts_per_step": float(np.mean(nd)),
+        "kernels": {st: {"ms_avg": stage_ms[j] / K, "share": stage_ms[j] / stage_ms.sum(),
+                         "gbs": tot[st] / K / (stage_ms[j] / K / 1e3) / 1e9} for j, st in enumerate(STAGES)},
+        "e2e": {"value": e2e_rate, "unit": "tokens/s", "h2d_bytes_per_step": T * s.hidden * 2,
+                "d2h_bytes_per_step": T * s.hidden * 2},
+        "gpu_launches": len(STAGES) * K,
+        "clocks": clk.summary(),
+        "device_status": status,
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        rate, done, el, threads, steps, t_dec = cpu_oracle_rate(wl, layer, T, args.cpu_seconds)
+        line["cpu_baseline"] = {"value": rate, "unit": "tokens/s", "cores": threads, "kind": "oracle",
+                                "sample": f"{steps} batches of T={T} fresh seeded tokens ({done} tokens, {el:.1f} s);"
+                                          f" weight decode ({t_dec:.1f} s) excluded"}
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,192 @@
+/*
+ * lmoe.h -- C ABI of the latent mixture-of-experts FFN block on NVIDIA B200
+ * (sm_100a).
+ *
+ * The block (teardown article "Edge0-145B: a Qwen MoE with its experts
+ * squeezed, and a 51B table left on the SSD", section "A latent in front of
+ * the experts", layer equation; Edge0 145B / 120B model page, "Model
+ * profile" and the architecture tables), per token x (width `hidden`):
+ *
+ *   router   l = W_r x + b; softmax over all experts; keep the top_k by
+ *            (logit desc, index asc); w_k = p_k / sum of the kept p
+ *   groups   every expert e carries a label group[e] in [0, n_groups)
+ *   D        h_g = D_g x                 for each group g hit by the token
+ *   experts  o_k = W_down (silu(W_gate h) * (W_up h)),  h = h_{group[e_k]}
+ *   U        y = sum_g U_g (sum_{k: group[e_k] = g} w_k o_k)
+ *   shared   y += S_down (silu(S_gate x) * (S_up x))    (full width)
+ *   residual y += residual                               (optional)
+ *
+ * Conventions for every call:
+ *   - Pointers named *_host are host memory; every other pointer is device
+ *     memory on the current device, owned by the caller.  The library never
+ *     allocates device memory; scratch comes from the caller's workspace
+ *     (size from lmoe_workspace_bytes, 256-byte aligned).
+ *   - `stream` is a cudaStream_t (NULL = legacy default stream).  Calls are
+ *     asynchronous on it.  A negative return means nothing was launched.
+ *   - All device pointers must be 16-byte aligned.
+ *   - A workspace may be used by one call at a time (calls on one stream
+ *     serialise; calls on different streams need different workspaces).
+ *   - Faults the kernels detect (an expert_group label >= n_groups, a
+ *     routed index out of range) are recorded in the workspace's status
+ *     word, read with lmoe_last_device_status.
+ *
+ * Storage layouts (all little-endian):
+ *   x, y, residual       bf16 [T][hidden]
+ *   router_w             fp32 or bf16 (cfg.router_dtype) [n_experts][hidden]
+ *   router_b             fp32 [n_experts] or NULL
+ *   expert_group         uint8 [n_experts]
+ *   shared.gate, .up     bf16 [shared_ffn][hidden]
+ *   shared.down          bf16 [hidden][shared_ffn]
+ *   D                    n_groups matrices [latent rows][hidden cols], then
+ *   U                    n_groups matrices [hidden rows][latent cols], each
+ *     Q8_0:  int8 q [cols/32][rows][32], then fp16 d [cols/32][rows];
+ *            weight(r, c) = d * q                       (34 bytes per 32)
+ *     Q4_0:  uint8 q [cols/32][rows][16] (byte j: low nibble element j,
+ *            high nibble element j+16), then fp16 d [cols/32][rows];
+ *            weight = d * (q - 8)                      (18 bytes per 32)
+ *   experts              n_experts records of lmoe_expert_record_bytes():
+ *     gate.q [latent/32][ffn][16] | up.q [latent/32][ffn][16] |
+ *     down.q [ffn/32][latent][16] | gate.s [latent/64][ffn][4] |
+ *     up.s [latent/64][ffn][4] | down.s [ffn/64][latent][4] |
+ *     fp32 ts_gate, ts_up, ts_down, uint32 0
+ *     q bytes hold E2M1 codes, element 2i in the low nibble of byte i;
+ *     s bytes are E4M3 scales, byte j of a word scales elements 16j..16j+15
+ *     of its 64-wide column group; weight = e2m1 * e4m3 * ts.
+ *     (1,935,376 bytes at latent 1792, ffn 640: the record size printed in
+ *     the teardown article, section "What is 4-bit".)
+ *
+ * Shape limits (lmoe_cfg_check): hidden, latent multiples of 128; ffn,
+ * shared_ffn multiples of 64; 1 <= top_k <= 16 and top_k <= n_experts <=
+ * 4096; 1 <= n_groups <= 64.
+ */
+#ifndef LMOE_H
+#define LMOE_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define LMOE_API __attribute__((visibility("default")))
+#else
+#define LMOE_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    LMOE_OK = 0,
+    LMOE_ERR_ARG = -1,           /* null pointer, bad size, misaligned pointer */
+    LMOE_ERR_UNSUPPORTED = -2,   /* shape or format outside the limits above */
+    LMOE_ERR_CUDA = -3,          /* a CUDA runtime call failed */
+    LMOE_ERR_WORKSPACE = -4,     /* workspace smaller than lmoe_workspace_bytes */
+    LMOE_ERR_TIMEOUT = -5,       /* a bounded device wait gave up */
+    LMOE_ERR_DEVICE_CHECK = -6   /* a kernel found an invalid input (see header) */
+} lmoe_status;
+
+typedef enum { LMOE_Q8_0 = 8, LMOE_Q4_0 = 4 } lmoe_du_fmt;   /* D/U block formats */
+typedef enum { LMOE_F32 = 0, LMOE_BF16 = 1 } lmoe_dtype;     /* router weight type */
+
+typedef struct {
+    int hidden;        /* model width (2560 for Edge0 145B / 120B) */
+    int latent;        /* latent width l (1792 / 1280) */
+    int n_experts;     /* routed experts per layer (512) */
+    int top_k;         /* experts per token (10) */
+    int n_groups;      /* D/U pairs per layer (8) */
+    int ffn;           /* expert SwiGLU width (640) */
+    int shared_ffn;    /* shared expert SwiGLU width (640) */
+    int du_fmt;        /* lmoe_du_fmt */
+    int router_dtype;  /* lmoe_dtype */
+} lmoe_cfg;
+
+typedef struct {
+    const void* gate;  /* bf16 [shared_ffn][hidden] */
+    const void* up;    /* bf16 [shared_ffn][hidden] */
+    const void* down;  /* bf16 [hidden][shared_ffn] */
+} lmoe_shared;
+
+/* One layer of a stack; all device pointers. */
+typedef struct {
+    const void* router_w;
+    const float* router_b;        /* may be NULL */
+    const uint8_t* expert_group;
+    const void* D;
+    const void* U;
+    const void* experts;
+    lmoe_shared shared;
+    const void* norm_gamma;       /* bf16 [hidden]: RMSNorm weight before the block */
+} lmoe_layer;
+
+/* LMOE_OK if the shape is supported, else LMOE_ERR_UNSUPPORTED / LMOE_ERR_ARG. */
+LMOE_API int lmoe_cfg_check(const lmoe_cfg* cfg);
+
+/* Bytes of one expert record, of one D (or U) blob holding all n_groups
+ * matrices, and of the workspace needed for up to T_max tokens.  0 if the
+ * configuration is unsupported. */
+LMOE_API size_t lmoe_expert_record_bytes(const lmoe_cfg* cfg);
+LMOE_API size_t lmoe_du_bytes(const lmoe_cfg* cfg);
+LMOE_API size_t lmoe_workspace_bytes(const lmoe_cfg* cfg, int T_max);
+
+/* Router only: logits, softmax, top_k and renormalised weights.
+ * topk_idx int32 [T][top_k] and topk_w fp32 [T][top_k], in selection order
+ * (logit descending, index ascending on ties). */
+LMOE_API int lmoe_route(const lmoe_cfg* cfg, const void* x, const void* router_w, const float* router_b, int T,
+               int32_t* topk_idx, float* topk_w, void* ws, size_t ws_bytes, void* stream);
+
+/* The block: y [T][hidden] bf16 = block(x). */
+LMOE_API int lmoe_forward(const lmoe_cfg* cfg, const void* x, const void* router_w, const uint8_t* expert_group,
+                 const void* D, const void* U, const void* experts, const lmoe_shared* shared,
+                 void* y, int T, void* ws, size_t ws_bytes, void* stream);
+
+/* The block with every option:
+ *   router_b     per-expert bias added to the logits, or NULL
+ *   residual     bf16 [T][hidden] added to y, or NULL; y overlaps neither x
+ *                nor residual
+ *   inject_idx / inject_w   when both non-NULL, the routing is taken from
+ *                them ([T][top_k]) instead of the router (the router still
+ *                runs; used where two logits are too close to compare)
+ *   out_idx / out_w         when non-NULL, receive the routing used. */
+LMOE_API int lmoe_forward_ex(const lmoe_cfg* cfg, const void* x, const void* router_w, const float* router_b,
+                    const uint8_t* expert_group, const void* D, const void* U, const void* experts,
+                    const lmoe_shared* shared, const void* residual,
+                    const int32_t* inject_idx, const float* inject_w, int32_t* out_idx, float* out_w,
+                    void* y, int T, void* ws, size_t ws_bytes, void* stream);
+
+/* As lmoe_forward, with x_host and y_host in host memory (page-locked for
+ * the copies to overlap): copies x in, runs the block, copies y out, all on
+ * `stream`.  The call returns once y_host is written. */
+LMOE_API int lmoe_forward_host(const lmoe_cfg* cfg, const void* x_host, const void* router_w, const float* router_b,
+                      const uint8_t* expert_group, const void* D, const void* U, const void* experts,
+                      const lmoe_shared* shared, void* y_host, int T, void* ws, size_t ws_bytes, void* stream);
+
+/* n_layers pre-norm residual layers: x <- x + block_l(RMSNorm_l(x)), the
+ * residual stream kept in bf16; RMSNorm(v) = gamma * v / sqrt(mean(v^2) + eps).
+ * x and y are bf16 [T][hidden] and may not alias.  `layers` is a host array. */
+LMOE_API int lmoe_stack_forward(const lmoe_cfg* cfg, int n_layers, const lmoe_layer* layers, const void* x, void* y,
+                       int T, float rms_eps, void* ws, size_t ws_bytes, void* stream);
+
+/* Waits for `stream`, then returns and clears the workspace status word
+ * (LMOE_OK, or LMOE_ERR_DEVICE_CHECK / LMOE_ERR_TIMEOUT set by a kernel). */
+LMOE_API int lmoe_last_device_status(void* ws, size_t ws_bytes, void* stream);
+
+/* Static text for a status code. */
+LMOE_API const char* lmoe_status_str(int status);
+
+/* Diagnostics: decode one stored matrix to fp32 [rows][cols] on the device
+ * with the same decoders the kernels use.  fmt: LMOE_Q8_0, LMOE_Q4_0, or 1
+ * for an NVFP4 matrix (q then s as in an expert record, scaled by ts). */
+LMOE_API int lmoe_debug_decode(int fmt, const void* blob, int rows, int cols, float ts, float* out, void* stream);
+
+/* Profiling: while n > 0, every later forward call records events[0] before
+ * its first kernel, events[i] before kernel i and one more event after its
+ * last kernel, on the call's stream, until the n events are used (each call
+ * starts again at events[0]).  `events` holds cudaEvent_t handles owned by
+ * the caller; n = 0 turns recording off.  At most 16 events. */
+LMOE_API int lmoe_profile_stage_events(void* const* events, int n);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* LMOE_H */

@@ -1,0 +1,307 @@
+// C ABI of the latent-MoE block: argument checks, workspace carve-up and
+// dispatch to the kernels.  Declarations and conventions: include/lmoe.h.
+
+#include <cstring>
+
+#include "lmoe_internal.cuh"
+
+using namespace lmoe;
+
+namespace {
+
+bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+int check_cfg(const lmoe_cfg* c) {
+    if (c == nullptr) return LMOE_ERR_ARG;
+    if (c->hidden <= 0 || c->latent <= 0 || c->n_experts <= 0 || c->top_k <= 0 || c->n_groups <= 0 ||
+        c->ffn <= 0 || c->shared_ffn <= 0)
+        return LMOE_ERR_ARG;
+    if (c->hidden % 128 || c->latent % 128 || c->ffn % 64 || c->shared_ffn % 64) return LMOE_ERR_UNSUPPORTED;
+    if (c->hidden > 960 * 32) return LMOE_ERR_UNSUPPORTED;
+    if (c->top_k > kMaxTopK || c->top_k > c->n_experts || c->n_experts > kMaxExpertsTopk) return LMOE_ERR_UNSUPPORTED;
+    if (c->n_groups > kMaxGroups || c->n_groups > 255) return LMOE_ERR_UNSUPPORTED;
+    if (c->du_fmt != LMOE_Q8_0 && c->du_fmt != LMOE_Q4_0) return LMOE_ERR_UNSUPPORTED;
+    if (c->router_dtype != LMOE_F32 && c->router_dtype != LMOE_BF16) return LMOE_ERR_UNSUPPORTED;
+    return LMOE_OK;
+}
+
+size_t du_matrix_bytes(const lmoe_cfg& c) {
+    return (size_t)c.latent * c.hidden / 32 * (c.du_fmt == LMOE_Q8_0 ? 34 : 18);
+}
+
+size_t record_bytes(const lmoe_cfg& c) {
+    const size_t lf = (size_t)c.latent * c.ffn;
+    return 3 * lf / 2 + 3 * lf / 16 + 16;
+}
+
+struct WsLayout {
+    size_t ctrl, idx, w, logits, n_unique, uexp, ucnt, uoff, slot_pair, pair_slot, ghit, tghit;
+    size_t h, zsh, z, o, ypart, xio, yio, xa, xb;
+    size_t total;
+};
+
+WsLayout ws_layout(const lmoe_cfg& c, int T) {
+    WsLayout L{};
+    size_t off = 0;
+    auto take = [&](size_t bytes) {
+        const size_t o = off;
+        off += (bytes + 255) & ~(size_t)255;
+        return o;
+    };
+    const size_t TK = (size_t)T * c.top_k;
+    L.ctrl = take(sizeof(Ctrl));
+    L.idx = take(TK * 4);
+    L.w = take(TK * 4);
+    L.logits = take((size_t)T * c.n_experts * 4);
+    L.n_unique = take(4);
+    L.uexp = take(TK * 4);
+    L.ucnt = take(TK * 4);
+    L.uoff = take(TK * 4);
+    L.slot_pair = take(TK * 4);
+    L.pair_slot = take(TK * 4);
+    L.ghit = take((size_t)c.n_groups * 4);
+    L.tghit = take((size_t)T * c.n_groups);
+    L.h = take((size_t)T * c.n_groups * c.latent * 4);
+    L.zsh = take((size_t)T * c.shared_ffn * 4);
+    L.z = take(TK * c.ffn * 4);
+    L.o = take(TK * c.latent * 4);
+    L.ypart = take((size_t)(c.n_groups + 1) * T * c.hidden * 4);
+    L.xio = take((size_t)T * c.hidden * 2);
+    L.yio = take((size_t)T * c.hidden * 2);
+    L.xa = take((size_t)T * c.hidden * 2);
+    L.xb = take((size_t)T * c.hidden * 2);
+    L.total = off;
+    return L;
+}
+
+FwdParams base_params(const lmoe_cfg& c, int T, void* ws, const WsLayout& L) {
+    FwdParams p;
+    std::memset(&p, 0, sizeof(p));
+    p.H = c.hidden; p.L = c.latent; p.E = c.n_experts; p.K = c.top_k; p.G = c.n_groups;
+    p.F = c.ffn; p.Fs = c.shared_ffn; p.du_fmt = c.du_fmt; p.router_bf16 = c.router_dtype == LMOE_BF16;
+    p.T = T;
+    char* b = static_cast<char*>(ws);
+    p.ctrl = reinterpret_cast<Ctrl*>(b + L.ctrl);
+    p.r.idx = reinterpret_cast<int32_t*>(b + L.idx);
+    p.r.w = reinterpret_cast<float*>(b + L.w);
+    p.r.logits = reinterpret_cast<float*>(b + L.logits);
+    p.r.n_unique = reinterpret_cast<int32_t*>(b + L.n_unique);
+    p.r.uexp = reinterpret_cast<int32_t*>(b + L.uexp);
+    p.r.ucnt = reinterpret_cast<int32_t*>(b + L.ucnt);
+    p.r.uoff = reinterpret_cast<int32_t*>(b + L.uoff);
+    p.r.slot_pair = reinterpret_cast<int32_t*>(b + L.slot_pair);
+    p.r.pair_slot = reinterpret_cast<int32_t*>(b + L.pair_slot);
+    p.r.ghit = reinterpret_cast<int32_t*>(b + L.ghit);
+    p.r.tghit = reinterpret_cast<uint8_t*>(b + L.tghit);
+    p.h = reinterpret_cast<float*>(b + L.h);
+    p.zsh = reinterpret_cast<float*>(b + L.zsh);
+    p.z = reinterpret_cast<float*>(b + L.z);
+    p.o = reinterpret_cast<float*>(b + L.o);
+    p.ypart = reinterpret_cast<float*>(b + L.ypart);
+    p.du_bytes_D = du_matrix_bytes(c);
+    p.du_bytes_U = du_matrix_bytes(c);
+    p.rec_bytes = record_bytes(c);
+    p.eps = 0.f;
+    return p;
+}
+
+int cuda_status(cudaError_t e) { return e == cudaSuccess ? LMOE_OK : LMOE_ERR_CUDA; }
+
+// Reset the CTA tickets (the status word is kept until it is read).
+cudaError_t reset_tickets(void* ws, cudaStream_t st) {
+    return cudaMemsetAsync(static_cast<char*>(ws) + offsetof(Ctrl, route_ticket), 0,
+                           sizeof(Ctrl) - offsetof(Ctrl, route_ticket), st);
+}
+
+int check_block_ptrs(const void* x, const void* router_w, const uint8_t* expert_group, const void* D, const void* U,
+                     const void* experts, const lmoe_shared* shared, const void* y) {
+    if (!x || !router_w || !expert_group || !D || !U || !experts || !shared || !y) return LMOE_ERR_ARG;
+    if (!shared->gate || !shared->up || !shared->down) return LMOE_ERR_ARG;
+    const void* p16[] = {x, router_w, D, U, experts, shared->gate, shared->up, shared->down, y};
+    for (const void* q : p16)
+        if (!aligned(q, 16)) return LMOE_ERR_ARG;
+    return LMOE_OK;
+}
+
+int forward_impl(const lmoe_cfg* cfg, const void* x, const void* router_w, const float* router_b,
+                 const uint8_t* expert_group, const void* D, const void* U, const void* experts,
+                 const lmoe_shared* shared, const void* residual, const int32_t* inject_idx, const float* inject_w,
+                 int32_t* out_idx, float* out_w, void* y, int T, void* ws, size_t ws_bytes, cudaStream_t st,
+                 const void* gamma, float eps) {
+    int s = check_cfg(cfg);
+    if (s != LMOE_OK) return s;
+    if (T < 0) return LMOE_ERR_ARG;
+    s = check_block_ptrs(x, router_w, expert_group, D, U, experts, shared, y);
+    if (s != LMOE_OK) return s;
+    if ((router_b && !aligned(router_b, 4)) || (residual && !aligned(residual, 16)) ||
+        (inject_idx && !aligned(inject_idx, 4)) || (inject_w && !aligned(inject_w, 4)) ||
+        (out_idx && !aligned(out_idx, 4)) || (out_w && !aligned(out_w, 4)) || (gamma && !aligned(gamma, 16)))
+        return LMOE_ERR_ARG;
+    if ((inject_idx == nullptr) != (inject_w == nullptr)) return LMOE_ERR_ARG;
+    if (T == 0) return LMOE_OK;
+    if (!ws || !aligned(ws, 256)) return LMOE_ERR_ARG;
+    const WsLayout L = ws_layout(*cfg, T);
+    if (L.total > ws_bytes) return LMOE_ERR_WORKSPACE;
+    FwdParams p = base_params(*cfg, T, ws, L);
+    p.x = static_cast<const uint16_t*>(x);
+    p.router_w = router_w;
+    p.router_b = router_b;
+    p.group = expert_group;
+    p.D = static_cast<const uint8_t*>(D);
+    p.U = static_cast<const uint8_t*>(U);
+    p.experts = static_cast<const uint8_t*>(experts);
+    p.sg = static_cast<const uint16_t*>(shared->gate);
+    p.su = static_cast<const uint16_t*>(shared->up);
+    p.sd = static_cast<const uint16_t*>(shared->down);
+    p.residual = static_cast<const uint16_t*>(residual);
+    p.gamma = static_cast<const uint16_t*>(gamma);
+    p.eps = eps;
+    p.inject_idx = inject_idx;
+    p.inject_w = inject_w;
+    p.out_idx = out_idx;
+    p.out_w = out_w;
+    p.y = static_cast<uint16_t*>(y);
+    cudaError_t e = reset_tickets(ws, st);
+    if (e != cudaSuccess) return LMOE_ERR_CUDA;
+    return cuda_status(run_gemv_path(p, st, false));
+}
+
+}  // namespace
+
+extern "C" {
+
+int lmoe_cfg_check(const lmoe_cfg* cfg) { return check_cfg(cfg); }
+
+size_t lmoe_expert_record_bytes(const lmoe_cfg* cfg) { return check_cfg(cfg) == LMOE_OK ? record_bytes(*cfg) : 0; }
+
+size_t lmoe_du_bytes(const lmoe_cfg* cfg) {
+    return check_cfg(cfg) == LMOE_OK ? du_matrix_bytes(*cfg) * cfg->n_groups : 0;
+}
+
+size_t lmoe_workspace_bytes(const lmoe_cfg* cfg, int T_max) {
+    if (check_cfg(cfg) != LMOE_OK || T_max < 0) return 0;
+    return ws_layout(*cfg, T_max < 1 ? 1 : T_max).total;
+}
+
+int lmoe_route(const lmoe_cfg* cfg, const void* x, const void* router_w, const float* router_b, int T,
+               int32_t* topk_idx, float* topk_w, void* ws, size_t ws_bytes, void* stream) {
+    int s = check_cfg(cfg);
+    if (s != LMOE_OK) return s;
+    if (T < 0 || !x || !router_w || !topk_idx || !topk_w) return LMOE_ERR_ARG;
+    if (!aligned(x, 16) || !aligned(router_w, 16) || !aligned(topk_idx, 4) || !aligned(topk_w, 4) ||
+        (router_b && !aligned(router_b, 4)))
+        return LMOE_ERR_ARG;
+    if (T == 0) return LMOE_OK;
+    if (!ws || !aligned(ws, 256)) return LMOE_ERR_ARG;
+    const WsLayout L = ws_layout(*cfg, T);
+    if (L.total > ws_bytes) return LMOE_ERR_WORKSPACE;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    FwdParams p = base_params(*cfg, T, ws, L);
+    p.x = static_cast<const uint16_t*>(x);
+    p.router_w = router_w;
+    p.router_b = router_b;
+    p.out_idx = topk_idx;
+    p.out_w = topk_w;
+    cudaError_t e = reset_tickets(ws, st);
+    if (e != cudaSuccess) return LMOE_ERR_CUDA;
+    return cuda_status(run_gemv_path(p, st, true));
+}
+
+int lmoe_forward(const lmoe_cfg* cfg, const void* x, const void* router_w, const uint8_t* expert_group,
+                 const void* D, const void* U, const void* experts, const lmoe_shared* shared, void* y, int T,
+                 void* ws, size_t ws_bytes, void* stream) {
+    return forward_impl(cfg, x, router_w, nullptr, expert_group, D, U, experts, shared, nullptr, nullptr, nullptr,
+                        nullptr, nullptr, y, T, ws, ws_bytes, static_cast<cudaStream_t>(stream), nullptr, 0.f);
+}
+
+int lmoe_forward_ex(const lmoe_cfg* cfg, const void* x, const void* router_w, const float* router_b,
+                    const uint8_t* expert_group, const void* D, const void* U, const void* experts,
+                    const lmoe_shared* shared, const void* residual, const int32_t* inject_idx, const float* inject_w,
+                    int32_t* out_idx, float* out_w, void* y, int T, void* ws, size_t ws_bytes, void* stream) {
+    return forward_impl(cfg, x, router_w, router_b, expert_group, D, U, experts, shared, residual, inject_idx,
+                        inject_w, out_idx, out_w, y, T, ws, ws_bytes, static_cast<cudaStream_t>(stream), nullptr,
+                        0.f);
+}
+
+int lmoe_forward_host(const lmoe_cfg* cfg, const void* x_host, const void* router_w, const float* router_b,
+                      const uint8_t* expert_group, const void* D, const void* U, const void* experts,
+                      const lmoe_shared* shared, void* y_host, int T, void* ws, size_t ws_bytes, void* stream) {
+    int s = check_cfg(cfg);
+    if (s != LMOE_OK) return s;
+    if (!x_host || !y_host || T < 0) return LMOE_ERR_ARG;
+    if (T == 0) return LMOE_OK;
+    if (!ws || !aligned(ws, 256)) return LMOE_ERR_ARG;
+    const WsLayout L = ws_layout(*cfg, T);
+    if (L.total > ws_bytes) return LMOE_ERR_WORKSPACE;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    char* b = static_cast<char*>(ws);
+    const size_t bytes = (size_t)T * cfg->hidden * 2;
+    if (cudaMemcpyAsync(b + L.xio, x_host, bytes, cudaMemcpyHostToDevice, st) != cudaSuccess) return LMOE_ERR_CUDA;
+    s = forward_impl(cfg, b + L.xio, router_w, router_b, expert_group, D, U, experts, shared, nullptr, nullptr,
+                     nullptr, nullptr, nullptr, b + L.yio, T, ws, ws_bytes, st, nullptr, 0.f);
+    if (s != LMOE_OK) return s;
+    if (cudaMemcpyAsync(y_host, b + L.yio, bytes, cudaMemcpyDeviceToHost, st) != cudaSuccess) return LMOE_ERR_CUDA;
+    return cuda_status(cudaStreamSynchronize(st));
+}
+
+int lmoe_stack_forward(const lmoe_cfg* cfg, int n_layers, const lmoe_layer* layers, const void* x, void* y, int T,
+                       float rms_eps, void* ws, size_t ws_bytes, void* stream) {
+    int s = check_cfg(cfg);
+    if (s != LMOE_OK) return s;
+    if (n_layers < 1 || !layers || !x || !y || T < 0 || !(rms_eps >= 0.f)) return LMOE_ERR_ARG;
+    for (int l = 0; l < n_layers; ++l)
+        if (!layers[l].norm_gamma) return LMOE_ERR_ARG;
+    if (T == 0) return LMOE_OK;
+    if (!ws || !aligned(ws, 256)) return LMOE_ERR_ARG;
+    const WsLayout L = ws_layout(*cfg, T);
+    if (L.total > ws_bytes) return LMOE_ERR_WORKSPACE;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    char* b = static_cast<char*>(ws);
+    const void* cur = x;
+    for (int l = 0; l < n_layers; ++l) {
+        void* out = l == n_layers - 1 ? y : (void*)(b + ((l & 1) ? L.xb : L.xa));
+        const lmoe_layer& ly = layers[l];
+        s = forward_impl(cfg, cur, ly.router_w, ly.router_b, ly.expert_group, ly.D, ly.U, ly.experts, &ly.shared,
+                         cur, nullptr, nullptr, nullptr, nullptr, out, T, ws, ws_bytes, st, ly.norm_gamma, rms_eps);
+        if (s != LMOE_OK) return s;
+        cur = out;
+    }
+    return LMOE_OK;
+}
+
+int lmoe_last_device_status(void* ws, size_t ws_bytes, void* stream) {
+    if (!ws || ws_bytes < sizeof(Ctrl)) return LMOE_ERR_ARG;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    int host = 0;
+    if (cudaStreamSynchronize(st) != cudaSuccess) return LMOE_ERR_CUDA;
+    if (cudaMemcpy(&host, ws, sizeof(int), cudaMemcpyDeviceToHost) != cudaSuccess) return LMOE_ERR_CUDA;
+    if (cudaMemset(ws, 0, sizeof(int)) != cudaSuccess) return LMOE_ERR_CUDA;
+    return host;
+}
+
+const char* lmoe_status_str(int s) {
+    switch (s) {
+        case LMOE_OK: return "ok";
+        case LMOE_ERR_ARG: return "invalid argument (null, size or alignment)";
+        case LMOE_ERR_UNSUPPORTED: return "unsupported shape or format";
+        case LMOE_ERR_CUDA: return "CUDA runtime error";
+        case LMOE_ERR_WORKSPACE: return "workspace too small";
+        case LMOE_ERR_TIMEOUT: return "a bounded device wait gave up";
+        case LMOE_ERR_DEVICE_CHECK: return "a kernel found an invalid input";
+        default: return "unknown status";
+    }
+}
+
+int lmoe_profile_stage_events(void* const* events, int n) {
+    if (n < 0 || n > kMaxStageEvents || (n > 0 && !events)) return LMOE_ERR_ARG;
+    set_stage_events(events, n);
+    return LMOE_OK;
+}
+
+int lmoe_debug_decode(int fmt, const void* blob, int rows, int cols, float ts, float* out, void* stream) {
+    if (!blob || !out || rows <= 0 || cols <= 0 || cols % 64 || !aligned(blob, 16)) return LMOE_ERR_ARG;
+    if (fmt != LMOE_Q8_0 && fmt != LMOE_Q4_0 && fmt != 1) return LMOE_ERR_UNSUPPORTED;
+    return cuda_status(run_debug_decode(fmt, blob, rows, cols, ts, out, static_cast<cudaStream_t>(stream)));
+}
+
+}  // extern "C"

@@ -1,0 +1,74 @@
+// Internal interface between the C-ABI layer and the kernels.
+#pragma once
+
+#include "lmoe_common.cuh"
+
+namespace lmoe {
+
+constexpr int kMaxExpertsTopk = 1024;   // experts a router warp holds in registers (32 per lane)
+
+// Streaming loads of weights that are read once: no L1 allocation.
+__device__ __forceinline__ uint4 ldg_stream(const uint4* p) {
+    uint4 v;
+    asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0, %1, %2, %3}, [%4];"
+                 : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+                 : "l"(p));
+    return v;
+}
+__device__ __forceinline__ float4 ldg_stream(const float4* p) {
+    float4 v;
+    asm volatile("ld.global.nc.L1::no_allocate.v4.f32 {%0, %1, %2, %3}, [%4];"
+                 : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w)
+                 : "l"(p));
+    return v;
+}
+
+__device__ __forceinline__ uint16_t f32_to_bf16_bits(float v) {
+    return __bfloat16_as_ushort(__float2bfloat16_rn(v));
+}
+
+struct FwdParams {
+    // shape
+    int H, L, E, K, G, F, Fs, du_fmt, router_bf16;
+    int T;
+    // inputs
+    const uint16_t* x;
+    const void* router_w;
+    const float* router_b;
+    const uint8_t* group;
+    const uint8_t* D;
+    const uint8_t* U;
+    const uint8_t* experts;
+    const uint16_t* sg;
+    const uint16_t* su;
+    const uint16_t* sd;
+    const uint16_t* residual;
+    const uint16_t* gamma;   // RMSNorm of x before the block (stack), nullptr: none
+    float eps;
+    const int32_t* inject_idx;
+    const float* inject_w;
+    // outputs
+    uint16_t* y;
+    int32_t* out_idx;
+    float* out_w;
+    // workspace
+    Ctrl* ctrl;
+    Routing r;
+    float* h;       // [T][G][L]
+    float* zsh;     // [T][Fs]
+    float* z;       // [T*K][F]   per slot
+    float* o;       // [T*K][L]   per slot
+    float* ypart;   // [G+1][T][H]
+    size_t du_bytes_D, du_bytes_U, rec_bytes;
+    // launch shape of the router kernel
+    int n_router_ctas, router_rows_per_warp;
+    bool do_shared, do_buckets;
+};
+
+constexpr int kMaxStageEvents = 16;
+
+cudaError_t run_gemv_path(const FwdParams& p, cudaStream_t st, bool route_only);
+void set_stage_events(void* const* events, int n);
+cudaError_t run_debug_decode(int fmt, const void* blob, int R, int C, float ts, float* out, cudaStream_t st);
+
+}  // namespace lmoe

@@ -1,0 +1,207 @@
+"""CUDA path (through the C ABI) against the fp64 oracle on seeded inputs."""
+import numpy as np
+import pytest
+import torch
+
+from latent_mixture_experts_softmax_b200 import binding as B
+from latent_mixture_experts_softmax_b200 import build, synth
+from latent_mixture_experts_softmax_b200.layer import DeviceLayer, to_device
+from oracle import lmoe_oracle as orc
+
+from parity import GAP, check_block, check_routing, small_workload, assert_close, bf16_bits_to_f64
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _built():
+    build.build_all()
+    assert torch.cuda.is_available()
+
+
+# ----------------------------------------------------------------------------
+# storage-format decoders of the kernels, bit for bit
+# ----------------------------------------------------------------------------
+
+@pytest.mark.parametrize("fmt", [synth.Q8_0, synth.Q4_0])
+def test_decode_du_matches_oracle(fmt):
+    R, C = 96, 256
+    blob = synth.qmatrix(fmt, 77, 0.03, R, C)
+    out = torch.empty(R, C, dtype=torch.float32, device="cuda")
+    B.lmoe_debug_decode(fmt, to_device(blob, "cuda"), R, C, 1.0, out)
+    ref = orc.decode_du(fmt, blob, R, C)
+    np.testing.assert_array_equal(out.cpu().numpy().astype(np.float64), ref)
+
+
+def test_decode_nvfp4_matches_oracle():
+    L_, F_ = 128, 64
+    rec = synth.experts_normal(5, 0.02, 1, L_, F_)
+    nq, ns = L_ * F_ // 2, L_ * F_ // 16
+    ts = np.frombuffer(rec[3 * nq + 3 * ns: 3 * nq + 3 * ns + 12].tobytes(), np.float32)
+    for m, (R, C) in enumerate([(F_, L_), (F_, L_), (L_, F_)]):
+        blob = np.concatenate([rec[m * nq:(m + 1) * nq], rec[3 * nq + m * ns:3 * nq + (m + 1) * ns]])
+        out = torch.empty(R, C, dtype=torch.float32, device="cuda")
+        B.lmoe_debug_decode(B.LMOE_NVFP4_DEBUG, to_device(blob, "cuda"), R, C, float(ts[m]), out)
+        ref = orc.decode_nvfp4(blob[:nq], blob[nq:], ts[m], R, C)
+        np.testing.assert_allclose(out.cpu().numpy().astype(np.float64), ref, rtol=2.0 ** -23, atol=0)
+
+
+# ----------------------------------------------------------------------------
+# router
+# ----------------------------------------------------------------------------
+
+@pytest.mark.parametrize("name", ["tiny", "edge0_120b_decode", "edge0_145b_decode"])
+def test_route_matches_oracle(name):
+    wl = synth.WORKLOADS[name]
+    layer = synth.make_layer(wl)
+    dev = DeviceLayer(wl.shape, layer)
+    n_ok = 0
+    for draw in range(4):
+        xb = synth.make_x(wl, T=16, draw=draw)
+        ws = dev.workspace(16)
+        idx, w = dev.route(to_device(xb, "cuda"), ws)
+        W = orc.Weights(wl.shape, layer)
+        idx_r, w_r, gap, _ = orc.route(orc.bf16_to_f64(xb), W.Wr, W.b, wl.shape.top_k)
+        n_ok += check_routing(idx.cpu().numpy(), w.cpu().numpy(), idx_r, w_r, gap)
+        # selection order is logit-descending: the weights must be non-increasing
+        assert np.all(np.diff(w.cpu().numpy(), axis=1) <= 1e-7)
+    assert n_ok >= 48
+
+
+def test_route_ties_pick_lowest_index():
+    s = synth.replace(synth.WORKLOADS["tiny"].shape, n_experts=64, top_k=4)
+    wl = synth.Workload("ties", s, T=3, bias_sigma=None)
+    layer = synth.make_layer(wl)
+    layer["router_w"] = np.zeros_like(layer["router_w"])
+    layer["router_b"] = np.zeros(64, np.float32)
+    layer["router_b"][[5, 9, 17, 33, 40]] = 1.0          # five-way tie for four places
+    dev = DeviceLayer(s, layer)
+    idx, w = dev.route(to_device(synth.make_x(wl), "cuda"), dev.workspace(3))
+    assert idx.cpu().tolist() == [[5, 9, 17, 33]] * 3
+    np.testing.assert_allclose(w.cpu().numpy(), 0.25, rtol=1e-6)
+
+
+# ----------------------------------------------------------------------------
+# the block
+# ----------------------------------------------------------------------------
+
+@pytest.mark.parametrize("T", [1, 2, 3, 4, 5, 8, 13, 37])
+def test_block_small_shape_ragged_tokens(T):
+    wl = small_workload(T)
+    layer = synth.make_layer(wl)
+    check_block(wl.shape, layer, synth.make_x(wl), what=f"T={T}")
+
+
+@pytest.mark.parametrize("fmt", [synth.Q8_0, synth.Q4_0])
+def test_block_small_shape_formats_with_residual(fmt):
+    wl = small_workload(11, du_fmt=fmt, router_dtype="f32")
+    layer = synth.make_layer(wl)
+    res = synth.bf16_normal(synth.key(1, 0, "residual"), 1.0, (11, wl.shape.hidden))
+    check_block(wl.shape, layer, synth.make_x(wl), residual_bits=res, what=f"fmt={fmt}")
+
+
+def test_block_one_hot_expert_and_unhit_groups():
+    """Every token routes to the same experts (one expert holds all T tokens,
+    more than one pass of the token chunk) and most groups are never hit."""
+    wl = small_workload(21)
+    layer = synth.make_layer(wl)
+    layer["router_b"] = np.full(wl.shape.n_experts, -50.0, np.float32)
+    layer["router_b"][:wl.shape.top_k] = 50.0 + np.arange(wl.shape.top_k, dtype=np.float32)
+    layer["expert_group"][:wl.shape.top_k] = 1
+    out = check_block(wl.shape, layer, synth.make_x(wl), what="one-hot")
+    assert np.all(np.sort(out["idx_gpu"], axis=1) == np.arange(wl.shape.top_k))
+
+
+def test_block_tiny_config():
+    wl = synth.WORKLOADS["tiny"]
+    check_block(wl.shape, synth.make_layer(wl), synth.make_x(wl), what="tiny")
+
+
+@pytest.mark.parametrize("name", ["edge0_120b_decode", "edge0_145b_decode"])
+def test_block_decode_configs(name):
+    wl = synth.WORKLOADS[name]
+    layer = synth.make_layer(wl)
+    dev = DeviceLayer(wl.shape, layer)
+    W = orc.Weights(wl.shape, layer, max_cached_experts=16)
+    for draw in range(3):
+        check_block(wl.shape, layer, synth.make_x(wl, draw=draw), dev=dev, weights=W, what=f"{name} draw {draw}")
+
+
+def test_block_prefill_config_sampled_tokens():
+    """T=4096 through the same launch sequence the benchmark times; the oracle
+    recomputes a sample of rows (the block is per token)."""
+    wl = synth.WORKLOADS["edge0_145b_prefill"]
+    layer = synth.make_layer(wl)
+    xb = synth.make_x(wl)
+    rows = np.array([0, 1, 777, 2048, 3001, 4095])
+    check_block(wl.shape, layer, xb, tokens=rows, what="prefill sample")
+
+
+def test_forward_host_matches_device_call():
+    wl = small_workload(6)
+    layer = synth.make_layer(wl)
+    dev = DeviceLayer(wl.shape, layer)
+    xb = synth.make_x(wl)
+    ws = dev.workspace(6)
+    y_dev = dev.forward(to_device(xb, "cuda"), ws)
+    x_h = torch.from_numpy(xb.view(np.int16)).pin_memory()
+    y_h = torch.empty_like(x_h).pin_memory()
+    B.lmoe_forward_host(dev.cfg, x_h, dev.router_w, dev.router_b, dev.expert_group, dev.D, dev.U, dev.experts,
+                        dev.shared, y_h, 6, ws)
+    assert torch.equal(y_h, y_dev.cpu())
+
+
+def test_forward_is_deterministic():
+    wl = small_workload(37)
+    layer = synth.make_layer(wl)
+    dev = DeviceLayer(wl.shape, layer)
+    x = to_device(synth.make_x(wl), "cuda")
+    ws = dev.workspace(37)
+    a = dev.forward(x, ws).clone()
+    b = dev.forward(x, ws).clone()
+    assert torch.equal(a, b)
+
+
+def test_empty_batch_is_noop():
+    wl = small_workload(4)
+    dev = DeviceLayer(wl.shape, synth.make_layer(wl))
+    y = torch.full((0, wl.shape.hidden), 7, dtype=torch.int16, device="cuda")
+    x = torch.zeros((0, wl.shape.hidden), dtype=torch.int16, device="cuda")
+    ws = dev.workspace(1)
+    # zero-size tensors may have a null data pointer: pass a valid one
+    B.lmoe_forward(dev.cfg, ws, dev.router_w, dev.expert_group, dev.D, dev.U, dev.experts, dev.shared, ws, 0, ws)
+
+
+def test_bad_group_label_is_reported_not_faulted():
+    wl = small_workload(4)
+    layer = synth.make_layer(wl)
+    layer["expert_group"][:] = 200                      # >= n_groups
+    dev = DeviceLayer(wl.shape, layer)
+    ws = dev.workspace(4)
+    dev.forward(to_device(synth.make_x(wl), "cuda"), ws)
+    assert B.lmoe_last_device_status(ws) == B.LMOE_ERR_DEVICE_CHECK
+    assert B.lmoe_last_device_status(ws) == B.LMOE_OK       # read clears it
+
+
+def test_stack_layers_against_oracle_layer_by_layer():
+    wl = small_workload(5).with_(n_layers=3)
+    s = wl.shape
+    layers = [synth.make_layer(wl, layer=l) for l in range(wl.n_layers)]
+    gammas = [synth.bf16_bits_from_f32(np.linspace(0.5, 1.5, s.hidden).astype(np.float32) + 0.1 * l)
+              for l in range(wl.n_layers)]
+    devs = [DeviceLayer(s, ly, gamma=g) for ly, g in zip(layers, gammas)]
+    xb = synth.make_x(wl)
+    x = to_device(xb, "cuda")
+    ws = devs[0].workspace(wl.T)
+    eps = 1e-6
+    # layer by layer through the stack call with 1..n layers: each output is
+    # checked against the oracle fed the GPU's own input of that layer
+    cur = xb
+    for l in range(wl.n_layers):
+        y = torch.empty_like(x)
+        B.lmoe_stack_forward(devs[0].cfg, [d.as_c_layer() for d in devs[:l + 1]], x, y, wl.T, eps, ws)
+        torch.cuda.synchronize()
+        y_ref, _, _, gap = orc.stack_layer_forward(s, layers[l], cur, orc.bf16_to_f64(gammas[l]), eps)
+        assert np.all(gap >= GAP)
+        assert_close(bf16_bits_to_f64(y), y_ref, f"stack layer {l}")
+        cur = y.cpu().numpy().view(np.uint16)
