@@ -1,9 +1,10 @@
 // C ABI of the latent-MoE block: argument checks, workspace carve-up and
 // dispatch to the kernels.  Declarations and conventions: include/lmoe.h.
 
+#include <algorithm>
 #include <cstring>
 
-#include "lmoe_internal.cuh"
+#include "lmoe_prefill.cuh"
 
 using namespace lmoe;
 
@@ -34,9 +35,23 @@ size_t record_bytes(const lmoe_cfg& c) {
     return 3 * lf / 2 + 3 * lf / 16 + 16;
 }
 
+// Token count from which the tensor-core path runs (bf16 router only).
+constexpr int kPrefillMinT = 64;
+
+// (the router GEMM tiles the experts by 128)
+bool use_prefill(const lmoe_cfg& c, int T) {
+    return T >= kPrefillMinT && c.router_dtype == LMOE_BF16 && c.n_experts % 128 == 0;
+}
+
+// Workspace of the few-token path (first) and of the tensor-core path; both
+// start after the control block, so one allocation serves either.
 struct WsLayout {
     size_t ctrl, idx, w, logits, n_unique, uexp, ucnt, uoff, slot_pair, pair_slot, ghit, tghit;
     size_t h, zsh, z, o, ypart, xio, yio, xa, xb;
+    // tensor-core path
+    size_t p_zero_begin, p_tgmask, p_cnt, p_fill, p_dhit, p_n_etiles, p_zero_end;
+    size_t p_n_unique, p_off, p_uexp, p_ucnt, p_uoff, p_etile, p_slot_pair, p_pair_slot, p_idx, p_w, p_logits;
+    size_t p_xh, p_xr, p_xr_lo, p_hperm, p_zperm, p_operm, p_s, p_zsh;
     size_t total;
 };
 
@@ -48,29 +63,67 @@ WsLayout ws_layout(const lmoe_cfg& c, int T) {
         off += (bytes + 255) & ~(size_t)255;
         return o;
     };
-    const size_t TK = (size_t)T * c.top_k;
     L.ctrl = take(sizeof(Ctrl));
-    L.idx = take(TK * 4);
-    L.w = take(TK * 4);
-    L.logits = take((size_t)T * c.n_experts * 4);
-    L.n_unique = take(4);
-    L.uexp = take(TK * 4);
-    L.ucnt = take(TK * 4);
-    L.uoff = take(TK * 4);
-    L.slot_pair = take(TK * 4);
-    L.pair_slot = take(TK * 4);
-    L.ghit = take((size_t)c.n_groups * 4);
-    L.tghit = take((size_t)T * c.n_groups);
-    L.h = take((size_t)T * c.n_groups * c.latent * 4);
-    L.zsh = take((size_t)T * c.shared_ffn * 4);
-    L.z = take(TK * c.ffn * 4);
-    L.o = take(TK * c.latent * 4);
-    L.ypart = take((size_t)(c.n_groups + 1) * T * c.hidden * 4);
     L.xio = take((size_t)T * c.hidden * 2);
     L.yio = take((size_t)T * c.hidden * 2);
     L.xa = take((size_t)T * c.hidden * 2);
     L.xb = take((size_t)T * c.hidden * 2);
-    L.total = off;
+    const size_t common = off;
+    // few-token path (used below kPrefillMinT tokens)
+    {
+        const int Td = use_prefill(c, T) ? kPrefillMinT - 1 : T;
+        const size_t TK = (size_t)Td * c.top_k;
+        L.idx = take(TK * 4);
+        L.w = take(TK * 4);
+        L.logits = take((size_t)Td * c.n_experts * 4);
+        L.n_unique = take(4);
+        L.uexp = take(TK * 4);
+        L.ucnt = take(TK * 4);
+        L.uoff = take(TK * 4);
+        L.slot_pair = take(TK * 4);
+        L.pair_slot = take(TK * 4);
+        L.ghit = take((size_t)c.n_groups * 4);
+        L.tghit = take((size_t)Td * c.n_groups);
+        L.h = take((size_t)Td * c.n_groups * c.latent * 4);
+        L.zsh = take((size_t)Td * c.shared_ffn * 4);
+        L.z = take(TK * c.ffn * 4);
+        L.o = take(TK * c.latent * 4);
+        L.ypart = take((size_t)(c.n_groups + 1) * Td * c.hidden * 4);
+    }
+    const size_t end_decode = off;
+    if (use_prefill(c, T)) {
+        off = common;
+        const size_t TK = (size_t)T * c.top_k;
+        const size_t ttiles = (T + kNtDense - 1) / kNtDense;
+        L.p_zero_begin = off;
+        L.p_tgmask = take((size_t)T * c.n_groups * 4);
+        L.p_cnt = take((size_t)c.n_experts * 4);
+        L.p_fill = take((size_t)c.n_experts * 4);
+        L.p_dhit = take(ttiles * c.n_groups);
+        L.p_n_etiles = take(4);
+        L.p_zero_end = off;
+        L.p_n_unique = take(4);
+        L.p_off = take((size_t)c.n_experts * 4);
+        const size_t nu = std::min((size_t)c.n_experts, TK);
+        L.p_uexp = take(nu * 4);
+        L.p_ucnt = take(nu * 4);
+        L.p_uoff = take(nu * 4);
+        L.p_etile = take((nu + TK / kNtExpert + 1) * 8);
+        L.p_slot_pair = take(TK * 4);
+        L.p_pair_slot = take(TK * 4);
+        L.p_idx = take(TK * 4);
+        L.p_w = take(TK * 4);
+        L.p_logits = take((size_t)T * c.n_experts * 4);
+        L.p_xh = take((size_t)T * c.hidden * 2);
+        L.p_xr = take((size_t)T * c.hidden * 2);
+        L.p_xr_lo = take((size_t)T * c.hidden * 2);
+        L.p_hperm = take(TK * c.latent * 2);
+        L.p_zperm = take(TK * c.ffn * 2);
+        L.p_operm = take(TK * c.latent * 2);
+        L.p_s = take((size_t)T * c.n_groups * c.latent * 2);
+        L.p_zsh = take((size_t)T * c.shared_ffn * 2);
+    }
+    L.total = std::max(off, end_decode);
     return L;
 }
 
@@ -123,6 +176,60 @@ int check_block_ptrs(const void* x, const void* router_w, const uint8_t* expert_
     return LMOE_OK;
 }
 
+// Fill the tensor-core path's parameters from the few-token ones and run it.
+int run_prefill(const lmoe_cfg& c, const FwdParams& f, const WsLayout& L, void* ws, cudaStream_t st) {
+    PrefillParams p;
+    std::memset(&p, 0, sizeof(p));
+    char* b = static_cast<char*>(ws);
+    p.H = f.H; p.L = f.L; p.E = f.E; p.K = f.K; p.G = f.G; p.F = f.F; p.Fs = f.Fs; p.du_fmt = f.du_fmt; p.T = f.T;
+    p.x = f.x;
+    p.router_w_bf16 = static_cast<const uint16_t*>(f.router_w);
+    p.router_b = f.router_b;
+    p.group = f.group;
+    p.D = f.D; p.U = f.U; p.experts = f.experts;
+    p.sg = f.sg; p.su = f.su; p.sd = f.sd;
+    p.residual = f.residual;
+    p.gamma = f.gamma;
+    p.eps = f.eps;
+    p.inject_idx = f.inject_idx;
+    p.inject_w = f.inject_w;
+    p.du_bytes = f.du_bytes_D;
+    p.rec_bytes = f.rec_bytes;
+    p.y = f.y;
+    p.out_idx = f.out_idx;
+    p.out_w = f.out_w;
+    p.ctrl = f.ctrl;
+    p.logits = reinterpret_cast<float*>(b + L.p_logits);
+    p.idx = reinterpret_cast<int32_t*>(b + L.p_idx);
+    p.w = reinterpret_cast<float*>(b + L.p_w);
+    p.tgmask = reinterpret_cast<uint32_t*>(b + L.p_tgmask);
+    p.cnt = reinterpret_cast<int32_t*>(b + L.p_cnt);
+    p.fill = reinterpret_cast<int32_t*>(b + L.p_fill);
+    p.dhit = reinterpret_cast<uint8_t*>(b + L.p_dhit);
+    p.n_etiles = reinterpret_cast<int32_t*>(b + L.p_n_etiles);
+    p.n_unique = reinterpret_cast<int32_t*>(b + L.p_n_unique);
+    p.off = reinterpret_cast<int32_t*>(b + L.p_off);
+    p.uexp = reinterpret_cast<int32_t*>(b + L.p_uexp);
+    p.ucnt = reinterpret_cast<int32_t*>(b + L.p_ucnt);
+    p.uoff = reinterpret_cast<int32_t*>(b + L.p_uoff);
+    p.etile = reinterpret_cast<int2*>(b + L.p_etile);
+    p.slot_pair = reinterpret_cast<int32_t*>(b + L.p_slot_pair);
+    p.pair_slot = reinterpret_cast<int32_t*>(b + L.p_pair_slot);
+    p.xh = reinterpret_cast<__half*>(b + L.p_xh);
+    if (f.gamma) {
+        p.xr = reinterpret_cast<uint16_t*>(b + L.p_xr);
+        p.xr_lo = reinterpret_cast<uint16_t*>(b + L.p_xr_lo);
+    }
+    p.hperm = reinterpret_cast<__half*>(b + L.p_hperm);
+    p.zperm = reinterpret_cast<__half*>(b + L.p_zperm);
+    p.operm = reinterpret_cast<__half*>(b + L.p_operm);
+    p.s = reinterpret_cast<__half*>(b + L.p_s);
+    p.zsh = reinterpret_cast<__half*>(b + L.p_zsh);
+    (void)c;
+    stage_reset();
+    return cuda_status(run_prefill_path(p, st, b + L.p_zero_begin, L.p_zero_end - L.p_zero_begin, stage_mark));
+}
+
 int forward_impl(const lmoe_cfg* cfg, const void* x, const void* router_w, const float* router_b,
                  const uint8_t* expert_group, const void* D, const void* U, const void* experts,
                  const lmoe_shared* shared, const void* residual, const int32_t* inject_idx, const float* inject_w,
@@ -161,6 +268,7 @@ int forward_impl(const lmoe_cfg* cfg, const void* x, const void* router_w, const
     p.out_idx = out_idx;
     p.out_w = out_w;
     p.y = static_cast<uint16_t*>(y);
+    if (use_prefill(*cfg, T)) return run_prefill(*cfg, p, L, ws, st);
     cudaError_t e = reset_tickets(ws, st);
     if (e != cudaSuccess) return LMOE_ERR_CUDA;
     return cuda_status(run_gemv_path(p, st, false));
@@ -202,6 +310,22 @@ int lmoe_route(const lmoe_cfg* cfg, const void* x, const void* router_w, const f
     p.router_b = router_b;
     p.out_idx = topk_idx;
     p.out_w = topk_w;
+    if (use_prefill(*cfg, T)) {
+        PrefillParams q;
+        std::memset(&q, 0, sizeof(q));
+        char* b = static_cast<char*>(ws);
+        q.H = p.H; q.E = p.E; q.K = p.K; q.T = T;
+        q.x = p.x;
+        q.router_w_bf16 = static_cast<const uint16_t*>(router_w);
+        q.router_b = router_b;
+        q.ctrl = p.ctrl;
+        q.logits = reinterpret_cast<float*>(b + L.p_logits);
+        q.idx = reinterpret_cast<int32_t*>(b + L.p_idx);
+        q.w = reinterpret_cast<float*>(b + L.p_w);
+        q.out_idx = topk_idx;
+        q.out_w = topk_w;
+        return cuda_status(run_prefill_route(q, st));
+    }
     cudaError_t e = reset_tickets(ws, st);
     if (e != cudaSuccess) return LMOE_ERR_CUDA;
     return cuda_status(run_gemv_path(p, st, true));

@@ -71,6 +71,35 @@ __device__ __forceinline__ float warp_sum(float v) {
 
 __device__ __forceinline__ float silu(float a) { return a / (1.0f + __expf(-a)); }
 
+// Block-wide exclusive scan of one int per thread; returns the total.
+__device__ __forceinline__ int block_exclusive_scan(int v, int* out, int* scratch) {
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nw = blockDim.x >> 5;
+    int x = v;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const int y = __shfl_up_sync(0xffffffffu, x, o);
+        if (lane >= o) x += y;
+    }
+    if (lane == 31) scratch[warp] = x;
+    __syncthreads();
+    if (warp == 0) {
+        int s = lane < nw ? scratch[lane] : 0;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const int y = __shfl_up_sync(0xffffffffu, s, o);
+            if (lane >= o) s += y;
+        }
+        if (lane < nw) scratch[lane] = s;
+    }
+    __syncthreads();
+    const int base = warp ? scratch[warp - 1] : 0;
+    *out = base + x - v;
+    const int total = scratch[nw - 1];
+    __syncthreads();
+    return total;
+}
+
+
 // ---------------------------------------------------------------------------
 // status word and tickets (first 4 KiB of the workspace)
 // ---------------------------------------------------------------------------

@@ -90,11 +90,9 @@ __device__ __forceinline__ void dot4_f32(float4 w, const float* xs, int k0, floa
     }
 }
 
-// One Q8_0 block (32 int8 at q, scale d) against xs[(k0 + j) * NT + t].
+// One Q8_0 block (32 int8 in a, b; scale d) against xs[(k0 + j) * NT + t].
 template <int NT>
-__device__ __forceinline__ void dot_q8_0_block(const uint8_t* q, float d, const float* xs, int k0, float (&acc)[NT]) {
-    const uint4 a = ldg_stream(reinterpret_cast<const uint4*>(q));
-    const uint4 b = ldg_stream(reinterpret_cast<const uint4*>(q) + 1);
+__device__ __forceinline__ void dot_q8_0_regs(uint4 a, uint4 b, float d, const float* xs, int k0, float (&acc)[NT]) {
     const uint32_t w8[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
     float blk[NT];
 #pragma unroll
@@ -115,8 +113,7 @@ __device__ __forceinline__ void dot_q8_0_block(const uint8_t* q, float d, const 
 
 // One Q4_0 block (16 bytes: byte j = elements j (low) and j+16 (high)).
 template <int NT>
-__device__ __forceinline__ void dot_q4_0_block(const uint8_t* q, float d, const float* xs, int k0, float (&acc)[NT]) {
-    const uint4 a = ldg_stream(reinterpret_cast<const uint4*>(q));
+__device__ __forceinline__ void dot_q4_0_regs(uint4 a, float d, const float* xs, int k0, float (&acc)[NT]) {
     const uint32_t w4[4] = {a.x, a.y, a.z, a.w};
     float blk[NT];
 #pragma unroll
@@ -171,24 +168,90 @@ __device__ __forceinline__ void dot_nvfp4_chunk(uint4 qv, float s0, float s1, co
     }
 }
 
+// One row of a plain bf16 / fp32 matrix (K contiguous) against xs, the warp's
+// lanes splitting K; ten 16-byte loads per lane are issued before any
+// arithmetic.  The per-lane partial sums are left in acc (reduce with warp_sum).
+template <int NT, bool kBF16>
+__device__ __forceinline__ void row_dot(const void* wrow, int K, const float* xs, int lane, float (&acc)[NT]) {
+    constexpr int kB = 10;
+    constexpr int kPer = kBF16 ? 8 : 4;          // elements per 16-byte load
+    constexpr int kStep = 32 * kPer;
+    for (int base = 0; base < K; base += kB * kStep) {
+        uint4 w[kB];
+#pragma unroll
+        for (int i = 0; i < kB; ++i) {
+            const int k0 = base + i * kStep + lane * kPer;
+            if (k0 < K) w[i] = ldg_stream(reinterpret_cast<const uint4*>(static_cast<const char*>(wrow) + (size_t)k0 * (kBF16 ? 2 : 4)));
+        }
+#pragma unroll
+        for (int i = 0; i < kB; ++i) {
+            const int k0 = base + i * kStep + lane * kPer;
+            if (k0 < K) {
+                if (kBF16) dot8_bf16<NT>(w[i], xs, k0, acc);
+                else dot4_f32<NT>(make_float4(__uint_as_float(w[i].x), __uint_as_float(w[i].y), __uint_as_float(w[i].z),
+                                              __uint_as_float(w[i].w)), xs, k0, acc);
+            }
+        }
+    }
+}
+
 // Row-tile GEMV over a D/U matrix [R rows][C cols] stored as Q8_0 / Q4_0:
-// lane = row (row0 + lane), warps split the 64-wide column groups.
+// lane = row, warps split the 64-wide column groups.  Each warp takes two
+// groups per pass and issues all their loads before any arithmetic.
 template <int NT>
 __device__ __forceinline__ void du_rows(int fmt, const uint8_t* mat, int R, int C, int row, const float* xs,
                                         float (&acc)[NT]) {
     const int warp = threadIdx.x >> 5;
     const int nwarps = blockDim.x >> 5;
-    const int nb = C / 32;
-    const size_t qrow = fmt == LMOE_Q8_0 ? 32 : 16;
-    const uint16_t* dsc = reinterpret_cast<const uint16_t*>(mat + (size_t)R * nb * qrow);
-    for (int kg = warp; kg < C / 64; kg += nwarps) {
+    const int ng = C / 64;
+    const uint16_t* dsc = reinterpret_cast<const uint16_t*>(mat + (size_t)R * C / 32 * (fmt == LMOE_Q8_0 ? 32 : 16));
+    for (int base = warp; base < ng; base += 2 * nwarps) {
+        const int kg[2] = {base, base + nwarps};
+        if (fmt == LMOE_Q8_0) {
+            uint4 q[2][4];
+            uint16_t d[2][2];
 #pragma unroll
-        for (int c = 0; c < 2; ++c) {
-            const int b = 2 * kg + c;
-            const float d = fp16_bits_to_f32(__ldg(dsc + (size_t)b * R + row));
-            const uint8_t* q = mat + ((size_t)b * R + row) * qrow;
-            if (fmt == LMOE_Q8_0) dot_q8_0_block<NT>(q, d, xs, 32 * b, acc);
-            else dot_q4_0_block<NT>(q, d, xs, 32 * b, acc);
+            for (int u = 0; u < 2; ++u) {
+                if (kg[u] < ng) {
+#pragma unroll
+                    for (int c = 0; c < 2; ++c) {
+                        const uint4* src = reinterpret_cast<const uint4*>(mat + ((size_t)(2 * kg[u] + c) * R + row) * 32);
+                        q[u][2 * c] = ldg_stream(src);
+                        q[u][2 * c + 1] = ldg_stream(src + 1);
+                        d[u][c] = __ldg(dsc + (size_t)(2 * kg[u] + c) * R + row);
+                    }
+                }
+            }
+#pragma unroll
+            for (int u = 0; u < 2; ++u) {
+                if (kg[u] < ng) {
+#pragma unroll
+                    for (int c = 0; c < 2; ++c)
+                        dot_q8_0_regs<NT>(q[u][2 * c], q[u][2 * c + 1], fp16_bits_to_f32(d[u][c]), xs,
+                                          64 * kg[u] + 32 * c, acc);
+                }
+            }
+        } else {
+            uint4 q[2][2];
+            uint16_t d[2][2];
+#pragma unroll
+            for (int u = 0; u < 2; ++u) {
+                if (kg[u] < ng) {
+#pragma unroll
+                    for (int c = 0; c < 2; ++c) {
+                        q[u][c] = ldg_stream(reinterpret_cast<const uint4*>(mat + ((size_t)(2 * kg[u] + c) * R + row) * 16));
+                        d[u][c] = __ldg(dsc + (size_t)(2 * kg[u] + c) * R + row);
+                    }
+                }
+            }
+#pragma unroll
+            for (int u = 0; u < 2; ++u) {
+                if (kg[u] < ng) {
+#pragma unroll
+                    for (int c = 0; c < 2; ++c)
+                        dot_q4_0_regs<NT>(q[u][c], fp16_bits_to_f32(d[u][c]), xs, 64 * kg[u] + 32 * c, acc);
+                }
+            }
         }
     }
 }
@@ -199,13 +262,28 @@ __device__ __forceinline__ void nvfp4_rows(const uint8_t* q, const uint8_t* s, i
                                            const float* xs, float (&acc)[NT]) {
     const int warp = threadIdx.x >> 5;
     const int nwarps = blockDim.x >> 5;
-    for (int kg = warp; kg < C / 64; kg += nwarps) {
-        float sc[4];
-        e4m3x4_to_f32x4(__ldg(reinterpret_cast<const uint32_t*>(s + ((size_t)kg * R + row) * 4)), sc);
+    const int ng = C / 64;
+    for (int base = warp; base < ng; base += 2 * nwarps) {
+        const int kg[2] = {base, base + nwarps};
+        uint4 qv[2][2];
+        uint32_t sw[2];
 #pragma unroll
-        for (int c = 0; c < 2; ++c) {
-            const uint4 qv = ldg_stream(reinterpret_cast<const uint4*>(q + ((size_t)(2 * kg + c) * R + row) * 16));
-            dot_nvfp4_chunk<NT>(qv, sc[2 * c], sc[2 * c + 1], xs, 64 * kg + 32 * c, acc);
+        for (int u = 0; u < 2; ++u) {
+            if (kg[u] < ng) {
+                sw[u] = __ldg(reinterpret_cast<const uint32_t*>(s + ((size_t)kg[u] * R + row) * 4));
+#pragma unroll
+                for (int c = 0; c < 2; ++c)
+                    qv[u][c] = ldg_stream(reinterpret_cast<const uint4*>(q + ((size_t)(2 * kg[u] + c) * R + row) * 16));
+            }
+        }
+#pragma unroll
+        for (int u = 0; u < 2; ++u) {
+            if (kg[u] < ng) {
+                float sc[4];
+                e4m3x4_to_f32x4(sw[u], sc);
+#pragma unroll
+                for (int c = 0; c < 2; ++c) dot_nvfp4_chunk<NT>(qv[u][c], sc[2 * c], sc[2 * c + 1], xs, 64 * kg[u] + 32 * c, acc);
+            }
         }
     }
 }
@@ -248,22 +326,13 @@ __global__ void __launch_bounds__(256) k_router_shared(FwdParams p) {
         stage_x<NT>(p, t0, nt, xs, rs);
         __syncthreads();
         if (router_cta) {
-            const int rows_per_cta = p.router_rows_per_warp * 8;
-            for (int r = 0; r < p.router_rows_per_warp; ++r) {
-                const int e = blockIdx.x * rows_per_cta + warp * p.router_rows_per_warp + r;
-                if (e >= p.E) break;
+            const int e = blockIdx.x * 8 + warp;
+            if (e < p.E) {
                 float acc[NT];
 #pragma unroll
                 for (int t = 0; t < NT; ++t) acc[t] = 0.f;
-                if (kRouterBF16) {
-                    const uint16_t* wr = static_cast<const uint16_t*>(p.router_w) + (size_t)e * H;
-                    for (int k0 = lane * 8; k0 < H; k0 += 256)
-                        dot8_bf16<NT>(ldg_stream(reinterpret_cast<const uint4*>(wr + k0)), xs, k0, acc);
-                } else {
-                    const float* wr = static_cast<const float*>(p.router_w) + (size_t)e * H;
-                    for (int k0 = lane * 4; k0 < H; k0 += 128)
-                        dot4_f32<NT>(ldg_stream(reinterpret_cast<const float4*>(wr + k0)), xs, k0, acc);
-                }
+                if (kRouterBF16) row_dot<NT, true>(static_cast<const uint16_t*>(p.router_w) + (size_t)e * H, H, xs, lane, acc);
+                else row_dot<NT, false>(static_cast<const float*>(p.router_w) + (size_t)e * H, H, xs, lane, acc);
                 const float b = p.router_b ? __ldg(p.router_b + e) : 0.f;
 #pragma unroll
                 for (int t = 0; t < NT; ++t) {
@@ -278,12 +347,8 @@ __global__ void __launch_bounds__(256) k_router_shared(FwdParams p) {
                 float a[NT], u[NT];
 #pragma unroll
                 for (int t = 0; t < NT; ++t) { a[t] = 0.f; u[t] = 0.f; }
-                const uint16_t* wg = p.sg + (size_t)f * H;
-                const uint16_t* wu = p.su + (size_t)f * H;
-                for (int k0 = lane * 8; k0 < H; k0 += 256) {
-                    dot8_bf16<NT>(ldg_stream(reinterpret_cast<const uint4*>(wg + k0)), xs, k0, a);
-                    dot8_bf16<NT>(ldg_stream(reinterpret_cast<const uint4*>(wu + k0)), xs, k0, u);
-                }
+                row_dot<NT, true>(p.sg + (size_t)f * H, H, xs, lane, a);
+                row_dot<NT, true>(p.su + (size_t)f * H, H, xs, lane, u);
 #pragma unroll
                 for (int t = 0; t < NT; ++t) {
                     const float av = warp_sum(a[t]), uv = warp_sum(u[t]);
@@ -318,34 +383,6 @@ __device__ __forceinline__ void warp_argmax(float& v, int& i) {
         const int oi = __shfl_xor_sync(0xffffffffu, i, o);
         if (ov > v || (ov == v && oi < i)) { v = ov; i = oi; }
     }
-}
-
-// Block-wide exclusive scan of one int per thread; returns the total.
-__device__ int block_exclusive_scan(int v, int* out, int* scratch) {
-    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nw = blockDim.x >> 5;
-    int x = v;
-#pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-        const int y = __shfl_up_sync(0xffffffffu, x, o);
-        if (lane >= o) x += y;
-    }
-    if (lane == 31) scratch[warp] = x;
-    __syncthreads();
-    if (warp == 0) {
-        int s = lane < nw ? scratch[lane] : 0;
-#pragma unroll
-        for (int o = 1; o < 32; o <<= 1) {
-            const int y = __shfl_up_sync(0xffffffffu, s, o);
-            if (lane >= o) s += y;
-        }
-        if (lane < nw) scratch[lane] = s;
-    }
-    __syncthreads();
-    const int base = warp ? scratch[warp - 1] : 0;
-    *out = base + x - v;
-    const int total = scratch[nw - 1];
-    __syncthreads();
-    return total;
 }
 
 __device__ void topk_and_buckets(const FwdParams& p) {
@@ -460,7 +497,7 @@ __device__ void topk_and_buckets(const FwdParams& p) {
 // ---------------------------------------------------------------------------
 
 template <int NT>
-__global__ void __launch_bounds__(256) k_dproj(FwdParams p) {
+__global__ void __launch_bounds__(512) k_dproj(FwdParams p) {
     extern __shared__ float smem[];
     __shared__ float rs[kChunk];
     const int g = blockIdx.y;
@@ -492,7 +529,7 @@ __global__ void __launch_bounds__(256) k_dproj(FwdParams p) {
 // ---------------------------------------------------------------------------
 
 template <int NT>
-__global__ void __launch_bounds__(256) k_expert_gateup(FwdParams p) {
+__global__ void __launch_bounds__(512) k_expert_gateup(FwdParams p) {
     extern __shared__ float smem[];
     const int j = blockIdx.y;
     const int n_unique = __ldcg(p.r.n_unique);
@@ -536,7 +573,7 @@ __global__ void __launch_bounds__(256) k_expert_gateup(FwdParams p) {
 }
 
 template <int NT>
-__global__ void __launch_bounds__(256) k_expert_down(FwdParams p) {
+__global__ void __launch_bounds__(512) k_expert_down(FwdParams p) {
     extern __shared__ float smem[];
     const int j = blockIdx.y;
     const int n_unique = __ldcg(p.r.n_unique);
@@ -576,13 +613,16 @@ __global__ void __launch_bounds__(256) k_expert_down(FwdParams p) {
 // ---------------------------------------------------------------------------
 
 template <int NT>
-__global__ void __launch_bounds__(256) k_uproj(FwdParams p) {
+__global__ void __launch_bounds__(512) k_uproj(FwdParams p) {
     extern __shared__ float smem[];
     const int part = blockIdx.y;            // 0..G-1: group; G: shared expert
     const int H = p.H, L = p.L, G = p.G, K = p.K, T = p.T;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int row0 = blockIdx.x * 32;
     const bool active = part == G || __ldcg(p.r.ghit + part) > 0;
+    __shared__ int lst_slot[kChunk * kMaxTopK];
+    __shared__ float lst_w[kChunk * kMaxTopK];
+    __shared__ int lst_n[kChunk];
     if (active) {
         float* as = smem;                                   // [max(L, Fs)][NT]
         float* red = smem + (size_t)max(L, p.Fs) * NT;
@@ -593,17 +633,28 @@ __global__ void __launch_bounds__(256) k_uproj(FwdParams p) {
             for (int t = 0; t < NT; ++t) acc[t] = 0.f;
             if (part < G) {
                 // s[t][k] = sum over the token's experts of group `part` of w * o
-                for (int i = threadIdx.x; i < NT * L; i += blockDim.x) {
-                    const int t = i / L, k = i - t * L;
-                    float s = 0.f;
+                if (threadIdx.x < NT) {
+                    const int t = threadIdx.x;
+                    int n = 0;
                     if (t < nt && p.r.tghit[(size_t)(t0 + t) * G + part]) {
                         for (int kk = 0; kk < K; ++kk) {
                             const int pair = (t0 + t) * K + kk;
                             const int e = __ldcg(p.r.idx + pair);
-                            if (p.group[e] == part)
-                                s = fmaf(__ldcg(p.r.w + pair), __ldcg(p.o + (size_t)__ldcg(p.r.pair_slot + pair) * L + k), s);
+                            if (p.group[e] == part) {
+                                lst_slot[t * kMaxTopK + n] = __ldcg(p.r.pair_slot + pair);
+                                lst_w[t * kMaxTopK + n] = __ldcg(p.r.w + pair);
+                                ++n;
+                            }
                         }
                     }
+                    lst_n[t] = n;
+                }
+                __syncthreads();
+                for (int i = threadIdx.x; i < NT * L; i += blockDim.x) {
+                    const int t = i / L, k = i - t * L;
+                    float s = 0.f;
+                    for (int j = 0; j < lst_n[t]; ++j)
+                        s = fmaf(lst_w[t * kMaxTopK + j], __ldcg(p.o + (size_t)lst_slot[t * kMaxTopK + j] * L + k), s);
                     as[k * NT + t] = s;
                 }
                 __syncthreads();
@@ -626,9 +677,7 @@ __global__ void __launch_bounds__(256) k_uproj(FwdParams p) {
                     float a2[NT];
 #pragma unroll
                     for (int t = 0; t < NT; ++t) a2[t] = 0.f;
-                    const uint16_t* wd = p.sd + (size_t)row * Fs;
-                    for (int k0 = lane * 8; k0 < Fs; k0 += 256)
-                        dot8_bf16<NT>(ldg_stream(reinterpret_cast<const uint4*>(wd + k0)), as, k0, a2);
+                    row_dot<NT, true>(p.sd + (size_t)row * Fs, Fs, as, lane, a2);
 #pragma unroll
                     for (int t = 0; t < NT; ++t) {
                         const float v = warp_sum(a2[t]);
@@ -676,47 +725,73 @@ void set_stage_events(void* const* events, int n) {
     for (int i = 0; i < n; ++i) g_stage_events[i] = static_cast<cudaEvent_t>(events[i]);
 }
 
-static void stage_mark(cudaStream_t st) {
+void stage_mark(cudaStream_t st) {
     if (g_stage_cursor < g_n_stage_events) cudaEventRecord(g_stage_events[g_stage_cursor++], st);
+}
+
+void stage_reset() { g_stage_cursor = 0; }
+
+// Raise a kernel's dynamic shared-memory limit when needed (static + dynamic
+// above 48 KiB needs the opt-in); remembered per kernel and device.
+cudaError_t ensure_smem(const void* kernel, size_t smem) {
+    struct Entry { const void* k; int dev; size_t bytes; };
+    static Entry table[128];
+    static int n = 0;
+    int dev = 0;
+    cudaGetDevice(&dev);
+    for (int i = 0; i < n; ++i)
+        if (table[i].k == kernel && table[i].dev == dev && table[i].bytes >= smem) return cudaSuccess;
+    cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    for (int i = 0; i < n; ++i)
+        if (table[i].k == kernel && table[i].dev == dev) { table[i].bytes = smem; return cudaSuccess; }
+    if (n < 128) table[n++] = {kernel, dev, smem};
+    return cudaSuccess;
 }
 
 template <typename Kern>
 static cudaError_t launch(Kern k, dim3 grid, int threads, size_t smem, cudaStream_t st, const FwdParams& p) {
     stage_mark(st);
-    if (smem > 48 * 1024) {
-        cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (smem > 0) {
+        cudaError_t e = ensure_smem(reinterpret_cast<const void*>(k), smem);
         if (e != cudaSuccess) return e;
     }
     k<<<grid, threads, smem, st>>>(p);
     return cudaGetLastError();
 }
 
+// Warps per CTA of a row-tile GEMV over C columns: two 64-column groups per warp.
+static int gemv_warps(int C) { return max(1, min(16, (C / 64 + 1) / 2)); }
+
 template <int NT>
 static cudaError_t run_gemv_path_nt(FwdParams p, cudaStream_t st, bool route_only) {
-    const int threads = 256;
-    const size_t red = (size_t)8 * 32 * NT * sizeof(float);
-    // 1. router (+ shared gate/up, top-k, buckets)
-    p.router_rows_per_warp = 2;
-    p.n_router_ctas = (p.E + 8 * p.router_rows_per_warp - 1) / (8 * p.router_rows_per_warp);
+    auto red = [](int warps) { return (size_t)warps * 32 * NT * sizeof(float); };
+    // 1. router (+ shared gate/up, top-k, buckets): one warp per router row / shared feature
+    p.router_rows_per_warp = 1;
+    p.n_router_ctas = (p.E + 7) / 8;
     p.do_shared = !route_only;
     p.do_buckets = !route_only;
     const int n_shared_ctas = route_only ? 0 : (p.Fs + 7) / 8;
     {
         const size_t sm = (size_t)p.H * NT * sizeof(float);
         cudaError_t e = p.router_bf16
-            ? launch(k_router_shared<NT, true>, dim3(p.n_router_ctas + n_shared_ctas), threads, sm, st, p)
-            : launch(k_router_shared<NT, false>, dim3(p.n_router_ctas + n_shared_ctas), threads, sm, st, p);
+            ? launch(k_router_shared<NT, true>, dim3(p.n_router_ctas + n_shared_ctas), 256, sm, st, p)
+            : launch(k_router_shared<NT, false>, dim3(p.n_router_ctas + n_shared_ctas), 256, sm, st, p);
         if (e != cudaSuccess || route_only) return e;
     }
     const int max_unique = min(p.T * p.K, p.E);
     cudaError_t e;
-    e = launch(k_dproj<NT>, dim3(p.L / 32, p.G), threads, (size_t)p.H * NT * 4 + red, st, p);
+    int w = gemv_warps(p.H);
+    e = launch(k_dproj<NT>, dim3(p.L / 32, p.G), 32 * w, (size_t)p.H * NT * 4 + red(w), st, p);
     if (e != cudaSuccess) return e;
-    e = launch(k_expert_gateup<NT>, dim3(p.F / 32, max_unique), threads, (size_t)p.L * NT * 4 + red, st, p);
+    w = gemv_warps(p.L);
+    e = launch(k_expert_gateup<NT>, dim3(p.F / 32, max_unique), 32 * w, (size_t)p.L * NT * 4 + red(w), st, p);
     if (e != cudaSuccess) return e;
-    e = launch(k_expert_down<NT>, dim3(p.L / 32, max_unique), threads, (size_t)p.F * NT * 4 + red, st, p);
+    w = gemv_warps(p.F);
+    e = launch(k_expert_down<NT>, dim3(p.L / 32, max_unique), 32 * w, (size_t)p.F * NT * 4 + red(w), st, p);
     if (e != cudaSuccess) return e;
-    e = launch(k_uproj<NT>, dim3(p.H / 32, p.G + 1), threads, (size_t)max(p.L, p.Fs) * NT * 4 + red, st, p);
+    w = max(gemv_warps(p.L), 8);
+    e = launch(k_uproj<NT>, dim3(p.H / 32, p.G + 1), 32 * w, (size_t)max(p.L, p.Fs) * NT * 4 + red(w), st, p);
     return e;
 }
 

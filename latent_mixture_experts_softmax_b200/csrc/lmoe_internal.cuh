@@ -69,6 +69,9 @@ constexpr int kMaxStageEvents = 16;
 
 cudaError_t run_gemv_path(const FwdParams& p, cudaStream_t st, bool route_only);
 void set_stage_events(void* const* events, int n);
+void stage_mark(cudaStream_t st);
+void stage_reset();
+cudaError_t ensure_smem(const void* kernel, size_t smem);
 cudaError_t run_debug_decode(int fmt, const void* blob, int R, int C, float ts, float* out, cudaStream_t st);
 
 }  // namespace lmoe

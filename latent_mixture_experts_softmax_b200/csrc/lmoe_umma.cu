@@ -1,0 +1,938 @@
+// Latent-MoE block for many tokens (prefill): the dense contractions run on
+// the 5th-generation tensor cores (tcgen05.mma, fp32 accumulators in TMEM)
+// in one warp-specialised, persistent GEMM kernel template:
+//
+//   warps 0-3  epilogue: TMEM -> registers -> fused epilogue -> global
+//   warps 4-7  producers: TMA for the activation operand; the weight operand
+//              is read from its storage format (Q8_0, Q4_0, NVFP4, bf16),
+//              dequantised in registers and written to shared memory in the
+//              UMMA K-major 128-byte-swizzled layout
+//   warp 8     TMEM allocation and the single-thread UMMA issue
+//
+// Operands are swapped with respect to the usual "tokens x weights" view:
+// the weight rows are the MMA's M = 128 side and the tokens (or expert
+// slots) are its N side, so one dequantised weight tile feeds up to 256
+// tokens.  Every accumulator is fp32 in TMEM, double-buffered so the
+// epilogue of one tile overlaps the main loop of the next.
+//
+// GEMMs of the block (teardown article "Edge0-145B: a Qwen MoE with its
+// experts squeezed", section "A latent in front of the experts"; Edge0
+// 145B / 120B model page, architecture tables):
+//   ROUTER        logits[t][e]   = W_r[e] . x_t + b_e          (bf16 x bf16)
+//   SHARED_GATEUP z_sh[t][f]     = silu(S_gate x_t) * (S_up x_t)  (bf16)
+//   DPROJ         h[slot][l]     = (D_g x_t)[l] for every slot (t, k) with
+//                                  group(e_k) = g               (fp16)
+//   GATEUP        z[slot][f]     = silu(W_gate h) * (W_up h)    (fp16)
+//   DOWN          o[slot][l]     = w_slot * (W_down z)[l]       (fp16)
+//   UPROJ         y[t]           = sum_g U_g s[t][g] + S_down z_sh[t]
+//                                  (+ residual)                 (fp16)
+// with s[t][g] = sum of o over the token's experts of group g (combine
+// kernel).  The routing, bucketing and combine steps are plain CUDA kernels
+// in this file.
+
+#include "lmoe_prefill.cuh"
+
+namespace lmoe {
+
+using namespace sm100;
+
+constexpr uint64_t kWaitLimitNs = 2000000000ull;   // 2 s per barrier wait
+
+// ---------------------------------------------------------------------------
+// tiles
+// ---------------------------------------------------------------------------
+
+struct TileRef {
+    int valid;
+    int mat;      // group (DPROJ) or expert (GATEUP / DOWN)
+    int m0;       // first A row of the tile (feature)
+    int b0;       // first B row (token or slot)
+    int n;        // valid B rows
+    int nq;       // token tile index (UPROJ / DPROJ hit flags)
+};
+
+template <int KIND, int NT>
+struct Sched {
+    __device__ static int m_tiles(const PrefillParams& p) {
+        switch (KIND) {
+            case G_ROUTER: return p.E / 128;
+            case G_SHARED_GATEUP: return p.Fs / 64;
+            case G_DPROJ: return p.G * (p.L / 128);
+            case G_GATEUP: return p.F / 64;
+            case G_DOWN: return p.L / 128;
+            default: return p.H / 128;
+        }
+    }
+    __device__ static int num_tiles(const PrefillParams& p) {
+        if (KIND == G_GATEUP || KIND == G_DOWN) return m_tiles(p) * __ldcg(p.n_etiles);
+        return m_tiles(p) * ((p.T + NT - 1) / NT);
+    }
+    __device__ static TileRef get(const PrefillParams& p, int i) {
+        TileRef t;
+        const int mt = m_tiles(p);
+        t.valid = 1;
+        t.mat = 0;
+        if (KIND == G_GATEUP || KIND == G_DOWN) {
+            // consecutive tiles share the expert's token rows
+            const int et = i / mt, m = i % mt;
+            const int2 d = p.etile[et];
+            const int j = d.x, n0 = d.y;
+            t.mat = __ldcg(p.uexp + j);
+            t.m0 = m * (KIND == G_GATEUP ? 64 : 128);
+            t.b0 = __ldcg(p.uoff + j) + n0;
+            t.n = min(NT, __ldcg(p.ucnt + j) - n0);
+            t.nq = 0;
+        } else {
+            // consecutive tiles share the weight tile (token tiles fastest)
+            const int ntt = (p.T + NT - 1) / NT;
+            const int m = i / ntt, q = i % ntt;
+            t.nq = q;
+            t.b0 = q * NT;
+            t.n = min(NT, p.T - t.b0);
+            if (KIND == G_DPROJ) {
+                const int mpg = p.L / 128;
+                t.mat = m / mpg;
+                t.m0 = (m % mpg) * 128;
+                t.valid = p.dhit[q * p.G + t.mat] != 0;
+            } else if (KIND == G_SHARED_GATEUP) {
+                t.m0 = m * 64;
+            } else {
+                t.m0 = m * 128;
+            }
+        }
+        return t;
+    }
+    // UPROJ: one segment per group, then the shared expert's down projection.
+    // ROUTER / SHARED_GATEUP on a normalised input: the input is split into
+    // bf16 high and low parts, one segment each, so the products stay exact.
+    __device__ static int num_segs(const PrefillParams& p) {
+        if (KIND == G_UPROJ) return p.G + 1;
+        if (KIND == G_ROUTER || KIND == G_SHARED_GATEUP) return p.xr ? 2 : 1;
+        return 1;
+    }
+    __device__ static bool seg_active(const PrefillParams& p, const TileRef& t, int seg) {
+        if (KIND != G_UPROJ || seg == p.G) return true;
+        return p.dhit[t.nq * p.G + seg] != 0;
+    }
+    __device__ static int seg_k(const PrefillParams& p, int seg) {
+        switch (KIND) {
+            case G_ROUTER:
+            case G_SHARED_GATEUP:
+            case G_DPROJ: return p.H;
+            case G_GATEUP: return p.L;
+            case G_DOWN: return p.F;
+            default: return seg == p.G ? p.Fs : p.L;
+        }
+    }
+    // A comes through TMA (plain bf16 weights) rather than the dequantising producers
+    static constexpr bool kTmaA = KIND == G_ROUTER || KIND == G_SHARED_GATEUP;
+    static constexpr int kBf16 = (KIND == G_ROUTER || KIND == G_SHARED_GATEUP) ? 1 : 0;
+};
+
+// Walks the (tile, segment, 64-wide K stage) sequence of one CTA.
+template <int KIND, int NT>
+struct Cursor {
+    using S = Sched<KIND, NT>;
+    int tile, seg, ks, nk, ntiles;
+    bool done;
+    TileRef t;
+    __device__ void begin(const PrefillParams& p) {
+        ntiles = S::num_tiles(p);
+        tile = (int)blockIdx.x - (int)gridDim.x;
+        done = false;
+        next_tile(p);
+    }
+    __device__ void next_tile(const PrefillParams& p) {
+        while (true) {
+            tile += gridDim.x;
+            if (tile >= ntiles) { done = true; return; }
+            t = S::get(p, tile);
+            if (!t.valid) continue;
+            seg = -1;
+            if (next_seg(p)) return;
+        }
+    }
+    // advance to the next active segment of the current tile; false if none
+    __device__ bool next_seg(const PrefillParams& p) {
+        while (++seg < S::num_segs(p)) {
+            if (S::seg_active(p, t, seg)) {
+                ks = 0;
+                nk = S::seg_k(p, seg) / 64;
+                return true;
+            }
+        }
+        return false;
+    }
+    __device__ void next_stage(const PrefillParams& p) {
+        if (++ks < nk) return;
+        if (next_seg(p)) return;
+        next_tile(p);
+    }
+    __device__ bool last_stage_of_tile(const PrefillParams& p) const {
+        if (ks + 1 < nk) return false;
+        for (int s2 = seg + 1; s2 < S::num_segs(p); ++s2)
+            if (S::seg_active(p, t, s2)) return false;
+        return true;
+    }
+};
+
+// ---------------------------------------------------------------------------
+// weight operand: raw loads and dequantisation to fp16 (one row, 64 columns)
+// ---------------------------------------------------------------------------
+
+struct RawRow {
+    uint4 q[8];
+    uint32_t s;
+};
+
+__device__ __forceinline__ uint4 ldg_nc(const void* ptr) { return ldg_stream(reinterpret_cast<const uint4*>(ptr)); }
+
+// Where row r (0..127) of the A tile of stage (tile, seg, ks) lives, and its load.
+template <int KIND, int NT>
+__device__ __forceinline__ void load_raw(const PrefillParams& p, const Cursor<KIND, NT>& c, int r, RawRow& raw) {
+    const int k0 = c.ks * 64;
+    if (KIND == G_DPROJ || (KIND == G_UPROJ && c.seg < p.G)) {
+        const int R = KIND == G_DPROJ ? p.L : p.H;
+        const int C = KIND == G_DPROJ ? p.H : p.L;
+        const uint8_t* mat = (KIND == G_DPROJ ? p.D : p.U) + (size_t)(KIND == G_DPROJ ? c.t.mat : c.seg) * p.du_bytes;
+        const int row = c.t.m0 + r;
+        const int kb = k0 / 32;
+        const uint16_t* dsc;
+        if (p.du_fmt == LMOE_Q8_0) {
+            raw.q[0] = ldg_nc(mat + ((size_t)kb * R + row) * 32);
+            raw.q[1] = ldg_nc(mat + ((size_t)kb * R + row) * 32 + 16);
+            raw.q[2] = ldg_nc(mat + ((size_t)(kb + 1) * R + row) * 32);
+            raw.q[3] = ldg_nc(mat + ((size_t)(kb + 1) * R + row) * 32 + 16);
+            dsc = reinterpret_cast<const uint16_t*>(mat + (size_t)R * C);
+        } else {
+            raw.q[0] = ldg_nc(mat + ((size_t)kb * R + row) * 16);
+            raw.q[1] = ldg_nc(mat + ((size_t)(kb + 1) * R + row) * 16);
+            dsc = reinterpret_cast<const uint16_t*>(mat + (size_t)R * C / 2);
+        }
+        raw.s = (uint32_t)__ldg(dsc + (size_t)kb * R + row) | ((uint32_t)__ldg(dsc + (size_t)(kb + 1) * R + row) << 16);
+    } else if (KIND == G_UPROJ) {
+        // shared expert down projection, bf16 [H][Fs]
+        const uint16_t* src = p.sd + (size_t)(c.t.m0 + r) * p.Fs + k0;
+#pragma unroll
+        for (int i = 0; i < 8; ++i) raw.q[i] = ldg_nc(src + 8 * i);
+    } else if (KIND == G_GATEUP || KIND == G_DOWN) {
+        const size_t nq = (size_t)p.L * p.F / 2, ns = (size_t)p.L * p.F / 16;
+        const uint8_t* rec = p.experts + (size_t)c.t.mat * p.rec_bytes;
+        const uint8_t *q, *s;
+        int R, row;
+        if (KIND == G_GATEUP) {
+            const bool up = r >= 64;
+            q = rec + (up ? nq : 0);
+            s = rec + 3 * nq + (up ? ns : 0);
+            R = p.F;
+            row = c.t.m0 + (r & 63);
+        } else {
+            q = rec + 2 * nq;
+            s = rec + 3 * nq + 2 * ns;
+            R = p.L;
+            row = c.t.m0 + r;
+        }
+        const int kc = k0 / 32;
+        raw.q[0] = ldg_nc(q + ((size_t)kc * R + row) * 16);
+        raw.q[1] = ldg_nc(q + ((size_t)(kc + 1) * R + row) * 16);
+        raw.s = __ldg(reinterpret_cast<const uint32_t*>(s + ((size_t)(k0 / 64) * R + row) * 4));
+    }
+}
+
+__device__ __forceinline__ uint32_t h2_bits(__half2 h) { return *reinterpret_cast<uint32_t*>(&h); }
+__device__ __forceinline__ __half2 bits_h2(uint32_t u) { return *reinterpret_cast<__half2*>(&u); }
+
+// 4 bytes holding values v+bias (0..255) -> two half2 of (1024 + byte)
+__device__ __forceinline__ void bytes_to_h2x2(uint32_t w, uint32_t& lo, uint32_t& hi) {
+    lo = __byte_perm(w, 0x64646464u, 0x4140);
+    hi = __byte_perm(w, 0x64646464u, 0x4342);
+}
+
+// Dequantise one row's 64 columns into 32 half2 (element order).
+template <int KIND>
+__device__ __forceinline__ void dequant_row(const PrefillParams& p, int seg, const RawRow& raw, uint32_t (&o)[32]) {
+    if (KIND == G_DPROJ || (KIND == G_UPROJ && seg < p.G)) {
+        const __half2 d0 = __half2half2(__ushort_as_half((unsigned short)(raw.s & 0xFFFF)));
+        const __half2 d1 = __half2half2(__ushort_as_half((unsigned short)(raw.s >> 16)));
+        if (p.du_fmt == LMOE_Q8_0) {
+            const __half2 off = __float2half2_rn(1152.f);          // 1024 + 128
+#pragma unroll
+            for (int b = 0; b < 2; ++b) {
+                const uint32_t w8[8] = {raw.q[2 * b].x, raw.q[2 * b].y, raw.q[2 * b].z, raw.q[2 * b].w,
+                                        raw.q[2 * b + 1].x, raw.q[2 * b + 1].y, raw.q[2 * b + 1].z,
+                                        raw.q[2 * b + 1].w};
+                const __half2 d = b ? d1 : d0;
+#pragma unroll
+                for (int i = 0; i < 8; ++i) {
+                    uint32_t lo, hi;
+                    bytes_to_h2x2(w8[i] ^ 0x80808080u, lo, hi);
+                    o[16 * b + 2 * i] = h2_bits(__hmul2(__hsub2(bits_h2(lo), off), d));
+                    o[16 * b + 2 * i + 1] = h2_bits(__hmul2(__hsub2(bits_h2(hi), off), d));
+                }
+            }
+        } else {
+            const __half2 off = __float2half2_rn(1032.f);          // 1024 + 8
+#pragma unroll
+            for (int b = 0; b < 2; ++b) {
+                const uint32_t w4[4] = {raw.q[b].x, raw.q[b].y, raw.q[b].z, raw.q[b].w};
+                const __half2 d = b ? d1 : d0;
+#pragma unroll
+                for (int i = 0; i < 4; ++i) {
+                    uint32_t lo, hi;
+                    bytes_to_h2x2(w4[i] & 0x0F0F0F0Fu, lo, hi);           // elements 4i .. 4i+3
+                    o[16 * b + 2 * i] = h2_bits(__hmul2(__hsub2(bits_h2(lo), off), d));
+                    o[16 * b + 2 * i + 1] = h2_bits(__hmul2(__hsub2(bits_h2(hi), off), d));
+                    bytes_to_h2x2((w4[i] >> 4) & 0x0F0F0F0Fu, lo, hi);    // elements 16+4i ..
+                    o[16 * b + 8 + 2 * i] = h2_bits(__hmul2(__hsub2(bits_h2(lo), off), d));
+                    o[16 * b + 8 + 2 * i + 1] = h2_bits(__hmul2(__hsub2(bits_h2(hi), off), d));
+                }
+            }
+        }
+    } else if (KIND == G_UPROJ) {
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+            const uint32_t w4[4] = {raw.q[i].x, raw.q[i].y, raw.q[i].z, raw.q[i].w};
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+                const float2 f = bf16x2_to_f32x2(w4[j]);
+                o[4 * i + j] = h2_bits(__floats2half2_rn(f.x, f.y));
+            }
+        }
+    } else {
+        // NVFP4: E2M1 x E4M3 is exact in fp16; the tensor scale is applied in the epilogue
+        uint32_t sc01, sc23;
+        asm("{\n\t.reg .b16 a, b;\n\tmov.b32 {a, b}, %2;\n\t"
+            "cvt.rn.f16x2.e4m3x2 %0, a;\n\tcvt.rn.f16x2.e4m3x2 %1, b;\n\t}"
+            : "=r"(sc01), "=r"(sc23)
+            : "r"(raw.s));
+        const __half2 s[4] = {__low2half2(bits_h2(sc01)), __high2half2(bits_h2(sc01)), __low2half2(bits_h2(sc23)),
+                              __high2half2(bits_h2(sc23))};
+#pragma unroll
+        for (int c = 0; c < 2; ++c) {
+            const uint32_t w4[4] = {raw.q[c].x, raw.q[c].y, raw.q[c].z, raw.q[c].w};
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                uint32_t h[4];
+                e2m1x8_to_f16x8(w4[i], h);
+                const __half2 sc = s[2 * c + (i >> 1)];
+#pragma unroll
+                for (int j = 0; j < 4; ++j) o[16 * c + 4 * i + j] = h2_bits(__hmul2(bits_h2(h[j]), sc));
+            }
+        }
+    }
+}
+
+// Row r of a 128-byte-swizzled K-major tile: 16-byte chunk c at (c ^ (r & 7)).
+__device__ __forceinline__ void store_row_swizzled(uint8_t* tile, int r, const uint32_t (&o)[32]) {
+    uint8_t* row = tile + r * 128;
+#pragma unroll
+    for (int c = 0; c < 8; ++c) {
+        const uint4 v = make_uint4(o[4 * c], o[4 * c + 1], o[4 * c + 2], o[4 * c + 3]);
+        *reinterpret_cast<uint4*>(row + ((c ^ (r & 7)) << 4)) = v;
+    }
+}
+
+// ---------------------------------------------------------------------------
+// epilogue
+// ---------------------------------------------------------------------------
+
+__device__ __forceinline__ float u2f(uint32_t u) { return __uint_as_float(u); }
+
+template <int KIND, int NT>
+__device__ __forceinline__ void epilogue_chunk(const PrefillParams& p, const TileRef& t, int warp, int lane, int c0,
+                                               const uint32_t (&r)[32], float* xchg) {
+    const int row = 32 * warp + lane;      // accumulator row (TMEM lane)
+    const int ncol = min(32, t.n - c0);
+    if (KIND == G_ROUTER) {
+        const int e = t.m0 + row;
+        const float b = p.router_b ? __ldg(p.router_b + e) : 0.f;
+        for (int j = 0; j < ncol; ++j) p.logits[(size_t)(t.b0 + c0 + j) * p.E + e] = u2f(r[j]) + b;
+    } else if (KIND == G_DPROJ) {
+        const int l = t.m0 + row;
+        const int g = t.mat;
+        for (int j = 0; j < ncol; ++j) {
+            const int tok = t.b0 + c0 + j;
+            uint32_t mask = __ldg(p.tgmask + (size_t)tok * p.G + g);
+            if (mask == 0) continue;
+            const __half v = __float2half_rn(u2f(r[j]));
+            while (mask) {
+                const int k = __ffs(mask) - 1;
+                mask &= mask - 1;
+                const int slot = __ldg(p.pair_slot + (size_t)tok * p.K + k);
+                p.hperm[(size_t)slot * p.L + l] = v;
+            }
+        }
+    } else if (KIND == G_GATEUP || KIND == G_SHARED_GATEUP) {
+        // rows 0-63: gate, rows 64-127: up (warps 2, 3 hand theirs to warps 0, 1)
+        if (warp >= 2) {
+#pragma unroll
+            for (int j = 0; j < 32; ++j) xchg[j * 64 + (row - 64)] = u2f(r[j]);
+        }
+        named_bar_sync(1, 128);
+        if (warp < 2) {
+            float tg = 1.f, tu = 1.f;
+            if (KIND == G_GATEUP) {
+                const size_t nq = (size_t)p.L * p.F / 2, ns = (size_t)p.L * p.F / 16;
+                const float* tail = reinterpret_cast<const float*>(p.experts + (size_t)t.mat * p.rec_bytes + 3 * nq + 3 * ns);
+                tg = __ldg(tail);
+                tu = __ldg(tail + 1);
+            }
+            const int f = t.m0 + row;
+            for (int j = 0; j < ncol; ++j) {
+                const float a = u2f(r[j]) * tg;
+                const float u = xchg[j * 64 + row] * tu;
+                const __half z = __float2half_rn(silu(a) * u);
+                if (KIND == G_GATEUP) p.zperm[(size_t)(t.b0 + c0 + j) * p.F + f] = z;
+                else p.zsh[(size_t)(t.b0 + c0 + j) * p.Fs + f] = z;
+            }
+        }
+        named_bar_sync(1, 128);
+    } else if (KIND == G_DOWN) {
+        const size_t nq = (size_t)p.L * p.F / 2, ns = (size_t)p.L * p.F / 16;
+        const float td = __ldg(reinterpret_cast<const float*>(p.experts + (size_t)t.mat * p.rec_bytes + 3 * nq + 3 * ns) + 2);
+        const int l = t.m0 + row;
+        for (int j = 0; j < ncol; ++j) {
+            const int slot = t.b0 + c0 + j;
+            const float w = __ldg(p.w + __ldg(p.slot_pair + slot));
+            p.operm[(size_t)slot * p.L + l] = __float2half_rn(u2f(r[j]) * td * w);
+        }
+    } else {  // UPROJ
+        const int hrow = t.m0 + row;
+        for (int j = 0; j < ncol; ++j) {
+            const int tok = t.b0 + c0 + j;
+            float v = u2f(r[j]);
+            if (p.residual) v += bf16_bits_to_f32(__ldg(p.residual + (size_t)tok * p.H + hrow));
+            p.y[(size_t)tok * p.H + hrow] = f32_to_bf16_bits(v);
+        }
+    }
+}
+
+// ---------------------------------------------------------------------------
+// the GEMM kernel
+// ---------------------------------------------------------------------------
+
+template <int NT, int STAGES>
+struct SmemPlan {
+    static constexpr int kA = 128 * 128;                 // bytes per A stage (128 rows x 64 x 16-bit)
+    static constexpr int kB = NT * 128;                  // bytes per B stage
+    static constexpr int kXchg = 32 * 64 * 4;            // gate/up exchange
+    static constexpr int kBars = (3 * STAGES + 5) * 8;
+    static constexpr int kTotal = 1024 /*alignment slack*/ + STAGES * (kA + kB) + kXchg + kBars + 16;
+};
+
+template <int KIND, int NT, int STAGES>
+__global__ void __launch_bounds__(288, 1) k_umma_gemm(const __grid_constant__ TmaMaps maps, const PrefillParams p) {
+    using S = Sched<KIND, NT>;
+    using Plan = SmemPlan<NT, STAGES>;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
+    uint8_t* sA = smem;
+    uint8_t* sB = smem + STAGES * Plan::kA;
+    float* xchg = reinterpret_cast<float*>(sB + STAGES * Plan::kB);
+    uint64_t* bars = reinterpret_cast<uint64_t*>(reinterpret_cast<uint8_t*>(xchg) + Plan::kXchg);
+    uint64_t* full_a = bars;
+    uint64_t* full_b = bars + STAGES;
+    uint64_t* empty = bars + 2 * STAGES;
+    uint64_t* tfull = bars + 3 * STAGES;
+    uint64_t* tempty = tfull + 2;
+    uint64_t* final_bar = tempty + 2;
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(final_bar + 1);
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    constexpr uint32_t kTmemCols = 2 * NT;
+
+    if (threadIdx.x == 256) {
+        for (int s = 0; s < STAGES; ++s) {
+            mbar_init(&full_a[s], 128);
+            mbar_init(&full_b[s], 1);
+            mbar_init(&empty[s], 1);
+        }
+        for (int a = 0; a < 2; ++a) {
+            mbar_init(&tfull[a], 1);
+            mbar_init(&tempty[a], 128);
+        }
+        mbar_init(final_bar, 1);
+        *abort_flag = 0;
+        fence_barrier_init();
+    }
+    if (warp == 8) {
+        tmem_alloc(tmem_slot, kTmemCols);
+        tmem_relinquish();
+    }
+    if (threadIdx.x == 128) tma_prefetch_desc(&maps.b);
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem_base = *tmem_slot;
+
+    if (warp >= 4 && warp < 8) {
+        // ------------------------------------------------------------ producers
+        const int r = threadIdx.x - 128;           // A row
+        Cursor<KIND, NT> cur, pre;
+        cur.begin(p);
+        pre = cur;
+        RawRow ring[2];
+        // prefetch the first two stages
+        if (!S::kTmaA) {
+            if (!pre.done) { load_raw<KIND, NT>(p, pre, r, ring[0]); pre.next_stage(p); }
+            if (!pre.done) { load_raw<KIND, NT>(p, pre, r, ring[1]); pre.next_stage(p); }
+        }
+        uint32_t it = 0;
+        uint32_t last_phase[STAGES];
+#pragma unroll
+        for (int s = 0; s < STAGES; ++s) last_phase[s] = 0xFFFFFFFFu;
+        while (!cur.done) {
+#pragma unroll
+            for (int slot = 0; slot < 2; ++slot) {
+                if (cur.done) break;
+                const int s = it % STAGES;
+                const uint32_t ph = (it / STAGES) & 1;
+                if (!mbar_wait(&empty[s], ph ^ 1, abort_flag, kWaitLimitNs)) goto producer_abort;
+                if (r == 0) {
+                    // activation operand (and plain bf16 weights) by TMA
+                    const int k0 = cur.ks * 64;
+                    uint32_t bytes = Plan::kB + (S::kTmaA ? Plan::kA : 0);
+                    mbar_arrive_expect_tx(&full_b[s], bytes);
+                    uint8_t* dB = sB + s * Plan::kB;
+                    if (KIND == G_UPROJ && cur.seg < p.G) tma_load_3d(dB, &maps.b, &full_b[s], k0, cur.seg, cur.t.b0);
+                    else if (cur.seg > 0) tma_load_2d(dB, &maps.b2, &full_b[s], k0, cur.t.b0);
+                    else tma_load_2d(dB, &maps.b, &full_b[s], k0, cur.t.b0);
+                    if (KIND == G_ROUTER) {
+                        tma_load_2d(sA + s * Plan::kA, &maps.a, &full_b[s], k0, cur.t.m0);
+                    } else if (KIND == G_SHARED_GATEUP) {
+                        tma_load_2d(sA + s * Plan::kA, &maps.a, &full_b[s], k0, cur.t.m0);
+                        tma_load_2d(sA + s * Plan::kA + 64 * 128, &maps.a2, &full_b[s], k0, cur.t.m0);
+                    }
+                    last_phase[s] = ph;
+                }
+                if (!S::kTmaA) {
+                    uint32_t o[32];
+                    dequant_row<KIND>(p, cur.seg, ring[slot], o);
+                    store_row_swizzled(sA + s * Plan::kA, r, o);
+                    fence_proxy_async_smem();
+                    mbar_arrive(&full_a[s]);
+                    if (!pre.done) { load_raw<KIND, NT>(p, pre, r, ring[slot]); pre.next_stage(p); }
+                }
+                cur.next_stage(p);
+                ++it;
+            }
+        }
+        goto producer_done;
+    producer_abort:
+        if (r == 0) {
+            // let every load already issued land before the CTA can leave
+            for (int s = 0; s < STAGES; ++s)
+                if (last_phase[s] != 0xFFFFFFFFu) {
+                    volatile int dummy = 0;
+                    mbar_wait(&full_b[s], last_phase[s], &dummy, kWaitLimitNs);
+                }
+        }
+    producer_done:;
+    } else if (warp == 8) {
+        // ------------------------------------------------------------ MMA issuer
+        if (lane == 0) {
+            Cursor<KIND, NT> cur;
+            cur.begin(p);
+            uint32_t it = 0, tcount = 0;
+            bool issued = false;
+            while (!cur.done) {
+                const int acc = tcount & 1;
+                const uint32_t aph = (tcount >> 1) & 1;
+                if (!mbar_wait(&tempty[acc], aph ^ 1, abort_flag, kWaitLimitNs)) break;
+                tc_fence_after();
+                const uint32_t d_tmem = tmem_base + acc * NT;
+                const int n_mma = (KIND == G_GATEUP || KIND == G_DOWN) ? ((cur.t.n + 15) & ~15) : NT;
+                const uint32_t idesc = idesc_f16(128, n_mma, S::kBf16);
+                bool first = true;
+                bool ok = true;
+                while (true) {
+                    const int s = it % STAGES;
+                    const uint32_t ph = (it / STAGES) & 1;
+                    if (!mbar_wait(&full_b[s], ph, abort_flag, kWaitLimitNs)) { ok = false; break; }
+                    if (!S::kTmaA && !mbar_wait(&full_a[s], ph, abort_flag, kWaitLimitNs)) { ok = false; break; }
+                    tc_fence_after();
+                    const uint64_t a_desc = sdesc_k128(smem_u32(sA + s * Plan::kA));
+                    const uint64_t b_desc = sdesc_k128(smem_u32(sB + s * Plan::kB));
+#pragma unroll
+                    for (int j = 0; j < 4; ++j)
+                        umma_f16(d_tmem, a_desc + 2 * j, b_desc + 2 * j, idesc, (first && j == 0) ? 0u : 1u);
+                    first = false;
+                    issued = true;
+                    umma_commit(&empty[s]);
+                    ++it;
+                    const bool last = cur.last_stage_of_tile(p);
+                    cur.next_stage(p);
+                    if (last) break;
+                }
+                if (!ok) break;
+                umma_commit(&tfull[acc]);
+                ++tcount;
+            }
+            if (issued) {
+                // all tensor-core work of this CTA done before TMEM is released
+                umma_commit(final_bar);
+                volatile int dummy = 0;
+                mbar_wait(final_bar, 0, &dummy, kWaitLimitNs);
+            }
+        }
+        __syncwarp();
+    } else {
+        // ------------------------------------------------------------ epilogue
+        Cursor<KIND, NT> cur;
+        cur.begin(p);
+        uint32_t tcount = 0;
+        while (!cur.done) {
+            const int acc = tcount & 1;
+            const uint32_t ph = (tcount >> 1) & 1;
+            if (!mbar_wait(&tfull[acc], ph, abort_flag, kWaitLimitNs)) break;
+            tc_fence_after();
+            const uint32_t taddr = tmem_base + ((uint32_t)(32 * warp) << 16) + acc * NT;
+            for (int c0 = 0; c0 < cur.t.n; c0 += 32) {
+                uint32_t rr[32];
+                tmem_ld_32x32b_x32(taddr + c0, rr);
+                tmem_ld_wait();
+                epilogue_chunk<KIND, NT>(p, cur.t, warp, lane, c0, rr, xchg);
+            }
+            tc_fence_before();
+            mbar_arrive(&tempty[acc]);
+            ++tcount;
+            // skip to the next tile
+            cur.next_tile(p);
+        }
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    if (*abort_flag && threadIdx.x == 0) set_status(p.ctrl, LMOE_ERR_TIMEOUT);
+    if (warp == 8) {
+        tc_fence_after();
+        tmem_dealloc(tmem_base, kTmemCols);
+    }
+}
+
+// ---------------------------------------------------------------------------
+// routing and bucketing for many tokens
+// ---------------------------------------------------------------------------
+
+// fp16 copy of the block input (RMS-normalised first when gamma is given);
+// values outside the fp16 range are reported as an invalid input.
+__global__ void k_x_to_fp16(const PrefillParams p) {
+    const int t = blockIdx.x;
+    const uint16_t* row = p.x + (size_t)t * p.H;
+    float scale = 1.f;
+    if (p.gamma) {
+        __shared__ float red[32];
+        float ss = 0.f;
+        for (int k = threadIdx.x; k < p.H; k += blockDim.x) {
+            const float v = bf16_bits_to_f32(row[k]);
+            ss += v * v;
+        }
+        ss = warp_sum(ss);
+        if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = ss;
+        __syncthreads();
+        if (threadIdx.x < 32) {
+            float v = threadIdx.x < (blockDim.x >> 5) ? red[threadIdx.x] : 0.f;
+            v = warp_sum(v);
+            if (threadIdx.x == 0) red[0] = rsqrtf(v / (float)p.H + p.eps);
+        }
+        __syncthreads();
+        scale = red[0];
+    }
+    bool bad = false;
+    for (int k = threadIdx.x; k < p.H; k += blockDim.x) {
+        float v = bf16_bits_to_f32(row[k]);
+        if (p.gamma) v *= scale * bf16_bits_to_f32(p.gamma[k]);
+        bad |= !(fabsf(v) <= 65504.f);
+        p.xh[(size_t)t * p.H + k] = __float2half_rn(v);
+        if (p.xr) {
+            const uint16_t hi = f32_to_bf16_bits(v);
+            p.xr[(size_t)t * p.H + k] = hi;
+            p.xr_lo[(size_t)t * p.H + k] = f32_to_bf16_bits(v - bf16_bits_to_f32(hi));
+        }
+    }
+    if (bad) set_status(p.ctrl, LMOE_ERR_DEVICE_CHECK);
+}
+
+// softmax top-k per token from the logits (warp per token)
+__global__ void k_topk(const PrefillParams p) {
+    const int warp = (blockIdx.x * blockDim.x + threadIdx.x) >> 5, lane = threadIdx.x & 31;
+    if (warp >= p.T) return;
+    const int t = warp, E = p.E, K = p.K;
+    if (p.inject_idx) {
+        if (lane < K) {
+            p.idx[(size_t)t * K + lane] = p.inject_idx[(size_t)t * K + lane];
+            p.w[(size_t)t * K + lane] = p.inject_w[(size_t)t * K + lane];
+        }
+    } else {
+        float v[kMaxExpertsTopk / 32];
+        uint32_t taken = 0;
+#pragma unroll
+        for (int j = 0; j < kMaxExpertsTopk / 32; ++j) {
+            const int e = lane + 32 * j;
+            v[j] = e < E ? __ldcg(p.logits + (size_t)t * E + e) : -INFINITY;
+        }
+        float lmax = 0.f, denom = 0.f, my_l = 0.f;
+        int my_e = 0;
+        for (int k = 0; k < K; ++k) {
+            float bv = -INFINITY;
+            int bi = 0x7fffffff;
+#pragma unroll
+            for (int j = 0; j < kMaxExpertsTopk / 32; ++j) {
+                const int e = lane + 32 * j;
+                if (e < E && !(taken >> j & 1u) && (v[j] > bv || (v[j] == bv && e < bi))) { bv = v[j]; bi = e; }
+            }
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1) {
+                const float ov = __shfl_xor_sync(0xffffffffu, bv, o);
+                const int oi = __shfl_xor_sync(0xffffffffu, bi, o);
+                if (ov > bv || (ov == bv && oi < bi)) { bv = ov; bi = oi; }
+            }
+            if ((bi & 31) == lane && bi < E) taken |= 1u << (bi >> 5);
+            if (k == 0) lmax = bv;
+            if (k == lane) { my_l = bv; my_e = bi; }
+            denom += expf(bv - lmax);
+        }
+        if (lane < K) {
+            p.idx[(size_t)t * K + lane] = my_e;
+            p.w[(size_t)t * K + lane] = expf(my_l - lmax) / denom;
+        }
+    }
+    if (lane < K) {
+        if (p.out_idx) p.out_idx[(size_t)t * K + lane] = p.idx[(size_t)t * K + lane];
+        if (p.out_w) p.out_w[(size_t)t * K + lane] = p.w[(size_t)t * K + lane];
+    }
+}
+
+// counts per expert, group masks per token, hit flags per token tile
+__global__ void k_bucket_count(const PrefillParams p) {
+    const int i = blockIdx.x * blockDim.x + threadIdx.x;
+    if (i >= p.T * p.K) return;
+    const int t = i / p.K, k = i - t * p.K;
+    int e = p.idx[i];
+    if (e < 0 || e >= p.E) { set_status(p.ctrl, LMOE_ERR_DEVICE_CHECK); e = 0; p.idx[i] = 0; }
+    int g = p.group[e];
+    if (g >= p.G) { set_status(p.ctrl, LMOE_ERR_DEVICE_CHECK); g = 0; }
+    atomicAdd(p.cnt + e, 1);
+    atomicOr(p.tgmask + (size_t)t * p.G + g, 1u << k);
+    p.dhit[(t / kNtDense) * p.G + g] = 1;
+}
+
+// offsets, distinct experts and the expert token tiles (one CTA)
+__global__ void k_bucket_scan(const PrefillParams p) {
+    __shared__ int scratch[32];
+    const int E = p.E;
+    const int per = (E + blockDim.x - 1) / blockDim.x;
+    const int e_lo = threadIdx.x * per, e_hi = min(E, e_lo + per);
+    int c = 0, f = 0, nt = 0;
+    for (int e = e_lo; e < e_hi; ++e) {
+        const int ce = p.cnt[e];
+        c += ce;
+        f += ce > 0;
+        nt += (ce + kNtExpert - 1) / kNtExpert;
+    }
+    int off0, u0, t0;
+    block_exclusive_scan(c, &off0, scratch);
+    const int n_unique = block_exclusive_scan(f, &u0, scratch);
+    const int n_tiles = block_exclusive_scan(nt, &t0, scratch);
+    for (int e = e_lo, o = off0, u = u0, tt = t0; e < e_hi; ++e) {
+        const int ce = p.cnt[e];
+        p.off[e] = o;
+        if (ce > 0) {
+            p.uexp[u] = e;
+            p.ucnt[u] = ce;
+            p.uoff[u] = o;
+            for (int n0 = 0; n0 < ce; n0 += kNtExpert) p.etile[tt++] = make_int2(u, n0);
+            ++u;
+        }
+        o += ce;
+    }
+    if (threadIdx.x == 0) {
+        *p.n_unique = n_unique;
+        *p.n_etiles = n_tiles;
+    }
+}
+
+__global__ void k_bucket_scatter(const PrefillParams p) {
+    const int i = blockIdx.x * blockDim.x + threadIdx.x;
+    if (i >= p.T * p.K) return;
+    const int e = p.idx[i];
+    const int slot = p.off[e] + atomicAdd(p.fill + e, 1);
+    p.slot_pair[slot] = i;
+    p.pair_slot[i] = slot;
+}
+
+// s[t][g] = sum over the token's experts of group g of o (already weighted);
+// zero for groups the token does not hit.  One CTA per token, 16 bytes per thread.
+__global__ void k_combine(const PrefillParams p) {
+    const int t = blockIdx.x;
+    const int nchunk = p.L / 8;
+    for (int g = 0; g < p.G; ++g) {
+        const uint32_t mask = __ldg(p.tgmask + (size_t)t * p.G + g);
+        for (int c = threadIdx.x; c < nchunk; c += blockDim.x) {
+            float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+            uint32_t m = mask;
+            while (m) {
+                const int k = __ffs(m) - 1;
+                m &= m - 1;
+                const int slot = __ldg(p.pair_slot + (size_t)t * p.K + k);
+                const uint4 v = __ldcg(reinterpret_cast<const uint4*>(p.operm + (size_t)slot * p.L) + c);
+                const uint32_t w4[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+                for (int j = 0; j < 4; ++j) {
+                    const float2 f = __half22float2(bits_h2(w4[j]));
+                    acc[2 * j] += f.x;
+                    acc[2 * j + 1] += f.y;
+                }
+            }
+            uint4 out;
+            out.x = h2_bits(__floats2half2_rn(acc[0], acc[1]));
+            out.y = h2_bits(__floats2half2_rn(acc[2], acc[3]));
+            out.z = h2_bits(__floats2half2_rn(acc[4], acc[5]));
+            out.w = h2_bits(__floats2half2_rn(acc[6], acc[7]));
+            reinterpret_cast<uint4*>(p.s + ((size_t)t * p.G + g) * p.L)[c] = out;
+        }
+    }
+}
+
+// ---------------------------------------------------------------------------
+// host side: tensor maps and the launch sequence
+// ---------------------------------------------------------------------------
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+static EncodeTiledFn encode_fn() {
+    static EncodeTiledFn fn = nullptr;
+    if (!fn) {
+        void* ptr = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<EncodeTiledFn>(ptr);
+    }
+    return fn;
+}
+
+// 2-D map over a row-major [rows][cols] 16-bit matrix, box = 64 columns x box_rows.
+static bool make_map_2d(CUtensorMap* m, const void* base, bool bf16, uint64_t rows, uint64_t cols, uint64_t row_stride_elems,
+                        uint32_t box_rows) {
+    EncodeTiledFn fn = encode_fn();
+    if (!fn) return false;
+    cuuint64_t dims[2] = {cols, rows};
+    cuuint64_t strides[1] = {row_stride_elems * 2};
+    cuuint32_t box[2] = {64, box_rows};
+    cuuint32_t es[2] = {1, 1};
+    return fn(m, bf16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, const_cast<void*>(base),
+              dims, strides, box, es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// 3-D map over s [T][G][L] fp16, box = 64 x 1 x box_rows.
+static bool make_map_s(CUtensorMap* m, const void* base, uint64_t T, uint64_t G, uint64_t L, uint32_t box_rows) {
+    EncodeTiledFn fn = encode_fn();
+    if (!fn) return false;
+    cuuint64_t dims[3] = {L, G, T};
+    cuuint64_t strides[2] = {L * 2, G * L * 2};
+    cuuint32_t box[3] = {64, 1, box_rows};
+    cuuint32_t es[3] = {1, 1, 1};
+    return fn(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 3, const_cast<void*>(base), dims, strides, box, es,
+              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+static int g_num_sms = 0;
+
+template <int KIND, int NT, int STAGES>
+static cudaError_t launch_gemm(const TmaMaps& maps, const PrefillParams& p, cudaStream_t st, int max_tiles) {
+    const size_t smem = SmemPlan<NT, STAGES>::kTotal;
+    auto kern = k_umma_gemm<KIND, NT, STAGES>;
+    cudaError_t e = ensure_smem(reinterpret_cast<const void*>(kern), smem);
+    if (e != cudaSuccess) return e;
+    if (g_num_sms == 0) {
+        int dev = 0;
+        cudaGetDevice(&dev);
+        cudaDeviceGetAttribute(&g_num_sms, cudaDevAttrMultiProcessorCount, dev);
+    }
+    const int grid = max(1, min(g_num_sms, max_tiles));
+    kern<<<grid, 288, smem, st>>>(maps, p);
+    return cudaGetLastError();
+}
+
+cudaError_t run_prefill_path(PrefillParams p, cudaStream_t st, void* memset_base, size_t memset_bytes,
+                             void (*mark)(cudaStream_t)) {
+    const int T = p.T, H = p.H, L = p.L, G = p.G, F = p.F, Fs = p.Fs, K = p.K, E = p.E;
+    cudaError_t e;
+    const int ttiles = (T + kNtDense - 1) / kNtDense;
+    TmaMaps m_router, m_shared, m_d, m_gu, m_down, m_u;
+    std::memset(&m_router, 0, sizeof(TmaMaps));
+    m_shared = m_d = m_gu = m_down = m_u = m_router;
+    (void)mark;
+    bool ok = true;
+    ok &= make_map_2d(&m_router.a, p.router_w_bf16, true, E, H, H, 128);
+    ok &= make_map_2d(&m_router.b, p.xr ? (const void*)p.xr : (const void*)p.x, true, T, H, H, kNtDense);
+    ok &= make_map_2d(&m_shared.a, p.sg, true, Fs, H, H, 64);
+    ok &= make_map_2d(&m_shared.a2, p.su, true, Fs, H, H, 64);
+    ok &= make_map_2d(&m_shared.b, p.xr ? (const void*)p.xr : (const void*)p.x, true, T, H, H, kNtDense);
+    if (p.xr) {
+        ok &= make_map_2d(&m_router.b2, p.xr_lo, true, T, H, H, kNtDense);
+        ok &= make_map_2d(&m_shared.b2, p.xr_lo, true, T, H, H, kNtDense);
+    }
+    ok &= make_map_2d(&m_d.b, p.xh, false, T, H, H, kNtDense);
+    ok &= make_map_2d(&m_gu.b, p.hperm, false, (uint64_t)T * K, L, L, kNtExpert);
+    ok &= make_map_2d(&m_down.b, p.zperm, false, (uint64_t)T * K, F, F, kNtExpert);
+    ok &= make_map_s(&m_u.b, p.s, T, G, L, kNtDense);
+    ok &= make_map_2d(&m_u.b2, p.zsh, false, T, Fs, Fs, kNtDense);
+    if (!ok) return cudaErrorInvalidValue;
+
+    if (memset_bytes) {
+        e = cudaMemsetAsync(memset_base, 0, memset_bytes, st);
+        if (e != cudaSuccess) return e;
+    }
+    mark(st);
+    k_x_to_fp16<<<T, 256, 0, st>>>(p);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    mark(st);
+    if ((e = launch_gemm<G_ROUTER, kNtDense, 4>(m_router, p, st, (E / 128) * ttiles)) != cudaSuccess) return e;
+    mark(st);
+    k_topk<<<(T * 32 + 255) / 256, 256, 0, st>>>(p);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    const int pairs = T * K;
+    k_bucket_count<<<(pairs + 255) / 256, 256, 0, st>>>(p);
+    k_bucket_scan<<<1, 1024, 0, st>>>(p);
+    k_bucket_scatter<<<(pairs + 255) / 256, 256, 0, st>>>(p);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    mark(st);
+    if ((e = launch_gemm<G_SHARED_GATEUP, kNtDense, 4>(m_shared, p, st, (Fs / 64) * ttiles)) != cudaSuccess) return e;
+    mark(st);
+    if ((e = launch_gemm<G_DPROJ, kNtDense, 4>(m_d, p, st, G * (L / 128) * ttiles)) != cudaSuccess) return e;
+    mark(st);
+    const int max_etiles = min(E, pairs) + pairs / kNtExpert + 1;
+    if ((e = launch_gemm<G_GATEUP, kNtExpert, 6>(m_gu, p, st, (F / 64) * max_etiles)) != cudaSuccess) return e;
+    mark(st);
+    if ((e = launch_gemm<G_DOWN, kNtExpert, 6>(m_down, p, st, (L / 128) * max_etiles)) != cudaSuccess) return e;
+    mark(st);
+    k_combine<<<T, 256, 0, st>>>(p);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    mark(st);
+    if ((e = launch_gemm<G_UPROJ, kNtDense, 4>(m_u, p, st, (H / 128) * ttiles)) != cudaSuccess) return e;
+    mark(st);
+    return cudaSuccess;
+}
+
+// Router only (logits GEMM + top-k) for many tokens.
+cudaError_t run_prefill_route(PrefillParams p, cudaStream_t st) {
+    TmaMaps m;
+    std::memset(&m, 0, sizeof(m));
+    bool ok = make_map_2d(&m.a, p.router_w_bf16, true, p.E, p.H, p.H, 128);
+    ok &= make_map_2d(&m.b, p.x, true, p.T, p.H, p.H, kNtDense);
+    if (!ok) return cudaErrorInvalidValue;
+    const int ttiles = (p.T + kNtDense - 1) / kNtDense;
+    cudaError_t e = launch_gemm<G_ROUTER, kNtDense, 4>(m, p, st, (p.E / 128) * ttiles);
+    if (e != cudaSuccess) return e;
+    k_topk<<<(p.T * 32 + 255) / 256, 256, 0, st>>>(p);
+    return cudaGetLastError();
+}
+
+}  // namespace lmoe

@@ -205,3 +205,76 @@ def test_stack_layers_against_oracle_layer_by_layer():
         assert np.all(gap >= GAP)
         assert_close(bf16_bits_to_f64(y), y_ref, f"stack layer {l}")
         cur = y.cpu().numpy().view(np.uint16)
+
+
+# ----------------------------------------------------------------------------
+# many tokens: the tensor-core path (every row compared)
+# ----------------------------------------------------------------------------
+
+def prefill_workload(T, seed=5, **kw):
+    shape = synth.LayerShape(hidden=256, latent=128, n_experts=128, top_k=6, n_groups=4, ffn=128, shared_ffn=64,
+                             du_fmt=synth.Q8_0, router_dtype="bf16")
+    return synth.Workload("prefill_small", synth.replace(shape, **kw), T=T, seed=seed, groups="uniform",
+                          bias_sigma=0.5, weight_sigma=0.05)
+
+
+@pytest.mark.parametrize("T", [64, 300, 777])
+def test_prefill_path_small_shape_all_rows(T):
+    wl = prefill_workload(T)
+    check_block(wl.shape, synth.make_layer(wl), synth.make_x(wl), what=f"prefill T={T}")
+
+
+@pytest.mark.parametrize("fmt", [synth.Q8_0, synth.Q4_0])
+def test_prefill_path_formats_with_residual(fmt):
+    wl = prefill_workload(260, du_fmt=fmt, latent=256)
+    res = synth.bf16_normal(synth.key(2, 0, "residual"), 1.0, (260, wl.shape.hidden))
+    check_block(wl.shape, synth.make_layer(wl), synth.make_x(wl), residual_bits=res, what=f"prefill fmt={fmt}")
+
+
+def test_prefill_path_skewed_expert_spans_several_tiles():
+    """One expert takes every token (several 128-slot tiles of the expert GEMMs)."""
+    wl = prefill_workload(400)
+    layer = synth.make_layer(wl)
+    layer["router_b"][7] = 40.0
+    out = check_block(wl.shape, layer, synth.make_x(wl), what="skewed")
+    assert np.all(out["idx_gpu"][:, 0] == 7)
+
+
+def test_prefill_route_matches_oracle():
+    wl = prefill_workload(500)
+    layer = synth.make_layer(wl)
+    dev = DeviceLayer(wl.shape, layer)
+    xb = synth.make_x(wl)
+    idx, w = dev.route(to_device(xb, "cuda"), dev.workspace(500))
+    W = orc.Weights(wl.shape, layer)
+    idx_r, w_r, gap, _ = orc.route(orc.bf16_to_f64(xb), W.Wr, W.b, wl.shape.top_k)
+    assert check_routing(idx.cpu().numpy(), w.cpu().numpy(), idx_r, w_r, gap) >= 490
+
+
+def test_prefill_stack_layers():
+    wl = prefill_workload(130).with_(n_layers=2)
+    s = wl.shape
+    layers = [synth.make_layer(wl, layer=l) for l in range(2)]
+    gammas = [synth.bf16_bits_from_f32(np.linspace(0.5, 1.5, s.hidden).astype(np.float32) + 0.2 * l) for l in range(2)]
+    devs = [DeviceLayer(s, ly, gamma=g) for ly, g in zip(layers, gammas)]
+    xb = synth.make_x(wl)
+    x = to_device(xb, "cuda")
+    ws = devs[0].workspace(wl.T)
+    cur = xb
+    for l in range(2):
+        y = torch.empty_like(x)
+        B.lmoe_stack_forward(devs[0].cfg, [d.as_c_layer() for d in devs[:l + 1]], x, y, wl.T, 1e-6, ws)
+        torch.cuda.synchronize()
+        y_ref, _, _, gap = orc.stack_layer_forward(s, layers[l], cur, orc.bf16_to_f64(gammas[l]), 1e-6)
+        assert np.all(gap >= GAP)
+        assert_close(bf16_bits_to_f64(y), y_ref, f"prefill stack layer {l}")
+        cur = y.cpu().numpy().view(np.uint16)
+    assert B.lmoe_last_device_status(ws) == B.LMOE_OK
+
+
+def test_prefill_16384_tokens_sampled():
+    """The largest configuration: 16384 tokens of the Edge0-145B-shaped layer."""
+    wl = synth.WORKLOADS["edge0_145b_prefill"].with_(T=16384)
+    layer = synth.make_layer(wl)
+    xb = synth.make_x(wl)
+    check_block(wl.shape, layer, xb, tokens=np.array([0, 5000, 16383]), what="prefill 16384")
