@@ -110,9 +110,11 @@ class ClockSampler:
 # algorithmic bytes of one step (from the routing actually taken)
 # ----------------------------------------------------------------------------
 
-def step_bytes(shape, idx: np.ndarray, groups: np.ndarray, T: int) -> dict:
-    """Bytes each kernel must move at least once: weights it reads plus its
-    activations in and out."""
+def step_cost(shape, idx: np.ndarray, groups: np.ndarray, T: int, prefill: bool) -> dict:
+    """Algorithmic bytes (few-token path) or FLOPs (tensor-core path) of each
+    kernel for one step, from the routing actually taken: the weights a kernel
+    must read at least once plus its activations in and out, or 2 x the
+    multiply-adds of the contraction it performs for the routed pairs only."""
     H, L, E, K, G, F, Fs = (shape.hidden, shape.latent, shape.n_experts, shape.top_k, shape.n_groups, shape.ffn,
                             shape.shared_ffn)
     du = L * H // 32 * (34 if shape.du_fmt == 8 else 18)
@@ -120,20 +122,38 @@ def step_bytes(shape, idx: np.ndarray, groups: np.ndarray, T: int) -> dict:
     rec_d = F * L // 2 + F * L // 16
     rw = E * H * (2 if shape.router_dtype == "bf16" else 4)
     hit = {int(groups[e]) for e in idx.reshape(-1)}
-    n_distinct = len(set(idx.reshape(-1).tolist()))
+    distinct = set(idx.reshape(-1).tolist())
+    pairs_tg = sum(len({int(groups[e]) for e in idx[t]}) for t in range(idx.shape[0]))   # hit (token, group) pairs
     b = {
         "k_router_shared": rw + 2 * Fs * H * 2 + T * H * 2,
         "k_dproj": len(hit) * du + T * H * 2,
-        "k_expert_gateup": n_distinct * rec_gu,
-        "k_expert_down": n_distinct * rec_d,
+        "k_expert_gateup": len(distinct) * rec_gu,
+        "k_expert_down": len(distinct) * rec_d,
         "k_uproj": len(hit) * du + H * Fs * 2 + 2 * T * H * 2,
     }
-    b["n_distinct"] = n_distinct
-    b["n_groups_hit"] = len(hit)
-    return b
+    f = {
+        "x_to_fp16": 0.0,
+        "router_gemm": 2.0 * T * E * H,
+        "topk_bucket": 0.0,
+        "shared_gateup": 2.0 * T * 2 * Fs * H,
+        "dproj": 2.0 * pairs_tg * L * H,
+        "gateup": 2.0 * T * K * 2 * F * L,
+        "down": 2.0 * T * K * L * F,
+        "combine": 0.0,
+        "uproj": 2.0 * pairs_tg * H * L + 2.0 * T * H * Fs,
+    }
+    weight_bytes = rw + 3 * Fs * H * 2 + len(hit) * 2 * du + len(distinct) * (rec_gu + rec_d)
+    out = dict(f if prefill else b)
+    out["bytes_total"] = weight_bytes + 2 * T * H * 2 if prefill else float(sum(b.values()))
+    out["flops_total"] = float(sum(f.values()))
+    out["n_distinct"] = len(distinct)
+    out["n_groups_hit"] = len(hit)
+    return out
 
 
 STAGES = ["k_router_shared", "k_dproj", "k_expert_gateup", "k_expert_down", "k_uproj"]
+PREFILL_STAGES = ["x_to_fp16", "router_gemm", "topk_bucket", "shared_gateup", "dproj", "gateup", "down", "combine",
+                  "uproj"]
 
 
 def workload_desc(wl, T):
@@ -252,26 +272,37 @@ def main():
         devs.append(d)
     ws = base.workspace(T)
     K, W = args.steps, args.warmup
-    n_steps = K + W
-    xs_host = [synth.make_x(wl, T=T, draw=rank * 100_003 + i) for i in range(n_steps)]
+    prefill = T >= 64 and s.router_dtype == "bf16" and s.n_experts % 128 == 0
+    stages = PREFILL_STAGES if prefill else STAGES
+    # one CUDA graph per distinct step (its own token batch, weight copy and
+    # output buffers); the timed loop replays them in turn
+    n_graphs = min(K, 8 if prefill else 64)
+    xs_host = [synth.make_x(wl, T=T, draw=rank * 100_003 + i) for i in range(n_graphs)]
     xs = [to_device(x, dev_name) for x in xs_host]
     ys = [torch.empty_like(x) for x in xs]
-    idx_all = torch.empty((n_steps, T, s.top_k), dtype=torch.int32, device=dev_name)
-    w_all = torch.empty((n_steps, T, s.top_k), dtype=torch.float32, device=dev_name)
+    idx_all = torch.empty((n_graphs, T, s.top_k), dtype=torch.int32, device=dev_name)
+    w_all = torch.empty((n_graphs, T, s.top_k), dtype=torch.float32, device=dev_name)
     stream = torch.cuda.current_stream()
 
-    def step(i):
-        d = devs[i % R]
-        B.lmoe_forward_ex(d.cfg, xs[i], d.router_w, d.router_b, d.expert_group, d.D, d.U, d.experts, d.shared,
-                          None, None, None, idx_all[i], w_all[i], ys[i], T, ws, stream)
+    def step(i, st=None):
+        g = i % n_graphs
+        d = devs[g % R]
+        B.lmoe_forward_ex(d.cfg, xs[g], d.router_w, d.router_b, d.expert_group, d.D, d.U, d.experts, d.shared,
+                          None, None, None, idx_all[g], w_all[g], ys[g], T, ws, st or torch.cuda.current_stream())
 
-    for i in range(W):
+    for i in range(max(W, n_graphs)):
         step(i)
     torch.cuda.synchronize()
+    graphs = []
+    for g in range(n_graphs):
+        cg = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(cg):
+            step(g)
+        graphs.append(cg)
+    for i in range(W):
+        graphs[i % n_graphs].replay()
+    torch.cuda.synchronize()
 
-    # per-kernel events inside the timed region
-    n_ev = len(STAGES) + 1
-    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(n_ev)] for _ in range(K)]
     start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     if world > 1:
         dist.barrier()
@@ -279,11 +310,9 @@ def main():
     with ClockSampler(local) as clk:
         start.record()
         for k in range(K):
-            B.lmoe_profile_stage_events(evs[k])
-            step(W + k)
+            graphs[(W + k) % n_graphs].replay()
         end.record()
         torch.cuda.synchronize()
-    B.lmoe_profile_stage_events([])
     if world > 1:
         dist.barrier()
     ms = start.elapsed_time(end)
@@ -292,40 +321,61 @@ def main():
         dist.all_reduce(ms_t, op=dist.ReduceOp.MAX)
     ms_max = float(ms_t.item())
     status = B.lmoe_last_device_status(ws)
+    del graphs
 
-    # per-kernel times and algorithmic bytes
-    stage_ms = np.zeros(len(STAGES))
-    for k in range(K):
-        for j in range(len(STAGES)):
+    # per-kernel durations: the same steps launched one by one with CUDA
+    # events recorded by the library between its kernels on the step's stream
+    K2 = min(K, 200)
+    n_ev = len(stages) + 1
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(n_ev)] for _ in range(K2)]
+    torch.cuda.synchronize()
+    for k in range(K2):
+        B.lmoe_profile_stage_events(evs[k])
+        step(k)
+    torch.cuda.synchronize()
+    B.lmoe_profile_stage_events([])
+    stage_ms = np.zeros(len(stages))
+    for k in range(K2):
+        for j in range(len(stages)):
             stage_ms[j] += evs[k][j].elapsed_time(evs[k][j + 1])
+    stage_ms /= K2
+
     idx_np = idx_all.cpu().numpy()
     groups = layer["expert_group"]
-    tot = {st: 0 for st in STAGES}
-    nd = []
-    for k in range(K):
-        b = step_bytes(s, idx_np[W + k], groups, T)
-        nd.append(b["n_distinct"])
-        for st in STAGES:
-            tot[st] += b[st]
-    step_alg_bytes = sum(tot.values()) / K
-    peaks = {}
+    per_graph = [step_cost(s, idx_np[g], groups, T, prefill) for g in range(n_graphs)]
+    cost = {st: float(np.mean([c[st] for c in per_graph])) for st in stages}
+    step_alg_bytes = float(np.mean([c["bytes_total"] for c in per_graph]))
+    step_flops = float(np.mean([c["flops_total"] for c in per_graph]))
+    nd = [c["n_distinct"] for c in per_graph]
     try:
         with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
             peaks = json.load(f)
-        hbm_peak, peak_src = float(peaks["hbm_gbs"]), "measured"
+        hbm_peak = float(peaks["hbm_gbs"])
+        tc_peak = float(peaks["bf16_tflops"])
+        peak_src = "measured"
     except Exception:
-        hbm_peak, peak_src = 6650.0, "fallback"
+        hbm_peak, tc_peak, peak_src = 6650.0, 1590.0, "fallback"
     dom = int(np.argmax(stage_ms))
-    dom_name = STAGES[dom]
-    dom_avg_s = stage_ms[dom] / K / 1e3
-    dom_gbs = tot[dom_name] / K / dom_avg_s / 1e9
+    dom_name = stages[dom]
+    dom_s = stage_ms[dom] / 1e3
+    if prefill:
+        dom_ach = cost[dom_name] / dom_s / 1e12
+        roof = {"bound": "tensor", "kernel": dom_name, "achieved": dom_ach, "peak": tc_peak, "unit": "TFLOP/s",
+                "frac": dom_ach / tc_peak, "peak_source": f"{peak_src} bf16 dense (fp16 operands run at the bf16 rate)",
+                "traffic": None}
+    else:
+        dom_ach = cost[dom_name] / dom_s / 1e9
+        roof = {"bound": "hbm", "kernel": dom_name, "achieved": dom_ach, "peak": hbm_peak, "unit": "GB/s",
+                "frac": dom_ach / hbm_peak, "peak_source": peak_src, "traffic": None}
+    t_step = ms_max / K / 1e3
+    t_lb = max(step_alg_bytes / (hbm_peak * 1e9), step_flops / (tc_peak * 1e12))
 
     # e2e through the host-buffer entry point (copies inside the timed region)
-    x_pin = [torch.from_numpy(x.view(np.int16)).pin_memory() for x in xs_host[:K]]
+    x_pin = [torch.from_numpy(x.view(np.int16)).pin_memory() for x in xs_host]
     y_pin = torch.empty((T, s.hidden), dtype=torch.int16).pin_memory()
     for i in range(min(W, K)):
         d = devs[i % R]
-        B.lmoe_forward_host(d.cfg, x_pin[i], d.router_w, d.router_b, d.expert_group, d.D, d.U, d.experts, d.shared,
+        B.lmoe_forward_host(d.cfg, x_pin[i % n_graphs], d.router_w, d.router_b, d.expert_group, d.D, d.U, d.experts, d.shared,
                             y_pin, T, ws, stream)
     if world > 1:
         dist.barrier()
@@ -334,7 +384,7 @@ def main():
     e0.record()
     for i in range(K):
         d = devs[i % R]
-        B.lmoe_forward_host(d.cfg, x_pin[i], d.router_w, d.router_b, d.expert_group, d.D, d.U, d.experts, d.shared,
+        B.lmoe_forward_host(d.cfg, x_pin[i % n_graphs], d.router_w, d.router_b, d.expert_group, d.D, d.U, d.experts, d.shared,
                             y_pin, T, ws, stream)
     e1.record()
     torch.cuda.synchronize()
@@ -347,23 +397,27 @@ def main():
     line = {
         "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": K, "warmup": W,
         "ms_per_step": ms_max / K, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
-        "dtype": "f32", "data": "synthetic",
+        "dtype": "f16" if prefill else "f32", "data": "synthetic",
         "config": {"workload": workload_desc(wl, T), "T": T, "parallelism": f"replicas x{world}",
                    "l2": f"inputs larger than L2: {R} weight copies rotated, "
                          f"{R * per_step_max / 1e6:.0f} MB touched between reuses",
                    "weights": "NVFP4 experts, Q8_0/Q4_0 D/U, bf16 router and shared expert; "
-                              "bf16 activations in and out, fp32 accumulation"},
-        "roofline": {"bound": "hbm", "kernel": dom_name, "achieved": dom_gbs, "peak": hbm_peak, "unit": "GB/s",
-                     "frac": dom_gbs / hbm_peak, "peak_source": peak_src, "traffic": None},
-        "layer_gbs": step_alg_bytes / (ms_max / K / 1e3) / 1e9,
-        "layer_frac_hbm": step_alg_bytes / (ms_max / K / 1e3) / 1e9 / hbm_peak,
-        "algorithmic_bytes_per_step": step_alg_bytes,
+                              "bf16 activations in and out, fp32 accumulation",
+                   "path": ("tensor cores (tcgen05): fp16 operands dequantised from the stored formats"
+                            if prefill else "CUDA-core weight streaming"),
+                   "timing": f"{n_graphs} captured CUDA graphs replayed in turn"},
+        "roofline": roof,
+        "layer": {"gbs": step_alg_bytes / t_step / 1e9, "tflops": step_flops / t_step / 1e12,
+                  "algorithmic_bytes": step_alg_bytes, "algorithmic_flops": step_flops,
+                  "roofline_time_us": t_lb * 1e6, "frac_of_roofline": t_lb / t_step},
         "distinct_experts_per_step": float(np.mean(nd)),
-        "kernels": {st: {"ms_avg": stage_ms[j] / K, "share": stage_ms[j] / stage_ms.sum(),
-                         "gbs": tot[st] / K / (stage_ms[j] / K / 1e3) / 1e9} for j, st in enumerate(STAGES)},
+        "kernels": {st: {"us_avg": 1e3 * stage_ms[j], "share": stage_ms[j] / stage_ms.sum(),
+                         ("tflops" if prefill else "gbs"): cost[st] / (stage_ms[j] / 1e3) / (1e12 if prefill else 1e9)}
+                    for j, st in enumerate(stages)},
+        "kernel_timing": f"CUDA events between the library's kernels over {K2} steps launched one by one",
         "e2e": {"value": e2e_rate, "unit": "tokens/s", "h2d_bytes_per_step": T * s.hidden * 2,
                 "d2h_bytes_per_step": T * s.hidden * 2},
-        "gpu_launches": len(STAGES) * K,
+        "gpu_launches": (len(stages) + (3 if prefill else 0)) * K,
         "clocks": clk.summary(),
         "device_status": status,
     }

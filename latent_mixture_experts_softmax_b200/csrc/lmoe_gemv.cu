@@ -320,6 +320,8 @@ __global__ void __launch_bounds__(256) k_router_shared(FwdParams p) {
     const int H = p.H;
     const bool router_cta = (int)blockIdx.x < p.n_router_ctas;
     if (!router_cta && !p.do_shared) return;
+    if (p.prefetch_l2 && blockIdx.x == 0 && p.T <= kChunk)
+        l2_prefetch_range(p.sd, (size_t)p.H * p.Fs * 2);
 
     for (int t0 = 0; t0 < p.T; t0 += NT) {
         const int nt = min(NT, p.T - t0);
@@ -489,6 +491,19 @@ __device__ void topk_and_buckets(const FwdParams& p) {
         const int slot = offs[e] + atomicAdd(&cnt[e], 1);
         r.slot_pair[slot] = i;
         r.pair_slot[i] = slot;
+    }
+    // Start streaming every weight the rest of the step reads into L2 now, in
+    // the order the kernels need them: D_g of the hit groups, the routed
+    // experts' records, U_g of the hit groups.  The later kernels then find
+    // their weights on chip while HBM stays busy across kernel boundaries.
+    if (p.prefetch_l2 && T <= kChunk) {
+        __syncthreads();
+        for (int g = 0; g < G; ++g)
+            if (gh[g]) l2_prefetch_range(p.D + (size_t)g * p.du_bytes_D, p.du_bytes_D);
+        for (int u = 0; u < n_unique; ++u)
+            l2_prefetch_range(p.experts + (size_t)__ldcg(r.uexp + u) * p.rec_bytes, p.rec_bytes);
+        for (int g = 0; g < G; ++g)
+            if (gh[g]) l2_prefetch_range(p.U + (size_t)g * p.du_bytes_U, p.du_bytes_U);
     }
 }
 
@@ -771,6 +786,7 @@ static cudaError_t run_gemv_path_nt(FwdParams p, cudaStream_t st, bool route_onl
     p.n_router_ctas = (p.E + 7) / 8;
     p.do_shared = !route_only;
     p.do_buckets = !route_only;
+    p.prefetch_l2 = !route_only;
     const int n_shared_ctas = route_only ? 0 : (p.Fs + 7) / 8;
     {
         const size_t sm = (size_t)p.H * NT * sizeof(float);

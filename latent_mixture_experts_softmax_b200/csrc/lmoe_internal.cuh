@@ -23,6 +23,19 @@ __device__ __forceinline__ float4 ldg_stream(const float4* p) {
     return v;
 }
 
+// The CTA's threads split [ptr, ptr + bytes) into 64 KiB pieces and ask the
+// TMA unit to bring each into L2 (a hint: nothing waits on it).
+__device__ __forceinline__ void l2_prefetch_range(const void* ptr, size_t bytes) {
+    constexpr size_t kPiece = 64 * 1024;
+    const char* base = static_cast<const char*>(ptr);
+    const size_t n = (bytes + kPiece - 1) / kPiece;
+    for (size_t i = threadIdx.x; i < n; i += blockDim.x) {
+        const size_t off = i * kPiece;
+        const uint32_t len = (uint32_t)min(kPiece, bytes - off) & ~15u;
+        if (len) asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(base + off), "r"(len) : "memory");
+    }
+}
+
 __device__ __forceinline__ uint16_t f32_to_bf16_bits(float v) {
     return __bfloat16_as_ushort(__float2bfloat16_rn(v));
 }
@@ -63,6 +76,7 @@ struct FwdParams {
     // launch shape of the router kernel
     int n_router_ctas, router_rows_per_warp;
     bool do_shared, do_buckets;
+    bool prefetch_l2;   // stream the step's weights into L2 ahead of use (few tokens)
 };
 
 constexpr int kMaxStageEvents = 16;
