@@ -185,6 +185,25 @@ LMOE_API int lmoe_debug_decode(int fmt, const void* blob, int rows, int cols, fl
  * the caller; n = 0 turns recording off.  At most 16 events. */
 LMOE_API int lmoe_profile_stage_events(void* const* events, int n);
 
+/* Router only, for callers that cannot call cudaMalloc (code inside a host
+ * framework that owns every device allocation, or a path where no workspace
+ * can be handed in).  Same results as lmoe_route, but the scratch lives in a
+ * fixed array of 274,432 bytes that is part of this library; every device
+ * that loads the library holds one copy until the process exits.  The paper
+ * has no counterpart to this call.
+ *   - Limits: T <= 64, n_experts <= 1024, top_k <= 16; larger sizes return
+ *     LMOE_ERR_WORKSPACE and launch nothing.
+ *   - Allocates nothing: no cudaMalloc, no cudaFree, no allocating library.
+ *   - The first call on a device looks up the array's device address (once
+ *     per device, with that device current); make that first call before
+ *     any stream capture.
+ *   - Every call on a device shares the one array and clears its control
+ *     words itself; calls that overlap on the GPU (other streams, other host
+ *     threads) race on it and must be serialised by the caller.
+ *   - topk_idx / topk_w as in lmoe_route; all pointers device memory. */
+LMOE_API int lmoe_route_noalloc(const lmoe_cfg* cfg, const void* x, const void* router_w, const float* router_b,
+                                int T, int32_t* topk_idx, float* topk_w, void* stream);
+
 #ifdef __cplusplus
 }
 #endif

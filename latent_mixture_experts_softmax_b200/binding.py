@@ -27,7 +27,8 @@ LMOE_NVFP4_DEBUG = 1
 # every symbol include/lmoe.h declares
 EXPORTS = ("lmoe_cfg_check", "lmoe_expert_record_bytes", "lmoe_du_bytes", "lmoe_workspace_bytes", "lmoe_route",
            "lmoe_forward", "lmoe_forward_ex", "lmoe_forward_host", "lmoe_stack_forward", "lmoe_last_device_status",
-           "lmoe_status_str", "lmoe_debug_decode", "lmoe_profile_stage_events")
+           "lmoe_status_str", "lmoe_debug_decode", "lmoe_profile_stage_events",
+           "lmoe_route_noalloc")
 
 
 class LmoeError(RuntimeError):
@@ -89,6 +90,8 @@ def lib() -> ctypes.CDLL:
         L.lmoe_debug_decode.restype = i32
         L.lmoe_profile_stage_events.argtypes = [ctypes.POINTER(ctypes.c_void_p), i32]
         L.lmoe_profile_stage_events.restype = i32
+        L.lmoe_route_noalloc.argtypes = [cfgp, vp, vp, vp, i32, vp, vp, vp]
+        L.lmoe_route_noalloc.restype = i32
         _lib = L
     return _lib
 
@@ -215,3 +218,9 @@ def lmoe_profile_stage_events(events) -> int:
         handles.append(ev.cuda_event)
     arr = (ctypes.c_void_p * max(1, len(handles)))(*handles)
     return _check(lib().lmoe_profile_stage_events(arr, len(handles)), "lmoe_profile_stage_events")
+
+
+def lmoe_route_noalloc(cfg, x, router_w, router_b, T, topk_idx, topk_w, stream=None):
+    """Router without a workspace (scratch is a fixed array inside the library)."""
+    return _check(lib().lmoe_route_noalloc(ctypes.byref(cfg), _ptr(x), _ptr(router_w), _ptr(router_b), T,
+                                           _ptr(topk_idx), _ptr(topk_w), _stream(stream)), "lmoe_route_noalloc")
