@@ -47,7 +47,7 @@ bool use_prefill(const lmoe_cfg& c, int T) {
 // start after the control block, so one allocation serves either.
 struct WsLayout {
     size_t ctrl, idx, w, logits, n_unique, uexp, ucnt, uoff, slot_pair, pair_slot, ghit, tghit;
-    size_t h, zsh, z, o, ypart, xio, yio, xa, xb;
+    size_t x16, h16, zsh, z16, s16, ypart, xio, yio, xa, xb;
     // tensor-core path
     size_t p_zero_begin, p_tgmask, p_cnt, p_fill, p_dhit, p_n_etiles, p_zero_end;
     size_t p_n_unique, p_off, p_uexp, p_ucnt, p_uoff, p_etile, p_slot_pair, p_pair_slot, p_idx, p_w, p_logits;
@@ -84,10 +84,11 @@ WsLayout ws_layout(const lmoe_cfg& c, int T) {
         L.pair_slot = take(TK * 4);
         L.ghit = take((size_t)c.n_groups * 4);
         L.tghit = take((size_t)Td * c.n_groups);
-        L.h = take((size_t)Td * c.n_groups * c.latent * 4);
+        L.x16 = take((size_t)Td * c.hidden * 2);
+        L.h16 = take((size_t)Td * c.n_groups * c.latent * 2);
         L.zsh = take((size_t)Td * c.shared_ffn * 4);
-        L.z = take(TK * c.ffn * 4);
-        L.o = take(TK * c.latent * 4);
+        L.z16 = take(TK * c.ffn * 2);
+        L.s16 = take((size_t)Td * c.n_groups * c.latent * 2);
         L.ypart = take((size_t)(c.n_groups + 1) * Td * c.hidden * 4);
     }
     const size_t end_decode = off;
@@ -121,7 +122,7 @@ WsLayout ws_layout(const lmoe_cfg& c, int T) {
         L.p_zperm = take(TK * c.ffn * 2);
         L.p_operm = take(TK * c.latent * 2);
         L.p_s = take((size_t)T * c.n_groups * c.latent * 2);
-        L.p_zsh = take((size_t)T * c.shared_ffn * 2);
+        L.p_zsh = take((size_t)2 * T * c.shared_ffn * 2);
     }
     L.total = std::max(off, end_decode);
     return L;
@@ -146,10 +147,11 @@ FwdParams base_params(const lmoe_cfg& c, int T, void* ws, const WsLayout& L) {
     p.r.pair_slot = reinterpret_cast<int32_t*>(b + L.pair_slot);
     p.r.ghit = reinterpret_cast<int32_t*>(b + L.ghit);
     p.r.tghit = reinterpret_cast<uint8_t*>(b + L.tghit);
-    p.h = reinterpret_cast<float*>(b + L.h);
+    p.x16 = reinterpret_cast<__half*>(b + L.x16);
+    p.h16 = reinterpret_cast<__half*>(b + L.h16);
     p.zsh = reinterpret_cast<float*>(b + L.zsh);
-    p.z = reinterpret_cast<float*>(b + L.z);
-    p.o = reinterpret_cast<float*>(b + L.o);
+    p.z16 = reinterpret_cast<__half*>(b + L.z16);
+    p.s16 = reinterpret_cast<__half*>(b + L.s16);
     p.ypart = reinterpret_cast<float*>(b + L.ypart);
     p.du_bytes_D = du_matrix_bytes(c);
     p.du_bytes_U = du_matrix_bytes(c);
@@ -224,7 +226,7 @@ int run_prefill(const lmoe_cfg& c, const FwdParams& f, const WsLayout& L, void* 
     p.zperm = reinterpret_cast<__half*>(b + L.p_zperm);
     p.operm = reinterpret_cast<__half*>(b + L.p_operm);
     p.s = reinterpret_cast<__half*>(b + L.p_s);
-    p.zsh = reinterpret_cast<__half*>(b + L.p_zsh);
+    p.zsh = reinterpret_cast<uint16_t*>(b + L.p_zsh);
     (void)c;
     stage_reset();
     return cuda_status(run_prefill_path(p, st, b + L.p_zero_begin, L.p_zero_end - L.p_zero_begin, stage_mark));

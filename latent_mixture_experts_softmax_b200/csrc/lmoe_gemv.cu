@@ -24,39 +24,85 @@
 namespace lmoe {
 
 // ---------------------------------------------------------------------------
-// activation staging: dst[k * NT + t] = act(t0 + t, k) for t < nt, 0 beyond
+// activation staging: xs[t * ld + k] = act(t0 + t, k) as fp32 for t < nt, 0
+// beyond (token-major rows padded by 4 floats so lanes reading 8 consecutive
+// columns of one row hit distinct bank pairs)
 // ---------------------------------------------------------------------------
 
-// x rows are bf16 [T][H]; with gamma != nullptr the row is RMS-normalised
-// first: gamma[k] * x[k] / sqrt(mean(x^2) + eps).
+__host__ __device__ constexpr int xs_ld(int K) { return K + 4; }
+
+// x rows are bf16 [T][H]; with gamma != nullptr the row is RMS-normalised:
+// gamma[k] * x[k] / sqrt(mean(x^2) + eps).  Every load of the CTA is issued
+// before any is used.  CTA 0 also writes the fp16 copy used by the D_g kernel.
 template <int NT>
 __device__ void stage_x(const FwdParams& p, int t0, int nt, float* xs, float* rs) {
-    const int H = p.H;
-    const int tid = threadIdx.x, nthr = blockDim.x;
-    if (p.gamma != nullptr) {
-        const int warp = tid >> 5, lane = tid & 31;
-        for (int t = warp; t < NT; t += nthr >> 5) {
-            float ss = 0.f;
-            if (t < nt) {
-                const uint16_t* row = p.x + (size_t)(t0 + t) * H;
-                for (int k = lane; k < H; k += 32) {
-                    float v = bf16_bits_to_f32(row[k]);
-                    ss += v * v;
-                }
+    const int H = p.H, ld = xs_ld(H);
+    const int nc = H / 8;                     // 16-byte chunks per row
+    __shared__ float ssq[NT][32];
+    float part[NT];
+#pragma unroll
+    for (int t = 0; t < NT; ++t) part[t] = 0.f;
+    for (int c = threadIdx.x; c < nc; c += blockDim.x) {
+        uint4 v[NT];
+#pragma unroll
+        for (int t = 0; t < NT; ++t)
+            v[t] = t < nt ? __ldg(reinterpret_cast<const uint4*>(p.x + (size_t)(t0 + t) * H) + c) : make_uint4(0, 0, 0, 0);
+#pragma unroll
+        for (int t = 0; t < NT; ++t) {
+            const uint32_t w4[4] = {v[t].x, v[t].y, v[t].z, v[t].w};
+            float f[8];
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+                const float2 q = bf16x2_to_f32x2(w4[j]);
+                f[2 * j] = q.x;
+                f[2 * j + 1] = q.y;
             }
-            ss = warp_sum(ss);
-            if (lane == 0) rs[t] = rsqrtf(ss / (float)H + p.eps);
+#pragma unroll
+            for (int j = 0; j < 8; ++j) part[t] = fmaf(f[j], f[j], part[t]);
+            *reinterpret_cast<float4*>(xs + t * ld + 8 * c) = make_float4(f[0], f[1], f[2], f[3]);
+            *reinterpret_cast<float4*>(xs + t * ld + 8 * c + 4) = make_float4(f[4], f[5], f[6], f[7]);
+        }
+    }
+    if (p.gamma != nullptr) {
+        const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, nw = blockDim.x >> 5;
+#pragma unroll
+        for (int t = 0; t < NT; ++t) {
+            const float v = warp_sum(part[t]);
+            if (lane == 0) ssq[t][warp] = v;
         }
         __syncthreads();
-    }
-    for (int i = tid; i < NT * H; i += nthr) {
-        const int t = i / H, k = i - t * H;
-        float v = 0.f;
-        if (t < nt) {
-            v = bf16_bits_to_f32(p.x[(size_t)(t0 + t) * H + k]);
-            if (p.gamma != nullptr) v *= rs[t] * bf16_bits_to_f32(p.gamma[k]);
+        if (threadIdx.x < NT) {
+            float tot = 0.f;
+            for (int w = 0; w < nw; ++w) tot += ssq[threadIdx.x][w];
+            rs[threadIdx.x] = rsqrtf(tot / (float)H + p.eps);
         }
-        xs[k * NT + t] = v;
+        __syncthreads();
+        for (int c = threadIdx.x; c < nc; c += blockDim.x) {
+            const uint4 gv = __ldg(reinterpret_cast<const uint4*>(p.gamma) + c);
+            const uint32_t g4[4] = {gv.x, gv.y, gv.z, gv.w};
+            float gf[8];
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+                const float2 q = bf16x2_to_f32x2(g4[j]);
+                gf[2 * j] = q.x;
+                gf[2 * j + 1] = q.y;
+            }
+#pragma unroll
+            for (int t = 0; t < NT; ++t)
+#pragma unroll
+                for (int j = 0; j < 8; ++j) xs[t * ld + 8 * c + j] *= rs[t] * gf[j];
+        }
+    }
+    if (blockIdx.x == 0 && p.x16) {
+        __syncthreads();
+        for (int i = threadIdx.x; i < nt * nc; i += blockDim.x) {
+            const int t = i / nc, c = i - t * nc;
+            const float* src = xs + t * ld + 8 * c;
+            __half2 h[4];
+#pragma unroll
+            for (int j = 0; j < 4; ++j) h[j] = __floats2half2_rn(src[2 * j], src[2 * j + 1]);
+            *reinterpret_cast<uint4*>(p.x16 + (size_t)(t0 + t) * H + 8 * c) = *reinterpret_cast<uint4*>(h);
+        }
     }
 }
 
@@ -64,107 +110,42 @@ __device__ void stage_x(const FwdParams& p, int t0, int nt, float* xs, float* rs
 // inner products of one stored row segment with NT staged activations
 // ---------------------------------------------------------------------------
 
-// 8 bf16 weights (one 16-byte load) against xs[(k0 + j) * NT + t].
+// 8 bf16 weights (one 16-byte load) against xs[t * ld + k0 + j].
 template <int NT>
-__device__ __forceinline__ void dot8_bf16(uint4 wv, const float* xs, int k0, float (&acc)[NT]) {
+__device__ __forceinline__ void dot8_bf16(uint4 wv, const float* xs, int ld, int k0, float (&acc)[NT]) {
     const uint32_t w4[4] = {wv.x, wv.y, wv.z, wv.w};
+    float w[8];
 #pragma unroll
-    for (int j2 = 0; j2 < 4; ++j2) {
-        const float2 w = bf16x2_to_f32x2(w4[j2]);
-        const float* x0 = xs + (k0 + 2 * j2) * NT;
+    for (int j = 0; j < 4; ++j) {
+        const float2 q = bf16x2_to_f32x2(w4[j]);
+        w[2 * j] = q.x;
+        w[2 * j + 1] = q.y;
+    }
 #pragma unroll
-        for (int t = 0; t < NT; ++t) acc[t] = fmaf(w.x, x0[t], acc[t]);
-#pragma unroll
-        for (int t = 0; t < NT; ++t) acc[t] = fmaf(w.y, x0[NT + t], acc[t]);
+    for (int t = 0; t < NT; ++t) {
+        const float4 a = *reinterpret_cast<const float4*>(xs + t * ld + k0);
+        const float4 b = *reinterpret_cast<const float4*>(xs + t * ld + k0 + 4);
+        acc[t] = fmaf(w[0], a.x, acc[t]);
+        acc[t] = fmaf(w[1], a.y, acc[t]);
+        acc[t] = fmaf(w[2], a.z, acc[t]);
+        acc[t] = fmaf(w[3], a.w, acc[t]);
+        acc[t] = fmaf(w[4], b.x, acc[t]);
+        acc[t] = fmaf(w[5], b.y, acc[t]);
+        acc[t] = fmaf(w[6], b.z, acc[t]);
+        acc[t] = fmaf(w[7], b.w, acc[t]);
     }
 }
 
 // 4 fp32 weights against xs.
 template <int NT>
-__device__ __forceinline__ void dot4_f32(float4 w, const float* xs, int k0, float (&acc)[NT]) {
-    const float wv[4] = {w.x, w.y, w.z, w.w};
+__device__ __forceinline__ void dot4_f32(float4 w, const float* xs, int ld, int k0, float (&acc)[NT]) {
 #pragma unroll
-    for (int j = 0; j < 4; ++j) {
-#pragma unroll
-        for (int t = 0; t < NT; ++t) acc[t] = fmaf(wv[j], xs[(k0 + j) * NT + t], acc[t]);
-    }
-}
-
-// One Q8_0 block (32 int8 in a, b; scale d) against xs[(k0 + j) * NT + t].
-template <int NT>
-__device__ __forceinline__ void dot_q8_0_regs(uint4 a, uint4 b, float d, const float* xs, int k0, float (&acc)[NT]) {
-    const uint32_t w8[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
-    float blk[NT];
-#pragma unroll
-    for (int t = 0; t < NT; ++t) blk[t] = 0.f;
-#pragma unroll
-    for (int i = 0; i < 8; ++i) {
-#pragma unroll
-        for (int j = 0; j < 4; ++j) {
-            const float wq = (float)(int8_t)((w8[i] >> (8 * j)) & 0xFF);
-            const float* xk = xs + (k0 + 4 * i + j) * NT;
-#pragma unroll
-            for (int t = 0; t < NT; ++t) blk[t] = fmaf(wq, xk[t], blk[t]);
-        }
-    }
-#pragma unroll
-    for (int t = 0; t < NT; ++t) acc[t] = fmaf(d, blk[t], acc[t]);
-}
-
-// One Q4_0 block (16 bytes: byte j = elements j (low) and j+16 (high)).
-template <int NT>
-__device__ __forceinline__ void dot_q4_0_regs(uint4 a, float d, const float* xs, int k0, float (&acc)[NT]) {
-    const uint32_t w4[4] = {a.x, a.y, a.z, a.w};
-    float blk[NT];
-#pragma unroll
-    for (int t = 0; t < NT; ++t) blk[t] = 0.f;
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-#pragma unroll
-        for (int j = 0; j < 4; ++j) {
-            const uint32_t byte = (w4[i] >> (8 * j)) & 0xFF;
-            const float lo = (float)((int)(byte & 0xF) - 8);
-            const float hi = (float)((int)(byte >> 4) - 8);
-            const float* xl = xs + (k0 + 4 * i + j) * NT;
-            const float* xh = xs + (k0 + 16 + 4 * i + j) * NT;
-#pragma unroll
-            for (int t = 0; t < NT; ++t) blk[t] = fmaf(lo, xl[t], blk[t]);
-#pragma unroll
-            for (int t = 0; t < NT; ++t) blk[t] = fmaf(hi, xh[t], blk[t]);
-        }
-    }
-#pragma unroll
-    for (int t = 0; t < NT; ++t) acc[t] = fmaf(d, blk[t], acc[t]);
-}
-
-// One 32-element NVFP4 chunk (16 bytes of codes) with the two E4M3 scales of
-// its halves (s0: elements 0..15, s1: 16..31).
-template <int NT>
-__device__ __forceinline__ void dot_nvfp4_chunk(uint4 qv, float s0, float s1, const float* xs, int k0,
-                                                float (&acc)[NT]) {
-    const uint32_t w4[4] = {qv.x, qv.y, qv.z, qv.w};
-#pragma unroll
-    for (int half = 0; half < 2; ++half) {
-        float blk[NT];
-#pragma unroll
-        for (int t = 0; t < NT; ++t) blk[t] = 0.f;
-#pragma unroll
-        for (int i = 0; i < 2; ++i) {
-            uint32_t h[4];
-            e2m1x8_to_f16x8(w4[2 * half + i], h);
-#pragma unroll
-            for (int j = 0; j < 4; ++j) {
-                const float2 v = f16x2_to_f32x2(h[j]);
-                const float* xk = xs + (k0 + 16 * half + 8 * i + 2 * j) * NT;
-#pragma unroll
-                for (int t = 0; t < NT; ++t) blk[t] = fmaf(v.x, xk[t], blk[t]);
-#pragma unroll
-                for (int t = 0; t < NT; ++t) blk[t] = fmaf(v.y, xk[NT + t], blk[t]);
-            }
-        }
-        const float s = half ? s1 : s0;
-#pragma unroll
-        for (int t = 0; t < NT; ++t) acc[t] = fmaf(s, blk[t], acc[t]);
+    for (int t = 0; t < NT; ++t) {
+        const float4 a = *reinterpret_cast<const float4*>(xs + t * ld + k0);
+        acc[t] = fmaf(w.x, a.x, acc[t]);
+        acc[t] = fmaf(w.y, a.y, acc[t]);
+        acc[t] = fmaf(w.z, a.z, acc[t]);
+        acc[t] = fmaf(w.w, a.w, acc[t]);
     }
 }
 
@@ -172,7 +153,7 @@ __device__ __forceinline__ void dot_nvfp4_chunk(uint4 qv, float s0, float s1, co
 // lanes splitting K; ten 16-byte loads per lane are issued before any
 // arithmetic.  The per-lane partial sums are left in acc (reduce with warp_sum).
 template <int NT, bool kBF16>
-__device__ __forceinline__ void row_dot(const void* wrow, int K, const float* xs, int lane, float (&acc)[NT]) {
+__device__ __forceinline__ void row_dot(const void* wrow, int K, const float* xs, int ld, int lane, float (&acc)[NT]) {
     constexpr int kB = 10;
     constexpr int kPer = kBF16 ? 8 : 4;          // elements per 16-byte load
     constexpr int kStep = 32 * kPer;
@@ -187,122 +168,12 @@ __device__ __forceinline__ void row_dot(const void* wrow, int K, const float* xs
         for (int i = 0; i < kB; ++i) {
             const int k0 = base + i * kStep + lane * kPer;
             if (k0 < K) {
-                if (kBF16) dot8_bf16<NT>(w[i], xs, k0, acc);
+                if (kBF16) dot8_bf16<NT>(w[i], xs, ld, k0, acc);
                 else dot4_f32<NT>(make_float4(__uint_as_float(w[i].x), __uint_as_float(w[i].y), __uint_as_float(w[i].z),
-                                              __uint_as_float(w[i].w)), xs, k0, acc);
+                                              __uint_as_float(w[i].w)), xs, ld, k0, acc);
             }
         }
     }
-}
-
-// Row-tile GEMV over a D/U matrix [R rows][C cols] stored as Q8_0 / Q4_0:
-// lane = row, warps split the 64-wide column groups.  Each warp takes two
-// groups per pass and issues all their loads before any arithmetic.
-template <int NT>
-__device__ __forceinline__ void du_rows(int fmt, const uint8_t* mat, int R, int C, int row, const float* xs,
-                                        float (&acc)[NT]) {
-    const int warp = threadIdx.x >> 5;
-    const int nwarps = blockDim.x >> 5;
-    const int ng = C / 64;
-    const uint16_t* dsc = reinterpret_cast<const uint16_t*>(mat + (size_t)R * C / 32 * (fmt == LMOE_Q8_0 ? 32 : 16));
-    for (int base = warp; base < ng; base += 2 * nwarps) {
-        const int kg[2] = {base, base + nwarps};
-        if (fmt == LMOE_Q8_0) {
-            uint4 q[2][4];
-            uint16_t d[2][2];
-#pragma unroll
-            for (int u = 0; u < 2; ++u) {
-                if (kg[u] < ng) {
-#pragma unroll
-                    for (int c = 0; c < 2; ++c) {
-                        const uint4* src = reinterpret_cast<const uint4*>(mat + ((size_t)(2 * kg[u] + c) * R + row) * 32);
-                        q[u][2 * c] = ldg_stream(src);
-                        q[u][2 * c + 1] = ldg_stream(src + 1);
-                        d[u][c] = __ldg(dsc + (size_t)(2 * kg[u] + c) * R + row);
-                    }
-                }
-            }
-#pragma unroll
-            for (int u = 0; u < 2; ++u) {
-                if (kg[u] < ng) {
-#pragma unroll
-                    for (int c = 0; c < 2; ++c)
-                        dot_q8_0_regs<NT>(q[u][2 * c], q[u][2 * c + 1], fp16_bits_to_f32(d[u][c]), xs,
-                                          64 * kg[u] + 32 * c, acc);
-                }
-            }
-        } else {
-            uint4 q[2][2];
-            uint16_t d[2][2];
-#pragma unroll
-            for (int u = 0; u < 2; ++u) {
-                if (kg[u] < ng) {
-#pragma unroll
-                    for (int c = 0; c < 2; ++c) {
-                        q[u][c] = ldg_stream(reinterpret_cast<const uint4*>(mat + ((size_t)(2 * kg[u] + c) * R + row) * 16));
-                        d[u][c] = __ldg(dsc + (size_t)(2 * kg[u] + c) * R + row);
-                    }
-                }
-            }
-#pragma unroll
-            for (int u = 0; u < 2; ++u) {
-                if (kg[u] < ng) {
-#pragma unroll
-                    for (int c = 0; c < 2; ++c)
-                        dot_q4_0_regs<NT>(q[u][c], fp16_bits_to_f32(d[u][c]), xs, 64 * kg[u] + 32 * c, acc);
-                }
-            }
-        }
-    }
-}
-
-// NVFP4 matrix [R rows][C cols] (codes at q, scales at s), rows as above.
-template <int NT>
-__device__ __forceinline__ void nvfp4_rows(const uint8_t* q, const uint8_t* s, int R, int C, int row,
-                                           const float* xs, float (&acc)[NT]) {
-    const int warp = threadIdx.x >> 5;
-    const int nwarps = blockDim.x >> 5;
-    const int ng = C / 64;
-    for (int base = warp; base < ng; base += 2 * nwarps) {
-        const int kg[2] = {base, base + nwarps};
-        uint4 qv[2][2];
-        uint32_t sw[2];
-#pragma unroll
-        for (int u = 0; u < 2; ++u) {
-            if (kg[u] < ng) {
-                sw[u] = __ldg(reinterpret_cast<const uint32_t*>(s + ((size_t)kg[u] * R + row) * 4));
-#pragma unroll
-                for (int c = 0; c < 2; ++c)
-                    qv[u][c] = ldg_stream(reinterpret_cast<const uint4*>(q + ((size_t)(2 * kg[u] + c) * R + row) * 16));
-            }
-        }
-#pragma unroll
-        for (int u = 0; u < 2; ++u) {
-            if (kg[u] < ng) {
-                float sc[4];
-                e4m3x4_to_f32x4(sw[u], sc);
-#pragma unroll
-                for (int c = 0; c < 2; ++c) dot_nvfp4_chunk<NT>(qv[u][c], sc[2 * c], sc[2 * c + 1], xs, 64 * kg[u] + 32 * c, acc);
-            }
-        }
-    }
-}
-
-// Sum per-warp partials red[warp][lane][t] into warp 0's acc (others get junk).
-template <int NT>
-__device__ __forceinline__ void reduce_warps(float (&acc)[NT], float* red) {
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int nwarps = blockDim.x >> 5;
-#pragma unroll
-    for (int t = 0; t < NT; ++t) red[(warp * 32 + lane) * NT + t] = acc[t];
-    __syncthreads();
-    if (warp == 0) {
-        for (int w = 1; w < nwarps; ++w) {
-#pragma unroll
-            for (int t = 0; t < NT; ++t) acc[t] += red[(w * 32 + lane) * NT + t];
-        }
-    }
-    __syncthreads();
 }
 
 // ---------------------------------------------------------------------------
@@ -333,8 +204,8 @@ __global__ void __launch_bounds__(256) k_router_shared(FwdParams p) {
                 float acc[NT];
 #pragma unroll
                 for (int t = 0; t < NT; ++t) acc[t] = 0.f;
-                if (kRouterBF16) row_dot<NT, true>(static_cast<const uint16_t*>(p.router_w) + (size_t)e * H, H, xs, lane, acc);
-                else row_dot<NT, false>(static_cast<const float*>(p.router_w) + (size_t)e * H, H, xs, lane, acc);
+                if (kRouterBF16) row_dot<NT, true>(static_cast<const uint16_t*>(p.router_w) + (size_t)e * H, H, xs, xs_ld(H), lane, acc);
+                else row_dot<NT, false>(static_cast<const float*>(p.router_w) + (size_t)e * H, H, xs, xs_ld(H), lane, acc);
                 const float b = p.router_b ? __ldg(p.router_b + e) : 0.f;
 #pragma unroll
                 for (int t = 0; t < NT; ++t) {
@@ -349,8 +220,8 @@ __global__ void __launch_bounds__(256) k_router_shared(FwdParams p) {
                 float a[NT], u[NT];
 #pragma unroll
                 for (int t = 0; t < NT; ++t) { a[t] = 0.f; u[t] = 0.f; }
-                row_dot<NT, true>(p.sg + (size_t)f * H, H, xs, lane, a);
-                row_dot<NT, true>(p.su + (size_t)f * H, H, xs, lane, u);
+                row_dot<NT, true>(p.sg + (size_t)f * H, H, xs, xs_ld(H), lane, a);
+                row_dot<NT, true>(p.su + (size_t)f * H, H, xs, xs_ld(H), lane, u);
 #pragma unroll
                 for (int t = 0; t < NT; ++t) {
                     const float av = warp_sum(a[t]), uv = warp_sum(u[t]);
@@ -508,193 +379,440 @@ __device__ void topk_and_buckets(const FwdParams& p) {
 }
 
 // ---------------------------------------------------------------------------
-// kernel 2: h[t][g] = D_g x_t
+// kernels 2-5 on the tensor pipe (mma.sync m16n8k16, fp16 operands, fp32
+// accumulation): at decode the arithmetic per weight byte, not the tensor
+// throughput, limits a CUDA-core GEMV (4-bit weights allow ~2.8 instructions
+// per weight at HBM speed; a CUDA-core dot product with the dequantisation
+// needs 4-6), so the dot products go to the tensor pipe and the CUDA cores
+// only unpack.  A warp owns 16 weight rows; the 8 token columns of the MMA
+// are the (up to 8) tokens of the pass, zero-padded.
+//
+// Fragment ownership (lane = 4 g + t): A rows g and g + 8; B column (token)
+// g; C rows g, g + 8 and columns 2t, 2t + 1.  Within a 32-element block the
+// thread feeds the k slots it owns with physical elements it loads itself;
+// the activation operand is read with the same permutation, so the sum over
+// k is unchanged.
 // ---------------------------------------------------------------------------
 
-template <int NT>
-__global__ void __launch_bounds__(512) k_dproj(FwdParams p) {
-    extern __shared__ float smem[];
-    __shared__ float rs[kChunk];
+__device__ __forceinline__ void mma16816(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
+                                         uint32_t b0, uint32_t b1) {
+    asm volatile(
+        "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, {%8, %9}, "
+        "{%0, %1, %2, %3};"
+        : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+        : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+
+__device__ __forceinline__ uint32_t hsub2_bits(uint32_t a, uint32_t b) {
+    __half2 r = __hsub2(*reinterpret_cast<__half2*>(&a), *reinterpret_cast<__half2*>(&b));
+    return *reinterpret_cast<uint32_t*>(&r);
+}
+__device__ __forceinline__ uint32_t hmul2_bits(uint32_t a, uint32_t b) {
+    __half2 r = __hmul2(*reinterpret_cast<__half2*>(&a), *reinterpret_cast<__half2*>(&b));
+    return *reinterpret_cast<uint32_t*>(&r);
+}
+
+// 4 signed int8 -> two f16x2 holding the exact integers (elements 0,1 and 2,3).
+__device__ __forceinline__ void i8x4_to_h2x2(uint32_t w, uint32_t& lo, uint32_t& hi) {
+    const uint32_t u = w ^ 0x80808080u;                   // q + 128
+    const uint32_t off = 0x64806480u;                     // fp16 1152 = 1024 + 128, twice
+    lo = hsub2_bits(__byte_perm(u, 0x64646464u, 0x4140), off);
+    hi = hsub2_bits(__byte_perm(u, 0x64646464u, 0x4342), off);
+}
+
+// 4 nibbles (in the low nibble of each byte) -> (q - 8) as two f16x2.
+__device__ __forceinline__ void u4x4_to_h2x2(uint32_t n, uint32_t& lo, uint32_t& hi) {
+    const uint32_t off = 0x64086408u;                     // fp16 1032 = 1024 + 8, twice
+    lo = hsub2_bits(__byte_perm(n, 0x64646464u, 0x4140), off);
+    hi = hsub2_bits(__byte_perm(n, 0x64646464u, 0x4342), off);
+}
+
+constexpr int kMmaWarps = 8;                      // warps per CTA: split of the reduction
+constexpr int kXPad = 32;                         // halves of padding per staged activation row
+
+// Stage 8 token rows of a 16-bit activation matrix (row stride `ld` halves,
+// K columns) into dst[8][K + kXPad]; rows at or beyond nt are zero.  Eight
+// 16-byte loads per thread are in flight before any store.
+__device__ __forceinline__ void stage_act16(__half* dst, int K, const __half* src, size_t ld, int nt) {
+    const int KP = K + kXPad;
+    const int n8 = K / 8, total = 8 * n8;
+    constexpr int kB = 8;
+    for (int i0 = threadIdx.x; i0 < total; i0 += kB * blockDim.x) {
+        uint4 v[kB];
+#pragma unroll
+        for (int u = 0; u < kB; ++u) {
+            const int i = i0 + u * blockDim.x, t = i / n8, c = i - t * n8;
+            v[u] = (i < total && t < nt) ? __ldcg(reinterpret_cast<const uint4*>(src + t * ld) + c) : make_uint4(0, 0, 0, 0);
+        }
+#pragma unroll
+        for (int u = 0; u < kB; ++u) {
+            const int i = i0 + u * blockDim.x, t = i / n8, c = i - t * n8;
+            if (i < total) *reinterpret_cast<uint4*>(dst + (size_t)t * KP + 8 * c) = v[u];
+        }
+    }
+}
+
+// Q8_0 / Q4_0 rows [r0, r0 + 16) of a matrix [R][C] against the staged
+// activations xs[8][C + kXPad], columns [kb0 * 32, kb1 * 32); acc += C frags.
+template <int FMT>
+__device__ __forceinline__ void mma_du_rows(const uint8_t* mat, int R, int C, int r0, int kb0, int kb1,
+                                            const __half* xs, float (&acc)[4]) {
+    const int lane = threadIdx.x & 31, g = lane >> 2, t = lane & 3;
+    const int KP = C + kXPad;
+    const size_t qrow = FMT == LMOE_Q8_0 ? 32 : 16;
+    const uint16_t* dsc = reinterpret_cast<const uint16_t*>(mat + (size_t)R * C / 32 * qrow);
+    const __half* xrow = xs + (size_t)g * KP;
+    constexpr int kU = 8;                                  // blocks whose loads are issued together
+    for (int kb = kb0; kb < kb1; kb += kU) {
+        uint32_t w[kU][4];
+        uint16_t d[kU][2];
+#pragma unroll
+        for (int u = 0; u < kU; ++u) {
+            if (kb + u < kb1) {
+                const size_t b = (size_t)(kb + u);
+                if (FMT == LMOE_Q8_0) {
+                    const uint2 lo = __ldg(reinterpret_cast<const uint2*>(mat + (b * R + r0 + g) * 32 + 8 * t));
+                    const uint2 hi = __ldg(reinterpret_cast<const uint2*>(mat + (b * R + r0 + g + 8) * 32 + 8 * t));
+                    w[u][0] = lo.x; w[u][1] = lo.y; w[u][2] = hi.x; w[u][3] = hi.y;
+                } else {
+                    w[u][0] = __ldg(reinterpret_cast<const uint32_t*>(mat + (b * R + r0 + g) * 16 + 4 * t));
+                    w[u][2] = __ldg(reinterpret_cast<const uint32_t*>(mat + (b * R + r0 + g + 8) * 16 + 4 * t));
+                }
+                d[u][0] = __ldg(dsc + b * R + r0 + g);
+                d[u][1] = __ldg(dsc + b * R + r0 + g + 8);
+            }
+        }
+#pragma unroll
+        for (int u = 0; u < kU; ++u) {
+            if (kb + u < kb1) {
+                const int k0 = (kb + u) * 32;
+                float c[4] = {0.f, 0.f, 0.f, 0.f};
+                if (FMT == LMOE_Q8_0) {
+                    // thread t: elements 8t .. 8t+7 of rows g and g + 8
+                    uint32_t ga0, ga1, ga2, ga3, ha0, ha1, ha2, ha3;
+                    i8x4_to_h2x2(w[u][0], ga0, ga1);
+                    i8x4_to_h2x2(w[u][1], ga2, ga3);
+                    i8x4_to_h2x2(w[u][2], ha0, ha1);
+                    i8x4_to_h2x2(w[u][3], ha2, ha3);
+                    const uint4 xv = *reinterpret_cast<const uint4*>(xrow + k0 + 8 * t);
+                    mma16816(c, ga0, ha0, ga1, ha1, xv.x, xv.y);
+                    mma16816(c, ga2, ha2, ga3, ha3, xv.z, xv.w);
+                } else {
+                    // thread t: elements 4t .. 4t+3 (low nibbles) and 16+4t .. (high)
+                    uint32_t gl0, gl1, gh0, gh1, hl0, hl1, hh0, hh1;
+                    u4x4_to_h2x2(w[u][0] & 0x0F0F0F0Fu, gl0, gl1);
+                    u4x4_to_h2x2((w[u][0] >> 4) & 0x0F0F0F0Fu, gh0, gh1);
+                    u4x4_to_h2x2(w[u][2] & 0x0F0F0F0Fu, hl0, hl1);
+                    u4x4_to_h2x2((w[u][2] >> 4) & 0x0F0F0F0Fu, hh0, hh1);
+                    const uint2 xl = *reinterpret_cast<const uint2*>(xrow + k0 + 4 * t);
+                    const uint2 xh = *reinterpret_cast<const uint2*>(xrow + k0 + 16 + 4 * t);
+                    mma16816(c, gl0, hl0, gl1, hl1, xl.x, xl.y);
+                    mma16816(c, gh0, hh0, gh1, hh1, xh.x, xh.y);
+                }
+                const float dg = fp16_bits_to_f32(d[u][0]), dh = fp16_bits_to_f32(d[u][1]);
+                acc[0] = fmaf(dg, c[0], acc[0]);
+                acc[1] = fmaf(dg, c[1], acc[1]);
+                acc[2] = fmaf(dh, c[2], acc[2]);
+                acc[3] = fmaf(dh, c[3], acc[3]);
+            }
+        }
+    }
+}
+
+// NVFP4 rows [r0, r0 + 16) of a matrix [R][C] (codes q, scales s), 32-column
+// chunks [kc0, kc1).  The E4M3 scale multiplies the E2M1 value in fp16
+// (exact); the tensor scale is left to the caller.
+__device__ __forceinline__ void mma_nvfp4_rows(const uint8_t* q, const uint8_t* s, int R, int C, int r0, int kc0,
+                                               int kc1, const __half* xs, float (&acc)[4]) {
+    const int lane = threadIdx.x & 31, g = lane >> 2, t = lane & 3;
+    const int KP = C + kXPad;
+    const __half* xrow = xs + (size_t)g * KP;
+    constexpr int kU = 8;
+    for (int kc = kc0; kc < kc1; kc += kU) {
+        uint32_t wg[kU], wh[kU], sg[kU], sh[kU];
+#pragma unroll
+        for (int u = 0; u < kU; ++u) {
+            if (kc + u < kc1) {
+                const size_t c = (size_t)(kc + u);
+                wg[u] = __ldg(reinterpret_cast<const uint32_t*>(q + (c * R + r0 + g) * 16 + 4 * t));
+                wh[u] = __ldg(reinterpret_cast<const uint32_t*>(q + (c * R + r0 + g + 8) * 16 + 4 * t));
+                sg[u] = __ldg(reinterpret_cast<const uint32_t*>(s + ((c / 2) * R + r0 + g) * 4));
+                sh[u] = __ldg(reinterpret_cast<const uint32_t*>(s + ((c / 2) * R + r0 + g + 8) * 4));
+            }
+        }
+#pragma unroll
+        for (int u = 0; u < kU; ++u) {
+            if (kc + u < kc1) {
+                const int kcu = kc + u;
+                // this thread's 8 elements (8t .. 8t+7 of the chunk) share one scale byte
+                const int sb = 2 * (kcu & 1) + (t >> 1);
+                uint32_t scg, sch;
+                {
+                    const uint32_t bg = (sg[u] >> (8 * sb)) & 0xFF, bh = (sh[u] >> (8 * sb)) & 0xFF;
+                    uint32_t hg, hh;
+                    asm("{\n\t.reg .b16 a, b;\n\tcvt.u16.u32 a, %2;\n\tcvt.u16.u32 b, %3;\n\t"
+                        "cvt.rn.f16x2.e4m3x2 %0, a;\n\tcvt.rn.f16x2.e4m3x2 %1, b;\n\t}"
+                        : "=r"(hg), "=r"(hh)
+                        : "r"(bg), "r"(bh));
+                    scg = (hg & 0xFFFF) | (hg << 16);
+                    sch = (hh & 0xFFFF) | (hh << 16);
+                }
+                uint32_t a[4], b[4];
+                e2m1x8_to_f16x8(wg[u], a);
+                e2m1x8_to_f16x8(wh[u], b);
+#pragma unroll
+                for (int j = 0; j < 4; ++j) {
+                    a[j] = hmul2_bits(a[j], scg);
+                    b[j] = hmul2_bits(b[j], sch);
+                }
+                const uint4 xv = *reinterpret_cast<const uint4*>(xrow + kcu * 32 + 8 * t);
+                mma16816(acc, a[0], b[0], a[1], b[1], xv.x, xv.y);
+                mma16816(acc, a[2], b[2], a[3], b[3], xv.z, xv.w);
+            }
+        }
+    }
+}
+
+// Sum the kMmaWarps partial C fragments into warp 0's (others get zeros).
+__device__ __forceinline__ void reduce_frags(float (&acc)[4], float* red) {
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+#pragma unroll
+    for (int i = 0; i < 4; ++i) red[(warp * 32 + lane) * 4 + i] = acc[i];
+    __syncthreads();
+    if (warp == 0) {
+        for (int w = 1; w < kMmaWarps; ++w)
+#pragma unroll
+            for (int i = 0; i < 4; ++i) acc[i] += red[(w * 32 + lane) * 4 + i];
+    }
+    __syncthreads();
+}
+
+// kernel 2: h16[t][g] = D_g x_t for hit groups; CTA = 16 rows of one group
+template <int FMT>
+__global__ void __launch_bounds__(32 * kMmaWarps) k_dproj_mma(FwdParams p) {
+    extern __shared__ __align__(16) uint8_t smem_u8[];
     const int g = blockIdx.y;
     if (__ldcg(p.r.ghit + g) == 0) return;
-    float* xs = smem;                       // [H][NT]
-    float* red = smem + (size_t)p.H * NT;   // [8][32][NT]
-    const int lane = threadIdx.x & 31;
-    const int row = blockIdx.x * 32 + lane;
+    const int H = p.H, L = p.L, r0 = blockIdx.x * 16;
+    __half* xs = reinterpret_cast<__half*>(smem_u8);
+    float* red = reinterpret_cast<float*>(smem_u8 + (size_t)8 * (H + kXPad) * 2);
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const uint8_t* Dg = p.D + (size_t)g * p.du_bytes_D;
-    for (int t0 = 0; t0 < p.T; t0 += NT) {
-        const int nt = min(NT, p.T - t0);
-        stage_x<NT>(p, t0, nt, xs, rs);
+    const int nb = H / 32, per = (nb + kMmaWarps - 1) / kMmaWarps;
+    for (int t0 = 0; t0 < p.T; t0 += 8) {
+        const int nt = min(8, p.T - t0);
+        stage_act16(xs, H, p.x16 + (size_t)t0 * H, H, nt);
         __syncthreads();
-        float acc[NT];
+        float acc[4] = {0.f, 0.f, 0.f, 0.f};
+        mma_du_rows<FMT>(Dg, L, H, r0, warp * per, min(nb, (warp + 1) * per), xs, acc);
+        reduce_frags(acc, red);
+        if (warp == 0) {
+            const int gg = lane >> 2, tt = lane & 3;
 #pragma unroll
-        for (int t = 0; t < NT; ++t) acc[t] = 0.f;
-        du_rows<NT>(p.du_fmt, Dg, p.L, p.H, row, xs, acc);
-        reduce_warps<NT>(acc, red);
-        if (threadIdx.x < 32) {
-#pragma unroll
-            for (int t = 0; t < NT; ++t)
-                if (t < nt) p.h[((size_t)(t0 + t) * p.G + g) * p.L + row] = acc[t];
+            for (int i = 0; i < 4; ++i) {
+                const int tok = 2 * tt + (i & 1), row = r0 + gg + 8 * (i >> 1);
+                if (tok < nt) p.h16[((size_t)(t0 + tok) * p.G + g) * L + row] = __float2half_rn(acc[i]);
+            }
         }
     }
 }
 
-// ---------------------------------------------------------------------------
-// kernels 3 and 4: experts (one CTA = 32 rows of one distinct expert)
-// ---------------------------------------------------------------------------
-
-template <int NT>
-__global__ void __launch_bounds__(512) k_expert_gateup(FwdParams p) {
-    extern __shared__ float smem[];
+// kernel 3: z16[slot] = silu(W_gate h) * (W_up h) for the expert's slots;
+// CTA = 16 features (gate and up rows) of one distinct expert
+__global__ void __launch_bounds__(32 * kMmaWarps) k_gateup_mma(FwdParams p) {
+    extern __shared__ __align__(16) uint8_t smem_u8[];
     const int j = blockIdx.y;
-    const int n_unique = __ldcg(p.r.n_unique);
-    if (j >= n_unique) return;
+    if (j >= __ldcg(p.r.n_unique)) return;
     const int e = __ldcg(p.r.uexp + j), cnt = __ldcg(p.r.ucnt + j), off = __ldcg(p.r.uoff + j);
     const int g = p.group[e] < p.G ? p.group[e] : 0;
-    const int L = p.L, F = p.F;
-    float* hs = smem;                        // [L][NT]
-    float* red = smem + (size_t)L * NT;      // [8][32][NT]
-    __shared__ int tok[kChunk];
-    const int lane = threadIdx.x & 31;
-    const int f = blockIdx.x * 32 + lane;
-    const uint8_t* rec = p.experts + (size_t)e * p.rec_bytes;
-    const size_t nq = (size_t)L * F / 2, ns = (size_t)L * F / 16;
-    float ts[2];
-    ts[0] = __ldg(reinterpret_cast<const float*>(rec + 3 * nq + 3 * ns));
-    ts[1] = __ldg(reinterpret_cast<const float*>(rec + 3 * nq + 3 * ns) + 1);
-    for (int c0 = 0; c0 < cnt; c0 += NT) {
-        const int nt = min(NT, cnt - c0);
-        if (threadIdx.x < NT) tok[threadIdx.x] = threadIdx.x < nt ? __ldcg(p.r.slot_pair + off + c0 + threadIdx.x) / p.K : -1;
-        __syncthreads();
-        for (int i = threadIdx.x; i < NT * L; i += blockDim.x) {
-            const int t = i / L, k = i - t * L;
-            hs[k * NT + t] = tok[t] >= 0 ? __ldcg(p.h + ((size_t)tok[t] * p.G + g) * L + k) : 0.f;
-        }
-        __syncthreads();
-        float a[NT], u[NT];
-#pragma unroll
-        for (int t = 0; t < NT; ++t) { a[t] = 0.f; u[t] = 0.f; }
-        nvfp4_rows<NT>(rec, rec + 3 * nq, F, L, f, hs, a);
-        nvfp4_rows<NT>(rec + nq, rec + 3 * nq + ns, F, L, f, hs, u);
-        reduce_warps<NT>(a, red);
-        reduce_warps<NT>(u, red);
-        if (threadIdx.x < 32) {
-#pragma unroll
-            for (int t = 0; t < NT; ++t)
-                if (t < nt) p.z[(size_t)(off + c0 + t) * F + f] = silu(a[t] * ts[0]) * (u[t] * ts[1]);
-        }
-        __syncthreads();
-    }
-}
-
-template <int NT>
-__global__ void __launch_bounds__(512) k_expert_down(FwdParams p) {
-    extern __shared__ float smem[];
-    const int j = blockIdx.y;
-    const int n_unique = __ldcg(p.r.n_unique);
-    if (j >= n_unique) return;
-    const int e = __ldcg(p.r.uexp + j), cnt = __ldcg(p.r.ucnt + j), off = __ldcg(p.r.uoff + j);
-    const int L = p.L, F = p.F;
-    float* zs = smem;                        // [F][NT]
-    float* red = smem + (size_t)F * NT;
-    const int lane = threadIdx.x & 31;
-    const int row = blockIdx.x * 32 + lane;
-    const uint8_t* rec = p.experts + (size_t)e * p.rec_bytes;
-    const size_t nq = (size_t)L * F / 2, ns = (size_t)L * F / 16;
-    const float ts = __ldg(reinterpret_cast<const float*>(rec + 3 * nq + 3 * ns) + 2);
-    for (int c0 = 0; c0 < cnt; c0 += NT) {
-        const int nt = min(NT, cnt - c0);
-        for (int i = threadIdx.x; i < NT * F; i += blockDim.x) {
-            const int t = i / F, k = i - t * F;
-            zs[k * NT + t] = t < nt ? __ldcg(p.z + (size_t)(off + c0 + t) * F + k) : 0.f;
-        }
-        __syncthreads();
-        float acc[NT];
-#pragma unroll
-        for (int t = 0; t < NT; ++t) acc[t] = 0.f;
-        nvfp4_rows<NT>(rec + 2 * nq, rec + 3 * nq + 2 * ns, L, F, row, zs, acc);
-        reduce_warps<NT>(acc, red);
-        if (threadIdx.x < 32) {
-#pragma unroll
-            for (int t = 0; t < NT; ++t)
-                if (t < nt) p.o[(size_t)(off + c0 + t) * L + row] = acc[t] * ts;
-        }
-        __syncthreads();
-    }
-}
-
-// ---------------------------------------------------------------------------
-// kernel 5: U_g of the per-group weighted sums, shared down, combine
-// ---------------------------------------------------------------------------
-
-template <int NT>
-__global__ void __launch_bounds__(512) k_uproj(FwdParams p) {
-    extern __shared__ float smem[];
-    const int part = blockIdx.y;            // 0..G-1: group; G: shared expert
-    const int H = p.H, L = p.L, G = p.G, K = p.K, T = p.T;
+    const int L = p.L, F = p.F, f0 = blockIdx.x * 16;
+    __half* hs = reinterpret_cast<__half*>(smem_u8);
+    float* red = reinterpret_cast<float*>(smem_u8 + (size_t)8 * (L + kXPad) * 2);
+    __shared__ int tok[8];
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int row0 = blockIdx.x * 32;
+    const uint8_t* rec = p.experts + (size_t)e * p.rec_bytes;
+    const size_t nq = (size_t)L * F / 2, ns = (size_t)L * F / 16;
+    const float* tail = reinterpret_cast<const float*>(rec + 3 * nq + 3 * ns);
+    const float ts_g = __ldg(tail), ts_u = __ldg(tail + 1);
+    const int nc = L / 32, per = (nc + kMmaWarps - 1) / kMmaWarps;
+    for (int c0 = 0; c0 < cnt; c0 += 8) {
+        const int nt = min(8, cnt - c0);
+        if (threadIdx.x < 8) tok[threadIdx.x] = threadIdx.x < nt ? __ldcg(p.r.slot_pair + off + c0 + threadIdx.x) / p.K : 0;
+        __syncthreads();
+        // gather the slots' latent inputs h16[token][g] (eight loads in flight per thread)
+        {
+            const int n8 = L / 8, total = 8 * n8;
+            for (int i0 = threadIdx.x; i0 < total; i0 += 8 * blockDim.x) {
+                uint4 v[8];
+#pragma unroll
+                for (int u = 0; u < 8; ++u) {
+                    const int i = i0 + u * blockDim.x, t = i / n8, c = i - t * n8;
+                    v[u] = (i < total && t < nt) ? __ldcg(reinterpret_cast<const uint4*>(p.h16 + ((size_t)tok[t] * p.G + g) * L) + c)
+                                                 : make_uint4(0, 0, 0, 0);
+                }
+#pragma unroll
+                for (int u = 0; u < 8; ++u) {
+                    const int i = i0 + u * blockDim.x, t = i / n8, c = i - t * n8;
+                    if (i < total) *reinterpret_cast<uint4*>(hs + (size_t)t * (L + kXPad) + 8 * c) = v[u];
+                }
+            }
+        }
+        __syncthreads();
+        float a[4] = {0.f, 0.f, 0.f, 0.f}, u[4] = {0.f, 0.f, 0.f, 0.f};
+        const int kc0 = warp * per, kc1 = min(nc, (warp + 1) * per);
+        mma_nvfp4_rows(rec, rec + 3 * nq, F, L, f0, kc0, kc1, hs, a);
+        mma_nvfp4_rows(rec + nq, rec + 3 * nq + ns, F, L, f0, kc0, kc1, hs, u);
+        reduce_frags(a, red);
+        reduce_frags(u, red);
+        if (warp == 0) {
+            const int gg = lane >> 2, tt = lane & 3;
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                const int col = 2 * tt + (i & 1), f = f0 + gg + 8 * (i >> 1);
+                if (col < nt) p.z16[(size_t)(off + c0 + col) * F + f] = __float2half_rn(silu(a[i] * ts_g) * (u[i] * ts_u));
+            }
+        }
+        __syncthreads();
+    }
+}
+
+// kernel 4: s16[t][g] = sum over the token's experts of group g of w * (W_down z);
+// CTA = 16 latent rows of one group; each warp takes whole experts of the
+// group (K = ffn in one warp, no reduction), the group sum is formed in a
+// fixed order afterwards.
+constexpr int kDownWarps = 8;
+
+__global__ void __launch_bounds__(32 * kDownWarps) k_down_mma(FwdParams p) {
+    extern __shared__ __align__(16) uint8_t smem_u8[];
+    const int g = blockIdx.y;
+    const int L = p.L, F = p.F, T = p.T, r0 = blockIdx.x * 16;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int KP = F + kXPad;
+    __half* zs = reinterpret_cast<__half*>(smem_u8);                       // [kDownWarps][8][F + pad]
+    float* part = reinterpret_cast<float*>(smem_u8 + (size_t)kDownWarps * 8 * KP * 2);  // [T * K][16] per slot
+    __shared__ int elist[kMaxTopK * kChunk];
+    __shared__ int n_e;
+    // group label and slot of every (token, k) pair, for the final sum
+    __shared__ uint8_t pg[kMaxTopK * 64];
+    __shared__ int pslot[kMaxTopK * 64];
+    for (int i = threadIdx.x; i < T * p.K; i += blockDim.x) {
+        const int e = __ldcg(p.r.idx + i);
+        pg[i] = p.group[e] < p.G ? p.group[e] : 0;
+        pslot[i] = __ldcg(p.r.pair_slot + i);
+    }
+    const int n_unique = __ldcg(p.r.n_unique);
+    const bool hit = __ldcg(p.r.ghit + g) > 0;
+    if (threadIdx.x == 0) {
+        int n = 0;
+        for (int j = 0; hit && j < n_unique; ++j)
+            if (p.group[__ldcg(p.r.uexp + j)] == g && n < kMaxTopK * kChunk) elist[n++] = j;
+        n_e = n;
+    }
+    __syncthreads();
+    const size_t nq = (size_t)L * F / 2, ns = (size_t)L * F / 16;
+    __half* zw = zs + (size_t)warp * 8 * KP;
+    for (int ii = warp; ii < n_e; ii += kDownWarps) {
+        const int j = elist[ii];
+        const int e = __ldcg(p.r.uexp + j), cnt = __ldcg(p.r.ucnt + j), off = __ldcg(p.r.uoff + j);
+        const uint8_t* rec = p.experts + (size_t)e * p.rec_bytes;
+        const float ts_d = __ldg(reinterpret_cast<const float*>(rec + 3 * nq + 3 * ns) + 2);
+        for (int c0 = 0; c0 < cnt; c0 += 8) {
+            const int nt = min(8, cnt - c0);
+            // this warp's 8 slot rows of z (fp16), zero beyond nt
+            for (int i = lane; i < 8 * (F / 8); i += 32) {
+                const int t = i / (F / 8), c = i - t * (F / 8);
+                const uint4 v = t < nt ? __ldcg(reinterpret_cast<const uint4*>(p.z16 + (size_t)(off + c0 + t) * F) + c)
+                                       : make_uint4(0, 0, 0, 0);
+                *reinterpret_cast<uint4*>(zw + (size_t)t * KP + 8 * c) = v;
+            }
+            __syncwarp();
+            float acc[4] = {0.f, 0.f, 0.f, 0.f};
+            mma_nvfp4_rows(rec + 2 * nq, rec + 3 * nq + 2 * ns, L, F, r0, 0, F / 32, zw, acc);
+            const int gg = lane >> 2, tt = lane & 3;
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                const int col = 2 * tt + (i & 1), row = gg + 8 * (i >> 1);
+                if (col < nt) {
+                    const int slot = off + c0 + col;
+                    part[(size_t)slot * 16 + row] = __ldcg(p.r.w + __ldcg(p.r.slot_pair + slot)) * (acc[i] * ts_d);
+                }
+            }
+            __syncwarp();
+        }
+    }
+    __syncthreads();
+    // group sum per (row, token), experts in ascending order (deterministic)
+    for (int i = threadIdx.x; i < 16 * T; i += blockDim.x) {
+        const int row = i / T, t = i - row * T;
+        float v = 0.f;
+        if (hit) {
+            for (int k = 0; k < p.K; ++k) {
+                const int pair = t * p.K + k;
+                if (pg[pair] == g) v += part[(size_t)pslot[pair] * 16 + row];
+            }
+        }
+        p.s16[((size_t)t * p.G + g) * L + r0 + row] = __float2half_rn(v);
+    }
+}
+
+// kernel 5: per 16 output rows, one part per hit group (U_g s16[t][g]) and
+// one for the shared expert's down projection; the last part of a row tile
+// to finish sums the parts in a fixed order, adds the residual, writes y.
+template <int FMT>
+__global__ void __launch_bounds__(32 * kMmaWarps) k_uproj_mma(FwdParams p) {
+    extern __shared__ __align__(16) uint8_t smem_u8[];
+    const int part = blockIdx.y;
+    const int H = p.H, L = p.L, G = p.G, T = p.T, r0 = blockIdx.x * 16;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const bool active = part == G || __ldcg(p.r.ghit + part) > 0;
-    __shared__ int lst_slot[kChunk * kMaxTopK];
-    __shared__ float lst_w[kChunk * kMaxTopK];
-    __shared__ int lst_n[kChunk];
     if (active) {
-        float* as = smem;                                   // [max(L, Fs)][NT]
-        float* red = smem + (size_t)max(L, p.Fs) * NT;
-        for (int t0 = 0; t0 < T; t0 += NT) {
-            const int nt = min(NT, T - t0);
-            float acc[NT];
-#pragma unroll
-            for (int t = 0; t < NT; ++t) acc[t] = 0.f;
+        for (int t0 = 0; t0 < T; t0 += 8) {
+            const int nt = min(8, T - t0);
             if (part < G) {
-                // s[t][k] = sum over the token's experts of group `part` of w * o
-                if (threadIdx.x < NT) {
-                    const int t = threadIdx.x;
-                    int n = 0;
-                    if (t < nt && p.r.tghit[(size_t)(t0 + t) * G + part]) {
-                        for (int kk = 0; kk < K; ++kk) {
-                            const int pair = (t0 + t) * K + kk;
-                            const int e = __ldcg(p.r.idx + pair);
-                            if (p.group[e] == part) {
-                                lst_slot[t * kMaxTopK + n] = __ldcg(p.r.pair_slot + pair);
-                                lst_w[t * kMaxTopK + n] = __ldcg(p.r.w + pair);
-                                ++n;
-                            }
-                        }
-                    }
-                    lst_n[t] = n;
-                }
+                __half* ss = reinterpret_cast<__half*>(smem_u8);
+                float* red = reinterpret_cast<float*>(smem_u8 + (size_t)8 * (L + kXPad) * 2);
+                stage_act16(ss, L, p.s16 + ((size_t)t0 * G + part) * L, (size_t)G * L, nt);
                 __syncthreads();
-                for (int i = threadIdx.x; i < NT * L; i += blockDim.x) {
-                    const int t = i / L, k = i - t * L;
-                    float s = 0.f;
-                    for (int j = 0; j < lst_n[t]; ++j)
-                        s = fmaf(lst_w[t * kMaxTopK + j], __ldcg(p.o + (size_t)lst_slot[t * kMaxTopK + j] * L + k), s);
-                    as[k * NT + t] = s;
-                }
-                __syncthreads();
-                du_rows<NT>(p.du_fmt, p.U + (size_t)part * p.du_bytes_U, H, L, row0 + lane, as, acc);
-                reduce_warps<NT>(acc, red);
-                if (threadIdx.x < 32) {
+                float acc[4] = {0.f, 0.f, 0.f, 0.f};
+                const int nb = L / 32, per = (nb + kMmaWarps - 1) / kMmaWarps;
+                mma_du_rows<FMT>(p.U + (size_t)part * p.du_bytes_U, H, L, r0, warp * per, min(nb, (warp + 1) * per),
+                                 ss, acc);
+                reduce_frags(acc, red);
+                if (warp == 0) {
+                    const int gg = lane >> 2, tt = lane & 3;
 #pragma unroll
-                    for (int t = 0; t < NT; ++t)
-                        if (t < nt) p.ypart[((size_t)part * T + t0 + t) * H + row0 + lane] = acc[t];
+                    for (int i = 0; i < 4; ++i) {
+                        const int tok = 2 * tt + (i & 1), row = r0 + gg + 8 * (i >> 1);
+                        if (tok < nt) p.ypart[((size_t)part * T + t0 + tok) * H + row] = acc[i];
+                    }
                 }
             } else {
-                const int Fs = p.Fs;
-                for (int i = threadIdx.x; i < NT * Fs; i += blockDim.x) {
-                    const int t = i / Fs, k = i - t * Fs;
-                    as[k * NT + t] = t < nt ? __ldcg(p.zsh + (size_t)(t0 + t) * Fs + k) : 0.f;
+                // shared expert: 4 rows per warp on CUDA cores (bf16 weights, fp32 hidden)
+                float* as = reinterpret_cast<float*>(smem_u8);      // [8][Fs + 4]
+                const int Fs = p.Fs, ld = xs_ld(Fs), n4 = Fs / 4;
+                for (int i0 = threadIdx.x; i0 < 8 * n4; i0 += 4 * blockDim.x) {
+                    float4 v[4];
+#pragma unroll
+                    for (int u = 0; u < 4; ++u) {
+                        const int i = i0 + u * blockDim.x, t = i / n4, c = i - t * n4;
+                        v[u] = (i < 8 * n4 && t < nt) ? __ldcg(reinterpret_cast<const float4*>(p.zsh + (size_t)(t0 + t) * Fs) + c)
+                                                      : make_float4(0.f, 0.f, 0.f, 0.f);
+                    }
+#pragma unroll
+                    for (int u = 0; u < 4; ++u) {
+                        const int i = i0 + u * blockDim.x, t = i / n4, c = i - t * n4;
+                        if (i < 8 * n4) *reinterpret_cast<float4*>(as + t * ld + 4 * c) = v[u];
+                    }
                 }
                 __syncthreads();
-                for (int rr = warp; rr < 32; rr += blockDim.x >> 5) {
-                    const int row = row0 + rr;
-                    float a2[NT];
+                for (int rr = warp; rr < 16; rr += kMmaWarps) {
+                    const int row = r0 + rr;
+                    float a2[8];
 #pragma unroll
-                    for (int t = 0; t < NT; ++t) a2[t] = 0.f;
-                    row_dot<NT, true>(p.sd + (size_t)row * Fs, Fs, as, lane, a2);
+                    for (int t = 0; t < 8; ++t) a2[t] = 0.f;
+                    row_dot<8, true>(p.sd + (size_t)row * Fs, Fs, as, ld, lane, a2);
 #pragma unroll
-                    for (int t = 0; t < NT; ++t) {
+                    for (int t = 0; t < 8; ++t) {
                         const float v = warp_sum(a2[t]);
                         if (lane == 0 && t < nt) p.ypart[((size_t)G * T + t0 + t) * H + row] = v;
                     }
@@ -703,7 +821,6 @@ __global__ void __launch_bounds__(512) k_uproj(FwdParams p) {
             __syncthreads();
         }
     }
-    // the last part of this row tile to finish writes y
     __shared__ int s_last;
     __syncthreads();
     if (threadIdx.x == 0) {
@@ -714,12 +831,14 @@ __global__ void __launch_bounds__(512) k_uproj(FwdParams p) {
     __syncthreads();
     if (!s_last) return;
     __threadfence();
-    for (int i = threadIdx.x; i < T * 32; i += blockDim.x) {
-        const int t = i >> 5, row = row0 + (i & 31);
-        float v = 0.f;
+    __shared__ uint8_t th[64 * kMaxGroups];
+    for (int i = threadIdx.x; i < T * G; i += blockDim.x) th[i] = p.r.tghit[i] && __ldcg(p.r.ghit + i % G) > 0;
+    __syncthreads();
+    for (int i = threadIdx.x; i < T * 16; i += blockDim.x) {
+        const int t = i >> 4, row = r0 + (i & 15);
+        float v = __ldcg(p.ypart + ((size_t)G * T + t) * H + row);
         for (int g = 0; g < G; ++g)
-            if (__ldcg(p.r.ghit + g) > 0 && p.r.tghit[(size_t)t * G + g]) v += __ldcg(p.ypart + ((size_t)g * T + t) * H + row);
-        v += __ldcg(p.ypart + ((size_t)G * T + t) * H + row);
+            if (th[t * G + g]) v += __ldcg(p.ypart + ((size_t)g * T + t) * H + row);
         if (p.residual) v += bf16_bits_to_f32(p.residual[(size_t)t * H + row]);
         p.y[(size_t)t * H + row] = f32_to_bf16_bits(v);
     }
@@ -775,39 +894,38 @@ static cudaError_t launch(Kern k, dim3 grid, int threads, size_t smem, cudaStrea
     return cudaGetLastError();
 }
 
-// Warps per CTA of a row-tile GEMV over C columns: two 64-column groups per warp.
-static int gemv_warps(int C) { return max(1, min(16, (C / 64 + 1) / 2)); }
-
 template <int NT>
 static cudaError_t run_gemv_path_nt(FwdParams p, cudaStream_t st, bool route_only) {
-    auto red = [](int warps) { return (size_t)warps * 32 * NT * sizeof(float); };
     // 1. router (+ shared gate/up, top-k, buckets): one warp per router row / shared feature
     p.router_rows_per_warp = 1;
     p.n_router_ctas = (p.E + 7) / 8;
     p.do_shared = !route_only;
     p.do_buckets = !route_only;
-    p.prefetch_l2 = !route_only;
+    p.prefetch_l2 = false;
     const int n_shared_ctas = route_only ? 0 : (p.Fs + 7) / 8;
     {
-        const size_t sm = (size_t)p.H * NT * sizeof(float);
+        const size_t sm = (size_t)xs_ld(p.H) * NT * sizeof(float);
         cudaError_t e = p.router_bf16
             ? launch(k_router_shared<NT, true>, dim3(p.n_router_ctas + n_shared_ctas), 256, sm, st, p)
             : launch(k_router_shared<NT, false>, dim3(p.n_router_ctas + n_shared_ctas), 256, sm, st, p);
         if (e != cudaSuccess || route_only) return e;
     }
     const int max_unique = min(p.T * p.K, p.E);
+    const size_t red = (size_t)kMmaWarps * 32 * 4 * sizeof(float);
+    const int thr = 32 * kMmaWarps;
     cudaError_t e;
-    int w = gemv_warps(p.H);
-    e = launch(k_dproj<NT>, dim3(p.L / 32, p.G), 32 * w, (size_t)p.H * NT * 4 + red(w), st, p);
+    const size_t sm_d = (size_t)8 * (p.H + kXPad) * 2 + red;
+    e = p.du_fmt == LMOE_Q8_0 ? launch(k_dproj_mma<LMOE_Q8_0>, dim3(p.L / 16, p.G), thr, sm_d, st, p)
+                              : launch(k_dproj_mma<LMOE_Q4_0>, dim3(p.L / 16, p.G), thr, sm_d, st, p);
     if (e != cudaSuccess) return e;
-    w = gemv_warps(p.L);
-    e = launch(k_expert_gateup<NT>, dim3(p.F / 32, max_unique), 32 * w, (size_t)p.L * NT * 4 + red(w), st, p);
+    e = launch(k_gateup_mma, dim3(p.F / 16, max_unique), thr, (size_t)8 * (p.L + kXPad) * 2 + red, st, p);
     if (e != cudaSuccess) return e;
-    w = gemv_warps(p.F);
-    e = launch(k_expert_down<NT>, dim3(p.L / 32, max_unique), 32 * w, (size_t)p.F * NT * 4 + red(w), st, p);
+    e = launch(k_down_mma, dim3(p.L / 16, p.G), 32 * kDownWarps,
+               (size_t)kDownWarps * 8 * (p.F + kXPad) * 2 + (size_t)p.T * p.K * 16 * 4, st, p);
     if (e != cudaSuccess) return e;
-    w = max(gemv_warps(p.L), 8);
-    e = launch(k_uproj<NT>, dim3(p.H / 32, p.G + 1), 32 * w, (size_t)max(p.L, p.Fs) * NT * 4 + red(w), st, p);
+    const size_t sm_u = max((size_t)8 * (p.L + kXPad) * 2 + red, (size_t)xs_ld(p.Fs) * 8 * 4);
+    e = p.du_fmt == LMOE_Q8_0 ? launch(k_uproj_mma<LMOE_Q8_0>, dim3(p.H / 16, p.G + 1), thr, sm_u, st, p)
+                              : launch(k_uproj_mma<LMOE_Q4_0>, dim3(p.H / 16, p.G + 1), thr, sm_u, st, p);
     return e;
 }
 

@@ -67,11 +67,12 @@ struct FwdParams {
     // workspace
     Ctrl* ctrl;
     Routing r;
-    float* h;       // [T][G][L]
-    float* zsh;     // [T][Fs]
-    float* z;       // [T*K][F]   per slot
-    float* o;       // [T*K][L]   per slot
-    float* ypart;   // [G+1][T][H]
+    __half* x16;    // [T][H]       block input (normalised for the stack), fp16
+    __half* h16;    // [T][G][L]    D_g x for the hit (token, group) pairs
+    float* zsh;     // [T][Fs]      shared-expert hidden
+    __half* z16;    // [T*K][F]     expert hidden per slot (slots grouped by expert)
+    __half* s16;    // [T][G][L]    per-group weighted expert sums
+    float* ypart;   // [G+1][T][H]  U_g parts and the shared part
     size_t du_bytes_D, du_bytes_U, rec_bytes;
     // launch shape of the router kernel
     int n_router_ctas, router_rows_per_warp;

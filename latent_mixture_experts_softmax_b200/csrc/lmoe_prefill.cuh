@@ -68,7 +68,7 @@ struct PrefillParams {
     __half* zperm;       // [T*K][F]
     __half* operm;       // [T*K][L] weighted expert outputs
     __half* s;           // [T][G][L]
-    __half* zsh;         // [T][Fs]
+    uint16_t* zsh;       // [2][T][Fs] shared-expert hidden as bf16 high and low parts
 };
 
 cudaError_t run_prefill_route(PrefillParams p, cudaStream_t st);

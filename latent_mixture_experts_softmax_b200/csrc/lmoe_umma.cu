@@ -105,13 +105,15 @@ struct Sched {
     // UPROJ: one segment per group, then the shared expert's down projection.
     // ROUTER / SHARED_GATEUP on a normalised input: the input is split into
     // bf16 high and low parts, one segment each, so the products stay exact.
+    // UPROJ segments G and G + 1: the shared expert's down projection on the
+    // bf16 high and low parts of its hidden activations.
     __device__ static int num_segs(const PrefillParams& p) {
-        if (KIND == G_UPROJ) return p.G + 1;
+        if (KIND == G_UPROJ) return p.G + 2;
         if (KIND == G_ROUTER || KIND == G_SHARED_GATEUP) return p.xr ? 2 : 1;
         return 1;
     }
     __device__ static bool seg_active(const PrefillParams& p, const TileRef& t, int seg) {
-        if (KIND != G_UPROJ || seg == p.G) return true;
+        if (KIND != G_UPROJ || seg >= p.G) return true;
         return p.dhit[t.nq * p.G + seg] != 0;
     }
     __device__ static int seg_k(const PrefillParams& p, int seg) {
@@ -121,12 +123,17 @@ struct Sched {
             case G_DPROJ: return p.H;
             case G_GATEUP: return p.L;
             case G_DOWN: return p.F;
-            default: return seg == p.G ? p.Fs : p.L;
+            default: return seg >= p.G ? p.Fs : p.L;
         }
     }
-    // A comes through TMA (plain bf16 weights) rather than the dequantising producers
-    static constexpr bool kTmaA = KIND == G_ROUTER || KIND == G_SHARED_GATEUP;
-    static constexpr int kBf16 = (KIND == G_ROUTER || KIND == G_SHARED_GATEUP) ? 1 : 0;
+    // A of this segment comes through TMA (plain bf16 weights: router, shared
+    // expert) rather than from the dequantising producers; those segments run
+    // bf16 x bf16.
+    __device__ static bool tma_a(const PrefillParams& p, int seg) {
+        if (KIND == G_ROUTER || KIND == G_SHARED_GATEUP) return true;
+        return KIND == G_UPROJ && seg >= p.G;
+    }
+    static constexpr bool kAnyTmaA = KIND == G_ROUTER || KIND == G_SHARED_GATEUP || KIND == G_UPROJ;
 };
 
 // Walks the (tile, segment, 64-wide K stage) sequence of one CTA.
@@ -180,62 +187,94 @@ struct Cursor {
 // weight operand: raw loads and dequantisation to fp16 (one row, 64 columns)
 // ---------------------------------------------------------------------------
 
-struct RawRow {
-    uint4 q[8];
-    uint32_t s;
-};
+// Raw weight bytes of one A stage (128 rows x 64 columns) as they are stored,
+// copied into a shared-memory slot by the TMA engine (1-D bulk copies):
+//   [part 0 | part 1 | scales]
+// part j = 32-column block (Q8_0 / Q4_0) or chunk (NVFP4) j of the stage,
+// 128 rows x (32 | 16) bytes, row r at r * bytes; scales: Q8_0 / Q4_0 two
+// fp16 arrays of 128 (block 0, block 1), NVFP4 one word per row.  For the
+// gate/up tiles rows 0-63 are gate rows and 64-127 the matching up rows.
+template <int KIND>
+__host__ __device__ constexpr int raw_part_bytes(int du_fmt) {
+    return KIND == G_DPROJ || KIND == G_UPROJ ? 128 * (du_fmt == LMOE_Q8_0 ? 32 : 16) : 128 * 16;
+}
+template <int KIND>
+__host__ __device__ constexpr int raw_slot_bytes(int du_fmt) {
+    return (KIND == G_ROUTER || KIND == G_SHARED_GATEUP) ? 0 : 2 * raw_part_bytes<KIND>(du_fmt) + 512;
+}
 
-__device__ __forceinline__ uint4 ldg_nc(const void* ptr) { return ldg_stream(reinterpret_cast<const uint4*>(ptr)); }
+__device__ __forceinline__ void bulk_g2s(void* dst, const void* src, uint32_t bytes, uint64_t* bar) {
+    asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
+                 ::"r"(smem_u32(dst)), "l"(src), "r"(bytes), "r"(smem_u32(bar))
+                 : "memory");
+}
 
-// Where row r (0..127) of the A tile of stage (tile, seg, ks) lives, and its load.
+// Arm `bar` and copy the raw weights of the cursor's stage into `slot`.
 template <int KIND, int NT>
-__device__ __forceinline__ void load_raw(const PrefillParams& p, const Cursor<KIND, NT>& c, int r, RawRow& raw) {
+__device__ __forceinline__ void issue_raw(const PrefillParams& p, const Cursor<KIND, NT>& c, uint8_t* slot,
+                                          uint64_t* bar) {
     const int k0 = c.ks * 64;
+    const uint32_t pb = raw_part_bytes<KIND>(p.du_fmt);
     if (KIND == G_DPROJ || (KIND == G_UPROJ && c.seg < p.G)) {
         const int R = KIND == G_DPROJ ? p.L : p.H;
         const int C = KIND == G_DPROJ ? p.H : p.L;
         const uint8_t* mat = (KIND == G_DPROJ ? p.D : p.U) + (size_t)(KIND == G_DPROJ ? c.t.mat : c.seg) * p.du_bytes;
-        const int row = c.t.m0 + r;
+        const size_t rowb = p.du_fmt == LMOE_Q8_0 ? 32 : 16;
+        const uint8_t* dsc = mat + (size_t)R * C / 32 * rowb;
         const int kb = k0 / 32;
-        const uint16_t* dsc;
-        if (p.du_fmt == LMOE_Q8_0) {
-            raw.q[0] = ldg_nc(mat + ((size_t)kb * R + row) * 32);
-            raw.q[1] = ldg_nc(mat + ((size_t)kb * R + row) * 32 + 16);
-            raw.q[2] = ldg_nc(mat + ((size_t)(kb + 1) * R + row) * 32);
-            raw.q[3] = ldg_nc(mat + ((size_t)(kb + 1) * R + row) * 32 + 16);
-            dsc = reinterpret_cast<const uint16_t*>(mat + (size_t)R * C);
-        } else {
-            raw.q[0] = ldg_nc(mat + ((size_t)kb * R + row) * 16);
-            raw.q[1] = ldg_nc(mat + ((size_t)(kb + 1) * R + row) * 16);
-            dsc = reinterpret_cast<const uint16_t*>(mat + (size_t)R * C / 2);
-        }
-        raw.s = (uint32_t)__ldg(dsc + (size_t)kb * R + row) | ((uint32_t)__ldg(dsc + (size_t)(kb + 1) * R + row) << 16);
-    } else if (KIND == G_UPROJ) {
-        // shared expert down projection, bf16 [H][Fs]
-        const uint16_t* src = p.sd + (size_t)(c.t.m0 + r) * p.Fs + k0;
-#pragma unroll
-        for (int i = 0; i < 8; ++i) raw.q[i] = ldg_nc(src + 8 * i);
-    } else if (KIND == G_GATEUP || KIND == G_DOWN) {
+        mbar_arrive_expect_tx(bar, 2 * pb + 512);
+        bulk_g2s(slot, mat + ((size_t)kb * R + c.t.m0) * rowb, pb, bar);
+        bulk_g2s(slot + pb, mat + ((size_t)(kb + 1) * R + c.t.m0) * rowb, pb, bar);
+        bulk_g2s(slot + 2 * pb, dsc + ((size_t)kb * R + c.t.m0) * 2, 256, bar);
+        bulk_g2s(slot + 2 * pb + 256, dsc + ((size_t)(kb + 1) * R + c.t.m0) * 2, 256, bar);
+    } else if (KIND == G_GATEUP) {
         const size_t nq = (size_t)p.L * p.F / 2, ns = (size_t)p.L * p.F / 16;
         const uint8_t* rec = p.experts + (size_t)c.t.mat * p.rec_bytes;
-        const uint8_t *q, *s;
-        int R, row;
-        if (KIND == G_GATEUP) {
-            const bool up = r >= 64;
-            q = rec + (up ? nq : 0);
-            s = rec + 3 * nq + (up ? ns : 0);
-            R = p.F;
-            row = c.t.m0 + (r & 63);
-        } else {
-            q = rec + 2 * nq;
-            s = rec + 3 * nq + 2 * ns;
-            R = p.L;
-            row = c.t.m0 + r;
+        const int kc = k0 / 32, R = p.F;
+        mbar_arrive_expect_tx(bar, 2 * pb + 512);
+#pragma unroll
+        for (int j = 0; j < 2; ++j) {
+            bulk_g2s(slot + j * pb, rec + ((size_t)(kc + j) * R + c.t.m0) * 16, 1024, bar);             // gate
+            bulk_g2s(slot + j * pb + 1024, rec + nq + ((size_t)(kc + j) * R + c.t.m0) * 16, 1024, bar);  // up
         }
-        const int kc = k0 / 32;
-        raw.q[0] = ldg_nc(q + ((size_t)kc * R + row) * 16);
-        raw.q[1] = ldg_nc(q + ((size_t)(kc + 1) * R + row) * 16);
-        raw.s = __ldg(reinterpret_cast<const uint32_t*>(s + ((size_t)(k0 / 64) * R + row) * 4));
+        bulk_g2s(slot + 2 * pb, rec + 3 * nq + ((size_t)(k0 / 64) * R + c.t.m0) * 4, 256, bar);
+        bulk_g2s(slot + 2 * pb + 256, rec + 3 * nq + ns + ((size_t)(k0 / 64) * R + c.t.m0) * 4, 256, bar);
+    } else if (KIND == G_DOWN) {
+        const size_t nq = (size_t)p.L * p.F / 2, ns = (size_t)p.L * p.F / 16;
+        const uint8_t* rec = p.experts + (size_t)c.t.mat * p.rec_bytes;
+        const int kc = k0 / 32, R = p.L;
+        mbar_arrive_expect_tx(bar, 2 * pb + 512);
+        bulk_g2s(slot, rec + 2 * nq + ((size_t)kc * R + c.t.m0) * 16, pb, bar);
+        bulk_g2s(slot + pb, rec + 2 * nq + ((size_t)(kc + 1) * R + c.t.m0) * 16, pb, bar);
+        bulk_g2s(slot + 2 * pb, rec + 3 * nq + 2 * ns + ((size_t)(k0 / 64) * R + c.t.m0) * 4, 512, bar);
+    } else {
+        mbar_arrive(bar);                          // nothing to copy for this stage
+    }
+}
+
+// Row r of a raw slot -> the register form the dequantiser takes.
+struct RawRow {
+    uint4 q[4];
+    uint32_t s;
+};
+
+template <int KIND>
+__device__ __forceinline__ void raw_row_from_smem(const PrefillParams& p, const uint8_t* slot, int r, RawRow& raw) {
+    const int pb = raw_part_bytes<KIND>(p.du_fmt);
+    if ((KIND == G_DPROJ || KIND == G_UPROJ) && p.du_fmt == LMOE_Q8_0) {
+        raw.q[0] = *reinterpret_cast<const uint4*>(slot + r * 32);
+        raw.q[1] = *reinterpret_cast<const uint4*>(slot + r * 32 + 16);
+        raw.q[2] = *reinterpret_cast<const uint4*>(slot + pb + r * 32);
+        raw.q[3] = *reinterpret_cast<const uint4*>(slot + pb + r * 32 + 16);
+    } else {
+        raw.q[0] = *reinterpret_cast<const uint4*>(slot + r * 16);
+        raw.q[1] = *reinterpret_cast<const uint4*>(slot + pb + r * 16);
+    }
+    if (KIND == G_DPROJ || KIND == G_UPROJ) {
+        const uint16_t* d = reinterpret_cast<const uint16_t*>(slot + 2 * pb);
+        raw.s = (uint32_t)d[r] | ((uint32_t)d[128 + r] << 16);
+    } else {
+        raw.s = reinterpret_cast<const uint32_t*>(slot + 2 * pb)[r];
     }
 }
 
@@ -288,16 +327,6 @@ __device__ __forceinline__ void dequant_row(const PrefillParams& p, int seg, con
                 }
             }
         }
-    } else if (KIND == G_UPROJ) {
-#pragma unroll
-        for (int i = 0; i < 8; ++i) {
-            const uint32_t w4[4] = {raw.q[i].x, raw.q[i].y, raw.q[i].z, raw.q[i].w};
-#pragma unroll
-            for (int j = 0; j < 4; ++j) {
-                const float2 f = bf16x2_to_f32x2(w4[j]);
-                o[4 * i + j] = h2_bits(__floats2half2_rn(f.x, f.y));
-            }
-        }
     } else {
         // NVFP4: E2M1 x E4M3 is exact in fp16; the tensor scale is applied in the epilogue
         uint32_t sc01, sc23;
@@ -346,20 +375,24 @@ __device__ __forceinline__ void epilogue_chunk(const PrefillParams& p, const Til
     if (KIND == G_ROUTER) {
         const int e = t.m0 + row;
         const float b = p.router_b ? __ldg(p.router_b + e) : 0.f;
-        for (int j = 0; j < ncol; ++j) p.logits[(size_t)(t.b0 + c0 + j) * p.E + e] = u2f(r[j]) + b;
+#pragma unroll
+        for (int j = 0; j < 32; ++j)
+            if (j < ncol) p.logits[(size_t)(t.b0 + c0 + j) * p.E + e] = u2f(r[j]) + b;
     } else if (KIND == G_DPROJ) {
+        // metadata staged by the epilogue warps: group masks and slots of the tile's tokens
+        const uint32_t* mmask = reinterpret_cast<const uint32_t*>(xchg);
+        const int* mslot = reinterpret_cast<const int*>(mmask + NT);
         const int l = t.m0 + row;
-        const int g = t.mat;
-        for (int j = 0; j < ncol; ++j) {
-            const int tok = t.b0 + c0 + j;
-            uint32_t mask = __ldg(p.tgmask + (size_t)tok * p.G + g);
-            if (mask == 0) continue;
-            const __half v = __float2half_rn(u2f(r[j]));
-            while (mask) {
-                const int k = __ffs(mask) - 1;
-                mask &= mask - 1;
-                const int slot = __ldg(p.pair_slot + (size_t)tok * p.K + k);
-                p.hperm[(size_t)slot * p.L + l] = v;
+#pragma unroll
+        for (int j = 0; j < 32; ++j) {
+            if (j < ncol) {
+                uint32_t mask = mmask[c0 + j];
+                const __half v = __float2half_rn(u2f(r[j]));
+                while (mask) {
+                    const int k = __ffs(mask) - 1;
+                    mask &= mask - 1;
+                    p.hperm[(size_t)mslot[(c0 + j) * p.K + k] * p.L + l] = v;
+                }
             }
         }
     } else if (KIND == G_GATEUP || KIND == G_SHARED_GATEUP) {
@@ -378,32 +411,44 @@ __device__ __forceinline__ void epilogue_chunk(const PrefillParams& p, const Til
                 tu = __ldg(tail + 1);
             }
             const int f = t.m0 + row;
-            for (int j = 0; j < ncol; ++j) {
-                const float a = u2f(r[j]) * tg;
-                const float u = xchg[j * 64 + row] * tu;
-                const __half z = __float2half_rn(silu(a) * u);
-                if (KIND == G_GATEUP) p.zperm[(size_t)(t.b0 + c0 + j) * p.F + f] = z;
-                else p.zsh[(size_t)(t.b0 + c0 + j) * p.Fs + f] = z;
+#pragma unroll
+            for (int j = 0; j < 32; ++j) {
+                if (j < ncol) {
+                    const float a = u2f(r[j]) * tg;
+                    const float u = xchg[j * 64 + row] * tu;
+                    const float z = silu(a) * u;
+                    if (KIND == G_GATEUP) {
+                        p.zperm[(size_t)(t.b0 + c0 + j) * p.F + f] = __float2half_rn(z);
+                    } else {
+                        const uint16_t hi = f32_to_bf16_bits(z);
+                        p.zsh[(size_t)(t.b0 + c0 + j) * p.Fs + f] = hi;
+                        p.zsh[((size_t)p.T + t.b0 + c0 + j) * p.Fs + f] = f32_to_bf16_bits(z - bf16_bits_to_f32(hi));
+                    }
+                }
             }
         }
         named_bar_sync(1, 128);
     } else if (KIND == G_DOWN) {
+        // routing weights of the tile's slots staged in xchg by the epilogue warps
         const size_t nq = (size_t)p.L * p.F / 2, ns = (size_t)p.L * p.F / 16;
         const float td = __ldg(reinterpret_cast<const float*>(p.experts + (size_t)t.mat * p.rec_bytes + 3 * nq + 3 * ns) + 2);
         const int l = t.m0 + row;
-        for (int j = 0; j < ncol; ++j) {
-            const int slot = t.b0 + c0 + j;
-            const float w = __ldg(p.w + __ldg(p.slot_pair + slot));
-            p.operm[(size_t)slot * p.L + l] = __float2half_rn(u2f(r[j]) * td * w);
+#pragma unroll
+        for (int j = 0; j < 32; ++j) {
+            if (j < ncol) {
+                const int slot = t.b0 + c0 + j;
+                p.operm[(size_t)slot * p.L + l] = __float2half_rn(u2f(r[j]) * td * xchg[c0 + j]);
+            }
         }
     } else {  // UPROJ
         const int hrow = t.m0 + row;
-        for (int j = 0; j < ncol; ++j) {
-            const int tok = t.b0 + c0 + j;
-            float v = u2f(r[j]);
-            if (p.residual) v += bf16_bits_to_f32(__ldg(p.residual + (size_t)tok * p.H + hrow));
-            p.y[(size_t)tok * p.H + hrow] = f32_to_bf16_bits(v);
-        }
+        float res[32];
+#pragma unroll
+        for (int j = 0; j < 32; ++j)
+            res[j] = (p.residual && j < ncol) ? bf16_bits_to_f32(__ldg(p.residual + (size_t)(t.b0 + c0 + j) * p.H + hrow)) : 0.f;
+#pragma unroll
+        for (int j = 0; j < 32; ++j)
+            if (j < ncol) p.y[(size_t)(t.b0 + c0 + j) * p.H + hrow] = f32_to_bf16_bits(u2f(r[j]) + res[j]);
     }
 }
 
@@ -411,29 +456,37 @@ __device__ __forceinline__ void epilogue_chunk(const PrefillParams& p, const Til
 // the GEMM kernel
 // ---------------------------------------------------------------------------
 
-template <int NT, int STAGES>
+template <int NT, int STAGES, int RS>
 struct SmemPlan {
     static constexpr int kA = 128 * 128;                 // bytes per A stage (128 rows x 64 x 16-bit)
     static constexpr int kB = NT * 128;                  // bytes per B stage
-    static constexpr int kXchg = 32 * 64 * 4;            // gate/up exchange
-    static constexpr int kBars = (3 * STAGES + 5) * 8;
-    static constexpr int kTotal = 1024 /*alignment slack*/ + STAGES * (kA + kB) + kXchg + kBars + 16;
+    static constexpr int kRaw = 8704;                    // bytes per raw weight slot (largest format)
+    // gate/up exchange (32 x 64 fp32) or a tile's routing metadata (NT x (1 + 16) words)
+    static constexpr int kXchg = (32 * 64 * 4 > NT * 4 * 17) ? 32 * 64 * 4 : NT * 4 * 17;
+    static constexpr int kBars = (3 * STAGES + 2 * RS + 5) * 8;
+    static constexpr int kTotal = 1024 /*alignment slack*/ + STAGES * (kA + kB) + RS * kRaw + kXchg + kBars + 16;
 };
 
-template <int KIND, int NT, int STAGES>
-__global__ void __launch_bounds__(288, 1) k_umma_gemm(const __grid_constant__ TmaMaps maps, const PrefillParams p) {
+constexpr int kConvWarps = 4;      // dequantising warps (one weight row per thread)
+constexpr int kGemmThreads = 320;  // 4 epilogue, 4 converter, 1 MMA, 1 loader warps
+
+template <int KIND, int NT, int STAGES, int RS>
+__global__ void __launch_bounds__(kGemmThreads, 1) k_umma_gemm(const __grid_constant__ TmaMaps maps, const PrefillParams p) {
     using S = Sched<KIND, NT>;
-    using Plan = SmemPlan<NT, STAGES>;
+    using Plan = SmemPlan<NT, STAGES, RS>;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
     uint8_t* sA = smem;
     uint8_t* sB = smem + STAGES * Plan::kA;
-    float* xchg = reinterpret_cast<float*>(sB + STAGES * Plan::kB);
+    uint8_t* sRaw = sB + STAGES * Plan::kB;
+    float* xchg = reinterpret_cast<float*>(sRaw + RS * Plan::kRaw);
     uint64_t* bars = reinterpret_cast<uint64_t*>(reinterpret_cast<uint8_t*>(xchg) + Plan::kXchg);
     uint64_t* full_a = bars;
     uint64_t* full_b = bars + STAGES;
     uint64_t* empty = bars + 2 * STAGES;
-    uint64_t* tfull = bars + 3 * STAGES;
+    uint64_t* raw_full = bars + 3 * STAGES;
+    uint64_t* raw_empty = raw_full + RS;
+    uint64_t* tfull = raw_empty + RS;
     uint64_t* tempty = tfull + 2;
     uint64_t* final_bar = tempty + 2;
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(final_bar + 1);
@@ -442,15 +495,19 @@ __global__ void __launch_bounds__(288, 1) k_umma_gemm(const __grid_constant__ Tm
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     constexpr uint32_t kTmemCols = 2 * NT;
 
-    if (threadIdx.x == 256) {
+    if (threadIdx.x == 0) {
         for (int s = 0; s < STAGES; ++s) {
-            mbar_init(&full_a[s], 128);
+            mbar_init(&full_a[s], kConvWarps);
             mbar_init(&full_b[s], 1);
             mbar_init(&empty[s], 1);
         }
+        for (int s = 0; s < RS; ++s) {
+            mbar_init(&raw_full[s], 1);
+            mbar_init(&raw_empty[s], kConvWarps);
+        }
         for (int a = 0; a < 2; ++a) {
             mbar_init(&tfull[a], 1);
-            mbar_init(&tempty[a], 128);
+            mbar_init(&tempty[a], 4);
         }
         mbar_init(final_bar, 1);
         *abort_flag = 0;
@@ -460,75 +517,99 @@ __global__ void __launch_bounds__(288, 1) k_umma_gemm(const __grid_constant__ Tm
         tmem_alloc(tmem_slot, kTmemCols);
         tmem_relinquish();
     }
-    if (threadIdx.x == 128) tma_prefetch_desc(&maps.b);
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem_base = *tmem_slot;
 
-    if (warp >= 4 && warp < 8) {
-        // ------------------------------------------------------------ producers
-        const int r = threadIdx.x - 128;           // A row
-        Cursor<KIND, NT> cur, pre;
-        cur.begin(p);
-        pre = cur;
-        RawRow ring[2];
-        // prefetch the first two stages
-        if (!S::kTmaA) {
-            if (!pre.done) { load_raw<KIND, NT>(p, pre, r, ring[0]); pre.next_stage(p); }
-            if (!pre.done) { load_raw<KIND, NT>(p, pre, r, ring[1]); pre.next_stage(p); }
-        }
-        uint32_t it = 0;
-        uint32_t last_phase[STAGES];
-#pragma unroll
-        for (int s = 0; s < STAGES; ++s) last_phase[s] = 0xFFFFFFFFu;
-        while (!cur.done) {
-#pragma unroll
-            for (int slot = 0; slot < 2; ++slot) {
-                if (cur.done) break;
-                const int s = it % STAGES;
-                const uint32_t ph = (it / STAGES) & 1;
-                if (!mbar_wait(&empty[s], ph ^ 1, abort_flag, kWaitLimitNs)) goto producer_abort;
-                if (r == 0) {
-                    // activation operand (and plain bf16 weights) by TMA
-                    const int k0 = cur.ks * 64;
-                    uint32_t bytes = Plan::kB + (S::kTmaA ? Plan::kA : 0);
-                    mbar_arrive_expect_tx(&full_b[s], bytes);
-                    uint8_t* dB = sB + s * Plan::kB;
-                    if (KIND == G_UPROJ && cur.seg < p.G) tma_load_3d(dB, &maps.b, &full_b[s], k0, cur.seg, cur.t.b0);
-                    else if (cur.seg > 0) tma_load_2d(dB, &maps.b2, &full_b[s], k0, cur.t.b0);
-                    else tma_load_2d(dB, &maps.b, &full_b[s], k0, cur.t.b0);
-                    if (KIND == G_ROUTER) {
-                        tma_load_2d(sA + s * Plan::kA, &maps.a, &full_b[s], k0, cur.t.m0);
-                    } else if (KIND == G_SHARED_GATEUP) {
-                        tma_load_2d(sA + s * Plan::kA, &maps.a, &full_b[s], k0, cur.t.m0);
-                        tma_load_2d(sA + s * Plan::kA + 64 * 128, &maps.a2, &full_b[s], k0, cur.t.m0);
+    if (warp == 9) {
+        // ------------------------------------------------------------ loader (one thread)
+        if (lane == 0) {
+            tma_prefetch_desc(&maps.b);
+            Cursor<KIND, NT> cb, cr;       // activation / plain-weight stages, raw-weight stages
+            cb.begin(p);
+            cr = cb;
+            uint32_t it_b = 0, it_r = 0;
+            uint32_t last_b[STAGES];
+            uint32_t last_r[RS];
+            for (int i = 0; i < STAGES; ++i) last_b[i] = 0xFFFFFFFFu;
+            for (int i = 0; i < RS; ++i) last_r[i] = 0xFFFFFFFFu;
+            bool ok = true;
+            while (ok && !cb.done) {
+                // raw weights run up to RS stages ahead of the activation tiles
+                while (!cr.done && it_r < it_b + RS) {
+                    const int rs = it_r % RS;
+                    const uint32_t ph = (it_r / RS) & 1;
+                    if (!mbar_wait(&raw_empty[rs], ph ^ 1, abort_flag, kWaitLimitNs)) { ok = false; break; }
+                    if (S::tma_a(p, cr.seg)) mbar_arrive(&raw_full[rs]);
+                    else issue_raw<KIND, NT>(p, cr, sRaw + rs * Plan::kRaw, &raw_full[rs]);
+                    last_r[rs] = ph;
+                    cr.next_stage(p);
+                    ++it_r;
+                }
+                if (!ok) break;
+                const int s = it_b % STAGES;
+                const uint32_t ph = (it_b / STAGES) & 1;
+                if (!mbar_wait(&empty[s], ph ^ 1, abort_flag, kWaitLimitNs)) break;
+                const bool ta = S::tma_a(p, cb.seg);
+                const int k0 = cb.ks * 64;
+                mbar_arrive_expect_tx(&full_b[s], Plan::kB + (ta ? Plan::kA : 0));
+                uint8_t* dB = sB + s * Plan::kB;
+                if (KIND == G_UPROJ && cb.seg < p.G) tma_load_3d(dB, &maps.b, &full_b[s], k0, cb.seg, cb.t.b0);
+                else if (KIND == G_UPROJ) tma_load_3d(dB, &maps.b2, &full_b[s], k0, cb.t.b0, cb.seg - p.G);
+                else if (cb.seg > 0) tma_load_2d(dB, &maps.b2, &full_b[s], k0, cb.t.b0);
+                else tma_load_2d(dB, &maps.b, &full_b[s], k0, cb.t.b0);
+                if (ta) {
+                    if (KIND == G_SHARED_GATEUP) {
+                        tma_load_2d(sA + s * Plan::kA, &maps.a, &full_b[s], k0, cb.t.m0);
+                        tma_load_2d(sA + s * Plan::kA + 64 * 128, &maps.a2, &full_b[s], k0, cb.t.m0);
+                    } else {
+                        tma_load_2d(sA + s * Plan::kA, &maps.a, &full_b[s], k0, cb.t.m0);
                     }
-                    last_phase[s] = ph;
                 }
-                if (!S::kTmaA) {
-                    uint32_t o[32];
-                    dequant_row<KIND>(p, cur.seg, ring[slot], o);
-                    store_row_swizzled(sA + s * Plan::kA, r, o);
-                    fence_proxy_async_smem();
-                    mbar_arrive(&full_a[s]);
-                    if (!pre.done) { load_raw<KIND, NT>(p, pre, r, ring[slot]); pre.next_stage(p); }
-                }
-                cur.next_stage(p);
-                ++it;
+                last_b[s] = ph;
+                cb.next_stage(p);
+                ++it_b;
+            }
+            if (*abort_flag) {
+                // let every copy already issued land before the CTA can leave
+                volatile int dummy = 0;
+                for (int i = 0; i < STAGES; ++i)
+                    if (last_b[i] != 0xFFFFFFFFu) mbar_wait(&full_b[i], last_b[i], &dummy, kWaitLimitNs);
+                for (int i = 0; i < RS; ++i)
+                    if (last_r[i] != 0xFFFFFFFFu) mbar_wait(&raw_full[i], last_r[i], &dummy, kWaitLimitNs);
             }
         }
-        goto producer_done;
-    producer_abort:
-        if (r == 0) {
-            // let every load already issued land before the CTA can leave
-            for (int s = 0; s < STAGES; ++s)
-                if (last_phase[s] != 0xFFFFFFFFu) {
-                    volatile int dummy = 0;
-                    mbar_wait(&full_b[s], last_phase[s], &dummy, kWaitLimitNs);
-                }
+        __syncwarp();
+    } else if (warp >= 4 && warp < 8) {
+        // ------------------------------------------------------------ converters
+        const int r = threadIdx.x - 128;           // A row
+        Cursor<KIND, NT> cur;
+        cur.begin(p);
+        uint32_t it = 0;
+        while (!cur.done) {
+            const int s = it % STAGES, rs = it % RS;
+            const uint32_t ph = (it / STAGES) & 1, rph = (it / RS) & 1;
+            const bool ta = S::tma_a(p, cur.seg);
+            if (!mbar_wait(&raw_full[rs], rph, abort_flag, kWaitLimitNs)) break;
+            if (!mbar_wait(&empty[s], ph ^ 1, abort_flag, kWaitLimitNs)) break;
+            if (!ta) {
+                RawRow raw;
+                raw_row_from_smem<KIND>(p, sRaw + rs * Plan::kRaw, r, raw);
+                uint32_t o[32];
+                dequant_row<KIND>(p, cur.seg, raw, o);
+                store_row_swizzled(sA + s * Plan::kA, r, o);
+                fence_proxy_async_smem();
+            }
+            __syncwarp();
+            if (lane == 0) {
+                // every stage completes a phase of full_a and raw_empty, so their parity stays in step
+                mbar_arrive(&full_a[s]);
+                mbar_arrive(&raw_empty[rs]);
+            }
+            cur.next_stage(p);
+            ++it;
         }
-    producer_done:;
     } else if (warp == 8) {
         // ------------------------------------------------------------ MMA issuer
         if (lane == 0) {
@@ -543,14 +624,15 @@ __global__ void __launch_bounds__(288, 1) k_umma_gemm(const __grid_constant__ Tm
                 tc_fence_after();
                 const uint32_t d_tmem = tmem_base + acc * NT;
                 const int n_mma = (KIND == G_GATEUP || KIND == G_DOWN) ? ((cur.t.n + 15) & ~15) : NT;
-                const uint32_t idesc = idesc_f16(128, n_mma, S::kBf16);
                 bool first = true;
                 bool ok = true;
                 while (true) {
                     const int s = it % STAGES;
                     const uint32_t ph = (it / STAGES) & 1;
+                    const bool ta = S::tma_a(p, cur.seg);
+                    const uint32_t idesc = idesc_f16(128, n_mma, ta ? 1 : 0);
                     if (!mbar_wait(&full_b[s], ph, abort_flag, kWaitLimitNs)) { ok = false; break; }
-                    if (!S::kTmaA && !mbar_wait(&full_a[s], ph, abort_flag, kWaitLimitNs)) { ok = false; break; }
+                    if (!mbar_wait(&full_a[s], ph, abort_flag, kWaitLimitNs)) { ok = false; break; }
                     tc_fence_after();
                     const uint64_t a_desc = sdesc_k128(smem_u32(sA + s * Plan::kA));
                     const uint64_t b_desc = sdesc_k128(smem_u32(sB + s * Plan::kB));
@@ -585,6 +667,19 @@ __global__ void __launch_bounds__(288, 1) k_umma_gemm(const __grid_constant__ Tm
         while (!cur.done) {
             const int acc = tcount & 1;
             const uint32_t ph = (tcount >> 1) & 1;
+            // the tile's routing metadata goes to shared memory while the
+            // accumulator is still being computed
+            if (KIND == G_DPROJ) {
+                uint32_t* mmask = reinterpret_cast<uint32_t*>(xchg);
+                int* mslot = reinterpret_cast<int*>(mmask + NT);
+                for (int i = threadIdx.x; i < cur.t.n; i += 128)
+                    mmask[i] = __ldg(p.tgmask + (size_t)(cur.t.b0 + i) * p.G + cur.t.mat);
+                for (int i = threadIdx.x; i < cur.t.n * p.K; i += 128)
+                    mslot[i] = __ldg(p.pair_slot + (size_t)cur.t.b0 * p.K + i);
+            } else if (KIND == G_DOWN) {
+                for (int i = threadIdx.x; i < cur.t.n; i += 128) xchg[i] = __ldg(p.w + __ldg(p.slot_pair + cur.t.b0 + i));
+            }
+            named_bar_sync(1, 128);
             if (!mbar_wait(&tfull[acc], ph, abort_flag, kWaitLimitNs)) break;
             tc_fence_after();
             const uint32_t taddr = tmem_base + ((uint32_t)(32 * warp) << 16) + acc * NT;
@@ -595,9 +690,10 @@ __global__ void __launch_bounds__(288, 1) k_umma_gemm(const __grid_constant__ Tm
                 epilogue_chunk<KIND, NT>(p, cur.t, warp, lane, c0, rr, xchg);
             }
             tc_fence_before();
-            mbar_arrive(&tempty[acc]);
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&tempty[acc]);
+            named_bar_sync(1, 128);
             ++tcount;
-            // skip to the next tile
             cur.next_tile(p);
         }
     }
@@ -842,12 +938,25 @@ static bool make_map_s(CUtensorMap* m, const void* base, uint64_t T, uint64_t G,
               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// 3-D map over the shared hidden [2][T][Fs] bf16 (high, low), box = 64 x box_rows x 1.
+static bool make_map_zsh(CUtensorMap* m, const void* base, uint64_t T, uint64_t Fs, uint32_t box_rows) {
+    EncodeTiledFn fn = encode_fn();
+    if (!fn) return false;
+    cuuint64_t dims[3] = {Fs, T, 2};
+    cuuint64_t strides[2] = {Fs * 2, T * Fs * 2};
+    cuuint32_t box[3] = {64, box_rows, 1};
+    cuuint32_t es[3] = {1, 1, 1};
+    return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, es,
+              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 static int g_num_sms = 0;
 
-template <int KIND, int NT, int STAGES>
+template <int KIND, int NT, int STAGES, int RS>
 static cudaError_t launch_gemm(const TmaMaps& maps, const PrefillParams& p, cudaStream_t st, int max_tiles) {
-    const size_t smem = SmemPlan<NT, STAGES>::kTotal;
-    auto kern = k_umma_gemm<KIND, NT, STAGES>;
+    const size_t smem = SmemPlan<NT, STAGES, RS>::kTotal;
+    auto kern = k_umma_gemm<KIND, NT, STAGES, RS>;
     cudaError_t e = ensure_smem(reinterpret_cast<const void*>(kern), smem);
     if (e != cudaSuccess) return e;
     if (g_num_sms == 0) {
@@ -856,7 +965,7 @@ static cudaError_t launch_gemm(const TmaMaps& maps, const PrefillParams& p, cuda
         cudaDeviceGetAttribute(&g_num_sms, cudaDevAttrMultiProcessorCount, dev);
     }
     const int grid = max(1, min(g_num_sms, max_tiles));
-    kern<<<grid, 288, smem, st>>>(maps, p);
+    kern<<<grid, kGemmThreads, smem, st>>>(maps, p);
     return cudaGetLastError();
 }
 
@@ -883,7 +992,8 @@ cudaError_t run_prefill_path(PrefillParams p, cudaStream_t st, void* memset_base
     ok &= make_map_2d(&m_gu.b, p.hperm, false, (uint64_t)T * K, L, L, kNtExpert);
     ok &= make_map_2d(&m_down.b, p.zperm, false, (uint64_t)T * K, F, F, kNtExpert);
     ok &= make_map_s(&m_u.b, p.s, T, G, L, kNtDense);
-    ok &= make_map_2d(&m_u.b2, p.zsh, false, T, Fs, Fs, kNtDense);
+    ok &= make_map_2d(&m_u.a, p.sd, true, H, Fs, Fs, 128);           // shared down weights (bf16)
+    ok &= make_map_zsh(&m_u.b2, p.zsh, T, Fs, kNtDense);               // shared hidden, bf16 high / low
     if (!ok) return cudaErrorInvalidValue;
 
     if (memset_bytes) {
@@ -894,7 +1004,7 @@ cudaError_t run_prefill_path(PrefillParams p, cudaStream_t st, void* memset_base
     k_x_to_fp16<<<T, 256, 0, st>>>(p);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
     mark(st);
-    if ((e = launch_gemm<G_ROUTER, kNtDense, 4>(m_router, p, st, (E / 128) * ttiles)) != cudaSuccess) return e;
+    if ((e = launch_gemm<G_ROUTER, kNtDense, 4, 1>(m_router, p, st, (E / 128) * ttiles)) != cudaSuccess) return e;
     mark(st);
     k_topk<<<(T * 32 + 255) / 256, 256, 0, st>>>(p);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
@@ -904,19 +1014,19 @@ cudaError_t run_prefill_path(PrefillParams p, cudaStream_t st, void* memset_base
     k_bucket_scatter<<<(pairs + 255) / 256, 256, 0, st>>>(p);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
     mark(st);
-    if ((e = launch_gemm<G_SHARED_GATEUP, kNtDense, 4>(m_shared, p, st, (Fs / 64) * ttiles)) != cudaSuccess) return e;
+    if ((e = launch_gemm<G_SHARED_GATEUP, kNtDense, 4, 1>(m_shared, p, st, (Fs / 64) * ttiles)) != cudaSuccess) return e;
     mark(st);
-    if ((e = launch_gemm<G_DPROJ, kNtDense, 4>(m_d, p, st, G * (L / 128) * ttiles)) != cudaSuccess) return e;
+    if ((e = launch_gemm<G_DPROJ, kNtDense, 3, 6>(m_d, p, st, G * (L / 128) * ttiles)) != cudaSuccess) return e;
     mark(st);
     const int max_etiles = min(E, pairs) + pairs / kNtExpert + 1;
-    if ((e = launch_gemm<G_GATEUP, kNtExpert, 6>(m_gu, p, st, (F / 64) * max_etiles)) != cudaSuccess) return e;
+    if ((e = launch_gemm<G_GATEUP, kNtExpert, 4, 8>(m_gu, p, st, (F / 64) * max_etiles)) != cudaSuccess) return e;
     mark(st);
-    if ((e = launch_gemm<G_DOWN, kNtExpert, 6>(m_down, p, st, (L / 128) * max_etiles)) != cudaSuccess) return e;
+    if ((e = launch_gemm<G_DOWN, kNtExpert, 4, 8>(m_down, p, st, (L / 128) * max_etiles)) != cudaSuccess) return e;
     mark(st);
     k_combine<<<T, 256, 0, st>>>(p);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
     mark(st);
-    if ((e = launch_gemm<G_UPROJ, kNtDense, 4>(m_u, p, st, (H / 128) * ttiles)) != cudaSuccess) return e;
+    if ((e = launch_gemm<G_UPROJ, kNtDense, 3, 6>(m_u, p, st, (H / 128) * ttiles)) != cudaSuccess) return e;
     mark(st);
     return cudaSuccess;
 }
@@ -929,7 +1039,7 @@ cudaError_t run_prefill_route(PrefillParams p, cudaStream_t st) {
     ok &= make_map_2d(&m.b, p.x, true, p.T, p.H, p.H, kNtDense);
     if (!ok) return cudaErrorInvalidValue;
     const int ttiles = (p.T + kNtDense - 1) / kNtDense;
-    cudaError_t e = launch_gemm<G_ROUTER, kNtDense, 4>(m, p, st, (p.E / 128) * ttiles);
+    cudaError_t e = launch_gemm<G_ROUTER, kNtDense, 4, 1>(m, p, st, (p.E / 128) * ttiles);
     if (e != cudaSuccess) return e;
     k_topk<<<(p.T * 32 + 255) / 256, 256, 0, st>>>(p);
     return cudaGetLastError();
