@@ -40,7 +40,7 @@ constexpr int kPrefillMinT = 64;
 
 // (the router GEMM tiles the experts by 128)
 bool use_prefill(const lmoe_cfg& c, int T) {
-    return T >= kPrefillMinT && c.router_dtype == LMOE_BF16 && c.n_experts % 128 == 0;
+    return T >= kPrefillMinT && c.router_dtype == LMOE_BF16 && c.n_experts % 128 == 0 && c.n_groups <= 62;
 }
 
 // Workspace of the few-token path (first) and of the tensor-core path; both

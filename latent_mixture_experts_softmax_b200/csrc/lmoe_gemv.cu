@@ -152,9 +152,8 @@ __device__ __forceinline__ void dot4_f32(float4 w, const float* xs, int ld, int 
 // One row of a plain bf16 / fp32 matrix (K contiguous) against xs, the warp's
 // lanes splitting K; ten 16-byte loads per lane are issued before any
 // arithmetic.  The per-lane partial sums are left in acc (reduce with warp_sum).
-template <int NT, bool kBF16>
+template <int NT, bool kBF16, int kB = 10>
 __device__ __forceinline__ void row_dot(const void* wrow, int K, const float* xs, int ld, int lane, float (&acc)[NT]) {
-    constexpr int kB = 10;
     constexpr int kPer = kBF16 ? 8 : 4;          // elements per 16-byte load
     constexpr int kStep = 32 * kPer;
     for (int base = 0; base < K; base += kB * kStep) {
@@ -258,6 +257,112 @@ __device__ __forceinline__ void warp_argmax(float& v, int& i) {
     }
 }
 
+// Softmax top-K of token t by one warp: NV logits per lane in registers; K
+// rounds of a warp arg-max (ties to the lower index); w_k = exp(l_k - l_1) /
+// sum over the kept of exp(l_j - l_1).
+template <int NV>
+__device__ __forceinline__ void topk_warp(const FwdParams& p, int t, int lane) {
+    const int E = p.E, K = p.K;
+    float v[NV];
+#pragma unroll
+    for (int j = 0; j < NV; ++j) {
+        const int e = lane + 32 * j;
+        v[j] = e < E ? __ldcg(p.r.logits + (size_t)t * E + e) : -INFINITY;
+    }
+    uint32_t taken = 0;
+    float lmax = 0.f, denom = 0.f, my_l = 0.f;
+    int my_e = 0;
+    for (int k = 0; k < K; ++k) {
+        float bv = -INFINITY;
+        int bi = 0x7fffffff;
+#pragma unroll
+        for (int j = 0; j < NV; ++j) {
+            const int e = lane + 32 * j;
+            if (e < E && !(taken >> j & 1u) && (v[j] > bv || (v[j] == bv && e < bi))) { bv = v[j]; bi = e; }
+        }
+        warp_argmax(bv, bi);
+        if ((bi & 31) == lane && bi < E) taken |= 1u << (bi >> 5);
+        if (k == 0) lmax = bv;
+        if (k == lane) { my_l = bv; my_e = bi; }
+        denom += expf(bv - lmax);
+    }
+    if (lane < K) {
+        p.r.idx[(size_t)t * K + lane] = my_e;
+        p.r.w[(size_t)t * K + lane] = expf(my_l - lmax) / denom;
+    }
+}
+
+// Bucketing of at most 64 (token, k) pairs by one warp: slots ordered by
+// (expert, pair index), distinct experts ascending; O(n^2) comparisons.
+__device__ void buckets_small_warp(const FwdParams& p, int lane) {
+    const int K = p.K, G = p.G, T = p.T, E = p.E, n = T * K;
+    const Routing& r = p.r;
+    __shared__ int se[64];
+    __shared__ uint8_t sf[64];
+    int e_i[2], g_i[2];
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+        const int i = lane + 32 * h;
+        e_i[h] = 0x7fffffff;
+        g_i[h] = 0;
+        if (i < n) {
+            int e = r.idx[i];
+            if (e < 0 || e >= E) { set_status(p.ctrl, LMOE_ERR_DEVICE_CHECK); e = 0; r.idx[i] = 0; }
+            int g = p.group[e];
+            if (g >= G) { set_status(p.ctrl, LMOE_ERR_DEVICE_CHECK); g = 0; }
+            e_i[h] = e;
+            g_i[h] = g;
+        }
+        se[i] = e_i[h];
+    }
+    for (int i = lane; i < T * G; i += 32) r.tghit[i] = 0;
+    for (int g = lane; g < G; g += 32) r.ghit[g] = 0;
+    __syncwarp();
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+        const int i = lane + 32 * h;
+        int before = 0;
+        for (int j = 0; j < i && j < n; ++j) before += se[j] == e_i[h];
+        sf[i] = (i < n && before == 0);
+    }
+    __syncwarp();
+    int n_first = 0;
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+        const int i = lane + 32 * h;
+        if (i >= n) continue;
+        int less = 0, same_before = 0, cnt = 0, u = 0;
+        for (int j = 0; j < n; ++j) {
+            const int ej = se[j];
+            less += ej < e_i[h];
+            same_before += (j < i && ej == e_i[h]);
+            cnt += ej == e_i[h];
+            u += (sf[j] && ej < e_i[h]);
+        }
+        const int slot = less + same_before;
+        r.slot_pair[slot] = i;
+        r.pair_slot[i] = slot;
+        if (sf[i]) {
+            r.uexp[u] = e_i[h];
+            r.ucnt[u] = cnt;
+            r.uoff[u] = less;
+            ++n_first;
+        }
+    }
+    __syncwarp();
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+        const int i = lane + 32 * h;
+        if (i < n) {
+            r.tghit[(i / K) * G + g_i[h]] = 1;
+            atomicAdd(r.ghit + g_i[h], 1);
+        }
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) n_first += __shfl_xor_sync(0xffffffffu, n_first, o);
+    if (lane == 0) *r.n_unique = n_first;
+}
+
 __device__ void topk_and_buckets(const FwdParams& p) {
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, nw = blockDim.x >> 5;
     const int E = p.E, K = p.K, G = p.G, T = p.T;
@@ -271,39 +376,11 @@ __device__ void topk_and_buckets(const FwdParams& p) {
         }
     } else {
         for (int t = warp; t < T; t += nw) {
-            float v[kMaxExpertsTopk / 32];
-            uint32_t taken = 0;
-#pragma unroll
-            for (int j = 0; j < kMaxExpertsTopk / 32; ++j) {
-                const int e = lane + 32 * j;
-                v[j] = e < E ? __ldcg(r.logits + (size_t)t * E + e) : -INFINITY;
-            }
-            float lmax = 0.f, denom = 0.f;
-            float sel_l[kMaxTopK];
-            int sel_e[kMaxTopK];
-            for (int k = 0; k < K; ++k) {
-                float bv = -INFINITY;
-                int bi = 0x7fffffff;
-#pragma unroll
-                for (int j = 0; j < kMaxExpertsTopk / 32; ++j) {
-                    const int e = lane + 32 * j;
-                    if (e < E && !(taken >> j & 1u) && (v[j] > bv || (v[j] == bv && e < bi))) { bv = v[j]; bi = e; }
-                }
-                warp_argmax(bv, bi);
-                if ((bi & 31) == lane && bi < E) taken |= 1u << (bi >> 5);
-                if (k == 0) lmax = bv;
-                sel_l[k] = bv;
-                sel_e[k] = bi;
-                denom += expf(bv - lmax);
-            }
-            if (lane < K) {
-                float lk = 0.f;
-                int ek = 0;
-#pragma unroll
-                for (int k = 0; k < kMaxTopK; ++k) if (k == lane) { lk = sel_l[k]; ek = sel_e[k]; }
-                r.idx[(size_t)t * K + lane] = ek;
-                r.w[(size_t)t * K + lane] = expf(lk - lmax) / denom;
-            }
+            if (E <= 64) topk_warp<2>(p, t, lane);
+            else if (E <= 128) topk_warp<4>(p, t, lane);
+            else if (E <= 256) topk_warp<8>(p, t, lane);
+            else if (E <= 512) topk_warp<16>(p, t, lane);
+            else topk_warp<32>(p, t, lane);
         }
     }
     __syncthreads();
@@ -314,6 +391,10 @@ __device__ void topk_and_buckets(const FwdParams& p) {
         }
     }
     if (!p.do_buckets) return;
+    if (T * K <= 64) {
+        if (warp == 0) buckets_small_warp(p, lane);
+        return;
+    }
 
     // --- bucketing: counts, distinct experts, slots, group hits
     __shared__ int cnt[kMaxExpertsTopk];
@@ -462,7 +543,7 @@ __device__ __forceinline__ void mma_du_rows(const uint8_t* mat, int R, int C, in
     const size_t qrow = FMT == LMOE_Q8_0 ? 32 : 16;
     const uint16_t* dsc = reinterpret_cast<const uint16_t*>(mat + (size_t)R * C / 32 * qrow);
     const __half* xrow = xs + (size_t)g * KP;
-    constexpr int kU = 8;                                  // blocks whose loads are issued together
+    constexpr int kU = 4;                                  // blocks whose loads are issued together
     for (int kb = kb0; kb < kb1; kb += kU) {
         uint32_t w[kU][4];
         uint16_t d[kU][2];
@@ -527,7 +608,7 @@ __device__ __forceinline__ void mma_nvfp4_rows(const uint8_t* q, const uint8_t* 
     const int lane = threadIdx.x & 31, g = lane >> 2, t = lane & 3;
     const int KP = C + kXPad;
     const __half* xrow = xs + (size_t)g * KP;
-    constexpr int kU = 8;
+    constexpr int kU = 4;
     for (int kc = kc0; kc < kc1; kc += kU) {
         uint32_t wg[kU], wh[kU], sg[kU], sh[kU];
 #pragma unroll
@@ -589,7 +670,7 @@ __device__ __forceinline__ void reduce_frags(float (&acc)[4], float* red) {
 
 // kernel 2: h16[t][g] = D_g x_t for hit groups; CTA = 16 rows of one group
 template <int FMT>
-__global__ void __launch_bounds__(32 * kMmaWarps) k_dproj_mma(FwdParams p) {
+__global__ void __launch_bounds__(32 * kMmaWarps, 4) k_dproj_mma(FwdParams p) {
     extern __shared__ __align__(16) uint8_t smem_u8[];
     const int g = blockIdx.y;
     if (__ldcg(p.r.ghit + g) == 0) return;
@@ -619,7 +700,7 @@ __global__ void __launch_bounds__(32 * kMmaWarps) k_dproj_mma(FwdParams p) {
 
 // kernel 3: z16[slot] = silu(W_gate h) * (W_up h) for the expert's slots;
 // CTA = 16 features (gate and up rows) of one distinct expert
-__global__ void __launch_bounds__(32 * kMmaWarps) k_gateup_mma(FwdParams p) {
+__global__ void __launch_bounds__(32 * kMmaWarps, 3) k_gateup_mma(FwdParams p) {
     extern __shared__ __align__(16) uint8_t smem_u8[];
     const int j = blockIdx.y;
     if (j >= __ldcg(p.r.n_unique)) return;
@@ -680,9 +761,9 @@ __global__ void __launch_bounds__(32 * kMmaWarps) k_gateup_mma(FwdParams p) {
 // CTA = 16 latent rows of one group; each warp takes whole experts of the
 // group (K = ffn in one warp, no reduction), the group sum is formed in a
 // fixed order afterwards.
-constexpr int kDownWarps = 8;
+constexpr int kDownWarps = 4;
 
-__global__ void __launch_bounds__(32 * kDownWarps) k_down_mma(FwdParams p) {
+__global__ void __launch_bounds__(32 * kDownWarps, 4) k_down_mma(FwdParams p) {
     extern __shared__ __align__(16) uint8_t smem_u8[];
     const int g = blockIdx.y;
     const int L = p.L, F = p.F, T = p.T, r0 = blockIdx.x * 16;
@@ -695,7 +776,8 @@ __global__ void __launch_bounds__(32 * kDownWarps) k_down_mma(FwdParams p) {
     // group label and slot of every (token, k) pair, for the final sum
     __shared__ uint8_t pg[kMaxTopK * 64];
     __shared__ int pslot[kMaxTopK * 64];
-    for (int i = threadIdx.x; i < T * p.K; i += blockDim.x) {
+    const bool pairs_in_smem = T * p.K <= kMaxTopK * 64;
+    for (int i = threadIdx.x; pairs_in_smem && i < T * p.K; i += blockDim.x) {
         const int e = __ldcg(p.r.idx + i);
         pg[i] = p.group[e] < p.G ? p.group[e] : 0;
         pslot[i] = __ldcg(p.r.pair_slot + i);
@@ -748,7 +830,11 @@ __global__ void __launch_bounds__(32 * kDownWarps) k_down_mma(FwdParams p) {
         if (hit) {
             for (int k = 0; k < p.K; ++k) {
                 const int pair = t * p.K + k;
-                if (pg[pair] == g) v += part[(size_t)pslot[pair] * 16 + row];
+                if (pairs_in_smem) {
+                    if (pg[pair] == g) v += part[(size_t)pslot[pair] * 16 + row];
+                } else if (p.group[__ldcg(p.r.idx + pair)] == g) {
+                    v += part[(size_t)__ldcg(p.r.pair_slot + pair) * 16 + row];
+                }
             }
         }
         p.s16[((size_t)t * p.G + g) * L + r0 + row] = __float2half_rn(v);
@@ -759,7 +845,7 @@ __global__ void __launch_bounds__(32 * kDownWarps) k_down_mma(FwdParams p) {
 // one for the shared expert's down projection; the last part of a row tile
 // to finish sums the parts in a fixed order, adds the residual, writes y.
 template <int FMT>
-__global__ void __launch_bounds__(32 * kMmaWarps) k_uproj_mma(FwdParams p) {
+__global__ void __launch_bounds__(32 * kMmaWarps, 3) k_uproj_mma(FwdParams p) {
     extern __shared__ __align__(16) uint8_t smem_u8[];
     const int part = blockIdx.y;
     const int H = p.H, L = p.L, G = p.G, T = p.T, r0 = blockIdx.x * 16;
@@ -810,7 +896,7 @@ __global__ void __launch_bounds__(32 * kMmaWarps) k_uproj_mma(FwdParams p) {
                     float a2[8];
 #pragma unroll
                     for (int t = 0; t < 8; ++t) a2[t] = 0.f;
-                    row_dot<8, true>(p.sd + (size_t)row * Fs, Fs, as, ld, lane, a2);
+                    row_dot<8, true, 3>(p.sd + (size_t)row * Fs, Fs, as, ld, lane, a2);
 #pragma unroll
                     for (int t = 0; t < 8; ++t) {
                         const float v = warp_sum(a2[t]);
@@ -832,13 +918,17 @@ __global__ void __launch_bounds__(32 * kMmaWarps) k_uproj_mma(FwdParams p) {
     if (!s_last) return;
     __threadfence();
     __shared__ uint8_t th[64 * kMaxGroups];
-    for (int i = threadIdx.x; i < T * G; i += blockDim.x) th[i] = p.r.tghit[i] && __ldcg(p.r.ghit + i % G) > 0;
+    const bool hits_in_smem = T * G <= 64 * kMaxGroups;
+    for (int i = threadIdx.x; hits_in_smem && i < T * G; i += blockDim.x)
+        th[i] = p.r.tghit[i] && __ldcg(p.r.ghit + i % G) > 0;
     __syncthreads();
     for (int i = threadIdx.x; i < T * 16; i += blockDim.x) {
         const int t = i >> 4, row = r0 + (i & 15);
         float v = __ldcg(p.ypart + ((size_t)G * T + t) * H + row);
-        for (int g = 0; g < G; ++g)
-            if (th[t * G + g]) v += __ldcg(p.ypart + ((size_t)g * T + t) * H + row);
+        for (int g = 0; g < G; ++g) {
+            const bool h = hits_in_smem ? th[t * G + g] != 0 : (p.r.tghit[(size_t)t * G + g] && __ldcg(p.r.ghit + g) > 0);
+            if (h) v += __ldcg(p.ypart + ((size_t)g * T + t) * H + row);
+        }
         if (p.residual) v += bf16_bits_to_f32(p.residual[(size_t)t * H + row]);
         p.y[(size_t)t * H + row] = f32_to_bf16_bits(v);
     }

@@ -13,12 +13,6 @@ __device__ __forceinline__ uint32_t smem_u32(const void* p) {
     return static_cast<uint32_t>(__cvta_generic_to_shared(p));
 }
 
-__device__ __forceinline__ uint64_t globaltimer_ns() {
-    uint64_t t;
-    asm volatile("mov.u64 %0, %globaltimer;" : "=l"(t));
-    return t;
-}
-
 // ---------------------------------------------------------------------------
 // mbarrier
 // ---------------------------------------------------------------------------
@@ -52,18 +46,21 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
     return ok != 0;
 }
 
-// Wait for the phase with the given parity to complete, at most `limit_ns`.
-// On timeout (or when another thread of the CTA already gave up, *abort != 0)
-// returns false after raising *abort.
-__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort, uint64_t limit_ns) {
+// Wait for the phase with the given parity to complete, for at most
+// `limit_cycles` SM clock cycles (the SM-local counter is cheap to read; the
+// global timer is not).  On timeout (or when another thread of the CTA already
+// gave up, *abort != 0) returns false after raising *abort.
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort, uint64_t limit_cycles) {
     if (mbar_try_wait(bar, parity)) return true;
-    const uint64_t t0 = globaltimer_ns();
-    while (true) {
-        if (*abort) return false;
+    const uint64_t t0 = clock64();
+    for (uint32_t i = 1;; ++i) {
         if (mbar_try_wait(bar, parity)) return true;
-        if (globaltimer_ns() - t0 > limit_ns) {
-            *abort = 1;
-            return false;
+        if ((i & 63) == 0) {
+            if (*abort) return false;
+            if ((uint64_t)(clock64() - t0) > limit_cycles) {
+                *abort = 1;
+                return false;
+            }
         }
     }
 }

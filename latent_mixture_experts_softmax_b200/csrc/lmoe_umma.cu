@@ -36,7 +36,7 @@ namespace lmoe {
 
 using namespace sm100;
 
-constexpr uint64_t kWaitLimitNs = 2000000000ull;   // 2 s per barrier wait
+constexpr uint64_t kWaitLimit = 4000000000ull;   // SM cycles per barrier wait (about 2 s)
 
 // ---------------------------------------------------------------------------
 // tiles
@@ -136,11 +136,13 @@ struct Sched {
     static constexpr bool kAnyTmaA = KIND == G_ROUTER || KIND == G_SHARED_GATEUP || KIND == G_UPROJ;
 };
 
-// Walks the (tile, segment, 64-wide K stage) sequence of one CTA.
+// Walks the (tile, segment, 64-wide K stage) sequence of one CTA.  The
+// active segments of a tile are read once, when the tile is entered.
 template <int KIND, int NT>
 struct Cursor {
     using S = Sched<KIND, NT>;
     int tile, seg, ks, nk, ntiles;
+    uint64_t segmask;
     bool done;
     TileRef t;
     __device__ void begin(const PrefillParams& p) {
@@ -155,20 +157,21 @@ struct Cursor {
             if (tile >= ntiles) { done = true; return; }
             t = S::get(p, tile);
             if (!t.valid) continue;
+            segmask = 0;
+            for (int sg = 0; sg < S::num_segs(p); ++sg)
+                if (S::seg_active(p, t, sg)) segmask |= 1ull << sg;
             seg = -1;
             if (next_seg(p)) return;
         }
     }
     // advance to the next active segment of the current tile; false if none
     __device__ bool next_seg(const PrefillParams& p) {
-        while (++seg < S::num_segs(p)) {
-            if (S::seg_active(p, t, seg)) {
-                ks = 0;
-                nk = S::seg_k(p, seg) / 64;
-                return true;
-            }
-        }
-        return false;
+        const uint64_t higher = seg < 0 ? segmask : (segmask & ~((2ull << seg) - 1));
+        if (!higher) return false;
+        seg = __ffsll((long long)higher) - 1;
+        ks = 0;
+        nk = S::seg_k(p, seg) / 64;
+        return true;
     }
     __device__ void next_stage(const PrefillParams& p) {
         if (++ks < nk) return;
@@ -177,9 +180,7 @@ struct Cursor {
     }
     __device__ bool last_stage_of_tile(const PrefillParams& p) const {
         if (ks + 1 < nk) return false;
-        for (int s2 = seg + 1; s2 < S::num_segs(p); ++s2)
-            if (S::seg_active(p, t, s2)) return false;
-        return true;
+        return (segmask & ~((2ull << seg) - 1)) == 0;
     }
 };
 
@@ -252,32 +253,6 @@ __device__ __forceinline__ void issue_raw(const PrefillParams& p, const Cursor<K
     }
 }
 
-// Row r of a raw slot -> the register form the dequantiser takes.
-struct RawRow {
-    uint4 q[4];
-    uint32_t s;
-};
-
-template <int KIND>
-__device__ __forceinline__ void raw_row_from_smem(const PrefillParams& p, const uint8_t* slot, int r, RawRow& raw) {
-    const int pb = raw_part_bytes<KIND>(p.du_fmt);
-    if ((KIND == G_DPROJ || KIND == G_UPROJ) && p.du_fmt == LMOE_Q8_0) {
-        raw.q[0] = *reinterpret_cast<const uint4*>(slot + r * 32);
-        raw.q[1] = *reinterpret_cast<const uint4*>(slot + r * 32 + 16);
-        raw.q[2] = *reinterpret_cast<const uint4*>(slot + pb + r * 32);
-        raw.q[3] = *reinterpret_cast<const uint4*>(slot + pb + r * 32 + 16);
-    } else {
-        raw.q[0] = *reinterpret_cast<const uint4*>(slot + r * 16);
-        raw.q[1] = *reinterpret_cast<const uint4*>(slot + pb + r * 16);
-    }
-    if (KIND == G_DPROJ || KIND == G_UPROJ) {
-        const uint16_t* d = reinterpret_cast<const uint16_t*>(slot + 2 * pb);
-        raw.s = (uint32_t)d[r] | ((uint32_t)d[128 + r] << 16);
-    } else {
-        raw.s = reinterpret_cast<const uint32_t*>(slot + 2 * pb)[r];
-    }
-}
-
 __device__ __forceinline__ uint32_t h2_bits(__half2 h) { return *reinterpret_cast<uint32_t*>(&h); }
 __device__ __forceinline__ __half2 bits_h2(uint32_t u) { return *reinterpret_cast<__half2*>(&u); }
 
@@ -287,77 +262,67 @@ __device__ __forceinline__ void bytes_to_h2x2(uint32_t w, uint32_t& lo, uint32_t
     hi = __byte_perm(w, 0x64646464u, 0x4342);
 }
 
-// Dequantise one row's 64 columns into 32 half2 (element order).
+// Half h (columns 32h .. 32h+31) of row r of a raw slot -> 16 half2.
 template <int KIND>
-__device__ __forceinline__ void dequant_row(const PrefillParams& p, int seg, const RawRow& raw, uint32_t (&o)[32]) {
-    if (KIND == G_DPROJ || (KIND == G_UPROJ && seg < p.G)) {
-        const __half2 d0 = __half2half2(__ushort_as_half((unsigned short)(raw.s & 0xFFFF)));
-        const __half2 d1 = __half2half2(__ushort_as_half((unsigned short)(raw.s >> 16)));
+__device__ __forceinline__ void dequant_half(const PrefillParams& p, const uint8_t* slot, int r, int h,
+                                             uint32_t (&o)[16]) {
+    const int pb = raw_part_bytes<KIND>(p.du_fmt);
+    if (KIND == G_DPROJ || KIND == G_UPROJ) {
+        const uint16_t dbits = reinterpret_cast<const uint16_t*>(slot + 2 * pb)[128 * h + r];
+        const __half2 d = __half2half2(__ushort_as_half(dbits));
         if (p.du_fmt == LMOE_Q8_0) {
-            const __half2 off = __float2half2_rn(1152.f);          // 1024 + 128
+            const uint4 a = *reinterpret_cast<const uint4*>(slot + h * pb + r * 32);
+            const uint4 b = *reinterpret_cast<const uint4*>(slot + h * pb + r * 32 + 16);
+            const uint32_t w8[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
+            const __half2 off = __float2half2_rn(1152.f);
 #pragma unroll
-            for (int b = 0; b < 2; ++b) {
-                const uint32_t w8[8] = {raw.q[2 * b].x, raw.q[2 * b].y, raw.q[2 * b].z, raw.q[2 * b].w,
-                                        raw.q[2 * b + 1].x, raw.q[2 * b + 1].y, raw.q[2 * b + 1].z,
-                                        raw.q[2 * b + 1].w};
-                const __half2 d = b ? d1 : d0;
-#pragma unroll
-                for (int i = 0; i < 8; ++i) {
-                    uint32_t lo, hi;
-                    bytes_to_h2x2(w8[i] ^ 0x80808080u, lo, hi);
-                    o[16 * b + 2 * i] = h2_bits(__hmul2(__hsub2(bits_h2(lo), off), d));
-                    o[16 * b + 2 * i + 1] = h2_bits(__hmul2(__hsub2(bits_h2(hi), off), d));
-                }
+            for (int i = 0; i < 8; ++i) {
+                uint32_t lo, hi;
+                bytes_to_h2x2(w8[i] ^ 0x80808080u, lo, hi);
+                o[2 * i] = h2_bits(__hmul2(__hsub2(bits_h2(lo), off), d));
+                o[2 * i + 1] = h2_bits(__hmul2(__hsub2(bits_h2(hi), off), d));
             }
         } else {
-            const __half2 off = __float2half2_rn(1032.f);          // 1024 + 8
+            const uint4 a = *reinterpret_cast<const uint4*>(slot + h * pb + r * 16);
+            const uint32_t w4[4] = {a.x, a.y, a.z, a.w};
+            const __half2 off = __float2half2_rn(1032.f);
 #pragma unroll
-            for (int b = 0; b < 2; ++b) {
-                const uint32_t w4[4] = {raw.q[b].x, raw.q[b].y, raw.q[b].z, raw.q[b].w};
-                const __half2 d = b ? d1 : d0;
-#pragma unroll
-                for (int i = 0; i < 4; ++i) {
-                    uint32_t lo, hi;
-                    bytes_to_h2x2(w4[i] & 0x0F0F0F0Fu, lo, hi);           // elements 4i .. 4i+3
-                    o[16 * b + 2 * i] = h2_bits(__hmul2(__hsub2(bits_h2(lo), off), d));
-                    o[16 * b + 2 * i + 1] = h2_bits(__hmul2(__hsub2(bits_h2(hi), off), d));
-                    bytes_to_h2x2((w4[i] >> 4) & 0x0F0F0F0Fu, lo, hi);    // elements 16+4i ..
-                    o[16 * b + 8 + 2 * i] = h2_bits(__hmul2(__hsub2(bits_h2(lo), off), d));
-                    o[16 * b + 8 + 2 * i + 1] = h2_bits(__hmul2(__hsub2(bits_h2(hi), off), d));
-                }
+            for (int i = 0; i < 4; ++i) {
+                uint32_t lo, hi;
+                bytes_to_h2x2(w4[i] & 0x0F0F0F0Fu, lo, hi);
+                o[2 * i] = h2_bits(__hmul2(__hsub2(bits_h2(lo), off), d));
+                o[2 * i + 1] = h2_bits(__hmul2(__hsub2(bits_h2(hi), off), d));
+                bytes_to_h2x2((w4[i] >> 4) & 0x0F0F0F0Fu, lo, hi);
+                o[8 + 2 * i] = h2_bits(__hmul2(__hsub2(bits_h2(lo), off), d));
+                o[8 + 2 * i + 1] = h2_bits(__hmul2(__hsub2(bits_h2(hi), off), d));
             }
         }
     } else {
-        // NVFP4: E2M1 x E4M3 is exact in fp16; the tensor scale is applied in the epilogue
-        uint32_t sc01, sc23;
-        asm("{\n\t.reg .b16 a, b;\n\tmov.b32 {a, b}, %2;\n\t"
-            "cvt.rn.f16x2.e4m3x2 %0, a;\n\tcvt.rn.f16x2.e4m3x2 %1, b;\n\t}"
-            : "=r"(sc01), "=r"(sc23)
-            : "r"(raw.s));
-        const __half2 s[4] = {__low2half2(bits_h2(sc01)), __high2half2(bits_h2(sc01)), __low2half2(bits_h2(sc23)),
-                              __high2half2(bits_h2(sc23))};
+        const uint4 a = *reinterpret_cast<const uint4*>(slot + h * pb + r * 16);
+        const uint32_t sw = reinterpret_cast<const uint32_t*>(slot + 2 * pb)[r];
+        const uint32_t s16 = (sw >> (16 * h)) & 0xFFFF;          // scales of columns 32h..+15 and +16..+31
+        uint32_t sc;
+        asm("{\n\t.reg .b16 a;\n\tcvt.u16.u32 a, %1;\n\tcvt.rn.f16x2.e4m3x2 %0, a;\n\t}" : "=r"(sc) : "r"(s16));
+        const __half2 s_lo = __low2half2(bits_h2(sc)), s_hi = __high2half2(bits_h2(sc));
+        const uint32_t w4[4] = {a.x, a.y, a.z, a.w};
 #pragma unroll
-        for (int c = 0; c < 2; ++c) {
-            const uint32_t w4[4] = {raw.q[c].x, raw.q[c].y, raw.q[c].z, raw.q[c].w};
+        for (int i = 0; i < 4; ++i) {
+            uint32_t hv[4];
+            e2m1x8_to_f16x8(w4[i], hv);
+            const __half2 sc2 = i < 2 ? s_lo : s_hi;
 #pragma unroll
-            for (int i = 0; i < 4; ++i) {
-                uint32_t h[4];
-                e2m1x8_to_f16x8(w4[i], h);
-                const __half2 sc = s[2 * c + (i >> 1)];
-#pragma unroll
-                for (int j = 0; j < 4; ++j) o[16 * c + 4 * i + j] = h2_bits(__hmul2(bits_h2(h[j]), sc));
-            }
+            for (int j = 0; j < 4; ++j) o[4 * i + j] = h2_bits(__hmul2(bits_h2(hv[j]), sc2));
         }
     }
 }
 
-// Row r of a 128-byte-swizzled K-major tile: 16-byte chunk c at (c ^ (r & 7)).
-__device__ __forceinline__ void store_row_swizzled(uint8_t* tile, int r, const uint32_t (&o)[32]) {
+// Half h of row r of a 128-byte-swizzled K-major tile (16-byte chunks 4h..4h+3).
+__device__ __forceinline__ void store_half_swizzled(uint8_t* tile, int r, int h, const uint32_t (&o)[16]) {
     uint8_t* row = tile + r * 128;
 #pragma unroll
-    for (int c = 0; c < 8; ++c) {
-        const uint4 v = make_uint4(o[4 * c], o[4 * c + 1], o[4 * c + 2], o[4 * c + 3]);
-        *reinterpret_cast<uint4*>(row + ((c ^ (r & 7)) << 4)) = v;
+    for (int c = 0; c < 4; ++c) {
+        const int cc = 4 * h + c;
+        *reinterpret_cast<uint4*>(row + ((cc ^ (r & 7)) << 4)) = make_uint4(o[4 * c], o[4 * c + 1], o[4 * c + 2], o[4 * c + 3]);
     }
 }
 
@@ -467,8 +432,8 @@ struct SmemPlan {
     static constexpr int kTotal = 1024 /*alignment slack*/ + STAGES * (kA + kB) + RS * kRaw + kXchg + kBars + 16;
 };
 
-constexpr int kConvWarps = 4;      // dequantising warps (one weight row per thread)
-constexpr int kGemmThreads = 320;  // 4 epilogue, 4 converter, 1 MMA, 1 loader warps
+constexpr int kConvWarps = 8;      // dequantising warps (half a weight row per thread)
+constexpr int kGemmThreads = 448;  // 4 epilogue, 8 converter, 1 MMA, 1 loader warps
 
 template <int KIND, int NT, int STAGES, int RS>
 __global__ void __launch_bounds__(kGemmThreads, 1) k_umma_gemm(const __grid_constant__ TmaMaps maps, const PrefillParams p) {
@@ -513,7 +478,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1) k_umma_gemm(const __grid_cons
         *abort_flag = 0;
         fence_barrier_init();
     }
-    if (warp == 8) {
+    if (warp == 12) {
         tmem_alloc(tmem_slot, kTmemCols);
         tmem_relinquish();
     }
@@ -522,7 +487,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1) k_umma_gemm(const __grid_cons
     tc_fence_after();
     const uint32_t tmem_base = *tmem_slot;
 
-    if (warp == 9) {
+    if (warp == 13) {
         // ------------------------------------------------------------ loader (one thread)
         if (lane == 0) {
             tma_prefetch_desc(&maps.b);
@@ -540,7 +505,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1) k_umma_gemm(const __grid_cons
                 while (!cr.done && it_r < it_b + RS) {
                     const int rs = it_r % RS;
                     const uint32_t ph = (it_r / RS) & 1;
-                    if (!mbar_wait(&raw_empty[rs], ph ^ 1, abort_flag, kWaitLimitNs)) { ok = false; break; }
+                    if (!mbar_wait(&raw_empty[rs], ph ^ 1, abort_flag, kWaitLimit)) { ok = false; break; }
                     if (S::tma_a(p, cr.seg)) mbar_arrive(&raw_full[rs]);
                     else issue_raw<KIND, NT>(p, cr, sRaw + rs * Plan::kRaw, &raw_full[rs]);
                     last_r[rs] = ph;
@@ -550,7 +515,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1) k_umma_gemm(const __grid_cons
                 if (!ok) break;
                 const int s = it_b % STAGES;
                 const uint32_t ph = (it_b / STAGES) & 1;
-                if (!mbar_wait(&empty[s], ph ^ 1, abort_flag, kWaitLimitNs)) break;
+                if (!mbar_wait(&empty[s], ph ^ 1, abort_flag, kWaitLimit)) break;
                 const bool ta = S::tma_a(p, cb.seg);
                 const int k0 = cb.ks * 64;
                 mbar_arrive_expect_tx(&full_b[s], Plan::kB + (ta ? Plan::kA : 0));
@@ -575,15 +540,16 @@ __global__ void __launch_bounds__(kGemmThreads, 1) k_umma_gemm(const __grid_cons
                 // let every copy already issued land before the CTA can leave
                 volatile int dummy = 0;
                 for (int i = 0; i < STAGES; ++i)
-                    if (last_b[i] != 0xFFFFFFFFu) mbar_wait(&full_b[i], last_b[i], &dummy, kWaitLimitNs);
+                    if (last_b[i] != 0xFFFFFFFFu) mbar_wait(&full_b[i], last_b[i], &dummy, kWaitLimit);
                 for (int i = 0; i < RS; ++i)
-                    if (last_r[i] != 0xFFFFFFFFu) mbar_wait(&raw_full[i], last_r[i], &dummy, kWaitLimitNs);
+                    if (last_r[i] != 0xFFFFFFFFu) mbar_wait(&raw_full[i], last_r[i], &dummy, kWaitLimit);
             }
         }
         __syncwarp();
-    } else if (warp >= 4 && warp < 8) {
+    } else if (warp >= 4 && warp < 12) {
         // ------------------------------------------------------------ converters
-        const int r = threadIdx.x - 128;           // A row
+        const int r = (threadIdx.x - 128) & 127;   // A row
+        const int hh = (threadIdx.x - 128) >> 7;   // half of the 64 columns
         Cursor<KIND, NT> cur;
         cur.begin(p);
         uint32_t it = 0;
@@ -591,14 +557,12 @@ __global__ void __launch_bounds__(kGemmThreads, 1) k_umma_gemm(const __grid_cons
             const int s = it % STAGES, rs = it % RS;
             const uint32_t ph = (it / STAGES) & 1, rph = (it / RS) & 1;
             const bool ta = S::tma_a(p, cur.seg);
-            if (!mbar_wait(&raw_full[rs], rph, abort_flag, kWaitLimitNs)) break;
-            if (!mbar_wait(&empty[s], ph ^ 1, abort_flag, kWaitLimitNs)) break;
+            if (!mbar_wait(&raw_full[rs], rph, abort_flag, kWaitLimit)) break;
+            if (!mbar_wait(&empty[s], ph ^ 1, abort_flag, kWaitLimit)) break;
             if (!ta) {
-                RawRow raw;
-                raw_row_from_smem<KIND>(p, sRaw + rs * Plan::kRaw, r, raw);
-                uint32_t o[32];
-                dequant_row<KIND>(p, cur.seg, raw, o);
-                store_row_swizzled(sA + s * Plan::kA, r, o);
+                uint32_t o[16];
+                dequant_half<KIND>(p, sRaw + rs * Plan::kRaw, r, hh, o);
+                store_half_swizzled(sA + s * Plan::kA, r, hh, o);
                 fence_proxy_async_smem();
             }
             __syncwarp();
@@ -610,7 +574,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1) k_umma_gemm(const __grid_cons
             cur.next_stage(p);
             ++it;
         }
-    } else if (warp == 8) {
+    } else if (warp == 12) {
         // ------------------------------------------------------------ MMA issuer
         if (lane == 0) {
             Cursor<KIND, NT> cur;
@@ -620,7 +584,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1) k_umma_gemm(const __grid_cons
             while (!cur.done) {
                 const int acc = tcount & 1;
                 const uint32_t aph = (tcount >> 1) & 1;
-                if (!mbar_wait(&tempty[acc], aph ^ 1, abort_flag, kWaitLimitNs)) break;
+                if (!mbar_wait(&tempty[acc], aph ^ 1, abort_flag, kWaitLimit)) break;
                 tc_fence_after();
                 const uint32_t d_tmem = tmem_base + acc * NT;
                 const int n_mma = (KIND == G_GATEUP || KIND == G_DOWN) ? ((cur.t.n + 15) & ~15) : NT;
@@ -631,8 +595,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1) k_umma_gemm(const __grid_cons
                     const uint32_t ph = (it / STAGES) & 1;
                     const bool ta = S::tma_a(p, cur.seg);
                     const uint32_t idesc = idesc_f16(128, n_mma, ta ? 1 : 0);
-                    if (!mbar_wait(&full_b[s], ph, abort_flag, kWaitLimitNs)) { ok = false; break; }
-                    if (!mbar_wait(&full_a[s], ph, abort_flag, kWaitLimitNs)) { ok = false; break; }
+                    if (!mbar_wait(&full_b[s], ph, abort_flag, kWaitLimit)) { ok = false; break; }
+                    if (!mbar_wait(&full_a[s], ph, abort_flag, kWaitLimit)) { ok = false; break; }
                     tc_fence_after();
                     const uint64_t a_desc = sdesc_k128(smem_u32(sA + s * Plan::kA));
                     const uint64_t b_desc = sdesc_k128(smem_u32(sB + s * Plan::kB));
@@ -655,7 +619,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1) k_umma_gemm(const __grid_cons
                 // all tensor-core work of this CTA done before TMEM is released
                 umma_commit(final_bar);
                 volatile int dummy = 0;
-                mbar_wait(final_bar, 0, &dummy, kWaitLimitNs);
+                mbar_wait(final_bar, 0, &dummy, kWaitLimit);
             }
         }
         __syncwarp();
@@ -680,7 +644,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1) k_umma_gemm(const __grid_cons
                 for (int i = threadIdx.x; i < cur.t.n; i += 128) xchg[i] = __ldg(p.w + __ldg(p.slot_pair + cur.t.b0 + i));
             }
             named_bar_sync(1, 128);
-            if (!mbar_wait(&tfull[acc], ph, abort_flag, kWaitLimitNs)) break;
+            if (!mbar_wait(&tfull[acc], ph, abort_flag, kWaitLimit)) break;
             tc_fence_after();
             const uint32_t taddr = tmem_base + ((uint32_t)(32 * warp) << 16) + acc * NT;
             for (int c0 = 0; c0 < cur.t.n; c0 += 32) {
@@ -701,7 +665,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1) k_umma_gemm(const __grid_cons
     tc_fence_before();
     __syncthreads();
     if (*abort_flag && threadIdx.x == 0) set_status(p.ctrl, LMOE_ERR_TIMEOUT);
-    if (warp == 8) {
+    if (warp == 12) {
         tc_fence_after();
         tmem_dealloc(tmem_base, kTmemCols);
     }
