@@ -126,10 +126,11 @@ def step_cost(shape, idx: np.ndarray, groups: np.ndarray, T: int, prefill: bool)
     pairs_tg = sum(len({int(groups[e]) for e in idx[t]}) for t in range(idx.shape[0]))   # hit (token, group) pairs
     b = {
         "k_router_shared": rw + 2 * Fs * H * 2 + T * H * 2,
-        "k_dproj": len(hit) * du + T * H * 2,
-        "k_expert_gateup": len(distinct) * rec_gu,
-        "k_expert_down": len(distinct) * rec_d,
-        "k_uproj": len(hit) * du + H * Fs * 2 + 2 * T * H * 2,
+        "k_stream_dproj": len(hit) * du + T * H * 2,
+        "k_stream_gateup": len(distinct) * rec_gu,
+        "k_stream_down": len(distinct) * rec_d,
+        "k_combine_small": 0,
+        "k_stream_uproj": len(hit) * du + H * Fs * 2 + 2 * T * H * 2,
     }
     f = {
         "x_to_fp16": 0.0,
@@ -151,7 +152,8 @@ def step_cost(shape, idx: np.ndarray, groups: np.ndarray, T: int, prefill: bool)
     return out
 
 
-STAGES = ["k_router_shared", "k_dproj", "k_expert_gateup", "k_expert_down", "k_uproj"]
+STAGES = ["k_router_shared", "k_stream_dproj", "k_stream_gateup", "k_stream_down", "k_combine_small",
+          "k_stream_uproj"]
 PREFILL_STAGES = ["x_to_fp16", "router_gemm", "topk_bucket", "shared_gateup", "dproj", "gateup", "down", "combine",
                   "uproj"]
 
@@ -163,6 +165,25 @@ def workload_desc(wl, T):
     return (f"{wl.name}: T={T}, hidden {s.hidden}, latent {s.latent}, {s.n_experts} experts top-{s.top_k}, "
             f"{s.n_groups} {fmt} D/U groups, NVFP4 experts ffn {s.ffn}, bf16 shared ffn {s.shared_ffn}, "
             f"{s.router_dtype} router, bias {bias}, expert_group {wl.groups}, x bf16 N(0,1), weights N(0,0.02)")
+
+
+# ----------------------------------------------------------------------------
+# multi-GPU: independent replicas, max over ranks
+# ----------------------------------------------------------------------------
+
+def max_over_ranks(ms: float, device=None) -> float:
+    """The slowest rank's time (every rank calls this in the same order)."""
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([ms], dtype=torch.float64, device=device)
+    if dist.is_available() and dist.is_initialized() and dist.get_world_size() > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def replica_throughput(world: int, tokens_per_step: int, steps: int, ms_max: float) -> float:
+    """Whole-job tokens/s: every rank processes its own batches (weak scaling)."""
+    return world * tokens_per_step * steps / (ms_max / 1e3)
 
 
 # ----------------------------------------------------------------------------
@@ -223,6 +244,101 @@ def run_reference(args, wl, T, rank, world):
 
 
 # ----------------------------------------------------------------------------
+# the 48-layer stack
+# ----------------------------------------------------------------------------
+
+def run_stack(args, wl, T, rank, world, local, dev_name, n_distinct=4):
+    """x <- x + block_l(RMSNorm_l(x)) over wl.n_layers layers in one call.
+    n_distinct independently seeded layers are generated and copied into
+    n_layers separate device buffers (layer l holds the bytes of layer
+    l % n_distinct): the time depends on the bytes each layer streams and on
+    its routing, which the changing residual stream drives."""
+    import numpy as np
+    import torch
+    from latent_mixture_experts_softmax_b200 import binding as B
+    from latent_mixture_experts_softmax_b200 import synth
+    from latent_mixture_experts_softmax_b200.layer import DeviceLayer, to_device
+    s = wl.shape
+    gamma = synth.bf16_bits_from_f32(np.ones(s.hidden, np.float32))
+    srcs = [synth.make_layer(wl, layer=l) for l in range(min(n_distinct, wl.n_layers))]
+    devs = [DeviceLayer(s, srcs[l % len(srcs)], device=dev_name, gamma=gamma) for l in range(wl.n_layers)]
+    layers = [d.as_c_layer() for d in devs]
+    ws = devs[0].workspace(T)
+    K, W = args.steps, args.warmup
+    n_in = 8
+    xs_host = [synth.make_x(wl, T=T, draw=rank * 100_003 + i) for i in range(n_in)]
+    xs = [to_device(x, dev_name) for x in xs_host]
+    ys = [torch.empty_like(x) for x in xs]
+    eps = 1e-6
+
+    def step(i):
+        B.lmoe_stack_forward(devs[0].cfg, layers, xs[i % n_in], ys[i % n_in], T, eps, ws)
+
+    for i in range(max(W, 1)):
+        step(i)
+    torch.cuda.synchronize()
+    graphs = []
+    if T <= 64:
+        for g in range(n_in):
+            cg = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(cg):
+                step(g)
+            graphs.append(cg)
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize()
+    with ClockSampler(local) as clk:
+        start.record()
+        for k in range(K):
+            if graphs:
+                graphs[k % n_in].replay()
+            else:
+                step(k)
+        end.record()
+        torch.cuda.synchronize()
+    ms_max = max_over_ranks(start.elapsed_time(end), dev_name)
+    status = B.lmoe_last_device_status(ws)
+    del graphs
+    # bytes per layer from the routing each layer actually takes (one untimed pass)
+    idx = torch.empty((T, s.top_k), dtype=torch.int32, device=dev_name)
+    wgt = torch.empty((T, s.top_k), dtype=torch.float32, device=dev_name)
+    cur = xs[0].clone()
+    nxt = torch.empty_like(cur)
+    prefill = T >= 64 and s.router_dtype == "bf16" and s.n_experts % 128 == 0
+    tot_b = tot_f = 0.0
+    for l, d in enumerate(devs):
+        B.lmoe_stack_forward(d.cfg, [layers[l]], cur, nxt, T, eps, ws)
+        # routing of this layer's normalised input, through the block call on it
+        xn = cur.view(torch.bfloat16).float()
+        xn = (xn * torch.rsqrt((xn * xn).mean(dim=1, keepdim=True) + eps)).to(torch.bfloat16).view(torch.int16)
+        B.lmoe_route(d.cfg, xn.contiguous(), d.router_w, d.router_b, T, idx, wgt, ws)
+        c = step_cost(s, idx.cpu().numpy(), srcs[l % len(srcs)]["expert_group"], T, prefill)
+        tot_b += c["bytes_total"]
+        tot_f += c["flops_total"]
+        cur, nxt = nxt, cur
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            peaks = json.load(f)
+        hbm_peak, tc_peak, src = float(peaks["hbm_gbs"]), float(peaks["bf16_tflops"]), "measured"
+    except Exception:
+        hbm_peak, tc_peak, src = 6650.0, 1590.0, "fallback"
+    t_step = ms_max / K / 1e3
+    t_lb = max(tot_b / (hbm_peak * 1e9), tot_f / (tc_peak * 1e12))
+    value = replica_throughput(world, T, K, ms_max)
+    line = {"metric": "latent-MoE 48-layer stack tokens/s", "value": value, "unit": "tokens/s", "n_gpus": world,
+            "steps": K, "warmup": W, "ms_per_step": ms_max / K, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f16" if prefill else "f32", "data": "synthetic",
+            "config": {"workload": workload_desc(wl, T), "T": T, "layers": wl.n_layers,
+                       "weights": f"{len(srcs)} seeded layers copied into {wl.n_layers} device buffers",
+                       "l2": f"{wl.n_layers} layers x {devs[0].weight_bytes() / 1e9:.2f} GB resident, larger than L2"},
+            "layer_equivalent": {"gbs": tot_b / t_step / 1e9, "tflops": tot_f / t_step / 1e12,
+                                 "roofline_time_us": t_lb * 1e6, "frac_of_roofline": t_lb / t_step,
+                                 "peak_source": src},
+            "clocks": clk.summary(), "device_status": status}
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+
+
+# ----------------------------------------------------------------------------
 # our arm
 # ----------------------------------------------------------------------------
 
@@ -252,6 +368,11 @@ def main():
         from datetime import timedelta
         dist.init_process_group("nccl", timeout=timedelta(seconds=120), device_id=dev_name)
     build.build_all()
+    if wl.n_layers > 1:
+        run_stack(args, wl, T, rank, world, local, dev_name)
+        if world > 1:
+            dist.destroy_process_group()
+        return
 
     layer = synth.make_layer(wl)
     base = DeviceLayer(wl.shape, layer, device=dev_name)
@@ -315,11 +436,7 @@ def main():
         torch.cuda.synchronize()
     if world > 1:
         dist.barrier()
-    ms = start.elapsed_time(end)
-    ms_t = torch.tensor([ms], dtype=torch.float64, device=dev_name)
-    if world > 1:
-        dist.all_reduce(ms_t, op=dist.ReduceOp.MAX)
-    ms_max = float(ms_t.item())
+    ms_max = max_over_ranks(start.elapsed_time(end), dev_name)
     status = B.lmoe_last_device_status(ws)
     del graphs
 
@@ -388,12 +505,9 @@ def main():
                             y_pin, T, ws, stream)
     e1.record()
     torch.cuda.synchronize()
-    e2e_ms = torch.tensor([e0.elapsed_time(e1)], dtype=torch.float64, device=dev_name)
-    if world > 1:
-        dist.all_reduce(e2e_ms, op=dist.ReduceOp.MAX)
-    e2e_rate = world * T * K / (float(e2e_ms.item()) / 1e3)
+    e2e_rate = replica_throughput(world, T, K, max_over_ranks(e0.elapsed_time(e1), dev_name))
 
-    value = world * T * K / (ms_max / 1e3)
+    value = replica_throughput(world, T, K, ms_max)
     line = {
         "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": K, "warmup": W,
         "ms_per_step": ms_max / K, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
@@ -418,6 +532,7 @@ def main():
         "e2e": {"value": e2e_rate, "unit": "tokens/s", "h2d_bytes_per_step": T * s.hidden * 2,
                 "d2h_bytes_per_step": T * s.hidden * 2},
         "gpu_launches": (len(stages) + (3 if prefill else 0)) * K,
+        "path": "prefill" if prefill else "decode",
         "clocks": clk.summary(),
         "device_status": status,
     }

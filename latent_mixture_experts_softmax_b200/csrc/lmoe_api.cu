@@ -47,7 +47,7 @@ bool use_prefill(const lmoe_cfg& c, int T) {
 // start after the control block, so one allocation serves either.
 struct WsLayout {
     size_t ctrl, idx, w, logits, n_unique, uexp, ucnt, uoff, slot_pair, pair_slot, ghit, tghit;
-    size_t x16, h16, zsh, z16, s16, ypart, xio, yio, xa, xb;
+    size_t x16, h16, zsh, zsh16, o16w, z16, s16, ypart, xio, yio, xa, xb;
     // tensor-core path
     size_t p_zero_begin, p_tgmask, p_cnt, p_fill, p_dhit, p_n_etiles, p_zero_end;
     size_t p_n_unique, p_off, p_uexp, p_ucnt, p_uoff, p_etile, p_slot_pair, p_pair_slot, p_idx, p_w, p_logits;
@@ -87,6 +87,8 @@ WsLayout ws_layout(const lmoe_cfg& c, int T) {
         L.x16 = take((size_t)Td * c.hidden * 2);
         L.h16 = take((size_t)Td * c.n_groups * c.latent * 2);
         L.zsh = take((size_t)Td * c.shared_ffn * 4);
+        L.zsh16 = take((size_t)Td * c.shared_ffn * 2);
+        L.o16w = take(TK * c.latent * 2);
         L.z16 = take(TK * c.ffn * 2);
         L.s16 = take((size_t)Td * c.n_groups * c.latent * 2);
         L.ypart = take((size_t)(c.n_groups + 1) * Td * c.hidden * 4);
@@ -150,6 +152,8 @@ FwdParams base_params(const lmoe_cfg& c, int T, void* ws, const WsLayout& L) {
     p.x16 = reinterpret_cast<__half*>(b + L.x16);
     p.h16 = reinterpret_cast<__half*>(b + L.h16);
     p.zsh = reinterpret_cast<float*>(b + L.zsh);
+    p.zsh16 = reinterpret_cast<__half*>(b + L.zsh16);
+    p.o16w = reinterpret_cast<__half*>(b + L.o16w);
     p.z16 = reinterpret_cast<__half*>(b + L.z16);
     p.s16 = reinterpret_cast<__half*>(b + L.s16);
     p.ypart = reinterpret_cast<float*>(b + L.ypart);

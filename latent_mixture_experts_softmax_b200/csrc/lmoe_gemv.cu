@@ -189,6 +189,8 @@ __global__ void __launch_bounds__(256) k_router_shared(FwdParams p) {
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int H = p.H;
     const bool router_cta = (int)blockIdx.x < p.n_router_ctas;
+    // the D_g kernel may launch now; it waits for this grid to complete
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
     if (!router_cta && !p.do_shared) return;
     if (p.prefetch_l2 && blockIdx.x == 0 && p.T <= kChunk)
         l2_prefetch_range(p.sd, (size_t)p.H * p.Fs * 2);
@@ -224,7 +226,11 @@ __global__ void __launch_bounds__(256) k_router_shared(FwdParams p) {
 #pragma unroll
                 for (int t = 0; t < NT; ++t) {
                     const float av = warp_sum(a[t]), uv = warp_sum(u[t]);
-                    if (lane == 0 && t < nt) p.zsh[(size_t)(t0 + t) * p.Fs + f] = silu(av) * uv;
+                    if (lane == 0 && t < nt) {
+                        const float z = silu(av) * uv;
+                        p.zsh[(size_t)(t0 + t) * p.Fs + f] = z;
+                        if (p.zsh16) p.zsh16[(size_t)(t0 + t) * p.Fs + f] = __float2half_rn(z);
+                    }
                 }
             }
         }
@@ -269,19 +275,32 @@ __device__ __forceinline__ void topk_warp(const FwdParams& p, int t, int lane) {
         const int e = lane + 32 * j;
         v[j] = e < E ? __ldcg(p.r.logits + (size_t)t * E + e) : -INFINITY;
     }
+    // each lane keeps its own best untaken (value, index); only the lane that
+    // supplied a round's winner rescans its values
     uint32_t taken = 0;
+    float lv = -INFINITY;
+    int li = 0x7fffffff;
+#pragma unroll
+    for (int j = 0; j < NV; ++j) {
+        const int e = lane + 32 * j;
+        if (e < E && v[j] > lv) { lv = v[j]; li = e; }
+    }
     float lmax = 0.f, denom = 0.f, my_l = 0.f;
     int my_e = 0;
     for (int k = 0; k < K; ++k) {
-        float bv = -INFINITY;
-        int bi = 0x7fffffff;
-#pragma unroll
-        for (int j = 0; j < NV; ++j) {
-            const int e = lane + 32 * j;
-            if (e < E && !(taken >> j & 1u) && (v[j] > bv || (v[j] == bv && e < bi))) { bv = v[j]; bi = e; }
-        }
+        float bv = lv;
+        int bi = li;
         warp_argmax(bv, bi);
-        if ((bi & 31) == lane && bi < E) taken |= 1u << (bi >> 5);
+        if (bi < E && (bi & 31) == lane) {
+            taken |= 1u << (bi >> 5);
+            lv = -INFINITY;
+            li = 0x7fffffff;
+#pragma unroll
+            for (int j = 0; j < NV; ++j) {
+                const int e = lane + 32 * j;
+                if (e < E && !(taken >> j & 1u) && (v[j] > lv || (v[j] == lv && e < li))) { lv = v[j]; li = e; }
+            }
+        }
         if (k == 0) lmax = bv;
         if (k == lane) { my_l = bv; my_e = bi; }
         denom += expf(bv - lmax);
@@ -1000,6 +1019,7 @@ static cudaError_t run_gemv_path_nt(FwdParams p, cudaStream_t st, bool route_onl
             : launch(k_router_shared<NT, false>, dim3(p.n_router_ctas + n_shared_ctas), 256, sm, st, p);
         if (e != cudaSuccess || route_only) return e;
     }
+    if (p.T <= 8) return run_stream_path(p, st);
     const int max_unique = min(p.T * p.K, p.E);
     const size_t red = (size_t)kMmaWarps * 32 * 4 * sizeof(float);
     const int thr = 32 * kMmaWarps;

@@ -70,6 +70,8 @@ struct FwdParams {
     __half* x16;    // [T][H]       block input (normalised for the stack), fp16
     __half* h16;    // [T][G][L]    D_g x for the hit (token, group) pairs
     float* zsh;     // [T][Fs]      shared-expert hidden
+    __half* zsh16;  // [T][Fs]      the same in fp16 (weight-streaming path)
+    __half* o16w;   // [T*K][L]     routing-weighted expert outputs per slot (weight-streaming path)
     __half* z16;    // [T*K][F]     expert hidden per slot (slots grouped by expert)
     __half* s16;    // [T][G][L]    per-group weighted expert sums
     float* ypart;   // [G+1][T][H]  U_g parts and the shared part
@@ -83,6 +85,7 @@ struct FwdParams {
 constexpr int kMaxStageEvents = 16;
 
 cudaError_t run_gemv_path(const FwdParams& p, cudaStream_t st, bool route_only);
+cudaError_t run_stream_path(const FwdParams& p, cudaStream_t st);
 void set_stage_events(void* const* events, int n);
 void stage_mark(cudaStream_t st);
 void stage_reset();
