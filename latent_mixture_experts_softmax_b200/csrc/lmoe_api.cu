@@ -46,7 +46,7 @@ bool use_prefill(const lmoe_cfg& c, int T) {
 // Workspace of the few-token path (first) and of the tensor-core path; both
 // start after the control block, so one allocation serves either.
 struct WsLayout {
-    size_t ctrl, idx, w, logits, n_unique, uexp, ucnt, uoff, slot_pair, pair_slot, ghit, tghit;
+    size_t ctrl, idx, w, logits, n_unique, uexp, ucnt, uoff, ugrp, slot_pair, pair_slot, ghit, tghit;
     size_t x16, h16, zsh, zsh16, o16w, z16, s16, ypart, xio, yio, xa, xb;
     // tensor-core path
     size_t p_zero_begin, p_tgmask, p_cnt, p_fill, p_dhit, p_n_etiles, p_zero_end;
@@ -80,6 +80,7 @@ WsLayout ws_layout(const lmoe_cfg& c, int T) {
         L.uexp = take(TK * 4);
         L.ucnt = take(TK * 4);
         L.uoff = take(TK * 4);
+        L.ugrp = take(TK * 4);
         L.slot_pair = take(TK * 4);
         L.pair_slot = take(TK * 4);
         L.ghit = take((size_t)c.n_groups * 4);
@@ -145,6 +146,7 @@ FwdParams base_params(const lmoe_cfg& c, int T, void* ws, const WsLayout& L) {
     p.r.uexp = reinterpret_cast<int32_t*>(b + L.uexp);
     p.r.ucnt = reinterpret_cast<int32_t*>(b + L.ucnt);
     p.r.uoff = reinterpret_cast<int32_t*>(b + L.uoff);
+    p.r.ugrp = reinterpret_cast<int32_t*>(b + L.ugrp);
     p.r.slot_pair = reinterpret_cast<int32_t*>(b + L.slot_pair);
     p.r.pair_slot = reinterpret_cast<int32_t*>(b + L.pair_slot);
     p.r.ghit = reinterpret_cast<int32_t*>(b + L.ghit);

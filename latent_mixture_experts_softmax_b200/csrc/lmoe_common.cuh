@@ -70,6 +70,9 @@ __device__ __forceinline__ float warp_sum(float v) {
 }
 
 __device__ __forceinline__ float silu(float a) { return a / (1.0f + __expf(-a)); }
+// The same with the approximate division (relative error ~1e-6; the
+// result is rounded to fp16 or bf16 right after).
+__device__ __forceinline__ float silu_fast(float a) { return __fdividef(a, 1.0f + __expf(-a)); }
 
 // Block-wide exclusive scan of one int per thread; returns the total.
 __device__ __forceinline__ int block_exclusive_scan(int v, int* out, int* scratch) {
@@ -126,6 +129,7 @@ struct Routing {
     int32_t* uexp;       // [T*K]    distinct experts, ascending
     int32_t* ucnt;       // [T*K]    (t, k) pairs per distinct expert
     int32_t* uoff;       // [T*K]    first slot of each distinct expert
+    int32_t* ugrp;       // [T*K]    group of each distinct expert (few-token path)
     int32_t* slot_pair;  // [T*K]    slot -> pair t*K + k (slots grouped by expert)
     int32_t* pair_slot;  // [T*K]    pair -> slot
     int32_t* ghit;       // [G]      tokens hitting each group (any > 0 means hit)

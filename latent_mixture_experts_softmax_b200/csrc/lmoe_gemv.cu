@@ -20,6 +20,7 @@
 // shared expert at full width, top-10 of 512).
 
 #include "lmoe_internal.cuh"
+#include "lmoe_route.cuh"
 
 namespace lmoe {
 
@@ -249,7 +250,15 @@ __global__ void __launch_bounds__(256) k_router_shared(FwdParams p) {
     __syncthreads();
     if (!s_last) return;
     __threadfence();
-    topk_and_buckets(p);
+    if (p.route_smem) {
+        __shared__ StreamShared rsh;
+        __shared__ uint8_t sgrp[kMaxExpertsTopk];
+        for (int e = threadIdx.x; e < p.E; e += blockDim.x) sgrp[e] = p.group[e];
+        __syncthreads();
+        route_in_cta(p, rsh, sgrp, true);
+    } else {
+        topk_and_buckets(p);
+    }
     if (threadIdx.x == 0) p.ctrl->route_ticket = 0;
 }
 
@@ -1010,6 +1019,9 @@ static cudaError_t run_gemv_path_nt(FwdParams p, cudaStream_t st, bool route_onl
     p.n_router_ctas = (p.E + 7) / 8;
     p.do_shared = !route_only;
     p.do_buckets = !route_only;
+    // few tokens, whole block: the routing is built in shared memory and
+    // published with every table the weight-streaming kernels read
+    p.route_smem = !route_only && p.T <= 8;
     p.prefetch_l2 = false;
     const int n_shared_ctas = route_only ? 0 : (p.Fs + 7) / 8;
     {

@@ -1,0 +1,212 @@
+// Routing of a few-token step (T <= 8) in one CTA's shared memory: softmax
+// top-K per token and the bucketing of the (token, k) pairs by expert.  Used
+// by the last CTA of the router kernel, which publishes the result to the
+// workspace for the kernels after it.
+#pragma once
+
+#include "lmoe_internal.cuh"
+
+namespace lmoe {
+
+constexpr int kMaxPairs = 8 * kMaxTopK;   // (token, k) pairs of at most 8 tokens
+
+// Routing of the step in shared memory.
+struct StreamShared {
+    int hg[kMaxGroups];        // hit groups, ascending
+    int n_hit;
+    int n_unique;              // distinct experts
+    int uexp[kMaxPairs];
+    int ucnt[kMaxPairs];
+    int uoff[kMaxPairs];
+    int ugrp[kMaxPairs];       // group of each distinct expert
+    int slot_tok[kMaxPairs];   // token of each slot (slots grouped by expert)
+    float slot_w[kMaxPairs];   // routing weight of each slot
+    // the routing itself (kernels that compute it rather than read it)
+    int idx[kMaxPairs];        // [T][K] selected experts
+    float w[kMaxPairs];        // [T][K] renormalised weights
+    int pe[kMaxPairs];         // pair -> expert (validated)
+    int pgrp[kMaxPairs];       // pair -> group
+    int slot_pair[kMaxPairs];
+    int pair_slot[kMaxPairs];
+    int gcnt[kMaxGroups];      // pairs per group
+    uint8_t pfirst[kMaxPairs]; // pair is the first of its expert
+};
+
+// ---------------------------------------------------------------------------
+// routing inside a kernel: every CTA derives the step's routing from the
+// router logits on its own (a few microseconds), so no kernel waits for a
+// single CTA to publish it
+// ---------------------------------------------------------------------------
+
+// Softmax top-K of one token by one warp (section "Routing" of the teardown
+// article: softmax over the E logits, top-K, renormalise over the kept):
+// K rounds of a warp arg-max, ties to the lower index; w_k = exp(l_k - l_1)
+// / sum over the kept of exp(l_j - l_1).  Writes idx[0..K), w[0..K).
+template <int NV>
+static __device__ void topk_row(const float* logits, int E, int K, int lane, int* idx, float* w) {
+    float v[NV];
+#pragma unroll
+    for (int j = 0; j < NV; ++j) {
+        const int e = lane + 32 * j;
+        v[j] = e < E ? __ldcg(logits + e) : -INFINITY;
+    }
+    uint32_t taken = 0;
+    float lv = -INFINITY;
+    int li = 0x7fffffff;
+#pragma unroll
+    for (int j = 0; j < NV; ++j) {
+        const int e = lane + 32 * j;
+        if (e < E && v[j] > lv) { lv = v[j]; li = e; }
+    }
+    float lmax = 0.f, denom = 0.f, my_l = 0.f;
+    int my_e = 0;
+    for (int k = 0; k < K; ++k) {
+        float bv = lv;
+        int bi = li;
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) {
+            const float ov = __shfl_xor_sync(0xffffffffu, bv, o);
+            const int oi = __shfl_xor_sync(0xffffffffu, bi, o);
+            if (ov > bv || (ov == bv && oi < bi)) { bv = ov; bi = oi; }
+        }
+        if (bi < E && (bi & 31) == lane) {
+            taken |= 1u << (bi >> 5);
+            lv = -INFINITY;
+            li = 0x7fffffff;
+#pragma unroll
+            for (int j = 0; j < NV; ++j) {
+                const int e = lane + 32 * j;
+                if (e < E && !(taken >> j & 1u) && (v[j] > lv || (v[j] == lv && e < li))) { lv = v[j]; li = e; }
+            }
+        }
+        if (k == 0) lmax = bv;
+        if (k == lane) { my_l = bv; my_e = bi; }
+        denom += expf(bv - lmax);
+    }
+    if (lane < K) {
+        idx[lane] = my_e;
+        w[lane] = expf(my_l - lmax) / denom;
+    }
+}
+
+// Bucketing of the T*K pairs by one warp, in shared memory: slots ordered by
+// (expert, pair index), distinct experts ascending, pairs per group.
+// `grp` is the expert -> group table (in shared memory).  Invalid indices
+// or labels are reported (report = true) and read as 0.
+static __device__ void bucket_pairs(const FwdParams& p, StreamShared& sh, const uint8_t* grp, int lane, bool report) {
+    const int K = p.K, G = p.G, E = p.E, n = p.T * K;
+    for (int g = lane; g < G; g += 32) sh.gcnt[g] = 0;
+    for (int i = lane; i < n; i += 32) {
+        int e = sh.idx[i];
+        if (e < 0 || e >= E) {
+            if (report) set_status(p.ctrl, LMOE_ERR_DEVICE_CHECK);
+            e = 0;
+        }
+        int g = grp[e];
+        if (g >= G) {
+            if (report) set_status(p.ctrl, LMOE_ERR_DEVICE_CHECK);
+            g = 0;
+        }
+        sh.pe[i] = e;
+        sh.pgrp[i] = g;
+    }
+    __syncwarp();
+    for (int i = lane; i < n; i += 32) {
+        bool first = true;
+#pragma unroll 8
+        for (int j = 0; j < i; ++j) first &= sh.pe[j] != sh.pe[i];
+        sh.pfirst[i] = first;
+    }
+    __syncwarp();
+    int n_first = 0;
+    for (int i = lane; i < n; i += 32) {
+        const int e = sh.pe[i];
+        int less = 0, same_before = 0, cnt = 0, u = 0;
+#pragma unroll 8
+        for (int j = 0; j < n; ++j) {
+            const int ej = sh.pe[j];
+            less += ej < e;
+            same_before += (j < i && ej == e);
+            cnt += ej == e;
+            u += (sh.pfirst[j] && ej < e);
+        }
+        const bool first = sh.pfirst[i];
+        const int slot = less + same_before;
+        sh.slot_pair[slot] = i;
+        sh.pair_slot[i] = slot;
+        sh.slot_tok[slot] = i / K;
+        sh.slot_w[slot] = sh.w[i];
+        if (first) {
+            sh.uexp[u] = e;
+            sh.ucnt[u] = cnt;
+            sh.uoff[u] = less;
+            sh.ugrp[u] = sh.pgrp[i];
+            ++n_first;
+        }
+        atomicAdd(&sh.gcnt[sh.pgrp[i]], 1);
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) n_first += __shfl_xor_sync(0xffffffffu, n_first, o);
+    __syncwarp();
+    if (lane == 0) {
+        sh.n_unique = n_first;
+        int nh = 0;
+        for (int g = 0; g < G; ++g)
+            if (sh.gcnt[g] > 0) sh.hg[nh++] = g;
+        sh.n_hit = nh;
+    }
+    __syncwarp();
+}
+
+// The step's routing into `sh`, by every thread of the CTA (contains
+// __syncthreads); `grp` is the expert -> group table in shared memory.
+// With publish, also written to the workspace for the kernels that read it
+// and to the caller's routing outputs.
+static __device__ void route_in_cta(const FwdParams& p, StreamShared& sh, const uint8_t* grp, bool publish) {
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int T = p.T, K = p.K, E = p.E, G = p.G, n = T * K;
+    if (p.inject_idx != nullptr && p.inject_w != nullptr) {
+        for (int i = threadIdx.x; i < n; i += blockDim.x) {
+            sh.idx[i] = __ldg(p.inject_idx + i);
+            sh.w[i] = __ldg(p.inject_w + i);
+        }
+    } else {
+        for (int t = warp; t < T; t += blockDim.x >> 5) {
+            const float* lg = p.r.logits + (size_t)t * E;
+            if (E <= 128) topk_row<4>(lg, E, K, lane, sh.idx + t * K, sh.w + t * K);
+            else if (E <= 256) topk_row<8>(lg, E, K, lane, sh.idx + t * K, sh.w + t * K);
+            else if (E <= 512) topk_row<16>(lg, E, K, lane, sh.idx + t * K, sh.w + t * K);
+            else topk_row<32>(lg, E, K, lane, sh.idx + t * K, sh.w + t * K);
+        }
+    }
+    __syncthreads();
+    if (warp == 0) bucket_pairs(p, sh, grp, lane, publish);
+    __syncthreads();
+    if (!publish) return;
+    const Routing& r = p.r;
+    for (int i = threadIdx.x; i < n; i += blockDim.x) {
+        r.idx[i] = sh.pe[i];
+        r.w[i] = sh.w[i];
+        if (p.out_idx) p.out_idx[i] = sh.idx[i];
+        if (p.out_w) p.out_w[i] = sh.w[i];
+        r.slot_pair[i] = sh.slot_pair[i];
+        r.pair_slot[i] = sh.pair_slot[i];
+        if (i < sh.n_unique) {
+            r.uexp[i] = sh.uexp[i];
+            r.ucnt[i] = sh.ucnt[i];
+            r.uoff[i] = sh.uoff[i];
+            r.ugrp[i] = sh.ugrp[i];
+        }
+    }
+    for (int i = threadIdx.x; i < T * G; i += blockDim.x) {
+        const int t = i / G, g = i - t * G;
+        uint8_t hit = 0;
+        for (int k = 0; k < K; ++k) hit |= sh.pgrp[t * K + k] == g;
+        r.tghit[i] = hit;
+    }
+    for (int g = threadIdx.x; g < G; g += blockDim.x) r.ghit[g] = sh.gcnt[g];
+    if (threadIdx.x == 0) *r.n_unique = sh.n_unique;
+}
+
+
+}  // namespace lmoe

@@ -18,8 +18,10 @@
 // per-group D/U); Edge0 145B / 120B model page, architecture tables.
 
 #include <cstring>
+#include <mutex>
 
 #include "lmoe_internal.cuh"
+#include "lmoe_route.cuh"
 #include "lmoe_sm100.cuh"
 
 namespace lmoe {
@@ -28,9 +30,11 @@ using namespace sm100;
 
 enum StreamPhase { SP_DPROJ = 0, SP_GATEUP = 1, SP_DOWN = 2, SP_UPROJ = 3 };
 
-constexpr int kSW = 8;                 // compute warps per CTA
+constexpr int kSW = 16;                // compute warps per CTA
 constexpr int kStreamThreads = 32 * (kSW + 2);   // + loader warp + reducer warp
 constexpr int kMaxSlots = 16;          // weight slots in the ring
+
+__host__ __device__ __forceinline__ int round128(int b) { return (b + 127) & ~127; }
 constexpr int kActPad = 32;            // halves of padding per staged activation row
 constexpr uint64_t kStreamWait = 4000000000ull;   // SM cycles per barrier wait
 
@@ -96,6 +100,7 @@ template <int FMT>
 __device__ __forceinline__ void tile_du(const uint8_t* q, const uint16_t* d, const __half* xs, int ld, int nt,
                                         int b0, int b1, float (&acc)[4]) {
     const int lane = threadIdx.x & 31, g = lane >> 2, t = lane & 3;
+#pragma unroll 2
     for (int b = b0; b < b1; ++b) {
         float c[4] = {0.f, 0.f, 0.f, 0.f};
         if (FMT == LMOE_Q8_0) {
@@ -137,6 +142,7 @@ __device__ __forceinline__ void tile_du(const uint8_t* q, const uint16_t* d, con
 __device__ __forceinline__ void tile_nvfp4(const uint8_t* q, const uint8_t* s, const __half* xs, int ld, int nt,
                                            int c0, int c1, float (&acc)[4]) {
     const int lane = threadIdx.x & 31, g = lane >> 2, t = lane & 3;
+#pragma unroll 2
     for (int c = c0; c < c1; ++c) {
         const uint32_t wg = *reinterpret_cast<const uint32_t*>(q + ((size_t)c * 16 + g) * 16 + 4 * t);
         const uint32_t wh = *reinterpret_cast<const uint32_t*>(q + ((size_t)c * 16 + g + 8) * 16 + 4 * t);
@@ -172,6 +178,7 @@ __device__ __forceinline__ void tile_nvfp4(const uint8_t* q, const uint8_t* s, c
 __device__ __forceinline__ void tile_bf16(const uint16_t* w, int K, const __half* xs, int ld, int nt, int b0, int b1,
                                           float (&acc)[4]) {
     const int lane = threadIdx.x & 31, g = lane >> 2, t = lane & 3;
+#pragma unroll 2
     for (int b = b0; b < b1; ++b) {
         const uint4 wg = *reinterpret_cast<const uint4*>(w + (size_t)g * K + 32 * b + 8 * t);
         const uint4 wh = *reinterpret_cast<const uint4*>(w + (size_t)(g + 8) * K + 32 * b + 8 * t);
@@ -190,26 +197,11 @@ __device__ __forceinline__ void tile_bf16(const uint16_t* w, int K, const __half
 // work items
 // ---------------------------------------------------------------------------
 
-constexpr int kMaxPairs = 8 * kMaxTopK;   // (token, k) pairs of at most 8 tokens
 
 template <int PHASE>
 __host__ __device__ __forceinline__ int stream_rows(int H, int L, int F) {
     return PHASE == SP_DPROJ ? L : PHASE == SP_GATEUP ? F : PHASE == SP_DOWN ? L : H;
 }
-
-// Routing of the step, staged once per CTA so that no per-item decision
-// waits on a global-memory round trip.
-struct StreamShared {
-    int hg[kMaxGroups];        // hit groups, ascending
-    int n_hit;
-    int n_unique;              // distinct experts
-    int uexp[kMaxPairs];
-    int ucnt[kMaxPairs];
-    int uoff[kMaxPairs];
-    int ugrp[kMaxPairs];       // group of each distinct expert
-    int slot_tok[kMaxPairs];   // token of each slot (slots grouped by expert)
-    float slot_w[kMaxPairs];   // routing weight of each slot
-};
 
 // What the compute and reducer warps need to know about the item in a slot.
 struct __align__(16) SlotMeta {
@@ -296,39 +288,35 @@ __global__ void __launch_bounds__(kStreamThreads, 1) k_stream(const __grid_const
     __shared__ __align__(8) uint64_t red_empty[2];
     __shared__ __align__(8) uint64_t xbar;
     __shared__ int abort_flag;
-    __shared__ float red[2][kSW][32][8];
+    constexpr int NV = PHASE == SP_GATEUP ? 8 : 4;   // partial values per lane (gate [+ up])
+    __shared__ float red[2][kSW][32][NV];
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int T = p.T, H = p.H, L = p.L, F = p.F, Fs = p.Fs, G = p.G, K = p.K;
     // the CTA-level activation buffer (D: x for all tokens) precedes the slots
-    const int xs_bytes = PHASE == SP_DPROJ ? 8 * (H + kActPad) * 2 : 0;
+    const int xs_bytes = PHASE == SP_DPROJ ? round128(T * (H + kActPad) * 2) : 0;
     uint8_t* slots = smem + xs_bytes;
 
-    // D reads the routing and x16 of the router kernel, its direct
-    // predecessor.  The later kernels read the routing only before their
-    // wait: their predecessor let them launch after its own wait, so the
-    // router kernel had completed by then.
+    // Routing, as the router kernel published it.  D runs right after the
+    // router kernel and waits for it first.  The later kernels read the
+    // routing before their own wait: their predecessor let them launch only
+    // after its own wait, so the router kernel had completed by then.
     if (PHASE == SP_DPROJ) {
         grid_dep_wait();
         grid_dep_launch();
     }
-    // ---- stage the routing in shared memory
     if (PHASE == SP_GATEUP || PHASE == SP_DOWN) {
         const int n = T * K;
         for (int i = threadIdx.x; i < n; i += blockDim.x) {
             sh.uexp[i] = __ldcg(p.r.uexp + i);
             sh.ucnt[i] = __ldcg(p.r.ucnt + i);
             sh.uoff[i] = __ldcg(p.r.uoff + i);
+            sh.ugrp[i] = __ldcg(p.r.ugrp + i);
             const int pr = __ldcg(p.r.slot_pair + i);
             sh.slot_tok[i] = pr / K;
             sh.slot_w[i] = __ldcg(p.r.w + pr);
         }
         if (threadIdx.x == 0) sh.n_unique = __ldcg(p.r.n_unique);
-        __syncthreads();
-        for (int i = threadIdx.x; i < sh.n_unique; i += blockDim.x) {
-            const int g = p.group[sh.uexp[i]];
-            sh.ugrp[i] = g < G ? g : 0;   // out-of-range labels were reported by the router
-        }
     } else {
         if (threadIdx.x < G) sh.hg[threadIdx.x] = __ldcg(p.r.ghit + threadIdx.x);
         __syncthreads();
@@ -517,7 +505,7 @@ __global__ void __launch_bounds__(kStreamThreads, 1) k_stream(const __grid_const
 #pragma unroll
                 for (int i4 = 0; i4 < 4; ++i4) {
                     red[b][warp][lane][i4] = a[i4];
-                    red[b][warp][lane][4 + i4] = u[i4];
+                    if (NV == 8) red[b][warp][lane][(4 + i4) % NV] = u[i4];
                 }
                 if (warp == 0 && lane == 0) red_meta[b] = m;
                 __syncwarp();
@@ -544,7 +532,7 @@ __global__ void __launch_bounds__(kStreamThreads, 1) k_stream(const __grid_const
 #pragma unroll
                 for (int w = 0; w < kSW; ++w) {
                     sa += red[b][w][lane][i4];
-                    su += red[b][w][lane][4 + i4];
+                    if (NV == 8) su += red[b][w][lane][(4 + i4) % NV];
                 }
                 a[i4] = sa;
                 u[i4] = su;
@@ -730,7 +718,17 @@ static cudaError_t launch_dependent(Kern kern, dim3 grid, dim3 block, size_t sme
 template <int PHASE, int FMT>
 static cudaError_t launch_stream(const StreamMaps& maps, const FwdParams& p, cudaStream_t st, int slot_bytes,
                                  int xs_bytes) {
-    const size_t budget = 192 * 1024;   // dynamic; about 22 KB of static shared memory come on top
+    // dynamic shared memory: what the device allows per block minus the kernel's static part
+    static size_t budget = 0;   // per kernel instance
+    if (!budget) {
+        cudaFuncAttributes fa;
+        int dev = 0, optin = 0;
+        cudaError_t e0 = cudaFuncGetAttributes(&fa, reinterpret_cast<const void*>(k_stream<PHASE, FMT>));
+        if (e0 == cudaSuccess) e0 = cudaGetDevice(&dev);
+        if (e0 == cudaSuccess) e0 = cudaDeviceGetAttribute(&optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev);
+        if (e0 != cudaSuccess) return e0;
+        budget = (size_t)optin - fa.sharedSizeBytes - 1024;
+    }
     const int n_slots = (int)std::min<size_t>(16, (budget - xs_bytes) / slot_bytes);
     if (n_slots < 2) return cudaErrorInvalidValue;
     const size_t smem = 128 + xs_bytes + (size_t)n_slots * slot_bytes;
@@ -746,17 +744,23 @@ static cudaError_t launch_stream(const StreamMaps& maps, const FwdParams& p, cud
     return launch_dependent(kern, dim3(g_sms), dim3(kStreamThreads), smem, st, maps, p, n_slots, slot_bytes);
 }
 
-static int round128(int b) { return (b + 127) & ~127; }
 
-// D, experts, combine, U for T <= 8 (the router kernel has run).
-cudaError_t run_stream_path(const FwdParams& p, cudaStream_t st) {
-    const int H = p.H, L = p.L, F = p.F, Fs = p.Fs, G = p.G, E = p.E;
+
+struct StreamMapSet {
+    StreamMaps d, gu, dn, u;
+};
+
+// Encode the four phases' tensor maps of one layer's weights.
+static bool encode_stream_maps(const FwdParams& p, StreamMapSet* out) {
+    const int H = p.H, L = p.L, F = p.F, G = p.G, E = p.E;
     const size_t qb = p.du_fmt == LMOE_Q8_0 ? 32 : 16;
     const size_t nq = (size_t)L * F / 2, ns = (size_t)L * F / 16;
     const uint8_t* ex = p.experts;
-    StreamMaps md, mgu, mdn, mu;
-    std::memset(&md, 0, sizeof(md));
-    mgu = mdn = mu = md;
+    StreamMaps& md = out->d;
+    StreamMaps& mgu = out->gu;
+    StreamMaps& mdn = out->dn;
+    StreamMaps& mu = out->u;
+    std::memset(out, 0, sizeof(*out));
     bool ok = true;
     const int qr = (int)qb / 2;
     // D: q [H/32][L][qb] + d [H/32][L] fp16 per group
@@ -776,17 +780,65 @@ cudaError_t run_stream_path(const FwdParams& p, cudaStream_t st) {
     ok &= map3(&mdn.wq, ex + 2 * nq, 8, L, F / 32, E, (uint64_t)L * 16, p.rec_bytes);
     ok &= map3(&mdn.ws, ex + 3 * nq + 2 * ns, 2, L, F / 64, E, (uint64_t)L * 4, p.rec_bytes);
     mdn.q_row = 8; mdn.s_row = 2;
-    if (!ok) return cudaErrorInvalidValue;
+    return ok;
+}
+
+// The maps depend only on the weight pointers and the shape, so each layer's
+// set is encoded once and kept (a small round-robin cache; a stack of layers
+// cycles through it).
+static bool stream_maps_for(const FwdParams& p, StreamMapSet* out) {
+    struct Key {
+        const void *D, *U, *ex;
+        int H, L, F, G, E, fmt;
+        size_t bd, bu, br;
+        bool operator==(const Key& o) const { return std::memcmp(this, &o, sizeof(Key)) == 0; }
+    };
+    constexpr int kCache = 64;
+    static Key keys[kCache];
+    static StreamMapSet sets[kCache];
+    static int n = 0, next = 0;
+    static std::mutex mu;
+    Key k;
+    std::memset(&k, 0, sizeof(k));
+    k.D = p.D; k.U = p.U; k.ex = p.experts;
+    k.H = p.H; k.L = p.L; k.F = p.F; k.G = p.G; k.E = p.E; k.fmt = p.du_fmt;
+    k.bd = p.du_bytes_D; k.bu = p.du_bytes_U; k.br = p.rec_bytes;
+    std::lock_guard<std::mutex> lock(mu);
+    for (int i = 0; i < n; ++i)
+        if (keys[i] == k) {
+            *out = sets[i];
+            return true;
+        }
+    if (!encode_stream_maps(p, out)) return false;
+    keys[next] = k;
+    sets[next] = *out;
+    next = (next + 1) % kCache;
+    if (n < kCache) ++n;
+    return true;
+}
+
+// D, experts, combine, U for T <= 8 (the router kernel has run).
+cudaError_t run_stream_path(const FwdParams& p, cudaStream_t st) {
+    const int H = p.H, L = p.L, F = p.F, Fs = p.Fs, G = p.G;
+    const size_t qb = p.du_fmt == LMOE_Q8_0 ? 32 : 16;
+    StreamMapSet ms;
+    if (!stream_maps_for(p, &ms)) return cudaErrorInvalidValue;
+    const StreamMaps& md = ms.d;
+    const StreamMaps& mgu = ms.gu;
+    const StreamMaps& mdn = ms.dn;
+    const StreamMaps& mu = ms.u;
 
     const int act_d = 0;
     const int slot_d = round128(16 * H * (int)qb / 32 + 16 * (H / 32) * 2);
-    const int slot_gu = round128(2 * (16 * L / 2 + 16 * (L / 64) * 4)) + 8 * (L + kActPad) * 2;
-    const int slot_dn = round128(16 * F / 2 + 16 * (F / 64) * 4) + 8 * F * 2;
-    const int slot_u = round128(std::max(16 * L * (int)qb / 32 + 16 * (L / 32) * 2, 32 * Fs)) +
-                       8 * std::max(L + kActPad, Fs) * 2;
+    // activation rows per slot: at most T (an expert sees each token once)
+    const int T = p.T;
+    const int slot_gu = round128(round128(2 * (16 * L / 2 + 16 * (L / 64) * 4)) + T * (L + kActPad) * 2);
+    const int slot_dn = round128(round128(16 * F / 2 + 16 * (F / 64) * 4) + T * F * 2);
+    const int slot_u = round128(round128(std::max(16 * L * (int)qb / 32 + 16 * (L / 32) * 2, 32 * Fs)) +
+                                T * std::max(L + kActPad, Fs) * 2);
     (void)act_d;
     cudaError_t e;
-    const int xs_d = 8 * (H + kActPad) * 2;
+    const int xs_d = round128(T * (H + kActPad) * 2);
     e = p.du_fmt == LMOE_Q8_0 ? launch_stream<SP_DPROJ, LMOE_Q8_0>(md, p, st, slot_d, xs_d)
                               : launch_stream<SP_DPROJ, LMOE_Q4_0>(md, p, st, slot_d, xs_d);
     if (e != cudaSuccess) return e;

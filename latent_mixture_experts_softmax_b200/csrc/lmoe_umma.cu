@@ -334,7 +334,7 @@ __device__ __forceinline__ float u2f(uint32_t u) { return __uint_as_float(u); }
 
 template <int KIND, int NT>
 __device__ __forceinline__ void epilogue_chunk(const PrefillParams& p, const TileRef& t, int warp, int lane, int c0,
-                                               const uint32_t (&r)[32], float* xchg) {
+                                               const uint32_t (&r)[32], float* xchg, const float* tscale) {
     const int row = 32 * warp + lane;      // accumulator row (TMEM lane)
     const int ncol = min(32, t.n - c0);
     if (KIND == G_ROUTER) {
@@ -361,42 +361,43 @@ __device__ __forceinline__ void epilogue_chunk(const PrefillParams& p, const Til
             }
         }
     } else if (KIND == G_GATEUP || KIND == G_SHARED_GATEUP) {
-        // rows 0-63: gate, rows 64-127: up (warps 2, 3 hand theirs to warps 0, 1)
-        if (warp >= 2) {
+        // rows 0-63: gate, rows 64-127: up.  Warps 0-1 finish columns 0-15
+        // of the chunk, warps 2-3 columns 16-31; each hands the other pair
+        // the half it does not finish.
+        float* xg = xchg;              // gate, columns 16-31: [16][64]
+        float* xu = xchg + 16 * 64;    // up, columns 0-15:    [16][64]
+        const int r64 = row & 63;
+        if (warp < 2) {
 #pragma unroll
-            for (int j = 0; j < 32; ++j) xchg[j * 64 + (row - 64)] = u2f(r[j]);
+            for (int j = 0; j < 16; ++j) xg[j * 64 + r64] = u2f(r[16 + j]);
+        } else {
+#pragma unroll
+            for (int j = 0; j < 16; ++j) xu[j * 64 + r64] = u2f(r[j]);
         }
         named_bar_sync(1, 128);
-        if (warp < 2) {
-            float tg = 1.f, tu = 1.f;
-            if (KIND == G_GATEUP) {
-                const size_t nq = (size_t)p.L * p.F / 2, ns = (size_t)p.L * p.F / 16;
-                const float* tail = reinterpret_cast<const float*>(p.experts + (size_t)t.mat * p.rec_bytes + 3 * nq + 3 * ns);
-                tg = __ldg(tail);
-                tu = __ldg(tail + 1);
-            }
-            const int f = t.m0 + row;
+        const float tg = tscale[0], tu = tscale[1];
+        const int f = t.m0 + r64;
+        const int jb = warp < 2 ? 0 : 16;
 #pragma unroll
-            for (int j = 0; j < 32; ++j) {
-                if (j < ncol) {
-                    const float a = u2f(r[j]) * tg;
-                    const float u = xchg[j * 64 + row] * tu;
-                    const float z = silu(a) * u;
-                    if (KIND == G_GATEUP) {
-                        p.zperm[(size_t)(t.b0 + c0 + j) * p.F + f] = __float2half_rn(z);
-                    } else {
-                        const uint16_t hi = f32_to_bf16_bits(z);
-                        p.zsh[(size_t)(t.b0 + c0 + j) * p.Fs + f] = hi;
-                        p.zsh[((size_t)p.T + t.b0 + c0 + j) * p.Fs + f] = f32_to_bf16_bits(z - bf16_bits_to_f32(hi));
-                    }
+        for (int j = 0; j < 16; ++j) {
+            if (jb + j < ncol) {
+                const float a = (warp < 2 ? u2f(r[j]) : xg[j * 64 + r64]) * tg;
+                const float u = (warp < 2 ? xu[j * 64 + r64] : u2f(r[16 + j])) * tu;
+                const float z = silu_fast(a) * u;
+                const int col = t.b0 + c0 + jb + j;
+                if (KIND == G_GATEUP) {
+                    p.zperm[(size_t)col * p.F + f] = __float2half_rn(z);
+                } else {
+                    const uint16_t hi = f32_to_bf16_bits(z);
+                    p.zsh[(size_t)col * p.Fs + f] = hi;
+                    p.zsh[((size_t)p.T + col) * p.Fs + f] = f32_to_bf16_bits(z - bf16_bits_to_f32(hi));
                 }
             }
         }
         named_bar_sync(1, 128);
     } else if (KIND == G_DOWN) {
         // routing weights of the tile's slots staged in xchg by the epilogue warps
-        const size_t nq = (size_t)p.L * p.F / 2, ns = (size_t)p.L * p.F / 16;
-        const float td = __ldg(reinterpret_cast<const float*>(p.experts + (size_t)t.mat * p.rec_bytes + 3 * nq + 3 * ns) + 2);
+        const float td = tscale[2];
         const int l = t.m0 + row;
 #pragma unroll
         for (int j = 0; j < 32; ++j) {
@@ -459,6 +460,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1) k_umma_gemm(const __grid_cons
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     constexpr uint32_t kTmemCols = 2 * NT;
+    __shared__ float tscale[4];   // the current tile's tensor scales (epilogue)
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < STAGES; ++s) {
@@ -636,12 +638,36 @@ __global__ void __launch_bounds__(kGemmThreads, 1) k_umma_gemm(const __grid_cons
             if (KIND == G_DPROJ) {
                 uint32_t* mmask = reinterpret_cast<uint32_t*>(xchg);
                 int* mslot = reinterpret_cast<int*>(mmask + NT);
-                for (int i = threadIdx.x; i < cur.t.n; i += 128)
-                    mmask[i] = __ldg(p.tgmask + (size_t)(cur.t.b0 + i) * p.G + cur.t.mat);
-                for (int i = threadIdx.x; i < cur.t.n * p.K; i += 128)
-                    mslot[i] = __ldg(p.pair_slot + (size_t)cur.t.b0 * p.K + i);
+                // batches of independent loads, then the shared-memory stores
+                const int nn = cur.t.n * p.K;
+                const int* src = p.pair_slot + (size_t)cur.t.b0 * p.K;
+                for (int i0 = threadIdx.x; i0 < nn; i0 += 128 * 8) {
+                    int v[8];
+#pragma unroll
+                    for (int u = 0; u < 8; ++u) v[u] = i0 + 128 * u < nn ? __ldg(src + i0 + 128 * u) : 0;
+#pragma unroll
+                    for (int u = 0; u < 8; ++u)
+                        if (i0 + 128 * u < nn) mslot[i0 + 128 * u] = v[u];
+                }
+                for (int i0 = threadIdx.x; i0 < cur.t.n; i0 += 128 * 2) {
+                    uint32_t v[2];
+#pragma unroll
+                    for (int u = 0; u < 2; ++u)
+                        v[u] = i0 + 128 * u < cur.t.n ? __ldg(p.tgmask + (size_t)(cur.t.b0 + i0 + 128 * u) * p.G + cur.t.mat) : 0u;
+#pragma unroll
+                    for (int u = 0; u < 2; ++u)
+                        if (i0 + 128 * u < cur.t.n) mmask[i0 + 128 * u] = v[u];
+                }
             } else if (KIND == G_DOWN) {
                 for (int i = threadIdx.x; i < cur.t.n; i += 128) xchg[i] = __ldg(p.w + __ldg(p.slot_pair + cur.t.b0 + i));
+            }
+            if ((KIND == G_GATEUP || KIND == G_DOWN) && threadIdx.x < 3) {
+                // the expert's tensor scales (gate, up, down) from its record tail
+                const size_t nq = (size_t)p.L * p.F / 2, ns = (size_t)p.L * p.F / 16;
+                tscale[threadIdx.x] =
+                    __ldg(reinterpret_cast<const float*>(p.experts + (size_t)cur.t.mat * p.rec_bytes + 3 * nq + 3 * ns) + threadIdx.x);
+            } else if (KIND == G_SHARED_GATEUP && threadIdx.x < 3) {
+                tscale[threadIdx.x] = 1.f;
             }
             named_bar_sync(1, 128);
             if (!mbar_wait(&tfull[acc], ph, abort_flag, kWaitLimit)) break;
@@ -651,7 +677,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1) k_umma_gemm(const __grid_cons
                 uint32_t rr[32];
                 tmem_ld_32x32b_x32(taddr + c0, rr);
                 tmem_ld_wait();
-                epilogue_chunk<KIND, NT>(p, cur.t, warp, lane, c0, rr, xchg);
+                epilogue_chunk<KIND, NT>(p, cur.t, warp, lane, c0, rr, xchg, tscale);
             }
             tc_fence_before();
             __syncwarp();
