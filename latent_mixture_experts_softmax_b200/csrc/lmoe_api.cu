@@ -46,7 +46,8 @@ bool use_prefill(const lmoe_cfg& c, int T) {
 // Workspace of the few-token path (first) and of the tensor-core path; both
 // start after the control block, so one allocation serves either.
 struct WsLayout {
-    size_t ctrl, idx, w, logits, n_unique, uexp, ucnt, uoff, ugrp, slot_pair, pair_slot, ghit, tghit;
+    size_t ctrl, idx, w, logits, n_unique, uexp, ucnt, uoff, ugrp, slot_pair, pair_slot, ghit, tghit, wpart, wtick;
+    size_t wtick_bytes;
     size_t x16, h16, zsh, zsh16, o16w, z16, s16, ypart, xio, yio, xa, xb;
     // tensor-core path
     size_t p_zero_begin, p_tgmask, p_cnt, p_fill, p_dhit, p_n_etiles, p_zero_end;
@@ -93,6 +94,12 @@ WsLayout ws_layout(const lmoe_cfg& c, int T) {
         L.z16 = take(TK * c.ffn * 2);
         L.s16 = take((size_t)Td * c.n_groups * c.latent * 2);
         L.ypart = take((size_t)(c.n_groups + 1) * Td * c.hidden * 4);
+        const int Ts = std::min(Td, 8);
+        L.wpart = take(stream_ws_part_bytes(c.hidden, c.latent, c.ffn, c.shared_ffn, c.n_groups, c.n_experts, c.top_k, Ts,
+                                            c.du_fmt));
+        L.wtick_bytes = stream_ws_tick_bytes(c.hidden, c.latent, c.ffn, c.shared_ffn, c.n_groups, c.n_experts, c.top_k, Ts,
+                                             c.du_fmt);
+        L.wtick = take(L.wtick_bytes);
     }
     const size_t end_decode = off;
     if (use_prefill(c, T)) {
@@ -159,6 +166,9 @@ FwdParams base_params(const lmoe_cfg& c, int T, void* ws, const WsLayout& L) {
     p.z16 = reinterpret_cast<__half*>(b + L.z16);
     p.s16 = reinterpret_cast<__half*>(b + L.s16);
     p.ypart = reinterpret_cast<float*>(b + L.ypart);
+    p.wpart = reinterpret_cast<float*>(b + L.wpart);
+    p.wtick = reinterpret_cast<int*>(b + L.wtick);
+    p.wtick_bytes = L.wtick_bytes;
     p.du_bytes_D = du_matrix_bytes(c);
     p.du_bytes_U = du_matrix_bytes(c);
     p.rec_bytes = record_bytes(c);

@@ -195,7 +195,6 @@ __global__ void __launch_bounds__(256) k_router_shared(FwdParams p) {
     if (!router_cta && !p.do_shared) return;
     if (p.prefetch_l2 && blockIdx.x == 0 && p.T <= kChunk)
         l2_prefetch_range(p.sd, (size_t)p.H * p.Fs * 2);
-
     for (int t0 = 0; t0 < p.T; t0 += NT) {
         const int nt = min(NT, p.T - t0);
         stage_x<NT>(p, t0, nt, xs, rs);
@@ -1024,6 +1023,11 @@ static cudaError_t run_gemv_path_nt(FwdParams p, cudaStream_t st, bool route_onl
     p.route_smem = !route_only && p.T <= 8;
     p.prefetch_l2 = false;
     const int n_shared_ctas = route_only ? 0 : (p.Fs + 7) / 8;
+    if (p.route_smem && p.wtick) {
+        // tickets of the split reductions of the weight-streaming kernels
+        cudaError_t e = cudaMemsetAsync(p.wtick, 0, p.wtick_bytes, st);
+        if (e != cudaSuccess) return e;
+    }
     {
         const size_t sm = (size_t)xs_ld(p.H) * NT * sizeof(float);
         cudaError_t e = p.router_bf16

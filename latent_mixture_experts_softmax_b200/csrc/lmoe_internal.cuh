@@ -75,6 +75,9 @@ struct FwdParams {
     __half* z16;    // [T*K][F]     expert hidden per slot (slots grouped by expert)
     __half* s16;    // [T][G][L]    per-group weighted expert sums
     float* ypart;   // [G+1][T][H]  U_g parts and the shared part
+    float* wpart;   // few-token path: partial 16x8 fragments of split reductions
+    int* wtick;     // few-token path: parts finished per output tile
+    size_t wtick_bytes;
     size_t du_bytes_D, du_bytes_U, rec_bytes;
     // launch shape of the router kernel
     int n_router_ctas, router_rows_per_warp;
@@ -87,6 +90,9 @@ constexpr int kMaxStageEvents = 16;
 
 cudaError_t run_gemv_path(const FwdParams& p, cudaStream_t st, bool route_only);
 cudaError_t run_stream_path(const FwdParams& p, cudaStream_t st);
+// workspace of the few-token path's split reductions, for up to T tokens
+size_t stream_ws_part_bytes(int H, int L, int F, int Fs, int G, int E, int K, int T, int du_fmt);
+size_t stream_ws_tick_bytes(int H, int L, int F, int Fs, int G, int E, int K, int T, int du_fmt);
 void set_stage_events(void* const* events, int n);
 void stage_mark(cudaStream_t st);
 void stage_reset();

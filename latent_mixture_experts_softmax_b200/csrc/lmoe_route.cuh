@@ -38,46 +38,58 @@ struct StreamShared {
 // single CTA to publish it
 // ---------------------------------------------------------------------------
 
+// Order-preserving map of a float onto an unsigned integer (larger float,
+// larger key; -0 and +0 map to the same key), and back.
+static __device__ __forceinline__ uint32_t order_key(float f) {
+    const uint32_t b = __float_as_uint(f + 0.0f);
+    return (b & 0x80000000u) ? ~b : (b | 0x80000000u);
+}
+static __device__ __forceinline__ float key_value(uint32_t k) {
+    return __uint_as_float((k & 0x80000000u) ? (k & 0x7fffffffu) : ~k);
+}
+
+// Largest of n packed (key, ~index) words, as a tree of comparisons.
+template <int N>
+static __device__ __forceinline__ uint64_t tree_max(const uint64_t (&pk)[N]) {
+    uint64_t m[N];
+#pragma unroll
+    for (int j = 0; j < N; ++j) m[j] = pk[j];
+#pragma unroll
+    for (int w = N / 2; w > 0; w >>= 1) {
+#pragma unroll
+        for (int j = 0; j < w; ++j) m[j] = m[j] > m[j + w] ? m[j] : m[j + w];
+    }
+    return m[0];
+}
+
 // Softmax top-K of one token by one warp (section "Routing" of the teardown
 // article: softmax over the E logits, top-K, renormalise over the kept):
-// K rounds of a warp arg-max, ties to the lower index; w_k = exp(l_k - l_1)
-// / sum over the kept of exp(l_j - l_1).  Writes idx[0..K), w[0..K).
+// ties go to the lower expert index; w_k = exp(l_k - l_1) / sum over the
+// kept of exp(l_j - l_1).  Writes idx[0..K), w[0..K).  Each lane packs its
+// NV logits as (order key, ~index) words and keeps its best; a round is two
+// warp reductions over the lanes' bests (largest key, then the lowest index
+// holding it) and, in the winning lane, a tree maximum over what is left.
 template <int NV>
 static __device__ void topk_row(const float* logits, int E, int K, int lane, int* idx, float* w) {
-    float v[NV];
+    uint64_t pk[NV];
 #pragma unroll
     for (int j = 0; j < NV; ++j) {
         const int e = lane + 32 * j;
-        v[j] = e < E ? __ldcg(logits + e) : -INFINITY;
+        pk[j] = e < E ? ((uint64_t)order_key(__ldcg(logits + e)) << 32) | (uint32_t)~e : 0ull;
     }
-    uint32_t taken = 0;
-    float lv = -INFINITY;
-    int li = 0x7fffffff;
-#pragma unroll
-    for (int j = 0; j < NV; ++j) {
-        const int e = lane + 32 * j;
-        if (e < E && v[j] > lv) { lv = v[j]; li = e; }
-    }
+    uint64_t best = tree_max(pk);
     float lmax = 0.f, denom = 0.f, my_l = 0.f;
     int my_e = 0;
     for (int k = 0; k < K; ++k) {
-        float bv = lv;
-        int bi = li;
+        const uint32_t key = (uint32_t)(best >> 32);
+        const uint32_t kmax = __reduce_max_sync(0xffffffffu, key);
+        const int bi = (int)__reduce_min_sync(0xffffffffu, key == kmax ? ~(uint32_t)best : 0xffffffffu);
+        const float bv = key_value(kmax);
+        if (~(uint32_t)best == (uint32_t)bi) {
 #pragma unroll
-        for (int o = 16; o > 0; o >>= 1) {
-            const float ov = __shfl_xor_sync(0xffffffffu, bv, o);
-            const int oi = __shfl_xor_sync(0xffffffffu, bi, o);
-            if (ov > bv || (ov == bv && oi < bi)) { bv = ov; bi = oi; }
-        }
-        if (bi < E && (bi & 31) == lane) {
-            taken |= 1u << (bi >> 5);
-            lv = -INFINITY;
-            li = 0x7fffffff;
-#pragma unroll
-            for (int j = 0; j < NV; ++j) {
-                const int e = lane + 32 * j;
-                if (e < E && !(taken >> j & 1u) && (v[j] > lv || (v[j] == lv && e < li))) { lv = v[j]; li = e; }
-            }
+            for (int j = 0; j < NV; ++j)
+                if (j == (bi >> 5)) pk[j] = 0ull;
+            best = tree_max(pk);
         }
         if (k == 0) lmax = bv;
         if (k == lane) { my_l = bv; my_e = bi; }
@@ -89,14 +101,16 @@ static __device__ void topk_row(const float* logits, int E, int K, int lane, int
     }
 }
 
-// Bucketing of the T*K pairs by one warp, in shared memory: slots ordered by
-// (expert, pair index), distinct experts ascending, pairs per group.
-// `grp` is the expert -> group table (in shared memory).  Invalid indices
-// or labels are reported (report = true) and read as 0.
-static __device__ void bucket_pairs(const FwdParams& p, StreamShared& sh, const uint8_t* grp, int lane, bool report) {
+// Bucketing of the T*K pairs by the whole CTA (one pair per thread), in
+// shared memory: slots ordered by (expert, pair index), distinct experts
+// ascending, pairs per group.  `grp` is the expert -> group table (in shared
+// memory).  Invalid indices or labels are reported (report = true) and read
+// as 0.  Contains __syncthreads.
+static __device__ void bucket_pairs(const FwdParams& p, StreamShared& sh, const uint8_t* grp, bool report) {
     const int K = p.K, G = p.G, E = p.E, n = p.T * K;
-    for (int g = lane; g < G; g += 32) sh.gcnt[g] = 0;
-    for (int i = lane; i < n; i += 32) {
+    for (int g = threadIdx.x; g < G; g += blockDim.x) sh.gcnt[g] = 0;
+    if (threadIdx.x == 0) sh.n_unique = 0;
+    for (int i = threadIdx.x; i < n; i += blockDim.x) {
         int e = sh.idx[i];
         if (e < 0 || e >= E) {
             if (report) set_status(p.ctrl, LMOE_ERR_DEVICE_CHECK);
@@ -110,16 +124,16 @@ static __device__ void bucket_pairs(const FwdParams& p, StreamShared& sh, const 
         sh.pe[i] = e;
         sh.pgrp[i] = g;
     }
-    __syncwarp();
-    for (int i = lane; i < n; i += 32) {
+    __syncthreads();
+    for (int i = threadIdx.x; i < n; i += blockDim.x) {
+        const int e = sh.pe[i];
         bool first = true;
 #pragma unroll 8
-        for (int j = 0; j < i; ++j) first &= sh.pe[j] != sh.pe[i];
+        for (int j = 0; j < i; ++j) first &= sh.pe[j] != e;
         sh.pfirst[i] = first;
     }
-    __syncwarp();
-    int n_first = 0;
-    for (int i = lane; i < n; i += 32) {
+    __syncthreads();
+    for (int i = threadIdx.x; i < n; i += blockDim.x) {
         const int e = sh.pe[i];
         int less = 0, same_before = 0, cnt = 0, u = 0;
 #pragma unroll 8
@@ -130,32 +144,28 @@ static __device__ void bucket_pairs(const FwdParams& p, StreamShared& sh, const 
             cnt += ej == e;
             u += (sh.pfirst[j] && ej < e);
         }
-        const bool first = sh.pfirst[i];
         const int slot = less + same_before;
         sh.slot_pair[slot] = i;
         sh.pair_slot[i] = slot;
         sh.slot_tok[slot] = i / K;
         sh.slot_w[slot] = sh.w[i];
-        if (first) {
+        if (sh.pfirst[i]) {
             sh.uexp[u] = e;
             sh.ucnt[u] = cnt;
             sh.uoff[u] = less;
             sh.ugrp[u] = sh.pgrp[i];
-            ++n_first;
+            atomicAdd(&sh.n_unique, 1);
         }
         atomicAdd(&sh.gcnt[sh.pgrp[i]], 1);
     }
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) n_first += __shfl_xor_sync(0xffffffffu, n_first, o);
-    __syncwarp();
-    if (lane == 0) {
-        sh.n_unique = n_first;
+    __syncthreads();
+    if (threadIdx.x == 0) {
         int nh = 0;
         for (int g = 0; g < G; ++g)
             if (sh.gcnt[g] > 0) sh.hg[nh++] = g;
         sh.n_hit = nh;
     }
-    __syncwarp();
+    __syncthreads();
 }
 
 // The step's routing into `sh`, by every thread of the CTA (contains
@@ -180,8 +190,7 @@ static __device__ void route_in_cta(const FwdParams& p, StreamShared& sh, const 
         }
     }
     __syncthreads();
-    if (warp == 0) bucket_pairs(p, sh, grp, lane, publish);
-    __syncthreads();
+    bucket_pairs(p, sh, grp, publish);
     if (!publish) return;
     const Routing& r = p.r;
     for (int i = threadIdx.x; i < n; i += blockDim.x) {

@@ -1,24 +1,29 @@
-// Few-token path (T <= 8), weight-streaming kernels: one persistent CTA per
-// SM streams 16-row weight tiles through a ring of shared-memory slots with
-// the TMA engine (tensor-map tile loads of the stored formats, no
-// conversion on the way) while eight compute warps dequantise each tile in
-// registers and multiply it with the staged activations on the tensor pipe
-// (mma.sync m16n8k16, fp16 operands, fp32 accumulation; the 8 MMA columns are
-// the up to 8 tokens).  Several tiles per SM are in flight at once, so HBM
-// streams without waiting on the arithmetic.
+// Few-token path (T <= 8), weight-streaming kernels.  One CTA per SM, 16
+// warps.  A work item is one 16-row tile of one matrix over one part of its
+// reduction (K); each warp streams its items' stored bytes (codes and
+// scales exactly as they sit in HBM) through its own ring of shared-memory
+// step buffers with per-thread asynchronous copies (cp.async, 16 bytes per
+// thread; the bulk-copy engine's fixed cost per copy would cap the rate),
+// dequantises in registers and multiplies on the tensor pipe (mma.sync
+// m16n8k16, fp16 operands, fp32 accumulation; the 8 MMA columns are the up
+// to 8 tokens).  Items are split into contiguous chunks per CTA; the
+// activations of a chunk are read once into a shared-memory cache.  When a
+// tile's reduction is split into parts, each part's 16x8 partial goes to
+// the workspace and the warp that completes the tile (ticket) adds the
+// parts in order and runs the epilogue.
 //
-//   k_stream<DPROJ>   h16[t][g]   = D_g x_t            (hit groups)
-//   k_stream<GATEUP>  z16[slot]   = silu(W_gate h) * (W_up h)
-//   k_stream<DOWN>    o16w[slot]  = w_slot * W_down z
-//   k_combine_small   s16[t][g]   = sum of o16w over the token's experts in g
-//   k_stream<UPROJ>   y           = sum_g U_g s16[t][g] + S_down z_sh (+ residual)
+//   k_wstream<DPROJ>   h16[t][g]   = D_g x_t            (hit groups)
+//   k_wstream<GATEUP>  z16[slot]   = silu(W_gate h) * (W_up h)
+//   k_wstream<DOWN>    o16w[slot]  = w_slot * W_down z
+//   k_combine_small    s16[g][t]   = sum of o16w over the token's experts in g
+//   k_wstream<UPROJ>   y           = sum_g U_g s16[g][t] + S_down z_sh (+ residual)
 //
 // Method: teardown article "Edge0-145B: a Qwen MoE with its experts
 // squeezed", section "A latent in front of the experts" (layer equation,
 // per-group D/U); Edge0 145B / 120B model page, architecture tables.
 
+#include <algorithm>
 #include <cstring>
-#include <mutex>
 
 #include "lmoe_internal.cuh"
 #include "lmoe_route.cuh"
@@ -30,32 +35,14 @@ using namespace sm100;
 
 enum StreamPhase { SP_DPROJ = 0, SP_GATEUP = 1, SP_DOWN = 2, SP_UPROJ = 3 };
 
-constexpr int kSW = 16;                // compute warps per CTA
-constexpr int kStreamThreads = 32 * (kSW + 2);   // + loader warp + reducer warp
-constexpr int kMaxSlots = 16;          // weight slots in the ring
+constexpr int kWW = 16;                     // warps per CTA
+constexpr int kWThreads = 32 * kWW;
+constexpr int kPD = 4;                      // step buffers per warp (3 steps in flight)
+constexpr int kStepBytes = 2304;            // largest step (see step_geom)
+constexpr int kMaxChunkParts = 8;           // distinct matrices in one CTA's chunk
+constexpr int kActPad = 32;                 // halves of padding per cached activation row
 
 __host__ __device__ __forceinline__ int round128(int b) { return (b + 127) & ~127; }
-constexpr int kActPad = 32;            // halves of padding per staged activation row
-constexpr uint64_t kStreamWait = 4000000000ull;   // SM cycles per barrier wait
-
-// Every weight map is 3-D over 16-bit units: (one K block's rows, contiguous;
-// K blocks; matrices).  A box takes 16 consecutive rows of every K block of
-// one matrix, so each TMA line is a 256-512 byte run, not one row.
-struct __align__(64) StreamMaps {
-    CUtensorMap wq;    // weight codes: D/U q (over groups) or expert gate/down q (over experts)
-    CUtensorMap ws;    // weight scales: D/U d or expert gate/down s
-    CUtensorMap wq2;   // expert up q
-    CUtensorMap ws2;   // expert up s
-    int q_row;         // 16-bit units per row of one K block in wq / wq2
-    int s_row;         // 16-bit units per row of one K block in ws / ws2
-};
-
-struct Item {
-    int kind;   // 0: weight tile of a group / expert, 1: shared-expert tile (UPROJ)
-    int mat;    // group g or expert e
-    int j;      // distinct-expert index (expert phases)
-    int r0;     // first of the tile's 16 output rows
-};
 
 __device__ __forceinline__ void mma16816s(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
                                           uint32_t b0, uint32_t b1) {
@@ -193,109 +180,195 @@ __device__ __forceinline__ void tile_bf16(const uint16_t* w, int K, const __half
     }
 }
 
+
 // ---------------------------------------------------------------------------
-// work items
+// items, steps and parts
 // ---------------------------------------------------------------------------
 
+// K blocks (32 elements) per step and the step's byte layout:
+//   D / U groups Q8_0: 4 blocks  codes [4][16][32] + scales [4][16] fp16 = 2176 B
+//   D / U groups Q4_0: 8 blocks  codes [8][16][16] + scales [8][16] fp16 = 2304 B
+//   gate/up NVFP4:     4 chunks  gate codes [4][16][16], up codes, gate scales [2][16][4], up scales = 2304 B
+//   down NVFP4:        8 chunks  codes [8][16][16] + scales [4][16][4] = 2304 B
+//   U shared bf16:     2 blocks  [16 rows][64] bf16 = 2048 B
+template <int PHASE, int FMT>
+__host__ __device__ __forceinline__ int step_blocks(bool shared_part) {
+    if (PHASE == SP_GATEUP) return 4;
+    if (PHASE == SP_DOWN) return 8;
+    if (PHASE == SP_UPROJ && shared_part) return 2;
+    return FMT == LMOE_Q8_0 ? 4 : 8;
+}
 
 template <int PHASE>
 __host__ __device__ __forceinline__ int stream_rows(int H, int L, int F) {
     return PHASE == SP_DPROJ ? L : PHASE == SP_GATEUP ? F : PHASE == SP_DOWN ? L : H;
 }
 
-// What the compute and reducer warps need to know about the item in a slot.
-struct __align__(16) SlotMeta {
-    float tail[4];   // expert record tail: tensor scales of gate, up, down
-    Item item;
-    int nt;          // activation rows (tokens or slots) of the item
-    int off;         // first slot of the expert (expert phases)
+// One decoded work item.
+struct WItem {
+    int mat;       // group (D, U), expert (gate/up, down); -1: the shared expert (U)
+    int j;         // distinct-expert index (gate/up, down) / part index (U)
+    int r0;        // first output row
+    int tile;      // output tile index
+    int q;         // reduction part
+    int kb0, kb1;  // K blocks of the part
 };
 
-template <int PHASE>
-__device__ __forceinline__ int stream_items(const FwdParams& p, const StreamShared& sh) {
-    const int tiles = stream_rows<PHASE>(p.H, p.L, p.F) / 16;
-    if (PHASE == SP_DPROJ) return sh.n_hit * tiles;
-    if (PHASE == SP_UPROJ) return (sh.n_hit + 1) * tiles;
-    return sh.n_unique * tiles;
-}
+struct WPlan {
+    int ks;        // reduction parts per tile
+    int tiles;     // output tiles per matrix
+    int n_mats;    // matrices (D: hit groups; experts; U: hit groups + shared)
+};
 
-// Item i: D / experts run matrix-major (consecutive items share a
-// matrix); U runs row-tile-major (consecutive items are the parts of one
-// output tile: the hit groups ascending, then the shared expert).
-template <int PHASE>
-__device__ __forceinline__ Item stream_item(const StreamShared& sh, int tiles, int i) {
-    Item it;
-    it.kind = 0;
-    it.j = 0;
-    if (PHASE == SP_UPROJ) {
-        const int parts = sh.n_hit + 1, part = i % parts;
-        it.r0 = (i / parts) * 16;
-        it.j = part;
-        if (part < sh.n_hit) it.mat = sh.hg[part];
-        else { it.kind = 1; it.mat = 0; }
-        return it;
-    }
-    const int m = i / tiles;
-    it.r0 = (i % tiles) * 16;
+// Items run matrix-major (consecutive items share a matrix, so a CTA's chunk
+// touches few of them), then tile, then part.
+template <int PHASE, int FMT>
+__device__ __forceinline__ WItem decode_item(const FwdParams& p, const StreamShared& sh, const WPlan& pl, int i) {
+    WItem it;
+    const int per_mat = pl.tiles * pl.ks;
+    const int m = i / per_mat, rem = i - m * per_mat;
+    it.tile = rem / pl.ks;
+    it.q = rem - it.tile * pl.ks;
+    it.r0 = it.tile * 16;
+    it.j = m;
+    bool shared_part = false;
+    int nb;
     if (PHASE == SP_DPROJ) {
         it.mat = sh.hg[m];
+        nb = p.H / 32;
+    } else if (PHASE == SP_UPROJ) {
+        shared_part = m == sh.n_hit;
+        it.mat = shared_part ? -1 : sh.hg[m];
+        nb = shared_part ? p.Fs / 32 : p.L / 32;
     } else {
-        it.j = m;
         it.mat = sh.uexp[m];
+        nb = (PHASE == SP_GATEUP ? p.L : p.F) / 32;
     }
+    const int sb = step_blocks<PHASE, FMT>(shared_part);
+    const int ns = (nb + sb - 1) / sb;
+    it.kb0 = min(nb, (it.q * ns / pl.ks) * sb);
+    it.kb1 = min(nb, ((it.q + 1) * ns / pl.ks) * sb);
     return it;
 }
 
-// First item of CTA c when n items are split into contiguous chunks.
 __device__ __forceinline__ int chunk_begin(int c, int n, int ctas) {
     return (int)(((long long)c * n) / ctas);
 }
 
-// Slot layout: weights (A, A2, S, S2) then the item's activations.
-template <int PHASE, int FMT>
-struct SlotPlan {
-    __device__ static int a_bytes(const FwdParams& p) {
-        if (PHASE == SP_DPROJ) return 16 * p.H * (FMT == LMOE_Q8_0 ? 32 : 16) / 32;
-        if (PHASE == SP_UPROJ) return 16 * p.L * (FMT == LMOE_Q8_0 ? 32 : 16) / 32;
-        if (PHASE == SP_GATEUP) return 16 * p.L / 2;
-        return 16 * p.F / 2;
-    }
-    __device__ static int s_bytes(const FwdParams& p) {
-        if (PHASE == SP_DPROJ) return 16 * (p.H / 32) * 2;
-        if (PHASE == SP_UPROJ) return 16 * (p.L / 32) * 2;
-        if (PHASE == SP_GATEUP) return 16 * (p.L / 64) * 4;
-        return 16 * (p.F / 64) * 4;
-    }
-};
+__device__ __forceinline__ void cp_async16(void* dst, const void* src) {
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_u32(dst)), "l"(src) : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+template <int N>
+__device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory"); }
 
-// Warp roles: kSW compute warps, one loader warp (one thread issues every
-// copy), one reducer warp.  The compute warps split each item's reduction
-// (K) evenly, hand their partial 16 x 8 fragments to the reducer through
-// one of two shared buffers and go straight on to the next item; the
-// reducer sums the partials and runs the epilogue.  No step of an item
-// waits for another item's epilogue.
+// Issue the copies of step `st` of item `it` into `buf` (every lane).
 template <int PHASE, int FMT>
-__global__ void __launch_bounds__(kStreamThreads, 1) k_stream(const __grid_constant__ StreamMaps maps, FwdParams p,
-                                                              int n_slots, int slot_bytes) {
+__device__ __forceinline__ void issue_step(const FwdParams& p, const WItem& it, int st, uint8_t* buf, int lane) {
+    const int L = p.L, F = p.F, H = p.H, Fs = p.Fs;
+    const bool shared_part = PHASE == SP_UPROJ && it.mat < 0;
+    const int sb = step_blocks<PHASE, FMT>(shared_part);
+    const int kb = it.kb0 + st * sb;
+    const int nblk = min(sb, it.kb1 - kb);
+    if (PHASE == SP_DPROJ || (PHASE == SP_UPROJ && !shared_part)) {
+        const int qb = FMT == LMOE_Q8_0 ? 32 : 16;
+        const int R = PHASE == SP_DPROJ ? L : H;
+        const int C = PHASE == SP_DPROJ ? H : L;
+        const uint8_t* mat = (PHASE == SP_DPROJ ? p.D + (size_t)it.mat * p.du_bytes_D : p.U + (size_t)it.mat * p.du_bytes_U);
+        const uint8_t* dsc = mat + (size_t)R * C / 32 * qb;
+        const int cpb = qb;                 // 16-byte chunks of codes per block (16 rows x qb bytes / 16)
+        const int n_codes = nblk * cpb, n_sc = nblk * 2;
+        for (int c = lane; c < n_codes + n_sc; c += 32) {
+            if (c < n_codes) {
+                const int b = c / cpb, o = (c - b * cpb) * 16;
+                cp_async16(buf + (size_t)c * 16, mat + ((size_t)(kb + b) * R + it.r0) * qb + o);
+            } else {
+                const int c2 = c - n_codes, b = c2 >> 1;
+                cp_async16(buf + (size_t)sb * 16 * qb + (size_t)c2 * 16, dsc + ((size_t)(kb + b) * R + it.r0) * 2 + (c2 & 1) * 16);
+            }
+        }
+    } else if (PHASE == SP_UPROJ) {
+        // shared expert down rows [H][Fs] bf16: 16 rows x 64 columns per 2 blocks
+        const int n = 16 * nblk * 4;        // 16-byte chunks: 4 per row per block
+        for (int c = lane; c < n; c += 32) {
+            const int row = c / (nblk * 4), o = (c - row * nblk * 4) * 16;
+            cp_async16(buf + (size_t)row * 128 + o, reinterpret_cast<const uint8_t*>(p.sd + (size_t)(it.r0 + row) * Fs) + (size_t)kb * 64 + o);
+        }
+    } else {
+        const size_t nq = (size_t)L * F / 2, ns = (size_t)L * F / 16;
+        const uint8_t* rec = p.experts + (size_t)it.mat * p.rec_bytes;
+        const int R = PHASE == SP_GATEUP ? F : L;
+        const uint8_t* q0 = rec + (PHASE == SP_GATEUP ? 0 : 2 * nq);
+        const uint8_t* s0 = rec + 3 * nq + (PHASE == SP_GATEUP ? 0 : 2 * ns);
+        const int nmat = PHASE == SP_GATEUP ? 2 : 1;      // gate and up
+        const int n_codes = nblk * 16, n_sc = ((nblk + 1) / 2) * 4;
+        const int qbytes = sb * 256, sbytes = (sb / 2) * 64;
+        for (int mm = 0; mm < nmat; ++mm) {
+            const uint8_t* qm = q0 + mm * nq;
+            const uint8_t* sm = s0 + mm * ns;
+            uint8_t* bq = buf + mm * qbytes;
+            uint8_t* bs = buf + nmat * qbytes + mm * sbytes;
+            for (int c = lane; c < n_codes + n_sc; c += 32) {
+                if (c < n_codes) {
+                    const int b = c >> 4, o = (c & 15) * 16;
+                    cp_async16(bq + (size_t)c * 16, qm + ((size_t)(kb + b) * R + it.r0) * 16 + o);
+                } else {
+                    const int c2 = c - n_codes, b = c2 >> 2;
+                    cp_async16(bs + (size_t)c2 * 16, sm + ((size_t)(kb / 2 + b) * R + it.r0) * 4 + (c2 & 3) * 16);
+                }
+            }
+        }
+    }
+}
+
+// Multiply step `st` (in `buf`) with the item's activations.
+template <int PHASE, int FMT>
+__device__ __forceinline__ void compute_step(const FwdParams& p, const WItem& it, int st, const uint8_t* buf,
+                                             const __half* xs, int ld, int nt, float (&a)[4], float (&u)[4]) {
+    const bool shared_part = PHASE == SP_UPROJ && it.mat < 0;
+    const int sb = step_blocks<PHASE, FMT>(shared_part);
+    const int kb = it.kb0 + st * sb;
+    const int nblk = min(sb, it.kb1 - kb);
+    const __half* x = xs + kb * 32;
+    if (PHASE == SP_DPROJ || (PHASE == SP_UPROJ && !shared_part)) {
+        const int qb = FMT == LMOE_Q8_0 ? 32 : 16;
+        tile_du<FMT>(buf, reinterpret_cast<const uint16_t*>(buf + sb * 16 * qb), x, ld, nt, 0, nblk, a);
+    } else if (PHASE == SP_UPROJ) {
+        tile_bf16(reinterpret_cast<const uint16_t*>(buf), 64, x, ld, nt, 0, nblk, a);
+    } else if (PHASE == SP_GATEUP) {
+        tile_nvfp4(buf, buf + 2 * 1024, x, ld, nt, 0, nblk, a);
+        tile_nvfp4(buf + 1024, buf + 2 * 1024 + 128, x, ld, nt, 0, nblk, u);
+    } else {
+        tile_nvfp4(buf, buf + 2048, x, ld, nt, 0, nblk, a);
+    }
+}
+
+template <int PHASE>
+__device__ __forceinline__ int n_steps(const WItem& it, int sb) { return (it.kb1 - it.kb0 + sb - 1) / sb; }
+
+// ---------------------------------------------------------------------------
+// the kernel
+// ---------------------------------------------------------------------------
+
+template <int PHASE, int FMT>
+__global__ void __launch_bounds__(kWThreads, 1) k_wstream(FwdParams p, WPlan pl, int cache_bytes) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 127) & ~(uintptr_t)127);
     __shared__ StreamShared sh;
-    __shared__ SlotMeta meta[kMaxSlots];
-    __shared__ SlotMeta red_meta[2];
-    __shared__ __align__(8) uint64_t full[kMaxSlots];
-    __shared__ __align__(8) uint64_t empty[kMaxSlots];
-    __shared__ __align__(8) uint64_t red_full[2];
-    __shared__ __align__(8) uint64_t red_empty[2];
-    __shared__ __align__(8) uint64_t xbar;
-    __shared__ int abort_flag;
-    constexpr int NV = PHASE == SP_GATEUP ? 8 : 4;   // partial values per lane (gate [+ up])
-    __shared__ float red[2][kSW][32][NV];
+    // the chunk's matrices: cache rows and (experts) tensor scales
+    __shared__ int c_m0, c_nm, c_skip, c_rows;
+    __shared__ int c_row0[kMaxChunkParts];
+    __shared__ int c_src[kMaxChunkParts * 8];
+    __shared__ float c_tail[kMaxChunkParts][4];
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int T = p.T, H = p.H, L = p.L, F = p.F, Fs = p.Fs, G = p.G, K = p.K;
-    // the CTA-level activation buffer (D: x for all tokens) precedes the slots
-    const int xs_bytes = PHASE == SP_DPROJ ? round128(T * (H + kActPad) * 2) : 0;
-    uint8_t* slots = smem + xs_bytes;
+    __half* cache = reinterpret_cast<__half*>(smem);
+    uint8_t* ring = smem + cache_bytes + (size_t)warp * kPD * kStepBytes;
+    const int ld = PHASE == SP_DPROJ ? H + kActPad
+                 : PHASE == SP_GATEUP ? L + kActPad
+                 : PHASE == SP_DOWN ? F + kActPad
+                                    : max(L, Fs) + kActPad;
 
     // Routing, as the router kernel published it.  D runs right after the
     // router kernel and waits for it first.  The later kernels read the
@@ -327,303 +400,204 @@ __global__ void __launch_bounds__(kStreamThreads, 1) k_stream(const __grid_const
             sh.n_hit = n;
         }
     }
+    __syncthreads();
+
+    WPlan plan = pl;
+    plan.n_mats = PHASE == SP_DPROJ ? sh.n_hit : PHASE == SP_UPROJ ? sh.n_hit + 1 : sh.n_unique;
+    const int n_items = plan.n_mats * plan.tiles * plan.ks;
+    const int i0 = chunk_begin(blockIdx.x, n_items, gridDim.x);
+    int i1 = chunk_begin(blockIdx.x + 1, n_items, gridDim.x);
+    const int per_mat = plan.tiles * plan.ks;
+
+    // the chunk's matrices and their activation rows
     if (threadIdx.x == 0) {
-        for (int s = 0; s < n_slots; ++s) {
-            mbar_init(&full[s], 1);
-            mbar_init(&empty[s], kSW);
+        const int m0 = i0 / per_mat, m1 = i0 < i1 ? (i1 - 1) / per_mat : m0 - 1;
+        const int nm = PHASE == SP_DPROJ ? 1 : m1 - m0 + 1;
+        int rows = 0;
+        bool fits = nm <= kMaxChunkParts;
+        for (int jj = 0; fits && jj < nm; ++jj) {
+            const int m = m0 + jj;
+            c_row0[jj] = rows;
+            const int nr = (PHASE == SP_GATEUP || PHASE == SP_DOWN) ? sh.ucnt[m] : T;
+            if (rows + nr > kMaxChunkParts * 8) { fits = false; break; }
+            for (int c = 0; c < nr; ++c, ++rows) {
+                int src;
+                if (PHASE == SP_DPROJ) src = c;                                           // x16 row
+                else if (PHASE == SP_GATEUP) src = sh.slot_tok[sh.uoff[m] + c] * G + sh.ugrp[m];   // h16 row
+                else if (PHASE == SP_DOWN) src = sh.uoff[m] + c;                          // z16 row
+                else src = m < sh.n_hit ? sh.hg[m] * T + c : -1 - c;                      // s16 row / shared hidden row
+                c_src[rows] = src;
+            }
         }
-        for (int b = 0; b < 2; ++b) {
-            mbar_init(&red_full[b], kSW);
-            mbar_init(&red_empty[b], 1);
+        fits = fits && (size_t)rows * ld * 2 <= (size_t)cache_bytes;
+        if (!fits) set_status(p.ctrl, LMOE_ERR_UNSUPPORTED);
+        c_m0 = m0;
+        c_nm = fits ? nm : 0;
+        c_skip = !fits;
+        c_rows = fits ? rows : 0;
+    }
+    __syncthreads();
+    if (c_skip) i1 = i0;
+    if ((PHASE == SP_GATEUP || PHASE == SP_DOWN) && threadIdx.x < 4 * c_nm) {
+        const int jj = threadIdx.x >> 2, qq = threadIdx.x & 3;
+        const size_t nq = (size_t)L * F / 2, ns = (size_t)L * F / 16;
+        const float* tail =
+            reinterpret_cast<const float*>(p.experts + (size_t)sh.uexp[c_m0 + jj] * p.rec_bytes + 3 * nq + 3 * ns);
+        c_tail[jj][qq] = __ldg(tail + qq);
+    }
+
+    // Every warp starts streaming its first steps' weights, which depend on
+    // the routing only, before the activations of the previous kernel exist.
+    const WItem none = {0, 0, 0, 0, 0, 0, 0};
+    int li = i0 + warp, ls = 0, l_ns = 0;      // load cursor: item, step, steps of the item
+    WItem lit = none;
+    if (li < i1) {
+        lit = decode_item<PHASE, FMT>(p, sh, plan, li);
+        l_ns = n_steps<PHASE>(lit, step_blocks<PHASE, FMT>(PHASE == SP_UPROJ && lit.mat < 0));
+    }
+    auto advance_load = [&]() {
+        if (li >= i1) return;
+        if (++ls < l_ns) return;
+        ls = 0;
+        li += kWW;
+        if (li < i1) {
+            lit = decode_item<PHASE, FMT>(p, sh, plan, li);
+            l_ns = n_steps<PHASE>(lit, step_blocks<PHASE, FMT>(PHASE == SP_UPROJ && lit.mat < 0));
         }
-        mbar_init(&xbar, 1);
-        abort_flag = 0;
-        fence_barrier_init();
+    };
+    int n_issued = 0;
+#pragma unroll
+    for (int k = 0; k < kPD - 1; ++k) {
+        if (li < i1) issue_step<PHASE, FMT>(p, lit, ls, ring + (size_t)(n_issued % kPD) * kStepBytes, lane);
+        cp_async_commit();
+        ++n_issued;
+        advance_load();
+    }
+
+    if (PHASE != SP_DPROJ) {
+        grid_dep_wait();
+        grid_dep_launch();
+    }
+    // the chunk's activations, by plain loads of every thread
+    {
+        const int rows = c_rows;
+        const int KC = PHASE == SP_DPROJ ? H : PHASE == SP_GATEUP ? L : PHASE == SP_DOWN ? F : max(L, Fs);
+        const int per = KC / 8;
+        for (int qv = threadIdx.x; qv < rows * per; qv += blockDim.x) {
+            const int r = qv / per, c = qv - r * per;
+            const int src = c_src[r];
+            const __half* s;
+            int w = KC;
+            if (PHASE == SP_DPROJ) s = p.x16 + (size_t)src * H;
+            else if (PHASE == SP_GATEUP) s = p.h16 + (size_t)src * L;
+            else if (PHASE == SP_DOWN) s = p.z16 + (size_t)src * F;
+            else if (src >= 0) { s = p.s16 + (size_t)src * L; w = L; }
+            else { s = p.zsh16 + (size_t)(-1 - src) * Fs; w = Fs; }
+            if (8 * c < w)
+                *reinterpret_cast<uint4*>(cache + (size_t)r * ld + 8 * c) = __ldcg(reinterpret_cast<const uint4*>(s) + c);
+        }
     }
     __syncthreads();
 
-    const int tiles = stream_rows<PHASE>(H, L, F) / 16;
-    const int n_items = stream_items<PHASE>(p, sh);
-    const int i0 = chunk_begin(blockIdx.x, n_items, gridDim.x);
-    const int i1 = chunk_begin(blockIdx.x + 1, n_items, gridDim.x);
-    using SP = SlotPlan<PHASE, FMT>;
-    const int abytes = SP::a_bytes(p), sbytes = SP::s_bytes(p);
-    // the item's activations follow its weights, 128-byte aligned (slots are);
-    // in U a slot may instead hold 16 shared-expert rows (16 x Fs bf16)
-    const int wbytes = (PHASE == SP_GATEUP ? 2 : 1) * (abytes + sbytes);
-    const int act_off = ((PHASE == SP_UPROJ ? max(wbytes, 32 * Fs) : wbytes) + 127) & ~127;
-    // reduction length and activation row stride (halves) inside a slot / the CTA buffer
-    const int KR = PHASE == SP_DPROJ ? H : PHASE == SP_GATEUP ? L : PHASE == SP_DOWN ? F : L;
-    const int ld = (PHASE == SP_DOWN) ? F : KR + kActPad;
-
-    if (warp == kSW) {
-        // ---------------------------------------------------------------- loader
-        if (lane == 0) {
-            uint32_t last_ph[kMaxSlots];
-            for (int s = 0; s < kMaxSlots; ++s) last_ph[s] = 0xFFFFFFFFu;
-            bool x_issued = false;
-            if (PHASE == SP_DPROJ && i0 < i1) {
-                mbar_arrive_expect_tx(&xbar, (uint32_t)T * H * 2);
-                for (int t = 0; t < T; ++t)
-                    asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
-                                 ::"r"(smem_u32(smem + (size_t)t * (H + kActPad) * 2)), "l"(p.x16 + (size_t)t * H),
-                                 "r"(H * 2), "r"(smem_u32(&xbar)) : "memory");
-                x_issued = true;
-            }
-            // Copies of item i into slot s: the weights (which depend on the
-            // routing only) and / or the activations (written by the
-            // previous kernel).
-            auto issue = [&](int i, int s, bool weights, bool acts) {
-                const Item item = stream_item<PHASE>(sh, tiles, i);
-                uint8_t* slot = slots + (size_t)s * slot_bytes;
-                uint8_t* act = slot + act_off;
-                SlotMeta& m = meta[s];
-                auto bulk = [&](void* dst, const void* src, uint32_t nb) {
-                    asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
-                                 ::"r"(smem_u32(dst)), "l"(src), "r"(nb), "r"(smem_u32(&full[s])) : "memory");
-                };
-                auto tma3 = [&](void* dst, const CUtensorMap* mp, int c0, int c2) {
-                    asm volatile(
-                        "cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes "
-                        "[%0], [%1, {%3, %4, %5}], [%2];"
-                        ::"r"(smem_u32(dst)), "l"(mp), "r"(smem_u32(&full[s])), "r"(c0), "r"(0), "r"(c2)
-                        : "memory");
-                };
-                int nact = T;
-                if (PHASE == SP_GATEUP || PHASE == SP_DOWN) nact = sh.ucnt[item.j];
-                if (weights) {
-                    m.item = item;
-                    m.nt = nact;
-                    m.off = (PHASE == SP_GATEUP || PHASE == SP_DOWN) ? sh.uoff[item.j] : 0;
-                    // one expect-tx for everything the slot will receive
-                    uint32_t bytes;
-                    if (PHASE == SP_UPROJ && item.kind == 1) bytes = 16 * Fs * 2 + T * Fs * 2;
-                    else if (PHASE == SP_GATEUP) bytes = wbytes + 16 + nact * L * 2;
-                    else if (PHASE == SP_DOWN) bytes = wbytes + 16 + nact * F * 2;
-                    else if (PHASE == SP_UPROJ) bytes = wbytes + T * L * 2;
-                    else bytes = wbytes;
-                    mbar_arrive_expect_tx(&full[s], bytes);
-                    if (PHASE == SP_UPROJ && item.kind == 1) {
-                        bulk(slot, p.sd + (size_t)item.r0 * Fs, 16 * Fs * 2);
-                    } else {
-                        const int cq = item.r0 * maps.q_row, cs = item.r0 * maps.s_row;
-                        tma3(slot, &maps.wq, cq, item.mat);
-                        tma3(slot + abytes, &maps.ws, cs, item.mat);
-                        if (PHASE == SP_GATEUP || PHASE == SP_DOWN) {
-                            const size_t nq = (size_t)L * F / 2, ns = (size_t)L * F / 16;
-                            bulk(m.tail, p.experts + (size_t)item.mat * p.rec_bytes + 3 * nq + 3 * ns, 16);
-                        }
-                        if (PHASE == SP_GATEUP) {
-                            tma3(slot + abytes + sbytes, &maps.wq2, cq, item.mat);
-                            tma3(slot + 2 * abytes + sbytes, &maps.ws2, cs, item.mat);
-                        }
-                    }
-                }
-                if (acts) {
-                    if (PHASE == SP_UPROJ && item.kind == 1) {
-                        bulk(act, p.zsh16, T * Fs * 2);
-                    } else if (PHASE == SP_GATEUP) {
-                        const int off = sh.uoff[item.j], g = sh.ugrp[item.j];
-                        for (int c = 0; c < nact; ++c)
-                            bulk(act + (size_t)c * ld * 2, p.h16 + ((size_t)sh.slot_tok[off + c] * G + g) * L, L * 2);
-                    } else if (PHASE == SP_DOWN) {
-                        bulk(act, p.z16 + (size_t)sh.uoff[item.j] * F, nact * F * 2);
-                    } else if (PHASE == SP_UPROJ) {
-                        for (int t = 0; t < T; ++t)
-                            bulk(act + (size_t)t * ld * 2, p.s16 + ((size_t)t * G + item.mat) * L, L * 2);
-                    }
-                }
-            };
-            // the first ring's worth of weights streams before the previous
-            // kernel has finished
-            const int n_pre = PHASE == SP_DPROJ ? 0 : min(n_slots, i1 - i0);
-            for (int k = 0; k < n_pre; ++k) {
-                issue(i0 + k, k, true, false);
-                last_ph[k] = 0;
-            }
-            if (PHASE != SP_DPROJ) {
-                grid_dep_wait();
-                grid_dep_launch();
-            }
-            for (int k = 0; k < n_pre; ++k) issue(i0 + k, k, false, true);
-            int it = n_pre;
-            for (int i = i0 + n_pre; i < i1; ++i, ++it) {
-                const int s = it % n_slots;
-                const uint32_t ph = (it / n_slots) & 1;
-                if (!mbar_wait(&empty[s], ph ^ 1, &abort_flag, kStreamWait)) break;
-                issue(i, s, true, true);
-                last_ph[s] = ph;
-            }
-            if (abort_flag) {
-                // let every copy already issued land before the CTA can leave
-                int dummy = 0;
-                for (int s = 0; s < n_slots; ++s)
-                    if (last_ph[s] != 0xFFFFFFFFu) mbar_wait(&full[s], last_ph[s], &dummy, kStreamWait);
-                if (x_issued) mbar_wait(&xbar, 0, &dummy, kStreamWait);
-            }
-        }
+    // ---- the warp's items: stream, multiply, finish
+    int ci = i0 + warp, cs = 0, c_nsteps = 0, n_done = 0;
+    WItem cit = none;
+    if (ci < i1) {
+        cit = decode_item<PHASE, FMT>(p, sh, plan, ci);
+        c_nsteps = n_steps<PHASE>(cit, step_blocks<PHASE, FMT>(PHASE == SP_UPROJ && cit.mat < 0));
+    }
+    float a[4] = {0.f, 0.f, 0.f, 0.f}, u[4] = {0.f, 0.f, 0.f, 0.f};
+    const int gg = lane >> 2, tt = lane & 3;
+    while (ci < i1) {
+        if (li < i1) issue_step<PHASE, FMT>(p, lit, ls, ring + (size_t)(n_issued % kPD) * kStepBytes, lane);
+        cp_async_commit();
+        ++n_issued;
+        advance_load();
+        cp_async_wait<kPD - 1>();
         __syncwarp();
-    } else if (warp < kSW) {
-        // ---------------------------------------------------------------- compute warps
-        if (PHASE != SP_DPROJ) {
-            grid_dep_wait();
-            grid_dep_launch();
+        // activations of the item
+        const int jj = cit.j - c_m0;
+        const __half* xs;
+        int nt = T;
+        if (PHASE == SP_DPROJ) xs = cache;
+        else if (PHASE == SP_UPROJ) xs = cache + (size_t)c_row0[jj] * ld;
+        else {
+            xs = cache + (size_t)c_row0[jj] * ld;
+            nt = sh.ucnt[cit.j];
         }
-        if (PHASE == SP_DPROJ && i0 < i1 && !mbar_wait(&xbar, 0, &abort_flag, kStreamWait)) goto done;
-        {
-            int it = 0;
-            for (int i = i0; i < i1; ++i, ++it) {
-                const int s = it % n_slots;
-                const uint32_t ph = (it / n_slots) & 1;
-                if (!mbar_wait(&full[s], ph, &abort_flag, kStreamWait)) break;
-                const SlotMeta m = meta[s];
-                const uint8_t* slot = slots + (size_t)s * slot_bytes;
-                const uint8_t* act = slot + act_off;
-                const __half* xs = PHASE == SP_DPROJ ? reinterpret_cast<const __half*>(smem) : reinterpret_cast<const __half*>(act);
-                const int nt = m.nt;
-                float a[4] = {0.f, 0.f, 0.f, 0.f}, u[4] = {0.f, 0.f, 0.f, 0.f};
-                if (PHASE == SP_DPROJ || (PHASE == SP_UPROJ && m.item.kind == 0)) {
-                    const int nb = KR / 32, per = (nb + kSW - 1) / kSW;
-                    tile_du<FMT>(slot, reinterpret_cast<const uint16_t*>(slot + abytes), xs, ld, nt, warp * per,
-                                 min(nb, (warp + 1) * per), a);
-                } else if (PHASE == SP_UPROJ) {
-                    const int nb = Fs / 32, per = (nb + kSW - 1) / kSW;
-                    tile_bf16(reinterpret_cast<const uint16_t*>(slot), Fs, xs, Fs, nt, warp * per,
-                              min(nb, (warp + 1) * per), a);
-                } else {
-                    const int nc = KR / 32, per = (nc + kSW - 1) / kSW;
-                    tile_nvfp4(slot, slot + abytes, xs, ld, nt, warp * per, min(nc, (warp + 1) * per), a);
-                    if (PHASE == SP_GATEUP)
-                        tile_nvfp4(slot + abytes + sbytes, slot + 2 * abytes + sbytes, xs, ld, nt, warp * per,
-                                   min(nc, (warp + 1) * per), u);
+        compute_step<PHASE, FMT>(p, cit, cs, ring + (size_t)(n_done % kPD) * kStepBytes, xs, ld, nt, a, u);
+        __syncwarp();
+        ++n_done;
+        if (++cs < c_nsteps) continue;
+
+        // ---- the item is complete: epilogue or partial
+        const int nparts = PHASE == SP_UPROJ ? plan.n_mats * plan.ks : plan.ks;
+        bool finish = nparts == 1;
+        int tick_base = 0, part = 0;
+        if (!finish) {
+            // partial of part (j, q) of tile (mat, tile); U: all matrices are parts of one tile
+            const int key = PHASE == SP_UPROJ ? cit.tile : cit.j * plan.tiles + cit.tile;
+            part = PHASE == SP_UPROJ ? cit.j * plan.ks + cit.q : cit.q;
+            tick_base = key;
+            float* dst = p.wpart + (((size_t)key * nparts + part) * 32 + lane) * 8;
+            *reinterpret_cast<float4*>(dst) = make_float4(a[0], a[1], a[2], a[3]);
+            if (PHASE == SP_GATEUP) *reinterpret_cast<float4*>(dst + 4) = make_float4(u[0], u[1], u[2], u[3]);
+            __threadfence();
+            __syncwarp();
+            int last = 0;
+            if (lane == 0) last = atomicAdd(p.wtick + key, 1) == nparts - 1;
+            last = __shfl_sync(0xffffffffu, last, 0);
+            if (last) {
+                __threadfence();
+                float sa[4] = {0.f, 0.f, 0.f, 0.f}, su[4] = {0.f, 0.f, 0.f, 0.f};
+                for (int q = 0; q < nparts; ++q) {
+                    const float* s = p.wpart + (((size_t)key * nparts + q) * 32 + lane) * 8;
+                    const float4 v = __ldcg(reinterpret_cast<const float4*>(s));
+                    sa[0] += v.x; sa[1] += v.y; sa[2] += v.z; sa[3] += v.w;
+                    if (PHASE == SP_GATEUP) {
+                        const float4 w4 = __ldcg(reinterpret_cast<const float4*>(s + 4));
+                        su[0] += w4.x; su[1] += w4.y; su[2] += w4.z; su[3] += w4.w;
+                    }
                 }
-                // every read of the slot is complete (the values are in registers)
-                __syncwarp();
-                if (lane == 0) mbar_arrive(&empty[s]);
-                const int b = it & 1;
-                if (!mbar_wait(&red_empty[b], ((it >> 1) & 1) ^ 1, &abort_flag, kStreamWait)) break;
 #pragma unroll
-                for (int i4 = 0; i4 < 4; ++i4) {
-                    red[b][warp][lane][i4] = a[i4];
-                    if (NV == 8) red[b][warp][lane][(4 + i4) % NV] = u[i4];
-                }
-                if (warp == 0 && lane == 0) red_meta[b] = m;
-                __syncwarp();
-                if (lane == 0) mbar_arrive(&red_full[b]);
+                for (int i4 = 0; i4 < 4; ++i4) { a[i4] = sa[i4]; u[i4] = su[i4]; }
+                if (lane == 0) p.wtick[key] = 0;
+                finish = true;
             }
         }
-    } else {
-        // ---------------------------------------------------------------- reducer + epilogue
-        if (PHASE != SP_DPROJ) {
-            grid_dep_wait();
-            grid_dep_launch();
-        }
-        const int gg = lane >> 2, tt = lane & 3;
-        float yacc[4] = {0.f, 0.f, 0.f, 0.f};   // U: running sum over the parts of one output tile
-        int seg_first = -1;                      // U: first part of the current run in this CTA
-        int it = 0;
-        for (int i = i0; i < i1; ++i, ++it) {
-            const int b = it & 1;
-            if (!mbar_wait(&red_full[b], (it >> 1) & 1, &abort_flag, kStreamWait)) break;
-            float a[4], u[4];
+        if (finish) {
+            const float* ts = (PHASE == SP_GATEUP || PHASE == SP_DOWN) ? c_tail[jj] : nullptr;
 #pragma unroll
             for (int i4 = 0; i4 < 4; ++i4) {
-                float sa = 0.f, su = 0.f;
-#pragma unroll
-                for (int w = 0; w < kSW; ++w) {
-                    sa += red[b][w][lane][i4];
-                    if (NV == 8) su += red[b][w][lane][(4 + i4) % NV];
-                }
-                a[i4] = sa;
-                u[i4] = su;
-            }
-            const SlotMeta m = red_meta[b];
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&red_empty[b]);
-            const Item item = m.item;
-            const int nt = m.nt;
-            if (PHASE != SP_UPROJ) {
-#pragma unroll
-                for (int i4 = 0; i4 < 4; ++i4) {
-                    const int col = 2 * tt + (i4 & 1), row = item.r0 + gg + 8 * (i4 >> 1);
-                    if (col >= nt) continue;
-                    if (PHASE == SP_DPROJ) {
-                        p.h16[((size_t)col * G + item.mat) * L + row] = __float2half_rn(a[i4]);
-                    } else if (PHASE == SP_GATEUP) {
-                        p.z16[(size_t)(m.off + col) * F + row] =
-                            __float2half_rn(silu(a[i4] * m.tail[0]) * (u[i4] * m.tail[1]));
-                    } else {
-                        p.o16w[(size_t)(m.off + col) * L + row] =
-                            __float2half_rn(sh.slot_w[m.off + col] * m.tail[2] * a[i4]);
-                    }
-                }
-                continue;
-            }
-            // U: accumulate the parts of this tile that run consecutively here
-            const int parts = sh.n_hit + 1;
-            if (seg_first < 0) seg_first = item.j;
-#pragma unroll
-            for (int i4 = 0; i4 < 4; ++i4) yacc[i4] += a[i4];
-            const bool tile_end = item.j == parts - 1;
-            if (!tile_end && i + 1 < i1) continue;
-            const int tile = item.r0 / 16;
-            const bool whole = seg_first == 0 && tile_end;
-            if (whole) {
-#pragma unroll
-                for (int i4 = 0; i4 < 4; ++i4) {
-                    const int col = 2 * tt + (i4 & 1), row = item.r0 + gg + 8 * (i4 >> 1);
-                    if (col >= T) continue;
-                    float v = yacc[i4];
+                const int col = 2 * tt + (i4 & 1), row = cit.r0 + gg + 8 * (i4 >> 1);
+                if (col >= nt) continue;
+                if (PHASE == SP_DPROJ) {
+                    p.h16[((size_t)col * G + cit.mat) * L + row] = __float2half_rn(a[i4]);
+                } else if (PHASE == SP_GATEUP) {
+                    p.z16[(size_t)(sh.uoff[cit.j] + col) * F + row] = __float2half_rn(silu(a[i4] * ts[0]) * (u[i4] * ts[1]));
+                } else if (PHASE == SP_DOWN) {
+                    const int slot = sh.uoff[cit.j] + col;
+                    p.o16w[(size_t)slot * L + row] = __float2half_rn(sh.slot_w[slot] * ts[2] * a[i4]);
+                } else {
+                    float v = a[i4];
                     if (p.residual) v += bf16_bits_to_f32(p.residual[(size_t)col * H + row]);
                     p.y[(size_t)col * H + row] = f32_to_bf16_bits(v);
                 }
-            } else {
-                // this CTA holds parts [seg_first, item.j] of the tile: park
-                // the partial sum under its first part; the CTA completing
-                // the tile's parts adds the partials in part order
-#pragma unroll
-                for (int i4 = 0; i4 < 4; ++i4) {
-                    const int col = 2 * tt + (i4 & 1), row = item.r0 + gg + 8 * (i4 >> 1);
-                    if (col < T) p.ypart[((size_t)seg_first * T + col) * H + row] = yacc[i4];
-                }
-                __threadfence();
-                __syncwarp();
-                int last = 0;
-                if (lane == 0) {
-                    const int n_mine = item.j - seg_first + 1;
-                    last = atomicAdd(&p.ctrl->tile_ticket[tile], n_mine) + n_mine == parts;
-                }
-                last = __shfl_sync(0xffffffffu, last, 0);
-                if (last) {
-                    __threadfence();
-                    const int base = tile * parts;
-                    for (int e2 = lane; e2 < T * 16; e2 += 32) {
-                        const int t = e2 >> 4, row = item.r0 + (e2 & 15);
-                        float v = 0.f;
-                        for (int q = 0; q < parts; ++q) {
-                            // q starts a run iff it starts the tile or some CTA's chunk
-                            const int gi = base + q;
-                            const int c = (int)(((long long)gi * gridDim.x + n_items - 1) / n_items);
-                            if (q == 0 || chunk_begin(c, n_items, gridDim.x) == gi)
-                                v += __ldcg(p.ypart + ((size_t)q * T + t) * H + row);
-                        }
-                        if (p.residual) v += bf16_bits_to_f32(p.residual[(size_t)t * H + row]);
-                        p.y[(size_t)t * H + row] = f32_to_bf16_bits(v);
-                    }
-                    if (lane == 0) p.ctrl->tile_ticket[tile] = 0;
-                }
             }
+        }
 #pragma unroll
-            for (int i4 = 0; i4 < 4; ++i4) yacc[i4] = 0.f;
-            seg_first = -1;
+        for (int i4 = 0; i4 < 4; ++i4) { a[i4] = 0.f; u[i4] = 0.f; }
+        cs = 0;
+        ci += kWW;
+        if (ci < i1) {
+            cit = decode_item<PHASE, FMT>(p, sh, plan, ci);
+            c_nsteps = n_steps<PHASE>(cit, step_blocks<PHASE, FMT>(PHASE == SP_UPROJ && cit.mat < 0));
         }
     }
-done:
-    __syncthreads();
-    if (abort_flag && threadIdx.x == 0) set_status(p.ctrl, LMOE_ERR_TIMEOUT);
+    cp_async_wait<0>();
 }
 
-// s16[t][g] = sum over the token's experts of group g of o16w (zero if none)
+// s16[g][t] = sum over the token's experts of group g of o16w (zero if none)
 __global__ void k_combine_small(FwdParams p) {
     const int t = blockIdx.y, g = blockIdx.x;
     const int L = p.L, K = p.K;
@@ -655,44 +629,13 @@ __global__ void k_combine_small(FwdParams p) {
         __half2 h[4];
 #pragma unroll
         for (int j = 0; j < 4; ++j) h[j] = __floats2half2_rn(acc[2 * j], acc[2 * j + 1]);
-        reinterpret_cast<uint4*>(p.s16 + ((size_t)t * p.G + g) * L)[c8] = *reinterpret_cast<uint4*>(h);
+        reinterpret_cast<uint4*>(p.s16 + ((size_t)g * p.T + t) * L)[c8] = *reinterpret_cast<uint4*>(h);
     }
 }
 
 // ---------------------------------------------------------------------------
-// host side
+// launch helpers
 // ---------------------------------------------------------------------------
-
-typedef CUresult (*EncodeFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
-                             const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
-                             CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
-
-static EncodeFn encode() {
-    static EncodeFn fn = nullptr;
-    if (!fn) {
-        void* ptr = nullptr;
-        cudaDriverEntryPointQueryResult q;
-        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) == cudaSuccess &&
-            q == cudaDriverEntryPointSuccess)
-            fn = reinterpret_cast<EncodeFn>(ptr);
-    }
-    return fn;
-}
-
-// 3-D tensor of 16-bit units: (row_u16 * rows: one K block, contiguous;
-// blocks; matrices), strides in bytes; the box is (row_u16 * 16, blocks, 1).
-static bool map3(CUtensorMap* m, const void* base, uint64_t row_u16, uint64_t rows, uint64_t blocks,
-                 uint64_t mats, uint64_t s_blk, uint64_t s_mat) {
-    EncodeFn fn = encode();
-    if (!fn || row_u16 * 16 > 256 || blocks > 256) return false;
-    cuuint64_t dims[3] = {row_u16 * rows, blocks, mats};
-    cuuint64_t strides[2] = {s_blk, s_mat};
-    cuuint32_t box[3] = {(cuuint32_t)(row_u16 * 16), (cuuint32_t)blocks, 1};
-    cuuint32_t es[3] = {1, 1, 1};
-    return fn(m, CU_TENSOR_MAP_DATA_TYPE_UINT16, 3, const_cast<void*>(base), dims, strides, box, es,
-              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
-}
 
 static int g_sms = 0;
 
@@ -715,24 +658,72 @@ static cudaError_t launch_dependent(Kern kern, dim3 grid, dim3 block, size_t sme
     return cudaLaunchKernelEx(&cfg, kern, args...);
 }
 
+
+// ---------------------------------------------------------------------------
+// host side
+// ---------------------------------------------------------------------------
+
+// Reduction parts per tile of each phase: enough items for about one per
+// warp of the GPU (148 SMs x 16 warps) counting every matrix that may be
+// hit, without a part smaller than one step.
+struct WPlans {
+    WPlan d, gu, dn, u;
+    size_t part_floats, ticks;
+};
+
 template <int PHASE, int FMT>
-static cudaError_t launch_stream(const StreamMaps& maps, const FwdParams& p, cudaStream_t st, int slot_bytes,
-                                 int xs_bytes) {
-    // dynamic shared memory: what the device allows per block minus the kernel's static part
-    static size_t budget = 0;   // per kernel instance
-    if (!budget) {
-        cudaFuncAttributes fa;
-        int dev = 0, optin = 0;
-        cudaError_t e0 = cudaFuncGetAttributes(&fa, reinterpret_cast<const void*>(k_stream<PHASE, FMT>));
-        if (e0 == cudaSuccess) e0 = cudaGetDevice(&dev);
-        if (e0 == cudaSuccess) e0 = cudaDeviceGetAttribute(&optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev);
-        if (e0 != cudaSuccess) return e0;
-        budget = (size_t)optin - fa.sharedSizeBytes - 1024;
+static WPlan plan_for(int H, int L, int F, int Fs, int G, int n_mats_max) {
+    WPlan w;
+    w.tiles = stream_rows<PHASE>(H, L, F) / 16;
+    w.n_mats = n_mats_max;
+    const int nb = PHASE == SP_DPROJ ? H / 32 : PHASE == SP_GATEUP ? L / 32 : PHASE == SP_DOWN ? F / 32 : L / 32;
+    int max_ks = (nb + step_blocks<PHASE, FMT>(false) - 1) / step_blocks<PHASE, FMT>(false);
+    if (PHASE == SP_UPROJ) max_ks = std::min(max_ks, (Fs / 32 + 1) / 2);
+    const int base = std::max(1, n_mats_max * w.tiles);
+    const int want = (148 * kWW + base - 1) / base;
+    w.ks = std::max(1, std::min({want, max_ks, 8}));
+    (void)G;
+    return w;
+}
+
+WPlans stream_plans(int H, int L, int F, int Fs, int G, int E, int K, int T, int du_fmt) {
+    WPlans P;
+    const int nu = std::min(T * K, E);
+    if (du_fmt == LMOE_Q8_0) {
+        P.d = plan_for<SP_DPROJ, LMOE_Q8_0>(H, L, F, Fs, G, G);
+        P.u = plan_for<SP_UPROJ, LMOE_Q8_0>(H, L, F, Fs, G, G + 1);
+    } else {
+        P.d = plan_for<SP_DPROJ, LMOE_Q4_0>(H, L, F, Fs, G, G);
+        P.u = plan_for<SP_UPROJ, LMOE_Q4_0>(H, L, F, Fs, G, G + 1);
     }
-    const int n_slots = (int)std::min<size_t>(16, (budget - xs_bytes) / slot_bytes);
-    if (n_slots < 2) return cudaErrorInvalidValue;
-    const size_t smem = 128 + xs_bytes + (size_t)n_slots * slot_bytes;
-    auto kern = k_stream<PHASE, FMT>;
+    P.gu = plan_for<SP_GATEUP, LMOE_Q8_0>(H, L, F, Fs, G, nu);
+    P.dn = plan_for<SP_DOWN, LMOE_Q8_0>(H, L, F, Fs, G, nu);
+    // partials (8 floats per lane, 32 lanes) and tickets, the largest phase
+    auto parts = [](const WPlan& w, bool all_parts_per_tile) {
+        return (size_t)w.n_mats * w.tiles * w.ks * (all_parts_per_tile ? 1 : 1);
+    };
+    P.part_floats = 256 * std::max({parts(P.d, false), parts(P.gu, false), parts(P.dn, false), parts(P.u, true)});
+    P.ticks = std::max({(size_t)P.d.n_mats * P.d.tiles, (size_t)P.gu.n_mats * P.gu.tiles, (size_t)P.dn.n_mats * P.dn.tiles,
+                        (size_t)P.u.tiles});
+    return P;
+}
+
+size_t stream_ws_part_bytes(int H, int L, int F, int Fs, int G, int E, int K, int T, int du_fmt) {
+    return stream_plans(H, L, F, Fs, G, E, K, T, du_fmt).part_floats * sizeof(float);
+}
+size_t stream_ws_tick_bytes(int H, int L, int F, int Fs, int G, int E, int K, int T, int du_fmt) {
+    return stream_plans(H, L, F, Fs, G, E, K, T, du_fmt).ticks * sizeof(int);
+}
+
+template <int PHASE, int FMT>
+static cudaError_t launch_wstream(const FwdParams& p, const WPlan& plan, int cache_rows, cudaStream_t st) {
+    const int ld = PHASE == SP_DPROJ ? p.H + kActPad
+                 : PHASE == SP_GATEUP ? p.L + kActPad
+                 : PHASE == SP_DOWN ? p.F + kActPad
+                                    : std::max(p.L, p.Fs) + kActPad;
+    const int cache_bytes = round128(cache_rows * ld * 2);
+    const size_t smem = 128 + (size_t)cache_bytes + (size_t)kWW * kPD * kStepBytes;
+    auto kern = k_wstream<PHASE, FMT>;
     cudaError_t e = ensure_smem(reinterpret_cast<const void*>(kern), smem);
     if (e != cudaSuccess) return e;
     if (!g_sms) {
@@ -741,115 +732,36 @@ static cudaError_t launch_stream(const StreamMaps& maps, const FwdParams& p, cud
         cudaDeviceGetAttribute(&g_sms, cudaDevAttrMultiProcessorCount, dev);
     }
     stage_mark(st);
-    return launch_dependent(kern, dim3(g_sms), dim3(kStreamThreads), smem, st, maps, p, n_slots, slot_bytes);
-}
-
-
-
-struct StreamMapSet {
-    StreamMaps d, gu, dn, u;
-};
-
-// Encode the four phases' tensor maps of one layer's weights.
-static bool encode_stream_maps(const FwdParams& p, StreamMapSet* out) {
-    const int H = p.H, L = p.L, F = p.F, G = p.G, E = p.E;
-    const size_t qb = p.du_fmt == LMOE_Q8_0 ? 32 : 16;
-    const size_t nq = (size_t)L * F / 2, ns = (size_t)L * F / 16;
-    const uint8_t* ex = p.experts;
-    StreamMaps& md = out->d;
-    StreamMaps& mgu = out->gu;
-    StreamMaps& mdn = out->dn;
-    StreamMaps& mu = out->u;
-    std::memset(out, 0, sizeof(*out));
-    bool ok = true;
-    const int qr = (int)qb / 2;
-    // D: q [H/32][L][qb] + d [H/32][L] fp16 per group
-    ok &= map3(&md.wq, p.D, qr, L, H / 32, G, (uint64_t)L * qb, p.du_bytes_D);
-    ok &= map3(&md.ws, p.D + (size_t)L * H / 32 * qb, 1, L, H / 32, G, (uint64_t)L * 2, p.du_bytes_D);
-    md.q_row = qr; md.s_row = 1;
-    // U: q [L/32][H][qb] + d [L/32][H]; the shared expert's down rows are plain copies
-    ok &= map3(&mu.wq, p.U, qr, H, L / 32, G, (uint64_t)H * qb, p.du_bytes_U);
-    ok &= map3(&mu.ws, p.U + (size_t)H * L / 32 * qb, 1, H, L / 32, G, (uint64_t)H * 2, p.du_bytes_U);
-    mu.q_row = qr; mu.s_row = 1;
-    // experts: gate/up q [L/32][F][16], s [L/64][F][4]; down q [F/32][L][16], s [F/64][L][4]
-    ok &= map3(&mgu.wq, ex, 8, F, L / 32, E, (uint64_t)F * 16, p.rec_bytes);
-    ok &= map3(&mgu.wq2, ex + nq, 8, F, L / 32, E, (uint64_t)F * 16, p.rec_bytes);
-    ok &= map3(&mgu.ws, ex + 3 * nq, 2, F, L / 64, E, (uint64_t)F * 4, p.rec_bytes);
-    ok &= map3(&mgu.ws2, ex + 3 * nq + ns, 2, F, L / 64, E, (uint64_t)F * 4, p.rec_bytes);
-    mgu.q_row = 8; mgu.s_row = 2;
-    ok &= map3(&mdn.wq, ex + 2 * nq, 8, L, F / 32, E, (uint64_t)L * 16, p.rec_bytes);
-    ok &= map3(&mdn.ws, ex + 3 * nq + 2 * ns, 2, L, F / 64, E, (uint64_t)L * 4, p.rec_bytes);
-    mdn.q_row = 8; mdn.s_row = 2;
-    return ok;
-}
-
-// The maps depend only on the weight pointers and the shape, so each layer's
-// set is encoded once and kept (a small round-robin cache; a stack of layers
-// cycles through it).
-static bool stream_maps_for(const FwdParams& p, StreamMapSet* out) {
-    struct Key {
-        const void *D, *U, *ex;
-        int H, L, F, G, E, fmt;
-        size_t bd, bu, br;
-        bool operator==(const Key& o) const { return std::memcmp(this, &o, sizeof(Key)) == 0; }
-    };
-    constexpr int kCache = 64;
-    static Key keys[kCache];
-    static StreamMapSet sets[kCache];
-    static int n = 0, next = 0;
-    static std::mutex mu;
-    Key k;
-    std::memset(&k, 0, sizeof(k));
-    k.D = p.D; k.U = p.U; k.ex = p.experts;
-    k.H = p.H; k.L = p.L; k.F = p.F; k.G = p.G; k.E = p.E; k.fmt = p.du_fmt;
-    k.bd = p.du_bytes_D; k.bu = p.du_bytes_U; k.br = p.rec_bytes;
-    std::lock_guard<std::mutex> lock(mu);
-    for (int i = 0; i < n; ++i)
-        if (keys[i] == k) {
-            *out = sets[i];
-            return true;
-        }
-    if (!encode_stream_maps(p, out)) return false;
-    keys[next] = k;
-    sets[next] = *out;
-    next = (next + 1) % kCache;
-    if (n < kCache) ++n;
-    return true;
+    return launch_dependent(kern, dim3(g_sms), dim3(kWThreads), smem, st, p, plan, cache_bytes);
 }
 
 // D, experts, combine, U for T <= 8 (the router kernel has run).
 cudaError_t run_stream_path(const FwdParams& p, cudaStream_t st) {
-    const int H = p.H, L = p.L, F = p.F, Fs = p.Fs, G = p.G;
-    const size_t qb = p.du_fmt == LMOE_Q8_0 ? 32 : 16;
-    StreamMapSet ms;
-    if (!stream_maps_for(p, &ms)) return cudaErrorInvalidValue;
-    const StreamMaps& md = ms.d;
-    const StreamMaps& mgu = ms.gu;
-    const StreamMaps& mdn = ms.dn;
-    const StreamMaps& mu = ms.u;
-
-    const int act_d = 0;
-    const int slot_d = round128(16 * H * (int)qb / 32 + 16 * (H / 32) * 2);
-    // activation rows per slot: at most T (an expert sees each token once)
-    const int T = p.T;
-    const int slot_gu = round128(round128(2 * (16 * L / 2 + 16 * (L / 64) * 4)) + T * (L + kActPad) * 2);
-    const int slot_dn = round128(round128(16 * F / 2 + 16 * (F / 64) * 4) + T * F * 2);
-    const int slot_u = round128(round128(std::max(16 * L * (int)qb / 32 + 16 * (L / 32) * 2, 32 * Fs)) +
-                                T * std::max(L + kActPad, Fs) * 2);
-    (void)act_d;
-    cudaError_t e;
-    const int xs_d = round128(T * (H + kActPad) * 2);
-    e = p.du_fmt == LMOE_Q8_0 ? launch_stream<SP_DPROJ, LMOE_Q8_0>(md, p, st, slot_d, xs_d)
-                              : launch_stream<SP_DPROJ, LMOE_Q4_0>(md, p, st, slot_d, xs_d);
+    const int H = p.H, L = p.L, F = p.F, Fs = p.Fs, G = p.G, T = p.T;
+    const WPlans P = stream_plans(H, L, F, Fs, G, p.E, p.K, T, p.du_fmt);
+    if (!g_sms) {
+        int dev = 0;
+        cudaGetDevice(&dev);
+        cudaDeviceGetAttribute(&g_sms, cudaDevAttrMultiProcessorCount, dev);
+    }
+    // cache rows: the distinct matrices one CTA's contiguous chunk can span, T rows each
+    auto chunk_rows = [&](const WPlan& w) {
+        const int per_mat = w.tiles * w.ks;
+        const int chunk = (w.n_mats * per_mat + g_sms - 1) / g_sms;
+        const int mats = std::min(w.n_mats, (chunk + per_mat - 1) / per_mat + 1);
+        return std::min(mats, kMaxChunkParts) * T;
+    };
+    cudaError_t e = p.du_fmt == LMOE_Q8_0 ? launch_wstream<SP_DPROJ, LMOE_Q8_0>(p, P.d, T, st)
+                              : launch_wstream<SP_DPROJ, LMOE_Q4_0>(p, P.d, T, st);
     if (e != cudaSuccess) return e;
-    e = launch_stream<SP_GATEUP, LMOE_Q8_0>(mgu, p, st, slot_gu, 0);
+    e = launch_wstream<SP_GATEUP, LMOE_Q8_0>(p, P.gu, chunk_rows(P.gu), st);
     if (e != cudaSuccess) return e;
-    e = launch_stream<SP_DOWN, LMOE_Q8_0>(mdn, p, st, slot_dn, 0);
+    e = launch_wstream<SP_DOWN, LMOE_Q8_0>(p, P.dn, chunk_rows(P.dn), st);
     if (e != cudaSuccess) return e;
     stage_mark(st);
     if ((e = launch_dependent(k_combine_small, dim3(G, p.T), dim3(128), 0, st, p)) != cudaSuccess) return e;
-    e = p.du_fmt == LMOE_Q8_0 ? launch_stream<SP_UPROJ, LMOE_Q8_0>(mu, p, st, slot_u, 0)
-                              : launch_stream<SP_UPROJ, LMOE_Q4_0>(mu, p, st, slot_u, 0);
+    e = p.du_fmt == LMOE_Q8_0 ? launch_wstream<SP_UPROJ, LMOE_Q8_0>(p, P.u, chunk_rows(P.u), st)
+                              : launch_wstream<SP_UPROJ, LMOE_Q4_0>(p, P.u, chunk_rows(P.u), st);
     return e;
 }
 
