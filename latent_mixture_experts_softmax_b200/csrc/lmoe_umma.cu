@@ -210,49 +210,6 @@ __device__ __forceinline__ void bulk_g2s(void* dst, const void* src, uint32_t by
                  : "memory");
 }
 
-// Arm `bar` and copy the raw weights of the cursor's stage into `slot`.
-template <int KIND, int NT>
-__device__ __forceinline__ void issue_raw(const PrefillParams& p, const Cursor<KIND, NT>& c, uint8_t* slot,
-                                          uint64_t* bar) {
-    const int k0 = c.ks * 64;
-    const uint32_t pb = raw_part_bytes<KIND>(p.du_fmt);
-    if (KIND == G_DPROJ || (KIND == G_UPROJ && c.seg < p.G)) {
-        const int R = KIND == G_DPROJ ? p.L : p.H;
-        const int C = KIND == G_DPROJ ? p.H : p.L;
-        const uint8_t* mat = (KIND == G_DPROJ ? p.D : p.U) + (size_t)(KIND == G_DPROJ ? c.t.mat : c.seg) * p.du_bytes;
-        const size_t rowb = p.du_fmt == LMOE_Q8_0 ? 32 : 16;
-        const uint8_t* dsc = mat + (size_t)R * C / 32 * rowb;
-        const int kb = k0 / 32;
-        mbar_arrive_expect_tx(bar, 2 * pb + 512);
-        bulk_g2s(slot, mat + ((size_t)kb * R + c.t.m0) * rowb, pb, bar);
-        bulk_g2s(slot + pb, mat + ((size_t)(kb + 1) * R + c.t.m0) * rowb, pb, bar);
-        bulk_g2s(slot + 2 * pb, dsc + ((size_t)kb * R + c.t.m0) * 2, 256, bar);
-        bulk_g2s(slot + 2 * pb + 256, dsc + ((size_t)(kb + 1) * R + c.t.m0) * 2, 256, bar);
-    } else if (KIND == G_GATEUP) {
-        const size_t nq = (size_t)p.L * p.F / 2, ns = (size_t)p.L * p.F / 16;
-        const uint8_t* rec = p.experts + (size_t)c.t.mat * p.rec_bytes;
-        const int kc = k0 / 32, R = p.F;
-        mbar_arrive_expect_tx(bar, 2 * pb + 512);
-#pragma unroll
-        for (int j = 0; j < 2; ++j) {
-            bulk_g2s(slot + j * pb, rec + ((size_t)(kc + j) * R + c.t.m0) * 16, 1024, bar);             // gate
-            bulk_g2s(slot + j * pb + 1024, rec + nq + ((size_t)(kc + j) * R + c.t.m0) * 16, 1024, bar);  // up
-        }
-        bulk_g2s(slot + 2 * pb, rec + 3 * nq + ((size_t)(k0 / 64) * R + c.t.m0) * 4, 256, bar);
-        bulk_g2s(slot + 2 * pb + 256, rec + 3 * nq + ns + ((size_t)(k0 / 64) * R + c.t.m0) * 4, 256, bar);
-    } else if (KIND == G_DOWN) {
-        const size_t nq = (size_t)p.L * p.F / 2, ns = (size_t)p.L * p.F / 16;
-        const uint8_t* rec = p.experts + (size_t)c.t.mat * p.rec_bytes;
-        const int kc = k0 / 32, R = p.L;
-        mbar_arrive_expect_tx(bar, 2 * pb + 512);
-        bulk_g2s(slot, rec + 2 * nq + ((size_t)kc * R + c.t.m0) * 16, pb, bar);
-        bulk_g2s(slot + pb, rec + 2 * nq + ((size_t)(kc + 1) * R + c.t.m0) * 16, pb, bar);
-        bulk_g2s(slot + 2 * pb, rec + 3 * nq + 2 * ns + ((size_t)(k0 / 64) * R + c.t.m0) * 4, 512, bar);
-    } else {
-        mbar_arrive(bar);                          // nothing to copy for this stage
-    }
-}
-
 __device__ __forceinline__ uint32_t h2_bits(__half2 h) { return *reinterpret_cast<uint32_t*>(&h); }
 __device__ __forceinline__ __half2 bits_h2(uint32_t u) { return *reinterpret_cast<__half2*>(&u); }
 
@@ -262,17 +219,48 @@ __device__ __forceinline__ void bytes_to_h2x2(uint32_t w, uint32_t& lo, uint32_t
     hi = __byte_perm(w, 0x64646464u, 0x4342);
 }
 
-// Half h (columns 32h .. 32h+31) of row r of a raw slot -> 16 half2.
+// The stored bytes one converter thread dequantises for one stage: half h
+// (columns 32h .. 32h+31 of the 64-column stage) of row r of the tile.
+struct RawHalf {
+    uint4 a, b;      // codes (Q8_0: 32 bytes; Q4_0, NVFP4: 16 bytes in a)
+    uint32_t s;      // scale: fp16 bits (Q8_0, Q4_0) or the row's four E4M3 bytes of the 64 columns (NVFP4)
+};
+
+// Fetch RawHalf of (row r, half h) of the cursor's stage with plain loads
+// (read-only path; the bulk-copy engine's fixed cost per copy would cap a
+// per-stage stream of small copies).
+template <int KIND, int NT>
+__device__ __forceinline__ void fetch_raw(const PrefillParams& p, const Cursor<KIND, NT>& c, int r, int h, RawHalf& o) {
+    const int k0 = c.ks * 64;
+    if (KIND == G_DPROJ || (KIND == G_UPROJ && c.seg < p.G)) {
+        const int R = KIND == G_DPROJ ? p.L : p.H;
+        const int C = KIND == G_DPROJ ? p.H : p.L;
+        const uint8_t* mat = (KIND == G_DPROJ ? p.D : p.U) + (size_t)(KIND == G_DPROJ ? c.t.mat : c.seg) * p.du_bytes;
+        const size_t rowb = p.du_fmt == LMOE_Q8_0 ? 32 : 16;
+        const size_t e = (size_t)(k0 / 32 + h) * R + c.t.m0 + r;
+        const uint4* q = reinterpret_cast<const uint4*>(mat + e * rowb);
+        o.a = __ldg(q);
+        if (p.du_fmt == LMOE_Q8_0) o.b = __ldg(q + 1);
+        o.s = __ldg(reinterpret_cast<const uint16_t*>(mat + (size_t)R * C / 32 * rowb) + e);
+    } else if (KIND == G_GATEUP || KIND == G_DOWN) {
+        const size_t nq = (size_t)p.L * p.F / 2, ns = (size_t)p.L * p.F / 16;
+        const uint8_t* rec = p.experts + (size_t)c.t.mat * p.rec_bytes;
+        const int R = KIND == G_GATEUP ? p.F : p.L;
+        const int row = KIND == G_GATEUP ? c.t.m0 + (r & 63) : c.t.m0 + r;
+        const int m = KIND == G_GATEUP ? (r >> 6) : 2;                  // gate, up, down
+        o.a = __ldg(reinterpret_cast<const uint4*>(rec + (size_t)m * nq + ((size_t)(k0 / 32 + h) * R + row) * 16));
+        o.s = __ldg(reinterpret_cast<const uint32_t*>(rec + 3 * nq + (size_t)m * ns + ((size_t)(k0 / 64) * R + row) * 4));
+    }
+}
+
+// RawHalf of (row r, half h) -> 16 half2 of the row's 32 columns.
 template <int KIND>
-__device__ __forceinline__ void dequant_half(const PrefillParams& p, const uint8_t* slot, int r, int h,
-                                             uint32_t (&o)[16]) {
-    const int pb = raw_part_bytes<KIND>(p.du_fmt);
+__device__ __forceinline__ void dequant_half(const PrefillParams& p, const RawHalf& raw, int h, uint32_t (&o)[16]) {
     if (KIND == G_DPROJ || KIND == G_UPROJ) {
-        const uint16_t dbits = reinterpret_cast<const uint16_t*>(slot + 2 * pb)[128 * h + r];
-        const __half2 d = __half2half2(__ushort_as_half(dbits));
+        const __half2 d = __half2half2(__ushort_as_half((uint16_t)raw.s));
         if (p.du_fmt == LMOE_Q8_0) {
-            const uint4 a = *reinterpret_cast<const uint4*>(slot + h * pb + r * 32);
-            const uint4 b = *reinterpret_cast<const uint4*>(slot + h * pb + r * 32 + 16);
+            const uint4 a = raw.a;
+            const uint4 b = raw.b;
             const uint32_t w8[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
             const __half2 off = __float2half2_rn(1152.f);
 #pragma unroll
@@ -283,7 +271,7 @@ __device__ __forceinline__ void dequant_half(const PrefillParams& p, const uint8
                 o[2 * i + 1] = h2_bits(__hmul2(__hsub2(bits_h2(hi), off), d));
             }
         } else {
-            const uint4 a = *reinterpret_cast<const uint4*>(slot + h * pb + r * 16);
+            const uint4 a = raw.a;
             const uint32_t w4[4] = {a.x, a.y, a.z, a.w};
             const __half2 off = __float2half2_rn(1032.f);
 #pragma unroll
@@ -298,8 +286,8 @@ __device__ __forceinline__ void dequant_half(const PrefillParams& p, const uint8
             }
         }
     } else {
-        const uint4 a = *reinterpret_cast<const uint4*>(slot + h * pb + r * 16);
-        const uint32_t sw = reinterpret_cast<const uint32_t*>(slot + 2 * pb)[r];
+        const uint4 a = raw.a;
+        const uint32_t sw = raw.s;
         const uint32_t s16 = (sw >> (16 * h)) & 0xFFFF;          // scales of columns 32h..+15 and +16..+31
         uint32_t sc;
         asm("{\n\t.reg .b16 a;\n\tcvt.u16.u32 a, %1;\n\tcvt.rn.f16x2.e4m3x2 %0, a;\n\t}" : "=r"(sc) : "r"(s16));
@@ -434,6 +422,7 @@ struct SmemPlan {
 };
 
 constexpr int kConvWarps = 8;      // dequantising warps (half a weight row per thread)
+constexpr int kRawAhead = 4;       // stages whose stored weight bytes a converter thread holds
 constexpr int kGemmThreads = 448;  // 4 epilogue, 8 converter, 1 MMA, 1 loader warps
 
 template <int KIND, int NT, int STAGES, int RS>
@@ -493,28 +482,12 @@ __global__ void __launch_bounds__(kGemmThreads, 1) k_umma_gemm(const __grid_cons
         // ------------------------------------------------------------ loader (one thread)
         if (lane == 0) {
             tma_prefetch_desc(&maps.b);
-            Cursor<KIND, NT> cb, cr;       // activation / plain-weight stages, raw-weight stages
+            Cursor<KIND, NT> cb;           // activation / plain-weight stages
             cb.begin(p);
-            cr = cb;
-            uint32_t it_b = 0, it_r = 0;
+            uint32_t it_b = 0;
             uint32_t last_b[STAGES];
-            uint32_t last_r[RS];
             for (int i = 0; i < STAGES; ++i) last_b[i] = 0xFFFFFFFFu;
-            for (int i = 0; i < RS; ++i) last_r[i] = 0xFFFFFFFFu;
-            bool ok = true;
-            while (ok && !cb.done) {
-                // raw weights run up to RS stages ahead of the activation tiles
-                while (!cr.done && it_r < it_b + RS) {
-                    const int rs = it_r % RS;
-                    const uint32_t ph = (it_r / RS) & 1;
-                    if (!mbar_wait(&raw_empty[rs], ph ^ 1, abort_flag, kWaitLimit)) { ok = false; break; }
-                    if (S::tma_a(p, cr.seg)) mbar_arrive(&raw_full[rs]);
-                    else issue_raw<KIND, NT>(p, cr, sRaw + rs * Plan::kRaw, &raw_full[rs]);
-                    last_r[rs] = ph;
-                    cr.next_stage(p);
-                    ++it_r;
-                }
-                if (!ok) break;
+            while (!cb.done) {
                 const int s = it_b % STAGES;
                 const uint32_t ph = (it_b / STAGES) & 1;
                 if (!mbar_wait(&empty[s], ph ^ 1, abort_flag, kWaitLimit)) break;
@@ -543,36 +516,46 @@ __global__ void __launch_bounds__(kGemmThreads, 1) k_umma_gemm(const __grid_cons
                 volatile int dummy = 0;
                 for (int i = 0; i < STAGES; ++i)
                     if (last_b[i] != 0xFFFFFFFFu) mbar_wait(&full_b[i], last_b[i], &dummy, kWaitLimit);
-                for (int i = 0; i < RS; ++i)
-                    if (last_r[i] != 0xFFFFFFFFu) mbar_wait(&raw_full[i], last_r[i], &dummy, kWaitLimit);
             }
         }
         __syncwarp();
     } else if (warp >= 4 && warp < 12) {
         // ------------------------------------------------------------ converters
+        // Each thread owns half a weight row of every stage; its stored bytes
+        // are fetched with plain loads kRawAhead - 1 stages ahead of use.
         const int r = (threadIdx.x - 128) & 127;   // A row
         const int hh = (threadIdx.x - 128) >> 7;   // half of the 64 columns
-        Cursor<KIND, NT> cur;
+        Cursor<KIND, NT> cur, cf;
         cur.begin(p);
+        cf = cur;
+        RawHalf raw[kRawAhead];
+#pragma unroll
+        for (int k = 0; k < kRawAhead - 1; ++k) {
+            if (!cf.done) {
+                if (!S::tma_a(p, cf.seg)) fetch_raw<KIND, NT>(p, cf, r, hh, raw[k]);
+                cf.next_stage(p);
+            }
+        }
         uint32_t it = 0;
         while (!cur.done) {
-            const int s = it % STAGES, rs = it % RS;
-            const uint32_t ph = (it / STAGES) & 1, rph = (it / RS) & 1;
+            if (!cf.done) {
+                if (!S::tma_a(p, cf.seg)) fetch_raw<KIND, NT>(p, cf, r, hh, raw[kRawAhead - 1]);
+                cf.next_stage(p);
+            }
+            const int s = it % STAGES;
+            const uint32_t ph = (it / STAGES) & 1;
             const bool ta = S::tma_a(p, cur.seg);
-            if (!mbar_wait(&raw_full[rs], rph, abort_flag, kWaitLimit)) break;
             if (!mbar_wait(&empty[s], ph ^ 1, abort_flag, kWaitLimit)) break;
             if (!ta) {
                 uint32_t o[16];
-                dequant_half<KIND>(p, sRaw + rs * Plan::kRaw, r, hh, o);
+                dequant_half<KIND>(p, raw[0], hh, o);
                 store_half_swizzled(sA + s * Plan::kA, r, hh, o);
                 fence_proxy_async_smem();
             }
             __syncwarp();
-            if (lane == 0) {
-                // every stage completes a phase of full_a and raw_empty, so their parity stays in step
-                mbar_arrive(&full_a[s]);
-                mbar_arrive(&raw_empty[rs]);
-            }
+            if (lane == 0) mbar_arrive(&full_a[s]);
+#pragma unroll
+            for (int k = 0; k + 1 < kRawAhead; ++k) raw[k] = raw[k + 1];
             cur.next_stage(p);
             ++it;
         }
@@ -994,7 +977,7 @@ cudaError_t run_prefill_path(PrefillParams p, cudaStream_t st, void* memset_base
     k_x_to_fp16<<<T, 256, 0, st>>>(p);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
     mark(st);
-    if ((e = launch_gemm<G_ROUTER, kNtDense, 4, 1>(m_router, p, st, (E / 128) * ttiles)) != cudaSuccess) return e;
+    if ((e = launch_gemm<G_ROUTER, kNtDense, 4, 0>(m_router, p, st, (E / 128) * ttiles)) != cudaSuccess) return e;
     mark(st);
     k_topk<<<(T * 32 + 255) / 256, 256, 0, st>>>(p);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
@@ -1004,19 +987,19 @@ cudaError_t run_prefill_path(PrefillParams p, cudaStream_t st, void* memset_base
     k_bucket_scatter<<<(pairs + 255) / 256, 256, 0, st>>>(p);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
     mark(st);
-    if ((e = launch_gemm<G_SHARED_GATEUP, kNtDense, 4, 1>(m_shared, p, st, (Fs / 64) * ttiles)) != cudaSuccess) return e;
+    if ((e = launch_gemm<G_SHARED_GATEUP, kNtDense, 4, 0>(m_shared, p, st, (Fs / 64) * ttiles)) != cudaSuccess) return e;
     mark(st);
-    if ((e = launch_gemm<G_DPROJ, kNtDense, 3, 6>(m_d, p, st, G * (L / 128) * ttiles)) != cudaSuccess) return e;
+    if ((e = launch_gemm<G_DPROJ, kNtDense, 4, 0>(m_d, p, st, G * (L / 128) * ttiles)) != cudaSuccess) return e;
     mark(st);
     const int max_etiles = min(E, pairs) + pairs / kNtExpert + 1;
-    if ((e = launch_gemm<G_GATEUP, kNtExpert, 4, 8>(m_gu, p, st, (F / 64) * max_etiles)) != cudaSuccess) return e;
+    if ((e = launch_gemm<G_GATEUP, kNtExpert, 6, 0>(m_gu, p, st, (F / 64) * max_etiles)) != cudaSuccess) return e;
     mark(st);
-    if ((e = launch_gemm<G_DOWN, kNtExpert, 4, 8>(m_down, p, st, (L / 128) * max_etiles)) != cudaSuccess) return e;
+    if ((e = launch_gemm<G_DOWN, kNtExpert, 6, 0>(m_down, p, st, (L / 128) * max_etiles)) != cudaSuccess) return e;
     mark(st);
     k_combine<<<T, 256, 0, st>>>(p);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
     mark(st);
-    if ((e = launch_gemm<G_UPROJ, kNtDense, 3, 6>(m_u, p, st, (H / 128) * ttiles)) != cudaSuccess) return e;
+    if ((e = launch_gemm<G_UPROJ, kNtDense, 4, 0>(m_u, p, st, (H / 128) * ttiles)) != cudaSuccess) return e;
     mark(st);
     return cudaSuccess;
 }
@@ -1029,7 +1012,7 @@ cudaError_t run_prefill_route(PrefillParams p, cudaStream_t st) {
     ok &= make_map_2d(&m.b, p.x, true, p.T, p.H, p.H, kNtDense);
     if (!ok) return cudaErrorInvalidValue;
     const int ttiles = (p.T + kNtDense - 1) / kNtDense;
-    cudaError_t e = launch_gemm<G_ROUTER, kNtDense, 4, 1>(m, p, st, (p.E / 128) * ttiles);
+    cudaError_t e = launch_gemm<G_ROUTER, kNtDense, 4, 0>(m, p, st, (p.E / 128) * ttiles);
     if (e != cudaSuccess) return e;
     k_topk<<<(p.T * 32 + 255) / 256, 256, 0, st>>>(p);
     return cudaGetLastError();
