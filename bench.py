@@ -126,11 +126,10 @@ def step_cost(shape, idx: np.ndarray, groups: np.ndarray, T: int, prefill: bool)
     pairs_tg = sum(len({int(groups[e]) for e in idx[t]}) for t in range(idx.shape[0]))   # hit (token, group) pairs
     b = {
         "k_router_shared": rw + 2 * Fs * H * 2 + T * H * 2,
-        "k_stream_dproj": len(hit) * du + T * H * 2,
-        "k_stream_gateup": len(distinct) * rec_gu,
-        "k_stream_down": len(distinct) * rec_d,
-        "k_combine_small": 0,
-        "k_stream_uproj": len(hit) * du + H * Fs * 2 + 2 * T * H * 2,
+        "k_wstream_dproj": len(hit) * du + T * H * 2,
+        "k_wstream_gateup": len(distinct) * rec_gu,
+        "k_wstream_down": len(distinct) * rec_d,
+        "k_wstream_uproj": len(hit) * du + H * Fs * 2 + 2 * T * H * 2,
     }
     f = {
         "x_to_fp16": 0.0,
@@ -152,8 +151,7 @@ def step_cost(shape, idx: np.ndarray, groups: np.ndarray, T: int, prefill: bool)
     return out
 
 
-STAGES = ["k_router_shared", "k_stream_dproj", "k_stream_gateup", "k_stream_down", "k_combine_small",
-          "k_stream_uproj"]
+STAGES = ["k_router_shared", "k_wstream_dproj", "k_wstream_gateup", "k_wstream_down", "k_wstream_uproj"]
 PREFILL_STAGES = ["x_to_fp16", "router_gemm", "topk_bucket", "shared_gateup", "dproj", "gateup", "down", "combine",
                   "uproj"]
 

@@ -15,8 +15,9 @@
 //   k_wstream<DPROJ>   h16[t][g]   = D_g x_t            (hit groups)
 //   k_wstream<GATEUP>  z16[slot]   = silu(W_gate h) * (W_up h)
 //   k_wstream<DOWN>    o16w[slot]  = w_slot * W_down z
-//   k_combine_small    s16[g][t]   = sum of o16w over the token's experts in g
-//   k_wstream<UPROJ>   y           = sum_g U_g s16[g][t] + S_down z_sh (+ residual)
+//   k_wstream<UPROJ>   y           = sum_g U_g s[g][t] + S_down z_sh (+ residual), where
+//                      s[g][t] = sum of o16w over token t's experts in group g is formed
+//                      while the CTA fills its activation cache
 //
 // Method: teardown article "Edge0-145B: a Qwen MoE with its experts
 // squeezed", section "A latent in front of the experts" (layer equation,
@@ -221,14 +222,17 @@ struct WPlan {
 };
 
 // Items run matrix-major (consecutive items share a matrix, so a CTA's chunk
-// touches few of them), then tile, then part.
+// touches few of them), then reduction part, then tile: the warps of a CTA
+// work on neighbouring row tiles of the same K blocks at the same time, so
+// together they read long contiguous runs of each stored K block (one
+// tile's 16 rows are only 256-512 bytes of it).
 template <int PHASE, int FMT>
 __device__ __forceinline__ WItem decode_item(const FwdParams& p, const StreamShared& sh, const WPlan& pl, int i) {
     WItem it;
     const int per_mat = pl.tiles * pl.ks;
     const int m = i / per_mat, rem = i - m * per_mat;
-    it.tile = rem / pl.ks;
-    it.q = rem - it.tile * pl.ks;
+    it.q = rem / pl.tiles;
+    it.tile = rem - it.q * pl.tiles;
     it.r0 = it.tile * 16;
     it.j = m;
     bool shared_part = false;
@@ -392,6 +396,15 @@ __global__ void __launch_bounds__(kWThreads, 1) k_wstream(FwdParams p, WPlan pl,
         if (threadIdx.x == 0) sh.n_unique = __ldcg(p.r.n_unique);
     } else {
         if (threadIdx.x < G) sh.hg[threadIdx.x] = __ldcg(p.r.ghit + threadIdx.x);
+        if (PHASE == SP_UPROJ) {
+            // U sums each token's expert outputs per group itself (below)
+            for (int i = threadIdx.x; i < T * K; i += blockDim.x) {
+                const int e = __ldcg(p.r.idx + i);
+                const int g = p.group[e];
+                sh.pgrp[i] = g < G ? g : 0;   // out-of-range labels were reported by the router
+                sh.pair_slot[i] = __ldcg(p.r.pair_slot + i);
+            }
+        }
         __syncthreads();
         if (threadIdx.x == 0) {
             int n = 0;
@@ -491,8 +504,30 @@ __global__ void __launch_bounds__(kWThreads, 1) k_wstream(FwdParams p, WPlan pl,
             if (PHASE == SP_DPROJ) s = p.x16 + (size_t)src * H;
             else if (PHASE == SP_GATEUP) s = p.h16 + (size_t)src * L;
             else if (PHASE == SP_DOWN) s = p.z16 + (size_t)src * F;
-            else if (src >= 0) { s = p.s16 + (size_t)src * L; w = L; }
-            else { s = p.zsh16 + (size_t)(-1 - src) * Fs; w = Fs; }
+            else if (src >= 0) {
+                // U: s[g][t] = sum of the weighted expert outputs of token t's
+                // experts in group g (fp32, in k order), rounded to fp16
+                if (8 * c < L) {
+                    const int g = src / T, t = src - g * T;
+                    float acc8[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+                    for (int k = 0; k < K; ++k) {
+                        if (sh.pgrp[t * K + k] != g) continue;
+                        const uint4 v = __ldcg(reinterpret_cast<const uint4*>(p.o16w + (size_t)sh.pair_slot[t * K + k] * L) + c);
+                        const uint32_t w4[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+                        for (int j = 0; j < 4; ++j) {
+                            const float2 f = __half22float2(*reinterpret_cast<const __half2*>(&w4[j]));
+                            acc8[2 * j] += f.x;
+                            acc8[2 * j + 1] += f.y;
+                        }
+                    }
+                    __half2 h[4];
+#pragma unroll
+                    for (int j = 0; j < 4; ++j) h[j] = __floats2half2_rn(acc8[2 * j], acc8[2 * j + 1]);
+                    *reinterpret_cast<uint4*>(cache + (size_t)r * ld + 8 * c) = *reinterpret_cast<uint4*>(h);
+                }
+                continue;
+            } else { s = p.zsh16 + (size_t)(-1 - src) * Fs; w = Fs; }
             if (8 * c < w)
                 *reinterpret_cast<uint4*>(cache + (size_t)r * ld + 8 * c) = __ldcg(reinterpret_cast<const uint4*>(s) + c);
         }
@@ -595,42 +630,6 @@ __global__ void __launch_bounds__(kWThreads, 1) k_wstream(FwdParams p, WPlan pl,
         }
     }
     cp_async_wait<0>();
-}
-
-// s16[g][t] = sum over the token's experts of group g of o16w (zero if none)
-__global__ void k_combine_small(FwdParams p) {
-    const int t = blockIdx.y, g = blockIdx.x;
-    const int L = p.L, K = p.K;
-    __shared__ int slots[kMaxTopK];
-    __shared__ int n;
-    grid_dep_wait();
-    grid_dep_launch();
-    if (threadIdx.x == 0) {
-        int c = 0;
-        for (int k = 0; k < K; ++k) {
-            const int e = __ldcg(p.r.idx + t * K + k);
-            if (p.group[e] == g) slots[c++] = __ldcg(p.r.pair_slot + t * K + k);
-        }
-        n = c;
-    }
-    __syncthreads();
-    for (int c8 = threadIdx.x; c8 < L / 8; c8 += blockDim.x) {
-        float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-        for (int i = 0; i < n; ++i) {
-            const uint4 v = __ldcg(reinterpret_cast<const uint4*>(p.o16w + (size_t)slots[i] * L) + c8);
-            const uint32_t w4[4] = {v.x, v.y, v.z, v.w};
-#pragma unroll
-            for (int j = 0; j < 4; ++j) {
-                const float2 f = __half22float2(*reinterpret_cast<const __half2*>(&w4[j]));
-                acc[2 * j] += f.x;
-                acc[2 * j + 1] += f.y;
-            }
-        }
-        __half2 h[4];
-#pragma unroll
-        for (int j = 0; j < 4; ++j) h[j] = __floats2half2_rn(acc[2 * j], acc[2 * j + 1]);
-        reinterpret_cast<uint4*>(p.s16 + ((size_t)g * p.T + t) * L)[c8] = *reinterpret_cast<uint4*>(h);
-    }
 }
 
 // ---------------------------------------------------------------------------
@@ -758,8 +757,6 @@ cudaError_t run_stream_path(const FwdParams& p, cudaStream_t st) {
     if (e != cudaSuccess) return e;
     e = launch_wstream<SP_DOWN, LMOE_Q8_0>(p, P.dn, chunk_rows(P.dn), st);
     if (e != cudaSuccess) return e;
-    stage_mark(st);
-    if ((e = launch_dependent(k_combine_small, dim3(G, p.T), dim3(128), 0, st, p)) != cudaSuccess) return e;
     e = p.du_fmt == LMOE_Q8_0 ? launch_wstream<SP_UPROJ, LMOE_Q8_0>(p, P.u, chunk_rows(P.u), st)
                               : launch_wstream<SP_UPROJ, LMOE_Q4_0>(p, P.u, chunk_rows(P.u), st);
     return e;
