@@ -131,6 +131,7 @@ def step_cost(shape, idx: np.ndarray, groups: np.ndarray, T: int, prefill: bool)
         "k_wstream_down": len(distinct) * rec_d,
         "k_wstream_uproj": len(hit) * du + H * Fs * 2 + 2 * T * H * 2,
     }
+    b_total = float(sum(b.values()))
     f = {
         "x_to_fp16": 0.0,
         "router_gemm": 2.0 * T * E * H,
@@ -144,7 +145,7 @@ def step_cost(shape, idx: np.ndarray, groups: np.ndarray, T: int, prefill: bool)
     }
     weight_bytes = rw + 3 * Fs * H * 2 + len(hit) * 2 * du + len(distinct) * (rec_gu + rec_d)
     out = dict(f if prefill else b)
-    out["bytes_total"] = weight_bytes + 2 * T * H * 2 if prefill else float(sum(b.values()))
+    out["bytes_total"] = weight_bytes + 2 * T * H * 2 if prefill else b_total
     out["flops_total"] = float(sum(f.values()))
     out["n_distinct"] = len(distinct)
     out["n_groups_hit"] = len(hit)
@@ -152,6 +153,7 @@ def step_cost(shape, idx: np.ndarray, groups: np.ndarray, T: int, prefill: bool)
 
 
 STAGES = ["k_router_shared", "k_wstream_dproj", "k_wstream_gateup", "k_wstream_down", "k_wstream_uproj"]
+
 PREFILL_STAGES = ["x_to_fp16", "router_gemm", "topk_bucket", "shared_gateup", "dproj", "gateup", "down", "combine",
                   "uproj"]
 
@@ -509,14 +511,15 @@ def main():
     line = {
         "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": K, "warmup": W,
         "ms_per_step": ms_max / K, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
-        "dtype": "f16" if prefill else "f32", "data": "synthetic",
+        "dtype": "f16", "data": "synthetic",
         "config": {"workload": workload_desc(wl, T), "T": T, "parallelism": f"replicas x{world}",
                    "l2": f"inputs larger than L2: {R} weight copies rotated, "
                          f"{R * per_step_max / 1e6:.0f} MB touched between reuses",
                    "weights": "NVFP4 experts, Q8_0/Q4_0 D/U, bf16 router and shared expert; "
                               "bf16 activations in and out, fp32 accumulation",
                    "path": ("tensor cores (tcgen05): fp16 operands dequantised from the stored formats"
-                            if prefill else "CUDA-core weight streaming"),
+                            if prefill else "weight streaming on the tensor pipe (mma.sync, fp16 operands, fp32 "
+                                            "accumulation), five kernels per layer"),
                    "timing": f"{n_graphs} captured CUDA graphs replayed in turn"},
         "roofline": roof,
         "layer": {"gbs": step_alg_bytes / t_step / 1e9, "tflops": step_flops / t_step / 1e12,

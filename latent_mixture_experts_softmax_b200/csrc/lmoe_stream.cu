@@ -351,213 +351,193 @@ template <int PHASE>
 __device__ __forceinline__ int n_steps(const WItem& it, int sb) { return (it.kb1 - it.kb0 + sb - 1) / sb; }
 
 // ---------------------------------------------------------------------------
-// the kernel
+// one phase: chunk, activation cache, per-warp pipeline
 // ---------------------------------------------------------------------------
 
+// The chunk of items of one CTA and the activation rows of its matrices.
+struct ChunkInfo {
+    int i0, i1;                  // items [i0, i1)
+    int m0, nm, rows, skip;      // first matrix, matrices, cached rows, refused
+    int row0[kMaxChunkParts];    // first cache row of each matrix
+    int src[kMaxChunkParts * 8]; // source of each cache row (phase-specific code)
+    float tail[kMaxChunkParts][4];  // experts: tensor scales of gate, up, down
+};
+
+// One warp's load cursor over its items' steps.
+struct LoadCursor {
+    int li, ls, l_ns, n_issued;
+    WItem lit;
+};
+
+template <int PHASE>
+__host__ __device__ __forceinline__ int cache_ld(int H, int L, int F, int Fs) {
+    return PHASE == SP_DPROJ ? H + kActPad : PHASE == SP_GATEUP ? L + kActPad : PHASE == SP_DOWN ? F + kActPad
+                                                                                               : (L > Fs ? L : Fs) + kActPad;
+}
+
+template <int PHASE>
+__device__ __forceinline__ int phase_mats(const StreamShared& sh) {
+    return PHASE == SP_DPROJ ? sh.n_hit : PHASE == SP_UPROJ ? sh.n_hit + 1 : sh.n_unique;
+}
+
+// Thread 0 decides the CTA's chunk and its cache rows; threads < 4 * nm
+// fetch the experts' tensor scales.  Ends with __syncthreads.
 template <int PHASE, int FMT>
-__global__ void __launch_bounds__(kWThreads, 1) k_wstream(FwdParams p, WPlan pl, int cache_bytes) {
-    extern __shared__ uint8_t smem_raw[];
-    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 127) & ~(uintptr_t)127);
-    __shared__ StreamShared sh;
-    // the chunk's matrices: cache rows and (experts) tensor scales
-    __shared__ int c_m0, c_nm, c_skip, c_rows;
-    __shared__ int c_row0[kMaxChunkParts];
-    __shared__ int c_src[kMaxChunkParts * 8];
-    __shared__ float c_tail[kMaxChunkParts][4];
-
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int T = p.T, H = p.H, L = p.L, F = p.F, Fs = p.Fs, G = p.G, K = p.K;
-    __half* cache = reinterpret_cast<__half*>(smem);
-    uint8_t* ring = smem + cache_bytes + (size_t)warp * kPD * kStepBytes;
-    const int ld = PHASE == SP_DPROJ ? H + kActPad
-                 : PHASE == SP_GATEUP ? L + kActPad
-                 : PHASE == SP_DOWN ? F + kActPad
-                                    : max(L, Fs) + kActPad;
-
-    // Routing, as the router kernel published it.  D runs right after the
-    // router kernel and waits for it first.  The later kernels read the
-    // routing before their own wait: their predecessor let them launch only
-    // after its own wait, so the router kernel had completed by then.
-    if (PHASE == SP_DPROJ) {
-        grid_dep_wait();
-        grid_dep_launch();
-    }
-    if (PHASE == SP_GATEUP || PHASE == SP_DOWN) {
-        const int n = T * K;
-        for (int i = threadIdx.x; i < n; i += blockDim.x) {
-            sh.uexp[i] = __ldcg(p.r.uexp + i);
-            sh.ucnt[i] = __ldcg(p.r.ucnt + i);
-            sh.uoff[i] = __ldcg(p.r.uoff + i);
-            sh.ugrp[i] = __ldcg(p.r.ugrp + i);
-            const int pr = __ldcg(p.r.slot_pair + i);
-            sh.slot_tok[i] = pr / K;
-            sh.slot_w[i] = __ldcg(p.r.w + pr);
-        }
-        if (threadIdx.x == 0) sh.n_unique = __ldcg(p.r.n_unique);
-    } else {
-        if (threadIdx.x < G) sh.hg[threadIdx.x] = __ldcg(p.r.ghit + threadIdx.x);
-        if (PHASE == SP_UPROJ) {
-            // U sums each token's expert outputs per group itself (below)
-            for (int i = threadIdx.x; i < T * K; i += blockDim.x) {
-                const int e = __ldcg(p.r.idx + i);
-                const int g = p.group[e];
-                sh.pgrp[i] = g < G ? g : 0;   // out-of-range labels were reported by the router
-                sh.pair_slot[i] = __ldcg(p.r.pair_slot + i);
-            }
-        }
-        __syncthreads();
-        if (threadIdx.x == 0) {
-            int n = 0;
-            for (int g = 0; g < G; ++g)
-                if (sh.hg[g] > 0) sh.hg[n++] = g;
-            sh.n_hit = n;
-        }
-    }
-    __syncthreads();
-
-    WPlan plan = pl;
-    plan.n_mats = PHASE == SP_DPROJ ? sh.n_hit : PHASE == SP_UPROJ ? sh.n_hit + 1 : sh.n_unique;
-    const int n_items = plan.n_mats * plan.tiles * plan.ks;
-    const int i0 = chunk_begin(blockIdx.x, n_items, gridDim.x);
-    int i1 = chunk_begin(blockIdx.x + 1, n_items, gridDim.x);
-    const int per_mat = plan.tiles * plan.ks;
-
-    // the chunk's matrices and their activation rows
+__device__ void phase_setup(const FwdParams& p, const StreamShared& sh, const WPlan& plan, int cache_bytes,
+                            ChunkInfo& ci) {
+    const int T = p.T, G = p.G;
+    const int ld = cache_ld<PHASE>(p.H, p.L, p.F, p.Fs);
     if (threadIdx.x == 0) {
+        const int n_items = phase_mats<PHASE>(sh) * plan.tiles * plan.ks;
+        const int per_mat = plan.tiles * plan.ks;
+        const int i0 = chunk_begin(blockIdx.x, n_items, gridDim.x);
+        const int i1 = chunk_begin(blockIdx.x + 1, n_items, gridDim.x);
         const int m0 = i0 / per_mat, m1 = i0 < i1 ? (i1 - 1) / per_mat : m0 - 1;
         const int nm = PHASE == SP_DPROJ ? 1 : m1 - m0 + 1;
         int rows = 0;
         bool fits = nm <= kMaxChunkParts;
         for (int jj = 0; fits && jj < nm; ++jj) {
             const int m = m0 + jj;
-            c_row0[jj] = rows;
+            ci.row0[jj] = rows;
             const int nr = (PHASE == SP_GATEUP || PHASE == SP_DOWN) ? sh.ucnt[m] : T;
             if (rows + nr > kMaxChunkParts * 8) { fits = false; break; }
             for (int c = 0; c < nr; ++c, ++rows) {
                 int src;
-                if (PHASE == SP_DPROJ) src = c;                                           // x16 row
-                else if (PHASE == SP_GATEUP) src = sh.slot_tok[sh.uoff[m] + c] * G + sh.ugrp[m];   // h16 row
-                else if (PHASE == SP_DOWN) src = sh.uoff[m] + c;                          // z16 row
-                else src = m < sh.n_hit ? sh.hg[m] * T + c : -1 - c;                      // s16 row / shared hidden row
-                c_src[rows] = src;
+                if (PHASE == SP_DPROJ) src = c;                                                     // x row
+                else if (PHASE == SP_GATEUP) src = sh.slot_tok[sh.uoff[m] + c] * G + sh.ugrp[m];  // h16 row
+                else if (PHASE == SP_DOWN) src = sh.uoff[m] + c;                                    // z16 row
+                else src = m < sh.n_hit ? sh.hg[m] * T + c : -1 - c;                               // s[g][t] / shared hidden
+                ci.src[rows] = src;
             }
         }
         fits = fits && (size_t)rows * ld * 2 <= (size_t)cache_bytes;
         if (!fits) set_status(p.ctrl, LMOE_ERR_UNSUPPORTED);
-        c_m0 = m0;
-        c_nm = fits ? nm : 0;
-        c_skip = !fits;
-        c_rows = fits ? rows : 0;
+        ci.i0 = i0;
+        ci.i1 = fits ? i1 : i0;
+        ci.m0 = m0;
+        ci.nm = fits ? nm : 0;
+        ci.rows = fits ? rows : 0;
+        ci.skip = !fits;
     }
     __syncthreads();
-    if (c_skip) i1 = i0;
-    if ((PHASE == SP_GATEUP || PHASE == SP_DOWN) && threadIdx.x < 4 * c_nm) {
+    if ((PHASE == SP_GATEUP || PHASE == SP_DOWN) && threadIdx.x < 4 * ci.nm) {
         const int jj = threadIdx.x >> 2, qq = threadIdx.x & 3;
-        const size_t nq = (size_t)L * F / 2, ns = (size_t)L * F / 16;
+        const size_t nq = (size_t)p.L * p.F / 2, ns = (size_t)p.L * p.F / 16;
         const float* tail =
-            reinterpret_cast<const float*>(p.experts + (size_t)sh.uexp[c_m0 + jj] * p.rec_bytes + 3 * nq + 3 * ns);
-        c_tail[jj][qq] = __ldg(tail + qq);
+            reinterpret_cast<const float*>(p.experts + (size_t)sh.uexp[ci.m0 + jj] * p.rec_bytes + 3 * nq + 3 * ns);
+        ci.tail[jj][qq] = __ldg(tail + qq);
     }
+}
 
-    // Every warp starts streaming its first steps' weights, which depend on
-    // the routing only, before the activations of the previous kernel exist.
-    const WItem none = {0, 0, 0, 0, 0, 0, 0};
-    int li = i0 + warp, ls = 0, l_ns = 0;      // load cursor: item, step, steps of the item
-    WItem lit = none;
-    if (li < i1) {
-        lit = decode_item<PHASE, FMT>(p, sh, plan, li);
-        l_ns = n_steps<PHASE>(lit, step_blocks<PHASE, FMT>(PHASE == SP_UPROJ && lit.mat < 0));
-    }
-    auto advance_load = [&]() {
-        if (li >= i1) return;
-        if (++ls < l_ns) return;
-        ls = 0;
-        li += kWW;
-        if (li < i1) {
-            lit = decode_item<PHASE, FMT>(p, sh, plan, li);
-            l_ns = n_steps<PHASE>(lit, step_blocks<PHASE, FMT>(PHASE == SP_UPROJ && lit.mat < 0));
-        }
-    };
-    int n_issued = 0;
-#pragma unroll
-    for (int k = 0; k < kPD - 1; ++k) {
-        if (li < i1) issue_step<PHASE, FMT>(p, lit, ls, ring + (size_t)(n_issued % kPD) * kStepBytes, lane);
-        cp_async_commit();
-        ++n_issued;
-        advance_load();
-    }
+template <int PHASE, int FMT>
+__device__ __forceinline__ void cursor_load_item(const FwdParams& p, const StreamShared& sh, const WPlan& plan,
+                                                 LoadCursor& c) {
+    c.lit = decode_item<PHASE, FMT>(p, sh, plan, c.li);
+    c.l_ns = n_steps<PHASE>(c.lit, step_blocks<PHASE, FMT>(PHASE == SP_UPROJ && c.lit.mat < 0));
+}
 
-    if (PHASE != SP_DPROJ) {
-        grid_dep_wait();
-        grid_dep_launch();
-    }
-    // the chunk's activations, by plain loads of every thread
-    {
-        const int rows = c_rows;
-        const int KC = PHASE == SP_DPROJ ? H : PHASE == SP_GATEUP ? L : PHASE == SP_DOWN ? F : max(L, Fs);
-        const int per = KC / 8;
-        for (int qv = threadIdx.x; qv < rows * per; qv += blockDim.x) {
-            const int r = qv / per, c = qv - r * per;
-            const int src = c_src[r];
-            const __half* s;
-            int w = KC;
-            if (PHASE == SP_DPROJ) s = p.x16 + (size_t)src * H;
-            else if (PHASE == SP_GATEUP) s = p.h16 + (size_t)src * L;
-            else if (PHASE == SP_DOWN) s = p.z16 + (size_t)src * F;
-            else if (src >= 0) {
-                // U: s[g][t] = sum of the weighted expert outputs of token t's
-                // experts in group g (fp32, in k order), rounded to fp16
-                if (8 * c < L) {
-                    const int g = src / T, t = src - g * T;
-                    float acc8[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-                    for (int k = 0; k < K; ++k) {
-                        if (sh.pgrp[t * K + k] != g) continue;
-                        const uint4 v = __ldcg(reinterpret_cast<const uint4*>(p.o16w + (size_t)sh.pair_slot[t * K + k] * L) + c);
-                        const uint32_t w4[4] = {v.x, v.y, v.z, v.w};
+// Issue the next step of the warp's stream (an empty commit group past its end).
+template <int PHASE, int FMT>
+__device__ __forceinline__ void cursor_issue(const FwdParams& p, const StreamShared& sh, const WPlan& plan,
+                                             const ChunkInfo& ci, uint8_t* ring, LoadCursor& c, int lane) {
+    if (c.li < ci.i1) issue_step<PHASE, FMT>(p, c.lit, c.ls, ring + (size_t)(c.n_issued % kPD) * kStepBytes, lane);
+    cp_async_commit();
+    ++c.n_issued;
+    if (c.li >= ci.i1) return;
+    if (++c.ls < c.l_ns) return;
+    c.ls = 0;
+    c.li += kWW;
+    if (c.li < ci.i1) cursor_load_item<PHASE, FMT>(p, sh, plan, c);
+}
+
+// The warp's first kPD - 1 steps (weights only: they depend on the routing).
+template <int PHASE, int FMT>
+__device__ void phase_prime(const FwdParams& p, const StreamShared& sh, const WPlan& plan, const ChunkInfo& ci,
+                            uint8_t* ring, LoadCursor& c) {
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    c.li = ci.i0 + warp;
+    c.ls = 0;
+    c.l_ns = 0;
+    c.n_issued = 0;
+    if (c.li < ci.i1) cursor_load_item<PHASE, FMT>(p, sh, plan, c);
 #pragma unroll
-                        for (int j = 0; j < 4; ++j) {
-                            const float2 f = __half22float2(*reinterpret_cast<const __half2*>(&w4[j]));
-                            acc8[2 * j] += f.x;
-                            acc8[2 * j + 1] += f.y;
-                        }
-                    }
-                    __half2 h[4];
+    for (int k = 0; k < kPD - 1; ++k) cursor_issue<PHASE, FMT>(p, sh, plan, ci, ring, c, lane);
+}
+
+// The chunk's activations from global memory, by plain loads of every thread.
+template <int PHASE>
+__device__ void phase_fill(const FwdParams& p, const StreamShared& sh, const ChunkInfo& ci, __half* cache) {
+    const int T = p.T, H = p.H, L = p.L, F = p.F, Fs = p.Fs, K = p.K;
+    const int ld = cache_ld<PHASE>(H, L, F, Fs);
+    const int KC = PHASE == SP_DPROJ ? H : PHASE == SP_GATEUP ? L : PHASE == SP_DOWN ? F : max(L, Fs);
+    const int per = KC / 8;
+    for (int qv = threadIdx.x; qv < ci.rows * per; qv += blockDim.x) {
+        const int r = qv / per, c = qv - r * per;
+        const int src = ci.src[r];
+        uint4 v;
+        if (PHASE == SP_DPROJ) {
+            v = __ldcg(reinterpret_cast<const uint4*>(p.x16 + (size_t)src * H) + c);
+        } else if (PHASE == SP_GATEUP) {
+            v = __ldcg(reinterpret_cast<const uint4*>(p.h16 + (size_t)src * L) + c);
+        } else if (PHASE == SP_DOWN) {
+            v = __ldcg(reinterpret_cast<const uint4*>(p.z16 + (size_t)src * F) + c);
+        } else if (src >= 0) {
+            // U: s[g][t] = sum of the weighted expert outputs of token t's
+            // experts in group g (fp32, in k order), rounded to fp16
+            if (8 * c >= L) continue;
+            const int g = src / T, t = src - g * T;
+            float acc8[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+            for (int k = 0; k < K; ++k) {
+                if (sh.pgrp[t * K + k] != g) continue;
+                const uint4 o = __ldcg(reinterpret_cast<const uint4*>(p.o16w + (size_t)sh.pair_slot[t * K + k] * L) + c);
+                const uint32_t w4[4] = {o.x, o.y, o.z, o.w};
 #pragma unroll
-                    for (int j = 0; j < 4; ++j) h[j] = __floats2half2_rn(acc8[2 * j], acc8[2 * j + 1]);
-                    *reinterpret_cast<uint4*>(cache + (size_t)r * ld + 8 * c) = *reinterpret_cast<uint4*>(h);
+                for (int j = 0; j < 4; ++j) {
+                    const float2 f = __half22float2(*reinterpret_cast<const __half2*>(&w4[j]));
+                    acc8[2 * j] += f.x;
+                    acc8[2 * j + 1] += f.y;
                 }
-                continue;
-            } else { s = p.zsh16 + (size_t)(-1 - src) * Fs; w = Fs; }
-            if (8 * c < w)
-                *reinterpret_cast<uint4*>(cache + (size_t)r * ld + 8 * c) = __ldcg(reinterpret_cast<const uint4*>(s) + c);
+            }
+            __half2 h[4];
+#pragma unroll
+            for (int j = 0; j < 4; ++j) h[j] = __floats2half2_rn(acc8[2 * j], acc8[2 * j + 1]);
+            v = *reinterpret_cast<uint4*>(h);
+        } else {
+            if (8 * c >= Fs) continue;
+            v = __ldcg(reinterpret_cast<const uint4*>(p.zsh16 + (size_t)(-1 - src) * Fs) + c);
         }
+        *reinterpret_cast<uint4*>(cache + (size_t)r * ld + 8 * c) = v;
     }
-    __syncthreads();
+}
 
-    // ---- the warp's items: stream, multiply, finish
-    int ci = i0 + warp, cs = 0, c_nsteps = 0, n_done = 0;
-    WItem cit = none;
-    if (ci < i1) {
-        cit = decode_item<PHASE, FMT>(p, sh, plan, ci);
+// The warp's items: stream, multiply, finish (epilogue, or partial + ticket).
+template <int PHASE, int FMT>
+__device__ void phase_run(const FwdParams& p, const StreamShared& sh, const WPlan& plan, const ChunkInfo& ci,
+                          uint8_t* ring, const __half* cache, LoadCursor& lc) {
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int T = p.T, H = p.H, L = p.L, F = p.F, G = p.G;
+    const int ld = cache_ld<PHASE>(H, L, F, p.Fs);
+    const int n_mats = phase_mats<PHASE>(sh);
+    int cidx = ci.i0 + warp, cs = 0, c_nsteps = 0, n_done = 0;
+    WItem cit = {0, 0, 0, 0, 0, 0, 0};
+    if (cidx < ci.i1) {
+        cit = decode_item<PHASE, FMT>(p, sh, plan, cidx);
         c_nsteps = n_steps<PHASE>(cit, step_blocks<PHASE, FMT>(PHASE == SP_UPROJ && cit.mat < 0));
     }
     float a[4] = {0.f, 0.f, 0.f, 0.f}, u[4] = {0.f, 0.f, 0.f, 0.f};
     const int gg = lane >> 2, tt = lane & 3;
-    while (ci < i1) {
-        if (li < i1) issue_step<PHASE, FMT>(p, lit, ls, ring + (size_t)(n_issued % kPD) * kStepBytes, lane);
-        cp_async_commit();
-        ++n_issued;
-        advance_load();
+    while (cidx < ci.i1) {
+        cursor_issue<PHASE, FMT>(p, sh, plan, ci, ring, lc, lane);
         cp_async_wait<kPD - 1>();
         __syncwarp();
         // activations of the item
-        const int jj = cit.j - c_m0;
+        const int jj = cit.j - ci.m0;
         const __half* xs;
         int nt = T;
         if (PHASE == SP_DPROJ) xs = cache;
-        else if (PHASE == SP_UPROJ) xs = cache + (size_t)c_row0[jj] * ld;
+        else if (PHASE == SP_UPROJ) xs = cache + (size_t)ci.row0[jj] * ld;
         else {
-            xs = cache + (size_t)c_row0[jj] * ld;
+            xs = cache + (size_t)ci.row0[jj] * ld;
             nt = sh.ucnt[cit.j];
         }
         compute_step<PHASE, FMT>(p, cit, cs, ring + (size_t)(n_done % kPD) * kStepBytes, xs, ld, nt, a, u);
@@ -566,14 +546,12 @@ __global__ void __launch_bounds__(kWThreads, 1) k_wstream(FwdParams p, WPlan pl,
         if (++cs < c_nsteps) continue;
 
         // ---- the item is complete: epilogue or partial
-        const int nparts = PHASE == SP_UPROJ ? plan.n_mats * plan.ks : plan.ks;
+        const int nparts = PHASE == SP_UPROJ ? n_mats * plan.ks : plan.ks;
         bool finish = nparts == 1;
-        int tick_base = 0, part = 0;
         if (!finish) {
             // partial of part (j, q) of tile (mat, tile); U: all matrices are parts of one tile
             const int key = PHASE == SP_UPROJ ? cit.tile : cit.j * plan.tiles + cit.tile;
-            part = PHASE == SP_UPROJ ? cit.j * plan.ks + cit.q : cit.q;
-            tick_base = key;
+            const int part = PHASE == SP_UPROJ ? cit.j * plan.ks + cit.q : cit.q;
             float* dst = p.wpart + (((size_t)key * nparts + part) * 32 + lane) * 8;
             *reinterpret_cast<float4*>(dst) = make_float4(a[0], a[1], a[2], a[3]);
             if (PHASE == SP_GATEUP) *reinterpret_cast<float4*>(dst + 4) = make_float4(u[0], u[1], u[2], u[3]);
@@ -586,11 +564,11 @@ __global__ void __launch_bounds__(kWThreads, 1) k_wstream(FwdParams p, WPlan pl,
                 __threadfence();
                 float sa[4] = {0.f, 0.f, 0.f, 0.f}, su[4] = {0.f, 0.f, 0.f, 0.f};
                 for (int q = 0; q < nparts; ++q) {
-                    const float* s = p.wpart + (((size_t)key * nparts + q) * 32 + lane) * 8;
-                    const float4 v = __ldcg(reinterpret_cast<const float4*>(s));
+                    const float* sp = p.wpart + (((size_t)key * nparts + q) * 32 + lane) * 8;
+                    const float4 v = __ldcg(reinterpret_cast<const float4*>(sp));
                     sa[0] += v.x; sa[1] += v.y; sa[2] += v.z; sa[3] += v.w;
                     if (PHASE == SP_GATEUP) {
-                        const float4 w4 = __ldcg(reinterpret_cast<const float4*>(s + 4));
+                        const float4 w4 = __ldcg(reinterpret_cast<const float4*>(sp + 4));
                         su[0] += w4.x; su[1] += w4.y; su[2] += w4.z; su[3] += w4.w;
                     }
                 }
@@ -601,7 +579,7 @@ __global__ void __launch_bounds__(kWThreads, 1) k_wstream(FwdParams p, WPlan pl,
             }
         }
         if (finish) {
-            const float* ts = (PHASE == SP_GATEUP || PHASE == SP_DOWN) ? c_tail[jj] : nullptr;
+            const float* ts = (PHASE == SP_GATEUP || PHASE == SP_DOWN) ? ci.tail[jj] : nullptr;
 #pragma unroll
             for (int i4 = 0; i4 < 4; ++i4) {
                 const int col = 2 * tt + (i4 & 1), row = cit.r0 + gg + 8 * (i4 >> 1);
@@ -623,12 +601,86 @@ __global__ void __launch_bounds__(kWThreads, 1) k_wstream(FwdParams p, WPlan pl,
 #pragma unroll
         for (int i4 = 0; i4 < 4; ++i4) { a[i4] = 0.f; u[i4] = 0.f; }
         cs = 0;
-        ci += kWW;
-        if (ci < i1) {
-            cit = decode_item<PHASE, FMT>(p, sh, plan, ci);
+        cidx += kWW;
+        if (cidx < ci.i1) {
+            cit = decode_item<PHASE, FMT>(p, sh, plan, cidx);
             c_nsteps = n_steps<PHASE>(cit, step_blocks<PHASE, FMT>(PHASE == SP_UPROJ && cit.mat < 0));
         }
     }
+}
+
+// Routing tables of a later kernel, as the router kernel published them.
+template <int PHASE>
+__device__ void stage_published_routing(const FwdParams& p, StreamShared& sh) {
+    const int T = p.T, G = p.G, K = p.K;
+    if (PHASE == SP_GATEUP || PHASE == SP_DOWN) {
+        const int n = T * K;
+        for (int i = threadIdx.x; i < n; i += blockDim.x) {
+            sh.uexp[i] = __ldcg(p.r.uexp + i);
+            sh.ucnt[i] = __ldcg(p.r.ucnt + i);
+            sh.uoff[i] = __ldcg(p.r.uoff + i);
+            sh.ugrp[i] = __ldcg(p.r.ugrp + i);
+            const int pr = __ldcg(p.r.slot_pair + i);
+            sh.slot_tok[i] = pr / K;
+            sh.slot_w[i] = __ldcg(p.r.w + pr);
+        }
+        if (threadIdx.x == 0) sh.n_unique = __ldcg(p.r.n_unique);
+    } else {
+        if (threadIdx.x < G) sh.hg[threadIdx.x] = __ldcg(p.r.ghit + threadIdx.x);
+        if (PHASE == SP_UPROJ) {
+            for (int i = threadIdx.x; i < T * K; i += blockDim.x) {
+                const int e = __ldcg(p.r.idx + i);
+                const int g = p.group[e];
+                sh.pgrp[i] = g < G ? g : 0;   // out-of-range labels were reported by the router
+                sh.pair_slot[i] = __ldcg(p.r.pair_slot + i);
+            }
+        }
+        __syncthreads();
+        if (threadIdx.x == 0) {
+            int n = 0;
+            for (int g = 0; g < G; ++g)
+                if (sh.hg[g] > 0) sh.hg[n++] = g;
+            sh.n_hit = n;
+        }
+    }
+    __syncthreads();
+}
+
+// ---------------------------------------------------------------------------
+// one kernel per phase (a router kernel ran before; routing published)
+// ---------------------------------------------------------------------------
+
+template <int PHASE, int FMT>
+__global__ void __launch_bounds__(kWThreads, 1) k_wstream(FwdParams p, WPlan pl, int cache_bytes) {
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 127) & ~(uintptr_t)127);
+    __shared__ StreamShared sh;
+    __shared__ ChunkInfo ci;
+    const int warp = threadIdx.x >> 5;
+    __half* cache = reinterpret_cast<__half*>(smem);
+    uint8_t* ring = smem + cache_bytes + (size_t)warp * kPD * kStepBytes;
+
+    // D runs right after the router kernel and waits for it first.  The
+    // later kernels read the routing before their own wait: their
+    // predecessor let them launch only after its own wait, so the router
+    // kernel had completed by then.
+    if (PHASE == SP_DPROJ) {
+        grid_dep_wait();
+        grid_dep_launch();
+    }
+    stage_published_routing<PHASE>(p, sh);
+    WPlan plan = pl;
+    plan.n_mats = phase_mats<PHASE>(sh);
+    phase_setup<PHASE, FMT>(p, sh, plan, cache_bytes, ci);
+    LoadCursor lc;
+    phase_prime<PHASE, FMT>(p, sh, plan, ci, ring, lc);
+    if (PHASE != SP_DPROJ) {
+        grid_dep_wait();
+        grid_dep_launch();
+    }
+    phase_fill<PHASE>(p, sh, ci, cache);
+    __syncthreads();
+    phase_run<PHASE, FMT>(p, sh, plan, ci, ring, cache, lc);
     cp_async_wait<0>();
 }
 
