@@ -326,7 +326,7 @@ def run_stack(args, wl, T, rank, world, local, dev_name, n_distinct=4):
     value = replica_throughput(world, T, K, ms_max)
     line = {"metric": "latent-MoE 48-layer stack tokens/s", "value": value, "unit": "tokens/s", "n_gpus": world,
             "steps": K, "warmup": W, "ms_per_step": ms_max / K, "higher_is_better": True, "scaling": "weak",
-            "vs_baseline": None, "dtype": "f16" if prefill else "f32", "data": "synthetic",
+            "vs_baseline": None, "dtype": "f16", "data": "synthetic",
             "config": {"workload": workload_desc(wl, T), "T": T, "layers": wl.n_layers,
                        "weights": f"{len(srcs)} seeded layers copied into {wl.n_layers} device buffers",
                        "l2": f"{wl.n_layers} layers x {devs[0].weight_bytes() / 1e9:.2f} GB resident, larger than L2"},

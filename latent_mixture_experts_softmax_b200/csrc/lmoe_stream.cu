@@ -127,38 +127,50 @@ __device__ __forceinline__ void tile_du(const uint8_t* q, const uint16_t* d, con
 // One 16-row NVFP4 tile in shared memory (codes [chunk][16 rows][16 B],
 // scales [chunk/2][16 rows][4 B]), chunks [c0, c1); the E4M3 scale is folded
 // into the fp16 operand (exact), the tensor scale is left to the caller.
+// Even and odd chunks accumulate separately so that consecutive MMAs do not
+// wait on each other; the two sums are added at the end.
+__device__ __forceinline__ void nvfp4_chunk(const uint8_t* q, const uint8_t* s, const __half* xs, int ld, int nt, int c,
+                                            float (&acc)[4]) {
+    const int lane = threadIdx.x & 31, g = lane >> 2, t = lane & 3;
+    const uint32_t wg = *reinterpret_cast<const uint32_t*>(q + ((size_t)c * 16 + g) * 16 + 4 * t);
+    const uint32_t wh = *reinterpret_cast<const uint32_t*>(q + ((size_t)c * 16 + g + 8) * 16 + 4 * t);
+    const uint32_t swg = *reinterpret_cast<const uint32_t*>(s + ((size_t)(c >> 1) * 16 + g) * 4);
+    const uint32_t swh = *reinterpret_cast<const uint32_t*>(s + ((size_t)(c >> 1) * 16 + g + 8) * 4);
+    const int sb = 2 * (c & 1) + (t >> 1);
+    uint32_t scg, sch;
+    {
+        uint32_t hg, hh;
+        asm("{\n\t.reg .b16 a, b;\n\tcvt.u16.u32 a, %2;\n\tcvt.u16.u32 b, %3;\n\t"
+            "cvt.rn.f16x2.e4m3x2 %0, a;\n\tcvt.rn.f16x2.e4m3x2 %1, b;\n\t}"
+            : "=r"(hg), "=r"(hh)
+            : "r"((swg >> (8 * sb)) & 0xFF), "r"((swh >> (8 * sb)) & 0xFF));
+        scg = (hg & 0xFFFF) | (hg << 16);
+        sch = (hh & 0xFFFF) | (hh << 16);
+    }
+    uint32_t a[4], b[4];
+    e2m1x8_to_f16x8(wg, a);
+    e2m1x8_to_f16x8(wh, b);
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+        a[j] = hmul2u(a[j], scg);
+        b[j] = hmul2u(b[j], sch);
+    }
+    const uint4 xv = act8(xs, ld, g, nt, c * 32 + 8 * t);
+    mma16816s(acc, a[0], b[0], a[1], b[1], xv.x, xv.y);
+    mma16816s(acc, a[2], b[2], a[3], b[3], xv.z, xv.w);
+}
+
 __device__ __forceinline__ void tile_nvfp4(const uint8_t* q, const uint8_t* s, const __half* xs, int ld, int nt,
                                            int c0, int c1, float (&acc)[4]) {
-    const int lane = threadIdx.x & 31, g = lane >> 2, t = lane & 3;
-#pragma unroll 2
-    for (int c = c0; c < c1; ++c) {
-        const uint32_t wg = *reinterpret_cast<const uint32_t*>(q + ((size_t)c * 16 + g) * 16 + 4 * t);
-        const uint32_t wh = *reinterpret_cast<const uint32_t*>(q + ((size_t)c * 16 + g + 8) * 16 + 4 * t);
-        const uint32_t swg = *reinterpret_cast<const uint32_t*>(s + ((size_t)(c >> 1) * 16 + g) * 4);
-        const uint32_t swh = *reinterpret_cast<const uint32_t*>(s + ((size_t)(c >> 1) * 16 + g + 8) * 4);
-        const int sb = 2 * (c & 1) + (t >> 1);
-        uint32_t scg, sch;
-        {
-            uint32_t hg, hh;
-            asm("{\n\t.reg .b16 a, b;\n\tcvt.u16.u32 a, %2;\n\tcvt.u16.u32 b, %3;\n\t"
-                "cvt.rn.f16x2.e4m3x2 %0, a;\n\tcvt.rn.f16x2.e4m3x2 %1, b;\n\t}"
-                : "=r"(hg), "=r"(hh)
-                : "r"((swg >> (8 * sb)) & 0xFF), "r"((swh >> (8 * sb)) & 0xFF));
-            scg = (hg & 0xFFFF) | (hg << 16);
-            sch = (hh & 0xFFFF) | (hh << 16);
-        }
-        uint32_t a[4], b[4];
-        e2m1x8_to_f16x8(wg, a);
-        e2m1x8_to_f16x8(wh, b);
-#pragma unroll
-        for (int j = 0; j < 4; ++j) {
-            a[j] = hmul2u(a[j], scg);
-            b[j] = hmul2u(b[j], sch);
-        }
-        const uint4 xv = act8(xs, ld, g, nt, c * 32 + 8 * t);
-        mma16816s(acc, a[0], b[0], a[1], b[1], xv.x, xv.y);
-        mma16816s(acc, a[2], b[2], a[3], b[3], xv.z, xv.w);
+    float acc2[4] = {0.f, 0.f, 0.f, 0.f};
+    int c = c0;
+    for (; c + 1 < c1; c += 2) {
+        nvfp4_chunk(q, s, xs, ld, nt, c, acc);
+        nvfp4_chunk(q, s, xs, ld, nt, c + 1, acc2);
     }
+    if (c < c1) nvfp4_chunk(q, s, xs, ld, nt, c, acc);
+#pragma unroll
+    for (int j = 0; j < 4; ++j) acc[j] += acc2[j];
 }
 
 // 16 rows of bf16 weights ([16][K] row-major) against fp16 activations,
