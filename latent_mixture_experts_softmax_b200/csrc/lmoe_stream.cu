@@ -726,9 +726,12 @@ static cudaError_t launch_dependent(Kern kern, dim3 grid, dim3 block, size_t sme
 // host side
 // ---------------------------------------------------------------------------
 
-// Reduction parts per tile of each phase: enough items for about one per
-// warp of the GPU (148 SMs x 16 warps) counting every matrix that may be
-// hit, without a part smaller than one step.
+// Reduction parts per tile of each phase.  Measured on B200: splitting a
+// tile's reduction over several warps (to have an item for every warp)
+// costs more in partial round trips and tickets than the parallelism
+// returns, so every tile is reduced by one warp (one part); U's tiles still
+// meet through a ticket, because the hit groups and the shared expert are
+// separate items of one output tile.
 struct WPlans {
     WPlan d, gu, dn, u;
     size_t part_floats, ticks;
@@ -739,12 +742,8 @@ static WPlan plan_for(int H, int L, int F, int Fs, int G, int n_mats_max) {
     WPlan w;
     w.tiles = stream_rows<PHASE>(H, L, F) / 16;
     w.n_mats = n_mats_max;
-    const int nb = PHASE == SP_DPROJ ? H / 32 : PHASE == SP_GATEUP ? L / 32 : PHASE == SP_DOWN ? F / 32 : L / 32;
-    int max_ks = (nb + step_blocks<PHASE, FMT>(false) - 1) / step_blocks<PHASE, FMT>(false);
-    if (PHASE == SP_UPROJ) max_ks = std::min(max_ks, (Fs / 32 + 1) / 2);
-    const int base = std::max(1, n_mats_max * w.tiles);
-    const int want = (148 * kWW + base - 1) / base;
-    w.ks = std::max(1, std::min({want, max_ks, 8}));
+    w.ks = 1;
+    (void)Fs;
     (void)G;
     return w;
 }
@@ -762,10 +761,8 @@ WPlans stream_plans(int H, int L, int F, int Fs, int G, int E, int K, int T, int
     P.gu = plan_for<SP_GATEUP, LMOE_Q8_0>(H, L, F, Fs, G, nu);
     P.dn = plan_for<SP_DOWN, LMOE_Q8_0>(H, L, F, Fs, G, nu);
     // partials (8 floats per lane, 32 lanes) and tickets, the largest phase
-    auto parts = [](const WPlan& w, bool all_parts_per_tile) {
-        return (size_t)w.n_mats * w.tiles * w.ks * (all_parts_per_tile ? 1 : 1);
-    };
-    P.part_floats = 256 * std::max({parts(P.d, false), parts(P.gu, false), parts(P.dn, false), parts(P.u, true)});
+    auto parts = [](const WPlan& w) { return (size_t)w.n_mats * w.tiles * w.ks; };
+    P.part_floats = 256 * std::max({parts(P.d), parts(P.gu), parts(P.dn), parts(P.u)});
     P.ticks = std::max({(size_t)P.d.n_mats * P.d.tiles, (size_t)P.gu.n_mats * P.gu.tiles, (size_t)P.dn.n_mats * P.dn.tiles,
                         (size_t)P.u.tiles});
     return P;
