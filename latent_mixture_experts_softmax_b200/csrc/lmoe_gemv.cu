@@ -102,7 +102,6 @@ __global__ void __launch_bounds__(256) k_router_shared(FwdParams p) {
         __shared__ StreamShared rsh;
         __shared__ uint8_t sgrp[kMaxExpertsTopk];
         for (int e = threadIdx.x; e < p.E; e += blockDim.x) sgrp[e] = p.group[e];
-        __syncthreads();
         route_in_cta(p, rsh, sgrp, true);
     } else {
         topk_and_buckets(p);

@@ -29,13 +29,11 @@ struct StreamShared {
     int slot_pair[kMaxPairs];
     int pair_slot[kMaxPairs];
     int gcnt[kMaxGroups];      // pairs per group
-    uint8_t pfirst[kMaxPairs]; // pair is the first of its expert
+    uint32_t emask[kMaxExpertsTopk / 32];  // experts selected by some pair
 };
 
 // ---------------------------------------------------------------------------
-// routing inside a kernel: every CTA derives the step's routing from the
-// router logits on its own (a few microseconds), so no kernel waits for a
-// single CTA to publish it
+// routing inside one CTA, from the router logits in global memory
 // ---------------------------------------------------------------------------
 
 // Order-preserving map of a float onto an unsigned integer (larger float,
@@ -62,42 +60,50 @@ static __device__ __forceinline__ uint64_t tree_max(const uint64_t (&pk)[N]) {
     return m[0];
 }
 
+static __device__ __forceinline__ uint64_t pack_logit(float l, int e) {
+    return ((uint64_t)order_key(l) << 32) | (uint32_t)~e;
+}
+
 // Softmax top-K of one token by one warp (section "Routing" of the teardown
-// article: softmax over the E logits, top-K, renormalise over the kept):
-// ties go to the lower expert index; w_k = exp(l_k - l_1) / sum over the
-// kept of exp(l_j - l_1).  Writes idx[0..K), w[0..K).  Each lane packs its
-// NV logits as (order key, ~index) words and keeps its best; a round is two
-// warp reductions over the lanes' bests (largest key, then the lowest index
-// holding it) and, in the winning lane, a tree maximum over what is left.
+// article: softmax over the E logits, top-K, renormalise over the kept).
+// A logit is packed as (order key, ~index), so the larger word is the larger
+// logit and, between equal logits, the lower expert index; the words of a
+// row are distinct.  Each lane keeps the largest of its NV words; a round
+// takes the warp's largest by a butterfly of shuffles, and the lane that
+// held it replaces its best by a tree maximum over what it has left.
+// w_k = exp(l_k - l_1) / sum over the kept of exp(l_j - l_1), the sum taken
+// in k order.  Writes idx[0..K), w[0..K).
 template <int NV>
 static __device__ void topk_row(const float* logits, int E, int K, int lane, int* idx, float* w) {
     uint64_t pk[NV];
 #pragma unroll
     for (int j = 0; j < NV; ++j) {
         const int e = lane + 32 * j;
-        pk[j] = e < E ? ((uint64_t)order_key(__ldcg(logits + e)) << 32) | (uint32_t)~e : 0ull;
+        pk[j] = e < E ? pack_logit(__ldcg(logits + e), e) : 0ull;
     }
-    uint64_t best = tree_max(pk);
-    float lmax = 0.f, denom = 0.f, my_l = 0.f;
-    int my_e = 0;
+    uint64_t best = tree_max(pk), mine = 0ull;
     for (int k = 0; k < K; ++k) {
-        const uint32_t key = (uint32_t)(best >> 32);
-        const uint32_t kmax = __reduce_max_sync(0xffffffffu, key);
-        const int bi = (int)__reduce_min_sync(0xffffffffu, key == kmax ? ~(uint32_t)best : 0xffffffffu);
-        const float bv = key_value(kmax);
-        if (~(uint32_t)best == (uint32_t)bi) {
+        uint64_t m = best;
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1) {
+            const uint64_t o = __shfl_xor_sync(0xffffffffu, m, off);
+            m = o > m ? o : m;
+        }
+        mine = k == lane ? m : mine;
+        if (m == best) {
+            const int jw = (int)(~(uint32_t)m) >> 5;
 #pragma unroll
             for (int j = 0; j < NV; ++j)
-                if (j == (bi >> 5)) pk[j] = 0ull;
+                if (j == jw) pk[j] = 0ull;
             best = tree_max(pk);
         }
-        if (k == 0) lmax = bv;
-        if (k == lane) { my_l = bv; my_e = bi; }
-        denom += expf(bv - lmax);
     }
+    const float lmax = key_value((uint32_t)(__shfl_sync(0xffffffffu, mine, 0) >> 32));
+    float denom = 0.f;
+    for (int k = 0; k < K; ++k) denom += expf(key_value((uint32_t)(__shfl_sync(0xffffffffu, mine, k) >> 32)) - lmax);
     if (lane < K) {
-        idx[lane] = my_e;
-        w[lane] = expf(my_l - lmax) / denom;
+        idx[lane] = (int)~(uint32_t)mine;
+        w[lane] = expf(key_value((uint32_t)(mine >> 32)) - lmax) / denom;
     }
 }
 
@@ -105,11 +111,11 @@ static __device__ void topk_row(const float* logits, int E, int K, int lane, int
 // shared memory: slots ordered by (expert, pair index), distinct experts
 // ascending, pairs per group.  `grp` is the expert -> group table (in shared
 // memory).  Invalid indices or labels are reported (report = true) and read
-// as 0.  Contains __syncthreads.
+// as 0.  sh.emask, sh.gcnt and sh.n_unique must be zero on entry (and that
+// ordered by a __syncthreads).  Contains __syncthreads.
 static __device__ void bucket_pairs(const FwdParams& p, StreamShared& sh, const uint8_t* grp, bool report) {
     const int K = p.K, G = p.G, E = p.E, n = p.T * K;
-    for (int g = threadIdx.x; g < G; g += blockDim.x) sh.gcnt[g] = 0;
-    if (threadIdx.x == 0) sh.n_unique = 0;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     for (int i = threadIdx.x; i < n; i += blockDim.x) {
         int e = sh.idx[i];
         if (e < 0 || e >= E) {
@@ -123,47 +129,47 @@ static __device__ void bucket_pairs(const FwdParams& p, StreamShared& sh, const 
         }
         sh.pe[i] = e;
         sh.pgrp[i] = g;
+        atomicOr(&sh.emask[e >> 5], 1u << (e & 31));
+        atomicAdd(&sh.gcnt[g], 1);
     }
     __syncthreads();
     for (int i = threadIdx.x; i < n; i += blockDim.x) {
         const int e = sh.pe[i];
-        bool first = true;
-#pragma unroll 8
-        for (int j = 0; j < i; ++j) first &= sh.pe[j] != e;
-        sh.pfirst[i] = first;
-    }
-    __syncthreads();
-    for (int i = threadIdx.x; i < n; i += blockDim.x) {
-        const int e = sh.pe[i];
-        int less = 0, same_before = 0, cnt = 0, u = 0;
+        int less = 0, same_before = 0, cnt = 0;
 #pragma unroll 8
         for (int j = 0; j < n; ++j) {
             const int ej = sh.pe[j];
             less += ej < e;
-            same_before += (j < i && ej == e);
+            same_before += (j < i) & (ej == e);
             cnt += ej == e;
-            u += (sh.pfirst[j] && ej < e);
         }
+        // distinct experts below e
+        int u = __popc(sh.emask[e >> 5] & ((1u << (e & 31)) - 1u));
+        for (int v = 0; v < (e >> 5); ++v) u += __popc(sh.emask[v]);
         const int slot = less + same_before;
         sh.slot_pair[slot] = i;
         sh.pair_slot[i] = slot;
         sh.slot_tok[slot] = i / K;
         sh.slot_w[slot] = sh.w[i];
-        if (sh.pfirst[i]) {
+        if (same_before == 0) {
             sh.uexp[u] = e;
             sh.ucnt[u] = cnt;
             sh.uoff[u] = less;
             sh.ugrp[u] = sh.pgrp[i];
             atomicAdd(&sh.n_unique, 1);
         }
-        atomicAdd(&sh.gcnt[sh.pgrp[i]], 1);
     }
-    __syncthreads();
-    if (threadIdx.x == 0) {
-        int nh = 0;
-        for (int g = 0; g < G; ++g)
-            if (sh.gcnt[g] > 0) sh.hg[nh++] = g;
-        sh.n_hit = nh;
+    // hit groups, ascending (warp 0, by ballots)
+    if (warp == 0) {
+        int base = 0;
+        for (int g0 = 0; g0 < G; g0 += 32) {
+            const int g = g0 + lane;
+            const bool hit = g < G && sh.gcnt[g] > 0;
+            const uint32_t bal = __ballot_sync(0xffffffffu, hit);
+            if (hit) sh.hg[base + __popc(bal & ((1u << lane) - 1u))] = g;
+            base += __popc(bal);
+        }
+        if (lane == 0) sh.n_hit = base;
     }
     __syncthreads();
 }
@@ -175,6 +181,9 @@ static __device__ void bucket_pairs(const FwdParams& p, StreamShared& sh, const 
 static __device__ void route_in_cta(const FwdParams& p, StreamShared& sh, const uint8_t* grp, bool publish) {
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int T = p.T, K = p.K, E = p.E, G = p.G, n = T * K;
+    for (int v = threadIdx.x; v < (E + 31) / 32; v += blockDim.x) sh.emask[v] = 0u;
+    for (int g = threadIdx.x; g < G; g += blockDim.x) sh.gcnt[g] = 0;
+    if (threadIdx.x == 0) sh.n_unique = 0;
     if (p.inject_idx != nullptr && p.inject_w != nullptr) {
         for (int i = threadIdx.x; i < n; i += blockDim.x) {
             sh.idx[i] = __ldg(p.inject_idx + i);

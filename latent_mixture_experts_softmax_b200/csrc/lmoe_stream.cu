@@ -12,7 +12,7 @@
 // the workspace and the warp that completes the tile (ticket) adds the
 // parts in order and runs the epilogue.
 //
-//   k_wstream<DPROJ>   h16[t][g]   = D_g x_t            (hit groups)
+//   k_wstream<DPROJ>   h16[t][g]   = D_g x_t            (every group)
 //   k_wstream<GATEUP>  z16[slot]   = silu(W_gate h) * (W_up h)
 //   k_wstream<DOWN>    o16w[slot]  = w_slot * W_down z
 //   k_wstream<UPROJ>   y           = sum_g U_g s[g][t] + S_down z_sh (+ residual), where
@@ -476,20 +476,70 @@ __device__ void phase_prime(const FwdParams& p, const StreamShared& sh, const WP
     for (int k = 0; k < kPD - 1; ++k) cursor_issue<PHASE, FMT>(p, sh, plan, ci, ring, c, lane);
 }
 
+// D's activations: the block input rows (bf16) as fp16, RMS-normalised
+// (gamma[k] x[k] / sqrt(mean(x^2) + eps), the stack's pre-norm) when gamma
+// is given.  D reads the input itself, so it depends on no earlier kernel
+// of the step.
+__device__ void fill_x(const FwdParams& p, __half* cache, int ld, float* rs) {
+    const int T = p.T, H = p.H, nc = H / 8;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    auto unpack = [](const uint4 v, float (&f)[8]) {
+        const uint32_t w4[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            const float2 q = bf16x2_to_f32x2(w4[j]);
+            f[2 * j] = q.x;
+            f[2 * j + 1] = q.y;
+        }
+    };
+    if (p.gamma != nullptr) {
+        for (int t = warp; t < T; t += blockDim.x >> 5) {
+            float ss = 0.f;
+            for (int c = lane; c < nc; c += 32) {
+                float f[8];
+                unpack(__ldg(reinterpret_cast<const uint4*>(p.x + (size_t)t * H) + c), f);
+#pragma unroll
+                for (int j = 0; j < 8; ++j) ss = fmaf(f[j], f[j], ss);
+            }
+            ss = warp_sum(ss);
+            if (lane == 0) rs[t] = rsqrtf(ss / (float)H + p.eps);
+        }
+        __syncthreads();
+    }
+    for (int i = threadIdx.x; i < T * nc; i += blockDim.x) {
+        const int t = i / nc, c = i - t * nc;
+        float f[8];
+        unpack(__ldg(reinterpret_cast<const uint4*>(p.x + (size_t)t * H) + c), f);
+        if (p.gamma != nullptr) {
+            float g[8];
+            unpack(__ldg(reinterpret_cast<const uint4*>(p.gamma) + c), g);
+#pragma unroll
+            for (int j = 0; j < 8; ++j) f[j] *= rs[t] * g[j];
+        }
+        __half2 h[4];
+#pragma unroll
+        for (int j = 0; j < 4; ++j) h[j] = __floats2half2_rn(f[2 * j], f[2 * j + 1]);
+        *reinterpret_cast<uint4*>(cache + (size_t)t * ld + 8 * c) = *reinterpret_cast<uint4*>(h);
+    }
+}
+
 // The chunk's activations from global memory, by plain loads of every thread.
 template <int PHASE>
 __device__ void phase_fill(const FwdParams& p, const StreamShared& sh, const ChunkInfo& ci, __half* cache) {
     const int T = p.T, H = p.H, L = p.L, F = p.F, Fs = p.Fs, K = p.K;
     const int ld = cache_ld<PHASE>(H, L, F, Fs);
+    if (PHASE == SP_DPROJ) {
+        __shared__ float rs[8];
+        if (ci.rows > 0) fill_x(p, cache, ld, rs);
+        return;
+    }
     const int KC = PHASE == SP_DPROJ ? H : PHASE == SP_GATEUP ? L : PHASE == SP_DOWN ? F : max(L, Fs);
     const int per = KC / 8;
     for (int qv = threadIdx.x; qv < ci.rows * per; qv += blockDim.x) {
         const int r = qv / per, c = qv - r * per;
         const int src = ci.src[r];
         uint4 v;
-        if (PHASE == SP_DPROJ) {
-            v = __ldcg(reinterpret_cast<const uint4*>(p.x16 + (size_t)src * H) + c);
-        } else if (PHASE == SP_GATEUP) {
+        if (PHASE == SP_GATEUP) {
             v = __ldcg(reinterpret_cast<const uint4*>(p.h16 + (size_t)src * L) + c);
         } else if (PHASE == SP_DOWN) {
             v = __ldcg(reinterpret_cast<const uint4*>(p.z16 + (size_t)src * F) + c);
@@ -621,6 +671,16 @@ __device__ void phase_run(const FwdParams& p, const StreamShared& sh, const WPla
     }
 }
 
+// D's matrices: every group, in order.  A few-token step hits nearly every
+// group (40 picks over 8 groups at 4 tokens), and h of a group no token hits
+// is never read, so D computes all of them and needs no routing: it runs
+// while the router kernel's last CTA is still routing.
+__device__ void stage_all_groups(const FwdParams& p, StreamShared& sh) {
+    for (int g = threadIdx.x; g < p.G; g += blockDim.x) sh.hg[g] = g;
+    if (threadIdx.x == 0) sh.n_hit = p.G;
+    __syncthreads();
+}
+
 // Routing tables of a later kernel, as the router kernel published them.
 template <int PHASE>
 __device__ void stage_published_routing(const FwdParams& p, StreamShared& sh) {
@@ -665,22 +725,22 @@ __device__ void stage_published_routing(const FwdParams& p, StreamShared& sh) {
 template <int PHASE, int FMT>
 __global__ void __launch_bounds__(kWThreads, 1) k_wstream(FwdParams p, WPlan pl, int cache_bytes) {
     extern __shared__ uint8_t smem_raw[];
-    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 127) & ~(uintptr_t)127);
+    // aligned by pointer arithmetic on the shared array, so that the compiler
+    // still knows every access through it is a shared-memory access
+    uint8_t* smem = smem_raw + ((128u - (smem_u32(smem_raw) & 127u)) & 127u);
     __shared__ StreamShared sh;
     __shared__ ChunkInfo ci;
     const int warp = threadIdx.x >> 5;
     __half* cache = reinterpret_cast<__half*>(smem);
     uint8_t* ring = smem + cache_bytes + (size_t)warp * kPD * kStepBytes;
 
-    // D runs right after the router kernel and waits for it first.  The
-    // later kernels read the routing before their own wait: their
-    // predecessor let them launch only after its own wait, so the router
-    // kernel had completed by then.
-    if (PHASE == SP_DPROJ) {
-        grid_dep_wait();
-        grid_dep_launch();
-    }
-    stage_published_routing<PHASE>(p, sh);
+    // D needs nothing from the router kernel and starts while it runs; it
+    // waits for it only at its end, so that D's completion implies the
+    // router kernel's.  The later kernels read the routing before their own
+    // wait: their predecessor let them launch only after its own wait, so
+    // the router kernel had completed by then.
+    if (PHASE == SP_DPROJ) stage_all_groups(p, sh);
+    else stage_published_routing<PHASE>(p, sh);
     WPlan plan = pl;
     plan.n_mats = phase_mats<PHASE>(sh);
     phase_setup<PHASE, FMT>(p, sh, plan, cache_bytes, ci);
@@ -694,6 +754,10 @@ __global__ void __launch_bounds__(kWThreads, 1) k_wstream(FwdParams p, WPlan pl,
     __syncthreads();
     phase_run<PHASE, FMT>(p, sh, plan, ci, ring, cache, lc);
     cp_async_wait<0>();
+    if (PHASE == SP_DPROJ) {
+        grid_dep_wait();
+        grid_dep_launch();
+    }
 }
 
 // ---------------------------------------------------------------------------
@@ -792,7 +856,9 @@ static cudaError_t launch_wstream(const FwdParams& p, const WPlan& plan, int cac
         cudaDeviceGetAttribute(&g_sms, cudaDevAttrMultiProcessorCount, dev);
     }
     stage_mark(st);
-    return launch_dependent(kern, dim3(g_sms), dim3(kWThreads), smem, st, p, plan, cache_bytes);
+    // D runs beside the router kernel's routing CTA, which keeps one SM
+    const int grid = PHASE == SP_DPROJ ? std::max(1, g_sms - 1) : g_sms;
+    return launch_dependent(kern, dim3(grid), dim3(kWThreads), smem, st, p, plan, cache_bytes);
 }
 
 // D, experts, combine, U for T <= 8 (the router kernel has run).

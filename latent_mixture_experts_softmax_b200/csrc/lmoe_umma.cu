@@ -430,7 +430,9 @@ __global__ void __launch_bounds__(kGemmThreads, 1) k_umma_gemm(const __grid_cons
     using S = Sched<KIND, NT>;
     using Plan = SmemPlan<NT, STAGES, RS>;
     extern __shared__ uint8_t smem_raw[];
-    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
+    // aligned by pointer arithmetic on the shared array, so that the compiler
+    // still knows every access through it is a shared-memory access
+    uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
     uint8_t* sA = smem;
     uint8_t* sB = smem + STAGES * Plan::kA;
     uint8_t* sRaw = sB + STAGES * Plan::kB;
