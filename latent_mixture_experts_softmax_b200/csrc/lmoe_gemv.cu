@@ -19,6 +19,8 @@
 // Edge0 145B / 120B model page, architecture tables (SwiGLU width 640, one
 // shared expert at full width, top-10 of 512).
 
+#include <algorithm>
+
 #include "lmoe_internal.cuh"
 #include "lmoe_route.cuh"
 #include "lmoe_rowdot.cuh"
@@ -42,6 +44,11 @@ __global__ void __launch_bounds__(256) k_router_shared(FwdParams p) {
     // the D_g kernel may launch now; it waits for this grid to complete
     asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
     if (!router_cta && !p.do_shared) return;
+    // expert -> group table, for the CTA that ends up routing (loaded while
+    // the logits are computed)
+    __shared__ uint8_t sgrp[kMaxExpertsTopk];
+    if (router_cta && p.route_smem)
+        for (int e = threadIdx.x; e < p.E; e += blockDim.x) sgrp[e] = p.group[e];
     if (p.prefetch_l2 && blockIdx.x == 0 && p.T <= kChunk)
         l2_prefetch_range(p.sd, (size_t)p.H * p.Fs * 2);
     for (int t0 = 0; t0 < p.T; t0 += NT) {
@@ -100,9 +107,8 @@ __global__ void __launch_bounds__(256) k_router_shared(FwdParams p) {
     __threadfence();
     if (p.route_smem) {
         __shared__ StreamShared rsh;
-        __shared__ uint8_t sgrp[kMaxExpertsTopk];
-        for (int e = threadIdx.x; e < p.E; e += blockDim.x) sgrp[e] = p.group[e];
-        route_in_cta(p, rsh, sgrp, true);
+        // the top-K scratch reuses the staged activations' space
+        route_in_cta(p, rsh, *reinterpret_cast<TopkScratch*>(smem), sgrp, true);
     } else {
         topk_and_buckets(p);
     }
@@ -877,7 +883,8 @@ static cudaError_t run_gemv_path_nt(FwdParams p, cudaStream_t st, bool route_onl
         if (e != cudaSuccess) return e;
     }
     {
-        const size_t sm = (size_t)xs_ld(p.H) * NT * sizeof(float);
+        size_t sm = (size_t)xs_ld(p.H) * NT * sizeof(float);
+        if (p.route_smem) sm = std::max(sm, sizeof(TopkScratch));
         cudaError_t e = p.router_bf16
             ? launch(k_router_shared<NT, true>, dim3(p.n_router_ctas + n_shared_ctas), 256, sm, st, p)
             : launch(k_router_shared<NT, false>, dim3(p.n_router_ctas + n_shared_ctas), 256, sm, st, p);

@@ -68,51 +68,75 @@ static __device__ __forceinline__ uint64_t pack_logit(float l, int e) {
 // article: softmax over the E logits, top-K, renormalise over the kept).
 // A logit is packed as (order key, ~index), so the larger word is the larger
 // logit and, between equal logits, the lower expert index; the words of a
-// row are distinct.  Each lane keeps the largest of its NV words; a round
-// takes the warp's largest by a butterfly of shuffles, and the lane that
-// held it replaces its best by a tree maximum over what it has left.
-// w_k = exp(l_k - l_1) / sum over the kept of exp(l_j - l_1), the sum taken
-// in k order.  Writes idx[0..K), w[0..K).
+// row are distinct.
+//  1. Each lane keeps NV words and their maximum.  tau = the K-th largest of
+//     the 32 lane maxima bounds the token's K largest words from below (the
+//     K largest lane maxima are K distinct words, all >= tau).
+//  2. The words >= tau (at most K * NV, typically a few more than K) are
+//     compacted into `cand`; a candidate's rank is the number of larger
+//     candidates, and the K of rank < K are the top K, in order.
+//  3. w_k = exp(l_k - l_1) / sum over the kept of exp(l_j - l_1), the sum
+//     taken in k order.
+// Writes idx[0..K), w[0..K); `cand` holds K * NV words, `sel` K.
 template <int NV>
-static __device__ void topk_row(const float* logits, int E, int K, int lane, int* idx, float* w) {
+static __device__ void topk_row(const float* logits, int E, int K, int lane, int* idx, float* w, uint64_t* cand,
+                                uint64_t* sel) {
     uint64_t pk[NV];
 #pragma unroll
     for (int j = 0; j < NV; ++j) {
         const int e = lane + 32 * j;
         pk[j] = e < E ? pack_logit(__ldcg(logits + e), e) : 0ull;
     }
-    uint64_t best = tree_max(pk), mine = 0ull;
-    for (int k = 0; k < K; ++k) {
-        uint64_t m = best;
+    const uint64_t lmx = tree_max(pk);
+    int r = 0;
 #pragma unroll
-        for (int off = 16; off > 0; off >>= 1) {
-            const uint64_t o = __shfl_xor_sync(0xffffffffu, m, off);
-            m = o > m ? o : m;
-        }
-        mine = k == lane ? m : mine;
-        if (m == best) {
-            const int jw = (int)(~(uint32_t)m) >> 5;
+    for (int l = 0; l < 32; ++l) r += __shfl_sync(0xffffffffu, lmx, l) > lmx;
+    const uint32_t bal = __ballot_sync(0xffffffffu, r == K - 1);
+    const uint64_t tau = __shfl_sync(0xffffffffu, lmx, __ffs(bal) - 1);
+    int c = 0;
 #pragma unroll
-            for (int j = 0; j < NV; ++j)
-                if (j == jw) pk[j] = 0ull;
-            best = tree_max(pk);
-        }
+    for (int j = 0; j < NV; ++j) c += pk[j] >= tau;
+    int pre = c;
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+        const int o = __shfl_up_sync(0xffffffffu, pre, off);
+        if (lane >= off) pre += o;
     }
-    const float lmax = key_value((uint32_t)(__shfl_sync(0xffffffffu, mine, 0) >> 32));
+    const int total = __shfl_sync(0xffffffffu, pre, 31);
+    pre -= c;
+#pragma unroll
+    for (int j = 0; j < NV; ++j)
+        if (pk[j] >= tau) cand[pre++] = pk[j];
+    __syncwarp();
+    for (int i = lane; i < total; i += 32) {
+        const uint64_t v = cand[i];
+        int rk = 0;
+        for (int j = 0; j < total; ++j) rk += cand[j] > v;
+        if (rk < K) sel[rk] = v;
+    }
+    __syncwarp();
+    const float lmax = key_value((uint32_t)(sel[0] >> 32));
     float denom = 0.f;
-    for (int k = 0; k < K; ++k) denom += expf(key_value((uint32_t)(__shfl_sync(0xffffffffu, mine, k) >> 32)) - lmax);
+    for (int k = 0; k < K; ++k) denom += expf(key_value((uint32_t)(sel[k] >> 32)) - lmax);
     if (lane < K) {
-        idx[lane] = (int)~(uint32_t)mine;
-        w[lane] = expf(key_value((uint32_t)(mine >> 32)) - lmax) / denom;
+        const uint64_t v = sel[lane];
+        idx[lane] = (int)~(uint32_t)v;
+        w[lane] = expf(key_value((uint32_t)(v >> 32)) - lmax) / denom;
     }
 }
+
+// Scratch of the top-K of up to 8 tokens.
+struct TopkScratch {
+    uint64_t cand[8][kMaxTopK * (kMaxExpertsTopk / 32)];
+    uint64_t sel[8][kMaxTopK];
+};
 
 // Bucketing of the T*K pairs by the whole CTA (one pair per thread), in
 // shared memory: slots ordered by (expert, pair index), distinct experts
 // ascending, pairs per group.  `grp` is the expert -> group table (in shared
 // memory).  Invalid indices or labels are reported (report = true) and read
-// as 0.  sh.emask, sh.gcnt and sh.n_unique must be zero on entry (and that
-// ordered by a __syncthreads).  Contains __syncthreads.
+// as 0.  sh.emask and sh.n_unique must be zero on entry (and that ordered by
+// a __syncthreads).  Contains __syncthreads.
 static __device__ void bucket_pairs(const FwdParams& p, StreamShared& sh, const uint8_t* grp, bool report) {
     const int K = p.K, G = p.G, E = p.E, n = p.T * K;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -130,9 +154,13 @@ static __device__ void bucket_pairs(const FwdParams& p, StreamShared& sh, const 
         sh.pe[i] = e;
         sh.pgrp[i] = g;
         atomicOr(&sh.emask[e >> 5], 1u << (e & 31));
-        atomicAdd(&sh.gcnt[g], 1);
     }
     __syncthreads();
+    for (int g = threadIdx.x; g < G; g += blockDim.x) {
+        int c = 0;
+        for (int i = 0; i < n; ++i) c += sh.pgrp[i] == g;
+        sh.gcnt[g] = c;
+    }
     for (int i = threadIdx.x; i < n; i += blockDim.x) {
         const int e = sh.pe[i];
         int less = 0, same_before = 0, cnt = 0;
@@ -159,6 +187,7 @@ static __device__ void bucket_pairs(const FwdParams& p, StreamShared& sh, const 
             atomicAdd(&sh.n_unique, 1);
         }
     }
+    __syncthreads();
     // hit groups, ascending (warp 0, by ballots)
     if (warp == 0) {
         int base = 0;
@@ -178,11 +207,11 @@ static __device__ void bucket_pairs(const FwdParams& p, StreamShared& sh, const 
 // __syncthreads); `grp` is the expert -> group table in shared memory.
 // With publish, also written to the workspace for the kernels that read it
 // and to the caller's routing outputs.
-static __device__ void route_in_cta(const FwdParams& p, StreamShared& sh, const uint8_t* grp, bool publish) {
+static __device__ void route_in_cta(const FwdParams& p, StreamShared& sh, TopkScratch& ts, const uint8_t* grp,
+                                    bool publish) {
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int T = p.T, K = p.K, E = p.E, G = p.G, n = T * K;
     for (int v = threadIdx.x; v < (E + 31) / 32; v += blockDim.x) sh.emask[v] = 0u;
-    for (int g = threadIdx.x; g < G; g += blockDim.x) sh.gcnt[g] = 0;
     if (threadIdx.x == 0) sh.n_unique = 0;
     if (p.inject_idx != nullptr && p.inject_w != nullptr) {
         for (int i = threadIdx.x; i < n; i += blockDim.x) {
@@ -192,10 +221,12 @@ static __device__ void route_in_cta(const FwdParams& p, StreamShared& sh, const 
     } else {
         for (int t = warp; t < T; t += blockDim.x >> 5) {
             const float* lg = p.r.logits + (size_t)t * E;
-            if (E <= 128) topk_row<4>(lg, E, K, lane, sh.idx + t * K, sh.w + t * K);
-            else if (E <= 256) topk_row<8>(lg, E, K, lane, sh.idx + t * K, sh.w + t * K);
-            else if (E <= 512) topk_row<16>(lg, E, K, lane, sh.idx + t * K, sh.w + t * K);
-            else topk_row<32>(lg, E, K, lane, sh.idx + t * K, sh.w + t * K);
+            int* ix = sh.idx + t * K;
+            float* wt = sh.w + t * K;
+            if (E <= 128) topk_row<4>(lg, E, K, lane, ix, wt, ts.cand[t], ts.sel[t]);
+            else if (E <= 256) topk_row<8>(lg, E, K, lane, ix, wt, ts.cand[t], ts.sel[t]);
+            else if (E <= 512) topk_row<16>(lg, E, K, lane, ix, wt, ts.cand[t], ts.sel[t]);
+            else topk_row<32>(lg, E, K, lane, ix, wt, ts.cand[t], ts.sel[t]);
         }
     }
     __syncthreads();

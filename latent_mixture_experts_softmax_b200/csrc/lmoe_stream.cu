@@ -362,6 +362,20 @@ __device__ __forceinline__ void compute_step(const FwdParams& p, const WItem& it
 template <int PHASE>
 __device__ __forceinline__ int n_steps(const WItem& it, int sb) { return (it.kb1 - it.kb0 + sb - 1) / sb; }
 
+// Steps of a phase's items in item order: items [0, nA) take nsA steps
+// each, the others nsB (U: the hit groups' matrices, then the shared
+// expert's); first(i) is item i's first step.  A CTA's steps are cut into
+// equal contiguous ranges, one per warp, so every warp streams the same
+// number of steps whatever the number of items.
+struct StepMap {
+    int nA, nsA, nsB;
+    __device__ __forceinline__ int first(int i) const { return i <= nA ? i * nsA : nA * nsA + (i - nA) * nsB; }
+    __device__ __forceinline__ int item(int st) const {
+        const int sA = nA * nsA;
+        return st < sA ? st / nsA : nA + (st - sA) / nsB;
+    }
+};
+
 // ---------------------------------------------------------------------------
 // one phase: chunk, activation cache, per-warp pipeline
 // ---------------------------------------------------------------------------
@@ -375,10 +389,12 @@ struct ChunkInfo {
     float tail[kMaxChunkParts][4];  // experts: tensor scales of gate, up, down
 };
 
-// One warp's load cursor over its items' steps.
+// One warp's load cursor over its range of steps.
 struct LoadCursor {
-    int li, ls, l_ns, n_issued;
-    WItem lit;
+    int st, s1;        // next step to issue, end of the range
+    int j, j0, j1;     // its item, the item's first step and end
+    int n_issued;
+    WItem it;
 };
 
 template <int PHASE>
@@ -442,38 +458,60 @@ __device__ void phase_setup(const FwdParams& p, const StreamShared& sh, const WP
 }
 
 template <int PHASE, int FMT>
-__device__ __forceinline__ void cursor_load_item(const FwdParams& p, const StreamShared& sh, const WPlan& plan,
-                                                 LoadCursor& c) {
-    c.lit = decode_item<PHASE, FMT>(p, sh, plan, c.li);
-    c.l_ns = n_steps<PHASE>(c.lit, step_blocks<PHASE, FMT>(PHASE == SP_UPROJ && c.lit.mat < 0));
+__device__ __forceinline__ StepMap step_map(const FwdParams& p, const StreamShared& sh, const WPlan& pl) {
+    const int nb = (PHASE == SP_DPROJ ? p.H : PHASE == SP_DOWN ? p.F : p.L) / 32;
+    const int sb = step_blocks<PHASE, FMT>(false);
+    StepMap m;
+    m.nsA = (nb + sb - 1) / sb;
+    if (PHASE == SP_UPROJ) {
+        m.nA = sh.n_hit * pl.tiles;
+        const int sbs = step_blocks<PHASE, FMT>(true);
+        m.nsB = (p.Fs / 32 + sbs - 1) / sbs;
+    } else {
+        m.nA = pl.n_mats * pl.tiles;
+        m.nsB = m.nsA;
+    }
+    return m;
 }
 
-// Issue the next step of the warp's stream (an empty commit group past its end).
+// First step of warp w's range in the CTA's chunk.
+__device__ __forceinline__ int range_start(const StepMap& m, const ChunkInfo& ci, int w) {
+    const int b = m.first(ci.i0), S = m.first(ci.i1) - b;
+    return b + (int)(((long long)w * S) / kWW);
+}
+
+// Issue the next step of the warp's range (an empty commit group past its end).
 template <int PHASE, int FMT>
 __device__ __forceinline__ void cursor_issue(const FwdParams& p, const StreamShared& sh, const WPlan& plan,
-                                             const ChunkInfo& ci, uint8_t* ring, LoadCursor& c, int lane) {
-    if (c.li < ci.i1) issue_step<PHASE, FMT>(p, c.lit, c.ls, ring + (size_t)(c.n_issued % kPD) * kStepBytes, lane);
+                                             const StepMap& m, uint8_t* ring, LoadCursor& c, int lane) {
+    if (c.st < c.s1) issue_step<PHASE, FMT>(p, c.it, c.st - c.j0, ring + (size_t)(c.n_issued % kPD) * kStepBytes, lane);
     cp_async_commit();
     ++c.n_issued;
-    if (c.li >= ci.i1) return;
-    if (++c.ls < c.l_ns) return;
-    c.ls = 0;
-    c.li += kWW;
-    if (c.li < ci.i1) cursor_load_item<PHASE, FMT>(p, sh, plan, c);
+    if (c.st >= c.s1) return;
+    if (++c.st == c.j1 && c.st < c.s1) {
+        ++c.j;
+        c.it = decode_item<PHASE, FMT>(p, sh, plan, c.j);
+        c.j0 = c.j1;
+        c.j1 = m.first(c.j + 1);
+    }
 }
 
 // The warp's first kPD - 1 steps (weights only: they depend on the routing).
 template <int PHASE, int FMT>
 __device__ void phase_prime(const FwdParams& p, const StreamShared& sh, const WPlan& plan, const ChunkInfo& ci,
-                            uint8_t* ring, LoadCursor& c) {
+                            const StepMap& m, uint8_t* ring, LoadCursor& c) {
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    c.li = ci.i0 + warp;
-    c.ls = 0;
-    c.l_ns = 0;
+    c.st = range_start(m, ci, warp);
+    c.s1 = range_start(m, ci, warp + 1);
     c.n_issued = 0;
-    if (c.li < ci.i1) cursor_load_item<PHASE, FMT>(p, sh, plan, c);
+    if (c.st < c.s1) {
+        c.j = m.item(c.st);
+        c.it = decode_item<PHASE, FMT>(p, sh, plan, c.j);
+        c.j0 = m.first(c.j);
+        c.j1 = m.first(c.j + 1);
+    }
 #pragma unroll
-    for (int k = 0; k < kPD - 1; ++k) cursor_issue<PHASE, FMT>(p, sh, plan, ci, ring, c, lane);
+    for (int k = 0; k < kPD - 1; ++k) cursor_issue<PHASE, FMT>(p, sh, plan, m, ring, c, lane);
 }
 
 // D's activations: the block input rows (bf16) as fp16, RMS-normalised
@@ -572,102 +610,148 @@ __device__ void phase_fill(const FwdParams& p, const StreamShared& sh, const Chu
     }
 }
 
-// The warp's items: stream, multiply, finish (epilogue, or partial + ticket).
+// An item's 16x8 result is complete: its epilogue, or (U, whose output tile
+// sums the hit groups' and the shared expert's items) its partial and, in
+// the warp that completes the tile (ticket), the ordered sum and epilogue.
+template <int PHASE, int FMT>
+__device__ __forceinline__ void item_finish(const FwdParams& p, const StreamShared& sh, const WPlan& plan,
+                                            const ChunkInfo& ci, const WItem& cit, float (&a)[4], float (&u)[4]) {
+    const int lane = threadIdx.x & 31;
+    const int T = p.T, H = p.H, L = p.L, F = p.F, G = p.G;
+    const int jj = cit.j - ci.m0;
+    const int nt = (PHASE == SP_GATEUP || PHASE == SP_DOWN) ? sh.ucnt[cit.j] : T;
+    const int gg = lane >> 2, tt = lane & 3;
+    const int nparts = PHASE == SP_UPROJ ? phase_mats<PHASE>(sh) * plan.ks : plan.ks;
+    bool finish = nparts == 1;
+    if (!finish) {
+        // partial of part (j, q) of tile (mat, tile); U: all matrices are parts of one tile
+        const int key = PHASE == SP_UPROJ ? cit.tile : cit.j * plan.tiles + cit.tile;
+        const int part = PHASE == SP_UPROJ ? cit.j * plan.ks + cit.q : cit.q;
+        float* dst = p.wpart + (((size_t)key * nparts + part) * 32 + lane) * 8;
+        *reinterpret_cast<float4*>(dst) = make_float4(a[0], a[1], a[2], a[3]);
+        if (PHASE == SP_GATEUP) *reinterpret_cast<float4*>(dst + 4) = make_float4(u[0], u[1], u[2], u[3]);
+        __threadfence();
+        __syncwarp();
+        int last = 0;
+        if (lane == 0) last = atomicAdd(p.wtick + key, 1) == nparts - 1;
+        last = __shfl_sync(0xffffffffu, last, 0);
+        if (last) {
+            __threadfence();
+            float sa[4] = {0.f, 0.f, 0.f, 0.f}, su[4] = {0.f, 0.f, 0.f, 0.f};
+            for (int q = 0; q < nparts; ++q) {
+                const float* sp = p.wpart + (((size_t)key * nparts + q) * 32 + lane) * 8;
+                const float4 v = __ldcg(reinterpret_cast<const float4*>(sp));
+                sa[0] += v.x; sa[1] += v.y; sa[2] += v.z; sa[3] += v.w;
+                if (PHASE == SP_GATEUP) {
+                    const float4 w4 = __ldcg(reinterpret_cast<const float4*>(sp + 4));
+                    su[0] += w4.x; su[1] += w4.y; su[2] += w4.z; su[3] += w4.w;
+                }
+            }
+#pragma unroll
+            for (int i4 = 0; i4 < 4; ++i4) { a[i4] = sa[i4]; u[i4] = su[i4]; }
+            if (lane == 0) p.wtick[key] = 0;
+            finish = true;
+        }
+    }
+    if (finish) {
+        const float* ts = (PHASE == SP_GATEUP || PHASE == SP_DOWN) ? ci.tail[jj] : nullptr;
+#pragma unroll
+        for (int i4 = 0; i4 < 4; ++i4) {
+            const int col = 2 * tt + (i4 & 1), row = cit.r0 + gg + 8 * (i4 >> 1);
+            if (col >= nt) continue;
+            if (PHASE == SP_DPROJ) {
+                p.h16[((size_t)col * G + cit.mat) * L + row] = __float2half_rn(a[i4]);
+            } else if (PHASE == SP_GATEUP) {
+                p.z16[(size_t)(sh.uoff[cit.j] + col) * F + row] = __float2half_rn(silu(a[i4] * ts[0]) * (u[i4] * ts[1]));
+            } else if (PHASE == SP_DOWN) {
+                const int slot = sh.uoff[cit.j] + col;
+                p.o16w[(size_t)slot * L + row] = __float2half_rn(sh.slot_w[slot] * ts[2] * a[i4]);
+            } else {
+                float v = a[i4];
+                if (p.residual) v += bf16_bits_to_f32(p.residual[(size_t)col * H + row]);
+                p.y[(size_t)col * H + row] = f32_to_bf16_bits(v);
+            }
+        }
+    }
+}
+
+// The warp's range of steps: stream, multiply, finish.  An item whose steps
+// all fall in the range is finished by the warp; an item cut by range
+// boundaries leaves one 16x8 partial per warp in shared memory (in the
+// warp's step ring, free once its range is done: slot 0 for the range's
+// first item, slot 1 for its last), and after a barrier the warp where the
+// item begins adds the partials in warp order (K order) and finishes it.
+// Contains __syncthreads.
 template <int PHASE, int FMT>
 __device__ void phase_run(const FwdParams& p, const StreamShared& sh, const WPlan& plan, const ChunkInfo& ci,
-                          uint8_t* ring, const __half* cache, LoadCursor& lc) {
+                          const StepMap& m, uint8_t* ring_base, const __half* cache, LoadCursor& lc) {
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int T = p.T, H = p.H, L = p.L, F = p.F, G = p.G;
+    const int T = p.T, H = p.H, L = p.L, F = p.F;
     const int ld = cache_ld<PHASE>(H, L, F, p.Fs);
-    const int n_mats = phase_mats<PHASE>(sh);
-    int cidx = ci.i0 + warp, cs = 0, c_nsteps = 0, n_done = 0;
-    WItem cit = {0, 0, 0, 0, 0, 0, 0};
-    if (cidx < ci.i1) {
-        cit = decode_item<PHASE, FMT>(p, sh, plan, cidx);
-        c_nsteps = n_steps<PHASE>(cit, step_blocks<PHASE, FMT>(PHASE == SP_UPROJ && cit.mat < 0));
-    }
+    uint8_t* ring = ring_base + (size_t)warp * kPD * kStepBytes;
+    const int s0 = range_start(m, ci, warp), s1 = range_start(m, ci, warp + 1);
     float a[4] = {0.f, 0.f, 0.f, 0.f}, u[4] = {0.f, 0.f, 0.f, 0.f};
-    const int gg = lane >> 2, tt = lane & 3;
-    while (cidx < ci.i1) {
-        cursor_issue<PHASE, FMT>(p, sh, plan, ci, ring, lc, lane);
-        cp_async_wait<kPD - 1>();
-        __syncwarp();
-        // activations of the item
+    float ha[4] = {0.f, 0.f, 0.f, 0.f}, hu[4] = {0.f, 0.f, 0.f, 0.f};
+    bool first_cut = false, last_cut = false;
+    int n_done = 0;
+    int st = s0;
+    while (st < s1) {
+        const int j = m.item(st);
+        const WItem cit = decode_item<PHASE, FMT>(p, sh, plan, j);
+        const int j0 = m.first(j), j1 = m.first(j + 1);
+        const int e = min(s1, j1);
         const int jj = cit.j - ci.m0;
-        const __half* xs;
-        int nt = T;
-        if (PHASE == SP_DPROJ) xs = cache;
-        else if (PHASE == SP_UPROJ) xs = cache + (size_t)ci.row0[jj] * ld;
-        else {
-            xs = cache + (size_t)ci.row0[jj] * ld;
-            nt = sh.ucnt[cit.j];
-        }
-        compute_step<PHASE, FMT>(p, cit, cs, ring + (size_t)(n_done % kPD) * kStepBytes, xs, ld, nt, a, u);
-        __syncwarp();
-        ++n_done;
-        if (++cs < c_nsteps) continue;
-
-        // ---- the item is complete: epilogue or partial
-        const int nparts = PHASE == SP_UPROJ ? n_mats * plan.ks : plan.ks;
-        bool finish = nparts == 1;
-        if (!finish) {
-            // partial of part (j, q) of tile (mat, tile); U: all matrices are parts of one tile
-            const int key = PHASE == SP_UPROJ ? cit.tile : cit.j * plan.tiles + cit.tile;
-            const int part = PHASE == SP_UPROJ ? cit.j * plan.ks + cit.q : cit.q;
-            float* dst = p.wpart + (((size_t)key * nparts + part) * 32 + lane) * 8;
-            *reinterpret_cast<float4*>(dst) = make_float4(a[0], a[1], a[2], a[3]);
-            if (PHASE == SP_GATEUP) *reinterpret_cast<float4*>(dst + 4) = make_float4(u[0], u[1], u[2], u[3]);
-            __threadfence();
+        const __half* xs = PHASE == SP_DPROJ ? cache : cache + (size_t)ci.row0[jj] * ld;
+        const int nt = (PHASE == SP_GATEUP || PHASE == SP_DOWN) ? sh.ucnt[cit.j] : T;
+        for (; st < e; ++st) {
+            cursor_issue<PHASE, FMT>(p, sh, plan, m, ring, lc, lane);
+            cp_async_wait<kPD - 1>();
             __syncwarp();
-            int last = 0;
-            if (lane == 0) last = atomicAdd(p.wtick + key, 1) == nparts - 1;
-            last = __shfl_sync(0xffffffffu, last, 0);
-            if (last) {
-                __threadfence();
-                float sa[4] = {0.f, 0.f, 0.f, 0.f}, su[4] = {0.f, 0.f, 0.f, 0.f};
-                for (int q = 0; q < nparts; ++q) {
-                    const float* sp = p.wpart + (((size_t)key * nparts + q) * 32 + lane) * 8;
-                    const float4 v = __ldcg(reinterpret_cast<const float4*>(sp));
-                    sa[0] += v.x; sa[1] += v.y; sa[2] += v.z; sa[3] += v.w;
-                    if (PHASE == SP_GATEUP) {
-                        const float4 w4 = __ldcg(reinterpret_cast<const float4*>(sp + 4));
-                        su[0] += w4.x; su[1] += w4.y; su[2] += w4.z; su[3] += w4.w;
-                    }
-                }
-#pragma unroll
-                for (int i4 = 0; i4 < 4; ++i4) { a[i4] = sa[i4]; u[i4] = su[i4]; }
-                if (lane == 0) p.wtick[key] = 0;
-                finish = true;
-            }
+            compute_step<PHASE, FMT>(p, cit, st - j0, ring + (size_t)(n_done % kPD) * kStepBytes, xs, ld, nt, a, u);
+            __syncwarp();
+            ++n_done;
         }
-        if (finish) {
-            const float* ts = (PHASE == SP_GATEUP || PHASE == SP_DOWN) ? ci.tail[jj] : nullptr;
+        if (j0 >= s0 && j1 <= s1) {
+            item_finish<PHASE, FMT>(p, sh, plan, ci, cit, a, u);
+        } else if (j0 < s0) {
+            first_cut = true;
 #pragma unroll
-            for (int i4 = 0; i4 < 4; ++i4) {
-                const int col = 2 * tt + (i4 & 1), row = cit.r0 + gg + 8 * (i4 >> 1);
-                if (col >= nt) continue;
-                if (PHASE == SP_DPROJ) {
-                    p.h16[((size_t)col * G + cit.mat) * L + row] = __float2half_rn(a[i4]);
-                } else if (PHASE == SP_GATEUP) {
-                    p.z16[(size_t)(sh.uoff[cit.j] + col) * F + row] = __float2half_rn(silu(a[i4] * ts[0]) * (u[i4] * ts[1]));
-                } else if (PHASE == SP_DOWN) {
-                    const int slot = sh.uoff[cit.j] + col;
-                    p.o16w[(size_t)slot * L + row] = __float2half_rn(sh.slot_w[slot] * ts[2] * a[i4]);
-                } else {
-                    float v = a[i4];
-                    if (p.residual) v += bf16_bits_to_f32(p.residual[(size_t)col * H + row]);
-                    p.y[(size_t)col * H + row] = f32_to_bf16_bits(v);
-                }
-            }
+            for (int i4 = 0; i4 < 4; ++i4) { ha[i4] = a[i4]; hu[i4] = u[i4]; }
+        } else {
+            last_cut = true;
+            break;
         }
 #pragma unroll
         for (int i4 = 0; i4 < 4; ++i4) { a[i4] = 0.f; u[i4] = 0.f; }
-        cs = 0;
-        cidx += kWW;
-        if (cidx < ci.i1) {
-            cit = decode_item<PHASE, FMT>(p, sh, plan, cidx);
-            c_nsteps = n_steps<PHASE>(cit, step_blocks<PHASE, FMT>(PHASE == SP_UPROJ && cit.mat < 0));
+    }
+    cp_async_wait<0>();
+    __syncwarp();
+    float* part = reinterpret_cast<float*>(ring);
+    if (first_cut) {
+        *reinterpret_cast<float4*>(part + lane * 8) = make_float4(ha[0], ha[1], ha[2], ha[3]);
+        if (PHASE == SP_GATEUP) *reinterpret_cast<float4*>(part + lane * 8 + 4) = make_float4(hu[0], hu[1], hu[2], hu[3]);
+    }
+    if (last_cut) {
+        *reinterpret_cast<float4*>(part + 256 + lane * 8) = make_float4(a[0], a[1], a[2], a[3]);
+        if (PHASE == SP_GATEUP) *reinterpret_cast<float4*>(part + 256 + lane * 8 + 4) = make_float4(u[0], u[1], u[2], u[3]);
+    }
+    __syncthreads();
+    if (last_cut) {
+        // the item begun here and continued by the next warps
+        const int j = m.item(s1 - 1);
+        const WItem cit = decode_item<PHASE, FMT>(p, sh, plan, j);
+        const int j1 = m.first(j + 1);
+        for (int w = warp + 1; w < kWW && range_start(m, ci, w) < j1; ++w) {
+            if (range_start(m, ci, w + 1) == range_start(m, ci, w)) continue;   // empty range
+            const float* q = reinterpret_cast<const float*>(ring_base + (size_t)w * kPD * kStepBytes) + lane * 8;
+            const float4 v = *reinterpret_cast<const float4*>(q);
+            a[0] += v.x; a[1] += v.y; a[2] += v.z; a[3] += v.w;
+            if (PHASE == SP_GATEUP) {
+                const float4 w4 = *reinterpret_cast<const float4*>(q + 4);
+                u[0] += w4.x; u[1] += w4.y; u[2] += w4.z; u[3] += w4.w;
+            }
         }
+        item_finish<PHASE, FMT>(p, sh, plan, ci, cit, a, u);
     }
 }
 
@@ -744,16 +828,16 @@ __global__ void __launch_bounds__(kWThreads, 1) k_wstream(FwdParams p, WPlan pl,
     WPlan plan = pl;
     plan.n_mats = phase_mats<PHASE>(sh);
     phase_setup<PHASE, FMT>(p, sh, plan, cache_bytes, ci);
+    const StepMap m = step_map<PHASE, FMT>(p, sh, plan);
     LoadCursor lc;
-    phase_prime<PHASE, FMT>(p, sh, plan, ci, ring, lc);
+    phase_prime<PHASE, FMT>(p, sh, plan, ci, m, ring, lc);
     if (PHASE != SP_DPROJ) {
         grid_dep_wait();
         grid_dep_launch();
     }
     phase_fill<PHASE>(p, sh, ci, cache);
     __syncthreads();
-    phase_run<PHASE, FMT>(p, sh, plan, ci, ring, cache, lc);
-    cp_async_wait<0>();
+    phase_run<PHASE, FMT>(p, sh, plan, ci, m, smem + cache_bytes, cache, lc);
     if (PHASE == SP_DPROJ) {
         grid_dep_wait();
         grid_dep_launch();
