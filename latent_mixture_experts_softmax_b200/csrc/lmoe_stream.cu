@@ -1,16 +1,18 @@
 // Few-token path (T <= 8), weight-streaming kernels.  One CTA per SM, 16
-// warps.  A work item is one 16-row tile of one matrix over one part of its
-// reduction (K); each warp streams its items' stored bytes (codes and
-// scales exactly as they sit in HBM) through its own ring of shared-memory
-// step buffers with per-thread asynchronous copies (cp.async, 16 bytes per
-// thread; the bulk-copy engine's fixed cost per copy would cap the rate),
-// dequantises in registers and multiplies on the tensor pipe (mma.sync
-// m16n8k16, fp16 operands, fp32 accumulation; the 8 MMA columns are the up
-// to 8 tokens).  Items are split into contiguous chunks per CTA; the
-// activations of a chunk are read once into a shared-memory cache.  When a
-// tile's reduction is split into parts, each part's 16x8 partial goes to
-// the workspace and the warp that completes the tile (ticket) adds the
-// parts in order and runs the epilogue.
+// warps.  A work item is one 16-row tile of one matrix over its reduction
+// (K), in steps of a few stored K blocks.  Items are split into contiguous
+// chunks per CTA, and a chunk's steps into equal contiguous ranges per warp;
+// each warp streams its range's stored bytes (codes and scales exactly as
+// they sit in HBM) through its own ring of shared-memory step buffers with
+// per-thread asynchronous copies (cp.async, 16 bytes per thread; the
+// bulk-copy engine's fixed cost per copy would cap the rate), dequantises in
+// registers and multiplies on the tensor pipe (mma.sync m16n8k16, fp16
+// operands, fp32 accumulation; the 8 MMA columns are the up to 8 tokens).
+// The activations of a chunk are read once into a shared-memory cache.  An
+// item cut by warp ranges is summed in shared memory, in K order; U's output
+// tiles, whose items (hit groups and the shared expert) sit in different
+// CTAs, meet in the workspace, and the warp that completes a tile (ticket)
+// adds the parts in order and runs the epilogue.
 //
 //   k_wstream<DPROJ>   h16[t][g]   = D_g x_t            (every group)
 //   k_wstream<GATEUP>  z16[slot]   = silu(W_gate h) * (W_up h)
