@@ -126,12 +126,13 @@ def step_cost(shape, idx: np.ndarray, groups: np.ndarray, T: int, prefill: bool)
     pairs_tg = sum(len({int(groups[e]) for e in idx[t]}) for t in range(idx.shape[0]))   # hit (token, group) pairs
     b = {
         "k_router_shared": rw + 2 * Fs * H * 2 + T * H * 2,
-        "k_wstream_dproj": len(hit) * du + T * H * 2,
+        "k_wstream_dproj": G * du + T * H * 2,     # every group (D runs before the routing is known)
         "k_wstream_gateup": len(distinct) * rec_gu,
         "k_wstream_down": len(distinct) * rec_d,
         "k_wstream_uproj": len(hit) * du + H * Fs * 2 + 2 * T * H * 2,
     }
-    b_total = float(sum(b.values()))
+    # the step's algorithmic bytes count only the hit groups' D
+    b_total = float(sum(b.values()) - (G - len(hit)) * du)
     f = {
         "x_to_fp16": 0.0,
         "router_gemm": 2.0 * T * E * H,
@@ -151,6 +152,15 @@ def step_cost(shape, idx: np.ndarray, groups: np.ndarray, T: int, prefill: bool)
     out["n_groups_hit"] = len(hit)
     return out
 
+
+# DRAM bytes per launch (dram__bytes_read.sum + dram__bytes_write.sum) of a
+# kernel, from one ncu capture (cold caches) of the current kernels on B200,
+# by (workload, T, kernel).  A kernel changed since its capture has no entry,
+# and its traffic is reported as null.
+NCU_TRAFFIC = {
+    ("edge0_120b_decode", 4, "k_router_shared"): 9.298176e6,
+    ("edge0_145b_prefill", 4096, "gateup"): 801.190656e6 + 51.464448e6,
+}
 
 STAGES = ["k_router_shared", "k_wstream_dproj", "k_wstream_gateup", "k_wstream_down", "k_wstream_uproj"]
 
@@ -479,11 +489,11 @@ def main():
         dom_ach = cost[dom_name] / dom_s / 1e12
         roof = {"bound": "tensor", "kernel": dom_name, "achieved": dom_ach, "peak": tc_peak, "unit": "TFLOP/s",
                 "frac": dom_ach / tc_peak, "peak_source": f"{peak_src} bf16 dense (fp16 operands run at the bf16 rate)",
-                "traffic": None}
+                "traffic": NCU_TRAFFIC.get((wl.name, T, dom_name))}
     else:
         dom_ach = cost[dom_name] / dom_s / 1e9
         roof = {"bound": "hbm", "kernel": dom_name, "achieved": dom_ach, "peak": hbm_peak, "unit": "GB/s",
-                "frac": dom_ach / hbm_peak, "peak_source": peak_src, "traffic": None}
+                "frac": dom_ach / hbm_peak, "peak_source": peak_src, "traffic": NCU_TRAFFIC.get((wl.name, T, dom_name))}
     t_step = ms_max / K / 1e3
     t_lb = max(step_alg_bytes / (hbm_peak * 1e9), step_flops / (tc_peak * 1e12))
 
