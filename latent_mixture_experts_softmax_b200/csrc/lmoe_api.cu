@@ -46,7 +46,8 @@ bool use_prefill(const lmoe_cfg& c, int T) {
 // Workspace of the few-token path (first) and of the tensor-core path; both
 // start after the control block, so one allocation serves either.
 struct WsLayout {
-    size_t ctrl, idx, w, logits, n_unique, uexp, ucnt, uoff, ugrp, slot_pair, pair_slot, ghit, tghit, wpart, wtick;
+    size_t ctrl, idx, w, logits, n_unique, uexp, ucnt, uoff, ugrp, slot_pair, pair_slot, slot_tok, slot_w, pgrp, ghit,
+        tghit, wpart, wtick;
     size_t wtick_bytes;
     size_t x16, h16, zsh, zsh16, o16w, z16, s16, ypart, xio, yio, xa, xb;
     // tensor-core path
@@ -84,6 +85,9 @@ WsLayout ws_layout(const lmoe_cfg& c, int T) {
         L.ugrp = take(TK * 4);
         L.slot_pair = take(TK * 4);
         L.pair_slot = take(TK * 4);
+        L.slot_tok = take(TK * 4);
+        L.slot_w = take(TK * 4);
+        L.pgrp = take(TK * 4);
         L.ghit = take((size_t)c.n_groups * 4);
         L.tghit = take((size_t)Td * c.n_groups);
         L.x16 = take((size_t)Td * c.hidden * 2);
@@ -156,6 +160,9 @@ FwdParams base_params(const lmoe_cfg& c, int T, void* ws, const WsLayout& L) {
     p.r.ugrp = reinterpret_cast<int32_t*>(b + L.ugrp);
     p.r.slot_pair = reinterpret_cast<int32_t*>(b + L.slot_pair);
     p.r.pair_slot = reinterpret_cast<int32_t*>(b + L.pair_slot);
+    p.r.slot_tok = reinterpret_cast<int32_t*>(b + L.slot_tok);
+    p.r.slot_w = reinterpret_cast<float*>(b + L.slot_w);
+    p.r.pgrp = reinterpret_cast<int32_t*>(b + L.pgrp);
     p.r.ghit = reinterpret_cast<int32_t*>(b + L.ghit);
     p.r.tghit = reinterpret_cast<uint8_t*>(b + L.tghit);
     p.x16 = reinterpret_cast<__half*>(b + L.x16);

@@ -132,6 +132,9 @@ struct Routing {
     int32_t* ugrp;       // [T*K]    group of each distinct expert (few-token path)
     int32_t* slot_pair;  // [T*K]    slot -> pair t*K + k (slots grouped by expert)
     int32_t* pair_slot;  // [T*K]    pair -> slot
+    int32_t* slot_tok;   // [T*K]    token of each slot (few-token path)
+    float* slot_w;       // [T*K]    routing weight of each slot (few-token path)
+    int32_t* pgrp;       // [T*K]    group of each pair (few-token path)
     int32_t* ghit;       // [G]      tokens hitting each group (any > 0 means hit)
     uint8_t* tghit;      // [T][G]   token t hits group g
 };

@@ -240,6 +240,9 @@ static __device__ void route_in_cta(const FwdParams& p, StreamShared& sh, TopkSc
         if (p.out_w) p.out_w[i] = sh.w[i];
         r.slot_pair[i] = sh.slot_pair[i];
         r.pair_slot[i] = sh.pair_slot[i];
+        r.slot_tok[i] = sh.slot_tok[i];
+        r.slot_w[i] = sh.slot_w[i];
+        r.pgrp[i] = sh.pgrp[i];
         if (i < sh.n_unique) {
             r.uexp[i] = sh.uexp[i];
             r.ucnt[i] = sh.ucnt[i];

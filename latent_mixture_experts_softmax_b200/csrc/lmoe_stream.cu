@@ -269,9 +269,8 @@ __device__ __forceinline__ WItem decode_item(const FwdParams& p, const StreamSha
     return it;
 }
 
-__device__ __forceinline__ int chunk_begin(int c, int n, int ctas) {
-    return (int)(((long long)c * n) / ctas);
-}
+// c * n stays far below 2^31 (at most 148 CTAs x a few thousand items)
+__device__ __forceinline__ int chunk_begin(int c, int n, int ctas) { return (c * n) / ctas; }
 
 __device__ __forceinline__ void cp_async16(void* dst, const void* src) {
     asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_u32(dst)), "l"(src) : "memory");
@@ -388,7 +387,7 @@ struct ChunkInfo {
     int m0, nm, rows, skip;      // first matrix, matrices, cached rows, refused
     int row0[kMaxChunkParts];    // first cache row of each matrix
     int src[kMaxChunkParts * 8]; // source of each cache row (phase-specific code)
-    float tail[kMaxChunkParts][4];  // experts: tensor scales of gate, up, down
+    alignas(16) float tail[kMaxChunkParts][4];  // experts: tensor scales of gate, up, down
 };
 
 // One warp's load cursor over its range of steps.
@@ -450,12 +449,16 @@ __device__ void phase_setup(const FwdParams& p, const StreamShared& sh, const WP
         ci.skip = !fits;
     }
     __syncthreads();
-    if ((PHASE == SP_GATEUP || PHASE == SP_DOWN) && threadIdx.x < 4 * ci.nm) {
-        const int jj = threadIdx.x >> 2, qq = threadIdx.x & 3;
-        const size_t nq = (size_t)p.L * p.F / 2, ns = (size_t)p.L * p.F / 16;
-        const float* tail =
-            reinterpret_cast<const float*>(p.experts + (size_t)sh.uexp[ci.m0 + jj] * p.rec_bytes + 3 * nq + 3 * ns);
-        ci.tail[jj][qq] = __ldg(tail + qq);
+    if ((PHASE == SP_GATEUP || PHASE == SP_DOWN) && (threadIdx.x >> 5) == kWW - 1) {
+        // the experts' tensor scales (16 bytes each), copied asynchronously by
+        // the last warp; it waits for them before the barrier that follows
+        // the activation fill
+        const int jj = threadIdx.x & 31;
+        if (jj < ci.nm) {
+            const size_t nq = (size_t)p.L * p.F / 2, ns = (size_t)p.L * p.F / 16;
+            cp_async16(&ci.tail[jj][0], p.experts + (size_t)sh.uexp[ci.m0 + jj] * p.rec_bytes + 3 * nq + 3 * ns);
+        }
+        cp_async_commit();
     }
 }
 
@@ -778,18 +781,15 @@ __device__ void stage_published_routing(const FwdParams& p, StreamShared& sh) {
             sh.ucnt[i] = __ldcg(p.r.ucnt + i);
             sh.uoff[i] = __ldcg(p.r.uoff + i);
             sh.ugrp[i] = __ldcg(p.r.ugrp + i);
-            const int pr = __ldcg(p.r.slot_pair + i);
-            sh.slot_tok[i] = pr / K;
-            sh.slot_w[i] = __ldcg(p.r.w + pr);
+            sh.slot_tok[i] = __ldcg(p.r.slot_tok + i);
+            sh.slot_w[i] = __ldcg(p.r.slot_w + i);
         }
         if (threadIdx.x == 0) sh.n_unique = __ldcg(p.r.n_unique);
     } else {
         if (threadIdx.x < G) sh.hg[threadIdx.x] = __ldcg(p.r.ghit + threadIdx.x);
         if (PHASE == SP_UPROJ) {
             for (int i = threadIdx.x; i < T * K; i += blockDim.x) {
-                const int e = __ldcg(p.r.idx + i);
-                const int g = p.group[e];
-                sh.pgrp[i] = g < G ? g : 0;   // out-of-range labels were reported by the router
+                sh.pgrp[i] = __ldcg(p.r.pgrp + i);
                 sh.pair_slot[i] = __ldcg(p.r.pair_slot + i);
             }
         }
@@ -838,6 +838,7 @@ __global__ void __launch_bounds__(kWThreads, 1) k_wstream(FwdParams p, WPlan pl,
         grid_dep_launch();
     }
     phase_fill<PHASE>(p, sh, ci, cache);
+    if ((PHASE == SP_GATEUP || PHASE == SP_DOWN) && warp == kWW - 1) cp_async_wait<kPD - 1>();   // tensor scales
     __syncthreads();
     phase_run<PHASE, FMT>(p, sh, plan, ci, m, smem + cache_bytes, cache, lc);
     if (PHASE == SP_DPROJ) {
