@@ -112,6 +112,33 @@ def test_block_one_hot_expert_and_unhit_groups():
     assert np.all(np.sort(out["idx_gpu"], axis=1) == np.arange(wl.shape.top_k))
 
 
+@pytest.mark.parametrize("T", [1, 8])
+def test_block_few_tokens_one_hot_expert_and_unhit_groups(T):
+    """The few-token path with every token on the same experts, all in one
+    group: the other groups' h is computed and never read, one expert holds
+    every token, and most warps of most CTAs get no steps."""
+    wl = small_workload(T)
+    layer = synth.make_layer(wl)
+    layer["router_b"] = np.full(wl.shape.n_experts, -50.0, np.float32)
+    layer["router_b"][:wl.shape.top_k] = 50.0 + np.arange(wl.shape.top_k, dtype=np.float32)
+    layer["expert_group"][:] = 0
+    layer["expert_group"][:wl.shape.top_k] = 2
+    out = check_block(wl.shape, layer, synth.make_x(wl), what=f"few-token one-hot T={T}")
+    assert np.all(np.sort(out["idx_gpu"], axis=1) == np.arange(wl.shape.top_k))
+
+
+@pytest.mark.parametrize("fmt,T", [(synth.Q8_0, 3), (synth.Q4_0, 7)])
+def test_block_few_tokens_ragged_steps(fmt, T):
+    """Few tokens with step counts that do not divide the reductions (down:
+    6 of 8 chunks in its only step) and a shared expert whose U items take
+    more steps than the groups' (5 against 2 or 3)."""
+    wl = small_workload(T, hidden=512, latent=384, n_experts=96, top_k=8, n_groups=6, ffn=192, shared_ffn=320,
+                        du_fmt=fmt)
+    layer = synth.make_layer(wl)
+    res = synth.bf16_normal(synth.key(2, 0, "residual"), 1.0, (T, wl.shape.hidden))
+    check_block(wl.shape, layer, synth.make_x(wl), residual_bits=res, what=f"ragged steps fmt={fmt} T={T}")
+
+
 def test_block_tiny_config():
     wl = synth.WORKLOADS["tiny"]
     check_block(wl.shape, synth.make_layer(wl), synth.make_x(wl), what="tiny")
