@@ -126,51 +126,59 @@ __device__ __forceinline__ void tile_du(const uint8_t* q, const uint16_t* d, con
     }
 }
 
-// One 16-row NVFP4 tile in shared memory (codes [chunk][16 rows][16 B],
-// scales [chunk/2][16 rows][4 B]), chunks [c0, c1); the E4M3 scale is folded
-// into the fp16 operand (exact), the tensor scale is left to the caller.
-// Even and odd chunks accumulate separately so that consecutive MMAs do not
-// wait on each other; the two sums are added at the end.
-__device__ __forceinline__ void nvfp4_chunk(const uint8_t* q, const uint8_t* s, const __half* xs, int ld, int nt, int c,
-                                            float (&acc)[4]) {
+// Four E4M3 scales (one stored word) -> two f16x2: bytes 0, 1 and bytes 2, 3.
+__device__ __forceinline__ void e4m3x4_to_f16x2x2(uint32_t w, uint32_t& lo, uint32_t& hi) {
+    asm("{\n\t.reg .b16 a, b;\n\tmov.b32 {a, b}, %2;\n\t"
+        "cvt.rn.f16x2.e4m3x2 %0, a;\n\tcvt.rn.f16x2.e4m3x2 %1, b;\n\t}"
+        : "=r"(lo), "=r"(hi)
+        : "r"(w));
+}
+
+// One 32-column NVFP4 chunk c of a 16-row tile: codes [chunk][16 rows][16 B];
+// sg / sh are the lane's E4M3 scales of rows g and g + 8 as f16x2 (both
+// halves equal), folded into the fp16 operand (exact); the tensor scale is
+// left to the caller.
+__device__ __forceinline__ void nvfp4_chunk_scaled(const uint8_t* q, const __half* xs, int ld, int nt, int c,
+                                                   uint32_t sg, uint32_t sh, float (&acc)[4]) {
     const int lane = threadIdx.x & 31, g = lane >> 2, t = lane & 3;
     const uint32_t wg = *reinterpret_cast<const uint32_t*>(q + ((size_t)c * 16 + g) * 16 + 4 * t);
     const uint32_t wh = *reinterpret_cast<const uint32_t*>(q + ((size_t)c * 16 + g + 8) * 16 + 4 * t);
-    const uint32_t swg = *reinterpret_cast<const uint32_t*>(s + ((size_t)(c >> 1) * 16 + g) * 4);
-    const uint32_t swh = *reinterpret_cast<const uint32_t*>(s + ((size_t)(c >> 1) * 16 + g + 8) * 4);
-    const int sb = 2 * (c & 1) + (t >> 1);
-    uint32_t scg, sch;
-    {
-        uint32_t hg, hh;
-        asm("{\n\t.reg .b16 a, b;\n\tcvt.u16.u32 a, %2;\n\tcvt.u16.u32 b, %3;\n\t"
-            "cvt.rn.f16x2.e4m3x2 %0, a;\n\tcvt.rn.f16x2.e4m3x2 %1, b;\n\t}"
-            : "=r"(hg), "=r"(hh)
-            : "r"((swg >> (8 * sb)) & 0xFF), "r"((swh >> (8 * sb)) & 0xFF));
-        scg = (hg & 0xFFFF) | (hg << 16);
-        sch = (hh & 0xFFFF) | (hh << 16);
-    }
     uint32_t a[4], b[4];
     e2m1x8_to_f16x8(wg, a);
     e2m1x8_to_f16x8(wh, b);
 #pragma unroll
     for (int j = 0; j < 4; ++j) {
-        a[j] = hmul2u(a[j], scg);
-        b[j] = hmul2u(b[j], sch);
+        a[j] = hmul2u(a[j], sg);
+        b[j] = hmul2u(b[j], sh);
     }
     const uint4 xv = act8(xs, ld, g, nt, c * 32 + 8 * t);
     mma16816s(acc, a[0], b[0], a[1], b[1], xv.x, xv.y);
     mma16816s(acc, a[2], b[2], a[3], b[3], xv.z, xv.w);
 }
 
+// One 16-row NVFP4 tile in shared memory (codes [chunk][16 rows][16 B],
+// scales [chunk/2][16 rows][4 B]: byte j of a row's word scales its 16-column
+// block j of the chunk pair), chunks [0, c1).  Chunks go in pairs (even,
+// odd) that share one scale word per row, converted once; lane t's columns
+// 8t..8t+7 of a chunk lie in the pair's block t/2 (even chunk) or 2 + t/2
+// (odd chunk).  Even and odd chunks accumulate separately so that
+// consecutive MMAs do not wait on each other; the two sums are added at the
+// end.
 __device__ __forceinline__ void tile_nvfp4(const uint8_t* q, const uint8_t* s, const __half* xs, int ld, int nt,
-                                           int c0, int c1, float (&acc)[4]) {
+                                           int c1, float (&acc)[4]) {
+    const int lane = threadIdx.x & 31, g = lane >> 2, t = lane & 3;
+    const uint32_t sel = (t >> 1) ? 0x3232u : 0x1010u;   // duplicate the high / low half
     float acc2[4] = {0.f, 0.f, 0.f, 0.f};
-    int c = c0;
-    for (; c + 1 < c1; c += 2) {
-        nvfp4_chunk(q, s, xs, ld, nt, c, acc);
-        nvfp4_chunk(q, s, xs, ld, nt, c + 1, acc2);
+    for (int c = 0; c < c1; c += 2) {
+        const uint32_t swg = *reinterpret_cast<const uint32_t*>(s + ((size_t)(c >> 1) * 16 + g) * 4);
+        const uint32_t swh = *reinterpret_cast<const uint32_t*>(s + ((size_t)(c >> 1) * 16 + g + 8) * 4);
+        uint32_t g01, g23, h01, h23;
+        e4m3x4_to_f16x2x2(swg, g01, g23);
+        e4m3x4_to_f16x2x2(swh, h01, h23);
+        nvfp4_chunk_scaled(q, xs, ld, nt, c, __byte_perm(g01, 0u, sel), __byte_perm(h01, 0u, sel), acc);
+        if (c + 1 < c1)
+            nvfp4_chunk_scaled(q, xs, ld, nt, c + 1, __byte_perm(g23, 0u, sel), __byte_perm(h23, 0u, sel), acc2);
     }
-    if (c < c1) nvfp4_chunk(q, s, xs, ld, nt, c, acc);
 #pragma unroll
     for (int j = 0; j < 4; ++j) acc[j] += acc2[j];
 }
@@ -353,10 +361,10 @@ __device__ __forceinline__ void compute_step(const FwdParams& p, const WItem& it
     } else if (PHASE == SP_UPROJ) {
         tile_bf16(reinterpret_cast<const uint16_t*>(buf), 64, x, ld, nt, 0, nblk, a);
     } else if (PHASE == SP_GATEUP) {
-        tile_nvfp4(buf, buf + 2 * 1024, x, ld, nt, 0, nblk, a);
-        tile_nvfp4(buf + 1024, buf + 2 * 1024 + 128, x, ld, nt, 0, nblk, u);
+        tile_nvfp4(buf, buf + 2 * 1024, x, ld, nt, nblk, a);
+        tile_nvfp4(buf + 1024, buf + 2 * 1024 + 128, x, ld, nt, nblk, u);
     } else {
-        tile_nvfp4(buf, buf + 2048, x, ld, nt, 0, nblk, a);
+        tile_nvfp4(buf, buf + 2048, x, ld, nt, nblk, a);
     }
 }
 
