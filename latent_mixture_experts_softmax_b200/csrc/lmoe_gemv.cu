@@ -77,8 +77,7 @@ __global__ void __launch_bounds__(256) k_router_shared(FwdParams p) {
                 float a[NT], u[NT];
 #pragma unroll
                 for (int t = 0; t < NT; ++t) { a[t] = 0.f; u[t] = 0.f; }
-                row_dot<NT, true>(p.sg + (size_t)f * H, H, xs, xs_ld(H), lane, a);
-                row_dot<NT, true>(p.su + (size_t)f * H, H, xs, xs_ld(H), lane, u);
+                row_dot2_bf16<NT>(p.sg + (size_t)f * H, p.su + (size_t)f * H, H, xs, xs_ld(H), lane, a, u);
 #pragma unroll
                 for (int t = 0; t < NT; ++t) {
                     const float av = warp_sum(a[t]), uv = warp_sum(u[t]);
@@ -875,6 +874,8 @@ static cudaError_t run_gemv_path_nt(FwdParams p, cudaStream_t st, bool route_onl
     // few tokens, whole block: the routing is built in shared memory and
     // published with every table the weight-streaming kernels read
     p.route_smem = !route_only && p.T <= 8;
+    // the weight-streaming kernels read the block input themselves
+    if (p.route_smem) p.x16 = nullptr;
     p.prefetch_l2 = false;
     const int n_shared_ctas = route_only ? 0 : (p.Fs + 7) / 8;
     if (p.route_smem && p.wtick) {

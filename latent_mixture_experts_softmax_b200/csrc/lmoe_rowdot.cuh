@@ -160,4 +160,31 @@ __device__ __forceinline__ void row_dot(const void* wrow, int K, const float* xs
     }
 }
 
+// Two rows of plain bf16 matrices (K contiguous) against xs, as row_dot:
+// both rows' loads are issued before any arithmetic.
+template <int NT, int kB = 10>
+__device__ __forceinline__ void row_dot2_bf16(const uint16_t* ra, const uint16_t* rb, int K, const float* xs, int ld,
+                                              int lane, float (&acc_a)[NT], float (&acc_b)[NT]) {
+    constexpr int kStep = 32 * 8;
+    for (int base = 0; base < K; base += kB * kStep) {
+        uint4 wa[kB], wb[kB];
+#pragma unroll
+        for (int i = 0; i < kB; ++i) {
+            const int k0 = base + i * kStep + lane * 8;
+            if (k0 < K) {
+                wa[i] = ldg_stream(reinterpret_cast<const uint4*>(ra + k0));
+                wb[i] = ldg_stream(reinterpret_cast<const uint4*>(rb + k0));
+            }
+        }
+#pragma unroll
+        for (int i = 0; i < kB; ++i) {
+            const int k0 = base + i * kStep + lane * 8;
+            if (k0 < K) {
+                dot8_bf16<NT>(wa[i], xs, ld, k0, acc_a);
+                dot8_bf16<NT>(wb[i], xs, ld, k0, acc_b);
+            }
+        }
+    }
+}
+
 }  // namespace lmoe
