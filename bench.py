@@ -158,7 +158,7 @@ def step_cost(shape, idx: np.ndarray, groups: np.ndarray, T: int, prefill: bool)
 # by (workload, T, kernel).  A kernel changed since its capture has no entry,
 # and its traffic is reported as null.
 NCU_TRAFFIC = {
-    ("edge0_120b_decode", 4, "k_router_shared"): 9.298432e6,
+    ("edge0_120b_decode", 4, "k_router_shared"): 9.297408e6,
     ("edge0_145b_prefill", 4096, "gateup"): 801.190656e6 + 51.464448e6,
 }
 
