@@ -40,7 +40,7 @@ enum StreamPhase { SP_DPROJ = 0, SP_GATEUP = 1, SP_DOWN = 2, SP_UPROJ = 3 };
 
 constexpr int kWW = 16;                     // warps per CTA
 constexpr int kWThreads = 32 * kWW;
-constexpr int kPD = 4;                      // step buffers per warp (3 steps in flight)
+constexpr int kPD = 3;                      // step buffers per warp (2 steps in flight)
 constexpr int kStepBytes = 2304;            // largest step (see step_geom)
 constexpr int kMaxChunkParts = 8;           // distinct matrices in one CTA's chunk
 constexpr int kActPad = 32;                 // halves of padding per cached activation row
