@@ -238,16 +238,14 @@ struct WItem {
 };
 
 struct WPlan {
-    int ks;        // reduction parts per tile
+    int ks;        // reduction parts per tile (1: a tile's K is cut only between warps)
     int tiles;     // output tiles per matrix
-    int n_mats;    // matrices (D: hit groups; experts; U: hit groups + shared)
+    int n_mats;    // matrices (D: every group; experts; U: hit groups + shared)
 };
 
 // Items run matrix-major (consecutive items share a matrix, so a CTA's chunk
-// touches few of them), then reduction part, then tile: the warps of a CTA
-// work on neighbouring row tiles of the same K blocks at the same time, so
-// together they read long contiguous runs of each stored K block (one
-// tile's 16 rows are only 256-512 bytes of it).
+// touches few of them and caches few activation rows), then reduction part,
+// then tile.
 template <int PHASE, int FMT>
 __device__ __forceinline__ WItem decode_item(const FwdParams& p, const StreamShared& sh, const WPlan& pl, int i) {
     WItem it;
