@@ -52,6 +52,7 @@ def lib():
         L.lmoe_synth_uniform.argtypes = [u64, u64]
         L.lmoe_synth_bf16.argtypes = [u64, dbl, vp, i64]
         L.lmoe_synth_f32.argtypes = [u64, dbl, vp, i64]
+        L.lmoe_synth_f64.argtypes = [u64, dbl, vp, i64]
         L.lmoe_synth_groups_uniform.argtypes = [u64, i32, i32, vp]
         L.lmoe_synth_q8_0.argtypes = [u64, dbl, i32, i32, vp]
         L.lmoe_synth_q4_0.argtypes = [u64, dbl, i32, i32, vp]
@@ -164,6 +165,20 @@ def f32_normal(k: int, sigma: float, shape) -> np.ndarray:
     out = np.empty(shape, np.float32)
     lib().lmoe_synth_f32(k, sigma, _p(out), out.size)
     return out
+
+
+def f64_normal(k: int, sigma: float, shape) -> np.ndarray:
+    """The unrounded draws sigma * normal(k, i) behind every generated tensor
+    (element i in row-major order)."""
+    out = np.empty(shape, np.float64)
+    lib().lmoe_synth_f64(k, sigma, _p(out), out.size)
+    return out
+
+
+def expert_key(k: int, e: int, m: int) -> int:
+    """Key of matrix m (0 gate, 1 up, 2 down) of expert e in experts_normal(k, ...)."""
+    L = lib()
+    return L.lmoe_synth_key(L.lmoe_synth_key(k, e), m)
 
 
 def qmatrix(fmt: int, k: int, sigma: float, rows: int, cols: int) -> np.ndarray:

@@ -131,6 +131,11 @@ void lmoe_synth_bf16(uint64_t key, double sigma, uint16_t* out, int64_t n) {
     for (int64_t i = 0; i < n; ++i) out[i] = f32_to_bf16_rne((float)(sigma * lmoe_synth_normal(key, (uint64_t)i)));
 }
 
+void lmoe_synth_f64(uint64_t key, double sigma, double* out, int64_t n) {
+#pragma omp parallel for schedule(static)
+    for (int64_t i = 0; i < n; ++i) out[i] = sigma * lmoe_synth_normal(key, (uint64_t)i);
+}
+
 void lmoe_synth_f32(uint64_t key, double sigma, float* out, int64_t n) {
 #pragma omp parallel for schedule(static)
     for (int64_t i = 0; i < n; ++i) out[i] = (float)(sigma * lmoe_synth_normal(key, (uint64_t)i));

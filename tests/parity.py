@@ -7,7 +7,7 @@ import torch
 
 from latent_mixture_experts_softmax_b200 import synth
 from latent_mixture_experts_softmax_b200.layer import DeviceLayer, to_device
-from oracle import lmoe_oracle as orc
+from oracle import native as orc
 
 # Tolerance of the block's output for bf16 activations with fp32 accumulation:
 # relative L2 error and the largest error relative to the output's RMS.

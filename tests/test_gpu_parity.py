@@ -6,7 +6,7 @@ import torch
 from latent_mixture_experts_softmax_b200 import binding as B
 from latent_mixture_experts_softmax_b200 import build, synth
 from latent_mixture_experts_softmax_b200.layer import DeviceLayer, to_device
-from oracle import lmoe_oracle as orc
+from oracle import native as orc
 
 from parity import GAP, check_block, check_routing, small_workload, assert_close, bf16_bits_to_f64
 

@@ -8,10 +8,18 @@ import numpy as np
 import pytest
 import torch
 
-from oracle import lmoe_oracle as orc
+from oracle import lmoe_oracle as np_oracle
+from oracle import native as cpp_oracle
 from latent_mixture_experts_softmax_b200 import synth
 
 GOLD = os.path.join(os.path.dirname(__file__), "golden")
+
+
+@pytest.fixture(params=["cpp", "numpy"])
+def orc(request):
+    """Every pin runs against both oracles: the C++ one (used by the parity
+    tests and the CPU baseline) and the numpy one (a second witness)."""
+    return cpp_oracle if request.param == "cpp" else np_oracle
 
 
 def _gold(name):
@@ -23,7 +31,7 @@ def _gold(name):
 # storage formats: byte totals the pages print
 # ----------------------------------------------------------------------------
 
-def test_record_and_build_sizes_match_pages():
+def test_record_and_build_sizes_match_pages(orc):
     g = _gold("page_figures.json")
     H, E, G, F, NL = (g[k]["value"] for k in ("hidden", "experts_per_layer", "groups", "swiglu_width", "layers"))
     L145, L120 = g["latent_145b"]["value"], g["latent_120b"]["value"]
@@ -53,14 +61,14 @@ def test_record_and_build_sizes_match_pages():
 # scalar formats against library conversions and the spec table
 # ----------------------------------------------------------------------------
 
-def test_e2m1_all_codes_match_spec_table():
+def test_e2m1_all_codes_match_spec_table(orc):
     want = np.array(_gold("e2m1_values.json")["values"])
     got = orc.e2m1_to_f64(np.arange(16))
     np.testing.assert_array_equal(got, want)
     assert np.all(np.signbit(got[8:]))
 
 
-def test_e4m3fn_all_codes_match_torch():
+def test_e4m3fn_all_codes_match_torch(orc):
     codes = torch.arange(256, dtype=torch.int32).to(torch.uint8)
     ref = codes.view(torch.float8_e4m3fn).to(torch.float64).numpy()
     got = orc.e4m3fn_to_f64(np.arange(256))
@@ -71,7 +79,7 @@ def test_e4m3fn_all_codes_match_torch():
     assert got[0x7E] == 448.0 and got[0x01] == 2.0 ** -9 and got[0x08] == 2.0 ** -6
 
 
-def test_fp16_all_codes_match_numpy():
+def test_fp16_all_codes_match_numpy(orc):
     codes = np.arange(65536, dtype=np.uint32).astype(np.uint16)
     ref = codes.view(np.float16).astype(np.float64)
     got = orc.fp16_to_f64(codes)
@@ -80,7 +88,7 @@ def test_fp16_all_codes_match_numpy():
     np.testing.assert_array_equal(got[~nan], ref[~nan])
 
 
-def test_bf16_matches_torch():
+def test_bf16_matches_torch(orc):
     rng = np.random.default_rng(3)
     codes = rng.integers(0, 65536, size=20000).astype(np.uint16)
     codes = codes[((codes >> 7) & 0xFF) != 0xFF]        # finite values only
@@ -96,7 +104,7 @@ def _fp16_bits(v):
     return int(np.array([v], np.float16).view(np.uint16)[0])
 
 
-def test_decode_q8_0_hand_packed():
+def test_decode_q8_0_hand_packed(orc):
     R, C = 3, 96
     rng = np.random.default_rng(1)
     q = rng.integers(-127, 128, size=(R, C))
@@ -116,7 +124,7 @@ def test_decode_q8_0_hand_packed():
     np.testing.assert_array_equal(got, want)
 
 
-def test_decode_q4_0_hand_packed():
+def test_decode_q4_0_hand_packed(orc):
     R, C = 2, 64
     rng = np.random.default_rng(2)
     q = rng.integers(0, 16, size=(R, C))
@@ -140,7 +148,7 @@ def test_decode_q4_0_hand_packed():
     np.testing.assert_array_equal(got, want)
 
 
-def test_decode_nvfp4_hand_packed():
+def test_decode_nvfp4_hand_packed(orc):
     R, C = 3, 128
     rng = np.random.default_rng(4)
     codes = rng.integers(0, 16, size=(R, C))
@@ -163,7 +171,7 @@ def test_decode_nvfp4_hand_packed():
     np.testing.assert_array_equal(got, want)
 
 
-def test_generator_round_trip_within_quantisation_error():
+def test_generator_round_trip_within_quantisation_error(orc):
     """Bytes from the generator decode to the matrix it was asked to encode,
     within each format's rounding step."""
     rng = np.random.default_rng(5)
@@ -197,7 +205,7 @@ def _brute_route(logits_row, K):
     return sel, [v / tot for v in ex]
 
 
-def test_route_matches_full_sort_and_closed_form_weights():
+def test_route_matches_full_sort_and_closed_form_weights(orc):
     rng = np.random.default_rng(7)
     T, E, H, K = 6, 40, 32, 10
     x = rng.normal(size=(T, H))
@@ -214,7 +222,7 @@ def test_route_matches_full_sort_and_closed_form_weights():
         assert abs(gap[t] - (srt[K - 1] - srt[K])) < 1e-12
 
 
-def test_route_ties_lowest_index_and_bias_moves_selection():
+def test_route_ties_lowest_index_and_bias_moves_selection(orc):
     E, K = 8, 3
     x = np.zeros((1, 4))
     Wr = np.zeros((E, 4))
@@ -226,7 +234,22 @@ def test_route_ties_lowest_index_and_bias_moves_selection():
     np.testing.assert_allclose(w[0], [e2 / (e2 + 2 * e1), e1 / (e2 + 2 * e1), e1 / (e2 + 2 * e1)], rtol=1e-14)
 
 
-def test_route_permutation_invariance():
+def test_route_many_ties_lowest_index_wins(orc):
+    """Hundreds of experts sharing a few logit values: the kept experts are
+    the first K of a full sort by (logit descending, index ascending)."""
+    rng = np.random.default_rng(12)
+    E, K, T = 300, 10, 4
+    x = np.zeros((T, 2))
+    Wr = np.zeros((E, 2))
+    for t in range(T):
+        b = rng.choice([0.0, 0.5, 1.0], size=E, p=[0.5, 0.3, 0.2])
+        idx, w, gap, _ = orc.route(x[t:t + 1], Wr, b, K)
+        want, ws = _brute_route(b.tolist(), K)
+        assert list(idx[0]) == want
+        np.testing.assert_allclose(w[0], ws, rtol=1e-14)
+
+
+def test_route_permutation_invariance(orc):
     rng = np.random.default_rng(8)
     T, E, H, K = 5, 32, 16, 4
     x = rng.normal(size=(T, H))
@@ -258,7 +281,7 @@ def _t(a):
 
 
 @pytest.mark.parametrize("fmt", [synth.Q8_0, synth.Q4_0])
-def test_block_equals_dense_masked_brute_force(fmt):
+def test_block_equals_dense_masked_brute_force(orc, fmt):
     wl, layer, xb = _tiny_layer(fmt=fmt)
     s = wl.shape
     y, idx, w, _ = orc.latent_moe_forward(s, layer, xb)
@@ -294,24 +317,29 @@ def test_block_equals_dense_masked_brute_force(fmt):
     np.testing.assert_allclose(M.numpy()[np.arange(T)[:, None], idx], w, rtol=1e-12)
 
 
-def test_block_linearity_of_U():
-    """U_g applied to the per-group sum equals the sum of U_g applied to each weighted expert output."""
+def test_block_linearity_of_U(orc):
+    """U_g applied to the per-group sum equals the sum of U_g applied to each
+    weighted expert output (the pieces recomputed here in torch from the
+    decoded matrices)."""
     wl, layer, xb = _tiny_layer()
     s = wl.shape
     y, idx, w, _ = orc.latent_moe_forward(s, layer, xb)
     W = orc.Weights(s, layer)
-    x = orc.bf16_to_f64(xb)
-    y2 = orc.shared_expert(x, W.Wsg, W.Wsu, W.Wsd)
+    F = torch.nn.functional
+    x = _t(orc.bf16_to_f64(xb))
+    y2 = (F.silu(x @ _t(W.Wsg).T) * (x @ _t(W.Wsu).T)) @ _t(W.Wsd).T
     for t in range(x.shape[0]):
         for k in range(s.top_k):
             e = int(idx[t, k])
             g = int(W.group[e])
-            o = orc.expert_apply(*W.expert(e), W.D(g) @ x[t])
-            y2[t] += W.U(g) @ (w[t, k] * o)
-    np.testing.assert_allclose(y, y2, rtol=1e-10, atol=1e-13)
+            Wg, Wu, Wd = (_t(m) for m in W.expert(e))
+            h = _t(W.D(g)) @ x[t]
+            o = Wd @ (F.silu(Wg @ h) * (Wu @ h))
+            y2[t] += _t(W.U(g)) @ (float(w[t, k]) * o)
+    np.testing.assert_allclose(y, y2.numpy(), rtol=1e-10, atol=1e-13)
 
 
-def test_block_single_expert_single_group_is_textbook_chain():
+def test_block_single_expert_single_group_is_textbook_chain(orc):
     s = synth.replace(TINY, n_experts=1, top_k=1, n_groups=1)
     wl, layer, xb = _tiny_layer(shape=s)
     y, idx, w, _ = orc.latent_moe_forward(s, layer, xb)
@@ -328,20 +356,23 @@ def test_block_single_expert_single_group_is_textbook_chain():
     np.testing.assert_allclose(y, want.numpy(), rtol=1e-11, atol=1e-14)
 
 
-def test_block_zero_input_gives_zero():
+def test_block_zero_input_gives_zero(orc):
     wl, layer, xb = _tiny_layer()
     y, _, _, _ = orc.latent_moe_forward(wl.shape, layer, np.zeros_like(xb))
     assert np.all(y == 0.0)
 
 
-def test_block_zero_experts_gives_shared_only():
+def test_block_zero_experts_gives_shared_only(orc):
     wl, layer, xb = _tiny_layer()
     layer = dict(layer)
     layer["experts"] = np.zeros_like(layer["experts"])
     y, _, _, _ = orc.latent_moe_forward(wl.shape, layer, xb)
-    W = orc.Weights(wl.shape, layer)
-    x = orc.bf16_to_f64(xb)
-    np.testing.assert_allclose(y, orc.shared_expert(x, W.Wsg, W.Wsu, W.Wsd), rtol=1e-13, atol=0)
+    F = torch.nn.functional
+    x = _t(orc.bf16_to_f64(xb))
+    bf = lambda a: torch.from_numpy(a.view(np.int16)).view(torch.bfloat16).double()
+    want = (F.silu(x @ bf(layer["shared_gate"]).T) * (x @ bf(layer["shared_up"]).T)) @ bf(layer["shared_down"]).T
+    # fp64 sums in another order: equal to rounding
+    np.testing.assert_allclose(y, want.numpy(), rtol=1e-12, atol=1e-14)
 
 
 def _identity_q8_0(n):
@@ -355,7 +386,7 @@ def _identity_q8_0(n):
     return np.frombuffer(bytes(blob), np.uint8)
 
 
-def test_block_identity_latent_reduces_to_standard_moe():
+def test_block_identity_latent_reduces_to_standard_moe(orc):
     s = synth.replace(TINY, latent=TINY.hidden)
     wl, layer, xb = _tiny_layer(shape=s)
     layer = dict(layer)
@@ -375,7 +406,7 @@ def test_block_identity_latent_reduces_to_standard_moe():
     np.testing.assert_allclose(y, want.numpy(), rtol=1e-11, atol=1e-14)
 
 
-def test_block_injection_overrides_routing():
+def test_block_injection_overrides_routing(orc):
     wl, layer, xb = _tiny_layer()
     s = wl.shape
     T = xb.shape[0]
@@ -387,7 +418,7 @@ def test_block_injection_overrides_routing():
     assert orc.rel_l2(y, y_ref) > 1e-3
 
 
-def test_residual_adds():
+def test_residual_adds(orc):
     wl, layer, xb = _tiny_layer()
     r = synth.bf16_normal(123, 1.0, xb.shape)
     y0, _, _, _ = orc.latent_moe_forward(wl.shape, layer, xb)
@@ -395,7 +426,7 @@ def test_residual_adds():
     np.testing.assert_allclose(y1 - y0, orc.bf16_to_f64(r), rtol=0, atol=1e-12)
 
 
-def test_rmsnorm_closed_form():
+def test_rmsnorm_closed_form(orc):
     v = np.array([[3.0, -4.0], [0.0, 0.0]])
     g = np.array([2.0, 0.5])
     out = orc.rmsnorm(v, g, 0.0 + 1e-30)
@@ -405,7 +436,7 @@ def test_rmsnorm_closed_form():
     np.testing.assert_allclose(orc.rmsnorm(np.array([[1.0, 1.0]]), np.ones(2), 1.0), [[1 / math.sqrt(2)] * 2])
 
 
-def test_stack_layer_is_residual_plus_block_of_norm():
+def test_stack_layer_is_residual_plus_block_of_norm(orc):
     wl, layer, xb = _tiny_layer()
     s = wl.shape
     gamma = np.linspace(0.5, 1.5, s.hidden)
@@ -415,3 +446,118 @@ def test_stack_layer_is_residual_plus_block_of_norm():
     xn = gamma[None, :] * x / np.sqrt(ms + 1e-6)
     blk, _, _, _ = orc.latent_moe_forward(s, layer, None, x_f64=xn)
     np.testing.assert_allclose(y, x + blk, rtol=1e-13, atol=1e-14)
+
+
+# ----------------------------------------------------------------------------
+# slicing of the D / U blobs and of the expert array, against the generator
+# ----------------------------------------------------------------------------
+
+def test_slices_match_the_generators_own_draws(orc):
+    """du_slice(g) and expert_slice(e) pick the bytes the generator wrote for
+    group g and expert e: re-encoding that index's own fp64 draws gives the
+    same bytes, and decoding the slice gives those draws back within each
+    format's rounding step.  An off-by-one group or record, or a transposed
+    decode, fails."""
+    s = synth.LayerShape(hidden=128, latent=64, n_experts=7, top_k=2, n_groups=3, ffn=64, shared_ffn=64,
+                         du_fmt=synth.Q8_0, router_dtype="bf16")
+    for fmt in (synth.Q8_0, synth.Q4_0):
+        wl = synth.Workload("slices", synth.replace(s, du_fmt=fmt), T=2, seed=21, weight_sigma=0.05)
+        layer = synth.make_layer(wl)
+        for name, R, C in (("D", s.latent, s.hidden), ("U", s.hidden, s.latent)):
+            for g in range(s.n_groups):
+                w = synth.f64_normal(synth.key(wl.seed, 0, name, g), wl.weight_sigma, (R, C))
+                sl = orc.du_slice(layer[name], fmt, g, R, C)
+                assert np.array_equal(sl, synth.qmatrix_encode(fmt, w)), (name, g)
+                amax = np.abs(w).reshape(R, C // 32, 32).max(axis=2)
+                step = np.repeat(amax / (127.0 if fmt == synth.Q8_0 else 8.0), 32, axis=1)
+                assert np.all(np.abs(orc.decode_du(fmt, sl, R, C) - w) <= step * 1.01 + 1e-12), (name, g)
+    wl = synth.Workload("slices", s, T=2, seed=22, weight_sigma=0.05)
+    layer = synth.make_layer(wl)
+    kx = synth.key(wl.seed, 0, "experts")
+    for e in (0, 3, s.n_experts - 1):
+        ws = [synth.f64_normal(synth.expert_key(kx, e, m), wl.weight_sigma, shp)
+              for m, shp in enumerate([(s.ffn, s.latent), (s.ffn, s.latent), (s.latent, s.ffn)])]
+        rec = orc.expert_slice(layer["experts"], e, s.latent, s.ffn)
+        assert np.array_equal(rec, synth.expert_record_encode(*ws)), e
+        for want, got in zip(ws, orc.decode_expert(rec, s.latent, s.ffn)):
+            # E2M1 with its E4M3 block scale: within half the widest grid gap
+            # (2 of the block's 6 levels) of the block maximum
+            amax16 = np.repeat(np.abs(want).reshape(want.shape[0], -1, 16).max(axis=2), 16, axis=1)
+            assert np.all(np.abs(got - want) <= amax16 / 6.0 * 1.0625 + 1e-12), e
+
+
+# ----------------------------------------------------------------------------
+# the stack: a closed-form two-layer case
+# ----------------------------------------------------------------------------
+
+def _exact_nvfp4_matrix(rng, R, C, unit):
+    """Values e2m1 * unit with +-6 * unit at the head of every 16-block, so
+    that NVFP4 encodes them exactly when unit / (6 * 448) * 6 is a power of
+    two (unit = 7 / 256 gives the tensor scale 2^-14 and block scale 448)."""
+    grid = np.array([0.0, 0.5, 1.0, 1.5, 2.0, 3.0, 4.0, 6.0])
+    v = grid[rng.integers(0, 8, size=(R, C))] * np.where(rng.random((R, C)) < 0.5, -1.0, 1.0)
+    v[:, ::16] = 6.0 * np.where(rng.random((R, C // 16)) < 0.5, -1.0, 1.0)
+    return v * unit
+
+
+def test_stack_two_layers_closed_form(orc):
+    """Two pre-norm residual layers with identity D and U (latent = hidden),
+    one expert always chosen with weight 1 and exactly representable NVFP4
+    weights: each layer is x + S(n(x)) + W_d(silu(W_g n(x)) * W_u n(x)) with
+    n = RMSNorm, written out here in torch; the second layer reads the first
+    layer's output rounded to bf16, as the stack keeps its residual stream."""
+    H = 64
+    s = synth.LayerShape(hidden=H, latent=H, n_experts=2, top_k=1, n_groups=1, ffn=64, shared_ffn=64,
+                         du_fmt=synth.Q8_0, router_dtype="f32")
+    rng = np.random.default_rng(31)
+    unit = 7.0 / 256.0
+    F = torch.nn.functional
+    bf = lambda a: torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).view(torch.bfloat16).double()
+    xb = synth.bf16_normal(synth.key(9, 0, "x"), 1.0, (3, H))
+    x_ref = bf(xb)
+    eps = 1e-6
+    for layer_i in range(2):
+        wl = synth.Workload("stack2", s, T=3, seed=40 + layer_i, weight_sigma=0.1)
+        layer = synth.make_layer(wl)
+        layer["router_w"] = np.zeros((2, H), np.float32)
+        layer["router_b"] = np.array([5.0, 0.0], np.float32)
+        layer["expert_group"] = np.zeros(2, np.uint8)
+        layer["D"] = _identity_q8_0(H)
+        layer["U"] = _identity_q8_0(H)
+        Wg, Wu, Wd = (_exact_nvfp4_matrix(rng, H, H, unit) for _ in range(3))
+        rec = synth.expert_record_encode(Wg, Wu, Wd)
+        layer["experts"] = np.concatenate([rec, np.zeros_like(rec)])
+        gamma = np.linspace(0.5, 1.5, H) + 0.25 * layer_i
+        y, idx, w, _ = orc.stack_layer_forward(s, layer, xb, gamma, eps)
+        assert np.all(idx == 0) and np.all(w == 1.0)
+        n = _t(gamma)[None, :] * x_ref / torch.sqrt((x_ref * x_ref).mean(dim=1, keepdim=True) + eps)
+        shared = (F.silu(n @ bf(layer["shared_gate"]).T) * (n @ bf(layer["shared_up"]).T)) @ bf(layer["shared_down"]).T
+        expert = (F.silu(n @ _t(Wg).T) * (n @ _t(Wu).T)) @ _t(Wd).T
+        want = x_ref + shared + expert
+        np.testing.assert_allclose(y, want.numpy(), rtol=1e-12, atol=1e-13)
+        # the next layer's input: this layer's output rounded to bf16 (here, by torch)
+        x_ref = want.to(torch.bfloat16).double()
+        xb = want.to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16)
+
+
+# ----------------------------------------------------------------------------
+# the two oracles against each other (independent implementations)
+# ----------------------------------------------------------------------------
+
+@pytest.mark.parametrize("fmt", [synth.Q8_0, synth.Q4_0])
+def test_cpp_and_numpy_oracles_agree(fmt):
+    s = synth.LayerShape(hidden=256, latent=128, n_experts=24, top_k=5, n_groups=4, ffn=128, shared_ffn=64,
+                         du_fmt=fmt, router_dtype="bf16")
+    wl = synth.Workload("agree", s, T=7, seed=17, bias_sigma=0.5, weight_sigma=0.05)
+    layer = synth.make_layer(wl)
+    xb = synth.make_x(wl)
+    res = synth.bf16_normal(synth.key(17, 0, "residual"), 1.0, xb.shape)
+    a = cpp_oracle.latent_moe_forward(s, layer, xb, residual_bits=res)
+    b = np_oracle.latent_moe_forward(s, layer, xb, residual_bits=res)
+    assert np.array_equal(a[1], b[1])
+    np.testing.assert_allclose(a[2], b[2], rtol=1e-13)
+    np.testing.assert_allclose(a[0], b[0], rtol=1e-11, atol=1e-13)
+    gamma = np.linspace(0.8, 1.2, s.hidden)
+    c = cpp_oracle.stack_layer_forward(s, layer, xb, gamma, 1e-6)
+    d = np_oracle.stack_layer_forward(s, layer, xb, gamma, 1e-6)
+    np.testing.assert_allclose(c[0], d[0], rtol=1e-11, atol=1e-13)
