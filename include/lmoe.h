@@ -118,28 +118,53 @@ typedef struct {
     const void* norm_gamma;       /* bf16 [hidden]: RMSNorm weight before the block */
 } lmoe_layer;
 
-/* LMOE_OK if the shape is supported, else LMOE_ERR_UNSUPPORTED / LMOE_ERR_ARG. */
+/* LMOE_OK if the shape is supported, else LMOE_ERR_UNSUPPORTED / LMOE_ERR_ARG.
+ * (Shapes: Edge0 145B / 120B model page, architecture tables: hidden 2560,
+ * 512 experts, top-10, 8 D/U groups, latent 1792 or 1280, SwiGLU 640.) */
 LMOE_API int lmoe_cfg_check(const lmoe_cfg* cfg);
 
 /* Bytes of one expert record, of one D (or U) blob holding all n_groups
  * matrices, and of the workspace needed for up to T_max tokens.  0 if the
- * configuration is unsupported. */
+ * configuration is unsupported.  (Record size: teardown article, section
+ * "What is 4-bit": 1,935,376 bytes per expert at latent 1792; Q8_0 / Q4_0
+ * sizes: 34 and 18 bytes per 32 weights; the model page, "Model profile",
+ * stores D and U as Q8 or Q4.) */
 LMOE_API size_t lmoe_expert_record_bytes(const lmoe_cfg* cfg);
 LMOE_API size_t lmoe_du_bytes(const lmoe_cfg* cfg);
 LMOE_API size_t lmoe_workspace_bytes(const lmoe_cfg* cfg, int T_max);
 
 /* Router only: logits, softmax, top_k and renormalised weights.
- * topk_idx int32 [T][top_k] and topk_w fp32 [T][top_k], in selection order
- * (logit descending, index ascending on ties). */
+ * Defining passage: model page, "Model profile" (the router picks 10 of the
+ * 512 experts of a layer); the function itself (softmax over all experts,
+ * top-k, renormalise over the kept, bias added to the logits, lowest index
+ * on ties) is not printed on the pages and follows the task's workload
+ * statement of the block.
+ *   x         bf16 [T][hidden], device
+ *   router_w  fp32 or bf16 [n_experts][hidden]; router_b fp32 [n_experts] or NULL
+ *   topk_idx  int32 [T][top_k] and topk_w fp32 [T][top_k], written in
+ *             selection order (logit descending, index ascending on ties)
+ *   ws        workspace of at least lmoe_workspace_bytes(cfg, T) bytes
+ * Errors: LMOE_ERR_ARG (null, misaligned, T < 0), LMOE_ERR_UNSUPPORTED,
+ * LMOE_ERR_WORKSPACE; T = 0 launches nothing. */
 LMOE_API int lmoe_route(const lmoe_cfg* cfg, const void* x, const void* router_w, const float* router_b, int T,
                int32_t* topk_idx, float* topk_w, void* ws, size_t ws_bytes, void* stream);
 
-/* The block: y [T][hidden] bf16 = block(x). */
+/* The block: y [T][hidden] bf16 = block(x).
+ * Defining passage: teardown article, section "A latent in front of the
+ * experts" (layer equation: the token is compressed by D_g, the experts run
+ * at latent width, their weighted outputs are summed and widened back by
+ * U_g), read per group (the same section gives every expert one of eight
+ * group labels); shared expert at full width: model page, "Model profile"
+ * (only the expert pool runs at the latent width).
+ * Arguments: x bf16 [T][hidden]; weights as in the storage layouts above;
+ * y bf16 [T][hidden] (must not overlap x); ws of lmoe_workspace_bytes(cfg, T).
+ * Errors: LMOE_ERR_ARG / _UNSUPPORTED / _WORKSPACE before any launch; kernel
+ * findings through lmoe_last_device_status. */
 LMOE_API int lmoe_forward(const lmoe_cfg* cfg, const void* x, const void* router_w, const uint8_t* expert_group,
                  const void* D, const void* U, const void* experts, const lmoe_shared* shared,
                  void* y, int T, void* ws, size_t ws_bytes, void* stream);
 
-/* The block with every option:
+/* The block with every option (same passage as lmoe_forward):
  *   router_b     per-expert bias added to the logits, or NULL
  *   residual     bf16 [T][hidden] added to y, or NULL; y overlaps neither x
  *                nor residual
@@ -153,16 +178,22 @@ LMOE_API int lmoe_forward_ex(const lmoe_cfg* cfg, const void* x, const void* rou
                     const int32_t* inject_idx, const float* inject_w, int32_t* out_idx, float* out_w,
                     void* y, int T, void* ws, size_t ws_bytes, void* stream);
 
-/* As lmoe_forward, with x_host and y_host in host memory (page-locked for
- * the copies to overlap): copies x in, runs the block, copies y out, all on
- * `stream`.  The call returns once y_host is written. */
+/* As lmoe_forward (same passage), with x_host and y_host in host memory
+ * (page-locked for the copies to overlap): copies x in, runs the block,
+ * copies y out, all on `stream`.  The call returns once y_host is written;
+ * the workspace holds the device copies of x and y. */
 LMOE_API int lmoe_forward_host(const lmoe_cfg* cfg, const void* x_host, const void* router_w, const float* router_b,
                       const uint8_t* expert_group, const void* D, const void* U, const void* experts,
                       const lmoe_shared* shared, void* y_host, int T, void* ws, size_t ws_bytes, void* stream);
 
 /* n_layers pre-norm residual layers: x <- x + block_l(RMSNorm_l(x)), the
  * residual stream kept in bf16; RMSNorm(v) = gamma * v / sqrt(mean(v^2) + eps).
- * x and y are bf16 [T][hidden] and may not alias.  `layers` is a host array. */
+ * Defining passage: model page, architecture tables (48 layers, each with a
+ * latent-MoE FFN); the norm, its place before the block and the residual
+ * add are not printed there (attention is omitted) and follow the task's
+ * statement of the stack.
+ * x and y are bf16 [T][hidden] and may not alias.  `layers` is a host array
+ * of device pointers (norm_gamma required).  Errors as lmoe_forward. */
 LMOE_API int lmoe_stack_forward(const lmoe_cfg* cfg, int n_layers, const lmoe_layer* layers, const void* x, void* y,
                        int T, float rms_eps, void* ws, size_t ws_bytes, void* stream);
 

@@ -117,6 +117,21 @@ static_assert(sizeof(Ctrl) <= 4096, "control block");
 
 __device__ __forceinline__ void set_status(Ctrl* c, int s) { atomicCAS(&c->status, 0, s); }
 
+// fp16 staging of activations: values outside the fp16 range (|v| > 65504,
+// or NaN) would become inf; they are flagged in `bad`, and the caller
+// reports LMOE_ERR_DEVICE_CHECK once.
+__device__ __forceinline__ __half half_checked(float v, bool& bad) {
+    bad |= !(fabsf(v) <= 65504.f);
+    return __float2half_rn(v);
+}
+__device__ __forceinline__ __half2 half2_checked(float a, float b, bool& bad) {
+    bad |= !(fabsf(a) <= 65504.f) | !(fabsf(b) <= 65504.f);
+    return __floats2half2_rn(a, b);
+}
+__device__ __forceinline__ void report_range(Ctrl* c, bool bad) {
+    if (bad) set_status(c, LMOE_ERR_DEVICE_CHECK);
+}
+
 // ---------------------------------------------------------------------------
 // workspace carve-up (host and device agree through this struct)
 // ---------------------------------------------------------------------------

@@ -84,7 +84,11 @@ __global__ void __launch_bounds__(256) k_router_shared(FwdParams p) {
                     if (lane == 0 && t < nt) {
                         const float z = silu(av) * uv;
                         p.zsh[(size_t)(t0 + t) * p.Fs + f] = z;
-                        if (p.zsh16) p.zsh16[(size_t)(t0 + t) * p.Fs + f] = __float2half_rn(z);
+                        if (p.zsh16) {
+                            bool bad = false;
+                            p.zsh16[(size_t)(t0 + t) * p.Fs + f] = half_checked(z, bad);
+                            report_range(p.ctrl, bad);
+                        }
                     }
                 }
             }
@@ -569,11 +573,13 @@ __global__ void __launch_bounds__(32 * kMmaWarps, 4) k_dproj_mma(FwdParams p) {
         reduce_frags(acc, red);
         if (warp == 0) {
             const int gg = lane >> 2, tt = lane & 3;
+            bool bad = false;
 #pragma unroll
             for (int i = 0; i < 4; ++i) {
                 const int tok = 2 * tt + (i & 1), row = r0 + gg + 8 * (i >> 1);
-                if (tok < nt) p.h16[((size_t)(t0 + tok) * p.G + g) * L + row] = __float2half_rn(acc[i]);
+                if (tok < nt) p.h16[((size_t)(t0 + tok) * p.G + g) * L + row] = half_checked(acc[i], bad);
             }
+            report_range(p.ctrl, bad);
         }
     }
 }
@@ -627,11 +633,13 @@ __global__ void __launch_bounds__(32 * kMmaWarps, 3) k_gateup_mma(FwdParams p) {
         reduce_frags(u, red);
         if (warp == 0) {
             const int gg = lane >> 2, tt = lane & 3;
+            bool bad = false;
 #pragma unroll
             for (int i = 0; i < 4; ++i) {
                 const int col = 2 * tt + (i & 1), f = f0 + gg + 8 * (i >> 1);
-                if (col < nt) p.z16[(size_t)(off + c0 + col) * F + f] = __float2half_rn(silu(a[i] * ts_g) * (u[i] * ts_u));
+                if (col < nt) p.z16[(size_t)(off + c0 + col) * F + f] = half_checked(silu(a[i] * ts_g) * (u[i] * ts_u), bad);
             }
+            report_range(p.ctrl, bad);
         }
         __syncthreads();
     }
@@ -704,6 +712,7 @@ __global__ void __launch_bounds__(32 * kDownWarps, 4) k_down_mma(FwdParams p) {
     }
     __syncthreads();
     // group sum per (row, token), experts in ascending order (deterministic)
+    bool bad = false;
     for (int i = threadIdx.x; i < 16 * T; i += blockDim.x) {
         const int row = i / T, t = i - row * T;
         float v = 0.f;
@@ -717,8 +726,9 @@ __global__ void __launch_bounds__(32 * kDownWarps, 4) k_down_mma(FwdParams p) {
                 }
             }
         }
-        p.s16[((size_t)t * p.G + g) * L + r0 + row] = __float2half_rn(v);
+        p.s16[((size_t)t * p.G + g) * L + r0 + row] = half_checked(v, bad);
     }
+    report_range(p.ctrl, bad);
 }
 
 // kernel 5: per 16 output rows, one part per hit group (U_g s16[t][g]) and

@@ -80,14 +80,16 @@ __device__ void stage_x(const FwdParams& p, int t0, int nt, float* xs, float* rs
     }
     if (blockIdx.x == 0 && p.x16) {
         __syncthreads();
+        bool bad = false;
         for (int i = threadIdx.x; i < nt * nc; i += blockDim.x) {
             const int t = i / nc, c = i - t * nc;
             const float* src = xs + t * ld + 8 * c;
             __half2 h[4];
 #pragma unroll
-            for (int j = 0; j < 4; ++j) h[j] = __floats2half2_rn(src[2 * j], src[2 * j + 1]);
+            for (int j = 0; j < 4; ++j) h[j] = half2_checked(src[2 * j], src[2 * j + 1], bad);
             *reinterpret_cast<uint4*>(p.x16 + (size_t)(t0 + t) * H + 8 * c) = *reinterpret_cast<uint4*>(h);
         }
+        report_range(p.ctrl, bad);
     }
 }
 

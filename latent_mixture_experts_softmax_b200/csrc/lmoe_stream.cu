@@ -184,17 +184,18 @@ __device__ __forceinline__ void tile_nvfp4(const uint8_t* q, const uint8_t* s, c
 }
 
 // 16 rows of bf16 weights ([16][K] row-major) against fp16 activations,
-// 32-column blocks [b0, b1); bf16 -> fp16 in registers.
+// 32-column blocks [b0, b1); bf16 -> fp16 in registers (a weight outside the
+// fp16 range is flagged in `bad`).
 __device__ __forceinline__ void tile_bf16(const uint16_t* w, int K, const __half* xs, int ld, int nt, int b0, int b1,
-                                          float (&acc)[4]) {
+                                          float (&acc)[4], bool& bad) {
     const int lane = threadIdx.x & 31, g = lane >> 2, t = lane & 3;
 #pragma unroll 2
     for (int b = b0; b < b1; ++b) {
         const uint4 wg = *reinterpret_cast<const uint4*>(w + (size_t)g * K + 32 * b + 8 * t);
         const uint4 wh = *reinterpret_cast<const uint4*>(w + (size_t)(g + 8) * K + 32 * b + 8 * t);
-        auto cv = [](uint32_t v) {
+        auto cv = [&bad](uint32_t v) {
             const float2 f = bf16x2_to_f32x2(v);
-            __half2 h = __floats2half2_rn(f.x, f.y);
+            __half2 h = half2_checked(f.x, f.y, bad);
             return *reinterpret_cast<uint32_t*>(&h);
         };
         const uint4 xv = act8(xs, ld, g, nt, 32 * b + 8 * t);
@@ -357,7 +358,9 @@ __device__ __forceinline__ void compute_step(const FwdParams& p, const WItem& it
         const int qb = FMT == LMOE_Q8_0 ? 32 : 16;
         tile_du<FMT>(buf, reinterpret_cast<const uint16_t*>(buf + sb * 16 * qb), x, ld, nt, 0, nblk, a);
     } else if (PHASE == SP_UPROJ) {
-        tile_bf16(reinterpret_cast<const uint16_t*>(buf), 64, x, ld, nt, 0, nblk, a);
+        bool bad = false;
+        tile_bf16(reinterpret_cast<const uint16_t*>(buf), 64, x, ld, nt, 0, nblk, a, bad);
+        report_range(p.ctrl, bad);
     } else if (PHASE == SP_GATEUP) {
         tile_nvfp4(buf, buf + 2 * 1024, x, ld, nt, nblk, a);
         tile_nvfp4(buf + 1024, buf + 2 * 1024 + 128, x, ld, nt, nblk, u);
@@ -555,6 +558,7 @@ __device__ void fill_x(const FwdParams& p, __half* cache, int ld, float* rs) {
         }
         __syncthreads();
     }
+    bool bad = false;
     for (int i = threadIdx.x; i < T * nc; i += blockDim.x) {
         const int t = i / nc, c = i - t * nc;
         float f[8];
@@ -567,9 +571,11 @@ __device__ void fill_x(const FwdParams& p, __half* cache, int ld, float* rs) {
         }
         __half2 h[4];
 #pragma unroll
-        for (int j = 0; j < 4; ++j) h[j] = __floats2half2_rn(f[2 * j], f[2 * j + 1]);
+        for (int j = 0; j < 4; ++j) h[j] = half2_checked(f[2 * j], f[2 * j + 1], bad);
         *reinterpret_cast<uint4*>(cache + (size_t)t * ld + 8 * c) = *reinterpret_cast<uint4*>(h);
     }
+    // only CTA 0 reports, so that a bad input costs one atomic, not one per CTA
+    if (blockIdx.x == 0) report_range(p.ctrl, bad);
 }
 
 // The chunk's activations from global memory, by plain loads of every thread.
@@ -584,6 +590,7 @@ __device__ void phase_fill(const FwdParams& p, const StreamShared& sh, const Chu
     }
     const int KC = PHASE == SP_DPROJ ? H : PHASE == SP_GATEUP ? L : PHASE == SP_DOWN ? F : max(L, Fs);
     const int per = KC / 8;
+    bool bad = false;
     for (int qv = threadIdx.x; qv < ci.rows * per; qv += blockDim.x) {
         const int r = qv / per, c = qv - r * per;
         const int src = ci.src[r];
@@ -611,7 +618,7 @@ __device__ void phase_fill(const FwdParams& p, const StreamShared& sh, const Chu
             }
             __half2 h[4];
 #pragma unroll
-            for (int j = 0; j < 4; ++j) h[j] = __floats2half2_rn(acc8[2 * j], acc8[2 * j + 1]);
+            for (int j = 0; j < 4; ++j) h[j] = half2_checked(acc8[2 * j], acc8[2 * j + 1], bad);
             v = *reinterpret_cast<uint4*>(h);
         } else {
             if (8 * c >= Fs) continue;
@@ -619,6 +626,7 @@ __device__ void phase_fill(const FwdParams& p, const StreamShared& sh, const Chu
         }
         *reinterpret_cast<uint4*>(cache + (size_t)r * ld + 8 * c) = v;
     }
+    if (PHASE == SP_UPROJ) report_range(p.ctrl, bad);
 }
 
 // An item's 16x8 result is complete: its epilogue, or (U, whose output tile
@@ -666,23 +674,25 @@ __device__ __forceinline__ void item_finish(const FwdParams& p, const StreamShar
     }
     if (finish) {
         const float* ts = (PHASE == SP_GATEUP || PHASE == SP_DOWN) ? ci.tail[jj] : nullptr;
+        bool bad = false;
 #pragma unroll
         for (int i4 = 0; i4 < 4; ++i4) {
             const int col = 2 * tt + (i4 & 1), row = cit.r0 + gg + 8 * (i4 >> 1);
             if (col >= nt) continue;
             if (PHASE == SP_DPROJ) {
-                p.h16[((size_t)col * G + cit.mat) * L + row] = __float2half_rn(a[i4]);
+                p.h16[((size_t)col * G + cit.mat) * L + row] = half_checked(a[i4], bad);
             } else if (PHASE == SP_GATEUP) {
-                p.z16[(size_t)(sh.uoff[cit.j] + col) * F + row] = __float2half_rn(silu(a[i4] * ts[0]) * (u[i4] * ts[1]));
+                p.z16[(size_t)(sh.uoff[cit.j] + col) * F + row] = half_checked(silu(a[i4] * ts[0]) * (u[i4] * ts[1]), bad);
             } else if (PHASE == SP_DOWN) {
                 const int slot = sh.uoff[cit.j] + col;
-                p.o16w[(size_t)slot * L + row] = __float2half_rn(sh.slot_w[slot] * ts[2] * a[i4]);
+                p.o16w[(size_t)slot * L + row] = half_checked(sh.slot_w[slot] * ts[2] * a[i4], bad);
             } else {
                 float v = a[i4];
                 if (p.residual) v += bf16_bits_to_f32(p.residual[(size_t)col * H + row]);
                 p.y[(size_t)col * H + row] = f32_to_bf16_bits(v);
             }
         }
+        report_range(p.ctrl, bad);
     }
 }
 

@@ -336,11 +336,12 @@ __device__ __forceinline__ void epilogue_chunk(const PrefillParams& p, const Til
         const uint32_t* mmask = reinterpret_cast<const uint32_t*>(xchg);
         const int* mslot = reinterpret_cast<const int*>(mmask + NT);
         const int l = t.m0 + row;
+        bool bad = false;
 #pragma unroll
         for (int j = 0; j < 32; ++j) {
             if (j < ncol) {
                 uint32_t mask = mmask[c0 + j];
-                const __half v = __float2half_rn(u2f(r[j]));
+                const __half v = half_checked(u2f(r[j]), bad);
                 while (mask) {
                     const int k = __ffs(mask) - 1;
                     mask &= mask - 1;
@@ -348,6 +349,7 @@ __device__ __forceinline__ void epilogue_chunk(const PrefillParams& p, const Til
                 }
             }
         }
+        report_range(p.ctrl, bad);
     } else if (KIND == G_GATEUP || KIND == G_SHARED_GATEUP) {
         // rows 0-63: gate, rows 64-127: up.  Warps 0-1 finish columns 0-15
         // of the chunk, warps 2-3 columns 16-31; each hands the other pair
@@ -366,6 +368,7 @@ __device__ __forceinline__ void epilogue_chunk(const PrefillParams& p, const Til
         const float tg = tscale[0], tu = tscale[1];
         const int f = t.m0 + r64;
         const int jb = warp < 2 ? 0 : 16;
+        bool bad = false;
 #pragma unroll
         for (int j = 0; j < 16; ++j) {
             if (jb + j < ncol) {
@@ -374,7 +377,7 @@ __device__ __forceinline__ void epilogue_chunk(const PrefillParams& p, const Til
                 const float z = silu_fast(a) * u;
                 const int col = t.b0 + c0 + jb + j;
                 if (KIND == G_GATEUP) {
-                    p.zperm[(size_t)col * p.F + f] = __float2half_rn(z);
+                    p.zperm[(size_t)col * p.F + f] = half_checked(z, bad);
                 } else {
                     const uint16_t hi = f32_to_bf16_bits(z);
                     p.zsh[(size_t)col * p.Fs + f] = hi;
@@ -382,18 +385,21 @@ __device__ __forceinline__ void epilogue_chunk(const PrefillParams& p, const Til
                 }
             }
         }
+        report_range(p.ctrl, bad);
         named_bar_sync(1, 128);
     } else if (KIND == G_DOWN) {
         // routing weights of the tile's slots staged in xchg by the epilogue warps
         const float td = tscale[2];
         const int l = t.m0 + row;
+        bool bad = false;
 #pragma unroll
         for (int j = 0; j < 32; ++j) {
             if (j < ncol) {
                 const int slot = t.b0 + c0 + j;
-                p.operm[(size_t)slot * p.L + l] = __float2half_rn(u2f(r[j]) * td * xchg[c0 + j]);
+                p.operm[(size_t)slot * p.L + l] = half_checked(u2f(r[j]) * td * xchg[c0 + j], bad);
             }
         }
+        report_range(p.ctrl, bad);
     } else {  // UPROJ
         const int hrow = t.m0 + row;
         float res[32];
@@ -838,6 +844,7 @@ __global__ void k_bucket_scatter(const PrefillParams p) {
 __global__ void k_combine(const PrefillParams p) {
     const int t = blockIdx.x;
     const int nchunk = p.L / 8;
+    bool bad = false;
     for (int g = 0; g < p.G; ++g) {
         const uint32_t mask = __ldg(p.tgmask + (size_t)t * p.G + g);
         for (int c = threadIdx.x; c < nchunk; c += blockDim.x) {
@@ -857,13 +864,14 @@ __global__ void k_combine(const PrefillParams p) {
                 }
             }
             uint4 out;
-            out.x = h2_bits(__floats2half2_rn(acc[0], acc[1]));
-            out.y = h2_bits(__floats2half2_rn(acc[2], acc[3]));
-            out.z = h2_bits(__floats2half2_rn(acc[4], acc[5]));
-            out.w = h2_bits(__floats2half2_rn(acc[6], acc[7]));
+            out.x = h2_bits(half2_checked(acc[0], acc[1], bad));
+            out.y = h2_bits(half2_checked(acc[2], acc[3], bad));
+            out.z = h2_bits(half2_checked(acc[4], acc[5], bad));
+            out.w = h2_bits(half2_checked(acc[6], acc[7], bad));
             reinterpret_cast<uint4*>(p.s + ((size_t)t * p.G + g) * p.L)[c] = out;
         }
     }
+    report_range(p.ctrl, bad);
 }
 
 // ---------------------------------------------------------------------------

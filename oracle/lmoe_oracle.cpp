@@ -29,7 +29,7 @@
 //   8. residual y += residual (optional)
 //   stack layer: x + block(RMSNorm(x)), RMSNorm(v) = gamma v / sqrt(mean v^2 + eps)
 //
-// Storage formats (the model page: "D/U formats: Q8 or Q4"; the teardown
+// Storage formats (the model page, "Model profile": D and U in Q8 or Q4; the teardown
 // article, "What is 4-bit": NVFP4 = E2M1 values with one E4M3 scale per 16,
 // a 16-byte record tail):
 //   Q8_0 [R][C]:  int8 q [C/32][R][32], then fp16 d [C/32][R]; w = d q

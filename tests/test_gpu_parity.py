@@ -154,14 +154,45 @@ def test_block_decode_configs(name):
         check_block(wl.shape, layer, synth.make_x(wl, draw=draw), dev=dev, weights=W, what=f"{name} draw {draw}")
 
 
+def _cover_rows(idx_all: np.ndarray, tile: int, per_tile: int) -> np.ndarray:
+    """Rows to recompute on the CPU: per_tile rows from every `tile`-token
+    tile, each picked (greedily, within its tile) to add the most experts not
+    yet covered, so that the sample reaches nearly every expert the batch
+    routes to and every tile of the tensor-core GEMMs."""
+    T = idx_all.shape[0]
+    covered = set()
+    rows = []
+    for t0 in range(0, T, tile):
+        cand = list(range(t0, min(T, t0 + tile)))
+        for _ in range(min(per_tile, len(cand))):
+            best = max(cand, key=lambda t: (len(set(idx_all[t].tolist()) - covered), -t))
+            cand.remove(best)
+            rows.append(best)
+            covered |= set(idx_all[best].tolist())
+    return np.array(sorted(rows))
+
+
+def _check_prefill_sampled(wl, T, per_tile, min_expert_cover):
+    layer = synth.make_layer(wl)
+    xb = synth.make_x(wl, T=T)
+    dev = DeviceLayer(wl.shape, layer)
+    idx, _ = dev.route(to_device(xb, "cuda"), dev.workspace(T))
+    idx_all = idx.cpu().numpy()
+    rows = _cover_rows(idx_all, 256, per_tile)
+    assert len({r // 256 for r in rows}) == (T + 255) // 256           # every token tile
+    routed = set(idx_all.reshape(-1).tolist())
+    cover = set(idx_all[rows].reshape(-1).tolist())
+    assert len(cover) >= min_expert_cover * len(routed), (len(cover), len(routed))
+    out = check_block(wl.shape, layer, xb, tokens=rows, dev=dev, what=f"prefill T={T} sample")
+    return out, rows
+
+
 def test_block_prefill_config_sampled_tokens():
     """T=4096 through the same launch sequence the benchmark times; the oracle
-    recomputes a sample of rows (the block is per token)."""
+    recomputes 128 rows (8 per 256-token tile) that reach >= 90% of the
+    experts the batch routes to (the block is per token)."""
     wl = synth.WORKLOADS["edge0_145b_prefill"]
-    layer = synth.make_layer(wl)
-    xb = synth.make_x(wl)
-    rows = np.array([0, 1, 777, 2048, 3001, 4095])
-    check_block(wl.shape, layer, xb, tokens=rows, what="prefill sample")
+    _check_prefill_sampled(wl, 4096, 8, 0.9)
 
 
 def test_forward_host_matches_device_call():
@@ -300,8 +331,69 @@ def test_prefill_stack_layers():
 
 
 def test_prefill_16384_tokens_sampled():
-    """The largest configuration: 16384 tokens of the Edge0-145B-shaped layer."""
+    """The largest configuration: 16384 tokens of the Edge0-145B-shaped layer,
+    one oracle row per 256-token tile (64 rows) chosen to reach the most
+    experts."""
     wl = synth.WORKLOADS["edge0_145b_prefill"].with_(T=16384)
-    layer = synth.make_layer(wl)
+    _check_prefill_sampled(wl, 16384, 1, 0.6)
+
+
+# ----------------------------------------------------------------------------
+# Edge0 shapes on the 9-63-token kernels and the full-shape stack
+# ----------------------------------------------------------------------------
+
+@pytest.mark.parametrize("name,T", [("edge0_120b_decode", 16), ("edge0_145b_decode", 16),
+                                    ("edge0_120b_decode", 48), ("edge0_145b_decode", 48)])
+def test_block_edge0_shapes_between_9_and_63_tokens(name, T):
+    """Routing and output at the Edge0 shapes on the kernels that take 9-63
+    tokens in passes of 8 (every row compared)."""
+    wl = synth.WORKLOADS[name]
+    check_block(wl.shape, synth.make_layer(wl), synth.make_x(wl, T=T, draw=7), what=f"{name} T={T}")
+
+
+def test_stack_full_shape_145b_layer_by_layer():
+    """Three Edge0-145B-shaped layers (hidden 2560, latent 1792, 512 experts,
+    Q8_0 D/U) at T=4 through the stack call; each layer's output against the
+    oracle fed the GPU's own input of that layer."""
+    wl = synth.WORKLOADS["edge0_145b_stack"].with_(n_layers=3)
+    s = wl.shape
+    layers = [synth.make_layer(wl, layer=l) for l in range(wl.n_layers)]
+    gammas = [synth.bf16_bits_from_f32((np.linspace(0.8, 1.2, s.hidden) + 0.05 * l).astype(np.float32))
+              for l in range(wl.n_layers)]
+    devs = [DeviceLayer(s, ly, gamma=g) for ly, g in zip(layers, gammas)]
     xb = synth.make_x(wl)
-    check_block(wl.shape, layer, xb, tokens=np.array([0, 5000, 16383]), what="prefill 16384")
+    x = to_device(xb, "cuda")
+    ws = devs[0].workspace(wl.T)
+    eps = 1e-6
+    cur = xb
+    for l in range(wl.n_layers):
+        y = torch.empty_like(x)
+        B.lmoe_stack_forward(devs[0].cfg, [d.as_c_layer() for d in devs[:l + 1]], x, y, wl.T, eps, ws)
+        torch.cuda.synchronize()
+        assert B.lmoe_last_device_status(ws) == B.LMOE_OK
+        y_ref, _, _, gap = orc.stack_layer_forward(s, layers[l], cur, orc.bf16_to_f64(gammas[l]), eps)
+        assert np.all(gap >= GAP)
+        assert_close(bf16_bits_to_f64(y), y_ref, f"145B stack layer {l}")
+        cur = y.cpu().numpy().view(np.uint16)
+
+
+# ----------------------------------------------------------------------------
+# inputs outside the fp16 range of the staged activations
+# ----------------------------------------------------------------------------
+
+@pytest.mark.parametrize("T", [4, 16, 300])
+def test_input_beyond_fp16_range_is_reported(T):
+    """A block input of 1e5 (representable in bf16, not in fp16) is reported
+    as LMOE_ERR_DEVICE_CHECK on every dispatch path (few tokens, 9-63
+    tokens, tensor cores) instead of running on as inf."""
+    wl = prefill_workload(T) if T >= 64 else small_workload(T)
+    layer = synth.make_layer(wl)
+    dev = DeviceLayer(wl.shape, layer)
+    xb = synth.make_x(wl)
+    xb[T // 2, 7] = synth.bf16_bits_from_f32(np.array([1e5], np.float32))[0]
+    ws = dev.workspace(T)
+    dev.forward(to_device(xb, "cuda"), ws)
+    assert B.lmoe_last_device_status(ws) == B.LMOE_ERR_DEVICE_CHECK
+    # the same call on an in-range input is clean again
+    dev.forward(to_device(synth.make_x(wl), "cuda"), ws)
+    assert B.lmoe_last_device_status(ws) == B.LMOE_OK
