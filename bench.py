@@ -48,6 +48,7 @@ def parse():
     ap.add_argument("--copies", type=int, default=0, help="weight copies to rotate (0: enough to defeat L2)")
     ap.add_argument("--cpu-seconds", type=float, default=12.0, help="CPU-oracle sample budget")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-sweep", action="store_true", help="skip the MTP verify-window sweep")
     return ap.parse_args()
 
 
@@ -130,6 +131,7 @@ def step_cost(shape, idx: np.ndarray, groups: np.ndarray, T: int, prefill: bool)
     distinct = set(idx.reshape(-1).tolist())
     pairs_tg = sum(len({int(groups[e]) for e in idx[t]}) for t in range(idx.shape[0]))   # hit (token, group) pairs
     b = {
+        "k_decode_step": 0.0,
         "k_router_shared": rw + 2 * Fs * H * 2 + T * H * 2,
         "k_wstream_dproj": G * du + T * H * 2,     # every group (D runs before the routing is known)
         "k_wstream_gateup": len(distinct) * rec_gu,
@@ -138,6 +140,7 @@ def step_cost(shape, idx: np.ndarray, groups: np.ndarray, T: int, prefill: bool)
     }
     # the step's algorithmic bytes count only the hit groups' D
     b_total = float(sum(b.values()) - (G - len(hit)) * du)
+    b["k_decode_step"] = b_total            # the whole step in one kernel
     f = {
         "x_to_fp16": 0.0,
         "router_gemm": 2.0 * T * E * H,
@@ -186,8 +189,12 @@ def ncu_traffic(workload: str, T: int, kernel: str):
     return e[0]
 
 
-def decode_stages():
-    return ["k_router_shared", "k_wstream_dproj", "k_wstream_gateup", "k_wstream_down", "k_wstream_uproj"]
+def decode_stages(T: int):
+    """Kernels of one few-token step: one persistent kernel up to 8 tokens
+    (every Edge0-shaped layer fits it), five kernels from 9 to 63."""
+    if T <= 8:
+        return ["k_decode_step"]
+    return ["k_router_shared", "k_dproj_mma", "k_gateup_mma", "k_down_mma", "k_uproj_mma"]
 
 
 PREFILL_STAGES = ["x_to_fp16", "router_gemm", "topk_bucket", "shared_gateup", "dproj", "gateup", "down", "combine",
@@ -399,28 +406,45 @@ def weight_copies(base, R):
     return devs
 
 
-def measure_layer(args, wl, T, K, W, rank, world, local, dev_name):
-    """Times K steps of one layer at T tokens (graph replay), then the same
-    steps launched one by one with events between the library's kernels,
-    then K end-to-end steps through the host-buffer entry point.  Returns
-    the fields of a bench line and the layer (for the CPU baseline)."""
+class LayerCtx:
+    """One layer's weights on the device in R copies, rotated between steps so
+    that R - 1 steps of at least T_min tokens touch more than twice the L2
+    before a copy is reused."""
+
+    def __init__(self, args, wl, T_min, dev_name):
+        from latent_mixture_experts_softmax_b200 import binding as B
+        from latent_mixture_experts_softmax_b200 import synth
+        from latent_mixture_experts_softmax_b200.layer import DeviceLayer
+        self.layer = synth.make_layer(wl)
+        self.base = DeviceLayer(wl.shape, self.layer, device=dev_name)
+        s = wl.shape
+        # bytes a step of T_min tokens touches at least: every weight except
+        # the experts, plus the records of its routed experts (at least top_k)
+        self.touch = min(self.base.weight_bytes(), self.base.weight_bytes() - self.base.experts.numel()
+                         + s.top_k * B.lmoe_expert_record_bytes(self.base.cfg))
+        self.R = args.copies or (1 if self.touch > 2 * 126e6 else int(np.ceil(2 * 126e6 / self.touch)) + 1)
+        self.devs = weight_copies(self.base, self.R)
+
+
+def measure_layer(args, wl, T, K, W, rank, world, local, dev_name, ctx=None, light=False):
+    """Times K steps of one layer at T tokens (graph replay); unless light,
+    then the same steps launched one by one with events between the
+    library's kernels, then K end-to-end steps through the host-buffer entry
+    point.  Returns the fields of a bench line and the layer's host arrays
+    (for the CPU baseline)."""
     import torch
     import torch.distributed as dist
     from latent_mixture_experts_softmax_b200 import binding as B
     from latent_mixture_experts_softmax_b200 import synth
-    from latent_mixture_experts_softmax_b200.layer import DeviceLayer, to_device
+    from latent_mixture_experts_softmax_b200.layer import to_device
 
-    layer = synth.make_layer(wl)
-    base = DeviceLayer(wl.shape, layer, device=dev_name)
+    own_ctx = ctx is None
+    ctx = ctx or LayerCtx(args, wl, T, dev_name)
+    layer, base, devs, R = ctx.layer, ctx.base, ctx.devs, ctx.R
     s = wl.shape
-    # bytes a step can touch: every weight except the experts not routed
-    per_step_max = base.weight_bytes() - base.experts.numel() + 2 * T * s.top_k * B.lmoe_expert_record_bytes(base.cfg)
-    R = args.copies or max(1, int(np.ceil(2 * 126e6 / min(per_step_max, base.weight_bytes()))) + (
-        1 if per_step_max < 2 * 126e6 else 0))
-    devs = weight_copies(base, R)
     ws = base.workspace(T)
     prefill = T >= 64 and s.router_dtype == "bf16" and s.n_experts % 128 == 0
-    stages = PREFILL_STAGES if prefill else decode_stages()
+    stages = PREFILL_STAGES if prefill else decode_stages(T)
     # one CUDA graph per distinct step (its own token batch, weight copy and
     # output buffers); the timed loop replays them in turn
     n_graphs = min(K, 8 if prefill else 64)
@@ -466,6 +490,22 @@ def measure_layer(args, wl, T, K, W, rank, world, local, dev_name):
     status = B.lmoe_last_device_status(ws)
     del graphs
 
+    idx_np = idx_all.cpu().numpy()
+    groups = layer["expert_group"]
+    per_graph = [step_cost(s, idx_np[g], groups, T, prefill) for g in range(n_graphs)]
+    step_alg_bytes = float(np.mean([c["bytes_total"] for c in per_graph]))
+    step_flops = float(np.mean([c["flops_total"] for c in per_graph]))
+    nd = [c["n_distinct"] for c in per_graph]
+    hbm_peak, tc_peak, peak_src = load_peaks()
+    t_step = ms_max / K / 1e3
+    t_lb = max(step_alg_bytes / (hbm_peak * 1e9), step_flops / (tc_peak * 1e12))
+    if light:
+        del graphs
+        return {"T": T, "value": replica_throughput(world, T, K, ms_max), "ms_per_step": ms_max / K,
+                "distinct_experts_per_step": float(np.mean(nd)), "algorithmic_bytes": step_alg_bytes,
+                "gbs": step_alg_bytes / t_step / 1e9, "frac_of_roofline": t_lb / t_step,
+                "clocks": clk.summary(), "device_status": status}, layer
+
     # per-kernel durations: the same steps launched one by one, with CUDA
     # events the library records between its kernels on the step's stream
     # (serialised: these launches lose the overlap of the graph replay)
@@ -484,14 +524,7 @@ def measure_layer(args, wl, T, K, W, rank, world, local, dev_name):
             stage_ms[j] += evs[k][j].elapsed_time(evs[k][j + 1])
     stage_ms /= K2
 
-    idx_np = idx_all.cpu().numpy()
-    groups = layer["expert_group"]
-    per_graph = [step_cost(s, idx_np[g], groups, T, prefill) for g in range(n_graphs)]
     cost = {st: float(np.mean([c[st] for c in per_graph])) for st in stages}
-    step_alg_bytes = float(np.mean([c["bytes_total"] for c in per_graph]))
-    step_flops = float(np.mean([c["flops_total"] for c in per_graph]))
-    nd = [c["n_distinct"] for c in per_graph]
-    hbm_peak, tc_peak, peak_src = load_peaks()
     dom = int(np.argmax(stage_ms))
     dom_name = stages[dom]
     dom_s = stage_ms[dom] / 1e3
@@ -506,9 +539,6 @@ def measure_layer(args, wl, T, K, W, rank, world, local, dev_name):
         roof = {"bound": "hbm", "kernel": dom_name, "achieved": dom_ach, "peak": hbm_peak, "unit": "GB/s",
                 "frac": dom_ach / hbm_peak, "peak_source": f"{peak_src} HBM copy",
                 "traffic": ncu_traffic(wl.name, T, dom_name)}
-    t_step = ms_max / K / 1e3
-    t_lb = max(step_alg_bytes / (hbm_peak * 1e9), step_flops / (tc_peak * 1e12))
-
     # e2e through the host-buffer entry point (copies inside the timed region)
     x_pin = [torch.from_numpy(x.view(np.int16)).pin_memory() for x in xs_host]
     y_pin = torch.empty((T, s.hidden), dtype=torch.int16).pin_memory()
@@ -533,13 +563,13 @@ def measure_layer(args, wl, T, K, W, rank, world, local, dev_name):
         "value": replica_throughput(world, T, K, ms_max), "unit": "tokens/s", "steps": K, "warmup": W,
         "ms_per_step": ms_max / K,
         "config": {"workload": workload_desc(wl, T), "T": T, "parallelism": f"replicas x{world}",
-                   "l2": (f"inputs larger than L2: {R} weight copies rotated, "
-                          f"{R * min(per_step_max, base.weight_bytes()) / 1e6:.0f} MB touched between reuses"),
+                   "l2": (f"inputs larger than L2: {R} weight copies rotated, at least "
+                          f"{(R - 1) * ctx.touch / 1e6:.0f} MB touched between reuses of one"),
                    "weights": "NVFP4 experts, Q8_0/Q4_0 D/U, bf16 router and shared expert; "
                               "bf16 activations in and out, fp32 accumulation",
                    "path": ("tensor cores (tcgen05): fp16 operands dequantised from the stored formats"
-                            if prefill else "weight streaming on the tensor pipe (mma.sync, fp16 operands, fp32 "
-                                            "accumulation)"),
+                            if prefill else "one persistent kernel per step: weight streaming on the tensor pipe "
+                                            "(mma.sync, fp16 operands, fp32 accumulation)"),
                    "timing": f"{n_graphs} captured CUDA graphs replayed in turn"},
         "roofline": roof,
         "layer": {"gbs": step_alg_bytes / t_step / 1e9, "tflops": step_flops / t_step / 1e12,
@@ -560,7 +590,9 @@ def measure_layer(args, wl, T, K, W, rank, world, local, dev_name):
         "clocks": clk.summary(),
         "device_status": status,
     }
-    del devs, base, xs, ys
+    del xs, ys
+    if own_ctx:
+        del devs, base, ctx
     torch.cuda.synchronize()
     torch.cuda.empty_cache()
     return out, layer
@@ -597,11 +629,34 @@ def main():
         return
 
     K, W = args.steps, args.warmup
-    head, layer = measure_layer(args, wl, T, K, W, rank, world, local, dev_name)
+    decode = T < 64
+    windows = [t for t in (1, 2, 3, 8) if t != T] if decode and not args.no_sweep else []
+    ctx = LayerCtx(args, wl, min([T] + windows), dev_name)
+    head, layer = measure_layer(args, wl, T, K, W, rank, world, local, dev_name, ctx=ctx)
     line = {"metric": METRIC, "value": head["value"], "unit": "tokens/s", "n_gpus": world, "steps": K, "warmup": W,
             "ms_per_step": head["ms_per_step"], "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
             "dtype": "f16", "data": "synthetic"}
     line.update({k: v for k, v in head.items() if k not in line})
+    if windows:
+        # MTP verify windows of other sizes on the same weights: distinct
+        # experts a window routes to, against 3.05 x one token's at 4 tokens
+        # (the teardown article, "The engine computes the misses where they lie")
+        sweep = {T: {"T": T, "value": head["value"], "ms_per_step": head["ms_per_step"],
+                     "distinct_experts_per_step": head["distinct_experts_per_step"],
+                     "algorithmic_bytes": head["layer"]["algorithmic_bytes"], "gbs": head["layer"]["gbs"],
+                     "frac_of_roofline": head["layer"]["frac_of_roofline"]}}
+        for t in windows:
+            sweep[t], _ = measure_layer(args, wl, t, K, W, rank, world, local, dev_name, ctx=ctx, light=True)
+        one = sweep[1]["distinct_experts_per_step"] if 1 in sweep else float(wl.shape.top_k)
+        line["mtp_window"] = {
+            "windows": [sweep[t] for t in sorted(sweep)],
+            "distinct_ratio_vs_one_token": {str(t): sweep[t]["distinct_experts_per_step"] / one for t in sorted(sweep)},
+            "pages_ratio_at_4_tokens": 3.05,
+            "note": "distinct experts per window divided by those of one token (top_k); the pages' constant is for "
+                    "real routing, these windows draw independent synthetic tokens with a N(0,1) expert bias"}
+    del ctx
+    torch.cuda.synchronize()
+    torch.cuda.empty_cache()
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(wl, layer, T, args.cpu_seconds)
     pre_wl = None if args.prefill_workload == "none" or T >= 64 else synth.WORKLOADS[args.prefill_workload]

@@ -294,6 +294,11 @@ int forward_impl(const lmoe_cfg* cfg, const void* x, const void* router_w, const
     p.out_w = out_w;
     p.y = static_cast<uint16_t*>(y);
     if (use_prefill(*cfg, T)) return run_prefill(*cfg, p, L, ws, st);
+    if (T <= 8 && decode_step_fits(p)) {
+        // one kernel; it clears its own counters, so no per-call reset
+        stage_reset();
+        return cuda_status(run_decode_step(p, st));
+    }
     cudaError_t e = reset_tickets(ws, st);
     if (e != cudaSuccess) return LMOE_ERR_CUDA;
     return cuda_status(run_gemv_path(p, st, false));

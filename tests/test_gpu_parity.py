@@ -139,6 +139,16 @@ def test_block_few_tokens_ragged_steps(fmt, T):
     check_block(wl.shape, layer, synth.make_x(wl), residual_bits=res, what=f"ragged steps fmt={fmt} T={T}")
 
 
+@pytest.mark.parametrize("T", [2, 8])
+def test_block_wide_hidden_one_kernel_and_five_kernel_steps(T):
+    """hidden 4096: at 8 tokens the one-kernel step's shared memory does not
+    fit and the five-kernel few-token path runs; at 2 tokens the one-kernel
+    step runs.  Both against the oracle."""
+    wl = small_workload(T, hidden=4096, latent=256, n_experts=48, top_k=6, n_groups=4, ffn=128, shared_ffn=128)
+    layer = synth.make_layer(wl)
+    check_block(wl.shape, layer, synth.make_x(wl), what=f"hidden 4096 T={T}")
+
+
 def test_block_tiny_config():
     wl = synth.WORKLOADS["tiny"]
     check_block(wl.shape, synth.make_layer(wl), synth.make_x(wl), what="tiny")
