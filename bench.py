@@ -500,7 +500,6 @@ def measure_layer(args, wl, T, K, W, rank, world, local, dev_name, ctx=None, lig
     t_step = ms_max / K / 1e3
     t_lb = max(step_alg_bytes / (hbm_peak * 1e9), step_flops / (tc_peak * 1e12))
     if light:
-        del graphs
         return {"T": T, "value": replica_throughput(world, T, K, ms_max), "ms_per_step": ms_max / K,
                 "distinct_experts_per_step": float(np.mean(nd)), "algorithmic_bytes": step_alg_bytes,
                 "gbs": step_alg_bytes / t_step / 1e9, "frac_of_roofline": t_lb / t_step,
@@ -598,6 +597,59 @@ def measure_layer(args, wl, T, K, W, rank, world, local, dev_name, ctx=None, lig
     return out, layer
 
 
+def dproj_ablation(ctx, wl, K, dev_name):
+    """D_g alone, as the reference kernel runs it (Q8_1 activations, every
+    group) and as this library needs it (fp16 activations, only the groups a
+    batch hits), at 1 and 4 tokens.  Each launch reads its D from one of the
+    R weight copies after an L2 flush; events bracket the kernels only."""
+    import torch
+    from latent_mixture_experts_softmax_b200 import binding as B
+    from latent_mixture_experts_softmax_b200 import synth
+    from latent_mixture_experts_softmax_b200.layer import to_device
+    s = wl.shape
+    G = s.n_groups
+    flush = torch.empty(256 * 2 ** 20, dtype=torch.uint8, device=dev_name)
+    du = B.lmoe_du_bytes(ctx.base.cfg) // G
+    hbm, _, src = load_peaks()
+    out = {"note": "weights read from HBM (L2 flushed before every launch); Q8_1: k_quantize_q8_1 + the D kernel",
+           "peak_gbs": hbm, "peak_source": src}
+    n = max(20, min(K, 100))
+    for T in (1, 4):
+        xs = [to_device(synth.make_x(wl, T=T, draw=700 + i), dev_name) for i in range(4)]
+        ws = ctx.base.workspace(T)
+        h = torch.empty((T, G, s.latent), dtype=torch.float32, device=dev_name)
+        idx = torch.empty((T, s.top_k), dtype=torch.int32, device=dev_name)
+        w = torch.empty((T, s.top_k), dtype=torch.float32, device=dev_name)
+        masks = []
+        for x in xs:
+            B.lmoe_route(ctx.base.cfg, x, ctx.base.router_w, ctx.base.router_b, T, idx, w, ws)
+            masks.append(sum(1 << int(g) for g in {int(ctx.layer["expert_group"][e]) for e in idx.cpu().numpy().ravel()}))
+        res = {}
+        for name, fmt, use_hit in (("q8_1_all_groups", 1, False), ("fp16_all_groups", 0, False),
+                                   ("fp16_hit_groups", 0, True)):
+            ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(n)]
+            groups = []
+            for i in range(n + 3):
+                d = ctx.devs[i % ctx.R]
+                mask = masks[i % 4] if use_hit else (1 << G) - 1
+                flush.zero_()
+                if i >= 3:
+                    ev[i - 3][0].record()
+                B.lmoe_dproj_ablation(d.cfg, xs[i % 4], d.D, fmt, mask, h, T, ws)
+                if i >= 3:
+                    ev[i - 3][1].record()
+                    groups.append(bin(mask).count("1"))
+            torch.cuda.synchronize()
+            us = float(np.mean([a.elapsed_time(b) for a, b in ev])) * 1e3
+            gb = float(np.mean(groups)) * du + T * s.hidden * 2
+            res[name] = {"us": us, "groups": float(np.mean(groups)), "gbs": gb / (us * 1e-6) / 1e9,
+                         "frac_of_hbm": gb / (us * 1e-6) / 1e9 / hbm}
+        res["speedup_ours_vs_reference"] = res["q8_1_all_groups"]["us"] / res["fp16_hit_groups"]["us"]
+        out[f"T{T}"] = res
+    del flush
+    return out
+
+
 def main():
     args = parse()
     rank = int(os.environ.get("RANK", "0"))
@@ -654,6 +706,8 @@ def main():
             "pages_ratio_at_4_tokens": 3.05,
             "note": "distinct experts per window divided by those of one token (top_k); the pages' constant is for "
                     "real routing, these windows draw independent synthetic tokens with a N(0,1) expert bias"}
+    if decode and not args.no_sweep:
+        line["ablation_dproj"] = dproj_ablation(ctx, wl, K, dev_name)
     del ctx
     torch.cuda.synchronize()
     torch.cuda.empty_cache()

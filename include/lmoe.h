@@ -216,6 +216,22 @@ LMOE_API int lmoe_debug_decode(int fmt, const void* blob, int rows, int cols, fl
  * the caller; n = 0 turns recording off.  At most 16 events. */
 LMOE_API int lmoe_profile_stage_events(void* const* events, int n);
 
+/* Ablation of D_g.  Defining passage: teardown article, section "A latent
+ * in front of the experts" -- its code excerpt shows the reference kernel
+ * quantising each token row to Q8_1 and running D over all 8 groups with
+ * integer dot products, where this library runs D on fp16 activations and
+ * needs only the groups a token hits.  h fp32 [T][n_groups][latent] =
+ * D_g x for every group g with bit g of group_mask set (other groups of h
+ * are not written):
+ *   act_fmt 0  fp16 activations, fp16 x fp16 tensor-core products, fp32 sums
+ *   act_fmt 1  Q8_1 activations: per block of 32, d = fp16(amax / 127) and
+ *              q = rint(x / d) clamped to +-127 (fp32 operations), then
+ *              integer products per block scaled by d_w * d
+ * x bf16 [T][hidden]; D as in lmoe_forward; ws of lmoe_workspace_bytes(cfg,
+ * T).  n_groups <= 32.  Errors: LMOE_ERR_ARG, _UNSUPPORTED, _WORKSPACE. */
+LMOE_API int lmoe_dproj_ablation(const lmoe_cfg* cfg, const void* x, const void* D, int act_fmt, uint32_t group_mask,
+                                 float* h, int T, void* ws, size_t ws_bytes, void* stream);
+
 /* Router only, for callers that cannot call cudaMalloc (code inside a host
  * framework that owns every device allocation, or a path where no workspace
  * can be handed in).  Same results as lmoe_route, but the scratch lives in a

@@ -28,7 +28,7 @@ LMOE_NVFP4_DEBUG = 1
 EXPORTS = ("lmoe_cfg_check", "lmoe_expert_record_bytes", "lmoe_du_bytes", "lmoe_workspace_bytes", "lmoe_route",
            "lmoe_forward", "lmoe_forward_ex", "lmoe_forward_host", "lmoe_stack_forward", "lmoe_last_device_status",
            "lmoe_status_str", "lmoe_debug_decode", "lmoe_profile_stage_events",
-           "lmoe_route_noalloc")
+           "lmoe_route_noalloc", "lmoe_dproj_ablation")
 
 
 class LmoeError(RuntimeError):
@@ -92,6 +92,8 @@ def lib() -> ctypes.CDLL:
         L.lmoe_profile_stage_events.restype = i32
         L.lmoe_route_noalloc.argtypes = [cfgp, vp, vp, vp, i32, vp, vp, vp]
         L.lmoe_route_noalloc.restype = i32
+        L.lmoe_dproj_ablation.argtypes = [cfgp, vp, vp, i32, ctypes.c_uint32, vp, i32, vp, sz, vp]
+        L.lmoe_dproj_ablation.restype = i32
         _lib = L
     return _lib
 
@@ -224,3 +226,10 @@ def lmoe_route_noalloc(cfg, x, router_w, router_b, T, topk_idx, topk_w, stream=N
     """Router without a workspace (scratch is a fixed array inside the library)."""
     return _check(lib().lmoe_route_noalloc(ctypes.byref(cfg), _ptr(x), _ptr(router_w), _ptr(router_b), T,
                                            _ptr(topk_idx), _ptr(topk_w), _stream(stream)), "lmoe_route_noalloc")
+
+
+def lmoe_dproj_ablation(cfg, x, D, act_fmt, group_mask, h, T, ws, stream=None):
+    """D_g x for the groups of group_mask, fp16 (act_fmt 0) or Q8_1 (1) activations."""
+    return _check(lib().lmoe_dproj_ablation(ctypes.byref(cfg), _ptr(x), _ptr(D), int(act_fmt), int(group_mask),
+                                            _ptr(h), T, _ptr(ws), _nbytes(ws), _stream(stream)),
+                  "lmoe_dproj_ablation")

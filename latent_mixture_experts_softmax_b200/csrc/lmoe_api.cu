@@ -452,6 +452,25 @@ int lmoe_profile_stage_events(void* const* events, int n) {
     return LMOE_OK;
 }
 
+int lmoe_dproj_ablation(const lmoe_cfg* cfg, const void* x, const void* D, int act_fmt, uint32_t group_mask, float* h,
+                        int T, void* ws, size_t ws_bytes, void* stream) {
+    int s = check_cfg(cfg);
+    if (s != LMOE_OK) return s;
+    if (!x || !D || !h || T < 0 || (act_fmt != 0 && act_fmt != 1)) return LMOE_ERR_ARG;
+    if (!aligned(x, 16) || !aligned(D, 16) || !aligned(h, 4)) return LMOE_ERR_ARG;
+    if (cfg->n_groups > 32) return LMOE_ERR_UNSUPPORTED;
+    if (T == 0) return LMOE_OK;
+    if (!ws || !aligned(ws, 256)) return LMOE_ERR_ARG;
+    const WsLayout L = ws_layout(*cfg, T);
+    if (L.total > ws_bytes) return LMOE_ERR_WORKSPACE;
+    // the Q8_1 rows use the workspace's two spare activation buffers
+    if (dproj_ablation_ws_bytes(T, cfg->hidden) > L.idx - L.xa) return LMOE_ERR_WORKSPACE;
+    return cuda_status(run_dproj_ablation(static_cast<const uint16_t*>(x), static_cast<const uint8_t*>(D), T,
+                                          cfg->hidden, cfg->latent, cfg->n_groups, cfg->du_fmt, act_fmt, group_mask,
+                                          du_matrix_bytes(*cfg), h, static_cast<char*>(ws) + L.xa,
+                                          static_cast<cudaStream_t>(stream)));
+}
+
 int lmoe_debug_decode(int fmt, const void* blob, int rows, int cols, float ts, float* out, void* stream) {
     if (!blob || !out || rows <= 0 || cols <= 0 || cols % 64 || !aligned(blob, 16)) return LMOE_ERR_ARG;
     if (fmt != LMOE_Q8_0 && fmt != LMOE_Q4_0 && fmt != 1) return LMOE_ERR_UNSUPPORTED;

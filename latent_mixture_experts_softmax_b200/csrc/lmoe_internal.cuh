@@ -101,5 +101,9 @@ void stage_mark(cudaStream_t st);
 void stage_reset();
 cudaError_t ensure_smem(const void* kernel, size_t smem);
 cudaError_t run_debug_decode(int fmt, const void* blob, int R, int C, float ts, float* out, cudaStream_t st);
+// D over a set of groups with fp16 or Q8_1 activations (the ablation)
+size_t dproj_ablation_ws_bytes(int T, int H);
+cudaError_t run_dproj_ablation(const uint16_t* x, const uint8_t* D, int T, int H, int L, int G, int fmt, int q81,
+                               uint32_t gmask, size_t du_bytes, float* h, void* ws, cudaStream_t st);
 
 }  // namespace lmoe

@@ -63,6 +63,12 @@ def lib():
         L.lmoe_synth_nvfp4_experts.argtypes = [u64, dbl, i32, i32, i32, vp]
         L.lmoe_synth_nvfp4_encode.restype = ctypes.c_float
         L.lmoe_synth_nvfp4_encode.argtypes = [vp, i32, i32, vp, vp]
+        for n in ("lmoe_synth_q3k_bytes", "lmoe_synth_iq4nl_bytes", "lmoe_synth_q3k_record_bytes"):
+            getattr(L, n).restype = ctypes.c_size_t
+            getattr(L, n).argtypes = [i32, i32]
+        L.lmoe_synth_q3k_encode.argtypes = [vp, i32, i32, vp]
+        L.lmoe_synth_iq4nl_encode.argtypes = [vp, i32, i32, vp]
+        L.lmoe_synth_q3k_experts.argtypes = [u64, dbl, i32, i32, i32, vp]
         _lib = L
     return _lib
 
@@ -87,6 +93,7 @@ class LayerShape:
     shared_ffn: int = 640
     du_fmt: int = Q8_0          # 8: Q8_0, 4: Q4_0
     router_dtype: str = "bf16"  # "f32" or "bf16"
+    expert_fmt: str = "nvfp4"   # "nvfp4", or "q3k" (Q3_K gate/up + IQ4_NL down)
 
 
 @dataclass(frozen=True)
@@ -108,6 +115,7 @@ class Workload:
 
 SHAPE_120B = LayerShape(latent=1280, du_fmt=Q4_0)
 SHAPE_145B = LayerShape(latent=1792, du_fmt=Q8_0)
+SHAPE_145B_Q3K = LayerShape(latent=1792, du_fmt=Q8_0, expert_fmt="q3k")
 
 WORKLOADS = {
     # 8 tokens, 64 experts, latent 1280, Q4_0 D/U, fp32 router, no bias, expert_group = e % 8
@@ -119,6 +127,11 @@ WORKLOADS = {
     "edge0_145b_decode": Workload("edge0_145b_decode", SHAPE_145B, T=4, groups="uniform", bias_sigma=1.0),
     # Edge0-145B-shaped layer, prefill of 4096 (and 16384) tokens
     "edge0_145b_prefill": Workload("edge0_145b_prefill", SHAPE_145B, T=4096, groups="uniform", bias_sigma=0.5),
+    # the same layer with the other expert build (Q3_K gate/up + IQ4_NL down)
+    "edge0_145b_q3k_decode": Workload("edge0_145b_q3k_decode", SHAPE_145B_Q3K, T=4, groups="uniform",
+                                      bias_sigma=1.0),
+    "edge0_145b_q3k_prefill": Workload("edge0_145b_q3k_prefill", SHAPE_145B_Q3K, T=4096, groups="uniform",
+                                       bias_sigma=0.5),
     # 48 stacked Edge0-145B-shaped layers with pre-RMSNorm and residual
     "edge0_145b_stack": Workload("edge0_145b_stack", SHAPE_145B, T=4, groups="uniform", bias_sigma=1.0,
                                  n_layers=48),
@@ -147,7 +160,9 @@ def du_matrix_bytes(fmt: int, rows: int, cols: int) -> int:
     return rows * cols // 32 * per32
 
 
-def expert_record_bytes(latent: int, ffn: int) -> int:
+def expert_record_bytes(latent: int, ffn: int, expert_fmt: str = "nvfp4") -> int:
+    if expert_fmt == "q3k":
+        return int(lib().lmoe_synth_q3k_record_bytes(latent, ffn))
     return int(lib().lmoe_synth_nvfp4_record_bytes(latent, ffn))
 
 
@@ -219,6 +234,33 @@ def expert_record_encode(w_gate: np.ndarray, w_up: np.ndarray, w_down: np.ndarra
     return rec
 
 
+def q3k_encode(w: np.ndarray) -> np.ndarray:
+    """Pack a matrix [rows, cols] (cols a multiple of 256) into the Q3_K planes."""
+    w = np.ascontiguousarray(w, np.float64)
+    out = np.zeros(int(lib().lmoe_synth_q3k_bytes(*w.shape)), np.uint8)
+    lib().lmoe_synth_q3k_encode(_p(w), w.shape[0], w.shape[1], _p(out))
+    return out
+
+
+def iq4nl_encode(w: np.ndarray) -> np.ndarray:
+    """Pack a matrix [rows, cols] (cols a multiple of 32) into the IQ4_NL planes."""
+    w = np.ascontiguousarray(w, np.float64)
+    out = np.zeros(int(lib().lmoe_synth_iq4nl_bytes(*w.shape)), np.uint8)
+    lib().lmoe_synth_iq4nl_encode(_p(w), w.shape[0], w.shape[1], _p(out))
+    return out
+
+
+def q3k_record_encode(w_gate: np.ndarray, w_up: np.ndarray, w_down: np.ndarray) -> np.ndarray:
+    """One expert of the Q3_K build from given gate [F, L], up [F, L], down [L, F]."""
+    return np.concatenate([q3k_encode(w_gate), q3k_encode(w_up), iq4nl_encode(w_down)])
+
+
+def q3k_experts(k: int, sigma: float, E: int, latent: int, ffn: int) -> np.ndarray:
+    out = np.zeros(E * expert_record_bytes(latent, ffn, "q3k"), np.uint8)
+    lib().lmoe_synth_q3k_experts(k, sigma, E, latent, ffn, _p(out))
+    return out
+
+
 def expert_groups(wl: Workload, layer: int = 0) -> np.ndarray:
     E, G = wl.shape.n_experts, wl.shape.n_groups
     if wl.groups == "mod":
@@ -248,7 +290,10 @@ def make_layer(wl: Workload, layer: int = 0) -> dict:
     out["expert_group"] = expert_groups(wl, layer)
     out["D"] = np.concatenate([qmatrix(s.du_fmt, key(seed, layer, "D", g), sig, L, H) for g in range(G)])
     out["U"] = np.concatenate([qmatrix(s.du_fmt, key(seed, layer, "U", g), sig, H, L) for g in range(G)])
-    out["experts"] = experts_normal(key(seed, layer, "experts"), sig, E, L, F)
+    if s.expert_fmt == "q3k":
+        out["experts"] = q3k_experts(key(seed, layer, "experts"), sig, E, L, F)
+    else:
+        out["experts"] = experts_normal(key(seed, layer, "experts"), sig, E, L, F)
     out["shared_gate"] = bf16_normal(key(seed, layer, "shared_gate"), sig, (Fs, H))
     out["shared_up"] = bf16_normal(key(seed, layer, "shared_up"), sig, (Fs, H))
     out["shared_down"] = bf16_normal(key(seed, layer, "shared_down"), sig, (H, Fs))

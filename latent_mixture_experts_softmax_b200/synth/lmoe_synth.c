@@ -287,3 +287,143 @@ float lmoe_synth_nvfp4_encode(const double* w, int R, int C, uint8_t* q, uint8_t
     memset(q, 0, (size_t)R * C / 2);
     return nvfp4_pack(w, R, C, q, s);
 }
+
+/* ---------------- Q3_K gate/up + IQ4_NL down expert records ----------------
+ * The other expert build of the pages: Q3_K for gate and up, IQ4_NL for
+ * down, 985,600 + 645,120 = 1,630,720 bytes per record at latent 1792 and
+ * ffn 640 (1,164,800 at latent 1280).  The pages give the type names and the
+ * byte totals, not the bit arrangement; the arrangement below is this
+ * project's, with exactly those byte counts:
+ *
+ *   Q3_K matrix [R, C] (C a multiple of 256): 110 bytes per 256 weights of a
+ *   row, stored as planes over 128-column halves h = c / 128:
+ *     lo [C/128][R][32]  2-bit low code parts; 32-bit word w (0..7) of a row's
+ *                        32 bytes covers elements 16w..16w+15, element
+ *                        16w + 4i + b in byte b, bits 2i..2i+1
+ *     hi [C/128][R][16]  high code bits; word v (0..3) covers elements
+ *                        32v..32v+31, element 32v + 4i + b in byte b, bit i
+ *     sc [C/128][R][6]   eight 6-bit sub-block scales (sub-block j = elements
+ *                        16j..16j+15 of the half) at bits 6j..6j+5 of the
+ *                        48-bit little-endian word
+ *     d  [C/256][R]      fp16 super-block scale
+ *     weight = d * (sc_j - 32) * (q - 4),  q = lo | hi << 2  in 0..7
+ *   IQ4_NL matrix [R, C] (C a multiple of 32): 18 bytes per 32 weights:
+ *     q  [C/32][R][16]   4-bit indices, byte j: element j (low nibble) and
+ *                        element j + 16 (high nibble)
+ *     d  [C/32][R]       fp16 block scale
+ *     weight = d * level[q]; the 16 levels are not printed on the pages: here
+ *     they are the standard normal quantiles at (i + 1/2) / 16, scaled so the
+ *     outermost is 127 and rounded (the table below, from that definition)
+ *   record: gate (Q3_K [F, L]) | up (Q3_K [F, L]) | down (IQ4_NL [L, F]).
+ */
+static const int kIq4Levels[16] = {-127, -90, -69, -53, -39, -27, -16, -5, 5, 16, 27, 39, 53, 69, 90, 127};
+
+size_t lmoe_synth_q3k_bytes(int R, int C) { return (size_t)R * C / 256 * 110; }
+size_t lmoe_synth_iq4nl_bytes(int R, int C) { return (size_t)R * C / 32 * 18; }
+size_t lmoe_synth_q3k_record_bytes(int L, int F) {
+    return 2 * lmoe_synth_q3k_bytes(F, L) + lmoe_synth_iq4nl_bytes(L, F);
+}
+
+/* Encode w [R, C] (row-major fp64) into the Q3_K planes at out. */
+void lmoe_synth_q3k_encode(const double* w, int R, int C, uint8_t* out) {
+    const size_t nh = (size_t)C / 128;
+    uint8_t* lo = out;
+    uint8_t* hi = lo + nh * R * 32;
+    uint8_t* sc = hi + nh * R * 16;
+    uint16_t* dd = (uint16_t*)(sc + nh * R * 6);
+    memset(out, 0, lmoe_synth_q3k_bytes(R, C));
+    for (int r = 0; r < R; ++r) {
+        for (int sb = 0; sb < C / 256; ++sb) {
+            const double* ws = w + (size_t)r * C + (size_t)sb * 256;
+            /* sub-block scales: the signed element of largest magnitude maps to -4 */
+            double s[16], smax = 0.0;
+            for (int j = 0; j < 16; ++j) {
+                double m = 0.0;
+                for (int k = 0; k < 16; ++k) if (fabs(ws[16 * j + k]) > fabs(m)) m = ws[16 * j + k];
+                s[j] = m / -4.0;
+                if (fabs(s[j]) > smax) smax = fabs(s[j]);
+            }
+            uint16_t dh = f64_to_fp16_rne(smax / 31.0);
+            double dv = fp16_value(dh);
+            dd[(size_t)sb * R + r] = dh;
+            for (int j = 0; j < 16; ++j) {
+                double f = dv > 0.0 ? rint(s[j] / dv) : 0.0;
+                if (f > 31.0) f = 31.0;
+                if (f < -32.0) f = -32.0;
+                const int scj = (int)f + 32;
+                const double e = dv * f;
+                const int h = (sb * 256 + 16 * j) / 128, jj = j % 8;
+                uint8_t* scp = sc + ((size_t)h * R + r) * 6;
+                /* 6 bits at bit 6*jj of the 48-bit little-endian word */
+                for (int b = 0; b < 6; ++b) {
+                    const int bit = 6 * jj + b;
+                    if ((scj >> b) & 1) scp[bit / 8] |= (uint8_t)(1u << (bit % 8));
+                }
+                for (int k = 0; k < 16; ++k) {
+                    const int c = sb * 256 + 16 * j + k, e128 = c % 128;
+                    double qv = e != 0.0 ? rint(ws[16 * j + k] / e) + 4.0 : 4.0;
+                    if (qv > 7.0) qv = 7.0;
+                    if (qv < 0.0) qv = 0.0;
+                    const int q = (int)qv;
+                    /* low bits: word e128/16, i = (e128 % 16) / 4, byte b = e128 % 4 */
+                    const int wlo = e128 / 16, ilo = (e128 % 16) / 4, blo = e128 % 4;
+                    lo[((size_t)h * R + r) * 32 + 4 * wlo + blo] |= (uint8_t)((q & 3) << (2 * ilo));
+                    const int whi = e128 / 32, ihi = (e128 % 32) / 4, bhi = e128 % 4;
+                    if (q & 4) hi[((size_t)h * R + r) * 16 + 4 * whi + bhi] |= (uint8_t)(1u << ihi);
+                }
+            }
+        }
+    }
+}
+
+/* Encode w [R, C] into the IQ4_NL planes at out: d = amax / 127, index of
+ * the nearest level (the lower one on a tie). */
+void lmoe_synth_iq4nl_encode(const double* w, int R, int C, uint8_t* out) {
+    uint8_t* qs = out;
+    uint16_t* dd = (uint16_t*)(out + (size_t)R * C / 2);
+    memset(out, 0, lmoe_synth_iq4nl_bytes(R, C));
+    for (int r = 0; r < R; ++r) {
+        for (int b = 0; b < C / 32; ++b) {
+            const double* wb = w + (size_t)r * C + (size_t)b * 32;
+            double amax = 0.0;
+            for (int j = 0; j < 32; ++j) if (fabs(wb[j]) > amax) amax = fabs(wb[j]);
+            uint16_t dh = f64_to_fp16_rne(amax / 127.0);
+            double dv = fp16_value(dh);
+            dd[(size_t)b * R + r] = dh;
+            uint8_t* q = qs + ((size_t)b * R + r) * 16;
+            for (int j = 0; j < 32; ++j) {
+                int best = 0;
+                if (dv > 0.0) {
+                    const double t = wb[j] / dv;
+                    for (int i = 1; i < 16; ++i)
+                        if (fabs(t - kIq4Levels[i]) < fabs(t - kIq4Levels[best])) best = i;
+                }
+                if (j < 16) q[j] |= (uint8_t)best;
+                else q[j - 16] |= (uint8_t)(best << 4);
+            }
+        }
+    }
+}
+
+/* E experts in the Q3_K build; matrix m (0 gate [F, L], 1 up, 2 down [L, F]) of
+ * expert e drawn as sigma * normal(key(key(key, e), m), r * C + c). */
+void lmoe_synth_q3k_experts(uint64_t key, double sigma, int E, int L, int F, uint8_t* out) {
+    const size_t rec = lmoe_synth_q3k_record_bytes(L, F);
+    const size_t gb = lmoe_synth_q3k_bytes(F, L);
+#pragma omp parallel
+    {
+        double* w = (double*)malloc(sizeof(double) * (size_t)L * F);
+#pragma omp for schedule(dynamic, 1)
+        for (int e = 0; e < E; ++e) {
+            uint8_t* r = out + rec * (size_t)e;
+            for (int m = 0; m < 3; ++m) {
+                int R = m < 2 ? F : L, C = m < 2 ? L : F;
+                uint64_t km = lmoe_synth_key(lmoe_synth_key(key, (uint64_t)e), (uint64_t)m);
+                for (size_t i = 0; i < (size_t)R * C; ++i) w[i] = sigma * lmoe_synth_normal(km, i);
+                if (m < 2) lmoe_synth_q3k_encode(w, R, C, r + gb * m);
+                else lmoe_synth_iq4nl_encode(w, R, C, r + 2 * gb);
+            }
+        }
+        free(w);
+    }
+}

@@ -143,32 +143,118 @@ double nvfp4_weight(const uint8_t* q, const uint8_t* s, double ts, int R, int r,
     return e2m1_value(code) * e4m3fn_value(scode) * ts;
 }
 
+// The other expert build (model page, "Model profile": Q3_K gate/up and
+// IQ4_NL down; teardown article, "What is 4-bit": 985,600 + 645,120 bytes is
+// the 1,630,720-byte record).  The pages give the type names and byte counts
+// only; the block arrangement is this project's (documented with the C ABI):
+//   Q3_K [R][C], 110 bytes per 256 weights of a row, planes over 128-column
+//   halves h: lo [C/128][R][32] (element 16w + 4i + b: byte 4w + b, bits
+//   2i..2i+1), hi [C/128][R][16] (element 32v + 4i + b: byte 4v + b, bit i),
+//   sc [C/128][R][6] (sub-block j of the half: bits 6j..6j+5, little-endian),
+//   d fp16 [C/256][R];  w = d * (sc_j - 32) * (q - 4), q = lo | hi << 2
+//   IQ4_NL [R][C], 18 bytes per 32: q [C/32][R][16] (as Q4_0), d fp16
+//   [C/32][R];  w = d * level[q]
+// The 16 IQ4_NL levels are not printed on the pages; they are read here as
+// the standard normal quantiles at (i + 1/2) / 16, scaled so that the
+// outermost is 127, rounded to integers (computed below from that definition).
+double normal_quantile(double p) {
+    double lo = -10.0, hi = 10.0;       // Phi(x) = erfc(-x / sqrt 2) / 2, by bisection
+    for (int it = 0; it < 200; ++it) {
+        const double mid = 0.5 * (lo + hi);
+        if (0.5 * std::erfc(-mid / std::sqrt(2.0)) < p) lo = mid;
+        else hi = mid;
+    }
+    return 0.5 * (lo + hi);
+}
+
+const double* iq4nl_levels() {
+    static double levels[16];
+    static bool done = false;
+    if (!done) {
+        const double top = normal_quantile(15.5 / 16.0);
+        for (int i = 0; i < 16; ++i) levels[i] = std::nearbyint(127.0 * normal_quantile((i + 0.5) / 16.0) / top);
+        done = true;
+    }
+    return levels;
+}
+
+int64_t q3k_matrix_bytes(int R, int C) { return (int64_t)R * C / 256 * 110; }
+int64_t iq4nl_matrix_bytes(int R, int C) { return (int64_t)R * C / 32 * 18; }
+
+double q3k_weight(const uint8_t* m, int R, int C, int r, int c) {
+    const int64_t nh = C / 128;
+    const uint8_t* lo = m;
+    const uint8_t* hi = lo + nh * R * 32;
+    const uint8_t* sc = hi + nh * R * 16;
+    const uint8_t* d = sc + nh * R * 6;
+    const int h = c / 128, e = c % 128;
+    const int q_lo = (lo[((int64_t)h * R + r) * 32 + 4 * (e / 16) + e % 4] >> (2 * ((e % 16) / 4))) & 3;
+    const int q_hi = (hi[((int64_t)h * R + r) * 16 + 4 * (e / 32) + e % 4] >> ((e % 32) / 4)) & 1;
+    const int q = q_lo | (q_hi << 2);
+    const int j = e / 16;
+    int scj = 0;
+    for (int b = 0; b < 6; ++b) {
+        const int bit = 6 * j + b;
+        scj |= ((sc[((int64_t)h * R + r) * 6 + bit / 8] >> (bit % 8)) & 1) << b;
+    }
+    const double dv = fp16_value(load_u16(d + 2 * ((int64_t)(c / 256) * R + r)));
+    return dv * (scj - 32) * (q - 4);
+}
+
+double iq4nl_weight(const uint8_t* m, int R, int C, int r, int c) {
+    const int64_t blk = (int64_t)(c / 32) * R + r;
+    const int j = c % 32;
+    const uint8_t byte = m[blk * 16 + (j % 16)];
+    const int q = j < 16 ? (byte & 0xF) : (byte >> 4);
+    const double d = fp16_value(load_u16(m + (int64_t)R * C / 2 + 2 * blk));
+    return d * iq4nl_levels()[q];
+}
+
 // Row r of a stored matrix into out[0..C).
 void du_row(int fmt, const uint8_t* m, int R, int C, int r, double* out) {
     for (int c = 0; c < C; ++c) out[c] = du_weight(fmt, m, R, C, r, c);
 }
 
-// One NVFP4 matrix of an expert record: which = 0 gate [F][L], 1 up [F][L], 2 down [L][F].
-struct Nvfp4View {
-    const uint8_t* q;
-    const uint8_t* s;
+// One matrix of an expert record: which = 0 gate [F][L], 1 up [F][L], 2 down
+// [L][F].  efmt 0: NVFP4 record (codes, scales, tensor-scale tail); efmt 1:
+// the Q3_K build (gate and up Q3_K, down IQ4_NL, no tail).
+struct ExpertMatrix {
+    int kind;            // 0 NVFP4, 1 Q3_K, 2 IQ4_NL
+    const uint8_t* q;    // NVFP4 codes, or the whole Q3_K / IQ4_NL matrix
+    const uint8_t* s;    // NVFP4 scales
     double ts;
     int R, C;
 };
 
-Nvfp4View expert_matrix(const uint8_t* rec, int L, int F, int which) {
+int64_t expert_record_bytes_fmt(int efmt, int L, int F) {
+    return efmt == 1 ? 2 * q3k_matrix_bytes(F, L) + iq4nl_matrix_bytes(L, F) : expert_record_bytes(L, F);
+}
+
+ExpertMatrix expert_matrix(const uint8_t* rec, int L, int F, int which, int efmt = 0) {
+    ExpertMatrix v;
+    v.R = which < 2 ? F : L;
+    v.C = which < 2 ? L : F;
+    v.s = nullptr;
+    v.ts = 1.0;
+    if (efmt == 1) {
+        v.kind = which < 2 ? 1 : 2;
+        v.q = rec + which * q3k_matrix_bytes(F, L);
+        return v;
+    }
     const int64_t nq = (int64_t)L * F / 2, ns = (int64_t)L * F / 16;
-    Nvfp4View v;
+    v.kind = 0;
     v.q = rec + which * nq;
     v.s = rec + 3 * nq + which * ns;
     v.ts = (double)load_f32(rec + 3 * nq + 3 * ns + 4 * which);
-    v.R = which < 2 ? F : L;
-    v.C = which < 2 ? L : F;
     return v;
 }
 
-void nvfp4_row(const Nvfp4View& v, int r, double* out) {
-    for (int c = 0; c < v.C; ++c) out[c] = nvfp4_weight(v.q, v.s, v.ts, v.R, r, c);
+void nvfp4_row(const ExpertMatrix& v, int r, double* out) {
+    for (int c = 0; c < v.C; ++c) {
+        if (v.kind == 0) out[c] = nvfp4_weight(v.q, v.s, v.ts, v.R, r, c);
+        else if (v.kind == 1) out[c] = q3k_weight(v.q, v.R, v.C, r, c);
+        else out[c] = iq4nl_weight(v.q, v.R, v.C, r, c);
+    }
 }
 
 double dot(const double* a, const double* b, int n) {
@@ -187,6 +273,7 @@ struct orc_shape {
     int hidden, latent, n_experts, top_k, n_groups, ffn, shared_ffn;
     int du_fmt;        // 8: Q8_0, 4: Q4_0
     int router_bf16;   // 1: router weights are bf16 bits, 0: fp32
+    int expert_fmt;    // 0: NVFP4 records, 1: Q3_K gate/up + IQ4_NL down records
 };
 
 struct orc_layer {
@@ -210,6 +297,7 @@ int64_t orc_expert_record_bytes(int L, int F) { return expert_record_bytes(L, F)
 // Byte offset of group g's matrix in a D or U blob, and of expert e's record.
 int64_t orc_du_offset(int fmt, int g, int R, int C) { return (int64_t)g * du_matrix_bytes(fmt, R, C); }
 int64_t orc_expert_offset(int e, int L, int F) { return (int64_t)e * expert_record_bytes(L, F); }
+int64_t orc_expert_offset_fmt(int efmt, int e, int L, int F) { return (int64_t)e * expert_record_bytes_fmt(efmt, L, F); }
 
 // ---- scalar decoders over arrays -----------------------------------------------
 
@@ -239,17 +327,43 @@ int orc_decode_du(int fmt, const uint8_t* blob, int R, int C, double* out) {
 // NVFP4 matrix [R][C] (codes q, scales s, tensor scale ts) -> out [R][C].
 int orc_decode_nvfp4(const uint8_t* q, const uint8_t* s, double ts, int R, int C, double* out) {
     if (C % 64) return -1;
-    Nvfp4View v{q, s, ts, R, C};
+    ExpertMatrix v{0, q, s, ts, R, C};
 #pragma omp parallel for schedule(static)
     for (int r = 0; r < R; ++r) nvfp4_row(v, r, out + (int64_t)r * C);
     return 0;
 }
 
-// Expert record -> gate [F][L], up [F][L], down [L][F].
+// Q3_K (kind 1) or IQ4_NL (kind 2) matrix [R][C] -> out [R][C].
+int orc_decode_q3k_iq4nl(int kind, const uint8_t* blob, int R, int C, double* out) {
+    if ((kind == 1 && C % 256) || (kind == 2 && C % 32) || (kind != 1 && kind != 2)) return -1;
+    ExpertMatrix v{kind, blob, nullptr, 1.0, R, C};
+#pragma omp parallel for schedule(static)
+    for (int r = 0; r < R; ++r) nvfp4_row(v, r, out + (int64_t)r * C);
+    return 0;
+}
+
+// The 16 IQ4_NL levels as this oracle computes them from their definition.
+void orc_iq4nl_levels(double* out) {
+    for (int i = 0; i < 16; ++i) out[i] = iq4nl_levels()[i];
+}
+
+int64_t orc_expert_record_bytes_fmt(int efmt, int L, int F) { return expert_record_bytes_fmt(efmt, L, F); }
+
+// Expert record (efmt 0 NVFP4, 1 Q3_K build) -> gate [F][L], up [F][L], down [L][F].
+void orc_decode_expert_fmt(int efmt, const uint8_t* rec, int L, int F, double* wg, double* wu, double* wd) {
+    double* outs[3] = {wg, wu, wd};
+    for (int m = 0; m < 3; ++m) {
+        const ExpertMatrix v = expert_matrix(rec, L, F, m, efmt);
+#pragma omp parallel for schedule(static)
+        for (int r = 0; r < v.R; ++r) nvfp4_row(v, r, outs[m] + (int64_t)r * v.C);
+    }
+}
+
+// NVFP4 expert record -> gate [F][L], up [F][L], down [L][F].
 void orc_decode_expert(const uint8_t* rec, int L, int F, double* wg, double* wu, double* wd) {
     double* outs[3] = {wg, wu, wd};
     for (int m = 0; m < 3; ++m) {
-        const Nvfp4View v = expert_matrix(rec, L, F, m);
+        const ExpertMatrix v = expert_matrix(rec, L, F, m);
 #pragma omp parallel for schedule(static)
         for (int r = 0; r < v.R; ++r) nvfp4_row(v, r, outs[m] + (int64_t)r * v.C);
     }
@@ -316,8 +430,9 @@ void orc_shared_expert(const orc_shape* s, const orc_layer* ly, const double* x,
 }
 
 // One expert on n latent vectors h [n][L] (step 4): o [n][L].
-void orc_expert_apply(const uint8_t* rec, int L, int F, const double* h, int n, double* o) {
-    const Nvfp4View vg = expert_matrix(rec, L, F, 0), vu = expert_matrix(rec, L, F, 1), vd = expert_matrix(rec, L, F, 2);
+void orc_expert_apply_fmt(int efmt, const uint8_t* rec, int L, int F, const double* h, int n, double* o) {
+    const ExpertMatrix vg = expert_matrix(rec, L, F, 0, efmt), vu = expert_matrix(rec, L, F, 1, efmt),
+                       vd = expert_matrix(rec, L, F, 2, efmt);
     std::vector<double> rg(L), ru(L), rd(F), z((size_t)n * F);
     for (int f = 0; f < F; ++f) {
         nvfp4_row(vg, f, rg.data());
@@ -331,6 +446,10 @@ void orc_expert_apply(const uint8_t* rec, int L, int F, const double* h, int n, 
         nvfp4_row(vd, r, rd.data());
         for (int i = 0; i < n; ++i) o[(int64_t)i * L + r] = dot(rd.data(), z.data() + (size_t)i * F, F);
     }
+}
+
+void orc_expert_apply(const uint8_t* rec, int L, int F, const double* h, int n, double* o) {
+    orc_expert_apply_fmt(0, rec, L, F, h, n, o);
 }
 
 // y [n][R] = M x for the stored Q8_0 / Q4_0 matrix M [R][C] and n vectors x [n][C].
@@ -401,7 +520,7 @@ int orc_forward(const orc_shape* s, const orc_layer* ly, const double* x, const 
     for (int e = 0; e < E; ++e)
         if (!pairs[e].empty()) used.push_back(e);
     std::vector<double> o((size_t)T * K * L);
-    const int64_t rec_b = expert_record_bytes(L, F);
+    const int64_t rec_b = expert_record_bytes_fmt(s->expert_fmt, L, F);
 #pragma omp parallel for schedule(dynamic, 1)
     for (int u = 0; u < (int)used.size(); ++u) {
         const int e = used[u];
@@ -410,7 +529,7 @@ int orc_forward(const orc_shape* s, const orc_layer* ly, const double* x, const 
         std::vector<double> hin(pe.size() * (size_t)L), out(pe.size() * (size_t)L);
         for (size_t i = 0; i < pe.size(); ++i)
             std::memcpy(&hin[i * L], &h[((size_t)(pe[i] / K) * G + g) * L], sizeof(double) * L);
-        orc_expert_apply(ly->experts + e * rec_b, L, F, hin.data(), (int)pe.size(), out.data());
+        orc_expert_apply_fmt(s->expert_fmt, ly->experts + e * rec_b, L, F, hin.data(), (int)pe.size(), out.data());
         for (size_t i = 0; i < pe.size(); ++i) std::memcpy(&o[(size_t)pe[i] * L], &out[i * L], sizeof(double) * L);
     }
     // step 7 first (the output starts as the shared expert), then steps 5, 6
@@ -439,6 +558,76 @@ int orc_forward(const orc_shape* s, const orc_layer* ly, const double* x, const 
     if (residual)
         for (int64_t i = 0; i < (int64_t)T * H; ++i) y[i] += bf16_value(residual[i]);
     return 0;
+}
+
+// ---- ablation: D over all groups with Q8_1 activations -------------------------------
+//
+// The teardown article's reference kernel (section "A latent in front of the
+// experts", its code excerpt) quantises each token row to Q8_1 and runs D over
+// all 8 groups with integer dot products.  Q8_1 as read here, per block of 32
+// consecutive elements of a row (the pages do not print it; every rounding
+// is an fp32 operation, so the GPU takes the same integer decisions):
+//   d = fp16(amax / 127)              amax = max |x_j| of the block (fp32)
+//   q_j = clamp(rint(x_j / float(d)), -127, 127)     (all zero when d == 0)
+// and the sum s = sum_j q_j (an integer; the fp16 d*s of the stored format
+// only matters for Q4_0 weights, whose -8 offset it cancels exactly here).
+// orc_quantize_q8_1: x [T][H] fp32 -> q int8 [T][H], d fp16 bits [T][H/32].
+void orc_quantize_q8_1(const float* x, int T, int H, int8_t* q, uint16_t* d_bits) {
+    for (int t = 0; t < T; ++t) {
+        for (int b = 0; b < H / 32; ++b) {
+            const float* xb = x + (int64_t)t * H + b * 32;
+            float amax = 0.f;
+            for (int j = 0; j < 32; ++j) amax = std::max(amax, std::fabs(xb[j]));
+            const float d32 = amax / 127.0f;
+            // fp32 -> fp16, round to nearest even (_Float16 conversion)
+            const _Float16 d16 = (_Float16)d32;
+            uint16_t bits;
+            std::memcpy(&bits, &d16, 2);
+            d_bits[(int64_t)t * (H / 32) + b] = bits;
+            const float dv = (float)d16;
+            for (int j = 0; j < 32; ++j) {
+                float v = dv > 0.f ? std::rint(xb[j] / dv) : 0.f;
+                v = std::min(127.f, std::max(-127.f, v));
+                q[(int64_t)t * H + b * 32 + j] = (int8_t)v;
+            }
+        }
+    }
+}
+
+// h [T][G][L] = D_g xq for every group g, where xq is the Q8_1 reading of the
+// fp32 rows x [T][H]: per block, d_w * d_x * sum_j w_j q_j (integer sum, exact).
+void orc_dproj_q8_1(int fmt, const uint8_t* D, int G, int L, int H, const float* x, int T, double* h) {
+    std::vector<int8_t> q((size_t)T * H);
+    std::vector<uint16_t> dx((size_t)T * (H / 32));
+    orc_quantize_q8_1(x, T, H, q.data(), dx.data());
+    const int64_t mb = du_matrix_bytes(fmt, L, H);
+    for (int g = 0; g < G; ++g) {
+        const uint8_t* m = D + g * mb;
+#pragma omp parallel for schedule(static)
+        for (int r = 0; r < L; ++r) {
+            for (int t = 0; t < T; ++t) {
+                double acc = 0.0;
+                for (int b = 0; b < H / 32; ++b) {
+                    const int64_t blk = (int64_t)b * L + r;
+                    int64_t isum = 0;
+                    double dw;
+                    for (int j = 0; j < 32; ++j) {
+                        int wq;
+                        if (fmt == kQ8_0) {
+                            wq = (int8_t)m[blk * 32 + j];
+                        } else {
+                            const uint8_t byte = m[blk * 16 + (j % 16)];
+                            wq = (j < 16 ? (byte & 0xF) : (byte >> 4)) - 8;
+                        }
+                        isum += (int64_t)wq * q[(size_t)t * H + b * 32 + j];
+                    }
+                    dw = fp16_value(load_u16(m + (int64_t)L * H / 32 * (fmt == kQ8_0 ? 32 : 16) + 2 * blk));
+                    acc += dw * fp16_value(dx[(size_t)t * (H / 32) + b]) * (double)isum;
+                }
+                h[((int64_t)t * G + g) * L + r] = acc;
+            }
+        }
+    }
 }
 
 // RMSNorm per row: out = gamma * v / sqrt(mean(v^2) + eps).

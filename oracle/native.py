@@ -79,6 +79,8 @@ def lib():
         L.orc_forward.restype = i32
         L.orc_forward.argtypes = [ctypes.POINTER(_Shape), ctypes.POINTER(_Layer), vp, vp, vp, vp, i32, vp, vp, vp, vp]
         L.orc_rmsnorm.argtypes = [vp, vp, dbl, i32, i32, vp]
+        L.orc_quantize_q8_1.argtypes = [vp, i32, i32, vp, vp]
+        L.orc_dproj_q8_1.argtypes = [i32, vp, i32, i32, i32, vp, i32, vp]
         L.orc_stack_layer.restype = i32
         L.orc_stack_layer.argtypes = [ctypes.POINTER(_Shape), ctypes.POINTER(_Layer), vp, vp, dbl, vp, vp, i32, vp,
                                       vp, vp, vp]
@@ -346,3 +348,27 @@ class Weights:
             s = self.s
             self._E[e] = decode_expert(expert_slice(self.layer["experts"], e, s.latent, s.ffn), s.latent, s.ffn)
         return self._E[e]
+
+
+# ----------------------------------------------------------------------------
+# ablation: D over all groups with Q8_1 activations
+# ----------------------------------------------------------------------------
+
+def quantize_q8_1(x):
+    """fp32 rows [T, H] -> (q int8 [T, H], d fp16 bits [T, H/32]), Q8_1 as read
+    in lmoe_oracle.cpp (every rounding an fp32 operation)."""
+    x = np.ascontiguousarray(x, np.float32)
+    T, H = x.shape
+    q = np.empty((T, H), np.int8)
+    d = np.empty((T, H // 32), np.uint16)
+    lib().orc_quantize_q8_1(_ptr(x), T, H, _ptr(q), _ptr(d))
+    return q, d
+
+
+def dproj_q8_1(fmt: int, D, G: int, L: int, H: int, x) -> np.ndarray:
+    """h [T, G, L] = D_g applied to the Q8_1 reading of x [T, H] (fp32), every group."""
+    Db, pD = _c(D, np.uint8)
+    x = np.ascontiguousarray(x, np.float32)
+    h = np.empty((x.shape[0], G, L))
+    lib().orc_dproj_q8_1(fmt, pD, G, L, H, _ptr(x), x.shape[0], _ptr(h))
+    return h

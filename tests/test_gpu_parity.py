@@ -407,3 +407,46 @@ def test_input_beyond_fp16_range_is_reported(T):
     # the same call on an in-range input is clean again
     dev.forward(to_device(synth.make_x(wl), "cuda"), ws)
     assert B.lmoe_last_device_status(ws) == B.LMOE_OK
+
+
+# ----------------------------------------------------------------------------
+# the reference-kernel ablation of D_g
+# ----------------------------------------------------------------------------
+
+def _d_only(name):
+    wl = synth.WORKLOADS[name]
+    s = wl.shape
+    D = np.concatenate([synth.qmatrix(s.du_fmt, synth.key(wl.seed, 0, "D", g), wl.weight_sigma, s.latent, s.hidden)
+                        for g in range(s.n_groups)])
+    return wl, s, D
+
+
+@pytest.mark.parametrize("name", ["edge0_145b_decode", "edge0_120b_decode"])
+@pytest.mark.parametrize("T", [1, 4, 11])
+def test_dproj_ablation_matches_oracle(name, T):
+    """Q8_1 activations over every group against the oracle's Q8_1 reading
+    (integer products exact on both sides, fp32 sums on the GPU), and fp16
+    activations over a subset of groups against D_g x (other groups left
+    untouched)."""
+    wl, s, D = _d_only(name)
+    xb = synth.make_x(wl, T=T, draw=3)
+    x32 = orc.bf16_to_f64(xb).astype(np.float32)
+    cfg = B.make_cfg(s)
+    ws = torch.zeros(B.lmoe_workspace_bytes(cfg, T), dtype=torch.uint8, device="cuda")
+    Dd, xd = to_device(D, "cuda"), to_device(xb, "cuda")
+    G, L, H = s.n_groups, s.latent, s.hidden
+    h = torch.full((T, G, L), float("nan"), dtype=torch.float32, device="cuda")
+    B.lmoe_dproj_ablation(cfg, xd, Dd, 1, (1 << G) - 1, h, T, ws)
+    ref = orc.dproj_q8_1(s.du_fmt, D, G, L, H, x32)
+    got = h.cpu().numpy().astype(np.float64)
+    assert orc.rel_l2(got, ref) < 1e-5 and orc.max_abs_over_rms(got, ref) < 1e-4
+    mask = 0b10110101 & ((1 << G) - 1)
+    h.fill_(float("nan"))
+    B.lmoe_dproj_ablation(cfg, xd, Dd, 0, mask, h, T, ws)
+    got = h.cpu().numpy().astype(np.float64)
+    for g in range(G):
+        if mask >> g & 1:
+            ref_g = orc.du_apply(s.du_fmt, orc.du_slice(D, s.du_fmt, g, L, H), L, H, x32)
+            assert orc.rel_l2(got[:, g], ref_g) < 1e-4, g
+        else:
+            assert np.all(np.isnan(got[:, g])), g

@@ -561,3 +561,60 @@ def test_cpp_and_numpy_oracles_agree(fmt):
     c = cpp_oracle.stack_layer_forward(s, layer, xb, gamma, 1e-6)
     d = np_oracle.stack_layer_forward(s, layer, xb, gamma, 1e-6)
     np.testing.assert_allclose(c[0], d[0], rtol=1e-11, atol=1e-13)
+
+
+# ----------------------------------------------------------------------------
+# the reference-kernel ablation: Q8_1 activations, D over every group
+# ----------------------------------------------------------------------------
+
+def test_q8_1_quantisation_rule():
+    """d = fp16(amax / 127), q = rint(x / d) (fp32): a hand case, a zero
+    block, and the rounding bound |x - d q| <= d / 2 on random rows."""
+    x = np.zeros((1, 64), np.float32)
+    x[0, :4] = [1.0, -0.5, 0.25, 127.0 / 128.0]          # amax 1: d = fp16(1/127)
+    q, d = cpp_oracle.quantize_q8_1(x)
+    dv = float(np.array([d[0, 0]], np.uint16).view(np.float16)[0])
+    assert dv == float(np.float16(np.float32(1.0) / np.float32(127.0)))
+    want = [int(np.rint(np.float32(v) / np.float32(dv))) for v in x[0, :4]]
+    assert q[0, :4].tolist() == want and want[0] == 127
+    assert np.all(q[0, 32:] == 0) and d[0, 1] == 0       # an all-zero block
+    rng = np.random.default_rng(41)
+    x = rng.normal(size=(5, 256)).astype(np.float32)
+    q, d = cpp_oracle.quantize_q8_1(x)
+    dv = d.view(np.float16).astype(np.float64).repeat(32, axis=1)
+    assert np.all(np.abs(q) <= 127)
+    assert np.all(np.abs(x - dv * q) <= dv * 0.5 * (1 + 1e-6) + 1e-12)
+
+
+@pytest.mark.parametrize("fmt", [synth.Q8_0, synth.Q4_0])
+def test_dproj_q8_1_exact_inputs_equal_plain_projection(fmt):
+    """Rows that Q8_1 represents exactly (d = 2^-6 and integer multiples,
+    +-127 d in every block) give exactly D_g x, with D decoded by the pinned
+    decoder and multiplied in torch."""
+    G, L, H = 3, 64, 128
+    wl = synth.Workload("abl", synth.LayerShape(hidden=H, latent=L, n_experts=4, top_k=2, n_groups=G, ffn=64,
+                                                 shared_ffn=64, du_fmt=fmt), T=3, seed=7, weight_sigma=0.05)
+    layer = synth.make_layer(wl)
+    rng = np.random.default_rng(43)
+    k = rng.integers(-127, 128, size=(3, H))
+    k[:, ::32] = 127 * np.where(rng.random((3, H // 32)) < 0.5, -1, 1)
+    x = (k * 2.0 ** -6).astype(np.float32)
+    h = cpp_oracle.dproj_q8_1(fmt, layer["D"], G, L, H, x)
+    for g in range(G):
+        Dg = torch.from_numpy(np_oracle.decode_du(fmt, np_oracle.du_slice(layer["D"], fmt, g, L, H), L, H))
+        want = torch.from_numpy(x.astype(np.float64)) @ Dg.T
+        np.testing.assert_allclose(h[:, g], want.numpy(), rtol=1e-12, atol=1e-12)
+
+
+def test_dproj_q8_1_equals_projection_of_the_dequantised_rows():
+    G, L, H = 2, 64, 256
+    wl = synth.Workload("abl", synth.LayerShape(hidden=H, latent=L, n_experts=4, top_k=2, n_groups=G, ffn=64,
+                                                 shared_ffn=64, du_fmt=synth.Q4_0), T=4, seed=8, weight_sigma=0.05)
+    layer = synth.make_layer(wl)
+    x = np.random.default_rng(44).normal(size=(4, H)).astype(np.float32)
+    q, d = cpp_oracle.quantize_q8_1(x)
+    xq = torch.from_numpy(q.astype(np.float64) * d.view(np.float16).astype(np.float64).repeat(32, axis=1))
+    h = cpp_oracle.dproj_q8_1(synth.Q4_0, layer["D"], G, L, H, x)
+    for g in range(G):
+        Dg = torch.from_numpy(np_oracle.decode_du(synth.Q4_0, np_oracle.du_slice(layer["D"], synth.Q4_0, g, L, H), L, H))
+        np.testing.assert_allclose(h[:, g], (xq @ Dg.T).numpy(), rtol=1e-12, atol=1e-13)
