@@ -54,10 +54,26 @@
  *     of its 64-wide column group; weight = e2m1 * e4m3 * ts.
  *     (1,935,376 bytes at latent 1792, ffn 640: the record size printed in
  *     the teardown article, section "What is 4-bit".)
+ *   experts, cfg.expert_fmt == LMOE_EXPERTS_Q3K: records of
+ *     gate (Q3_K [ffn][latent]) | up (Q3_K [ffn][latent]) | down (IQ4_NL
+ *     [latent][ffn]), no tail (1,630,720 bytes at latent 1792, 1,164,800 at
+ *     1280: the Q3_K record sizes the pages print; they give the type names
+ *     and byte counts only, the arrangement is this library's):
+ *     Q3_K [R][C], 110 bytes per 256 weights of a row, planes over 128-column
+ *       halves h:  lo [C/128][R][32] (element 16w + 4i + b of the half in
+ *       byte 4w + b, bits 2i..2i+1) | hi [C/128][R][16] (element 32v + 4i + b
+ *       in byte 4v + b, bit i) | sc [C/128][R][6] (sub-block j = elements
+ *       16j..16j+15 at bits 6j..6j+5, little-endian) | d fp16 [C/256][R];
+ *       weight = d * (sc_j - 32) * (q - 4), q = lo | hi << 2
+ *     IQ4_NL [R][C], 18 bytes per 32: codes [C/32][R][16] (byte j: element j
+ *       low nibble, element j+16 high) | d fp16 [C/32][R];
+ *       weight = d * level[code], the 16 levels being the standard normal
+ *       quantiles at (i + 1/2) / 16 scaled to an outermost 127 and rounded:
+ *       -127 -90 -69 -53 -39 -27 -16 -5 5 16 27 39 53 69 90 127
  *
  * Shape limits (lmoe_cfg_check): hidden, latent multiples of 128; ffn,
  * shared_ffn multiples of 64; 1 <= top_k <= 16 and top_k <= n_experts <=
- * 4096; 1 <= n_groups <= 64.
+ * 1024; 1 <= n_groups <= 64; with Q3_K experts latent a multiple of 256.
  */
 #ifndef LMOE_H
 #define LMOE_H
@@ -87,6 +103,7 @@ typedef enum {
 
 typedef enum { LMOE_Q8_0 = 8, LMOE_Q4_0 = 4 } lmoe_du_fmt;   /* D/U block formats */
 typedef enum { LMOE_F32 = 0, LMOE_BF16 = 1 } lmoe_dtype;     /* router weight type */
+typedef enum { LMOE_EXPERTS_NVFP4 = 0, LMOE_EXPERTS_Q3K = 1 } lmoe_expert_fmt;   /* expert records */
 
 typedef struct {
     int hidden;        /* model width (2560 for Edge0 145B / 120B) */
@@ -98,6 +115,7 @@ typedef struct {
     int shared_ffn;    /* shared expert SwiGLU width (640) */
     int du_fmt;        /* lmoe_du_fmt */
     int router_dtype;  /* lmoe_dtype */
+    int expert_fmt;    /* lmoe_expert_fmt (0: NVFP4 records) */
 } lmoe_cfg;
 
 typedef struct {
@@ -205,8 +223,9 @@ LMOE_API int lmoe_last_device_status(void* ws, size_t ws_bytes, void* stream);
 LMOE_API const char* lmoe_status_str(int status);
 
 /* Diagnostics: decode one stored matrix to fp32 [rows][cols] on the device
- * with the same decoders the kernels use.  fmt: LMOE_Q8_0, LMOE_Q4_0, or 1
- * for an NVFP4 matrix (q then s as in an expert record, scaled by ts). */
+ * with the same decoders the kernels use.  fmt: LMOE_Q8_0, LMOE_Q4_0, 1 for
+ * an NVFP4 matrix (q then s as in an expert record, scaled by ts), 2 for a
+ * Q3_K matrix, 3 for an IQ4_NL matrix (layouts above; ts unused). */
 LMOE_API int lmoe_debug_decode(int fmt, const void* blob, int rows, int cols, float ts, float* out, void* stream);
 
 /* Profiling: while n > 0, every later forward call records events[0] before

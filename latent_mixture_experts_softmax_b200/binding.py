@@ -23,6 +23,10 @@ LMOE_Q4_0 = 4
 LMOE_F32 = 0
 LMOE_BF16 = 1
 LMOE_NVFP4_DEBUG = 1
+LMOE_Q3K_DEBUG = 2
+LMOE_IQ4NL_DEBUG = 3
+LMOE_EXPERTS_NVFP4 = 0
+LMOE_EXPERTS_Q3K = 1
 
 # every symbol include/lmoe.h declares
 EXPORTS = ("lmoe_cfg_check", "lmoe_expert_record_bytes", "lmoe_du_bytes", "lmoe_workspace_bytes", "lmoe_route",
@@ -39,7 +43,7 @@ class LmoeError(RuntimeError):
 
 class lmoe_cfg(ctypes.Structure):
     _fields_ = [(n, ctypes.c_int) for n in ("hidden", "latent", "n_experts", "top_k", "n_groups", "ffn",
-                                            "shared_ffn", "du_fmt", "router_dtype")]
+                                            "shared_ffn", "du_fmt", "router_dtype", "expert_fmt")]
 
 
 class lmoe_shared(ctypes.Structure):
@@ -135,8 +139,11 @@ def make_cfg(shape) -> lmoe_cfg:
     rd = shape.router_dtype
     if isinstance(rd, str):
         rd = LMOE_BF16 if rd == "bf16" else LMOE_F32
+    ef = getattr(shape, "expert_fmt", "nvfp4")
+    if isinstance(ef, str):
+        ef = LMOE_EXPERTS_Q3K if ef == "q3k" else LMOE_EXPERTS_NVFP4
     return lmoe_cfg(shape.hidden, shape.latent, shape.n_experts, shape.top_k, shape.n_groups, shape.ffn,
-                    shape.shared_ffn, shape.du_fmt, rd)
+                    shape.shared_ffn, shape.du_fmt, rd, ef)
 
 
 def make_shared(gate, up, down) -> lmoe_shared:

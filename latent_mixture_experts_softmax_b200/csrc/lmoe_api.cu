@@ -23,6 +23,8 @@ int check_cfg(const lmoe_cfg* c) {
     if (c->n_groups > kMaxGroups || c->n_groups > 255) return LMOE_ERR_UNSUPPORTED;
     if (c->du_fmt != LMOE_Q8_0 && c->du_fmt != LMOE_Q4_0) return LMOE_ERR_UNSUPPORTED;
     if (c->router_dtype != LMOE_F32 && c->router_dtype != LMOE_BF16) return LMOE_ERR_UNSUPPORTED;
+    if (c->expert_fmt != LMOE_EXPERTS_NVFP4 && c->expert_fmt != LMOE_EXPERTS_Q3K) return LMOE_ERR_UNSUPPORTED;
+    if (c->expert_fmt == LMOE_EXPERTS_Q3K && c->latent % 256) return LMOE_ERR_UNSUPPORTED;
     return LMOE_OK;
 }
 
@@ -32,6 +34,7 @@ size_t du_matrix_bytes(const lmoe_cfg& c) {
 
 size_t record_bytes(const lmoe_cfg& c) {
     const size_t lf = (size_t)c.latent * c.ffn;
+    if (c.expert_fmt == LMOE_EXPERTS_Q3K) return 2 * (lf / 256 * 110) + lf / 32 * 18;
     return 3 * lf / 2 + 3 * lf / 16 + 16;
 }
 
@@ -147,6 +150,7 @@ FwdParams base_params(const lmoe_cfg& c, int T, void* ws, const WsLayout& L) {
     std::memset(&p, 0, sizeof(p));
     p.H = c.hidden; p.L = c.latent; p.E = c.n_experts; p.K = c.top_k; p.G = c.n_groups;
     p.F = c.ffn; p.Fs = c.shared_ffn; p.du_fmt = c.du_fmt; p.router_bf16 = c.router_dtype == LMOE_BF16;
+    p.efmt = c.expert_fmt;
     p.T = T;
     char* b = static_cast<char*>(ws);
     p.ctrl = reinterpret_cast<Ctrl*>(b + L.ctrl);
@@ -207,6 +211,7 @@ int run_prefill(const lmoe_cfg& c, const FwdParams& f, const WsLayout& L, void* 
     std::memset(&p, 0, sizeof(p));
     char* b = static_cast<char*>(ws);
     p.H = f.H; p.L = f.L; p.E = f.E; p.K = f.K; p.G = f.G; p.F = f.F; p.Fs = f.Fs; p.du_fmt = f.du_fmt; p.T = f.T;
+    p.efmt = f.efmt;
     p.x = f.x;
     p.router_w_bf16 = static_cast<const uint16_t*>(f.router_w);
     p.router_b = f.router_b;
@@ -298,6 +303,28 @@ int forward_impl(const lmoe_cfg* cfg, const void* x, const void* router_w, const
         // one kernel; it clears its own counters, so no per-call reset
         stage_reset();
         return cuda_status(run_decode_step(p, st));
+    }
+    if (cfg->expert_fmt == LMOE_EXPERTS_Q3K) {
+        // the Q3_K build between 9 and 63 tokens: the one-kernel step on
+        // passes of at most 8 tokens (the five-kernel path of that range
+        // reads NVFP4 records only)
+        FwdParams q = p;
+        q.T = std::min(T, 8);
+        if (!decode_step_fits(q)) return LMOE_ERR_UNSUPPORTED;
+        stage_reset();
+        for (int t0 = 0; t0 < T; t0 += 8) {
+            q = p;
+            q.T = std::min(8, T - t0);
+            q.x = p.x + (size_t)t0 * p.H;
+            q.y = p.y + (size_t)t0 * p.H;
+            if (p.residual) q.residual = p.residual + (size_t)t0 * p.H;
+            if (p.inject_idx) { q.inject_idx = p.inject_idx + (size_t)t0 * p.K; q.inject_w = p.inject_w + (size_t)t0 * p.K; }
+            if (p.out_idx) q.out_idx = p.out_idx + (size_t)t0 * p.K;
+            if (p.out_w) q.out_w = p.out_w + (size_t)t0 * p.K;
+            const cudaError_t e = run_decode_step(q, st);
+            if (e != cudaSuccess) return LMOE_ERR_CUDA;
+        }
+        return LMOE_OK;
     }
     cudaError_t e = reset_tickets(ws, st);
     if (e != cudaSuccess) return LMOE_ERR_CUDA;
@@ -473,7 +500,8 @@ int lmoe_dproj_ablation(const lmoe_cfg* cfg, const void* x, const void* D, int a
 
 int lmoe_debug_decode(int fmt, const void* blob, int rows, int cols, float ts, float* out, void* stream) {
     if (!blob || !out || rows <= 0 || cols <= 0 || cols % 64 || !aligned(blob, 16)) return LMOE_ERR_ARG;
-    if (fmt != LMOE_Q8_0 && fmt != LMOE_Q4_0 && fmt != 1) return LMOE_ERR_UNSUPPORTED;
+    if (fmt != LMOE_Q8_0 && fmt != LMOE_Q4_0 && fmt != 1 && fmt != 2 && fmt != 3) return LMOE_ERR_UNSUPPORTED;
+    if (fmt == 2 && cols % 256) return LMOE_ERR_ARG;
     return cuda_status(run_debug_decode(fmt, blob, rows, cols, ts, out, static_cast<cudaStream_t>(stream)));
 }
 

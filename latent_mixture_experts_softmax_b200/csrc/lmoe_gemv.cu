@@ -22,6 +22,7 @@
 #include <algorithm>
 
 #include "lmoe_internal.cuh"
+#include "lmoe_q3k.cuh"
 #include "lmoe_route.cuh"
 #include "lmoe_rowdot.cuh"
 
@@ -941,7 +942,11 @@ __global__ void k_debug_decode(int fmt, const uint8_t* blob, int R, int C, float
     const int r = blockIdx.x;
     for (int c = threadIdx.x; c < C; c += blockDim.x) {
         float v;
-        if (fmt == LMOE_Q8_0 || fmt == LMOE_Q4_0) {
+        if (fmt == 2) {
+            v = q3k_element(blob, R, C, r, c);
+        } else if (fmt == 3) {
+            v = iq4nl_element(blob, R, C, r, c);
+        } else if (fmt == LMOE_Q8_0 || fmt == LMOE_Q4_0) {
             const int b = c / 32, j = c % 32;
             const size_t qrow = fmt == LMOE_Q8_0 ? 32 : 16;
             const uint16_t d = reinterpret_cast<const uint16_t*>(blob + (size_t)R * (C / 32) * qrow)[(size_t)b * R + r];

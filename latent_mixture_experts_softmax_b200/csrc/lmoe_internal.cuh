@@ -43,6 +43,7 @@ __device__ __forceinline__ uint16_t f32_to_bf16_bits(float v) {
 struct FwdParams {
     // shape
     int H, L, E, K, G, F, Fs, du_fmt, router_bf16;
+    int efmt;   // expert records: LMOE_EXPERTS_NVFP4 or LMOE_EXPERTS_Q3K
     int T;
     // inputs
     const uint16_t* x;

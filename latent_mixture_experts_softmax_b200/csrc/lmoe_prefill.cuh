@@ -22,6 +22,7 @@ struct __align__(64) TmaMaps {
 
 struct PrefillParams {
     int H, L, E, K, G, F, Fs, du_fmt, T;
+    int efmt;            // expert records: LMOE_EXPERTS_NVFP4 or LMOE_EXPERTS_Q3K
     // inputs
     const uint16_t* x;
     const uint16_t* router_w_bf16;

@@ -29,6 +29,7 @@
 #include <cstring>
 
 #include "lmoe_internal.cuh"
+#include "lmoe_q3k.cuh"
 #include "lmoe_route.cuh"
 #include "lmoe_rowdot.cuh"
 #include "lmoe_sm100.cuh"
@@ -38,6 +39,11 @@ namespace lmoe {
 using namespace sm100;
 
 enum StreamPhase { SP_DPROJ = 0, SP_GATEUP = 1, SP_DOWN = 2, SP_UPROJ = 3 };
+
+// The format parameter of the phase templates: the D/U format (LMOE_Q8_0 /
+// LMOE_Q4_0) for D and U, the expert format for gate/up and down.
+constexpr int kEfNvfp4 = LMOE_EXPERTS_NVFP4;
+constexpr int kEfQ3k = LMOE_EXPERTS_Q3K;
 
 constexpr int kWW = 16;                     // warps per CTA
 constexpr int kWThreads = 32 * kWW;
@@ -206,6 +212,88 @@ __device__ __forceinline__ void tile_bf16(const uint16_t* w, int K, const __half
 }
 
 
+// The IQ4_NL byte -> (level of the low nibble, level of the high nibble)
+// table of the CTA (fp16 pairs), filled at kernel start.
+__device__ __forceinline__ uint32_t* iq4nl_lut() {
+    __shared__ uint32_t lut[256];
+    return lut;
+}
+
+// One 128-column half of a 16-row Q3_K tile in shared memory (planes lo
+// [16][32], hi [16][16], sc [16][6], d [16] fp16) times the activations at
+// columns [0, 128) of xs.  Sub-block j is one k16 MMA: lane t takes the
+// elements 16j + 4t .. 16j + 4t + 3 of rows g and g + 8, whose code bits sit
+// in bits 2t.. of lo word j and bits 4(j & 1) + t of hi word j / 2; the
+// operand is (q - 4) * (sc_j - 32), an integer of at most 128 (exact in
+// fp16); the super-block scale d multiplies the step's sum.
+__device__ __forceinline__ void tile_q3k_half(const uint8_t* m, const __half* xs, int ld, int nt, float (&acc)[4]) {
+    const int lane = threadIdx.x & 31, g = lane >> 2, t = lane & 3;
+    const uint8_t* lo = m;
+    const uint8_t* hi = m + 512;
+    const uint8_t* sc = m + 768;
+    const uint16_t* dd = reinterpret_cast<const uint16_t*>(m + 864);
+    auto sc48 = [&](int row) {
+        const uint16_t* p16 = reinterpret_cast<const uint16_t*>(sc + row * 6);
+        return (uint64_t)p16[0] | ((uint64_t)p16[1] << 16) | ((uint64_t)p16[2] << 32);
+    };
+    const uint64_t sg = sc48(g), sh = sc48(g + 8);
+    float c[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+        const uint32_t lg = *reinterpret_cast<const uint32_t*>(lo + g * 32 + 4 * j);
+        const uint32_t lh = *reinterpret_cast<const uint32_t*>(lo + (g + 8) * 32 + 4 * j);
+        const uint32_t hg = *reinterpret_cast<const uint32_t*>(hi + g * 16 + 4 * (j >> 1));
+        const uint32_t hh = *reinterpret_cast<const uint32_t*>(hi + (g + 8) * 16 + 4 * (j >> 1));
+        const int hs = 4 * (j & 1) + t;
+        const uint32_t qg = ((lg >> (2 * t)) & 0x03030303u) | (((hg >> hs) & 0x01010101u) << 2);
+        const uint32_t qh = ((lh >> (2 * t)) & 0x03030303u) | (((hh >> hs) & 0x01010101u) << 2);
+        const __half2 fg = __half2half2(__int2half_rn((int)((sg >> (6 * j)) & 63) - 32));
+        const __half2 fh = __half2half2(__int2half_rn((int)((sh >> (6 * j)) & 63) - 32));
+        auto op = [](uint32_t q, uint32_t sel, __half2 f) {
+            uint32_t v = hsub2u(__byte_perm(q, 0x64646464u, sel), 0x64046404u);     // (q - 4) pairs
+            return hmul2u(v, *reinterpret_cast<const uint32_t*>(&f));
+        };
+        const uint2 xv = g < nt ? *reinterpret_cast<const uint2*>(xs + (size_t)g * ld + 16 * j + 4 * t)
+                                : make_uint2(0, 0);
+        mma16816s(c, op(qg, 0x4140u, fg), op(qh, 0x4140u, fh), op(qg, 0x4342u, fg), op(qh, 0x4342u, fh), xv.x, xv.y);
+    }
+    const float dg = __half2float(__ushort_as_half(dd[g])), dh = __half2float(__ushort_as_half(dd[g + 8]));
+    acc[0] = fmaf(dg, c[0], acc[0]);
+    acc[1] = fmaf(dg, c[1], acc[1]);
+    acc[2] = fmaf(dh, c[2], acc[2]);
+    acc[3] = fmaf(dh, c[3], acc[3]);
+}
+
+// A 16-row IQ4_NL tile in shared memory (codes [block][16 rows][16 B], d
+// [block][16 rows] fp16), blocks [0, b1): as Q4_0 with the level table in
+// place of q - 8 (lane t: elements 4t..4t+3 from the low nibbles of its
+// 4 bytes, 16 + 4t.. from the high ones).
+__device__ __forceinline__ void tile_iq4nl(const uint8_t* q, const uint16_t* d, const __half* xs, int ld, int nt,
+                                           int b1, float (&acc)[4]) {
+    const int lane = threadIdx.x & 31, g = lane >> 2, t = lane & 3;
+    const uint32_t* lut = iq4nl_lut();
+#pragma unroll 2
+    for (int b = 0; b < b1; ++b) {
+        const uint32_t wg = *reinterpret_cast<const uint32_t*>(q + ((size_t)b * 16 + g) * 16 + 4 * t);
+        const uint32_t wh = *reinterpret_cast<const uint32_t*>(q + ((size_t)b * 16 + g + 8) * 16 + 4 * t);
+        const uint32_t g0 = lut[wg & 0xFF], g1 = lut[(wg >> 8) & 0xFF], g2 = lut[(wg >> 16) & 0xFF], g3 = lut[wg >> 24];
+        const uint32_t h0 = lut[wh & 0xFF], h1 = lut[(wh >> 8) & 0xFF], h2 = lut[(wh >> 16) & 0xFF], h3 = lut[wh >> 24];
+        const uint2 xl = act4(xs, ld, g, nt, 32 * b + 4 * t);
+        const uint2 xh = act4(xs, ld, g, nt, 32 * b + 16 + 4 * t);
+        float c[4] = {0.f, 0.f, 0.f, 0.f};
+        mma16816s(c, __byte_perm(g0, g1, 0x5410), __byte_perm(h0, h1, 0x5410), __byte_perm(g2, g3, 0x5410),
+                  __byte_perm(h2, h3, 0x5410), xl.x, xl.y);
+        mma16816s(c, __byte_perm(g0, g1, 0x7632), __byte_perm(h0, h1, 0x7632), __byte_perm(g2, g3, 0x7632),
+                  __byte_perm(h2, h3, 0x7632), xh.x, xh.y);
+        const float dg = __half2float(__ushort_as_half(d[b * 16 + g]));
+        const float dh = __half2float(__ushort_as_half(d[b * 16 + g + 8]));
+        acc[0] = fmaf(dg, c[0], acc[0]);
+        acc[1] = fmaf(dg, c[1], acc[1]);
+        acc[2] = fmaf(dh, c[2], acc[2]);
+        acc[3] = fmaf(dh, c[3], acc[3]);
+    }
+}
+
 // ---------------------------------------------------------------------------
 // items, steps and parts
 // ---------------------------------------------------------------------------
@@ -319,6 +407,50 @@ __device__ __forceinline__ void issue_step(const FwdParams& p, const WItem& it, 
             const int row = c / (nblk * 4), o = (c - row * nblk * 4) * 16;
             cp_async16(buf + (size_t)row * 128 + o, reinterpret_cast<const uint8_t*>(p.sd + (size_t)(it.r0 + row) * Fs) + (size_t)kb * 64 + o);
         }
+    } else if (FMT == kEfQ3k) {
+        const uint8_t* rec = p.experts + (size_t)it.mat * p.rec_bytes;
+        const size_t gb = q3k_matrix_bytes(F, L);
+        if (PHASE == SP_GATEUP) {
+            // one 128-column half h for gate and up: planes lo 512 | hi 256 | sc 96 | d 32 bytes each
+            const int h = kb / 4;
+            const size_t nh = (size_t)L / 128;
+            for (int mm = 0; mm < 2; ++mm) {
+                const uint8_t* m = rec + mm * gb;
+                uint8_t* bm = buf + mm * 896;
+                for (int c = lane; c < 56; c += 32) {
+                    const uint8_t* src;
+                    uint8_t* dst;
+                    if (c < 32) {
+                        src = m + ((size_t)h * F + it.r0) * 32 + c * 16;
+                        dst = bm + c * 16;
+                    } else if (c < 48) {
+                        src = m + nh * F * 32 + ((size_t)h * F + it.r0) * 16 + (c - 32) * 16;
+                        dst = bm + 512 + (c - 32) * 16;
+                    } else if (c < 54) {
+                        src = m + nh * F * 48 + ((size_t)h * F + it.r0) * 6 + (c - 48) * 16;
+                        dst = bm + 768 + (c - 48) * 16;
+                    } else {
+                        src = m + nh * F * 54 + ((size_t)(h / 2) * F + it.r0) * 2 + (c - 54) * 16;
+                        dst = bm + 864 + (c - 54) * 16;
+                    }
+                    cp_async16(dst, src);
+                }
+            }
+        } else {
+            // IQ4_NL down [L][F]: as the Q4_0 steps (8 blocks of 16 rows x 16 B, then the fp16 d)
+            const uint8_t* mat = rec + 2 * gb;
+            const uint8_t* dsc = mat + (size_t)L * F / 2;
+            const int n_codes = nblk * 16, n_sc = nblk * 2;
+            for (int c = lane; c < n_codes + n_sc; c += 32) {
+                if (c < n_codes) {
+                    const int b = c / 16, o = (c - b * 16) * 16;
+                    cp_async16(buf + (size_t)c * 16, mat + ((size_t)(kb + b) * L + it.r0) * 16 + o);
+                } else {
+                    const int c2 = c - n_codes, b = c2 >> 1;
+                    cp_async16(buf + (size_t)sb * 256 + (size_t)c2 * 16, dsc + ((size_t)(kb + b) * L + it.r0) * 2 + (c2 & 1) * 16);
+                }
+            }
+        }
     } else {
         const size_t nq = (size_t)L * F / 2, ns = (size_t)L * F / 16;
         const uint8_t* rec = p.experts + (size_t)it.mat * p.rec_bytes;
@@ -362,9 +494,14 @@ __device__ __forceinline__ void compute_step(const FwdParams& p, const WItem& it
         bool bad = false;
         tile_bf16(reinterpret_cast<const uint16_t*>(buf), 64, x, ld, nt, 0, nblk, a, bad);
         report_range(p.ctrl, bad);
+    } else if (PHASE == SP_GATEUP && FMT == kEfQ3k) {
+        tile_q3k_half(buf, x, ld, nt, a);
+        tile_q3k_half(buf + 896, x, ld, nt, u);
     } else if (PHASE == SP_GATEUP) {
         tile_nvfp4(buf, buf + 2 * 1024, x, ld, nt, nblk, a);
         tile_nvfp4(buf + 1024, buf + 2 * 1024 + 128, x, ld, nt, nblk, u);
+    } else if (FMT == kEfQ3k) {
+        tile_iq4nl(buf, reinterpret_cast<const uint16_t*>(buf + sb * 256), x, ld, nt, nblk, a);
     } else {
         tile_nvfp4(buf, buf + 2048, x, ld, nt, nblk, a);
     }
@@ -465,10 +602,11 @@ __device__ void phase_setup(const FwdParams& p, const StreamShared& sh, const WP
     __syncthreads();
     if ((PHASE == SP_GATEUP || PHASE == SP_DOWN) && threadIdx.x < 4 * ci.nm) {
         // the experts' tensor scales (gate, up, down; plain loads, read only
-        // by the epilogues, after later barriers)
+        // by the epilogues, after later barriers); the Q3_K build has none
         const int jj = threadIdx.x >> 2, k = threadIdx.x & 3;
         const size_t nq = (size_t)p.L * p.F / 2, ns = (size_t)p.L * p.F / 16;
-        ci.tail[jj][k] = __ldg(reinterpret_cast<const float*>(p.experts + (size_t)sh.uexp[ci.m0 + jj] * p.rec_bytes +
+        ci.tail[jj][k] = FMT == kEfQ3k ? 1.f
+                       : __ldg(reinterpret_cast<const float*>(p.experts + (size_t)sh.uexp[ci.m0 + jj] * p.rec_bytes +
                                                               3 * nq + 3 * ns) + k);
     }
 }
@@ -828,6 +966,7 @@ __global__ void __launch_bounds__(kWThreads, 1) k_wstream(FwdParams p, WPlan pl,
     __half* cache = reinterpret_cast<__half*>(smem);
     uint8_t* ring = smem + cache_bytes + (size_t)warp * kPD * kStepBytes;
 
+    if (PHASE == SP_DOWN && FMT == kEfQ3k) iq4nl_fill_lut(iq4nl_lut());   // ordered by the barriers below
     // D needs nothing from the router kernel and starts while it runs; it
     // waits for it only at its end, so that D's completion implies the
     // router kernel's.  The later kernels read the routing before their own
@@ -1061,7 +1200,7 @@ __device__ __noinline__ bool decode_first(const FwdParams& p, const DecodeLayout
     return true;
 }
 
-template <int FMT>
+template <int FMT, int EF>
 __global__ void __launch_bounds__(kWThreads, 1)
     k_decode_step(const __grid_constant__ FwdParams p, const __grid_constant__ DecodeLayout dl) {
     extern __shared__ uint8_t smem_raw[];
@@ -1077,13 +1216,14 @@ __global__ void __launch_bounds__(kWThreads, 1)
     float* xs = reinterpret_cast<float*>(ring_base + (size_t)kWW * kPD * kStepBytes);
 
     for (int e = threadIdx.x; e < p.E; e += blockDim.x) sgrp[e] = p.group[e];
+    if (EF == kEfQ3k) iq4nl_fill_lut(iq4nl_lut());
     // U's output-tile tickets are first used after three grid barriers
     if (blockIdx.x == 0)
         for (size_t i = threadIdx.x; i < p.wtick_bytes / sizeof(int); i += blockDim.x) p.wtick[i] = 0;
     __syncthreads();
     const bool ok = decode_first<FMT>(p, dl, sh, ci, sgrp, ring_base, cache, xs, rs, &s_ok) &&
-                    decode_phase<SP_GATEUP, FMT>(p, sh, dl.gu, ci, dl.cache_bytes, ring_base, cache, &ctrl->dec_phase[0], &s_ok) &&
-                    decode_phase<SP_DOWN, FMT>(p, sh, dl.dn, ci, dl.cache_bytes, ring_base, cache, &ctrl->dec_phase[1], &s_ok) &&
+                    decode_phase<SP_GATEUP, EF>(p, sh, dl.gu, ci, dl.cache_bytes, ring_base, cache, &ctrl->dec_phase[0], &s_ok) &&
+                    decode_phase<SP_DOWN, EF>(p, sh, dl.dn, ci, dl.cache_bytes, ring_base, cache, &ctrl->dec_phase[1], &s_ok) &&
                     decode_phase<SP_UPROJ, FMT>(p, sh, dl.u, ci, dl.cache_bytes, ring_base, cache, &ctrl->dec_phase[2], &s_ok);
     (void)ok;
     // leave; the last CTA out clears the step's counters
@@ -1220,9 +1360,11 @@ cudaError_t run_stream_path(const FwdParams& p, cudaStream_t st) {
     cudaError_t e = p.du_fmt == LMOE_Q8_0 ? launch_wstream<SP_DPROJ, LMOE_Q8_0>(p, P.d, T, st)
                               : launch_wstream<SP_DPROJ, LMOE_Q4_0>(p, P.d, T, st);
     if (e != cudaSuccess) return e;
-    e = launch_wstream<SP_GATEUP, LMOE_Q8_0>(p, P.gu, chunk_rows(P.gu), st);
+    e = p.efmt == kEfQ3k ? launch_wstream<SP_GATEUP, kEfQ3k>(p, P.gu, chunk_rows(P.gu), st)
+                         : launch_wstream<SP_GATEUP, kEfNvfp4>(p, P.gu, chunk_rows(P.gu), st);
     if (e != cudaSuccess) return e;
-    e = launch_wstream<SP_DOWN, LMOE_Q8_0>(p, P.dn, chunk_rows(P.dn), st);
+    e = p.efmt == kEfQ3k ? launch_wstream<SP_DOWN, kEfQ3k>(p, P.dn, chunk_rows(P.dn), st)
+                         : launch_wstream<SP_DOWN, kEfNvfp4>(p, P.dn, chunk_rows(P.dn), st);
     if (e != cudaSuccess) return e;
     e = p.du_fmt == LMOE_Q8_0 ? launch_wstream<SP_UPROJ, LMOE_Q8_0>(p, P.u, chunk_rows(P.u), st)
                               : launch_wstream<SP_UPROJ, LMOE_Q4_0>(p, P.u, chunk_rows(P.u), st);
@@ -1255,6 +1397,14 @@ static int chunk_cache_rows(const WPlan& w, int T) {
     return std::min(mats, kMaxChunkParts) * T;
 }
 
+typedef void (*DecodeKernel)(FwdParams, DecodeLayout);
+
+// The instance of the one-kernel step for the D/U and expert formats.
+static DecodeKernel decode_kernel(const FwdParams& p) {
+    if (p.du_fmt == LMOE_Q8_0) return p.efmt == kEfQ3k ? k_decode_step<LMOE_Q8_0, kEfQ3k> : k_decode_step<LMOE_Q8_0, kEfNvfp4>;
+    return p.efmt == kEfQ3k ? k_decode_step<LMOE_Q4_0, kEfQ3k> : k_decode_step<LMOE_Q4_0, kEfNvfp4>;
+}
+
 static DecodeLayout decode_layout(const FwdParams& p) {
     const WPlans P = stream_plans(p.H, p.L, p.F, p.Fs, p.G, p.E, p.K, p.T, p.du_fmt);
     DecodeLayout dl;
@@ -1284,8 +1434,7 @@ bool decode_step_fits(const FwdParams& p) {
     int dev = 0, optin = 0;
     cudaGetDevice(&dev);
     cudaDeviceGetAttribute(&optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev);
-    const void* k = p.du_fmt == LMOE_Q8_0 ? reinterpret_cast<const void*>(k_decode_step<LMOE_Q8_0>)
-                                          : reinterpret_cast<const void*>(k_decode_step<LMOE_Q4_0>);
+    const void* k = reinterpret_cast<const void*>(decode_kernel(p));
     cudaFuncAttributes fa;
     if (cudaFuncGetAttributes(&fa, k) != cudaSuccess) return false;
     return fa.sharedSizeBytes + dyn <= (size_t)optin;
@@ -1296,7 +1445,7 @@ cudaError_t run_decode_step(FwdParams p, cudaStream_t st) {
     p.route_smem = true;
     const DecodeLayout dl = decode_layout(p);
     const size_t smem = decode_dyn_smem(p, dl);
-    auto kern = p.du_fmt == LMOE_Q8_0 ? k_decode_step<LMOE_Q8_0> : k_decode_step<LMOE_Q4_0>;
+    auto kern = decode_kernel(p);
     cudaError_t e = ensure_smem(reinterpret_cast<const void*>(kern), smem);
     if (e != cudaSuccess) return e;
     int per_sm = 0;

@@ -31,6 +31,7 @@
 // in this file.
 
 #include "lmoe_prefill.cuh"
+#include "lmoe_q3k.cuh"
 
 namespace lmoe {
 
@@ -242,6 +243,30 @@ __device__ __forceinline__ void fetch_raw(const PrefillParams& p, const Cursor<K
         o.a = __ldg(q);
         if (p.du_fmt == LMOE_Q8_0) o.b = __ldg(q + 1);
         o.s = __ldg(reinterpret_cast<const uint16_t*>(mat + (size_t)R * C / 32 * rowb) + e);
+    } else if ((KIND == G_GATEUP || KIND == G_DOWN) && p.efmt == LMOE_EXPERTS_Q3K) {
+        const uint8_t* rec = p.experts + (size_t)c.t.mat * p.rec_bytes;
+        const size_t gb = q3k_matrix_bytes(p.F, p.L);
+        if (KIND == G_GATEUP) {
+            // 32 columns e0 .. e0 + 31 of one 128-column half h of a Q3_K row:
+            // lo words e0/16, e0/16 + 1; hi word e0/32; the half's 6 scale
+            // bytes; the super-block d
+            const int row = c.t.m0 + (r & 63), R = p.F;
+            const uint8_t* m = rec + (r >> 6) * gb;
+            const int col = k0 + 32 * h, hf = col / 128, e0 = col % 128;
+            const size_t nh = (size_t)p.L / 128;
+            const uint2 lo = __ldg(reinterpret_cast<const uint2*>(m + ((size_t)hf * R + row) * 32 + 4 * (e0 / 16)));
+            const uint32_t hi = __ldg(reinterpret_cast<const uint32_t*>(m + nh * R * 32 + ((size_t)hf * R + row) * 16 + 4 * (e0 / 32)));
+            const uint16_t* scp = reinterpret_cast<const uint16_t*>(m + nh * R * 48 + ((size_t)hf * R + row) * 6);
+            const uint16_t d = __ldg(reinterpret_cast<const uint16_t*>(m + nh * R * 54) + (size_t)(col / 256) * R + row);
+            o.a = make_uint4(lo.x, lo.y, hi, d);
+            o.b = make_uint4(__ldg(scp), __ldg(scp + 1), __ldg(scp + 2), (uint32_t)(e0 / 16));
+        } else {
+            // IQ4_NL down [L][F]: 32-column block k0 / 32 + h of row m0 + r
+            const uint8_t* m = rec + 2 * gb;
+            const size_t e = (size_t)(k0 / 32 + h) * p.L + c.t.m0 + r;
+            o.a = __ldg(reinterpret_cast<const uint4*>(m + e * 16));
+            o.s = __ldg(reinterpret_cast<const uint16_t*>(m + (size_t)p.L * p.F / 2) + e);
+        }
     } else if (KIND == G_GATEUP || KIND == G_DOWN) {
         const size_t nq = (size_t)p.L * p.F / 2, ns = (size_t)p.L * p.F / 16;
         const uint8_t* rec = p.experts + (size_t)c.t.mat * p.rec_bytes;
@@ -284,6 +309,38 @@ __device__ __forceinline__ void dequant_half(const PrefillParams& p, const RawHa
                 o[8 + 2 * i] = h2_bits(__hmul2(__hsub2(bits_h2(lo), off), d));
                 o[8 + 2 * i + 1] = h2_bits(__hmul2(__hsub2(bits_h2(hi), off), d));
             }
+        }
+    } else if (p.efmt == LMOE_EXPERTS_Q3K && KIND == G_GATEUP) {
+        // w = d * (sc_j - 32) * (q - 4): exact in fp32, one rounding to fp16
+        const float d = __half2float(__ushort_as_half((uint16_t)raw.a.w));
+        const uint64_t sc = (uint64_t)raw.b.x | ((uint64_t)raw.b.y << 16) | ((uint64_t)raw.b.z << 32);
+        const int j0 = (int)raw.b.w;
+        const uint32_t lo2[2] = {raw.a.x, raw.a.y};
+#pragma unroll
+        for (int k = 0; k < 16; ++k) {
+            float v[2];
+#pragma unroll
+            for (int u = 0; u < 2; ++u) {
+                const int i = 2 * k + u, b = i % 4, ii = (i % 16) / 4;
+                const int q = ((lo2[i / 16] >> (8 * b + 2 * ii)) & 3) | (((raw.a.z >> (8 * b + i / 4)) & 1) << 2);
+                const int f = (int)((sc >> (6 * (j0 + i / 16))) & 63) - 32;
+                v[u] = d * (float)(f * (q - 4));
+            }
+            o[k] = h2_bits(__floats2half2_rn(v[0], v[1]));
+        }
+    } else if (p.efmt == LMOE_EXPERTS_Q3K) {
+        // IQ4_NL: w = d * level[q], one rounding to fp16
+        const float d = __half2float(__ushort_as_half((uint16_t)raw.s));
+        const uint32_t w4[4] = {raw.a.x, raw.a.y, raw.a.z, raw.a.w};
+#pragma unroll
+        for (int k = 0; k < 16; ++k) {
+            float v[2];
+#pragma unroll
+            for (int u = 0; u < 2; ++u) {
+                const int i = 2 * k + u, byte = (w4[(i % 16) / 4] >> (8 * (i % 4))) & 0xFF;
+                v[u] = d * (float)iq4nl_level(i < 16 ? (byte & 15) : (byte >> 4));
+            }
+            o[k] = h2_bits(__floats2half2_rn(v[0], v[1]));
         }
     } else {
         const uint4 a = raw.a;
@@ -653,9 +710,10 @@ __global__ void __launch_bounds__(kGemmThreads, 1) k_umma_gemm(const __grid_cons
                 for (int i = threadIdx.x; i < cur.t.n; i += 128) xchg[i] = __ldg(p.w + __ldg(p.slot_pair + cur.t.b0 + i));
             }
             if ((KIND == G_GATEUP || KIND == G_DOWN) && threadIdx.x < 3) {
-                // the expert's tensor scales (gate, up, down) from its record tail
+                // the expert's tensor scales (gate, up, down) from its record
+                // tail; the Q3_K build has none
                 const size_t nq = (size_t)p.L * p.F / 2, ns = (size_t)p.L * p.F / 16;
-                tscale[threadIdx.x] =
+                tscale[threadIdx.x] = p.efmt == LMOE_EXPERTS_Q3K ? 1.f :
                     __ldg(reinterpret_cast<const float*>(p.experts + (size_t)cur.t.mat * p.rec_bytes + 3 * nq + 3 * ns) + threadIdx.x);
             } else if (KIND == G_SHARED_GATEUP && threadIdx.x < 3) {
                 tscale[threadIdx.x] = 1.f;

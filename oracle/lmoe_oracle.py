@@ -94,10 +94,13 @@ def nvfp4_matrix_bytes(rows: int, cols: int) -> int:
     return rows * cols // 2 + rows * cols // 16
 
 
-def expert_record_bytes(latent: int, ffn: int) -> int:
+def expert_record_bytes(latent: int, ffn: int, expert_fmt: str = "nvfp4") -> int:
     """gate [ffn, latent], up [ffn, latent], down [latent, ffn] in NVFP4 plus a
     16-byte tail holding the three fp32 tensor scales (teardown article, "What
-    is 4-bit": 1,935,376 B for 3,440,640 weights at latent 1792)."""
+    is 4-bit": 1,935,376 B for 3,440,640 weights at latent 1792); or the Q3_K
+    build: Q3_K gate and up, IQ4_NL down, no tail (1,630,720 B)."""
+    if expert_fmt == "q3k":
+        return 2 * (ffn * latent // 256 * 110) + latent * ffn // 32 * 18
     return 3 * nvfp4_matrix_bytes(ffn, latent) + 16
 
 
@@ -147,7 +150,71 @@ def decode_nvfp4(qbytes: np.ndarray, sbytes: np.ndarray, ts: float, rows: int, c
     return vals * np.repeat(scale, 16, axis=1) * float(ts)
 
 
-def decode_expert(record: np.ndarray, latent: int, ffn: int):
+# The other expert build (model page, "Model profile": Q3_K gate/up, IQ4_NL
+# down; teardown article, "What is 4-bit": 985,600 + 645,120 bytes per record
+# at latent 1792).  The pages give names and byte counts; the arrangement is
+# the one documented with the C ABI (planes over 128-column halves for Q3_K,
+# Q4_0-like planes for IQ4_NL).
+
+def iq4nl_levels() -> np.ndarray:
+    """The 16 IQ4_NL levels as read here: standard normal quantiles at
+    (i + 1/2) / 16, scaled so that the outermost is 127, rounded."""
+    from statistics import NormalDist
+    z = [NormalDist().inv_cdf((i + 0.5) / 16.0) for i in range(16)]
+    return np.rint(127.0 * np.array(z) / z[-1])
+
+
+def q3k_matrix_bytes(rows: int, cols: int) -> int:
+    return rows * cols // 256 * 110
+
+
+def iq4nl_matrix_bytes(rows: int, cols: int) -> int:
+    return rows * cols // 32 * 18
+
+
+def decode_q3k(blob, rows: int, cols: int) -> np.ndarray:
+    """Q3_K matrix [rows, cols]: w = d * (sc_j - 32) * (q - 4)."""
+    R, C = rows, cols
+    nh = C // 128
+    b = np.asarray(blob, np.uint8)
+    lo = b[: nh * R * 32].reshape(nh, R, 32).astype(np.int64)
+    hi = b[nh * R * 32: nh * R * 48].reshape(nh, R, 16).astype(np.int64)
+    sc = b[nh * R * 48: nh * R * 54].reshape(nh, R, 6).astype(np.int64)
+    d = fp16_to_f64(np.frombuffer(b[nh * R * 54: nh * R * 54 + 2 * (C // 256) * R].tobytes(), np.uint16)
+                    .reshape(C // 256, R))
+    e = np.arange(128)
+    q_lo = (lo[:, :, 4 * (e // 16) + e % 4] >> (2 * ((e % 16) // 4))) & 3           # [nh, R, 128]
+    q_hi = (hi[:, :, 4 * (e // 32) + e % 4] >> ((e % 32) // 4)) & 1
+    q = q_lo | (q_hi << 2)
+    word = sum(sc[:, :, k] << (8 * k) for k in range(6))                            # 48-bit words [nh, R]
+    j = e // 16
+    scj = (word[:, :, None] >> (6 * j)[None, None, :]) & 63                        # [nh, R, 128]
+    dv = np.repeat(d, 2, axis=0)[:, :, None]                                       # d of each half
+    w = dv * (scj - 32) * (q - 4)
+    return w.transpose(1, 0, 2).reshape(R, C)
+
+
+def decode_iq4nl(blob, rows: int, cols: int) -> np.ndarray:
+    """IQ4_NL matrix [rows, cols]: w = d * level[q], q as in Q4_0."""
+    nb = cols // 32
+    b = np.asarray(blob, np.uint8)[: rows * cols // 2].reshape(nb, rows, 16).astype(np.int64)
+    q = np.concatenate([b & 0xF, b >> 4], axis=2)
+    dbits = np.frombuffer(np.asarray(blob, np.uint8)[rows * cols // 2: rows * cols // 2 + 2 * nb * rows].tobytes(),
+                          np.uint16).reshape(nb, rows)
+    w = iq4nl_levels()[q] * fp16_to_f64(dbits)[:, :, None]
+    return w.transpose(1, 0, 2).reshape(rows, cols)
+
+
+def decode_expert(record: np.ndarray, latent: int, ffn: int, expert_fmt: str = "nvfp4"):
+    if expert_fmt == "q3k":
+        rec = np.asarray(record, np.uint8)
+        gb = q3k_matrix_bytes(ffn, latent)
+        return (decode_q3k(rec[:gb], ffn, latent), decode_q3k(rec[gb:2 * gb], ffn, latent),
+                decode_iq4nl(rec[2 * gb:2 * gb + iq4nl_matrix_bytes(latent, ffn)], latent, ffn))
+    return _decode_expert_nvfp4(record, latent, ffn)
+
+
+def _decode_expert_nvfp4(record: np.ndarray, latent: int, ffn: int):
     """-> (W_gate [ffn, latent], W_up [ffn, latent], W_down [latent, ffn]) in fp64."""
     nq = latent * ffn // 2
     ns = latent * ffn // 16
@@ -160,8 +227,8 @@ def decode_expert(record: np.ndarray, latent: int, ffn: int):
     return tuple(mats)
 
 
-def expert_slice(experts: np.ndarray, e: int, latent: int, ffn: int) -> np.ndarray:
-    rb = expert_record_bytes(latent, ffn)
+def expert_slice(experts: np.ndarray, e: int, latent: int, ffn: int, expert_fmt: str = "nvfp4") -> np.ndarray:
+    rb = expert_record_bytes(latent, ffn, expert_fmt)
     return experts[e * rb:(e + 1) * rb]
 
 
@@ -262,7 +329,8 @@ class Weights:
             if len(self._E) >= self._max:
                 self._E.pop(next(iter(self._E)))
             s = self.s
-            self._E[e] = decode_expert(expert_slice(self.layer["experts"], e, s.latent, s.ffn), s.latent, s.ffn)
+            f = getattr(s, "expert_fmt", "nvfp4")
+            self._E[e] = decode_expert(expert_slice(self.layer["experts"], e, s.latent, s.ffn, f), s.latent, s.ffn, f)
         return self._E[e]
 
 

@@ -44,7 +44,7 @@ def build(force: bool = False) -> str:
 
 class _Shape(ctypes.Structure):
     _fields_ = [(n, ctypes.c_int) for n in ("hidden", "latent", "n_experts", "top_k", "n_groups", "ffn",
-                                            "shared_ffn", "du_fmt", "router_bf16")]
+                                            "shared_ffn", "du_fmt", "router_bf16", "expert_fmt")]
 
 
 class _Layer(ctypes.Structure):
@@ -80,6 +80,14 @@ def lib():
         L.orc_forward.argtypes = [ctypes.POINTER(_Shape), ctypes.POINTER(_Layer), vp, vp, vp, vp, i32, vp, vp, vp, vp]
         L.orc_rmsnorm.argtypes = [vp, vp, dbl, i32, i32, vp]
         L.orc_quantize_q8_1.argtypes = [vp, i32, i32, vp, vp]
+        L.orc_decode_q3k_iq4nl.restype = i32
+        L.orc_decode_q3k_iq4nl.argtypes = [i32, vp, i32, i32, vp]
+        L.orc_iq4nl_levels.argtypes = [vp]
+        L.orc_expert_record_bytes_fmt.restype = i64
+        L.orc_expert_record_bytes_fmt.argtypes = [i32, i32, i32]
+        L.orc_expert_offset_fmt.restype = i64
+        L.orc_expert_offset_fmt.argtypes = [i32, i32, i32, i32]
+        L.orc_decode_expert_fmt.argtypes = [i32, vp, i32, i32, vp, vp, vp]
         L.orc_dproj_q8_1.argtypes = [i32, vp, i32, i32, i32, vp, i32, vp]
         L.orc_stack_layer.restype = i32
         L.orc_stack_layer.argtypes = [ctypes.POINTER(_Shape), ctypes.POINTER(_Layer), vp, vp, dbl, vp, vp, i32, vp,
@@ -133,8 +141,34 @@ def du_matrix_bytes(fmt: int, rows: int, cols: int) -> int:
     return int(lib().orc_du_matrix_bytes(fmt, rows, cols))
 
 
-def expert_record_bytes(latent: int, ffn: int) -> int:
-    return int(lib().orc_expert_record_bytes(latent, ffn))
+def _efmt(expert_fmt) -> int:
+    return 1 if expert_fmt == "q3k" else 0
+
+
+def expert_record_bytes(latent: int, ffn: int, expert_fmt: str = "nvfp4") -> int:
+    return int(lib().orc_expert_record_bytes_fmt(_efmt(expert_fmt), latent, ffn))
+
+
+def iq4nl_levels() -> np.ndarray:
+    out = np.empty(16)
+    lib().orc_iq4nl_levels(_ptr(out))
+    return out
+
+
+def decode_q3k(blob, rows: int, cols: int) -> np.ndarray:
+    b, p = _c(blob, np.uint8)
+    out = np.empty((rows, cols))
+    if lib().orc_decode_q3k_iq4nl(1, p, rows, cols, _ptr(out)) != 0:
+        raise ValueError("Q3_K columns must be a multiple of 256")
+    return out
+
+
+def decode_iq4nl(blob, rows: int, cols: int) -> np.ndarray:
+    b, p = _c(blob, np.uint8)
+    out = np.empty((rows, cols))
+    if lib().orc_decode_q3k_iq4nl(2, p, rows, cols, _ptr(out)) != 0:
+        raise ValueError("IQ4_NL columns must be a multiple of 32")
+    return out
 
 
 def decode_du(fmt: int, blob, rows: int, cols: int) -> np.ndarray:
@@ -164,19 +198,19 @@ def decode_nvfp4(qbytes, sbytes, ts, rows: int, cols: int) -> np.ndarray:
     return out
 
 
-def decode_expert(record, latent: int, ffn: int):
+def decode_expert(record, latent: int, ffn: int, expert_fmt: str = "nvfp4"):
     r, p = _c(record, np.uint8)
-    assert r.size >= expert_record_bytes(latent, ffn)
+    assert r.size >= expert_record_bytes(latent, ffn, expert_fmt)
     wg = np.empty((ffn, latent))
     wu = np.empty((ffn, latent))
     wd = np.empty((latent, ffn))
-    lib().orc_decode_expert(p, latent, ffn, _ptr(wg), _ptr(wu), _ptr(wd))
+    lib().orc_decode_expert_fmt(_efmt(expert_fmt), p, latent, ffn, _ptr(wg), _ptr(wu), _ptr(wd))
     return wg, wu, wd
 
 
-def expert_slice(experts: np.ndarray, e: int, latent: int, ffn: int) -> np.ndarray:
-    o = int(lib().orc_expert_offset(e, latent, ffn))
-    return experts[o:o + expert_record_bytes(latent, ffn)]
+def expert_slice(experts: np.ndarray, e: int, latent: int, ffn: int, expert_fmt: str = "nvfp4") -> np.ndarray:
+    o = int(lib().orc_expert_offset_fmt(_efmt(expert_fmt), e, latent, ffn))
+    return experts[o:o + expert_record_bytes(latent, ffn, expert_fmt)]
 
 
 def du_slice(blob: np.ndarray, fmt: int, g: int, rows: int, cols: int) -> np.ndarray:
@@ -205,7 +239,8 @@ def route(x, Wr, b, top_k: int):
 
 def _shape(shape) -> _Shape:
     return _Shape(shape.hidden, shape.latent, shape.n_experts, shape.top_k, shape.n_groups, shape.ffn,
-                  shape.shared_ffn, shape.du_fmt, 1 if shape.router_dtype == "bf16" else 0)
+                  shape.shared_ffn, shape.du_fmt, 1 if shape.router_dtype == "bf16" else 0,
+                  _efmt(getattr(shape, "expert_fmt", "nvfp4")))
 
 
 class _LayerRef:
@@ -346,7 +381,8 @@ class Weights:
             if len(self._E) >= self._max:
                 self._E.pop(next(iter(self._E)))
             s = self.s
-            self._E[e] = decode_expert(expert_slice(self.layer["experts"], e, s.latent, s.ffn), s.latent, s.ffn)
+            f = getattr(s, "expert_fmt", "nvfp4")
+            self._E[e] = decode_expert(expert_slice(self.layer["experts"], e, s.latent, s.ffn, f), s.latent, s.ffn, f)
         return self._E[e]
 
 

@@ -450,3 +450,39 @@ def test_dproj_ablation_matches_oracle(name, T):
             assert orc.rel_l2(got[:, g], ref_g) < 1e-4, g
         else:
             assert np.all(np.isnan(got[:, g])), g
+
+
+# ----------------------------------------------------------------------------
+# the Q3_K gate/up + IQ4_NL down expert build
+# ----------------------------------------------------------------------------
+
+def test_decode_q3k_iq4nl_match_oracle_bit_for_bit():
+    rng = np.random.default_rng(61)
+    w = rng.normal(0, 0.03, size=(48, 512))
+    for fmt, blob, dec in ((B.LMOE_Q3K_DEBUG, synth.q3k_encode(w), orc.decode_q3k),
+                           (B.LMOE_IQ4NL_DEBUG, synth.iq4nl_encode(w), orc.decode_iq4nl)):
+        out = torch.empty(48, 512, dtype=torch.float32, device="cuda")
+        B.lmoe_debug_decode(fmt, to_device(blob, "cuda"), 48, 512, 1.0, out)
+        np.testing.assert_array_equal(out.cpu().numpy().astype(np.float64), dec(blob, 48, 512))
+
+
+@pytest.mark.parametrize("T", [1, 4, 8, 13, 37])
+def test_block_q3k_experts_few_tokens(T):
+    """The one-kernel step with Q3_K gate/up and IQ4_NL down records (T <= 8),
+    and the same step on passes of 8 tokens (9-63)."""
+    wl = small_workload(T, latent=256, expert_fmt="q3k")
+    check_block(wl.shape, synth.make_layer(wl), synth.make_x(wl), what=f"q3k T={T}")
+
+
+def test_block_q3k_experts_tensor_cores():
+    wl = prefill_workload(300, latent=256, expert_fmt="q3k")
+    res = synth.bf16_normal(synth.key(4, 0, "residual"), 1.0, (300, wl.shape.hidden))
+    check_block(wl.shape, synth.make_layer(wl), synth.make_x(wl), residual_bits=res, what="q3k prefill")
+
+
+def test_block_q3k_145b_decode_config():
+    wl = synth.WORKLOADS["edge0_145b_q3k_decode"]
+    layer = synth.make_layer(wl)
+    dev = DeviceLayer(wl.shape, layer)
+    for draw in range(2):
+        check_block(wl.shape, layer, synth.make_x(wl, draw=draw), dev=dev, what=f"145B q3k draw {draw}")

@@ -618,3 +618,132 @@ def test_dproj_q8_1_equals_projection_of_the_dequantised_rows():
     for g in range(G):
         Dg = torch.from_numpy(np_oracle.decode_du(synth.Q4_0, np_oracle.du_slice(layer["D"], synth.Q4_0, g, L, H), L, H))
         np.testing.assert_allclose(h[:, g], (xq @ Dg.T).numpy(), rtol=1e-12, atol=1e-13)
+
+
+# ----------------------------------------------------------------------------
+# the Q3_K gate/up + IQ4_NL down expert build
+# ----------------------------------------------------------------------------
+
+def test_q3k_build_sizes_match_pages(orc):
+    """The record sizes and build totals the pages print for the Q3_K build,
+    with the Q8_0 (145B) and Q4_0 (120B) D/U of the NVFP4 builds."""
+    g = _gold("page_figures.json")
+    H, E, G, F, NL = (g[k]["value"] for k in ("hidden", "experts_per_layer", "groups", "swiglu_width", "layers"))
+    L145, L120 = g["latent_145b"]["value"], g["latent_120b"]["value"]
+    assert orc.expert_record_bytes(L145, F, "q3k") == g["q3k_record_bytes_latent1792"]["value"]
+    assert 2 * (F * L145 // 256 * 110) == g["q3k_record_gateup_bytes_latent1792"]["value"]
+    assert L145 * F // 32 * 18 == g["q3k_record_down_bytes_latent1792"]["value"]
+    assert orc.expert_record_bytes(L120, F, "q3k") == g["q3k_record_bytes_latent1280"]["value"]
+    b145 = NL * (E * orc.expert_record_bytes(L145, F, "q3k") + 2 * G * orc.du_matrix_bytes(orc.Q8_0, L145, H))
+    b120 = NL * (E * orc.expert_record_bytes(L120, F, "q3k") + 2 * G * orc.du_matrix_bytes(orc.Q4_0, L120, H))
+    assert round(b145 / 2 ** 30, 2) == g["weights_145b_q3k_gib"]["value"]
+    assert round(b120 / 2 ** 30, 2) == g["weights_120b_q3k_gib"]["value"]
+
+
+def test_iq4nl_levels_are_the_scaled_normal_quantiles(orc):
+    from scipy.stats import norm
+    z = norm.ppf((np.arange(16) + 0.5) / 16.0)
+    np.testing.assert_array_equal(orc.iq4nl_levels(), np.rint(127.0 * z / z[-1]))
+    assert orc.iq4nl_levels()[0] == -127 and orc.iq4nl_levels()[15] == 127
+
+
+def test_decode_q3k_hand_packed(orc):
+    """Codes, sub-block scales and super-block scales placed bit by bit from
+    the documented arrangement; w = d * (sc - 32) * (q - 4)."""
+    R, C = 3, 512
+    rng = np.random.default_rng(51)
+    q = rng.integers(0, 8, size=(R, C))
+    sc = rng.integers(0, 64, size=(R, C // 16))
+    d = rng.choice([0.5, 0.25, 0.0078125, 1.5], size=(R, C // 256))
+    nh = C // 128
+    lo = bytearray(nh * R * 32)
+    hi = bytearray(nh * R * 16)
+    scb = bytearray(nh * R * 6)
+    db = bytearray(2 * (C // 256) * R)
+    want = np.zeros((R, C))
+    for r in range(R):
+        for c in range(C):
+            h, e = divmod(c, 128)
+            lo[(h * R + r) * 32 + 4 * (e // 16) + e % 4] |= (int(q[r, c]) & 3) << (2 * ((e % 16) // 4))
+            if q[r, c] & 4:
+                hi[(h * R + r) * 16 + 4 * (e // 32) + e % 4] |= 1 << ((e % 32) // 4)
+            want[r, c] = d[r, c // 256] * (sc[r, c // 16] - 32) * (q[r, c] - 4)
+        for h in range(nh):
+            word = sum(int(sc[r, h * 8 + j]) << (6 * j) for j in range(8))
+            for k in range(6):
+                scb[(h * R + r) * 6 + k] = (word >> (8 * k)) & 0xFF
+        for sb in range(C // 256):
+            bits = _fp16_bits(d[r, sb])
+            db[2 * (sb * R + r)], db[2 * (sb * R + r) + 1] = bits & 0xFF, bits >> 8
+    blob = np.frombuffer(bytes(lo + hi + scb + db), np.uint8)
+    assert blob.size == R * C // 256 * 110
+    np.testing.assert_array_equal(orc.decode_q3k(blob, R, C), want)
+
+
+def test_decode_iq4nl_hand_packed(orc):
+    R, C = 2, 64
+    rng = np.random.default_rng(52)
+    q = rng.integers(0, 16, size=(R, C))
+    d = rng.choice([0.5, -0.25, 2.0 ** -10], size=(R, C // 32))
+    from scipy.stats import norm
+    z = norm.ppf((np.arange(16) + 0.5) / 16.0)
+    lev = np.rint(127.0 * z / z[-1])
+    blob = bytearray(R * C // 2 + R * C // 16)
+    want = np.zeros((R, C))
+    for r in range(R):
+        for c in range(C):
+            b, j = divmod(c, 32)
+            blob[(b * R + r) * 16 + j % 16] |= int(q[r, c]) << (0 if j < 16 else 4)
+            want[r, c] = lev[q[r, c]] * d[r, b]
+        for b in range(C // 32):
+            bits = _fp16_bits(d[r, b])
+            off = R * C // 2 + 2 * (b * R + r)
+            blob[off], blob[off + 1] = bits & 0xFF, bits >> 8
+    np.testing.assert_array_equal(orc.decode_iq4nl(np.frombuffer(bytes(blob), np.uint8), R, C), want)
+
+
+def test_q3k_generator_round_trip(orc):
+    """The generator's Q3_K / IQ4_NL bytes decode to the matrices it encoded,
+    within each format's grid: Q3_K within one sub-block step (|s| <= amax/4
+    of the 16 elements, plus the 6-bit rounding of s), IQ4_NL within the
+    widest half-gap of the levels (37/2 of d = amax/127)."""
+    rng = np.random.default_rng(53)
+    w = rng.normal(0, 0.02, size=(32, 512))
+    back = orc.decode_q3k(synth.q3k_encode(w), 32, 512)
+    amax16 = np.repeat(np.abs(w).reshape(32, -1, 16).max(axis=2), 16, axis=1)
+    assert np.all(np.abs(back - w) <= amax16 * 0.35 + 1e-12)
+    assert orc.rel_l2(back, w) < 0.2
+    back = orc.decode_iq4nl(synth.iq4nl_encode(w), 32, 512)
+    amax32 = np.repeat(np.abs(w).reshape(32, -1, 32).max(axis=2), 32, axis=1)
+    assert np.all(np.abs(back - w) <= amax32 / 127.0 * 18.6 + 1e-12)
+    assert orc.rel_l2(back, w) < 0.12
+
+
+def test_q3k_block_equals_dense_masked_brute_force(orc):
+    """The block with Q3_K experts: every expert on every token, masked by the
+    routing weights, in torch from the decoded matrices."""
+    s = synth.replace(TINY, latent=256, expert_fmt="q3k")
+    wl, layer, xb = _tiny_layer(shape=s)
+    y, idx, w, _ = orc.latent_moe_forward(s, layer, xb)
+    F = torch.nn.functional
+    x = _t(orc.bf16_to_f64(xb))
+    logits = x @ _t(layer["router_w"].astype(np.float64)).T + _t(layer["router_b"].astype(np.float64))
+    grp = layer["expert_group"].astype(np.int64)
+    bf = lambda a: torch.from_numpy(a.view(np.int16)).view(torch.bfloat16).double()
+    want = (F.silu(x @ bf(layer["shared_gate"]).T) * (x @ bf(layer["shared_up"]).T)) @ bf(layer["shared_down"]).T
+    for t in range(x.shape[0]):
+        sel, ws = _brute_route(logits[t].tolist(), s.top_k)
+        assert list(idx[t]) == sel
+        for g in sorted({int(grp[e]) for e in sel}):
+            Dg = _t(orc.decode_du(s.du_fmt, orc.du_slice(layer["D"], s.du_fmt, g, s.latent, s.hidden), s.latent, s.hidden))
+            Ug = _t(orc.decode_du(s.du_fmt, orc.du_slice(layer["U"], s.du_fmt, g, s.hidden, s.latent), s.hidden, s.latent))
+            h = Dg @ x[t]
+            acc = torch.zeros(s.latent, dtype=torch.float64)
+            for e, wk in zip(sel, ws):
+                if grp[e] != g:
+                    continue
+                Wg, Wu, Wd = (_t(m) for m in orc.decode_expert(orc.expert_slice(layer["experts"], e, s.latent, s.ffn, "q3k"),
+                                                               s.latent, s.ffn, "q3k"))
+                acc += wk * (Wd @ (F.silu(Wg @ h) * (Wu @ h)))
+            want[t] += Ug @ acc
+    np.testing.assert_allclose(y, want.numpy(), rtol=1e-10, atol=1e-12)
