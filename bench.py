@@ -131,7 +131,6 @@ def step_cost(shape, idx: np.ndarray, groups: np.ndarray, T: int, prefill: bool)
     distinct = set(idx.reshape(-1).tolist())
     pairs_tg = sum(len({int(groups[e]) for e in idx[t]}) for t in range(idx.shape[0]))   # hit (token, group) pairs
     b = {
-        "k_decode_step": 0.0,
         "k_router_shared": rw + 2 * Fs * H * 2 + T * H * 2,
         "k_wstream_dproj": G * du + T * H * 2,     # every group (D runs before the routing is known)
         "k_wstream_gateup": len(distinct) * rec_gu,
@@ -140,7 +139,10 @@ def step_cost(shape, idx: np.ndarray, groups: np.ndarray, T: int, prefill: bool)
     }
     # the step's algorithmic bytes count only the hit groups' D
     b_total = float(sum(b.values()) - (G - len(hit)) * du)
-    b["k_decode_step"] = b_total            # the whole step in one kernel
+    # the 9-63-token kernels read the same bytes per pass of 8 tokens
+    for a, c in (("k_dproj_mma", "k_wstream_dproj"), ("k_gateup_mma", "k_wstream_gateup"),
+                 ("k_down_mma", "k_wstream_down"), ("k_uproj_mma", "k_wstream_uproj")):
+        b[a] = b[c]
     f = {
         "x_to_fp16": 0.0,
         "router_gemm": 2.0 * T * E * H,
@@ -190,10 +192,11 @@ def ncu_traffic(workload: str, T: int, kernel: str):
 
 
 def decode_stages(T: int):
-    """Kernels of one few-token step: one persistent kernel up to 8 tokens
-    (every Edge0-shaped layer fits it), five kernels from 9 to 63."""
+    """Kernels of one few-token step (NVFP4 experts): the router kernel and
+    four weight-streaming kernels up to 8 tokens, the passes-of-8 kernels
+    from 9 to 63."""
     if T <= 8:
-        return ["k_decode_step"]
+        return ["k_router_shared", "k_wstream_dproj", "k_wstream_gateup", "k_wstream_down", "k_wstream_uproj"]
     return ["k_router_shared", "k_dproj_mma", "k_gateup_mma", "k_down_mma", "k_uproj_mma"]
 
 
@@ -567,8 +570,8 @@ def measure_layer(args, wl, T, K, W, rank, world, local, dev_name, ctx=None, lig
                    "weights": "NVFP4 experts, Q8_0/Q4_0 D/U, bf16 router and shared expert; "
                               "bf16 activations in and out, fp32 accumulation",
                    "path": ("tensor cores (tcgen05): fp16 operands dequantised from the stored formats"
-                            if prefill else "one persistent kernel per step: weight streaming on the tensor pipe "
-                                            "(mma.sync, fp16 operands, fp32 accumulation)"),
+                            if prefill else "router kernel + four weight-streaming kernels (mma.sync, fp16 "
+                                            "operands, fp32 accumulation), programmatic dependent launch"),
                    "timing": f"{n_graphs} captured CUDA graphs replayed in turn"},
         "roofline": roof,
         "layer": {"gbs": step_alg_bytes / t_step / 1e9, "tflops": step_flops / t_step / 1e12,

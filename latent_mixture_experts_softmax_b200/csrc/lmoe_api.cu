@@ -299,21 +299,12 @@ int forward_impl(const lmoe_cfg* cfg, const void* x, const void* router_w, const
     p.out_w = out_w;
     p.y = static_cast<uint16_t*>(y);
     if (use_prefill(*cfg, T)) return run_prefill(*cfg, p, L, ws, st);
-    if (T <= 8 && decode_step_fits(p)) {
-        // one kernel; it clears its own counters, so no per-call reset
-        stage_reset();
-        return cuda_status(run_decode_step(p, st));
-    }
-    if (cfg->expert_fmt == LMOE_EXPERTS_Q3K) {
-        // the Q3_K build between 9 and 63 tokens: the one-kernel step on
-        // passes of at most 8 tokens (the five-kernel path of that range
-        // reads NVFP4 records only)
-        FwdParams q = p;
-        q.T = std::min(T, 8);
-        if (!decode_step_fits(q)) return LMOE_ERR_UNSUPPORTED;
-        stage_reset();
+    if (cfg->expert_fmt == LMOE_EXPERTS_Q3K && T > 8) {
+        // the Q3_K build between 9 and 63 tokens: the few-token step on
+        // passes of at most 8 tokens (the kernels of that range read NVFP4
+        // records only)
         for (int t0 = 0; t0 < T; t0 += 8) {
-            q = p;
+            FwdParams q = p;
             q.T = std::min(8, T - t0);
             q.x = p.x + (size_t)t0 * p.H;
             q.y = p.y + (size_t)t0 * p.H;
@@ -321,7 +312,8 @@ int forward_impl(const lmoe_cfg* cfg, const void* x, const void* router_w, const
             if (p.inject_idx) { q.inject_idx = p.inject_idx + (size_t)t0 * p.K; q.inject_w = p.inject_w + (size_t)t0 * p.K; }
             if (p.out_idx) q.out_idx = p.out_idx + (size_t)t0 * p.K;
             if (p.out_w) q.out_w = p.out_w + (size_t)t0 * p.K;
-            const cudaError_t e = run_decode_step(q, st);
+            if (reset_tickets(ws, st) != cudaSuccess) return LMOE_ERR_CUDA;
+            const cudaError_t e = run_gemv_path(q, st, false);
             if (e != cudaSuccess) return LMOE_ERR_CUDA;
         }
         return LMOE_OK;

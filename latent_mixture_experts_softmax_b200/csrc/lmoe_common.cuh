@@ -110,13 +110,7 @@ __device__ __forceinline__ int block_exclusive_scan(int v, int* out, int* scratc
 struct Ctrl {
     int status;                 // lmoe_status set by kernels
     int route_ticket;           // CTAs of the router that finished
-    // one-kernel decode step: arrivals counted per step and cleared by the
-    // last CTA to leave (zero between calls)
-    unsigned dec_rows;          // router rows whose logits are written
-    unsigned dec_phase[3];      // CTAs done with D, gate/up, down
-    unsigned dec_exit;          // CTAs that left the kernel
-    int dec_abort;              // a bounded wait gave up: skip the rest
-    int pad[56];
+    int pad[62];
     int tile_ticket[960];       // per output row tile of the U stage
 };
 static_assert(sizeof(Ctrl) <= 4096, "control block");

@@ -91,9 +91,6 @@ constexpr int kMaxStageEvents = 16;
 
 cudaError_t run_gemv_path(const FwdParams& p, cudaStream_t st, bool route_only);
 cudaError_t run_stream_path(const FwdParams& p, cudaStream_t st);
-// the whole few-token step (T <= 8) in one persistent kernel, when it fits
-bool decode_step_fits(const FwdParams& p);
-cudaError_t run_decode_step(FwdParams p, cudaStream_t st);
 // workspace of the few-token path's split reductions, for up to T tokens
 size_t stream_ws_part_bytes(int H, int L, int F, int Fs, int G, int E, int K, int T, int du_fmt);
 size_t stream_ws_tick_bytes(int H, int L, int F, int Fs, int G, int E, int K, int T, int du_fmt);

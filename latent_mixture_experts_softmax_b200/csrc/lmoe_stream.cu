@@ -31,7 +31,6 @@
 #include "lmoe_internal.cuh"
 #include "lmoe_q3k.cuh"
 #include "lmoe_route.cuh"
-#include "lmoe_rowdot.cuh"
 #include "lmoe_sm100.cuh"
 
 namespace lmoe {
@@ -993,254 +992,6 @@ __global__ void __launch_bounds__(kWThreads, 1) k_wstream(FwdParams p, WPlan pl,
 }
 
 // ---------------------------------------------------------------------------
-// the whole few-token step in one persistent kernel
-// ---------------------------------------------------------------------------
-//
-// One CTA per SM, all resident (cooperative launch).  Per CTA:
-//   1. D's plan and first weight steps (D needs no routing), then its share of
-//      the router rows (logits) and of the shared expert's gate/up rows
-//   2. the routing, computed in every CTA from all logits once every row is
-//      written (counted in the control block); the routed experts' records,
-//      the hit groups' U_g and the shared down projection are then streamed
-//      into L2 (bulk prefetch, a hint), so HBM stays busy across the phase
-//      boundaries that follow
-//   3. D, gate/up, down, U as in the per-phase kernels; between two phases a
-//      CTA counts itself done, issues the next phase's first weight steps
-//      (they depend only on the routing) and then waits for every CTA
-// Every wait is bounded (about 2 s of SM clock): on timeout the CTA raises
-// an abort word that makes every other wait give up, the step records
-// LMOE_ERR_TIMEOUT, and each CTA drains its copies and leaves.  The last CTA
-// to leave clears the step's counters.
-
-constexpr uint64_t kDecodeWaitCycles = 4000000000ull;
-
-__device__ __forceinline__ unsigned ld_acquire_u32(const unsigned* ptr) {
-    unsigned v;
-    asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(ptr) : "memory");
-    return v;
-}
-
-// One thread: wait until *ctr >= target.  False if the wait gave up (the
-// step's abort word and status are then set) or another CTA had given up.
-__device__ bool wait_at_least(const unsigned* ctr, unsigned target, Ctrl* c) {
-    if (ld_acquire_u32(ctr) >= target) return true;
-    const uint64_t t0 = clock64();
-    while (true) {
-        if (ld_acquire_u32(ctr) >= target) return true;
-        if (*reinterpret_cast<volatile int*>(&c->dec_abort)) return false;
-        if ((uint64_t)(clock64() - t0) > kDecodeWaitCycles) {
-            atomicExch(&c->dec_abort, 1);
-            set_status(c, LMOE_ERR_TIMEOUT);
-            return false;
-        }
-        __nanosleep(20);
-    }
-}
-
-// This CTA's phase is complete: every thread's global writes of the phase
-// are made visible to the whole GPU before the CTA is counted.
-__device__ __forceinline__ void phase_arrive(unsigned* ctr) {
-    __syncthreads();
-    if (threadIdx.x == 0) {
-        __threadfence();
-        atomicAdd(ctr, 1u);
-    }
-}
-
-// Wait until every CTA has arrived (all threads return the same answer).
-__device__ __forceinline__ bool phase_wait(const unsigned* ctr, Ctrl* c, int* s_ok) {
-    if (threadIdx.x == 0) *s_ok = wait_at_least(ctr, gridDim.x, c);
-    __syncthreads();
-    return *s_ok != 0;
-}
-
-// Router logits and the shared expert's hidden state.  Item i (router row
-// i < E, then shared feature i - E) is taken by warp i / grid of CTA
-// i % grid; the block input is staged as fp32, 4 tokens per pass.  Each warp
-// counts its router rows once all their logits are written.
-template <bool kBF16>
-__device__ __noinline__ void decode_rows(const FwdParams& p, float* xs, float* rs) {
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int n_items = p.E + p.Fs, H = p.H, ld = xs_ld(H);
-    bool bad = false;
-    for (int t0 = 0; t0 < p.T; t0 += 4) {
-        const int nt = min(4, p.T - t0);
-        stage_x<4>(p, t0, nt, xs, rs);
-        __syncthreads();
-        for (int i = blockIdx.x + gridDim.x * warp; i < n_items; i += gridDim.x * kWW) {
-            if (i < p.E) {
-                float acc[4] = {0.f, 0.f, 0.f, 0.f};
-                if (kBF16) row_dot<4, true>(static_cast<const uint16_t*>(p.router_w) + (size_t)i * H, H, xs, ld, lane, acc);
-                else row_dot<4, false>(static_cast<const float*>(p.router_w) + (size_t)i * H, H, xs, ld, lane, acc);
-                const float b = p.router_b ? __ldg(p.router_b + i) : 0.f;
-#pragma unroll
-                for (int t = 0; t < 4; ++t) {
-                    const float v = warp_sum(acc[t]);
-                    if (lane == 0 && t < nt) p.r.logits[(size_t)(t0 + t) * p.E + i] = v + b;
-                }
-            } else {
-                const int f = i - p.E;
-                float a[4] = {0.f, 0.f, 0.f, 0.f}, u[4] = {0.f, 0.f, 0.f, 0.f};
-                row_dot2_bf16<4, 5>(p.sg + (size_t)f * H, p.su + (size_t)f * H, H, xs, ld, lane, a, u);
-#pragma unroll
-                for (int t = 0; t < 4; ++t) {
-                    const float av = warp_sum(a[t]), uv = warp_sum(u[t]);
-                    if (lane == 0 && t < nt) p.zsh16[(size_t)(t0 + t) * p.Fs + f] = half_checked(silu(av) * uv, bad);
-                }
-            }
-        }
-        __syncthreads();
-    }
-    report_range(p.ctrl, bad);
-    if (lane == 0) {
-        unsigned mine = 0;
-        for (int i = blockIdx.x + gridDim.x * warp; i < p.E; i += gridDim.x * kWW) ++mine;
-        if (mine) {
-            __threadfence();
-            atomicAdd(&p.ctrl->dec_rows, mine);
-        }
-    }
-}
-
-// Bring the rest of the step's weights into L2 while D streams: the routed
-// experts' records, U_g of the hit groups, the shared down projection, in
-// 32 KiB pieces spread over every CTA's threads.
-__device__ __noinline__ void prefetch_step_weights(const FwdParams& p, const StreamShared& sh) {
-    constexpr uint32_t kPiece = 32768;
-    const size_t sd_bytes = (size_t)p.H * p.Fs * 2;
-    const uint32_t per_rec = (uint32_t)((p.rec_bytes + kPiece - 1) / kPiece);
-    const uint32_t per_u = (uint32_t)((p.du_bytes_U + kPiece - 1) / kPiece);
-    const uint32_t per_sd = (uint32_t)((sd_bytes + kPiece - 1) / kPiece);
-    const uint32_t n_rec = (uint32_t)sh.n_unique * per_rec, n_u = (uint32_t)sh.n_hit * per_u;
-    const uint32_t total = n_rec + n_u + per_sd;
-    for (uint32_t i = blockIdx.x + gridDim.x * threadIdx.x; i < total; i += gridDim.x * blockDim.x) {
-        const uint8_t* base;
-        size_t bytes;
-        uint32_t j;
-        if (i < n_rec) {
-            j = i % per_rec;
-            base = p.experts + (size_t)sh.uexp[i / per_rec] * p.rec_bytes;
-            bytes = p.rec_bytes;
-        } else if (i < n_rec + n_u) {
-            const uint32_t k = i - n_rec;
-            j = k % per_u;
-            base = p.U + (size_t)sh.hg[k / per_u] * p.du_bytes_U;
-            bytes = p.du_bytes_U;
-        } else {
-            j = i - n_rec - n_u;
-            base = reinterpret_cast<const uint8_t*>(p.sd);
-            bytes = sd_bytes;
-        }
-        const size_t off = (size_t)j * kPiece;
-        const uint32_t len = (uint32_t)min((size_t)kPiece, bytes - off) & ~15u;
-        if (len) asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(base + off), "r"(len) : "memory");
-    }
-}
-
-// The routing of the step in this CTA (a function of its own, so that its
-// registers are not held across the streaming loops).
-__device__ __noinline__ void decode_route(const FwdParams& p, StreamShared& sh, TopkScratch& ts, const uint8_t* grp) {
-    route_in_cta(p, sh, ts, grp, blockIdx.x == 0);
-}
-
-// Plans and sizes of the one-kernel step, fixed on the host.
-struct DecodeLayout {
-    WPlan d, gu, dn, u;
-    int cache_bytes;
-};
-
-// One phase after the first: count the previous phase done, issue this
-// phase's first weight steps, wait for every CTA, fill the activations, run.
-template <int PHASE, int FMT>
-__device__ __noinline__ bool decode_phase(const FwdParams& p, StreamShared& sh, const WPlan& base_plan, ChunkInfo& ci,
-                             int cache_bytes, uint8_t* ring_base, __half* cache, unsigned* prev_done, int* s_ok) {
-    phase_arrive(prev_done);
-    WPlan plan = base_plan;
-    plan.n_mats = phase_mats<PHASE>(p, sh);
-    phase_setup<PHASE, FMT>(p, sh, plan, cache_bytes, ci);
-    const StepMap m = step_map<PHASE, FMT>(p, sh, plan);
-    LoadCursor lc;
-    phase_prime<PHASE, FMT>(p, sh, plan, ci, m, ring_base + (size_t)(threadIdx.x >> 5) * kPD * kStepBytes, lc);
-    if (!phase_wait(prev_done, p.ctrl, s_ok)) {
-        cp_async_wait<0>();
-        return false;
-    }
-    phase_fill<PHASE>(p, sh, ci, cache);
-    __syncthreads();
-    phase_run<PHASE, FMT>(p, sh, plan, ci, m, ring_base, cache, lc);
-    return true;
-}
-
-// The first phase: D's first weight steps, the router and shared-expert
-// rows, the routing and the L2 prefetch, then D itself.  False if a wait
-// gave up.
-template <int FMT>
-__device__ __noinline__ bool decode_first(const FwdParams& p, const DecodeLayout& dl, StreamShared& sh, ChunkInfo& ci,
-                                          const uint8_t* sgrp, uint8_t* ring_base, __half* cache, float* xs, float* rs,
-                                          int* s_ok) {
-    WPlan pd = dl.d;
-    pd.n_mats = p.G;
-    phase_setup<SP_DPROJ, FMT>(p, sh, pd, dl.cache_bytes, ci);
-    const StepMap md = step_map<SP_DPROJ, FMT>(p, sh, pd);
-    LoadCursor lc;
-    phase_prime<SP_DPROJ, FMT>(p, sh, pd, ci, md, ring_base + (size_t)(threadIdx.x >> 5) * kPD * kStepBytes, lc);
-    if (p.router_bf16) decode_rows<true>(p, xs, rs);
-    else decode_rows<false>(p, xs, rs);
-    if (threadIdx.x == 0) *s_ok = wait_at_least(&p.ctrl->dec_rows, (unsigned)p.E, p.ctrl);
-    __syncthreads();
-    if (!*s_ok) {
-        cp_async_wait<0>();
-        return false;
-    }
-    decode_route(p, sh, *reinterpret_cast<TopkScratch*>(xs), sgrp);
-    prefetch_step_weights(p, sh);
-    phase_fill<SP_DPROJ>(p, sh, ci, cache);
-    __syncthreads();
-    phase_run<SP_DPROJ, FMT>(p, sh, pd, ci, md, ring_base, cache, lc);
-    return true;
-}
-
-template <int FMT, int EF>
-__global__ void __launch_bounds__(kWThreads, 1)
-    k_decode_step(const __grid_constant__ FwdParams p, const __grid_constant__ DecodeLayout dl) {
-    extern __shared__ uint8_t smem_raw[];
-    uint8_t* smem = smem_raw + ((128u - (smem_u32(smem_raw) & 127u)) & 127u);
-    __shared__ StreamShared sh;
-    __shared__ ChunkInfo ci;                   // the phase being primed or run
-    __shared__ uint8_t sgrp[kMaxExpertsTopk];
-    __shared__ float rs[8];
-    __shared__ int s_ok;
-    Ctrl* ctrl = p.ctrl;
-    __half* cache = reinterpret_cast<__half*>(smem);
-    uint8_t* ring_base = smem + dl.cache_bytes;
-    float* xs = reinterpret_cast<float*>(ring_base + (size_t)kWW * kPD * kStepBytes);
-
-    for (int e = threadIdx.x; e < p.E; e += blockDim.x) sgrp[e] = p.group[e];
-    if (EF == kEfQ3k) iq4nl_fill_lut(iq4nl_lut());
-    // U's output-tile tickets are first used after three grid barriers
-    if (blockIdx.x == 0)
-        for (size_t i = threadIdx.x; i < p.wtick_bytes / sizeof(int); i += blockDim.x) p.wtick[i] = 0;
-    __syncthreads();
-    const bool ok = decode_first<FMT>(p, dl, sh, ci, sgrp, ring_base, cache, xs, rs, &s_ok) &&
-                    decode_phase<SP_GATEUP, EF>(p, sh, dl.gu, ci, dl.cache_bytes, ring_base, cache, &ctrl->dec_phase[0], &s_ok) &&
-                    decode_phase<SP_DOWN, EF>(p, sh, dl.dn, ci, dl.cache_bytes, ring_base, cache, &ctrl->dec_phase[1], &s_ok) &&
-                    decode_phase<SP_UPROJ, FMT>(p, sh, dl.u, ci, dl.cache_bytes, ring_base, cache, &ctrl->dec_phase[2], &s_ok);
-    (void)ok;
-    // leave; the last CTA out clears the step's counters
-    __syncthreads();
-    if (threadIdx.x == 0) {
-        __threadfence();
-        if (atomicAdd(&ctrl->dec_exit, 1u) == gridDim.x - 1) {
-            ctrl->dec_rows = 0;
-            ctrl->dec_phase[0] = ctrl->dec_phase[1] = ctrl->dec_phase[2] = 0;
-            ctrl->dec_abort = 0;
-            __threadfence();
-            ctrl->dec_exit = 0;
-        }
-    }
-}
-
-// ---------------------------------------------------------------------------
 // launch helpers
 // ---------------------------------------------------------------------------
 
@@ -1373,100 +1124,3 @@ cudaError_t run_stream_path(const FwdParams& p, cudaStream_t st) {
 
 }  // namespace lmoe
 
-namespace lmoe {
-
-// ---------------------------------------------------------------------------
-// host side of the one-kernel step
-// ---------------------------------------------------------------------------
-
-static int sm_count() {
-    if (!g_sms) {
-        int dev = 0;
-        cudaGetDevice(&dev);
-        cudaDeviceGetAttribute(&g_sms, cudaDevAttrMultiProcessorCount, dev);
-    }
-    return g_sms;
-}
-
-// Cache rows of a phase: the distinct matrices one CTA's contiguous chunk
-// can span, T rows each.
-static int chunk_cache_rows(const WPlan& w, int T) {
-    const int per_mat = w.tiles * w.ks;
-    const int chunk = (w.n_mats * per_mat + sm_count() - 1) / sm_count();
-    const int mats = std::min(w.n_mats, (chunk + per_mat - 1) / per_mat + 1);
-    return std::min(mats, kMaxChunkParts) * T;
-}
-
-typedef void (*DecodeKernel)(FwdParams, DecodeLayout);
-
-// The instance of the one-kernel step for the D/U and expert formats.
-static DecodeKernel decode_kernel(const FwdParams& p) {
-    if (p.du_fmt == LMOE_Q8_0) return p.efmt == kEfQ3k ? k_decode_step<LMOE_Q8_0, kEfQ3k> : k_decode_step<LMOE_Q8_0, kEfNvfp4>;
-    return p.efmt == kEfQ3k ? k_decode_step<LMOE_Q4_0, kEfQ3k> : k_decode_step<LMOE_Q4_0, kEfNvfp4>;
-}
-
-static DecodeLayout decode_layout(const FwdParams& p) {
-    const WPlans P = stream_plans(p.H, p.L, p.F, p.Fs, p.G, p.E, p.K, p.T, p.du_fmt);
-    DecodeLayout dl;
-    dl.d = P.d;
-    dl.gu = P.gu;
-    dl.dn = P.dn;
-    dl.u = P.u;
-    const size_t b_d = (size_t)p.T * (p.H + kActPad) * 2;
-    const size_t b_gu = (size_t)chunk_cache_rows(P.gu, p.T) * (p.L + kActPad) * 2;
-    const size_t b_dn = (size_t)chunk_cache_rows(P.dn, p.T) * (p.F + kActPad) * 2;
-    const size_t b_u = (size_t)chunk_cache_rows(P.u, p.T) * (std::max(p.L, p.Fs) + kActPad) * 2;
-    dl.cache_bytes = round128((int)std::max({b_d, b_gu, b_dn, b_u}));
-    return dl;
-}
-
-static size_t decode_dyn_smem(const FwdParams& p, const DecodeLayout& dl) {
-    const size_t xs = std::max((size_t)xs_ld(p.H) * 4 * sizeof(float), sizeof(TopkScratch));
-    return 128 + (size_t)dl.cache_bytes + (size_t)kWW * kPD * kStepBytes + ((xs + 15) & ~(size_t)15);
-}
-
-// The step fits one kernel when its shared memory does and one CTA per SM
-// can be resident (checked once per kernel and device).
-bool decode_step_fits(const FwdParams& p) {
-    if (p.T < 1 || p.T > 8) return false;
-    const DecodeLayout dl = decode_layout(p);
-    const size_t dyn = decode_dyn_smem(p, dl);
-    int dev = 0, optin = 0;
-    cudaGetDevice(&dev);
-    cudaDeviceGetAttribute(&optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev);
-    const void* k = reinterpret_cast<const void*>(decode_kernel(p));
-    cudaFuncAttributes fa;
-    if (cudaFuncGetAttributes(&fa, k) != cudaSuccess) return false;
-    return fa.sharedSizeBytes + dyn <= (size_t)optin;
-}
-
-cudaError_t run_decode_step(FwdParams p, cudaStream_t st) {
-    p.x16 = nullptr;
-    p.route_smem = true;
-    const DecodeLayout dl = decode_layout(p);
-    const size_t smem = decode_dyn_smem(p, dl);
-    auto kern = decode_kernel(p);
-    cudaError_t e = ensure_smem(reinterpret_cast<const void*>(kern), smem);
-    if (e != cudaSuccess) return e;
-    int per_sm = 0;
-    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, kWThreads, smem);
-    if (e != cudaSuccess) return e;
-    if (per_sm < 1) return cudaErrorInvalidConfiguration;
-    stage_mark(st);
-    cudaLaunchConfig_t cfg;
-    std::memset(&cfg, 0, sizeof(cfg));
-    cfg.gridDim = dim3(sm_count());
-    cfg.blockDim = dim3(kWThreads);
-    cfg.dynamicSmemBytes = smem;
-    cfg.stream = st;
-    cudaLaunchAttribute attr[1];
-    attr[0].id = cudaLaunchAttributeCooperative;
-    attr[0].val.cooperative = 1;
-    cfg.attrs = attr;
-    cfg.numAttrs = 1;
-    e = cudaLaunchKernelEx(&cfg, kern, p, dl);
-    stage_mark(st);
-    return e;
-}
-
-}  // namespace lmoe
