@@ -111,8 +111,7 @@ __global__ void __launch_bounds__(256) k_router_shared(FwdParams p) {
     __threadfence();
     if (p.route_smem) {
         __shared__ StreamShared rsh;
-        // the top-K scratch reuses the staged activations' space
-        route_in_cta(p, rsh, *reinterpret_cast<TopkScratch*>(smem), sgrp, true);
+        route_in_cta(p, rsh, sgrp, true);
     } else {
         topk_and_buckets(p);
     }
@@ -880,7 +879,11 @@ static cudaError_t run_gemv_path_nt(FwdParams p, cudaStream_t st, bool route_onl
     // 1. router (+ shared gate/up, top-k, buckets): one warp per router row / shared feature
     p.router_rows_per_warp = 1;
     p.n_router_ctas = (p.E + 7) / 8;
-    p.do_shared = !route_only;
+    // few tokens, whole block: the routing is built in shared memory (see
+    // below) and the shared expert's gate/up run in the D kernel, so the
+    // router kernel holds only the router rows' SMs
+    p.shared_in_d = !route_only && p.T <= 8;
+    p.do_shared = !route_only && !p.shared_in_d;
     p.do_buckets = !route_only;
     // few tokens, whole block: the routing is built in shared memory and
     // published with every table the weight-streaming kernels read
@@ -888,7 +891,7 @@ static cudaError_t run_gemv_path_nt(FwdParams p, cudaStream_t st, bool route_onl
     // the weight-streaming kernels read the block input themselves
     if (p.route_smem) p.x16 = nullptr;
     p.prefetch_l2 = false;
-    const int n_shared_ctas = route_only ? 0 : (p.Fs + 7) / 8;
+    const int n_shared_ctas = p.do_shared ? (p.Fs + 7) / 8 : 0;
     if (p.route_smem && p.wtick) {
         // tickets of the split reductions of the weight-streaming kernels
         cudaError_t e = cudaMemsetAsync(p.wtick, 0, p.wtick_bytes, st);
@@ -896,7 +899,6 @@ static cudaError_t run_gemv_path_nt(FwdParams p, cudaStream_t st, bool route_onl
     }
     {
         size_t sm = (size_t)xs_ld(p.H) * NT * sizeof(float);
-        if (p.route_smem) sm = std::max(sm, sizeof(TopkScratch));
         cudaError_t e = p.router_bf16
             ? launch(k_router_shared<NT, true>, dim3(p.n_router_ctas + n_shared_ctas), 256, sm, st, p)
             : launch(k_router_shared<NT, false>, dim3(p.n_router_ctas + n_shared_ctas), 256, sm, st, p);

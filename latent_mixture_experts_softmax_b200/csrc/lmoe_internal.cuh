@@ -83,6 +83,7 @@ struct FwdParams {
     // launch shape of the router kernel
     int n_router_ctas, router_rows_per_warp;
     bool do_shared, do_buckets;
+    bool shared_in_d;   // few tokens: the shared expert's gate/up run as items of the D kernel
     bool route_smem;    // few tokens: routing built in shared memory, all tables published
     bool prefetch_l2;   // stream the step's weights into L2 ahead of use (few tokens)
 };

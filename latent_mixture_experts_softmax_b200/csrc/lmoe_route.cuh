@@ -46,90 +46,58 @@ static __device__ __forceinline__ float key_value(uint32_t k) {
     return __uint_as_float((k & 0x80000000u) ? (k & 0x7fffffffu) : ~k);
 }
 
-// Largest of n packed (key, ~index) words, as a tree of comparisons.
-template <int N>
-static __device__ __forceinline__ uint64_t tree_max(const uint64_t (&pk)[N]) {
-    uint64_t m[N];
-#pragma unroll
-    for (int j = 0; j < N; ++j) m[j] = pk[j];
-#pragma unroll
-    for (int w = N / 2; w > 0; w >>= 1) {
-#pragma unroll
-        for (int j = 0; j < w; ++j) m[j] = m[j] > m[j + w] ? m[j] : m[j + w];
-    }
-    return m[0];
-}
-
 static __device__ __forceinline__ uint64_t pack_logit(float l, int e) {
     return ((uint64_t)order_key(l) << 32) | (uint32_t)~e;
 }
 
-// Softmax top-K of one token by one warp (section "Routing" of the teardown
-// article: softmax over the E logits, top-K, renormalise over the kept).
-// A logit is packed as (order key, ~index), so the larger word is the larger
-// logit and, between equal logits, the lower expert index; the words of a
-// row are distinct.
-//  1. Each lane keeps NV words and their maximum.  tau = the K-th largest of
-//     the 32 lane maxima bounds the token's K largest words from below (the
-//     K largest lane maxima are K distinct words, all >= tau).
-//  2. The words >= tau (at most K * NV, typically a few more than K) are
-//     compacted into `cand`; a candidate's rank is the number of larger
-//     candidates, and the K of rank < K are the top K, in order.
-//  3. w_k = exp(l_k - l_1) / sum over the kept of exp(l_j - l_1), the sum
-//     taken in k order.
-// Writes idx[0..K), w[0..K); `cand` holds K * NV words, `sel` K.
+// Softmax top-K of one token by one warp (the router of the model page's
+// "Model profile": softmax over the E logits, top-K, renormalise over the
+// kept).  A logit is packed as (order key, ~index), so the larger word is the
+// larger logit and, between equal logits, the lower expert index; the words
+// of a row are distinct.  Each lane holds NV words; K rounds each take the
+// warp's largest word: the largest order key by a warp max reduction, then
+// the lowest index among the lanes whose own largest word carries that key
+// by a warp min reduction; the owning lane clears that word.  The rounds
+// share one short loop body (this runs once per step, with its instructions
+// fetched cold, so code size counts more than cycles).
+//   w_k = exp(l_k - l_1) / sum over the kept of exp(l_j - l_1), summed in k
+//   order.  Writes idx[0..K), w[0..K).
 template <int NV>
-static __device__ void topk_row(const float* logits, int E, int K, int lane, int* idx, float* w, uint64_t* cand,
-                                uint64_t* sel) {
+static __device__ void topk_row(const float* logits, int E, int K, int lane, int* idx, float* w) {
     uint64_t pk[NV];
 #pragma unroll
     for (int j = 0; j < NV; ++j) {
         const int e = lane + 32 * j;
         pk[j] = e < E ? pack_logit(__ldcg(logits + e), e) : 0ull;
     }
-    const uint64_t lmx = tree_max(pk);
-    int r = 0;
+    float l1 = 0.f, denom = 0.f, my_l = 0.f;
+    int my_e = 0;
+#pragma unroll 1
+    for (int k = 0; k < K; ++k) {
+        uint64_t m = pk[0];
 #pragma unroll
-    for (int l = 0; l < 32; ++l) r += __shfl_sync(0xffffffffu, lmx, l) > lmx;
-    const uint32_t bal = __ballot_sync(0xffffffffu, r == K - 1);
-    const uint64_t tau = __shfl_sync(0xffffffffu, lmx, __ffs(bal) - 1);
-    int c = 0;
+        for (int j = 1; j < NV; ++j) m = pk[j] > m ? pk[j] : m;
+        const uint32_t key = (uint32_t)(m >> 32);
+        const uint32_t kmax = __reduce_max_sync(0xffffffffu, key);
+        const uint32_t e = __reduce_min_sync(0xffffffffu, key == kmax ? ~(uint32_t)m : 0xffffffffu);
+        if ((int)(e & 31) == lane) {
 #pragma unroll
-    for (int j = 0; j < NV; ++j) c += pk[j] >= tau;
-    int pre = c;
-#pragma unroll
-    for (int off = 1; off < 32; off <<= 1) {
-        const int o = __shfl_up_sync(0xffffffffu, pre, off);
-        if (lane >= off) pre += o;
+            for (int j = 0; j < NV; ++j)
+                if (j == (int)(e >> 5)) pk[j] = 0ull;
+        }
+        const float l = key_value(kmax);
+        if (k == 0) l1 = l;
+        denom += expf(l - l1);
+        if (k == lane) {
+            my_l = l;
+            my_e = (int)e;
+        }
     }
-    const int total = __shfl_sync(0xffffffffu, pre, 31);
-    pre -= c;
-#pragma unroll
-    for (int j = 0; j < NV; ++j)
-        if (pk[j] >= tau) cand[pre++] = pk[j];
-    __syncwarp();
-    for (int i = lane; i < total; i += 32) {
-        const uint64_t v = cand[i];
-        int rk = 0;
-        for (int j = 0; j < total; ++j) rk += cand[j] > v;
-        if (rk < K) sel[rk] = v;
-    }
-    __syncwarp();
-    const float lmax = key_value((uint32_t)(sel[0] >> 32));
-    float denom = 0.f;
-    for (int k = 0; k < K; ++k) denom += expf(key_value((uint32_t)(sel[k] >> 32)) - lmax);
     if (lane < K) {
-        const uint64_t v = sel[lane];
-        idx[lane] = (int)~(uint32_t)v;
-        w[lane] = expf(key_value((uint32_t)(v >> 32)) - lmax) / denom;
+        idx[lane] = my_e;
+        w[lane] = expf(my_l - l1) / denom;
     }
 }
-
-// Scratch of the top-K of up to 8 tokens.
-struct TopkScratch {
-    uint64_t cand[8][kMaxTopK * (kMaxExpertsTopk / 32)];
-    uint64_t sel[8][kMaxTopK];
-};
 
 // Bucketing of the T*K pairs by the whole CTA (one pair per thread), in
 // shared memory: slots ordered by (expert, pair index), distinct experts
@@ -164,7 +132,7 @@ static __device__ void bucket_pairs(const FwdParams& p, StreamShared& sh, const 
     for (int i = threadIdx.x; i < n; i += blockDim.x) {
         const int e = sh.pe[i];
         int less = 0, same_before = 0, cnt = 0;
-#pragma unroll 8
+#pragma unroll 2
         for (int j = 0; j < n; ++j) {
             const int ej = sh.pe[j];
             less += ej < e;
@@ -207,8 +175,7 @@ static __device__ void bucket_pairs(const FwdParams& p, StreamShared& sh, const 
 // __syncthreads); `grp` is the expert -> group table in shared memory.
 // With publish, also written to the workspace for the kernels that read it
 // and to the caller's routing outputs.
-static __device__ void route_in_cta(const FwdParams& p, StreamShared& sh, TopkScratch& ts, const uint8_t* grp,
-                                    bool publish) {
+static __device__ void route_in_cta(const FwdParams& p, StreamShared& sh, const uint8_t* grp, bool publish) {
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int T = p.T, K = p.K, E = p.E, G = p.G, n = T * K;
     for (int v = threadIdx.x; v < (E + 31) / 32; v += blockDim.x) sh.emask[v] = 0u;
@@ -223,10 +190,10 @@ static __device__ void route_in_cta(const FwdParams& p, StreamShared& sh, TopkSc
             const float* lg = p.r.logits + (size_t)t * E;
             int* ix = sh.idx + t * K;
             float* wt = sh.w + t * K;
-            if (E <= 128) topk_row<4>(lg, E, K, lane, ix, wt, ts.cand[t], ts.sel[t]);
-            else if (E <= 256) topk_row<8>(lg, E, K, lane, ix, wt, ts.cand[t], ts.sel[t]);
-            else if (E <= 512) topk_row<16>(lg, E, K, lane, ix, wt, ts.cand[t], ts.sel[t]);
-            else topk_row<32>(lg, E, K, lane, ix, wt, ts.cand[t], ts.sel[t]);
+            if (E <= 128) topk_row<4>(lg, E, K, lane, ix, wt);
+            else if (E <= 256) topk_row<8>(lg, E, K, lane, ix, wt);
+            else if (E <= 512) topk_row<16>(lg, E, K, lane, ix, wt);
+            else topk_row<32>(lg, E, K, lane, ix, wt);
         }
     }
     __syncthreads();

@@ -303,11 +303,13 @@ __device__ __forceinline__ void tile_iq4nl(const uint8_t* q, const uint16_t* d, 
 //   gate/up NVFP4:     4 chunks  gate codes [4][16][16], up codes, gate scales [2][16][4], up scales = 2304 B
 //   down NVFP4:        8 chunks  codes [8][16][16] + scales [4][16][4] = 2304 B
 //   U shared bf16:     2 blocks  [16 rows][64] bf16 = 2048 B
+//   D shared gate/up:  1 block   gate [16 rows][32] bf16, then up = 2048 B
 template <int PHASE, int FMT>
 __host__ __device__ __forceinline__ int step_blocks(bool shared_part) {
     if (PHASE == SP_GATEUP) return 4;
     if (PHASE == SP_DOWN) return 8;
     if (PHASE == SP_UPROJ && shared_part) return 2;
+    if (PHASE == SP_DPROJ && shared_part) return 1;
     return FMT == LMOE_Q8_0 ? 4 : 8;
 }
 
@@ -338,6 +340,18 @@ struct WPlan {
 template <int PHASE, int FMT>
 __device__ __forceinline__ WItem decode_item(const FwdParams& p, const StreamShared& sh, const WPlan& pl, int i) {
     WItem it;
+    if (PHASE == SP_DPROJ && i >= p.G * pl.tiles) {
+        // the shared expert's gate and up rows (16 features over the whole
+        // block input), after every group's D items; one 32-column block per step
+        it.mat = -1;
+        it.j = p.G;
+        it.q = 0;
+        it.tile = i - p.G * pl.tiles;
+        it.r0 = it.tile * 16;
+        it.kb0 = 0;
+        it.kb1 = p.H / 32;
+        return it;
+    }
     const int per_mat = pl.tiles * pl.ks;
     const int m = i / per_mat, rem = i - m * per_mat;
     it.q = rem / pl.tiles;
@@ -378,11 +392,18 @@ __device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_gr
 template <int PHASE, int FMT>
 __device__ __forceinline__ void issue_step(const FwdParams& p, const WItem& it, int st, uint8_t* buf, int lane) {
     const int L = p.L, F = p.F, H = p.H, Fs = p.Fs;
-    const bool shared_part = PHASE == SP_UPROJ && it.mat < 0;
+    const bool shared_part = (PHASE == SP_UPROJ || PHASE == SP_DPROJ) && it.mat < 0;
     const int sb = step_blocks<PHASE, FMT>(shared_part);
     const int kb = it.kb0 + st * sb;
     const int nblk = min(sb, it.kb1 - kb);
-    if (PHASE == SP_DPROJ || (PHASE == SP_UPROJ && !shared_part)) {
+    if (PHASE == SP_DPROJ && shared_part) {
+        // gate then up rows r0 .. r0 + 15, columns 32 kb .. + 31 (64 bytes a row)
+        for (int c = lane; c < 128; c += 32) {
+            const int mm = c >> 6, row = (c >> 2) & 15, o = (c & 3) * 16;
+            const uint16_t* src = (mm ? p.su : p.sg) + (size_t)(it.r0 + row) * H + (size_t)kb * 32;
+            cp_async16(buf + (size_t)mm * 1024 + row * 64 + o, reinterpret_cast<const uint8_t*>(src) + o);
+        }
+    } else if (PHASE == SP_DPROJ || (PHASE == SP_UPROJ && !shared_part)) {
         const int qb = FMT == LMOE_Q8_0 ? 32 : 16;
         const int R = PHASE == SP_DPROJ ? L : H;
         const int C = PHASE == SP_DPROJ ? H : L;
@@ -481,12 +502,17 @@ __device__ __forceinline__ void issue_step(const FwdParams& p, const WItem& it, 
 template <int PHASE, int FMT>
 __device__ __forceinline__ void compute_step(const FwdParams& p, const WItem& it, int st, const uint8_t* buf,
                                              const __half* xs, int ld, int nt, float (&a)[4], float (&u)[4]) {
-    const bool shared_part = PHASE == SP_UPROJ && it.mat < 0;
+    const bool shared_part = (PHASE == SP_UPROJ || PHASE == SP_DPROJ) && it.mat < 0;
     const int sb = step_blocks<PHASE, FMT>(shared_part);
     const int kb = it.kb0 + st * sb;
     const int nblk = min(sb, it.kb1 - kb);
     const __half* x = xs + kb * 32;
-    if (PHASE == SP_DPROJ || (PHASE == SP_UPROJ && !shared_part)) {
+    if (PHASE == SP_DPROJ && shared_part) {
+        bool bad = false;
+        tile_bf16(reinterpret_cast<const uint16_t*>(buf), 32, x, ld, nt, 0, 1, a, bad);
+        tile_bf16(reinterpret_cast<const uint16_t*>(buf + 1024), 32, x, ld, nt, 0, 1, u, bad);
+        report_range(p.ctrl, bad);
+    } else if (PHASE == SP_DPROJ || (PHASE == SP_UPROJ && !shared_part)) {
         const int qb = FMT == LMOE_Q8_0 ? 32 : 16;
         tile_du<FMT>(buf, reinterpret_cast<const uint16_t*>(buf + sb * 16 * qb), x, ld, nt, 0, nblk, a);
     } else if (PHASE == SP_UPROJ) {
@@ -558,7 +584,7 @@ __device__ __forceinline__ int phase_mats(const FwdParams& p, const StreamShared
     return PHASE == SP_DPROJ ? p.G : PHASE == SP_UPROJ ? sh.n_hit + 1 : sh.n_unique;
 }
 
-// Thread 0 decides the CTA's chunk and its cache rows (visible to all after
+// Warp 0 decides the CTA's chunk and its cache rows (visible to all after
 // the __syncthreads in here); threads < 4 * nm then fetch the experts'
 // tensor scales (visible after the caller's next __syncthreads).
 template <int PHASE, int FMT>
@@ -566,37 +592,49 @@ __device__ void phase_setup(const FwdParams& p, const StreamShared& sh, const WP
                             ChunkInfo& ci) {
     const int T = p.T, G = p.G;
     const int ld = cache_ld<PHASE>(p.H, p.L, p.F, p.Fs);
-    if (threadIdx.x == 0) {
-        const int n_items = phase_mats<PHASE>(p, sh) * plan.tiles * plan.ks;
+    if (threadIdx.x < 32) {
+        // warp 0: every lane computes the chunk; lane jj lays out the cache
+        // rows of the chunk's matrix jj (at most T rows each)
+        const int lane = threadIdx.x;
+        const int n_items = phase_mats<PHASE>(p, sh) * plan.tiles * plan.ks +
+                            (PHASE == SP_DPROJ && p.shared_in_d ? p.Fs / 16 : 0);
         const int per_mat = plan.tiles * plan.ks;
         const int i0 = chunk_begin(blockIdx.x, n_items, gridDim.x);
         const int i1 = chunk_begin(blockIdx.x + 1, n_items, gridDim.x);
         const int m0 = i0 / per_mat, m1 = i0 < i1 ? (i1 - 1) / per_mat : m0 - 1;
         const int nm = PHASE == SP_DPROJ ? 1 : m1 - m0 + 1;
-        int rows = 0;
-        bool fits = nm <= kMaxChunkParts;
-        for (int jj = 0; fits && jj < nm; ++jj) {
-            const int m = m0 + jj;
-            ci.row0[jj] = rows;
-            const int nr = (PHASE == SP_GATEUP || PHASE == SP_DOWN) ? sh.ucnt[m] : T;
-            if (rows + nr > kMaxChunkParts * 8) { fits = false; break; }
-            for (int c = 0; c < nr; ++c, ++rows) {
+        const int m = m0 + lane;
+        const bool act = lane < nm && lane < kMaxChunkParts;
+        const int nr = act ? ((PHASE == SP_GATEUP || PHASE == SP_DOWN) ? sh.ucnt[m] : T) : 0;
+        int pre = nr;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const int v = __shfl_up_sync(0xffffffffu, pre, o);
+            if (lane >= o) pre += v;
+        }
+        const int rows = __shfl_sync(0xffffffffu, pre, 31);
+        const bool fits = nm <= kMaxChunkParts && rows <= kMaxChunkParts * 8 && (size_t)rows * ld * 2 <= (size_t)cache_bytes;
+        if (act && fits) {
+            const int r0 = pre - nr;
+            ci.row0[lane] = r0;
+            for (int c = 0; c < nr; ++c) {
                 int src;
                 if (PHASE == SP_DPROJ) src = c;                                                     // x row
                 else if (PHASE == SP_GATEUP) src = sh.slot_tok[sh.uoff[m] + c] * G + sh.ugrp[m];  // h16 row
                 else if (PHASE == SP_DOWN) src = sh.uoff[m] + c;                                    // z16 row
                 else src = m < sh.n_hit ? sh.hg[m] * T + c : -1 - c;                               // s[g][t] / shared hidden
-                ci.src[rows] = src;
+                ci.src[r0 + c] = src;
             }
         }
-        fits = fits && (size_t)rows * ld * 2 <= (size_t)cache_bytes;
-        if (!fits) set_status(p.ctrl, LMOE_ERR_UNSUPPORTED);
-        ci.i0 = i0;
-        ci.i1 = fits ? i1 : i0;
-        ci.m0 = m0;
-        ci.nm = fits ? nm : 0;
-        ci.rows = fits ? rows : 0;
-        ci.skip = !fits;
+        if (lane == 0) {
+            if (!fits) set_status(p.ctrl, LMOE_ERR_UNSUPPORTED);
+            ci.i0 = i0;
+            ci.i1 = fits ? i1 : i0;
+            ci.m0 = m0;
+            ci.nm = fits ? nm : 0;
+            ci.rows = fits ? rows : 0;
+            ci.skip = !fits;
+        }
     }
     __syncthreads();
     if ((PHASE == SP_GATEUP || PHASE == SP_DOWN) && threadIdx.x < 4 * ci.nm) {
@@ -622,7 +660,8 @@ __device__ __forceinline__ StepMap step_map(const FwdParams& p, const StreamShar
         m.nsB = (p.Fs / 32 + sbs - 1) / sbs;
     } else {
         m.nA = pl.n_mats * pl.tiles;
-        m.nsB = m.nsA;
+        // D's shared-expert items: one 32-column block per step
+        m.nsB = PHASE == SP_DPROJ ? p.H / 32 : m.nsA;
     }
     return m;
 }
@@ -818,7 +857,9 @@ __device__ __forceinline__ void item_finish(const FwdParams& p, const StreamShar
         for (int i4 = 0; i4 < 4; ++i4) {
             const int col = 2 * tt + (i4 & 1), row = cit.r0 + gg + 8 * (i4 >> 1);
             if (col >= nt) continue;
-            if (PHASE == SP_DPROJ) {
+            if (PHASE == SP_DPROJ && cit.mat < 0) {
+                p.zsh16[(size_t)col * p.Fs + row] = half_checked(silu(a[i4]) * u[i4], bad);
+            } else if (PHASE == SP_DPROJ) {
                 p.h16[((size_t)col * G + cit.mat) * L + row] = half_checked(a[i4], bad);
             } else if (PHASE == SP_GATEUP) {
                 p.z16[(size_t)(sh.uoff[cit.j] + col) * F + row] = half_checked(silu(a[i4] * ts[0]) * (u[i4] * ts[1]), bad);
@@ -887,13 +928,14 @@ __device__ void phase_run(const FwdParams& p, const StreamShared& sh, const WPla
     cp_async_wait<0>();
     __syncwarp();
     float* part = reinterpret_cast<float*>(ring);
+    constexpr bool kTwoSums = PHASE == SP_GATEUP || PHASE == SP_DPROJ;   // gate and up (D: shared expert)
     if (first_cut) {
         *reinterpret_cast<float4*>(part + lane * 8) = make_float4(ha[0], ha[1], ha[2], ha[3]);
-        if (PHASE == SP_GATEUP) *reinterpret_cast<float4*>(part + lane * 8 + 4) = make_float4(hu[0], hu[1], hu[2], hu[3]);
+        if (kTwoSums) *reinterpret_cast<float4*>(part + lane * 8 + 4) = make_float4(hu[0], hu[1], hu[2], hu[3]);
     }
     if (last_cut) {
         *reinterpret_cast<float4*>(part + 256 + lane * 8) = make_float4(a[0], a[1], a[2], a[3]);
-        if (PHASE == SP_GATEUP) *reinterpret_cast<float4*>(part + 256 + lane * 8 + 4) = make_float4(u[0], u[1], u[2], u[3]);
+        if (kTwoSums) *reinterpret_cast<float4*>(part + 256 + lane * 8 + 4) = make_float4(u[0], u[1], u[2], u[3]);
     }
     __syncthreads();
     if (last_cut) {
@@ -906,7 +948,7 @@ __device__ void phase_run(const FwdParams& p, const StreamShared& sh, const WPla
             const float* q = reinterpret_cast<const float*>(ring_base + (size_t)w * kPD * kStepBytes) + lane * 8;
             const float4 v = *reinterpret_cast<const float4*>(q);
             a[0] += v.x; a[1] += v.y; a[2] += v.z; a[3] += v.w;
-            if (PHASE == SP_GATEUP) {
+            if (kTwoSums) {
                 const float4 w4 = *reinterpret_cast<const float4*>(q + 4);
                 u[0] += w4.x; u[1] += w4.y; u[2] += w4.z; u[3] += w4.w;
             }
