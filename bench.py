@@ -130,12 +130,9 @@ def step_cost(shape, idx: np.ndarray, groups: np.ndarray, T: int, prefill: bool)
     hit = {int(groups[e]) for e in idx.reshape(-1)}
     distinct = set(idx.reshape(-1).tolist())
     pairs_tg = sum(len({int(groups[e]) for e in idx[t]}) for t in range(idx.shape[0]))   # hit (token, group) pairs
-    # up to 8 tokens the shared expert's gate/up rows are read by the D kernel,
-    # from 9 to 63 tokens by the router kernel
-    sh_gu = 2 * Fs * H * 2
     b = {
-        "k_router_shared": rw + T * H * 2 + (0 if T <= 8 else sh_gu),
-        "k_wstream_dproj": G * du + T * H * 2 + (sh_gu if T <= 8 else 0),   # every group (D runs before the routing)
+        "k_router_shared": rw + 2 * Fs * H * 2 + T * H * 2,
+        "k_wstream_dproj": G * du + T * H * 2,     # every group (D runs before the routing is known)
         "k_wstream_gateup": len(distinct) * rec_gu,
         "k_wstream_down": len(distinct) * rec_d,
         "k_wstream_uproj": len(hit) * du + H * Fs * 2 + 2 * T * H * 2,

@@ -879,11 +879,11 @@ static cudaError_t run_gemv_path_nt(FwdParams p, cudaStream_t st, bool route_onl
     // 1. router (+ shared gate/up, top-k, buckets): one warp per router row / shared feature
     p.router_rows_per_warp = 1;
     p.n_router_ctas = (p.E + 7) / 8;
-    // few tokens, whole block: the routing is built in shared memory (see
-    // below) and the shared expert's gate/up run in the D kernel, so the
-    // router kernel holds only the router rows' SMs
-    p.shared_in_d = !route_only && p.T <= 8;
-    p.do_shared = !route_only && !p.shared_in_d;
+    // the shared expert's gate/up run in the router kernel's other CTAs (as
+    // items of the D kernel, whose items are split by count, their 80-step
+    // items left a few CTAs four times the work of the rest)
+    p.shared_in_d = false;
+    p.do_shared = !route_only;
     p.do_buckets = !route_only;
     // few tokens, whole block: the routing is built in shared memory and
     // published with every table the weight-streaming kernels read

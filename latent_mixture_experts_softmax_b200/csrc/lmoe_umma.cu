@@ -211,6 +211,16 @@ __device__ __forceinline__ void bulk_g2s(void* dst, const void* src, uint32_t by
                  : "memory");
 }
 
+__device__ __forceinline__ void cp_async16_sh(void* dst, const void* src) {
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_u32(dst)), "l"(src) : "memory");
+}
+__device__ __forceinline__ void cp_async4_sh(void* dst, const void* src) {
+    asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(smem_u32(dst)), "l"(src) : "memory");
+}
+__device__ __forceinline__ void cp_async_commit_grp() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+template <int N>
+__device__ __forceinline__ void cp_async_wait_grp() { asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory"); }
+
 __device__ __forceinline__ uint32_t h2_bits(__half2 h) { return *reinterpret_cast<uint32_t*>(&h); }
 __device__ __forceinline__ __half2 bits_h2(uint32_t u) { return *reinterpret_cast<__half2*>(&u); }
 
@@ -276,6 +286,22 @@ __device__ __forceinline__ void fetch_raw(const PrefillParams& p, const Cursor<K
         o.a = __ldg(reinterpret_cast<const uint4*>(rec + (size_t)m * nq + ((size_t)(k0 / 32 + h) * R + row) * 16));
         o.s = __ldg(reinterpret_cast<const uint32_t*>(rec + 3 * nq + (size_t)m * ns + ((size_t)(k0 / 64) * R + row) * 4));
     }
+}
+
+// The NVFP4 expert bytes of (row r, half h) of the cursor's stage, copied
+// into this thread's ring slot: 16 code bytes at slot[0, 16), the row's
+// 4-byte scale word at slot[16, 20).
+template <int KIND, int NT>
+__device__ __forceinline__ void fetch_raw_async(const PrefillParams& p, const Cursor<KIND, NT>& c, int r, int h,
+                                                uint8_t* slot) {
+    const int k0 = c.ks * 64;
+    const size_t nq = (size_t)p.L * p.F / 2, ns = (size_t)p.L * p.F / 16;
+    const uint8_t* rec = p.experts + (size_t)c.t.mat * p.rec_bytes;
+    const int R = KIND == G_GATEUP ? p.F : p.L;
+    const int row = KIND == G_GATEUP ? c.t.m0 + (r & 63) : c.t.m0 + r;
+    const int m = KIND == G_GATEUP ? (r >> 6) : 2;                  // gate, up, down
+    cp_async16_sh(slot, rec + (size_t)m * nq + ((size_t)(k0 / 32 + h) * R + row) * 16);
+    cp_async4_sh(slot + 16, rec + 3 * nq + (size_t)m * ns + ((size_t)(k0 / 64) * R + row) * 4);
 }
 
 // RawHalf of (row r, half h) -> 16 half2 of the row's 32 columns.
@@ -477,10 +503,12 @@ template <int NT, int STAGES, int RS>
 struct SmemPlan {
     static constexpr int kA = 128 * 128;                 // bytes per A stage (128 rows x 64 x 16-bit)
     static constexpr int kB = NT * 128;                  // bytes per B stage
-    static constexpr int kRaw = 8704;                    // bytes per raw weight slot (largest format)
+    // a stage of the converters' ring of stored expert bytes: 32 bytes for
+    // each of the 256 converter threads (16 code bytes, the 4-byte scale word)
+    static constexpr int kRaw = 256 * 32;
     // gate/up exchange (32 x 64 fp32) or a tile's routing metadata (NT x (1 + 16) words)
     static constexpr int kXchg = (32 * 64 * 4 > NT * 4 * 17) ? 32 * 64 * 4 : NT * 4 * 17;
-    static constexpr int kBars = (3 * STAGES + 2 * RS + 5) * 8;
+    static constexpr int kBars = (3 * STAGES + 5) * 8;
     static constexpr int kTotal = 1024 /*alignment slack*/ + STAGES * (kA + kB) + RS * kRaw + kXchg + kBars + 16;
 };
 
@@ -504,9 +532,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1) k_umma_gemm(const __grid_cons
     uint64_t* full_a = bars;
     uint64_t* full_b = bars + STAGES;
     uint64_t* empty = bars + 2 * STAGES;
-    uint64_t* raw_full = bars + 3 * STAGES;
-    uint64_t* raw_empty = raw_full + RS;
-    uint64_t* tfull = raw_empty + RS;
+    uint64_t* tfull = bars + 3 * STAGES;
     uint64_t* tempty = tfull + 2;
     uint64_t* final_bar = tempty + 2;
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(final_bar + 1);
@@ -521,10 +547,6 @@ __global__ void __launch_bounds__(kGemmThreads, 1) k_umma_gemm(const __grid_cons
             mbar_init(&full_a[s], kConvWarps);
             mbar_init(&full_b[s], 1);
             mbar_init(&empty[s], 1);
-        }
-        for (int s = 0; s < RS; ++s) {
-            mbar_init(&raw_full[s], 1);
-            mbar_init(&raw_empty[s], kConvWarps);
         }
         for (int a = 0; a < 2; ++a) {
             mbar_init(&tfull[a], 1);
@@ -586,13 +608,52 @@ __global__ void __launch_bounds__(kGemmThreads, 1) k_umma_gemm(const __grid_cons
         __syncwarp();
     } else if (warp >= 4 && warp < 12) {
         // ------------------------------------------------------------ converters
-        // Each thread owns half a weight row of every stage; its stored bytes
-        // are fetched with plain loads kRawAhead - 1 stages ahead of use.
+        // Each thread owns half a weight row of every stage.  NVFP4 expert
+        // weights come through a ring of RS stages in shared memory filled
+        // by the thread's own cp.async copies (deep enough to keep the loads
+        // of the stored bytes in flight); the other formats are fetched with
+        // plain loads kRawAhead - 1 stages ahead of use.
         const int r = (threadIdx.x - 128) & 127;   // A row
         const int hh = (threadIdx.x - 128) >> 7;   // half of the 64 columns
         Cursor<KIND, NT> cur, cf;
         cur.begin(p);
         cf = cur;
+        if (RS > 0 && (KIND == G_GATEUP || KIND == G_DOWN) && p.efmt == LMOE_EXPERTS_NVFP4) {
+            uint8_t* ring = sRaw + (size_t)(threadIdx.x - 128) * 32;       // + stage * Plan::kRaw
+#pragma unroll 1
+            for (int k = 0; k < RS - 1; ++k) {
+                if (!cf.done) {
+                    fetch_raw_async<KIND, NT>(p, cf, r, hh, ring + (size_t)k * Plan::kRaw);
+                    cf.next_stage(p);
+                }
+                cp_async_commit_grp();
+            }
+            uint32_t it = 0;
+            while (!cur.done) {
+                if (!cf.done) {
+                    fetch_raw_async<KIND, NT>(p, cf, r, hh, ring + (size_t)((it + RS - 1) % RS) * Plan::kRaw);
+                    cf.next_stage(p);
+                }
+                cp_async_commit_grp();
+                const int s = it % STAGES;
+                const uint32_t ph = (it / STAGES) & 1;
+                if (!mbar_wait(&empty[s], ph ^ 1, abort_flag, kWaitLimit)) break;
+                cp_async_wait_grp<RS - 1>();
+                const uint8_t* slot = ring + (size_t)(it % RS) * Plan::kRaw;
+                RawHalf raw;
+                raw.a = *reinterpret_cast<const uint4*>(slot);
+                raw.s = *reinterpret_cast<const uint32_t*>(slot + 16);
+                uint32_t o[16];
+                dequant_half<KIND>(p, raw, hh, o);
+                store_half_swizzled(sA + s * Plan::kA, r, hh, o);
+                fence_proxy_async_smem();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&full_a[s]);
+                cur.next_stage(p);
+                ++it;
+            }
+            cp_async_wait_grp<0>();
+        } else {
         RawHalf raw[kRawAhead];
 #pragma unroll
         for (int k = 0; k < kRawAhead - 1; ++k) {
@@ -623,6 +684,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1) k_umma_gemm(const __grid_cons
             for (int k = 0; k + 1 < kRawAhead; ++k) raw[k] = raw[k + 1];
             cur.next_stage(p);
             ++it;
+        }
         }
     } else if (warp == 12) {
         // ------------------------------------------------------------ MMA issuer
@@ -1060,9 +1122,9 @@ cudaError_t run_prefill_path(PrefillParams p, cudaStream_t st, void* memset_base
     if ((e = launch_gemm<G_DPROJ, kNtDense, 4, 0>(m_d, p, st, G * (L / 128) * ttiles)) != cudaSuccess) return e;
     mark(st);
     const int max_etiles = min(E, pairs) + pairs / kNtExpert + 1;
-    if ((e = launch_gemm<G_GATEUP, kNtExpert, 6, 0>(m_gu, p, st, (F / 64) * max_etiles)) != cudaSuccess) return e;
+    if ((e = launch_gemm<G_GATEUP, kNtExpert, 4, 8>(m_gu, p, st, (F / 64) * max_etiles)) != cudaSuccess) return e;
     mark(st);
-    if ((e = launch_gemm<G_DOWN, kNtExpert, 6, 0>(m_down, p, st, (L / 128) * max_etiles)) != cudaSuccess) return e;
+    if ((e = launch_gemm<G_DOWN, kNtExpert, 4, 8>(m_down, p, st, (L / 128) * max_etiles)) != cudaSuccess) return e;
     mark(st);
     k_combine<<<T, 256, 0, st>>>(p);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
