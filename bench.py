@@ -168,7 +168,13 @@ def step_cost(shape, idx: np.ndarray, groups: np.ndarray, T: int, prefill: bool)
 # whose hash is given (cold caches, one launch), by (workload, T, kernel).
 # When the sources have changed since the capture, or the kernel has no
 # capture, its traffic is reported as null.
-NCU_TRAFFIC = {}
+NCU_TRAFFIC = {
+    ("edge0_145b_decode", 4, "k_router_shared"): (9280000, "c93e26cfd6b4"),
+    ("edge0_145b_decode", 4, "k_wstream_dproj"): (39070000, "c93e26cfd6b4"),
+    ("edge0_145b_decode", 4, "k_wstream_gateup"): (42850000, "c93e26cfd6b4"),
+    ("edge0_145b_decode", 4, "k_wstream_down"): (21390000, "c93e26cfd6b4"),
+    ("edge0_145b_decode", 4, "k_wstream_uproj"): (43960000, "c93e26cfd6b4"),
+}
 
 
 def cuda_source_hash() -> str:
