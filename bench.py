@@ -141,7 +141,8 @@ def step_cost(shape, idx: np.ndarray, groups: np.ndarray, T: int, prefill: bool)
     b_total = float(sum(b.values()) - (G - len(hit)) * du)
     # the 9-63-token kernels read the same bytes per pass of 8 tokens
     for a, c in (("k_dproj_mma", "k_wstream_dproj"), ("k_gateup_mma", "k_wstream_gateup"),
-                 ("k_down_mma", "k_wstream_down"), ("k_uproj_mma", "k_wstream_uproj")):
+                 ("k_down_mma", "k_wstream_down"), ("k_uproj_mma", "k_wstream_uproj"),
+                 ("k_nvf4_gateup", "k_wstream_gateup"), ("k_nvf4_down", "k_wstream_down")):
         b[a] = b[c]
     f = {
         "x_to_fp16": 0.0,
@@ -197,11 +198,23 @@ def ncu_traffic(workload: str, T: int, kernel: str):
     return e[0]
 
 
-def decode_stages(T: int):
-    """Kernels of one few-token step (NVFP4 experts): the router kernel and
-    four weight-streaming kernels up to 8 tokens, the passes-of-8 kernels
-    from 9 to 63."""
+def tensor_core_experts(shape, T: int) -> bool:
+    """Whether the library runs the few-token NVFP4 expert phases on the
+    tensor cores (kind::mxf4nvf4): LMOE_FEW_TOKEN_EXPERTS=tensor_cores, at
+    most 8 tokens, ffn and latent multiples of 128 up to 2048 (the rule
+    stated in include/lmoe.h)."""
+    L, F = shape.latent, shape.ffn
+    return (shape.expert_fmt == "nvfp4" and 1 <= T <= 8 and L % 128 == 0 and F % 128 == 0 and L <= 2048
+            and F <= 2048 and os.environ.get("LMOE_FEW_TOKEN_EXPERTS") == "tensor_cores")
+
+
+def decode_stages(T: int, shape=None):
+    """Kernels of one few-token step: the router kernel and four
+    weight-streaming kernels up to 8 tokens (NVFP4 gate/up and down on the
+    tensor cores where they can), the passes-of-8 kernels from 9 to 63."""
     if T <= 8:
+        if shape is not None and tensor_core_experts(shape, T):
+            return ["k_router_shared", "k_wstream_dproj", "k_nvf4_gateup", "k_nvf4_down", "k_wstream_uproj"]
         return ["k_router_shared", "k_wstream_dproj", "k_wstream_gateup", "k_wstream_down", "k_wstream_uproj"]
     return ["k_router_shared", "k_dproj_mma", "k_gateup_mma", "k_down_mma", "k_uproj_mma"]
 
@@ -453,7 +466,7 @@ def measure_layer(args, wl, T, K, W, rank, world, local, dev_name, ctx=None, lig
     s = wl.shape
     ws = base.workspace(T)
     prefill = T >= 64 and s.router_dtype == "bf16" and s.n_experts % 128 == 0
-    stages = PREFILL_STAGES if prefill else decode_stages(T)
+    stages = PREFILL_STAGES if prefill else decode_stages(T, s)
     # one CUDA graph per distinct step (its own token batch, weight copy and
     # output buffers); the timed loop replays them in turn
     n_graphs = min(K, 8 if prefill else 64)
@@ -576,8 +589,13 @@ def measure_layer(args, wl, T, K, W, rank, world, local, dev_name, ctx=None, lig
                    "weights": "NVFP4 experts, Q8_0/Q4_0 D/U, bf16 router and shared expert; "
                               "bf16 activations in and out, fp32 accumulation",
                    "path": ("tensor cores (tcgen05): fp16 operands dequantised from the stored formats"
-                            if prefill else "router kernel + four weight-streaming kernels (mma.sync, fp16 "
-                                            "operands, fp32 accumulation), programmatic dependent launch"),
+                            if prefill else
+                            ("router kernel, D and U weight-streaming kernels (mma.sync, fp16 operands), NVFP4 "
+                             "gate/up and down on the tensor cores as stored (tcgen05 kind::mxf4nvf4, "
+                             "activations as six E2M1 terms), fp32 accumulation, programmatic dependent launch"
+                             if tensor_core_experts(s, T) else
+                             "router kernel + four weight-streaming kernels (mma.sync, fp16 operands, fp32 "
+                             "accumulation), programmatic dependent launch")),
                    "timing": f"{n_graphs} captured CUDA graphs replayed in turn"},
         "roofline": roof,
         "layer": {"gbs": step_alg_bytes / t_step / 1e9, "tflops": step_flops / t_step / 1e12,

@@ -95,6 +95,12 @@ cudaError_t run_stream_path(const FwdParams& p, cudaStream_t st);
 // workspace of the few-token path's split reductions, for up to T tokens
 size_t stream_ws_part_bytes(int H, int L, int F, int Fs, int G, int E, int K, int T, int du_fmt);
 size_t stream_ws_tick_bytes(int H, int L, int F, int Fs, int G, int E, int K, int T, int du_fmt);
+// Few-token expert phases on the tensor cores (kind::mxf4nvf4): whether a
+// step can take them, the workspace floats of their partial sums, launches.
+bool nvf4_usable(const FwdParams& p);
+size_t nvf4_part_floats();
+cudaError_t run_nvf4_gateup(const FwdParams& p, cudaStream_t st);
+cudaError_t run_nvf4_down(const FwdParams& p, cudaStream_t st);
 void set_stage_events(void* const* events, int n);
 void stage_mark(cudaStream_t st);
 void stage_reset();

@@ -191,9 +191,11 @@ __device__ __forceinline__ void tmem_ld_wait() { asm volatile("tcgen05.wait::ld.
 __device__ __forceinline__ void grid_dep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
 __device__ __forceinline__ void grid_dep_launch() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
 
-// Named barrier among `count` threads (id 1..15; 0 is __syncthreads).
+// Named barrier among `count` threads (id 1..15; 0 is __syncthreads).  The
+// non-aligned form: the threads of a warp may arrive from divergent paths
+// (bar.sync is the .aligned form, which requires them to arrive together).
 __device__ __forceinline__ void named_bar_sync(int id, int count) {
-    asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(count) : "memory");
+    asm volatile("barrier.sync %0, %1;" ::"r"(id), "r"(count) : "memory");
 }
 
 }  // namespace sm100

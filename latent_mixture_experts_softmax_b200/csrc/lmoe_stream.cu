@@ -26,7 +26,9 @@
 // per-group D/U); Edge0 145B / 120B model page, architecture tables.
 
 #include <algorithm>
+#include <cstdlib>
 #include <cstring>
+
 
 #include "lmoe_internal.cuh"
 #include "lmoe_q3k.cuh"
@@ -1099,7 +1101,7 @@ WPlans stream_plans(int H, int L, int F, int Fs, int G, int E, int K, int T, int
     P.dn = plan_for<SP_DOWN, LMOE_Q8_0>(H, L, F, Fs, G, nu);
     // partials (8 floats per lane, 32 lanes) and tickets, the largest phase
     auto parts = [](const WPlan& w) { return (size_t)w.n_mats * w.tiles * w.ks; };
-    P.part_floats = 256 * std::max({parts(P.d), parts(P.gu), parts(P.dn), parts(P.u)});
+    P.part_floats = std::max(256 * std::max({parts(P.d), parts(P.gu), parts(P.dn), parts(P.u)}), nvf4_part_floats());
     P.ticks = std::max({(size_t)P.d.n_mats * P.d.tiles, (size_t)P.gu.n_mats * P.gu.tiles, (size_t)P.dn.n_mats * P.dn.tiles,
                         (size_t)P.u.tiles});
     return P;
@@ -1134,6 +1136,16 @@ static cudaError_t launch_wstream(const FwdParams& p, const WPlan& plan, int cac
     return launch_dependent(kern, dim3(grid), dim3(kWThreads), smem, st, p, plan, cache_bytes);
 }
 
+// LMOE_FEW_TOKEN_EXPERTS selects the few-token NVFP4 expert phases:
+// "tensor_cores" runs them on the tensor-core kernels (kind::mxf4nvf4, the
+// weights as stored); anything else (the default) on the weight-streaming
+// kernels (mma.sync, weights dequantised in registers), which measure
+// faster on the Edge0 shapes.  Read at every call.
+static bool tensor_core_experts() {
+    const char* s = std::getenv("LMOE_FEW_TOKEN_EXPERTS");
+    return s && std::strcmp(s, "tensor_cores") == 0;
+}
+
 // D, experts, combine, U for T <= 8 (the router kernel has run).
 cudaError_t run_stream_path(const FwdParams& p, cudaStream_t st) {
     const int H = p.H, L = p.L, F = p.F, Fs = p.Fs, G = p.G, T = p.T;
@@ -1153,12 +1165,18 @@ cudaError_t run_stream_path(const FwdParams& p, cudaStream_t st) {
     cudaError_t e = p.du_fmt == LMOE_Q8_0 ? launch_wstream<SP_DPROJ, LMOE_Q8_0>(p, P.d, T, st)
                               : launch_wstream<SP_DPROJ, LMOE_Q4_0>(p, P.d, T, st);
     if (e != cudaSuccess) return e;
-    e = p.efmt == kEfQ3k ? launch_wstream<SP_GATEUP, kEfQ3k>(p, P.gu, chunk_rows(P.gu), st)
-                         : launch_wstream<SP_GATEUP, kEfNvfp4>(p, P.gu, chunk_rows(P.gu), st);
-    if (e != cudaSuccess) return e;
-    e = p.efmt == kEfQ3k ? launch_wstream<SP_DOWN, kEfQ3k>(p, P.dn, chunk_rows(P.dn), st)
-                         : launch_wstream<SP_DOWN, kEfNvfp4>(p, P.dn, chunk_rows(P.dn), st);
-    if (e != cudaSuccess) return e;
+    if (nvf4_usable(p) && tensor_core_experts()) {
+        // NVFP4 experts on the tensor cores, weights as stored
+        if ((e = run_nvf4_gateup(p, st)) != cudaSuccess) return e;
+        if ((e = run_nvf4_down(p, st)) != cudaSuccess) return e;
+    } else {
+        e = p.efmt == kEfQ3k ? launch_wstream<SP_GATEUP, kEfQ3k>(p, P.gu, chunk_rows(P.gu), st)
+                             : launch_wstream<SP_GATEUP, kEfNvfp4>(p, P.gu, chunk_rows(P.gu), st);
+        if (e != cudaSuccess) return e;
+        e = p.efmt == kEfQ3k ? launch_wstream<SP_DOWN, kEfQ3k>(p, P.dn, chunk_rows(P.dn), st)
+                             : launch_wstream<SP_DOWN, kEfNvfp4>(p, P.dn, chunk_rows(P.dn), st);
+        if (e != cudaSuccess) return e;
+    }
     e = p.du_fmt == LMOE_Q8_0 ? launch_wstream<SP_UPROJ, LMOE_Q8_0>(p, P.u, chunk_rows(P.u), st)
                               : launch_wstream<SP_UPROJ, LMOE_Q4_0>(p, P.u, chunk_rows(P.u), st);
     return e;

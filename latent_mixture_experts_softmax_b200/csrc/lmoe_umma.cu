@@ -557,10 +557,12 @@ __global__ void __launch_bounds__(kGemmThreads, 1) k_umma_gemm(const __grid_cons
         fence_barrier_init();
     }
     if (warp == 12) {
+        __syncwarp();
         tmem_alloc(tmem_slot, kTmemCols);
         tmem_relinquish();
     }
     tc_fence_before();
+    __syncwarp();
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem_base = *tmem_slot;
@@ -619,9 +621,10 @@ __global__ void __launch_bounds__(kGemmThreads, 1) k_umma_gemm(const __grid_cons
         cur.begin(p);
         cf = cur;
         if (RS > 0 && (KIND == G_GATEUP || KIND == G_DOWN) && p.efmt == LMOE_EXPERTS_NVFP4) {
+            constexpr int kRS = RS > 0 ? RS : 1;
             uint8_t* ring = sRaw + (size_t)(threadIdx.x - 128) * 32;       // + stage * Plan::kRaw
 #pragma unroll 1
-            for (int k = 0; k < RS - 1; ++k) {
+            for (int k = 0; k < kRS - 1; ++k) {
                 if (!cf.done) {
                     fetch_raw_async<KIND, NT>(p, cf, r, hh, ring + (size_t)k * Plan::kRaw);
                     cf.next_stage(p);
@@ -631,15 +634,15 @@ __global__ void __launch_bounds__(kGemmThreads, 1) k_umma_gemm(const __grid_cons
             uint32_t it = 0;
             while (!cur.done) {
                 if (!cf.done) {
-                    fetch_raw_async<KIND, NT>(p, cf, r, hh, ring + (size_t)((it + RS - 1) % RS) * Plan::kRaw);
+                    fetch_raw_async<KIND, NT>(p, cf, r, hh, ring + (size_t)((it + kRS - 1) % kRS) * Plan::kRaw);
                     cf.next_stage(p);
                 }
                 cp_async_commit_grp();
                 const int s = it % STAGES;
                 const uint32_t ph = (it / STAGES) & 1;
                 if (!mbar_wait(&empty[s], ph ^ 1, abort_flag, kWaitLimit)) break;
-                cp_async_wait_grp<RS - 1>();
-                const uint8_t* slot = ring + (size_t)(it % RS) * Plan::kRaw;
+                cp_async_wait_grp<kRS - 1>();
+                const uint8_t* slot = ring + (size_t)(it % kRS) * Plan::kRaw;
                 RawHalf raw;
                 raw.a = *reinterpret_cast<const uint4*>(slot);
                 raw.s = *reinterpret_cast<const uint32_t*>(slot + 16);
@@ -737,9 +740,14 @@ __global__ void __launch_bounds__(kGemmThreads, 1) k_umma_gemm(const __grid_cons
         __syncwarp();
     } else {
         // ------------------------------------------------------------ epilogue
+        // Every epilogue warp walks every tile and reaches every named
+        // barrier; after a timeout (dead) the work is skipped.  The TMEM
+        // loads are warp-collective, so the wait's outcome is made
+        // warp-uniform and the warp converges before each load.
         Cursor<KIND, NT> cur;
         cur.begin(p);
         uint32_t tcount = 0;
+        bool dead = false;
         while (!cur.done) {
             const int acc = tcount & 1;
             const uint32_t ph = (tcount >> 1) & 1;
@@ -781,18 +789,22 @@ __global__ void __launch_bounds__(kGemmThreads, 1) k_umma_gemm(const __grid_cons
                 tscale[threadIdx.x] = 1.f;
             }
             named_bar_sync(1, 128);
-            if (!mbar_wait(&tfull[acc], ph, abort_flag, kWaitLimit)) break;
-            tc_fence_after();
-            const uint32_t taddr = tmem_base + ((uint32_t)(32 * warp) << 16) + acc * NT;
-            for (int c0 = 0; c0 < cur.t.n; c0 += 32) {
-                uint32_t rr[32];
-                tmem_ld_32x32b_x32(taddr + c0, rr);
-                tmem_ld_wait();
-                epilogue_chunk<KIND, NT>(p, cur.t, warp, lane, c0, rr, xchg, tscale);
+            if (!dead) dead = !mbar_wait(&tfull[acc], ph, abort_flag, kWaitLimit);
+            dead = __any_sync(0xffffffffu, dead);
+            if (!dead) {
+                tc_fence_after();
+                const uint32_t taddr = tmem_base + ((uint32_t)(32 * warp) << 16) + acc * NT;
+                for (int c0 = 0; c0 < cur.t.n; c0 += 32) {
+                    uint32_t rr[32];
+                    __syncwarp();
+                    tmem_ld_32x32b_x32(taddr + c0, rr);
+                    tmem_ld_wait();
+                    epilogue_chunk<KIND, NT>(p, cur.t, warp, lane, c0, rr, xchg, tscale);
+                }
+                tc_fence_before();
             }
-            tc_fence_before();
             __syncwarp();
-            if (lane == 0) mbar_arrive(&tempty[acc]);
+            if (lane == 0 && !dead) mbar_arrive(&tempty[acc]);
             named_bar_sync(1, 128);
             ++tcount;
             cur.next_tile(p);
@@ -800,10 +812,12 @@ __global__ void __launch_bounds__(kGemmThreads, 1) k_umma_gemm(const __grid_cons
     }
 
     tc_fence_before();
+    __syncwarp();
     __syncthreads();
     if (*abort_flag && threadIdx.x == 0) set_status(p.ctrl, LMOE_ERR_TIMEOUT);
     if (warp == 12) {
         tc_fence_after();
+        __syncwarp();
         tmem_dealloc(tmem_base, kTmemCols);
     }
 }

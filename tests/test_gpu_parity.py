@@ -140,10 +140,11 @@ def test_block_few_tokens_ragged_steps(fmt, T):
 
 
 @pytest.mark.parametrize("T", [2, 8])
-def test_block_wide_hidden_one_kernel_and_five_kernel_steps(T):
-    """hidden 4096: at 8 tokens the one-kernel step's shared memory does not
-    fit and the five-kernel few-token path runs; at 2 tokens the one-kernel
-    step runs.  Both against the oracle."""
+def test_block_wide_hidden_few_token_steps(T):
+    """hidden 4096 (the D kernel's activation cache at its widest) with
+    latent 256 and ffn 128 (one 256-column stage per gate/up item, a
+    half-filled stage per down item on the tensor-core expert kernels), at 2
+    and 8 tokens, against the oracle."""
     wl = small_workload(T, hidden=4096, latent=256, n_experts=48, top_k=6, n_groups=4, ffn=128, shared_ffn=128)
     layer = synth.make_layer(wl)
     check_block(wl.shape, layer, synth.make_x(wl), what=f"hidden 4096 T={T}")
@@ -468,8 +469,9 @@ def test_decode_q3k_iq4nl_match_oracle_bit_for_bit():
 
 @pytest.mark.parametrize("T", [1, 4, 8, 13, 37])
 def test_block_q3k_experts_few_tokens(T):
-    """The one-kernel step with Q3_K gate/up and IQ4_NL down records (T <= 8),
-    and the same step on passes of 8 tokens (9-63)."""
+    """The few-token step with Q3_K gate/up and IQ4_NL down records (T <= 8:
+    the weight-streaming kernels), and the same step on passes of 8 tokens
+    (9-63)."""
     wl = small_workload(T, latent=256, expert_fmt="q3k")
     check_block(wl.shape, synth.make_layer(wl), synth.make_x(wl), what=f"q3k T={T}")
 
