@@ -358,7 +358,7 @@ template <int PHASE>
 __global__ void __launch_bounds__(kNvThreads, 1) k_nvf4(const __grid_constant__ NvArgs a) {
     using Geo = NvGeom<PHASE>;
     constexpr int NM = Geo::NM, STAGES = Geo::STAGES;
-    constexpr int LA = STAGES - 1;   // stages a loader thread keeps in flight
+    constexpr int LA = STAGES - 2;   // stages in flight ahead; one more slot gives the MMA a stage of slack
     const FwdParams& p = a.p;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
