@@ -94,6 +94,7 @@ class LayerShape:
     du_fmt: int = Q8_0          # 8: Q8_0, 4: Q4_0
     router_dtype: str = "bf16"  # "f32" or "bf16"
     expert_fmt: str = "nvfp4"   # "nvfp4", or "q3k" (Q3_K gate/up + IQ4_NL down)
+    act_fmt: str = "fp16"       # expert inputs: "fp16" (as computed), or "nvfp4" (W4A4)
 
 
 @dataclass(frozen=True)

@@ -265,6 +265,83 @@ double dot(const double* a, const double* b, int n) {
 
 double silu(double a) { return a / (1.0 + std::exp(-a)); }
 
+// ---------------------------------------------------------------------------
+// NVFP4 activations (the W4A4 mode)
+// ---------------------------------------------------------------------------
+//
+// The teardown article's "What is 4-bit" section gives the NVFP4 format (E2M1
+// values, one E4M3 scale per 16) for the weights.  The W4A4 mode applies it to
+// the routed experts' inputs as well (h before gate/up, z before down); the
+// pages give no rule for choosing activation scales, so this library uses
+// the plainest one that keeps every block scale in the E4M3 range: one fp32
+// scale per row, G = max|v| / (6 * 448), and per 16-element block the
+// smallest E4M3 value s >= max|v_block| / (6 G), codes = E2M1 nearest (ties
+// to the even code, saturating at 6) of v / (s G).  The kernels take these
+// decisions in fp32 on the fp16 activations they store, so the oracle rounds
+// the row to fp16 first and repeats the same fp32 operations; the products
+// and sums after that are fp64.
+
+// Round to the nearest IEEE binary16 value (ties to even), as a double.
+double fp16_round(double x) {
+    if (!std::isfinite(x)) return x;
+    const double a = std::fabs(x);
+    if (a >= 65520.0) return std::copysign(std::numeric_limits<double>::infinity(), x);
+    int e;
+    std::frexp(a, &e);                          // a = f 2^e, f in [0.5, 1)
+    const int lead = std::max(e - 1, -14);      // exponent of the leading bit (subnormals: -14)
+    const double quantum = std::ldexp(1.0, lead - 10);
+    return std::copysign(std::nearbyint(a / quantum) * quantum, x);
+}
+
+// Code of the smallest E4M3 value not below s (0 < s), at most 448.
+int e4m3_code_up(float s) {
+    for (int c = 1; c < 0x7E; ++c)
+        if ((float)e4m3fn_value(c) >= s) return c;
+    return 0x7E;
+}
+
+// E2M1 code nearest to v (ties to the even code), saturating at +-6.
+int e2m1_code_rn(float v) {
+    const float a = std::fabs(v);
+    int best = 0;
+    double bd = std::numeric_limits<double>::infinity();
+    for (int c = 0; c < 8; ++c) {
+        const double d = std::fabs((double)a - e2m1_value(c));
+        if (d < bd || (d == bd && (c & 1) == 0 && (best & 1) == 1)) {
+            bd = d;
+            best = c;
+        }
+    }
+    return (v < 0.f ? 8 : 0) | best;
+}
+
+// One activation row v [K] (K % 16 == 0, fp16-representable values) ->
+// out [K] = its NVFP4 value q * s * G; codes [K] (E2M1, low 4 bits),
+// scales [K/16] (E4M3 codes) and G when not NULL.
+void nvfp4_act_row(const double* v, int K, double* out, uint8_t* codes, uint8_t* scales, float* Gout) {
+    float amax = 0.f;
+    for (int k = 0; k < K; ++k) amax = std::max(amax, std::fabs((float)v[k]));
+    const float G = amax > 0.f ? amax * (1.f / (6.f * 448.f)) : 1.f;
+    if (Gout) *Gout = G;
+    for (int b = 0; b < K / 16; ++b) {
+        float bmax = 0.f;
+        for (int e = 0; e < 16; ++e) bmax = std::max(bmax, std::fabs((float)v[16 * b + e]));
+        int sc = 0;
+        float sd = 0.f;
+        if (bmax > 0.f) {
+            sc = e4m3_code_up(bmax / (6.f * G));
+            sd = (float)e4m3fn_value(sc) * G;
+        }
+        if (scales) scales[b] = (uint8_t)sc;
+        const float inv = sc ? 1.f / sd : 0.f;
+        for (int e = 0; e < 16; ++e) {
+            const int q = sc ? e2m1_code_rn((float)v[16 * b + e] * inv) : 0;
+            if (codes) codes[16 * b + e] = (uint8_t)q;
+            out[16 * b + e] = sc ? e2m1_value(q) * e4m3fn_value(sc) * (double)G : 0.0;
+        }
+    }
+}
+
 }  // namespace
 
 extern "C" {
@@ -274,6 +351,7 @@ struct orc_shape {
     int du_fmt;        // 8: Q8_0, 4: Q4_0
     int router_bf16;   // 1: router weights are bf16 bits, 0: fp32
     int expert_fmt;    // 0: NVFP4 records, 1: Q3_K gate/up + IQ4_NL down records
+    int act_fmt;       // 0: expert inputs as computed, 1: NVFP4 expert inputs (W4A4)
 };
 
 struct orc_layer {
@@ -429,11 +507,22 @@ void orc_shared_expert(const orc_shape* s, const orc_layer* ly, const double* x,
     }
 }
 
-// One expert on n latent vectors h [n][L] (step 4): o [n][L].
-void orc_expert_apply_fmt(int efmt, const uint8_t* rec, int L, int F, const double* h, int n, double* o) {
+// One expert on n latent vectors h [n][L] (step 4): o [n][L].  act = 1:
+// h and then z are taken as their NVFP4 activation values (W4A4 mode).
+void orc_expert_apply_act(int efmt, int act, const uint8_t* rec, int L, int F, const double* h_in, int n, double* o) {
     const ExpertMatrix vg = expert_matrix(rec, L, F, 0, efmt), vu = expert_matrix(rec, L, F, 1, efmt),
                        vd = expert_matrix(rec, L, F, 2, efmt);
-    std::vector<double> rg(L), ru(L), rd(F), z((size_t)n * F);
+    std::vector<double> rg(L), ru(L), rd(F), z((size_t)n * F), hq;
+    const double* h = h_in;
+    if (act == 1) {
+        hq.resize((size_t)n * L);
+        std::vector<double> r16(L);
+        for (int i = 0; i < n; ++i) {
+            for (int k = 0; k < L; ++k) r16[k] = fp16_round(h_in[(int64_t)i * L + k]);
+            nvfp4_act_row(r16.data(), L, hq.data() + (size_t)i * L, nullptr, nullptr, nullptr);
+        }
+        h = hq.data();
+    }
     for (int f = 0; f < F; ++f) {
         nvfp4_row(vg, f, rg.data());
         nvfp4_row(vu, f, ru.data());
@@ -442,15 +531,37 @@ void orc_expert_apply_fmt(int efmt, const uint8_t* rec, int L, int F, const doub
             z[(size_t)i * F + f] = silu(dot(rg.data(), hi, L)) * dot(ru.data(), hi, L);
         }
     }
+    if (act == 1) {
+        std::vector<double> r16(F);
+        for (int i = 0; i < n; ++i) {
+            for (int f = 0; f < F; ++f) r16[f] = fp16_round(z[(size_t)i * F + f]);
+            nvfp4_act_row(r16.data(), F, z.data() + (size_t)i * F, nullptr, nullptr, nullptr);
+        }
+    }
     for (int r = 0; r < L; ++r) {
         nvfp4_row(vd, r, rd.data());
         for (int i = 0; i < n; ++i) o[(int64_t)i * L + r] = dot(rd.data(), z.data() + (size_t)i * F, F);
     }
 }
 
+void orc_expert_apply_fmt(int efmt, const uint8_t* rec, int L, int F, const double* h, int n, double* o) {
+    orc_expert_apply_act(efmt, 0, rec, L, F, h, n, o);
+}
+
 void orc_expert_apply(const uint8_t* rec, int L, int F, const double* h, int n, double* o) {
     orc_expert_apply_fmt(0, rec, L, F, h, n, o);
 }
+
+// One activation row quantised as the W4A4 mode does (fp16 rounding first):
+// out [K] its NVFP4 values, codes [K], scales [K/16], G [1] (any may be NULL
+// except out).  K % 16 == 0.
+void orc_nvfp4_act_quantize(const double* v, int K, double* out, uint8_t* codes, uint8_t* scales, float* G) {
+    std::vector<double> r16(K);
+    for (int k = 0; k < K; ++k) r16[k] = fp16_round(v[k]);
+    nvfp4_act_row(r16.data(), K, out, codes, scales, G);
+}
+
+double orc_fp16_round(double x) { return fp16_round(x); }
 
 // y [n][R] = M x for the stored Q8_0 / Q4_0 matrix M [R][C] and n vectors x [n][C].
 void orc_du_apply(int fmt, const uint8_t* m, int R, int C, const double* x, int n, double* y) {
@@ -529,7 +640,8 @@ int orc_forward(const orc_shape* s, const orc_layer* ly, const double* x, const 
         std::vector<double> hin(pe.size() * (size_t)L), out(pe.size() * (size_t)L);
         for (size_t i = 0; i < pe.size(); ++i)
             std::memcpy(&hin[i * L], &h[((size_t)(pe[i] / K) * G + g) * L], sizeof(double) * L);
-        orc_expert_apply_fmt(s->expert_fmt, ly->experts + e * rec_b, L, F, hin.data(), (int)pe.size(), out.data());
+        orc_expert_apply_act(s->expert_fmt, s->act_fmt, ly->experts + e * rec_b, L, F, hin.data(), (int)pe.size(),
+                             out.data());
         for (size_t i = 0; i < pe.size(); ++i) std::memcpy(&o[(size_t)pe[i] * L], &out[i * L], sizeof(double) * L);
     }
     // step 7 first (the output starts as the shared expert), then steps 5, 6

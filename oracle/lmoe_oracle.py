@@ -287,11 +287,67 @@ def shared_expert(x: np.ndarray, Wsg: np.ndarray, Wsu: np.ndarray, Wsd: np.ndarr
     return (silu(a) * u) @ Wsd.T
 
 
-def expert_apply(Wg: np.ndarray, Wu: np.ndarray, Wd: np.ndarray, h: np.ndarray) -> np.ndarray:
-    """E_e : R^l -> R^F -> R^l, SwiGLU: W_down (silu(W_gate h) * (W_up h))."""
+def expert_apply(Wg: np.ndarray, Wu: np.ndarray, Wd: np.ndarray, h: np.ndarray, act: str = "fp16") -> np.ndarray:
+    """E_e : R^l -> R^F -> R^l, SwiGLU: W_down (silu(W_gate h) * (W_up h)).
+    act = "nvfp4": h and z enter as their NVFP4 activation values (W4A4)."""
+    if act == "nvfp4":
+        h = nvfp4_act(h)
     a = Wg @ h
     u = Wu @ h
-    return Wd @ (silu(a) * u)
+    z = silu(a) * u
+    if act == "nvfp4":
+        z = nvfp4_act(z)
+    return Wd @ z
+
+
+# ---- NVFP4 activations (the W4A4 mode) -------------------------------------
+# The teardown article ("What is 4-bit") gives NVFP4 for the weights; the
+# W4A4 mode applies it to the experts' inputs with the rule the pages leave
+# open read plainly: one fp32 scale per row G = max|v| / (6 * 448), per 16
+# elements the smallest E4M3 value s >= max|v_block| / (6 G), E2M1 codes
+# nearest (ties to even, saturating) to v / (s G).  The decisions are taken
+# in fp32 on the fp16-rounded row, as the kernels take them.
+
+def _e4m3_positive() -> np.ndarray:
+    return e4m3fn_to_f64(np.arange(0x7F))          # codes 0 .. 0x7E by value, 0x7F is NaN
+
+
+def _e2m1_nearest(v: np.ndarray) -> np.ndarray:
+    """Value of the E2M1 code nearest to each float32 v (ties to the even code, +-6 at most)."""
+    mags = e2m1_to_f64(np.arange(8))
+    a = np.abs(v.astype(np.float64))
+    d = np.abs(a[..., None] - mags)
+    dmin = d.min(-1, keepdims=True)
+    cand = d == dmin
+    even = cand & (np.arange(8) % 2 == 0)
+    code = np.where(even.any(-1), np.argmax(even, -1), np.argmax(cand, -1))
+    return np.where(v < 0, -mags[code], mags[code])
+
+
+def nvfp4_act(v: np.ndarray) -> np.ndarray:
+    """NVFP4 activation values of one row v [K] (K % 16 == 0), fp64 out."""
+    r = fp16_round(np.asarray(v, np.float64)).astype(np.float32)
+    amax = np.float32(np.abs(r).max())
+    G = np.float32(amax * np.float32(1.0 / 2688.0)) if amax > 0 else np.float32(1.0)
+    e4 = _e4m3_positive()
+    blocks = r.reshape(-1, 16)
+    bmax = np.abs(blocks).max(1)
+    with np.errstate(divide="ignore", invalid="ignore"):
+        s = (bmax / np.float32(np.float32(6.0) * G)).astype(np.float32)
+    code = np.minimum(np.searchsorted(e4.astype(np.float32), s, side="left"), 0x7E)
+    code = np.where(bmax > 0, np.maximum(code, 1), 0)
+    sval = e4[code].astype(np.float32)
+    sd = (sval * G).astype(np.float32)
+    with np.errstate(divide="ignore", invalid="ignore"):
+        inv = np.where(sd > 0, np.float32(1.0) / sd, np.float32(0.0)).astype(np.float32)
+    q = _e2m1_nearest((blocks * inv[:, None]).astype(np.float32))
+    out = q * e4[code][:, None] * np.float64(G)
+    return np.where(bmax[:, None] > 0, out, 0.0).reshape(-1)
+
+
+def fp16_round(v: np.ndarray) -> np.ndarray:
+    """Nearest binary16 values (ties to even), as fp64."""
+    return np.asarray(v, np.float64).astype(np.float16).astype(np.float64)
 
 
 class Weights:
@@ -369,7 +425,7 @@ def latent_moe_forward(shape, layer: dict, x_bits: np.ndarray, residual_bits: np
         for (t, k) in pairs[e]:
             if (t, g) not in h_cache:
                 h_cache[(t, g)] = W.D(g) @ x[t]
-            o[t, k] = expert_apply(Wg, Wu, Wd, h_cache[(t, g)])
+            o[t, k] = expert_apply(Wg, Wu, Wd, h_cache[(t, g)], getattr(shape, "act_fmt", "fp16"))
     for t in range(T):
         hit = sorted({int(W.group[e]) for e in idx[t]})
         for g in hit:

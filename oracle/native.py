@@ -44,7 +44,7 @@ def build(force: bool = False) -> str:
 
 class _Shape(ctypes.Structure):
     _fields_ = [(n, ctypes.c_int) for n in ("hidden", "latent", "n_experts", "top_k", "n_groups", "ffn",
-                                            "shared_ffn", "du_fmt", "router_bf16", "expert_fmt")]
+                                            "shared_ffn", "du_fmt", "router_bf16", "expert_fmt", "act_fmt")]
 
 
 class _Layer(ctypes.Structure):
@@ -89,6 +89,9 @@ def lib():
         L.orc_expert_offset_fmt.argtypes = [i32, i32, i32, i32]
         L.orc_decode_expert_fmt.argtypes = [i32, vp, i32, i32, vp, vp, vp]
         L.orc_dproj_q8_1.argtypes = [i32, vp, i32, i32, i32, vp, i32, vp]
+        L.orc_nvfp4_act_quantize.argtypes = [vp, i32, vp, vp, vp, vp]
+        L.orc_fp16_round.restype = dbl
+        L.orc_fp16_round.argtypes = [dbl]
         L.orc_stack_layer.restype = i32
         L.orc_stack_layer.argtypes = [ctypes.POINTER(_Shape), ctypes.POINTER(_Layer), vp, vp, dbl, vp, vp, i32, vp,
                                       vp, vp, vp]
@@ -240,7 +243,7 @@ def route(x, Wr, b, top_k: int):
 def _shape(shape) -> _Shape:
     return _Shape(shape.hidden, shape.latent, shape.n_experts, shape.top_k, shape.n_groups, shape.ffn,
                   shape.shared_ffn, shape.du_fmt, 1 if shape.router_dtype == "bf16" else 0,
-                  _efmt(getattr(shape, "expert_fmt", "nvfp4")))
+                  _efmt(getattr(shape, "expert_fmt", "nvfp4")), 1 if getattr(shape, "act_fmt", "fp16") == "nvfp4" else 0)
 
 
 class _LayerRef:
@@ -408,3 +411,21 @@ def dproj_q8_1(fmt: int, D, G: int, L: int, H: int, x) -> np.ndarray:
     h = np.empty((x.shape[0], G, L))
     lib().orc_dproj_q8_1(fmt, pD, G, L, H, _ptr(x), x.shape[0], _ptr(h))
     return h
+
+
+def nvfp4_act_quantize(v):
+    """One activation row as the W4A4 mode quantises it: (values fp64 [K],
+    E2M1 codes [K], E4M3 scale codes [K/16], G)."""
+    v = np.ascontiguousarray(v, np.float64)
+    K = v.size
+    assert K % 16 == 0
+    out = np.empty(K, np.float64)
+    codes = np.empty(K, np.uint8)
+    scales = np.empty(K // 16, np.uint8)
+    G = np.empty(1, np.float32)
+    lib().orc_nvfp4_act_quantize(_ptr(v), K, _ptr(out), _ptr(codes), _ptr(scales), _ptr(G))
+    return out, codes, scales, float(G[0])
+
+
+def fp16_round(x: float) -> float:
+    return float(lib().orc_fp16_round(float(x)))
