@@ -49,6 +49,7 @@ def parse():
     ap.add_argument("--cpu-seconds", type=float, default=12.0, help="CPU-oracle sample budget")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-sweep", action="store_true", help="skip the MTP verify-window sweep")
+    ap.add_argument("--no-w4a4", action="store_true", help="skip the W4A4 prefill object")
     return ap.parse_args()
 
 
@@ -229,7 +230,8 @@ def workload_desc(wl, T):
     bias = "none" if wl.bias_sigma is None else f"N(0,{wl.bias_sigma:g})"
     return (f"{wl.name}: T={T}, hidden {s.hidden}, latent {s.latent}, {s.n_experts} experts top-{s.top_k}, "
             f"{s.n_groups} {fmt} D/U groups, NVFP4 experts ffn {s.ffn}, bf16 shared ffn {s.shared_ffn}, "
-            f"{s.router_dtype} router, bias {bias}, expert_group {wl.groups}, x bf16 N(0,1), weights N(0,0.02)")
+            f"{s.router_dtype} router, bias {bias}, expert_group {wl.groups}, x bf16 N(0,1), weights N(0,0.02)"
+            + (", NVFP4 expert inputs (W4A4)" if getattr(s, "act_fmt", "fp16") == "nvfp4" else ""))
 
 
 def load_peaks():
@@ -551,10 +553,14 @@ def measure_layer(args, wl, T, K, W, rank, world, local, dev_name, ctx=None, lig
     dom_s = stage_ms[dom] / 1e3
     if prefill:
         dom_ach = cost[dom_name] / dom_s / 1e12
-        roof = {"bound": "tensor", "kernel": dom_name, "achieved": dom_ach, "peak": tc_peak, "unit": "TFLOP/s",
-                "frac": dom_ach / tc_peak,
-                "peak_source": f"{peak_src} bf16 dense burst (fp16 operands run at the bf16 rate)",
-                "traffic": ncu_traffic(wl.name, T, dom_name)}
+        if getattr(s, "act_fmt", "fp16") == "nvfp4" and dom_name in ("gateup", "down"):
+            # W4A4 expert GEMMs run kind::mxf4nvf4: the FP4 peak, taken as the
+            # measured bf16 peak times the nominal dense ratio 9 / 2.25 = 4
+            peak, psrc = 4.0 * tc_peak, f"{peak_src} bf16 dense burst x 4 (nominal fp4 / bf16 dense ratio)"
+        else:
+            peak, psrc = tc_peak, f"{peak_src} bf16 dense burst (fp16 operands run at the bf16 rate)"
+        roof = {"bound": "tensor", "kernel": dom_name, "achieved": dom_ach, "peak": peak, "unit": "TFLOP/s",
+                "frac": dom_ach / peak, "peak_source": psrc, "traffic": ncu_traffic(wl.name, T, dom_name)}
     else:
         dom_ach = cost[dom_name] / dom_s / 1e9
         roof = {"bound": "hbm", "kernel": dom_name, "achieved": dom_ach, "peak": hbm_peak, "unit": "GB/s",
@@ -748,6 +754,13 @@ def main():
             pre["cpu_baseline"] = cpu_baseline(pre_wl, pre_layer, pre_wl.T, args.cpu_seconds, sample_tokens=16)
         line["prefill"] = pre
         line["gpu_launches"] = head["gpu_launches"] + pre["gpu_launches"]
+        if not args.no_w4a4 and pre_wl.shape.expert_fmt == "nvfp4":
+            # the same prefill with NVFP4 expert inputs (W4A4, lmoe_cfg.act_fmt)
+            w4_wl = pre_wl.with_(shape=synth.replace(pre_wl.shape, act_fmt="nvfp4"))
+            w4, _ = measure_layer(args, w4_wl, w4_wl.T, K, W, rank, world, local, dev_name)
+            w4["metric"] = "latent-MoE layer tokens/s, prefill, W4A4 (NVFP4 expert inputs)"
+            line["prefill_w4a4"] = w4
+            line["gpu_launches"] += w4["gpu_launches"]
     if rank == 0:
         print(json.dumps(line), flush=True)
     if world > 1:

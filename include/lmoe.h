@@ -104,6 +104,16 @@ typedef enum {
 typedef enum { LMOE_Q8_0 = 8, LMOE_Q4_0 = 4 } lmoe_du_fmt;   /* D/U block formats */
 typedef enum { LMOE_F32 = 0, LMOE_BF16 = 1 } lmoe_dtype;     /* router weight type */
 typedef enum { LMOE_EXPERTS_NVFP4 = 0, LMOE_EXPERTS_Q3K = 1 } lmoe_expert_fmt;   /* expert records */
+/* Expert inputs.  LMOE_ACT_FP16: h and z enter the expert contractions as
+ * computed (staged in fp16, fp32 accumulation).  LMOE_ACT_NVFP4 (W4A4, NVFP4
+ * expert records only): the teardown article's NVFP4 format ("What is
+ * 4-bit") applied to h before gate/up and to z before down, each row
+ * quantised on its fp16 values in fp32: G = max|v| / (6 * 448), per 16
+ * elements the smallest E4M3 scale s >= max|v_block| / (6 G), E2M1 codes
+ * nearest (ties to even, saturating) to v / (s G); the contractions then run
+ * as NVFP4 x NVFP4 on the tensor cores (tcgen05 kind::mxf4nvf4).  Needs
+ * latent and ffn multiples of 128 up to 2048. */
+typedef enum { LMOE_ACT_FP16 = 0, LMOE_ACT_NVFP4 = 1 } lmoe_act_fmt;
 
 typedef struct {
     int hidden;        /* model width (2560 for Edge0 145B / 120B) */
@@ -116,6 +126,7 @@ typedef struct {
     int du_fmt;        /* lmoe_du_fmt */
     int router_dtype;  /* lmoe_dtype */
     int expert_fmt;    /* lmoe_expert_fmt (0: NVFP4 records) */
+    int act_fmt;       /* lmoe_act_fmt (0: fp16 expert inputs) */
 } lmoe_cfg;
 
 typedef struct {
@@ -177,7 +188,12 @@ LMOE_API int lmoe_route(const lmoe_cfg* cfg, const void* x, const void* router_w
  * Arguments: x bf16 [T][hidden]; weights as in the storage layouts above;
  * y bf16 [T][hidden] (must not overlap x); ws of lmoe_workspace_bytes(cfg, T).
  * Errors: LMOE_ERR_ARG / _UNSUPPORTED / _WORKSPACE before any launch; kernel
- * findings through lmoe_last_device_status. */
+ * findings through lmoe_last_device_status.
+ * Environment: LMOE_FEW_TOKEN_EXPERTS=tensor_cores (read at every call)
+ * runs the NVFP4 expert contractions of steps of T <= 8 on the tensor cores
+ * (kind::mxf4nvf4 on the stored bytes, the fp16 activations as six E2M1
+ * terms) instead of the weight-streaming kernels; the result agrees within
+ * the same tolerance, the default is faster on the Edge0 shapes. */
 LMOE_API int lmoe_forward(const lmoe_cfg* cfg, const void* x, const void* router_w, const uint8_t* expert_group,
                  const void* D, const void* U, const void* experts, const lmoe_shared* shared,
                  void* y, int T, void* ws, size_t ws_bytes, void* stream);
@@ -227,6 +243,17 @@ LMOE_API const char* lmoe_status_str(int status);
  * an NVFP4 matrix (q then s as in an expert record, scaled by ts), 2 for a
  * Q3_K matrix, 3 for an IQ4_NL matrix (layouts above; ts unused). */
 LMOE_API int lmoe_debug_decode(int fmt, const void* blob, int rows, int cols, float ts, float* out, void* stream);
+
+/* Diagnostics: the W4A4 mode's activation quantiser on its own.  Defining
+ * passage: teardown article, section "What is 4-bit" (NVFP4: E2M1 values,
+ * one E4M3 scale per 16), applied to activations by the rule under
+ * lmoe_act_fmt.  src: fp16 [n][cols] (device, 16-byte aligned), cols a
+ * multiple of 64.  Outputs (device, caller-owned): codes [cols/32][n][16]
+ * bytes (element 2i of a row's 32-column chunk in the low nibble of byte i),
+ * scales [cols/64][n] 32-bit words (byte j: the E4M3 code of the row's
+ * 16-column block 4k + j), G [n] fp32.  Returns LMOE_ERR_ARG for null,
+ * misaligned or badly sized arguments. */
+LMOE_API int lmoe_debug_act_quant(const void* src, int n, int cols, void* codes, void* scales, float* G, void* stream);
 
 /* Profiling: while n > 0, every later forward call records events[0] before
  * its first kernel, events[i] before kernel i and one more event after its

@@ -27,11 +27,13 @@ LMOE_Q3K_DEBUG = 2
 LMOE_IQ4NL_DEBUG = 3
 LMOE_EXPERTS_NVFP4 = 0
 LMOE_EXPERTS_Q3K = 1
+LMOE_ACT_FP16 = 0
+LMOE_ACT_NVFP4 = 1
 
 # every symbol include/lmoe.h declares
 EXPORTS = ("lmoe_cfg_check", "lmoe_expert_record_bytes", "lmoe_du_bytes", "lmoe_workspace_bytes", "lmoe_route",
            "lmoe_forward", "lmoe_forward_ex", "lmoe_forward_host", "lmoe_stack_forward", "lmoe_last_device_status",
-           "lmoe_status_str", "lmoe_debug_decode", "lmoe_profile_stage_events",
+           "lmoe_status_str", "lmoe_debug_decode", "lmoe_debug_act_quant", "lmoe_profile_stage_events",
            "lmoe_route_noalloc", "lmoe_dproj_ablation")
 
 
@@ -43,7 +45,7 @@ class LmoeError(RuntimeError):
 
 class lmoe_cfg(ctypes.Structure):
     _fields_ = [(n, ctypes.c_int) for n in ("hidden", "latent", "n_experts", "top_k", "n_groups", "ffn",
-                                            "shared_ffn", "du_fmt", "router_dtype", "expert_fmt")]
+                                            "shared_ffn", "du_fmt", "router_dtype", "expert_fmt", "act_fmt")]
 
 
 class lmoe_shared(ctypes.Structure):
@@ -92,6 +94,8 @@ def lib() -> ctypes.CDLL:
         L.lmoe_status_str.restype = ctypes.c_char_p
         L.lmoe_debug_decode.argtypes = [i32, vp, i32, i32, f32, vp, vp]
         L.lmoe_debug_decode.restype = i32
+        L.lmoe_debug_act_quant.argtypes = [vp, i32, i32, vp, vp, vp, vp]
+        L.lmoe_debug_act_quant.restype = i32
         L.lmoe_profile_stage_events.argtypes = [ctypes.POINTER(ctypes.c_void_p), i32]
         L.lmoe_profile_stage_events.restype = i32
         L.lmoe_route_noalloc.argtypes = [cfgp, vp, vp, vp, i32, vp, vp, vp]
@@ -142,8 +146,11 @@ def make_cfg(shape) -> lmoe_cfg:
     ef = getattr(shape, "expert_fmt", "nvfp4")
     if isinstance(ef, str):
         ef = LMOE_EXPERTS_Q3K if ef == "q3k" else LMOE_EXPERTS_NVFP4
+    af = getattr(shape, "act_fmt", "fp16")
+    if isinstance(af, str):
+        af = LMOE_ACT_NVFP4 if af == "nvfp4" else LMOE_ACT_FP16
     return lmoe_cfg(shape.hidden, shape.latent, shape.n_experts, shape.top_k, shape.n_groups, shape.ffn,
-                    shape.shared_ffn, shape.du_fmt, rd, ef)
+                    shape.shared_ffn, shape.du_fmt, rd, ef, af)
 
 
 def make_shared(gate, up, down) -> lmoe_shared:
@@ -212,6 +219,11 @@ def lmoe_stack_forward(cfg, layers, x, y, T, rms_eps, ws, stream=None):
 
 def lmoe_last_device_status(ws, stream=None) -> int:
     return lib().lmoe_last_device_status(_ptr(ws), _nbytes(ws), _stream(stream))
+
+
+def lmoe_debug_act_quant(src, n, cols, codes, scales, G, stream=None):
+    return _check(lib().lmoe_debug_act_quant(_ptr(src), n, cols, _ptr(codes), _ptr(scales), _ptr(G), _stream(stream)),
+                  "lmoe_debug_act_quant")
 
 
 def lmoe_debug_decode(fmt, blob, rows, cols, ts, out, stream=None):

@@ -25,6 +25,10 @@ int check_cfg(const lmoe_cfg* c) {
     if (c->router_dtype != LMOE_F32 && c->router_dtype != LMOE_BF16) return LMOE_ERR_UNSUPPORTED;
     if (c->expert_fmt != LMOE_EXPERTS_NVFP4 && c->expert_fmt != LMOE_EXPERTS_Q3K) return LMOE_ERR_UNSUPPORTED;
     if (c->expert_fmt == LMOE_EXPERTS_Q3K && c->latent % 256) return LMOE_ERR_UNSUPPORTED;
+    if (c->act_fmt != LMOE_ACT_FP16 && c->act_fmt != LMOE_ACT_NVFP4) return LMOE_ERR_UNSUPPORTED;
+    if (c->act_fmt == LMOE_ACT_NVFP4 && (c->expert_fmt != LMOE_EXPERTS_NVFP4 || c->latent % 128 || c->ffn % 128 ||
+                                         c->latent > 2048 || c->ffn > 2048))
+        return LMOE_ERR_UNSUPPORTED;
     return LMOE_OK;
 }
 
@@ -56,7 +60,7 @@ struct WsLayout {
     // tensor-core path
     size_t p_zero_begin, p_tgmask, p_cnt, p_fill, p_dhit, p_n_etiles, p_zero_end;
     size_t p_n_unique, p_off, p_uexp, p_ucnt, p_uoff, p_etile, p_slot_pair, p_pair_slot, p_idx, p_w, p_logits;
-    size_t p_xh, p_xr, p_xr_lo, p_hperm, p_zperm, p_operm, p_s, p_zsh;
+    size_t p_xh, p_xr, p_xr_lo, p_hperm, p_zperm, p_operm, p_s, p_zsh, p_aq, p_asf, p_aG;
     size_t total;
 };
 
@@ -140,6 +144,12 @@ WsLayout ws_layout(const lmoe_cfg& c, int T) {
         L.p_operm = take(TK * c.latent * 2);
         L.p_s = take((size_t)T * c.n_groups * c.latent * 2);
         L.p_zsh = take((size_t)2 * T * c.shared_ffn * 2);
+        if (c.act_fmt == LMOE_ACT_NVFP4) {
+            const size_t Kmax = std::max(c.latent, c.ffn);
+            L.p_aq = take(TK * Kmax / 2);
+            L.p_asf = take(TK * Kmax / 16);
+            L.p_aG = take(TK * 4);
+        }
     }
     L.total = std::max(off, end_decode);
     return L;
@@ -151,6 +161,7 @@ FwdParams base_params(const lmoe_cfg& c, int T, void* ws, const WsLayout& L) {
     p.H = c.hidden; p.L = c.latent; p.E = c.n_experts; p.K = c.top_k; p.G = c.n_groups;
     p.F = c.ffn; p.Fs = c.shared_ffn; p.du_fmt = c.du_fmt; p.router_bf16 = c.router_dtype == LMOE_BF16;
     p.efmt = c.expert_fmt;
+    p.act = c.act_fmt;
     p.T = T;
     char* b = static_cast<char*>(ws);
     p.ctrl = reinterpret_cast<Ctrl*>(b + L.ctrl);
@@ -212,6 +223,7 @@ int run_prefill(const lmoe_cfg& c, const FwdParams& f, const WsLayout& L, void* 
     char* b = static_cast<char*>(ws);
     p.H = f.H; p.L = f.L; p.E = f.E; p.K = f.K; p.G = f.G; p.F = f.F; p.Fs = f.Fs; p.du_fmt = f.du_fmt; p.T = f.T;
     p.efmt = f.efmt;
+    p.act = f.act;
     p.x = f.x;
     p.router_w_bf16 = static_cast<const uint16_t*>(f.router_w);
     p.router_b = f.router_b;
@@ -255,6 +267,11 @@ int run_prefill(const lmoe_cfg& c, const FwdParams& f, const WsLayout& L, void* 
     p.operm = reinterpret_cast<__half*>(b + L.p_operm);
     p.s = reinterpret_cast<__half*>(b + L.p_s);
     p.zsh = reinterpret_cast<uint16_t*>(b + L.p_zsh);
+    if (f.act == LMOE_ACT_NVFP4) {
+        p.aq = reinterpret_cast<uint8_t*>(b + L.p_aq);
+        p.asf = reinterpret_cast<uint32_t*>(b + L.p_asf);
+        p.aG = reinterpret_cast<float*>(b + L.p_aG);
+    }
     (void)c;
     stage_reset();
     return cuda_status(run_prefill_path(p, st, b + L.p_zero_begin, L.p_zero_end - L.p_zero_begin, stage_mark));
@@ -298,11 +315,17 @@ int forward_impl(const lmoe_cfg* cfg, const void* x, const void* router_w, const
     p.out_idx = out_idx;
     p.out_w = out_w;
     p.y = static_cast<uint16_t*>(y);
+    if (cfg->act_fmt == LMOE_ACT_NVFP4) {
+        FwdParams q = p;
+        q.T = std::min(T, 8);
+        if (!nvf4_usable(q)) return LMOE_ERR_UNSUPPORTED;
+    }
     if (use_prefill(*cfg, T)) return run_prefill(*cfg, p, L, ws, st);
-    if (cfg->expert_fmt == LMOE_EXPERTS_Q3K && T > 8) {
-        // the Q3_K build between 9 and 63 tokens: the few-token step on
-        // passes of at most 8 tokens (the kernels of that range read NVFP4
-        // records only)
+    if ((cfg->expert_fmt == LMOE_EXPERTS_Q3K || cfg->act_fmt == LMOE_ACT_NVFP4) && T > 8) {
+        // the Q3_K build between 9 and 63 tokens, and NVFP4 expert inputs
+        // above 8 tokens: the few-token step on passes of at most 8 tokens
+        // (the kernels of 9-63 tokens read NVFP4 records with fp16 inputs
+        // only)
         for (int t0 = 0; t0 < T; t0 += 8) {
             FwdParams q = p;
             q.T = std::min(8, T - t0);
@@ -495,6 +518,14 @@ int lmoe_debug_decode(int fmt, const void* blob, int rows, int cols, float ts, f
     if (fmt != LMOE_Q8_0 && fmt != LMOE_Q4_0 && fmt != 1 && fmt != 2 && fmt != 3) return LMOE_ERR_UNSUPPORTED;
     if (fmt == 2 && cols % 256) return LMOE_ERR_ARG;
     return cuda_status(run_debug_decode(fmt, blob, rows, cols, ts, out, static_cast<cudaStream_t>(stream)));
+}
+
+int lmoe_debug_act_quant(const void* src, int n, int cols, void* codes, void* scales, float* G, void* stream) {
+    if (!src || !codes || !scales || !G || n <= 0 || cols <= 0 || cols % 64 || !aligned(src, 16) || !aligned(codes, 16) ||
+        !aligned(scales, 4) || !aligned(G, 4))
+        return LMOE_ERR_ARG;
+    return cuda_status(run_act_quant(static_cast<const __half*>(src), n, cols, static_cast<uint8_t*>(codes),
+                                     static_cast<uint32_t*>(scales), G, static_cast<cudaStream_t>(stream)));
 }
 
 }  // extern "C"

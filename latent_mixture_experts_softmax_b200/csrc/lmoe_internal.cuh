@@ -44,6 +44,7 @@ struct FwdParams {
     // shape
     int H, L, E, K, G, F, Fs, du_fmt, router_bf16;
     int efmt;   // expert records: LMOE_EXPERTS_NVFP4 or LMOE_EXPERTS_Q3K
+    int act;    // expert inputs: LMOE_ACT_FP16 or LMOE_ACT_NVFP4 (W4A4)
     int T;
     // inputs
     const uint16_t* x;

@@ -56,7 +56,8 @@ using namespace sm100;
 
 enum NvPhase { NV_GATEUP = 0, NV_DOWN = 1 };
 
-constexpr int kNvJ = 6;                  // E2M1 terms per activation row
+constexpr int kNvJExact = 6;             // E2M1 terms per activation row (fp16-level inputs)
+constexpr int kNvJW4A4 = 1;              // one term: NVFP4 activations (W4A4)
 constexpr int kNvThreads = 288;
 constexpr int kNvMaxN = 48;              // B columns: 8 tokens x 6 terms
 constexpr int kNvMaxCtas = 160;
@@ -238,11 +239,11 @@ __device__ __forceinline__ const __half* act_row(const FwdParams& p, const NvSha
 // Rows i*J + jj of the B operand (codes in [K/32][npad][16 B], scale bytes
 // [npad][K/16]) and their fp32 term scales; then the scale words to TMEM
 // columns kColSFB + 4k + n/32, lane n%32 of every subpartition.
-template <int PHASE>
+template <int PHASE, int J>
 __device__ void build_b(const FwdParams& p, NvShared& sh, int j, int K, uint8_t* sB, uint8_t* sfbb, float* cs,
                         uint32_t tmem_base, bool& bad) {
     const int tid = threadIdx.x - 128, warp = tid >> 5, lane = tid & 31;   // warps 4-7: subpartitions 0-3
-    const int ne = sh.ucnt[j], N = ne * kNvJ, npad = (N + 15) & ~15;
+    const int ne = sh.ucnt[j], N = ne * J, npad = (N + 15) & ~15;
     const int nb = K / 16;
     // 1. row maxima
     for (int i = 0; i < ne; ++i) {
@@ -263,7 +264,7 @@ __device__ void build_b(const FwdParams& p, NvShared& sh, int j, int K, uint8_t*
     }
     named_bar_sync(2, 128);
     if (tid < N) {
-        const int i = tid / kNvJ, jj = tid - i * kNvJ;
+        const int i = tid / J, jj = tid - i * J;
         const float amax = fmaxf(fmaxf(sh.red[0][i], sh.red[1][i]), fmaxf(sh.red[2][i], sh.red[3][i]));
         float g = amax > 0.f ? amax * (1.f / (6.f * 448.f)) : 1.f;
         for (int u = 0; u < jj; ++u) g *= 0.2f;
@@ -286,8 +287,8 @@ __device__ void build_b(const FwdParams& p, NvShared& sh, int j, int K, uint8_t*
             }
         }
 #pragma unroll 1
-        for (int jj = 0; jj < kNvJ; ++jj) {
-            const int n = i * kNvJ + jj;
+        for (int jj = 0; jj < J; ++jj) {
+            const int n = i * J + jj;
             const float g = cs[n];
             float amax = 0.f;
 #pragma unroll
@@ -354,7 +355,7 @@ __device__ void build_b(const FwdParams& p, NvShared& sh, int j, int K, uint8_t*
 // the kernel
 // ---------------------------------------------------------------------------
 
-template <int PHASE>
+template <int PHASE, int J>
 __global__ void __launch_bounds__(kNvThreads, 1) k_nvf4(const __grid_constant__ NvArgs a) {
     using Geo = NvGeom<PHASE>;
     constexpr int NM = Geo::NM, STAGES = Geo::STAGES;
@@ -516,7 +517,7 @@ __global__ void __launch_bounds__(kNvThreads, 1) k_nvf4(const __grid_constant__ 
                 if (!mbar_wait(&tempty[d], ((pc >> 1) & 1) ^ 1, abort_flag, kNvWaitLimit)) { dead = true; break; }
                 tc_fence_after();
                 const int jd = (s / w.spi) / w.tiles;
-                const int npad = (sh.ucnt[jd] * kNvJ + 15) & ~15;
+                const int npad = (sh.ucnt[jd] * J + 15) & ~15;
                 const uint32_t idesc = idesc_mxf4nvf4(npad);
                 const uint32_t d_tmem = tmem_base + kColD + d * 128;
                 for (int st = s; st < e_end; ++st) {
@@ -576,7 +577,7 @@ __global__ void __launch_bounds__(kNvThreads, 1) k_nvf4(const __grid_constant__ 
             if (nbuilt >= 1 && !dead) dead = !mbar_wait(b_empty, (nbuilt - 1) & 1, abort_flag, kNvWaitLimit);
             dead = __any_sync(0xffffffffu, dead);
             tc_fence_after();
-            if (!dead) build_b<PHASE>(p, sh, jd, K, sB, sfbb, cs + (nbuilt & 1) * ncap, tmem_base, bad);
+            if (!dead) build_b<PHASE, J>(p, sh, jd, K, sB, sfbb, cs + (nbuilt & 1) * ncap, tmem_base, bad);
             else {
                 named_bar_sync(2, 128);
                 named_bar_sync(2, 128);
@@ -595,7 +596,7 @@ __global__ void __launch_bounds__(kNvThreads, 1) k_nvf4(const __grid_constant__ 
             const float* csb = cs + (cur_b & 1) * ncap;
             const int item = s / w.spi;
             const int jd = item / w.tiles, tile = item - jd * w.tiles;
-            const int ne = sh.ucnt[jd], N = ne * kNvJ, npad = (N + 15) & ~15;
+            const int ne = sh.ucnt[jd], N = ne * J, npad = (N + 15) & ~15;
             const int d = pc & 1;
             const int row = tile * 128 + et;
             // the expert's tensor scales
@@ -623,7 +624,7 @@ __global__ void __launch_bounds__(kNvThreads, 1) k_nvf4(const __grid_constant__ 
 #pragma unroll
                             for (int u = 0; u < 16; ++u) {
                                 const int n = c0 + u;
-                                if (n < N) P[m][n / kNvJ] = fmaf(csb[n], __uint_as_float(v[u]), P[m][n / kNvJ]);
+                                if (n < N) P[m][n / J] = fmaf(csb[n], __uint_as_float(v[u]), P[m][n / J]);
                             }
                         }
                     }
@@ -721,14 +722,14 @@ int nv_sms() {
     return n;
 }
 
-template <int PHASE>
+template <int PHASE, int J>
 cudaError_t launch_nvf4(const FwdParams& p, cudaStream_t st) {
     NvArgs a;
     std::memset(&a, 0, sizeof(a));
     a.p = p;
-    a.ncap = (p.T * kNvJ + 15) & ~15;
+    a.ncap = (p.T * J + 15) & ~15;
     const size_t smem = nv_smem_bytes<PHASE>(p, a.ncap);
-    auto kern = k_nvf4<PHASE>;
+    auto kern = k_nvf4<PHASE, J>;
     cudaError_t e = ensure_smem(reinterpret_cast<const void*>(kern), smem);
     if (e != cudaSuccess) return e;
     const int grid = std::min(nv_sms(), kNvMaxCtas);
@@ -758,14 +759,20 @@ bool nvf4_usable(const FwdParams& p) {
     if (p.L > kNvMaxK || p.F > kNvMaxK) return false;
     if (p.rec_bytes % 16 || (reinterpret_cast<uintptr_t>(p.experts) & 15)) return false;
     if (nv_sms() > kNvMaxCtas) return false;
-    const int ncap = (p.T * kNvJ + 15) & ~15;
+    const int ncap = (p.T * (p.act == LMOE_ACT_NVFP4 ? kNvJW4A4 : kNvJExact) + 15) & ~15;
     return nv_smem_bytes<NV_GATEUP>(p, ncap) <= 227 * 1024 && nv_smem_bytes<NV_DOWN>(p, ncap) <= 227 * 1024;
 }
 
 // Workspace floats the phases' partial sums need (2 pieces per CTA).
 size_t nvf4_part_floats() { return (size_t)kNvMaxCtas * 2 * 2 * 1024; }
 
-cudaError_t run_nvf4_gateup(const FwdParams& p, cudaStream_t st) { return launch_nvf4<NV_GATEUP>(p, st); }
-cudaError_t run_nvf4_down(const FwdParams& p, cudaStream_t st) { return launch_nvf4<NV_DOWN>(p, st); }
+// W4A4 (p.act == LMOE_ACT_NVFP4): one E2M1 term per activation row, the
+// NVFP4 activation rule of include/lmoe.h; otherwise six terms (fp16-level).
+cudaError_t run_nvf4_gateup(const FwdParams& p, cudaStream_t st) {
+    return p.act == LMOE_ACT_NVFP4 ? launch_nvf4<NV_GATEUP, kNvJW4A4>(p, st) : launch_nvf4<NV_GATEUP, kNvJExact>(p, st);
+}
+cudaError_t run_nvf4_down(const FwdParams& p, cudaStream_t st) {
+    return p.act == LMOE_ACT_NVFP4 ? launch_nvf4<NV_DOWN, kNvJW4A4>(p, st) : launch_nvf4<NV_DOWN, kNvJExact>(p, st);
+}
 
 }  // namespace lmoe

@@ -23,6 +23,7 @@ struct __align__(64) TmaMaps {
 struct PrefillParams {
     int H, L, E, K, G, F, Fs, du_fmt, T;
     int efmt;            // expert records: LMOE_EXPERTS_NVFP4 or LMOE_EXPERTS_Q3K
+    int act;             // expert inputs: LMOE_ACT_FP16 or LMOE_ACT_NVFP4 (W4A4)
     // inputs
     const uint16_t* x;
     const uint16_t* router_w_bf16;
@@ -70,9 +71,18 @@ struct PrefillParams {
     __half* operm;       // [T*K][L] weighted expert outputs
     __half* s;           // [T][G][L]
     uint16_t* zsh;       // [2][T][Fs] shared-expert hidden as bf16 high and low parts
+    // W4A4: NVFP4 activations of hperm, then of zperm (one buffer serves both)
+    uint8_t* aq;         // codes [K/32][T*K][16]
+    uint32_t* asf;       // scale words [K/64][T*K]
+    float* aG;           // [T*K]
 };
 
 cudaError_t run_prefill_route(PrefillParams p, cudaStream_t st);
+cudaError_t run_act_quant(const __half* src, int n, int K, uint8_t* codes, uint32_t* sfw, float* G, cudaStream_t st);
+cudaError_t run_w4a4_gateup(const PrefillParams& p, const uint8_t* aq, const uint32_t* asf, const float* aG, int n,
+                            cudaStream_t st);
+cudaError_t run_w4a4_down(const PrefillParams& p, const uint8_t* aq, const uint32_t* asf, const float* aG, int n,
+                          cudaStream_t st);
 cudaError_t run_prefill_path(PrefillParams p, cudaStream_t st, void* memset_base, size_t memset_bytes,
                              void (*mark)(cudaStream_t));
 

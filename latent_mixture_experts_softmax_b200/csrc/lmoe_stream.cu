@@ -1165,7 +1165,7 @@ cudaError_t run_stream_path(const FwdParams& p, cudaStream_t st) {
     cudaError_t e = p.du_fmt == LMOE_Q8_0 ? launch_wstream<SP_DPROJ, LMOE_Q8_0>(p, P.d, T, st)
                               : launch_wstream<SP_DPROJ, LMOE_Q4_0>(p, P.d, T, st);
     if (e != cudaSuccess) return e;
-    if (nvf4_usable(p) && tensor_core_experts()) {
+    if (p.act == LMOE_ACT_NVFP4 || (nvf4_usable(p) && tensor_core_experts())) {
         // NVFP4 experts on the tensor cores, weights as stored
         if ((e = run_nvf4_gateup(p, st)) != cudaSuccess) return e;
         if ((e = run_nvf4_down(p, st)) != cudaSuccess) return e;

@@ -1136,10 +1136,20 @@ cudaError_t run_prefill_path(PrefillParams p, cudaStream_t st, void* memset_base
     if ((e = launch_gemm<G_DPROJ, kNtDense, 4, 0>(m_d, p, st, G * (L / 128) * ttiles)) != cudaSuccess) return e;
     mark(st);
     const int max_etiles = min(E, pairs) + pairs / kNtExpert + 1;
-    if ((e = launch_gemm<G_GATEUP, kNtExpert, 4, 8>(m_gu, p, st, (F / 64) * max_etiles)) != cudaSuccess) return e;
-    mark(st);
-    if ((e = launch_gemm<G_DOWN, kNtExpert, 4, 8>(m_down, p, st, (L / 128) * max_etiles)) != cudaSuccess) return e;
-    mark(st);
+    if (p.act == LMOE_ACT_NVFP4) {
+        // W4A4: h, then z, as NVFP4 activations, times the NVFP4 weights
+        if ((e = run_act_quant(p.hperm, pairs, L, p.aq, p.asf, p.aG, st)) != cudaSuccess) return e;
+        if ((e = run_w4a4_gateup(p, p.aq, p.asf, p.aG, pairs, st)) != cudaSuccess) return e;
+        mark(st);
+        if ((e = run_act_quant(p.zperm, pairs, F, p.aq, p.asf, p.aG, st)) != cudaSuccess) return e;
+        if ((e = run_w4a4_down(p, p.aq, p.asf, p.aG, pairs, st)) != cudaSuccess) return e;
+        mark(st);
+    } else {
+        if ((e = launch_gemm<G_GATEUP, kNtExpert, 4, 8>(m_gu, p, st, (F / 64) * max_etiles)) != cudaSuccess) return e;
+        mark(st);
+        if ((e = launch_gemm<G_DOWN, kNtExpert, 4, 8>(m_down, p, st, (L / 128) * max_etiles)) != cudaSuccess) return e;
+        mark(st);
+    }
     k_combine<<<T, 256, 0, st>>>(p);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
     mark(st);

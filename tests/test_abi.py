@@ -80,3 +80,17 @@ def test_stack_needs_gamma(L):
     layer = B.lmoe_layer(16, None, 16, 16, 16, 16, B.lmoe_shared(16, 16, 16), None)
     arr = (B.lmoe_layer * 1)(layer)
     assert L.lmoe_stack_forward(ctypes.byref(cfg), 1, arr, 16, 32, 4, 1e-6, 256, 1 << 30, None) == B.LMOE_ERR_ARG
+
+
+def test_w4a4_needs_nvfp4_records_and_128_multiples():
+    """lmoe_cfg.act_fmt = LMOE_ACT_NVFP4 (W4A4) runs on the tensor-core expert
+    kernels: NVFP4 records, latent and ffn multiples of 128 up to 2048."""
+    from parity import small_workload
+    ok = small_workload(4, latent=256, ffn=128, act_fmt="nvfp4")
+    assert B.lmoe_cfg_check(B.make_cfg(ok.shape)) == B.LMOE_OK
+    for kw in ({"ffn": 192}, {"latent": 2176}, {"expert_fmt": "q3k"}):
+        wl = small_workload(4, **{"latent": 256, "ffn": 128, "act_fmt": "nvfp4", **kw})
+        assert B.lmoe_cfg_check(B.make_cfg(wl.shape)) == B.LMOE_ERR_UNSUPPORTED, kw
+    cfg = B.make_cfg(ok.shape)
+    cfg.act_fmt = 2
+    assert B.lmoe_cfg_check(cfg) == B.LMOE_ERR_UNSUPPORTED
