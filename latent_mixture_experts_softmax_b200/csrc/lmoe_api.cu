@@ -130,7 +130,7 @@ WsLayout ws_layout(const lmoe_cfg& c, int T) {
         L.p_uexp = take(nu * 4);
         L.p_ucnt = take(nu * 4);
         L.p_uoff = take(nu * 4);
-        L.p_etile = take((nu + TK / kNtExpert + 1) * 8);
+        L.p_etile = take((nu + TK / kNtExpert + 1) * 16);
         L.p_slot_pair = take(TK * 4);
         L.p_pair_slot = take(TK * 4);
         L.p_idx = take(TK * 4);
@@ -254,7 +254,7 @@ int run_prefill(const lmoe_cfg& c, const FwdParams& f, const WsLayout& L, void* 
     p.uexp = reinterpret_cast<int32_t*>(b + L.p_uexp);
     p.ucnt = reinterpret_cast<int32_t*>(b + L.p_ucnt);
     p.uoff = reinterpret_cast<int32_t*>(b + L.p_uoff);
-    p.etile = reinterpret_cast<int2*>(b + L.p_etile);
+    p.etile = reinterpret_cast<int4*>(b + L.p_etile);
     p.slot_pair = reinterpret_cast<int32_t*>(b + L.p_slot_pair);
     p.pair_slot = reinterpret_cast<int32_t*>(b + L.p_pair_slot);
     p.xh = reinterpret_cast<__half*>(b + L.p_xh);

@@ -60,7 +60,7 @@ struct PrefillParams {
     int32_t* uexp;       // [min(E, T*K)]
     int32_t* ucnt;
     int32_t* uoff;
-    int2* etile;         // expert token tiles {distinct index, first row}
+    int4* etile;         // expert token tiles {expert, first slot, slots (<= 128), distinct index}
     int32_t* slot_pair;  // [T*K]
     int32_t* pair_slot;  // [T*K]
     __half* xh;          // [T][H]   fp16 block input

@@ -76,12 +76,11 @@ struct Sched {
         if (KIND == G_GATEUP || KIND == G_DOWN) {
             // consecutive tiles share the expert's token rows
             const int et = i / mt, m = i % mt;
-            const int2 d = p.etile[et];
-            const int j = d.x, n0 = d.y;
-            t.mat = __ldcg(p.uexp + j);
+            const int4 d = __ldcg(p.etile + et);
+            t.mat = d.x;
             t.m0 = m * (KIND == G_GATEUP ? 64 : 128);
-            t.b0 = __ldcg(p.uoff + j) + n0;
-            t.n = min(NT, __ldcg(p.ucnt + j) - n0);
+            t.b0 = d.y;
+            t.n = min(NT, d.z);
             t.nq = 0;
         } else {
             // consecutive tiles share the weight tile (token tiles fastest)
@@ -953,7 +952,7 @@ __global__ void k_bucket_scan(const PrefillParams p) {
             p.uexp[u] = e;
             p.ucnt[u] = ce;
             p.uoff[u] = o;
-            for (int n0 = 0; n0 < ce; n0 += kNtExpert) p.etile[tt++] = make_int2(u, n0);
+            for (int n0 = 0; n0 < ce; n0 += kNtExpert) p.etile[tt++] = make_int4(e, o + n0, min(kNtExpert, ce - n0), u);
             ++u;
         }
         o += ce;

@@ -19,15 +19,20 @@
 //
 // The GEMM (one CTA per SM, persistent over its items): an item is one
 // expert token tile (at most 128 slots, from the tile list the bucketing
-// kernels built) times one 128-row tile of the weight matrix (gate and up
-// together for gate/up), over the whole K in 256-column stages.  Warps:
-//   0-3  loaders: cp.async copies of each stage's weight codes, weight scale
-//        words, activation codes and activation scale words into a ring of
-//        shared-memory slots; once a stage has landed, each warp copies the
-//        stage's weight and activation scale words to its 32-lane TMEM
-//        subpartition (scale columns 4k + b: rows / slots b*32 .. b*32+31)
-//   4-7  epilogue: accumulators (TMEM) -> * G * ts -> SwiGLU (gate/up) or
-//        routing weight (down) -> fp16 zperm / operm
+// kernels built) times one 128-row tile of the weight operand, over the whole
+// K in 256-column stages.  For gate/up the 128 rows are 64 output rows of
+// both matrices, interleaved by TMEM subpartition: lanes 0-15 of
+// subpartition b hold gate rows m0 + 16b .. m0 + 16b + 15 and lanes 16-31 the
+// up rows of the same outputs, so the SwiGLU pairs meet by a warp shuffle.
+// Warps:
+//   0-3  loaders: per stage, thread r copies operand row r (its codes and
+//        E4M3 scale words) and activation slot r with cp.async into a ring of
+//        STAGES shared-memory slots, STAGES - 2 stages ahead of the MMA (one
+//        slot of slack); once a stage has landed, each warp copies its
+//        weight and activation scale words to its 32-lane TMEM subpartition
+//        (scale columns 4k + b: rows / slots b*32 .. b*32+31)
+//   4-7  epilogue: accumulators (TMEM, two buffers) -> * G * ts -> SwiGLU
+//        (gate/up) or routing weight (down) -> fp16 zperm / operm
 //   8    MMA issue (one thread), TMEM allocation
 
 #include <cstring>
@@ -45,11 +50,13 @@ constexpr uint32_t kW4TmemCols = 512;
 constexpr int kW4CodeBox = 128 * 128;    // bytes: 8 chunks x 128 rows x 16 B
 constexpr int kW4ScaleBox = 4 * 128 * 4; // bytes: 4 64-column groups x 128 rows x 4 B
 
-template <int KIND>
-struct W4Geom {
-    static constexpr int NM = KIND == G_GATEUP ? 2 : 1;
-    static constexpr int STAGES = KIND == G_GATEUP ? 3 : 4;
-};
+// 256-column stages of 36 KB (weight codes and scale words of 128 rows,
+// activation codes and scale words of up to 128 slots); six fill 216 KB.
+constexpr int kW4Stages = 6;
+constexpr int kW4Ahead = kW4Stages - 2;
+constexpr int kW4StageBytes = 2 * (kW4CodeBox + kW4ScaleBox);
+constexpr uint32_t kW4ColSfa = 256, kW4ColSfb = 256 + 16 * kW4Stages;
+static_assert(kW4ColSfb + 16 * kW4Stages <= kW4TmemCols, "TMEM columns");
 
 struct __align__(64) W4Args {
     PrefillParams p;
@@ -177,29 +184,25 @@ __global__ void __launch_bounds__(256) k_act_quant(const __half* src, int n, int
 
 template <int KIND>
 __global__ void __launch_bounds__(kW4Threads, 1) k_w4a4(const __grid_constant__ W4Args a) {
-    using Geo = W4Geom<KIND>;
-    constexpr int NM = Geo::NM, STAGES = Geo::STAGES;
-    constexpr int LA = STAGES - 1;
+    constexpr int STAGES = kW4Stages, LA = kW4Ahead;
     const PrefillParams& p = a.p;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
     const int K = KIND == G_GATEUP ? p.L : p.F;
     const int R = KIND == G_GATEUP ? p.F : p.L;
-    const int mt = R / 128;
-    uint8_t* sA = smem;                                      // [slot][m] weight codes
-    uint8_t* sSA = sA + STAGES * NM * kW4CodeBox;            // [slot][m] weight scale words [4][128]
-    uint8_t* sB = sSA + STAGES * NM * kW4ScaleBox;           // [slot] activation codes [8][128][16]
-    uint8_t* sSB = sB + STAGES * kW4CodeBox;                 // [slot] activation scale words [4][128]
-    float* meta = reinterpret_cast<float*>(sSB + STAGES * kW4ScaleBox);   // [2][128]: G, routing weight
-    uint64_t* bars = reinterpret_cast<uint64_t*>(meta + 256);
+    const int mt = KIND == G_GATEUP ? R / 64 : R / 128;
+    // slot s: weight codes [8][128][16] | weight scale words [4][128] |
+    //         activation codes [8][128][16] | activation scale words [4][128]
+    uint8_t* ring = smem;
+    float* meta = reinterpret_cast<float*>(ring + STAGES * kW4StageBytes);   // [2 buffers][G | weight][128]
+    uint64_t* bars = reinterpret_cast<uint64_t*>(meta + 512);
     uint64_t* full = bars;               // [STAGES] (4 loader warps)
     uint64_t* empty = full + STAGES;     // [STAGES] (commit)
-    uint64_t* tfull = empty + STAGES;    // item accumulated (commit)
-    uint64_t* tempty = tfull + 1;        // accumulator read (4 epilogue warps)
-    uint64_t* final_bar = tempty + 1;
+    uint64_t* tfull = empty + STAGES;    // [2] item accumulated (commit)
+    uint64_t* tempty = tfull + 2;        // [2] accumulator read (4 epilogue warps)
+    uint64_t* final_bar = tempty + 2;
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(final_bar + 1);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
-    const uint32_t col_sfa = 256, col_sfb = 256 + STAGES * NM * 16;
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     if (threadIdx.x == 0) {
@@ -207,8 +210,10 @@ __global__ void __launch_bounds__(kW4Threads, 1) k_w4a4(const __grid_constant__ 
             mbar_init(&full[s], 4);
             mbar_init(&empty[s], 1);
         }
-        mbar_init(tfull, 1);
-        mbar_init(tempty, 4);
+        for (int b = 0; b < 2; ++b) {
+            mbar_init(&tfull[b], 1);
+            mbar_init(&tempty[b], 4);
+        }
         mbar_init(final_bar, 1);
         *abort_flag = 0;
         fence_barrier_init();
@@ -228,58 +233,72 @@ __global__ void __launch_bounds__(kW4Threads, 1) k_w4a4(const __grid_constant__ 
     const int n_items = __ldcg(p.n_etiles) * mt;
     const int spi = (K + 255) / 256;
     const size_t nq = (size_t)p.L * p.F / 2, ns = (size_t)p.L * p.F / 16;
-    auto item_of = [&](int i, int& mat, int& m0, int& b0, int& nrow) {
-        const int et = i / mt, t = i - et * mt;
-        const int2 d = p.etile[et];
-        mat = __ldcg(p.uexp + d.x);
-        m0 = t * 128;
-        b0 = __ldcg(p.uoff + d.x) + d.y;
-        nrow = min(128, __ldcg(p.ucnt + d.x) - d.y);
+    // item i: the expert tile {expert, first slot, slots} (fetched one item
+    // ahead by every role) and the row tile
+    auto tile_of = [&](int i) -> int4 {
+        return i < n_items ? __ldcg(p.etile + i / mt) : make_int4(0, 0, 0, 0);
     };
+    auto m0_of = [&](int i) { return (i % mt) * (KIND == G_GATEUP ? 64 : 128); };
 
     if (warp < 4) {
         // -------------------------------------------------------- loaders
-        const int lt = threadIdx.x;
+        const int r = threadIdx.x;    // operand row and activation slot of this thread
         bool dead = false;
         int n_st = 0;
         for (int i = blockIdx.x; i < n_items; i += gridDim.x) n_st += spi;
         int it_item = blockIdx.x, q = 0;
-        int mat = 0, m0 = 0, b0 = 0, nrow = 0;
-        if (it_item < n_items) item_of(it_item, mat, m0, b0, nrow);
+        const uint8_t* wq = nullptr;   // this row's codes, chunk 0
+        const uint8_t* wsc = nullptr;  // this row's scale words, group 0
+        const uint8_t* aq = nullptr;   // this slot's codes, chunk 0 (nullptr: past the tile)
+        const uint32_t* as = nullptr;
+        int4 nxt = tile_of(it_item);
+        auto start_item = [&]() {
+            const int4 d = nxt;
+            nxt = tile_of(it_item + gridDim.x);
+            const int mat = d.x, b0 = d.y, nrow = d.z, m0 = m0_of(it_item);
+            const uint8_t* rec = p.experts + (size_t)mat * p.rec_bytes;
+            int m = 2, row = m0 + r;
+            if (KIND == G_GATEUP) {
+                m = (r & 31) >> 4;                                   // 0 gate, 1 up
+                row = m0 + 16 * (r >> 5) + (r & 15);
+            }
+            wq = rec + m * nq + (size_t)row * 16;
+            wsc = rec + 3 * nq + m * ns + (size_t)row * 4;
+            aq = r < nrow ? a.aq + (size_t)(b0 + r) * 16 : nullptr;
+            as = r < nrow ? a.asf + b0 + r : nullptr;
+        };
+        if (it_item < n_items) start_item();
+        const size_t wstep = (size_t)R * 16, sstep = (size_t)R * 4, astep = (size_t)a.n * 16;
         for (int i = 0; i < n_st + LA; ++i) {
             if (i < n_st) {
                 const int slot = i % STAGES;
                 if (!dead) dead = !mbar_wait(&empty[slot], ((i / STAGES) & 1) ^ 1, abort_flag, kW4WaitLimit);
                 if (!dead) {
-                    const uint8_t* rec = p.experts + (size_t)mat * p.rec_bytes;
-                    const int nch = min(8, K / 32 - q * 8), ncp = min(4, K / 64 - q * 4);
-                    for (int x = lt; x < NM * nch * 128; x += 128) {
-                        const int m = x / (nch * 128), rem = x - m * nch * 128, c = rem >> 7, r = rem & 127;
-                        const uint8_t* qm = rec + (KIND == G_GATEUP ? m : 2) * nq;
-                        cp16(sA + (slot * NM + m) * kW4CodeBox + c * 2048 + r * 16,
-                             qm + ((size_t)(q * 8 + c) * R + m0 + r) * 16);
-                    }
-                    for (int x = lt; x < NM * ncp * 32; x += 128) {
-                        const int m = x / (ncp * 32), rem = x - m * ncp * 32, cp = rem >> 5, r4 = rem & 31;
-                        const uint8_t* sm = rec + 3 * nq + (KIND == G_GATEUP ? m : 2) * ns;
-                        cp16(sSA + (slot * NM + m) * kW4ScaleBox + cp * 512 + r4 * 16,
-                             sm + ((size_t)(q * 4 + cp) * R + m0 + 4 * r4) * 4);
-                    }
-                    // activation rows b0 .. b0 + nrow (the tile's slots)
-                    for (int x = lt; x < nch * 128; x += 128) {
-                        const int c = x >> 7, s = x & 127;
-                        if (s < nrow)
-                            cp16(sB + slot * kW4CodeBox + c * 2048 + s * 16, a.aq + ((size_t)(q * 8 + c) * a.n + b0 + s) * 16);
-                    }
-                    for (int x = lt; x < ncp * 128; x += 128) {
-                        const int cp = x >> 7, s = x & 127;
-                        if (s < nrow) cp4(sSB + slot * kW4ScaleBox + cp * 512 + s * 4, a.asf + (size_t)(q * 4 + cp) * a.n + b0 + s);
+                    uint8_t* sl = ring + slot * kW4StageBytes;
+                    const int nch = min(8, K / 32 - q * 8), ngr = min(4, K / 64 - q * 4);
+                    const uint8_t* wqq = wq + (size_t)(q * 8) * wstep;
+                    const uint8_t* wss = wsc + (size_t)(q * 4) * sstep;
+#pragma unroll
+                    for (int c = 0; c < 8; ++c)
+                        if (c < nch) cp16(sl + c * 2048 + r * 16, wqq + c * wstep);
+#pragma unroll
+                    for (int g = 0; g < 4; ++g)
+                        if (g < ngr) cp4(sl + kW4CodeBox + g * 512 + r * 4, wss + g * sstep);
+                    if (aq) {
+                        const uint8_t* aqq = aq + (size_t)(q * 8) * astep;
+                        const uint32_t* ass = as + (size_t)(q * 4) * a.n;
+#pragma unroll
+                        for (int c = 0; c < 8; ++c)
+                            if (c < nch) cp16(sl + kW4CodeBox + kW4ScaleBox + c * 2048 + r * 16, aqq + c * astep);
+#pragma unroll
+                        for (int g = 0; g < 4; ++g)
+                            if (g < ngr) cp4(sl + 2 * kW4CodeBox + kW4ScaleBox + g * 512 + r * 4, ass + (size_t)g * a.n);
                     }
                 }
                 if (++q == spi) {
                     q = 0;
                     it_item += gridDim.x;
-                    if (it_item < n_items) item_of(it_item, mat, m0, b0, nrow);
+                    if (it_item < n_items) start_item();
                 }
             }
             cp_commit();
@@ -290,26 +309,22 @@ __global__ void __launch_bounds__(kW4Threads, 1) k_w4a4(const __grid_constant__ 
                 dead = __any_sync(0xffffffffu, dead);
                 named_bar_sync(1, 128);
                 if (!dead) {
-                    // weight scales: lane a of warp w holds rows a + 32b in columns 4k + b
-                    const uint32_t* src = reinterpret_cast<const uint32_t*>(sSA);
-#pragma unroll
-                    for (int m = 0; m < NM; ++m) {
-                        uint32_t v[16];
-#pragma unroll
-                        for (int k = 0; k < 4; ++k)
-#pragma unroll
-                            for (int bb = 0; bb < 4; ++bb) v[k * 4 + bb] = src[(slot * NM + m) * 512 + k * 128 + lane + 32 * bb];
-                        __syncwarp();
-                        tst_x16(tmem_base + ((uint32_t)(32 * warp) << 16) + col_sfa + (uint32_t)((slot * NM + m) * 16), v);
-                    }
-                    const uint32_t* srcb = reinterpret_cast<const uint32_t*>(sSB);
-                    uint32_t v[16];
+                    // scale words: lane a of warp w holds rows / slots a + 32b in columns 4k + b
+                    const uint32_t* sw = reinterpret_cast<const uint32_t*>(ring + slot * kW4StageBytes + kW4CodeBox);
+                    const uint32_t* sa =
+                        reinterpret_cast<const uint32_t*>(ring + slot * kW4StageBytes + 2 * kW4CodeBox + kW4ScaleBox);
+                    uint32_t v[16], u[16];
 #pragma unroll
                     for (int k = 0; k < 4; ++k)
 #pragma unroll
-                        for (int bb = 0; bb < 4; ++bb) v[k * 4 + bb] = srcb[slot * 512 + k * 128 + lane + 32 * bb];
+                        for (int bb = 0; bb < 4; ++bb) {
+                            v[k * 4 + bb] = sw[k * 128 + lane + 32 * bb];
+                            u[k * 4 + bb] = sa[k * 128 + lane + 32 * bb];
+                        }
+                    const uint32_t lanes = (uint32_t)(32 * warp) << 16;
                     __syncwarp();
-                    tst_x16(tmem_base + ((uint32_t)(32 * warp) << 16) + col_sfb + (uint32_t)(slot * 16), v);
+                    tst_x16(tmem_base + lanes + kW4ColSfa + (uint32_t)(slot * 16), v);
+                    tst_x16(tmem_base + lanes + kW4ColSfb + (uint32_t)(slot * 16), u);
                     __syncwarp();
                     tst_wait();
                     tc_fence_before();
@@ -317,105 +332,128 @@ __global__ void __launch_bounds__(kW4Threads, 1) k_w4a4(const __grid_constant__ 
                 __syncwarp();
                 if (lane == 0 && !dead) mbar_arrive(&full[slot]);
             }
-            if (i == LA - 1) {
-                grid_dep_wait();
-                grid_dep_launch();
-            }
         }
         cp_wait<0>();
     } else if (warp == 8) {
         // -------------------------------------------------------- MMA issue
-        grid_dep_wait();
-        grid_dep_launch();
         if (lane == 0) {
             uint32_t it = 0, pc = 0;
             bool dead = false, issued = false;
+            int4 nxt = tile_of(blockIdx.x);
             for (int i = blockIdx.x; i < n_items && !dead; i += gridDim.x, ++pc) {
-                int mat, m0, b0, nrow;
-                item_of(i, mat, m0, b0, nrow);
-                const int npad = (nrow + 15) & ~15;
-                const uint32_t idesc = idesc_fp4(npad);
-                if (!mbar_wait(tempty, (pc & 1) ^ 1, abort_flag, kW4WaitLimit)) { dead = true; break; }
+                const int nrow = nxt.z;
+                nxt = tile_of(i + gridDim.x);
+                const uint32_t idesc = idesc_fp4((nrow + 15) & ~15);
+                const uint32_t acc = pc & 1;
+                if (!mbar_wait(&tempty[acc], ((pc >> 1) & 1) ^ 1, abort_flag, kW4WaitLimit)) { dead = true; break; }
                 tc_fence_after();
                 for (int q = 0; q < spi; ++q, ++it) {
                     const int slot = it % STAGES;
                     if (!mbar_wait(&full[slot], (it / STAGES) & 1, abort_flag, kW4WaitLimit)) { dead = true; break; }
                     tc_fence_after();
+                    const uint32_t sl = smem_u32(ring + slot * kW4StageBytes);
                     const int kk = min(4, (K - q * 256) / 64);
                     for (int k = 0; k < kk; ++k) {
-                        const uint64_t bdesc = sdesc_plain(smem_u32(sB + slot * kW4CodeBox) + (uint32_t)(k * 4096), 2048, 128);
-#pragma unroll
-                        for (int m = 0; m < NM; ++m) {
-                            const uint64_t adesc =
-                                sdesc_plain(smem_u32(sA + (slot * NM + m) * kW4CodeBox) + (uint32_t)(k * 4096), 2048, 128);
-                            umma_fp4(tmem_base + (uint32_t)(m * 128), adesc, bdesc, idesc,
-                                     tmem_base + col_sfa + (uint32_t)((slot * NM + m) * 16 + 4 * k),
-                                     tmem_base + col_sfb + (uint32_t)(slot * 16 + 4 * k), (q > 0 || k > 0) ? 1u : 0u);
-                        }
+                        const uint64_t adesc = sdesc_plain(sl + (uint32_t)(k * 4096), 2048, 128);
+                        const uint64_t bdesc = sdesc_plain(sl + kW4CodeBox + kW4ScaleBox + (uint32_t)(k * 4096), 2048, 128);
+                        umma_fp4(tmem_base + acc * 128, adesc, bdesc, idesc, tmem_base + kW4ColSfa + (uint32_t)(slot * 16 + 4 * k),
+                                 tmem_base + kW4ColSfb + (uint32_t)(slot * 16 + 4 * k), (q > 0 || k > 0) ? 1u : 0u);
                     }
                     issued = true;
                     umma_commit(&empty[slot]);
                 }
                 if (dead) break;
-                umma_commit(tfull);
+                umma_commit(&tfull[acc]);
             }
             if (issued) {
+                // every MMA done before TMEM is freed, even after an abort
                 umma_commit(final_bar);
-                volatile int dummy = 0;
-                mbar_wait(final_bar, 0, &dummy, kW4WaitLimit);
+                volatile int no_abort = 0;
+                mbar_wait(final_bar, 0, &no_abort, kW4WaitLimit);
             }
         }
         __syncwarp();
     } else {
         // -------------------------------------------------------- epilogue (warps 4-7)
-        grid_dep_wait();
-        grid_dep_launch();
         const int et = threadIdx.x - 128;
         const int sub = warp & 3;
         uint32_t pc = 0;
         bool dead = false, bad = false;
-        for (int i = blockIdx.x; i < n_items; i += gridDim.x, ++pc) {
-            int mat, m0, b0, nrow;
-            item_of(i, mat, m0, b0, nrow);
-            // per-slot scales of the tile: G, and the routing weight (down)
-            if (et < nrow) {
-                meta[et] = __ldcg(a.aG + b0 + et);
-                if (KIND == G_DOWN) meta[128 + et] = __ldcg(p.w + __ldcg(p.slot_pair + b0 + et));
+        // the next item's tile, per-slot scales (G; the routing weight for
+        // down) and tensor scales are fetched while this item drains
+        int4 cur = tile_of(blockIdx.x), nxt = tile_of(blockIdx.x + gridDim.x);
+        float nG = 0.f, nW = 0.f, nts0 = 0.f, nts1 = 0.f;
+        auto fetch = [&](const int4& d, float& g, int& sp, float& t0, float& t1) {
+            if (et < d.z) {
+                g = __ldcg(a.aG + d.y + et);
+                if (KIND == G_DOWN) sp = __ldcg(p.slot_pair + d.y + et);
             }
-            const float* tsp = reinterpret_cast<const float*>(p.experts + (size_t)mat * p.rec_bytes + 3 * nq + 3 * ns);
-            const float ts0 = __ldg(tsp + (KIND == G_GATEUP ? 0 : 2)), ts1 = __ldg(tsp + 1);
+            const float* tsp = reinterpret_cast<const float*>(p.experts + (size_t)d.x * p.rec_bytes + 3 * nq + 3 * ns);
+            t0 = __ldg(tsp + (KIND == G_GATEUP ? 0 : 2));
+            t1 = __ldg(tsp + 1);
+        };
+        int nsp = 0;
+        if (blockIdx.x < n_items) {
+            fetch(cur, nG, nsp, nts0, nts1);
+            if (KIND == G_DOWN && et < cur.z) nW = __ldcg(p.w + nsp);
+        }
+        for (int i = blockIdx.x; i < n_items; i += gridDim.x, ++pc) {
+            const int mat = cur.x, b0 = cur.y, nrow = cur.z, m0 = m0_of(i);
+            (void)mat;
+            const uint32_t acc = pc & 1;
+            float* mG = meta + acc * 256;
+            if (et < nrow) {
+                mG[et] = nG;
+                if (KIND == G_DOWN) mG[128 + et] = nW;
+            }
+            const float ts0 = nts0, ts1 = nts1;
+            const bool more = i + gridDim.x < n_items;
+            if (more) fetch(nxt, nG, nsp, nts0, nts1);
             named_bar_sync(2, 128);
-            if (!dead) dead = !mbar_wait(tfull, pc & 1, abort_flag, kW4WaitLimit);
+            if (!dead) dead = !mbar_wait(&tfull[acc], (pc >> 1) & 1, abort_flag, kW4WaitLimit);
             dead = __any_sync(0xffffffffu, dead);
             if (!dead) {
                 tc_fence_after();
-                const uint32_t taddr = tmem_base + ((uint32_t)(32 * sub) << 16);
-                const int row = m0 + et;
+                const uint32_t taddr = tmem_base + ((uint32_t)(32 * sub) << 16) + acc * 128;
+                const bool hi = lane >= 16;
+                const int row = KIND == G_GATEUP ? m0 + 16 * sub + (lane & 15) : m0 + 32 * sub + lane;
                 for (int c0 = 0; c0 < nrow; c0 += 16) {
-                    uint32_t vg[16], vu[16];
+                    uint32_t v[16];
                     __syncwarp();
-                    tld_x16(taddr + c0, vg);
-                    if (NM == 2) tld_x16(taddr + 128 + c0, vu);
+                    tld_x16(taddr + c0, v);
                     asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+                    if (KIND == G_GATEUP) {
+                        // lanes < 16: gate of columns c0..c0+7, partner's up; lanes >= 16:
+                        // partner's gate of columns c0+8..c0+15, own up
 #pragma unroll
-                    for (int u = 0; u < 16; ++u) {
-                        const int s = c0 + u;
-                        if (s >= nrow) break;
-                        const float g = meta[s];
-                        if (KIND == G_GATEUP) {
-                            const float gv = __uint_as_float(vg[u]) * g * ts0, uv = __uint_as_float(vu[u]) * g * ts1;
-                            p.zperm[(size_t)(b0 + s) * p.F + row] = half_checked(silu(gv) * uv, bad);
-                        } else {
-                            const float o = __uint_as_float(vg[u]) * g * ts0 * meta[128 + s];
-                            p.operm[(size_t)(b0 + s) * p.L + row] = half_checked(o, bad);
+                        for (int u = 0; u < 8; ++u) {
+                            const float mine = __uint_as_float(hi ? v[u + 8] : v[u]);
+                            const float other = __shfl_xor_sync(0xffffffffu, __uint_as_float(hi ? v[u] : v[u + 8]), 16);
+                            const int s = c0 + u + (hi ? 8 : 0);
+                            if (s < nrow) {
+                                const float g = mG[s];
+                                const float gv = (hi ? other : mine) * g * ts0, uv = (hi ? mine : other) * g * ts1;
+                                p.zperm[(size_t)(b0 + s) * p.F + row] = half_checked(silu(gv) * uv, bad);
+                            }
+                        }
+                    } else {
+#pragma unroll
+                        for (int u = 0; u < 16; ++u) {
+                            const int s = c0 + u;
+                            if (s < nrow) {
+                                const float o = __uint_as_float(v[u]) * mG[s] * ts0 * mG[128 + s];
+                                p.operm[(size_t)(b0 + s) * p.L + row] = half_checked(o, bad);
+                            }
                         }
                     }
                 }
                 tc_fence_before();
             }
             __syncwarp();
-            if (lane == 0 && !dead) mbar_arrive(tempty);
-            named_bar_sync(2, 128);
+            if (lane == 0 && !dead) mbar_arrive(&tempty[acc]);
+            if (KIND == G_DOWN && more && et < nxt.z) nW = __ldcg(p.w + nsp);
+            cur = nxt;
+            nxt = tile_of(i + 2 * gridDim.x);
         }
         report_range(p.ctrl, bad);
     }
@@ -441,12 +479,7 @@ int w4_sms() {
     return n;
 }
 
-template <int KIND>
-size_t w4_smem() {
-    using Geo = W4Geom<KIND>;
-    return 1024 + (size_t)Geo::STAGES * (Geo::NM * (kW4CodeBox + kW4ScaleBox) + kW4CodeBox + kW4ScaleBox) + 256 * 4 +
-           (2 * Geo::STAGES + 3) * 8 + 16;
-}
+constexpr size_t kW4Smem = 1024 + (size_t)kW4Stages * kW4StageBytes + 512 * 4 + (2 * kW4Stages + 5) * 8 + 16;
 
 template <int KIND>
 cudaError_t launch_w4a4(const PrefillParams& p, const uint8_t* aq, const uint32_t* asf, const float* aG, int n,
@@ -458,7 +491,7 @@ cudaError_t launch_w4a4(const PrefillParams& p, const uint8_t* aq, const uint32_
     a.asf = asf;
     a.aG = aG;
     a.n = n;
-    const size_t smem = w4_smem<KIND>();
+    const size_t smem = kW4Smem;
     auto kern = k_w4a4<KIND>;
     cudaError_t e = ensure_smem(reinterpret_cast<const void*>(kern), smem);
     if (e != cudaSuccess) return e;
