@@ -59,7 +59,7 @@ struct WsLayout {
     size_t x16, h16, zsh, zsh16, o16w, z16, s16, ypart, xio, yio, xa, xb;
     // tensor-core path
     size_t p_zero_begin, p_tgmask, p_cnt, p_fill, p_dhit, p_n_etiles, p_zero_end;
-    size_t p_n_unique, p_off, p_uexp, p_ucnt, p_uoff, p_etile, p_slot_pair, p_pair_slot, p_idx, p_w, p_logits;
+    size_t p_n_unique, p_off, p_uexp, p_ucnt, p_uoff, p_etile, p_slot_pair, p_wslot, p_pair_slot, p_idx, p_w, p_logits;
     size_t p_xh, p_xr, p_xr_lo, p_hperm, p_zperm, p_operm, p_s, p_zsh, p_aq, p_asf, p_aG;
     size_t total;
 };
@@ -132,6 +132,7 @@ WsLayout ws_layout(const lmoe_cfg& c, int T) {
         L.p_uoff = take(nu * 4);
         L.p_etile = take((nu + TK / kNtExpert + 1) * 16);
         L.p_slot_pair = take(TK * 4);
+        L.p_wslot = take(TK * 4);
         L.p_pair_slot = take(TK * 4);
         L.p_idx = take(TK * 4);
         L.p_w = take(TK * 4);
@@ -256,6 +257,7 @@ int run_prefill(const lmoe_cfg& c, const FwdParams& f, const WsLayout& L, void* 
     p.uoff = reinterpret_cast<int32_t*>(b + L.p_uoff);
     p.etile = reinterpret_cast<int4*>(b + L.p_etile);
     p.slot_pair = reinterpret_cast<int32_t*>(b + L.p_slot_pair);
+    p.wslot = reinterpret_cast<float*>(b + L.p_wslot);
     p.pair_slot = reinterpret_cast<int32_t*>(b + L.p_pair_slot);
     p.xh = reinterpret_cast<__half*>(b + L.p_xh);
     if (f.gamma) {

@@ -62,6 +62,7 @@ struct PrefillParams {
     int32_t* uoff;
     int4* etile;         // expert token tiles {expert, first slot, slots (<= 128), distinct index}
     int32_t* slot_pair;  // [T*K]
+    float* wslot;        // [T*K] routing weight of each expert slot
     int32_t* pair_slot;  // [T*K]
     __half* xh;          // [T][H]   fp16 block input
     uint16_t* xr;        // [T][H]   bf16 normalised input (stack) or nullptr

@@ -776,7 +776,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1) k_umma_gemm(const __grid_cons
                         if (i0 + 128 * u < cur.t.n) mmask[i0 + 128 * u] = v[u];
                 }
             } else if (KIND == G_DOWN) {
-                for (int i = threadIdx.x; i < cur.t.n; i += 128) xchg[i] = __ldg(p.w + __ldg(p.slot_pair + cur.t.b0 + i));
+                for (int i = threadIdx.x; i < cur.t.n; i += 128) xchg[i] = __ldcg(p.wslot + cur.t.b0 + i);
             }
             if ((KIND == G_GATEUP || KIND == G_DOWN) && threadIdx.x < 3) {
                 // the expert's tensor scales (gate, up, down) from its record
@@ -970,6 +970,7 @@ __global__ void k_bucket_scatter(const PrefillParams p) {
     const int slot = p.off[e] + atomicAdd(p.fill + e, 1);
     p.slot_pair[slot] = i;
     p.pair_slot[i] = slot;
+    p.wslot[slot] = p.w[i];
 }
 
 // s[t][g] = sum over the token's experts of group g of o (already weighted);

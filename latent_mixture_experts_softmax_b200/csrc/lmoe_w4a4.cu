@@ -383,20 +383,16 @@ __global__ void __launch_bounds__(kW4Threads, 1) k_w4a4(const __grid_constant__ 
         // down) and tensor scales are fetched while this item drains
         int4 cur = tile_of(blockIdx.x), nxt = tile_of(blockIdx.x + gridDim.x);
         float nG = 0.f, nW = 0.f, nts0 = 0.f, nts1 = 0.f;
-        auto fetch = [&](const int4& d, float& g, int& sp, float& t0, float& t1) {
+        auto fetch = [&](const int4& d, float& g, float& w, float& t0, float& t1) {
             if (et < d.z) {
                 g = __ldcg(a.aG + d.y + et);
-                if (KIND == G_DOWN) sp = __ldcg(p.slot_pair + d.y + et);
+                if (KIND == G_DOWN) w = __ldcg(p.wslot + d.y + et);
             }
             const float* tsp = reinterpret_cast<const float*>(p.experts + (size_t)d.x * p.rec_bytes + 3 * nq + 3 * ns);
             t0 = __ldg(tsp + (KIND == G_GATEUP ? 0 : 2));
             t1 = __ldg(tsp + 1);
         };
-        int nsp = 0;
-        if (blockIdx.x < n_items) {
-            fetch(cur, nG, nsp, nts0, nts1);
-            if (KIND == G_DOWN && et < cur.z) nW = __ldcg(p.w + nsp);
-        }
+        if (blockIdx.x < n_items) fetch(cur, nG, nW, nts0, nts1);
         for (int i = blockIdx.x; i < n_items; i += gridDim.x, ++pc) {
             const int mat = cur.x, b0 = cur.y, nrow = cur.z, m0 = m0_of(i);
             (void)mat;
@@ -408,7 +404,7 @@ __global__ void __launch_bounds__(kW4Threads, 1) k_w4a4(const __grid_constant__ 
             }
             const float ts0 = nts0, ts1 = nts1;
             const bool more = i + gridDim.x < n_items;
-            if (more) fetch(nxt, nG, nsp, nts0, nts1);
+            if (more) fetch(nxt, nG, nW, nts0, nts1);
             named_bar_sync(2, 128);
             if (!dead) dead = !mbar_wait(&tfull[acc], (pc >> 1) & 1, abort_flag, kW4WaitLimit);
             dead = __any_sync(0xffffffffu, dead);
@@ -451,7 +447,6 @@ __global__ void __launch_bounds__(kW4Threads, 1) k_w4a4(const __grid_constant__ 
             }
             __syncwarp();
             if (lane == 0 && !dead) mbar_arrive(&tempty[acc]);
-            if (KIND == G_DOWN && more && et < nxt.z) nW = __ldcg(p.w + nsp);
             cur = nxt;
             nxt = tile_of(i + 2 * gridDim.x);
         }
