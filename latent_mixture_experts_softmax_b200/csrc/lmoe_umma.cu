@@ -402,9 +402,15 @@ __device__ __forceinline__ void store_half_swizzled(uint8_t* tile, int r, int h,
 
 __device__ __forceinline__ float u2f(uint32_t u) { return __uint_as_float(u); }
 
+// Per epilogue warp, a 32-column x 32-row fp16 transpose buffer: row-major
+// outputs ([column][row], rows contiguous in memory) leave a warp as 16-byte
+// stores of 8 rows of one column instead of 2-byte stores of one row.
+constexpr int kTrPitch = 40;   // halves per buffered column (80 bytes: 16-byte aligned, spreads banks)
+
 template <int KIND, int NT>
 __device__ __forceinline__ void epilogue_chunk(const PrefillParams& p, const TileRef& t, int warp, int lane, int c0,
-                                               const uint32_t (&r)[32], float* xchg, const float* tscale) {
+                                               const uint32_t (&r)[32], float* xchg, const float* tscale,
+                                               uint16_t* trw) {
     const int row = 32 * warp + lane;      // accumulator row (TMEM lane)
     const int ncol = min(32, t.n - c0);
     if (KIND == G_ROUTER) {
@@ -417,20 +423,29 @@ __device__ __forceinline__ void epilogue_chunk(const PrefillParams& p, const Til
         // metadata staged by the epilogue warps: group masks and slots of the tile's tokens
         const uint32_t* mmask = reinterpret_cast<const uint32_t*>(xchg);
         const int* mslot = reinterpret_cast<const int*>(mmask + NT);
-        const int l = t.m0 + row;
         bool bad = false;
+        // lane = row: the chunk's fp16 values into the transpose buffer; then
+        // lane (column j, rows 8q .. 8q+7) writes them to every slot of the
+        // token whose expert is in this group
 #pragma unroll
-        for (int j = 0; j < 32; ++j) {
+        for (int j = 0; j < 32; ++j)
+            trw[j * kTrPitch + lane] = j < ncol ? __half_as_ushort(half_checked(u2f(r[j]), bad)) : (uint16_t)0;
+        __syncwarp();
+        const int lbase = t.m0 + 32 * warp;
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            const int idx = lane + 32 * i, j = idx >> 2, q = idx & 3;
             if (j < ncol) {
+                const uint4 v = *reinterpret_cast<const uint4*>(trw + j * kTrPitch + 8 * q);
                 uint32_t mask = mmask[c0 + j];
-                const __half v = half_checked(u2f(r[j]), bad);
                 while (mask) {
                     const int k = __ffs(mask) - 1;
                     mask &= mask - 1;
-                    p.hperm[(size_t)mslot[(c0 + j) * p.K + k] * p.L + l] = v;
+                    *reinterpret_cast<uint4*>(p.hperm + (size_t)mslot[(c0 + j) * p.K + k] * p.L + lbase + 8 * q) = v;
                 }
             }
         }
+        __syncwarp();
         report_range(p.ctrl, bad);
     } else if (KIND == G_GATEUP || KIND == G_SHARED_GATEUP) {
         // rows 0-63: gate, rows 64-127: up.  Warps 0-1 finish columns 0-15
@@ -472,15 +487,22 @@ __device__ __forceinline__ void epilogue_chunk(const PrefillParams& p, const Til
     } else if (KIND == G_DOWN) {
         // routing weights of the tile's slots staged in xchg by the epilogue warps
         const float td = tscale[2];
-        const int l = t.m0 + row;
         bool bad = false;
+        // lane = row into the transpose buffer, then 8 rows of one slot per 16-byte store
 #pragma unroll
-        for (int j = 0; j < 32; ++j) {
-            if (j < ncol) {
-                const int slot = t.b0 + c0 + j;
-                p.operm[(size_t)slot * p.L + l] = half_checked(u2f(r[j]) * td * xchg[c0 + j], bad);
-            }
+        for (int j = 0; j < 32; ++j)
+            trw[j * kTrPitch + lane] =
+                j < ncol ? __half_as_ushort(half_checked(u2f(r[j]) * td * xchg[c0 + j], bad)) : (uint16_t)0;
+        __syncwarp();
+        const int lbase = t.m0 + 32 * warp;
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            const int idx = lane + 32 * i, j = idx >> 2, q = idx & 3;
+            if (j < ncol)
+                *reinterpret_cast<uint4*>(p.operm + (size_t)(t.b0 + c0 + j) * p.L + lbase + 8 * q) =
+                    *reinterpret_cast<const uint4*>(trw + j * kTrPitch + 8 * q);
         }
+        __syncwarp();
         report_range(p.ctrl, bad);
     } else {  // UPROJ
         const int hrow = t.m0 + row;
@@ -507,8 +529,9 @@ struct SmemPlan {
     static constexpr int kRaw = 256 * 32;
     // gate/up exchange (32 x 64 fp32) or a tile's routing metadata (NT x (1 + 16) words)
     static constexpr int kXchg = (32 * 64 * 4 > NT * 4 * 17) ? 32 * 64 * 4 : NT * 4 * 17;
+    static constexpr int kTr = 4 * 32 * kTrPitch * 2;     // the epilogue warps' transpose buffers
     static constexpr int kBars = (3 * STAGES + 5) * 8;
-    static constexpr int kTotal = 1024 /*alignment slack*/ + STAGES * (kA + kB) + RS * kRaw + kXchg + kBars + 16;
+    static constexpr int kTotal = 1024 /*alignment slack*/ + STAGES * (kA + kB) + RS * kRaw + kXchg + kTr + kBars + 16;
 };
 
 constexpr int kConvWarps = 8;      // dequantising warps (half a weight row per thread)
@@ -527,7 +550,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1) k_umma_gemm(const __grid_cons
     uint8_t* sB = smem + STAGES * Plan::kA;
     uint8_t* sRaw = sB + STAGES * Plan::kB;
     float* xchg = reinterpret_cast<float*>(sRaw + RS * Plan::kRaw);
-    uint64_t* bars = reinterpret_cast<uint64_t*>(reinterpret_cast<uint8_t*>(xchg) + Plan::kXchg);
+    uint16_t* trbuf = reinterpret_cast<uint16_t*>(reinterpret_cast<uint8_t*>(xchg) + Plan::kXchg);
+    uint64_t* bars = reinterpret_cast<uint64_t*>(reinterpret_cast<uint8_t*>(trbuf) + Plan::kTr);
     uint64_t* full_a = bars;
     uint64_t* full_b = bars + STAGES;
     uint64_t* empty = bars + 2 * STAGES;
@@ -798,7 +822,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1) k_umma_gemm(const __grid_cons
                     __syncwarp();
                     tmem_ld_32x32b_x32(taddr + c0, rr);
                     tmem_ld_wait();
-                    epilogue_chunk<KIND, NT>(p, cur.t, warp, lane, c0, rr, xchg, tscale);
+                    epilogue_chunk<KIND, NT>(p, cur.t, warp, lane, c0, rr, xchg, tscale, trbuf + warp * 32 * kTrPitch);
                 }
                 tc_fence_before();
             }
