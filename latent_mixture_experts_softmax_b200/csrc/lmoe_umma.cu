@@ -530,7 +530,7 @@ struct SmemPlan {
     // gate/up exchange (32 x 64 fp32) or a tile's routing metadata (NT x (1 + 16) words)
     static constexpr int kXchg = (32 * 64 * 4 > NT * 4 * 17) ? 32 * 64 * 4 : NT * 4 * 17;
     static constexpr int kTr = 4 * 32 * kTrPitch * 2;     // the epilogue warps' transpose buffers
-    static constexpr int kBars = (3 * STAGES + 5) * 8;
+    static constexpr int kBars = (2 * STAGES + 5) * 8;
     static constexpr int kTotal = 1024 /*alignment slack*/ + STAGES * (kA + kB) + RS * kRaw + kXchg + kTr + kBars + 16;
 };
 
@@ -552,10 +552,12 @@ __global__ void __launch_bounds__(kGemmThreads, 1) k_umma_gemm(const __grid_cons
     float* xchg = reinterpret_cast<float*>(sRaw + RS * Plan::kRaw);
     uint16_t* trbuf = reinterpret_cast<uint16_t*>(reinterpret_cast<uint8_t*>(xchg) + Plan::kXchg);
     uint64_t* bars = reinterpret_cast<uint64_t*>(reinterpret_cast<uint8_t*>(trbuf) + Plan::kTr);
-    uint64_t* full_a = bars;
-    uint64_t* full_b = bars + STAGES;
-    uint64_t* empty = bars + 2 * STAGES;
-    uint64_t* tfull = bars + 3 * STAGES;
+    // full[s]: the converter warps' arrivals and the loader's expect-tx
+    // arrival with its copies' bytes (one barrier, so the MMA issuer waits
+    // once per stage)
+    uint64_t* full = bars;
+    uint64_t* empty = bars + STAGES;
+    uint64_t* tfull = bars + 2 * STAGES;
     uint64_t* tempty = tfull + 2;
     uint64_t* final_bar = tempty + 2;
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(final_bar + 1);
@@ -567,8 +569,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1) k_umma_gemm(const __grid_cons
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < STAGES; ++s) {
-            mbar_init(&full_a[s], kConvWarps);
-            mbar_init(&full_b[s], 1);
+            mbar_init(&full[s], kConvWarps + 1);
             mbar_init(&empty[s], 1);
         }
         for (int a = 0; a < 2; ++a) {
@@ -605,18 +606,18 @@ __global__ void __launch_bounds__(kGemmThreads, 1) k_umma_gemm(const __grid_cons
                 if (!mbar_wait(&empty[s], ph ^ 1, abort_flag, kWaitLimit)) break;
                 const bool ta = S::tma_a(p, cb.seg);
                 const int k0 = cb.ks * 64;
-                mbar_arrive_expect_tx(&full_b[s], Plan::kB + (ta ? Plan::kA : 0));
+                mbar_arrive_expect_tx(&full[s], Plan::kB + (ta ? Plan::kA : 0));
                 uint8_t* dB = sB + s * Plan::kB;
-                if (KIND == G_UPROJ && cb.seg < p.G) tma_load_3d(dB, &maps.b, &full_b[s], k0, cb.seg, cb.t.b0);
-                else if (KIND == G_UPROJ) tma_load_3d(dB, &maps.b2, &full_b[s], k0, cb.t.b0, cb.seg - p.G);
-                else if (cb.seg > 0) tma_load_2d(dB, &maps.b2, &full_b[s], k0, cb.t.b0);
-                else tma_load_2d(dB, &maps.b, &full_b[s], k0, cb.t.b0);
+                if (KIND == G_UPROJ && cb.seg < p.G) tma_load_3d(dB, &maps.b, &full[s], k0, cb.seg, cb.t.b0);
+                else if (KIND == G_UPROJ) tma_load_3d(dB, &maps.b2, &full[s], k0, cb.t.b0, cb.seg - p.G);
+                else if (cb.seg > 0) tma_load_2d(dB, &maps.b2, &full[s], k0, cb.t.b0);
+                else tma_load_2d(dB, &maps.b, &full[s], k0, cb.t.b0);
                 if (ta) {
                     if (KIND == G_SHARED_GATEUP) {
-                        tma_load_2d(sA + s * Plan::kA, &maps.a, &full_b[s], k0, cb.t.m0);
-                        tma_load_2d(sA + s * Plan::kA + 64 * 128, &maps.a2, &full_b[s], k0, cb.t.m0);
+                        tma_load_2d(sA + s * Plan::kA, &maps.a, &full[s], k0, cb.t.m0);
+                        tma_load_2d(sA + s * Plan::kA + 64 * 128, &maps.a2, &full[s], k0, cb.t.m0);
                     } else {
-                        tma_load_2d(sA + s * Plan::kA, &maps.a, &full_b[s], k0, cb.t.m0);
+                        tma_load_2d(sA + s * Plan::kA, &maps.a, &full[s], k0, cb.t.m0);
                     }
                 }
                 last_b[s] = ph;
@@ -624,10 +625,13 @@ __global__ void __launch_bounds__(kGemmThreads, 1) k_umma_gemm(const __grid_cons
                 ++it_b;
             }
             if (*abort_flag) {
-                // let every copy already issued land before the CTA can leave
+                // let every copy already issued land before the CTA can leave;
+                // the phase also needs the converters' arrivals, which may
+                // never come after an abort, so this wait is short (about
+                // 0.1 s: the copies themselves take microseconds)
                 volatile int dummy = 0;
                 for (int i = 0; i < STAGES; ++i)
-                    if (last_b[i] != 0xFFFFFFFFu) mbar_wait(&full_b[i], last_b[i], &dummy, kWaitLimit);
+                    if (last_b[i] != 0xFFFFFFFFu) mbar_wait(&full[i], last_b[i], &dummy, kWaitLimit / 16);
             }
         }
         __syncwarp();
@@ -674,7 +678,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1) k_umma_gemm(const __grid_cons
                 store_half_swizzled(sA + s * Plan::kA, r, hh, o);
                 fence_proxy_async_smem();
                 __syncwarp();
-                if (lane == 0) mbar_arrive(&full_a[s]);
+                if (lane == 0) mbar_arrive(&full[s]);
                 cur.next_stage(p);
                 ++it;
             }
@@ -705,7 +709,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1) k_umma_gemm(const __grid_cons
                 fence_proxy_async_smem();
             }
             __syncwarp();
-            if (lane == 0) mbar_arrive(&full_a[s]);
+            if (lane == 0) mbar_arrive(&full[s]);
 #pragma unroll
             for (int k = 0; k + 1 < kRawAhead; ++k) raw[k] = raw[k + 1];
             cur.next_stage(p);
@@ -733,8 +737,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1) k_umma_gemm(const __grid_cons
                     const uint32_t ph = (it / STAGES) & 1;
                     const bool ta = S::tma_a(p, cur.seg);
                     const uint32_t idesc = idesc_f16(128, n_mma, ta ? 1 : 0);
-                    if (!mbar_wait(&full_b[s], ph, abort_flag, kWaitLimit)) { ok = false; break; }
-                    if (!mbar_wait(&full_a[s], ph, abort_flag, kWaitLimit)) { ok = false; break; }
+                    if (!mbar_wait(&full[s], ph, abort_flag, kWaitLimit)) { ok = false; break; }
                     tc_fence_after();
                     const uint64_t a_desc = sdesc_k128(smem_u32(sA + s * Plan::kA));
                     const uint64_t b_desc = sdesc_k128(smem_u32(sB + s * Plan::kB));
