@@ -50,6 +50,8 @@ def parse():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-sweep", action="store_true", help="skip the MTP verify-window sweep")
     ap.add_argument("--no-w4a4", action="store_true", help="skip the W4A4 prefill object")
+    ap.add_argument("--act-fmt", choices=["fp16", "nvfp4"], default=None,
+                    help="expert input format of the workload (nvfp4: W4A4); default: the workload's own")
     return ap.parse_args()
 
 
@@ -171,11 +173,16 @@ def step_cost(shape, idx: np.ndarray, groups: np.ndarray, T: int, prefill: bool)
 # When the sources have changed since the capture, or the kernel has no
 # capture, its traffic is reported as null.
 NCU_TRAFFIC = {
-    ("edge0_145b_decode", 4, "k_router_shared"): (9280000, "c93e26cfd6b4"),
-    ("edge0_145b_decode", 4, "k_wstream_dproj"): (39070000, "c93e26cfd6b4"),
-    ("edge0_145b_decode", 4, "k_wstream_gateup"): (42850000, "c93e26cfd6b4"),
-    ("edge0_145b_decode", 4, "k_wstream_down"): (21390000, "c93e26cfd6b4"),
-    ("edge0_145b_decode", 4, "k_wstream_uproj"): (43960000, "c93e26cfd6b4"),
+    ("edge0_145b_decode", 4, "k_router_shared"): (9282560, "eb4da6755108"),
+    ("edge0_145b_decode", 4, "k_wstream_dproj"): (39070720, "eb4da6755108"),
+    ("edge0_145b_decode", 4, "k_wstream_gateup"): (42732544, "eb4da6755108"),
+    ("edge0_145b_decode", 4, "k_wstream_down"): (21392128, "eb4da6755108"),
+    ("edge0_145b_decode", 4, "k_wstream_uproj"): (43962112, "eb4da6755108"),
+    ("edge0_145b_prefill", 4096, "gateup"): (849587370, "eb4da6755108"),
+    ("edge0_145b_prefill", 4096, "uproj"): (447073280, "eb4da6755108"),
+    ("edge0_145b_prefill+w4a4", 4096, "uproj"): (446979754, "eb4da6755108"),
+    ("edge0_145b_prefill+w4a4", 4096, "gateup"): (745645568, "eb4da6755108"),
+    ("edge0_145b_prefill+w4a4", 4096, "down"): (464022442, "eb4da6755108"),
 }
 
 
@@ -192,8 +199,12 @@ def cuda_source_hash() -> str:
     return h.hexdigest()[:12]
 
 
-def ncu_traffic(workload: str, T: int, kernel: str):
-    e = NCU_TRAFFIC.get((workload, T, kernel))
+def ncu_traffic(wl, T: int, kernel: str):
+    """DRAM bytes per launch of `kernel` from the table above (keyed by the
+    workload name, "+w4a4" for NVFP4 expert inputs), if taken of the current
+    sources."""
+    name = wl.name + ("+w4a4" if getattr(wl.shape, "act_fmt", "fp16") == "nvfp4" else "")
+    e = NCU_TRAFFIC.get((name, T, kernel))
     if e is None or e[1] != cuda_source_hash():
         return None
     return e[0]
@@ -560,12 +571,12 @@ def measure_layer(args, wl, T, K, W, rank, world, local, dev_name, ctx=None, lig
         else:
             peak, psrc = tc_peak, f"{peak_src} bf16 dense burst (fp16 operands run at the bf16 rate)"
         roof = {"bound": "tensor", "kernel": dom_name, "achieved": dom_ach, "peak": peak, "unit": "TFLOP/s",
-                "frac": dom_ach / peak, "peak_source": psrc, "traffic": ncu_traffic(wl.name, T, dom_name)}
+                "frac": dom_ach / peak, "peak_source": psrc, "traffic": ncu_traffic(wl, T, dom_name)}
     else:
         dom_ach = cost[dom_name] / dom_s / 1e9
         roof = {"bound": "hbm", "kernel": dom_name, "achieved": dom_ach, "peak": hbm_peak, "unit": "GB/s",
                 "frac": dom_ach / hbm_peak, "peak_source": f"{peak_src} HBM copy",
-                "traffic": ncu_traffic(wl.name, T, dom_name)}
+                "traffic": ncu_traffic(wl, T, dom_name)}
     # e2e through the host-buffer entry point (copies inside the timed region)
     x_pin = [torch.from_numpy(x.view(np.int16)).pin_memory() for x in xs_host]
     y_pin = torch.empty((T, s.hidden), dtype=torch.int16).pin_memory()
@@ -691,6 +702,8 @@ def main():
 
     from latent_mixture_experts_softmax_b200 import synth
     wl = synth.WORKLOADS[args.workload]
+    if args.act_fmt:
+        wl = wl.with_(shape=synth.replace(wl.shape, act_fmt=args.act_fmt))
     T = args.T or wl.T
 
     if args.impl == "reference":
