@@ -50,17 +50,23 @@ struct TileRef {
     int b0;       // first B row (token or slot)
     int n;        // valid B rows
     int nq;       // token tile index (UPROJ / DPROJ hit flags)
+    int na;       // 128-row A tiles of the item (2 in the two-tile expert GEMMs, else 1)
 };
 
-template <int KIND, int NT>
+// MA = 2 (expert GEMMs only): an item covers two 128-row A tiles that share
+// each B stage, two MMAs per K step into two accumulators.  Gate/up: tile a
+// holds gate and up rows m0 + 64a .. m0 + 64a + 63; down: rows m0 + 128a ..
+// m0 + 128a + 127.  The last item of a matrix may have one.
+template <int KIND, int NT, int MA = 1>
 struct Sched {
+    static_assert(MA == 1 || KIND == G_GATEUP || KIND == G_DOWN, "two A tiles: expert GEMMs only");
     __device__ static int m_tiles(const PrefillParams& p) {
         switch (KIND) {
             case G_ROUTER: return p.E / 128;
             case G_SHARED_GATEUP: return p.Fs / 64;
             case G_DPROJ: return p.G * (p.L / 128);
-            case G_GATEUP: return p.F / 64;
-            case G_DOWN: return p.L / 128;
+            case G_GATEUP: return (p.F / 64 + MA - 1) / MA;
+            case G_DOWN: return (p.L / 128 + MA - 1) / MA;
             default: return p.H / 128;
         }
     }
@@ -73,15 +79,18 @@ struct Sched {
         const int mt = m_tiles(p);
         t.valid = 1;
         t.mat = 0;
+        t.na = 1;
         if (KIND == G_GATEUP || KIND == G_DOWN) {
             // consecutive tiles share the expert's token rows
             const int et = i / mt, m = i % mt;
             const int4 d = __ldcg(p.etile + et);
+            const int rows = KIND == G_GATEUP ? 64 : 128;           // output rows per A tile
             t.mat = d.x;
-            t.m0 = m * (KIND == G_GATEUP ? 64 : 128);
+            t.m0 = m * rows * MA;
             t.b0 = d.y;
             t.n = min(NT, d.z);
             t.nq = 0;
+            t.na = min(MA, ((KIND == G_GATEUP ? p.F : p.L) - t.m0) / rows);
         } else {
             // consecutive tiles share the weight tile (token tiles fastest)
             const int ntt = (p.T + NT - 1) / NT;
@@ -138,9 +147,9 @@ struct Sched {
 
 // Walks the (tile, segment, 64-wide K stage) sequence of one CTA.  The
 // active segments of a tile are read once, when the tile is entered.
-template <int KIND, int NT>
+template <int KIND, int NT, int MA = 1>
 struct Cursor {
-    using S = Sched<KIND, NT>;
+    using S = Sched<KIND, NT, MA>;
     int tile, seg, ks, nk, ntiles;
     uint64_t segmask;
     bool done;
@@ -239,8 +248,8 @@ struct RawHalf {
 // Fetch RawHalf of (row r, half h) of the cursor's stage with plain loads
 // (read-only path; the bulk-copy engine's fixed cost per copy would cap a
 // per-stage stream of small copies).
-template <int KIND, int NT>
-__device__ __forceinline__ void fetch_raw(const PrefillParams& p, const Cursor<KIND, NT>& c, int r, int h, RawHalf& o) {
+template <int KIND, int NT, class Cur>
+__device__ __forceinline__ void fetch_raw(const PrefillParams& p, const Cur& c, int r, int h, RawHalf& o) {
     const int k0 = c.ks * 64;
     if (KIND == G_DPROJ || (KIND == G_UPROJ && c.seg < p.G)) {
         const int R = KIND == G_DPROJ ? p.L : p.H;
@@ -290,8 +299,8 @@ __device__ __forceinline__ void fetch_raw(const PrefillParams& p, const Cursor<K
 // The NVFP4 expert bytes of (row r, half h) of the cursor's stage, copied
 // into this thread's ring slot: 16 code bytes at slot[0, 16), the row's
 // 4-byte scale word at slot[16, 20).
-template <int KIND, int NT>
-__device__ __forceinline__ void fetch_raw_async(const PrefillParams& p, const Cursor<KIND, NT>& c, int r, int h,
+template <int KIND, int NT, class Cur>
+__device__ __forceinline__ void fetch_raw_async(const PrefillParams& p, const Cur& c, int r, int h,
                                                 uint8_t* slot) {
     const int k0 = c.ks * 64;
     const size_t nq = (size_t)p.L * p.F / 2, ns = (size_t)p.L * p.F / 16;
@@ -301,6 +310,25 @@ __device__ __forceinline__ void fetch_raw_async(const PrefillParams& p, const Cu
     const int m = KIND == G_GATEUP ? (r >> 6) : 2;                  // gate, up, down
     cp_async16_sh(slot, rec + (size_t)m * nq + ((size_t)(k0 / 32 + h) * R + row) * 16);
     cp_async4_sh(slot + 16, rec + 3 * nq + (size_t)m * ns + ((size_t)(k0 / 64) * R + row) * 4);
+}
+
+// Two-tile expert items: the NVFP4 bytes of row rr of A tile a (both
+// 32-column halves of the stage), copied into this thread's ring slot: code
+// chunks at slot[0, 16) and [16, 32), the row's 4-byte scale word at
+// slot[32, 36).
+template <int KIND>
+__device__ __forceinline__ void fetch_row_async(const PrefillParams& p, const TileRef& t, int ks, int a, int rr,
+                                                uint8_t* slot) {
+    const int k0 = ks * 64;
+    const size_t nq = (size_t)p.L * p.F / 2, ns = (size_t)p.L * p.F / 16;
+    const uint8_t* rec = p.experts + (size_t)t.mat * p.rec_bytes;
+    const int R = KIND == G_GATEUP ? p.F : p.L;
+    const int row = KIND == G_GATEUP ? t.m0 + 64 * a + (rr & 63) : t.m0 + 128 * a + rr;
+    const int m = KIND == G_GATEUP ? (rr >> 6) : 2;                  // gate, up, down
+    const uint8_t* q = rec + (size_t)m * nq + ((size_t)(k0 / 32) * R + row) * 16;
+    cp_async16_sh(slot, q);
+    cp_async16_sh(slot + 16, q + (size_t)R * 16);
+    cp_async4_sh(slot + 32, rec + 3 * nq + (size_t)m * ns + ((size_t)(k0 / 64) * R + row) * 4);
 }
 
 // RawHalf of (row r, half h) -> 16 half2 of the row's 32 columns.
@@ -520,13 +548,14 @@ __device__ __forceinline__ void epilogue_chunk(const PrefillParams& p, const Til
 // the GEMM kernel
 // ---------------------------------------------------------------------------
 
-template <int NT, int STAGES, int RS>
+template <int NT, int STAGES, int RS, int MA = 1>
 struct SmemPlan {
-    static constexpr int kA = 128 * 128;                 // bytes per A stage (128 rows x 64 x 16-bit)
+    static constexpr int kA = MA * 128 * 128;            // bytes per A stage (MA x 128 rows x 64 x 16-bit)
     static constexpr int kB = NT * 128;                  // bytes per B stage
     // a stage of the converters' ring of stored expert bytes: 32 bytes for
     // each of the 256 converter threads (16 code bytes, the 4-byte scale word)
-    static constexpr int kRaw = 256 * 32;
+    // (two-tile items: 48 bytes, a whole row's 32 code bytes and scale word)
+    static constexpr int kRaw = 256 * (MA == 2 ? 48 : 32);
     // gate/up exchange (32 x 64 fp32) or a tile's routing metadata (NT x (1 + 16) words)
     static constexpr int kXchg = (32 * 64 * 4 > NT * 4 * 17) ? 32 * 64 * 4 : NT * 4 * 17;
     static constexpr int kTr = 4 * 32 * kTrPitch * 2;     // the epilogue warps' transpose buffers
@@ -538,10 +567,10 @@ constexpr int kConvWarps = 8;      // dequantising warps (half a weight row per 
 constexpr int kRawAhead = 4;       // stages whose stored weight bytes a converter thread holds
 constexpr int kGemmThreads = 448;  // 4 epilogue, 8 converter, 1 MMA, 1 loader warps
 
-template <int KIND, int NT, int STAGES, int RS>
+template <int KIND, int NT, int STAGES, int RS, int MA = 1>
 __global__ void __launch_bounds__(kGemmThreads, 1) k_umma_gemm(const __grid_constant__ TmaMaps maps, const PrefillParams p) {
-    using S = Sched<KIND, NT>;
-    using Plan = SmemPlan<NT, STAGES, RS>;
+    using S = Sched<KIND, NT, MA>;
+    using Plan = SmemPlan<NT, STAGES, RS, MA>;
     extern __shared__ uint8_t smem_raw[];
     // aligned by pointer arithmetic on the shared array, so that the compiler
     // still knows every access through it is a shared-memory access
@@ -564,7 +593,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1) k_umma_gemm(const __grid_cons
     volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    constexpr uint32_t kTmemCols = 2 * NT;
+    constexpr uint32_t kTmemCols = 2 * NT * MA;
     __shared__ float tscale[4];   // the current tile's tensor scales (epilogue)
 
     if (threadIdx.x == 0) {
@@ -595,7 +624,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1) k_umma_gemm(const __grid_cons
         // ------------------------------------------------------------ loader (one thread)
         if (lane == 0) {
             tma_prefetch_desc(&maps.b);
-            Cursor<KIND, NT> cb;           // activation / plain-weight stages
+            Cursor<KIND, NT, MA> cb;           // activation / plain-weight stages
             cb.begin(p);
             uint32_t it_b = 0;
             uint32_t last_b[STAGES];
@@ -644,10 +673,56 @@ __global__ void __launch_bounds__(kGemmThreads, 1) k_umma_gemm(const __grid_cons
         // plain loads kRawAhead - 1 stages ahead of use.
         const int r = (threadIdx.x - 128) & 127;   // A row
         const int hh = (threadIdx.x - 128) >> 7;   // half of the 64 columns
-        Cursor<KIND, NT> cur, cf;
+        Cursor<KIND, NT, MA> cur, cf;
         cur.begin(p);
         cf = cur;
-        if (RS > 0 && (KIND == G_GATEUP || KIND == G_DOWN) && p.efmt == LMOE_EXPERTS_NVFP4) {
+        if (MA == 2) {
+            // two-tile items: thread c converts the whole 64-column row
+            // c & 127 of A tile c >> 7, through its own ring of RS slots
+            constexpr int kRS = RS > 0 ? RS : 1;
+            const int c2 = threadIdx.x - 128, a2 = c2 >> 7, rr = c2 & 127;
+            uint8_t* ring = sRaw + (size_t)c2 * 48;                          // + stage * Plan::kRaw
+#pragma unroll 1
+            for (int k = 0; k < kRS - 1; ++k) {
+                if (!cf.done) {
+                    if (a2 < cf.t.na) fetch_row_async<KIND>(p, cf.t, cf.ks, a2, rr, ring + (size_t)k * Plan::kRaw);
+                    cf.next_stage(p);
+                }
+                cp_async_commit_grp();
+            }
+            uint32_t it = 0;
+            while (!cur.done) {
+                if (!cf.done) {
+                    if (a2 < cf.t.na)
+                        fetch_row_async<KIND>(p, cf.t, cf.ks, a2, rr, ring + (size_t)((it + kRS - 1) % kRS) * Plan::kRaw);
+                    cf.next_stage(p);
+                }
+                cp_async_commit_grp();
+                const int s = it % STAGES;
+                const uint32_t ph = (it / STAGES) & 1;
+                if (!mbar_wait(&empty[s], ph ^ 1, abort_flag, kWaitLimit)) break;
+                cp_async_wait_grp<kRS - 1>();
+                if (a2 < cur.t.na) {
+                    const uint8_t* slot = ring + (size_t)(it % kRS) * Plan::kRaw;
+                    uint8_t* tile = sA + s * Plan::kA + a2 * (128 * 128);
+                    RawHalf raw;
+                    raw.s = *reinterpret_cast<const uint32_t*>(slot + 32);
+#pragma unroll
+                    for (int h = 0; h < 2; ++h) {
+                        raw.a = *reinterpret_cast<const uint4*>(slot + 16 * h);
+                        uint32_t o[16];
+                        dequant_half<KIND>(p, raw, h, o);
+                        store_half_swizzled(tile, rr, h, o);
+                    }
+                    fence_proxy_async_smem();
+                }
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&full[s]);
+                cur.next_stage(p);
+                ++it;
+            }
+            cp_async_wait_grp<0>();
+        } else if (RS > 0 && (KIND == G_GATEUP || KIND == G_DOWN) && p.efmt == LMOE_EXPERTS_NVFP4) {
             constexpr int kRS = RS > 0 ? RS : 1;
             uint8_t* ring = sRaw + (size_t)(threadIdx.x - 128) * 32;       // + stage * Plan::kRaw
 #pragma unroll 1
@@ -719,7 +794,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1) k_umma_gemm(const __grid_cons
     } else if (warp == 12) {
         // ------------------------------------------------------------ MMA issuer
         if (lane == 0) {
-            Cursor<KIND, NT> cur;
+            Cursor<KIND, NT, MA> cur;
             cur.begin(p);
             uint32_t it = 0, tcount = 0;
             bool issued = false;
@@ -728,8 +803,9 @@ __global__ void __launch_bounds__(kGemmThreads, 1) k_umma_gemm(const __grid_cons
                 const uint32_t aph = (tcount >> 1) & 1;
                 if (!mbar_wait(&tempty[acc], aph ^ 1, abort_flag, kWaitLimit)) break;
                 tc_fence_after();
-                const uint32_t d_tmem = tmem_base + acc * NT;
+                const uint32_t d_tmem = tmem_base + acc * NT * MA;
                 const int n_mma = (KIND == G_GATEUP || KIND == G_DOWN) ? ((cur.t.n + 15) & ~15) : NT;
+                const int na = cur.t.na;
                 bool first = true;
                 bool ok = true;
                 while (true) {
@@ -739,11 +815,16 @@ __global__ void __launch_bounds__(kGemmThreads, 1) k_umma_gemm(const __grid_cons
                     const uint32_t idesc = idesc_f16(128, n_mma, ta ? 1 : 0);
                     if (!mbar_wait(&full[s], ph, abort_flag, kWaitLimit)) { ok = false; break; }
                     tc_fence_after();
-                    const uint64_t a_desc = sdesc_k128(smem_u32(sA + s * Plan::kA));
                     const uint64_t b_desc = sdesc_k128(smem_u32(sB + s * Plan::kB));
 #pragma unroll
-                    for (int j = 0; j < 4; ++j)
-                        umma_f16(d_tmem, a_desc + 2 * j, b_desc + 2 * j, idesc, (first && j == 0) ? 0u : 1u);
+                    for (int a = 0; a < MA; ++a) {
+                        if (a >= na) break;
+                        // A tile a of the stage; both tiles share the B stage
+                        const uint64_t a_desc = sdesc_k128(smem_u32(sA + s * Plan::kA + a * (128 * 128)));
+#pragma unroll
+                        for (int j = 0; j < 4; ++j)
+                            umma_f16(d_tmem + a * NT, a_desc + 2 * j, b_desc + 2 * j, idesc, (first && j == 0) ? 0u : 1u);
+                    }
                     first = false;
                     issued = true;
                     umma_commit(&empty[s]);
@@ -770,7 +851,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1) k_umma_gemm(const __grid_cons
         // barrier; after a timeout (dead) the work is skipped.  The TMEM
         // loads are warp-collective, so the wait's outcome is made
         // warp-uniform and the warp converges before each load.
-        Cursor<KIND, NT> cur;
+        Cursor<KIND, NT, MA> cur;
         cur.begin(p);
         uint32_t tcount = 0;
         bool dead = false;
@@ -819,13 +900,18 @@ __global__ void __launch_bounds__(kGemmThreads, 1) k_umma_gemm(const __grid_cons
             dead = __any_sync(0xffffffffu, dead);
             if (!dead) {
                 tc_fence_after();
-                const uint32_t taddr = tmem_base + ((uint32_t)(32 * warp) << 16) + acc * NT;
-                for (int c0 = 0; c0 < cur.t.n; c0 += 32) {
-                    uint32_t rr[32];
-                    __syncwarp();
-                    tmem_ld_32x32b_x32(taddr + c0, rr);
-                    tmem_ld_wait();
-                    epilogue_chunk<KIND, NT>(p, cur.t, warp, lane, c0, rr, xchg, tscale, trbuf + warp * 32 * kTrPitch);
+                for (int a = 0; a < cur.t.na; ++a) {
+                    // accumulator a of the item: A tile a's output rows
+                    TileRef ta = cur.t;
+                    ta.m0 += a * (KIND == G_GATEUP ? 64 : 128);
+                    const uint32_t taddr = tmem_base + ((uint32_t)(32 * warp) << 16) + acc * NT * MA + a * NT;
+                    for (int c0 = 0; c0 < cur.t.n; c0 += 32) {
+                        uint32_t rr[32];
+                        __syncwarp();
+                        tmem_ld_32x32b_x32(taddr + c0, rr);
+                        tmem_ld_wait();
+                        epilogue_chunk<KIND, NT>(p, ta, warp, lane, c0, rr, xchg, tscale, trbuf + warp * 32 * kTrPitch);
+                    }
                 }
                 tc_fence_before();
             }
@@ -1097,10 +1183,10 @@ static bool make_map_zsh(CUtensorMap* m, const void* base, uint64_t T, uint64_t 
 
 static int g_num_sms = 0;
 
-template <int KIND, int NT, int STAGES, int RS>
+template <int KIND, int NT, int STAGES, int RS, int MA = 1>
 static cudaError_t launch_gemm(const TmaMaps& maps, const PrefillParams& p, cudaStream_t st, int max_tiles) {
-    const size_t smem = SmemPlan<NT, STAGES, RS>::kTotal;
-    auto kern = k_umma_gemm<KIND, NT, STAGES, RS>;
+    const size_t smem = SmemPlan<NT, STAGES, RS, MA>::kTotal;
+    auto kern = k_umma_gemm<KIND, NT, STAGES, RS, MA>;
     cudaError_t e = ensure_smem(reinterpret_cast<const void*>(kern), smem);
     if (e != cudaSuccess) return e;
     if (g_num_sms == 0) {
@@ -1172,9 +1258,18 @@ cudaError_t run_prefill_path(PrefillParams p, cudaStream_t st, void* memset_base
         if ((e = run_w4a4_down(p, p.aq, p.asf, p.aG, pairs, st)) != cudaSuccess) return e;
         mark(st);
     } else {
-        if ((e = launch_gemm<G_GATEUP, kNtExpert, 4, 8>(m_gu, p, st, (F / 64) * max_etiles)) != cudaSuccess) return e;
-        mark(st);
-        if ((e = launch_gemm<G_DOWN, kNtExpert, 4, 8>(m_down, p, st, (L / 128) * max_etiles)) != cudaSuccess) return e;
+        if (p.efmt == LMOE_EXPERTS_NVFP4) {
+            // two 128-row A tiles per item (one B stage feeds both)
+            if ((e = launch_gemm<G_GATEUP, kNtExpert, 3, 4, 2>(m_gu, p, st, (F / 128 + 1) * max_etiles)) != cudaSuccess)
+                return e;
+            mark(st);
+            if ((e = launch_gemm<G_DOWN, kNtExpert, 3, 4, 2>(m_down, p, st, (L / 256 + 1) * max_etiles)) != cudaSuccess)
+                return e;
+        } else {
+            if ((e = launch_gemm<G_GATEUP, kNtExpert, 4, 8>(m_gu, p, st, (F / 64) * max_etiles)) != cudaSuccess) return e;
+            mark(st);
+            if ((e = launch_gemm<G_DOWN, kNtExpert, 4, 8>(m_down, p, st, (L / 128) * max_etiles)) != cudaSuccess) return e;
+        }
         mark(st);
     }
     k_combine<<<T, 256, 0, st>>>(p);

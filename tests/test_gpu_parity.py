@@ -300,6 +300,15 @@ def test_prefill_path_formats_with_residual(fmt):
     check_block(wl.shape, synth.make_layer(wl), synth.make_x(wl), residual_bits=res, what=f"prefill fmt={fmt}")
 
 
+@pytest.mark.parametrize("latent,ffn", [(384, 192), (128, 320)])
+def test_prefill_path_odd_row_tile_counts(latent, ffn):
+    """The expert GEMMs take two 128-row weight tiles per item (gate/up: 64
+    output features of gate and of up per tile; down: 128 rows of h); an odd
+    number of tiles leaves the last item of each matrix with one."""
+    wl = prefill_workload(200, latent=latent, ffn=ffn)
+    check_block(wl.shape, synth.make_layer(wl), synth.make_x(wl), what=f"prefill latent={latent} ffn={ffn}")
+
+
 def test_prefill_path_skewed_expert_spans_several_tiles():
     """One expert takes every token (several 128-slot tiles of the expert GEMMs)."""
     wl = prefill_workload(400)
