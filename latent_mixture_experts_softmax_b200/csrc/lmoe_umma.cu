@@ -92,9 +92,13 @@ struct Sched {
             t.nq = 0;
             t.na = min(MA, ((KIND == G_GATEUP ? p.F : p.L) - t.m0) / rows);
         } else {
-            // consecutive tiles share the weight tile (token tiles fastest)
+            // consecutive tiles share the weight tile (token tiles fastest),
+            // except U: there the token tile's B operand (the group sums s
+            // of every hit group, 28 KB a token at the Edge0 shapes) is what
+            // outgrows L2 when all of it is in flight, so consecutive tiles
+            // share the token tile and its B stages (weight tiles fastest)
             const int ntt = (p.T + NT - 1) / NT;
-            const int m = i / ntt, q = i % ntt;
+            const int m = KIND == G_UPROJ ? i % mt : i / ntt, q = KIND == G_UPROJ ? i / mt : i % ntt;
             t.nq = q;
             t.b0 = q * NT;
             t.n = min(NT, p.T - t.b0);
