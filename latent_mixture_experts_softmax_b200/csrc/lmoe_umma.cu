@@ -300,22 +300,6 @@ __device__ __forceinline__ void fetch_raw(const PrefillParams& p, const Cur& c, 
     }
 }
 
-// The NVFP4 expert bytes of (row r, half h) of the cursor's stage, copied
-// into this thread's ring slot: 16 code bytes at slot[0, 16), the row's
-// 4-byte scale word at slot[16, 20).
-template <int KIND, int NT, class Cur>
-__device__ __forceinline__ void fetch_raw_async(const PrefillParams& p, const Cur& c, int r, int h,
-                                                uint8_t* slot) {
-    const int k0 = c.ks * 64;
-    const size_t nq = (size_t)p.L * p.F / 2, ns = (size_t)p.L * p.F / 16;
-    const uint8_t* rec = p.experts + (size_t)c.t.mat * p.rec_bytes;
-    const int R = KIND == G_GATEUP ? p.F : p.L;
-    const int row = KIND == G_GATEUP ? c.t.m0 + (r & 63) : c.t.m0 + r;
-    const int m = KIND == G_GATEUP ? (r >> 6) : 2;                  // gate, up, down
-    cp_async16_sh(slot, rec + (size_t)m * nq + ((size_t)(k0 / 32 + h) * R + row) * 16);
-    cp_async4_sh(slot + 16, rec + 3 * nq + (size_t)m * ns + ((size_t)(k0 / 64) * R + row) * 4);
-}
-
 // Two-tile expert items: the NVFP4 bytes of row rr of A tile a (both
 // 32-column halves of the stage), copied into this thread's ring slot: code
 // chunks at slot[0, 16) and [16, 32), the row's 4-byte scale word at
@@ -558,8 +542,9 @@ struct SmemPlan {
     static constexpr int kB = NT * 128;                  // bytes per B stage
     // a stage of the converters' ring of stored expert bytes: 32 bytes for
     // each of the 256 converter threads (16 code bytes, the 4-byte scale word)
-    // (two-tile items: 48 bytes, a whole row's 32 code bytes and scale word)
-    static constexpr int kRaw = 256 * (MA == 2 ? 48 : 32);
+    // a stage of the two-tile expert GEMMs' ring: 48 bytes for each of the
+    // 256 converter threads (a whole row's 32 code bytes and its scale word)
+    static constexpr int kRaw = 256 * 48;
     // gate/up exchange (32 x 64 fp32) or a tile's routing metadata (NT x (1 + 16) words)
     static constexpr int kXchg = (32 * 64 * 4 > NT * 4 * 17) ? 32 * 64 * 4 : NT * 4 * 17;
     static constexpr int kTr = 4 * 32 * kTrPitch * 2;     // the epilogue warps' transpose buffers
@@ -670,11 +655,14 @@ __global__ void __launch_bounds__(kGemmThreads, 1) k_umma_gemm(const __grid_cons
         __syncwarp();
     } else if (warp >= 4 && warp < 12) {
         // ------------------------------------------------------------ converters
-        // Each thread owns half a weight row of every stage.  NVFP4 expert
-        // weights come through a ring of RS stages in shared memory filled
-        // by the thread's own cp.async copies (deep enough to keep the loads
-        // of the stored bytes in flight); the other formats are fetched with
-        // plain loads kRawAhead - 1 stages ahead of use.
+        // Each thread owns half a weight row of every stage (a whole row of
+        // one of the two A tiles in the two-tile expert GEMMs).  The stored
+        // NVFP4 expert bytes come through a ring of RS stages in shared
+        // memory filled by the thread's own cp.async copies (deep enough to
+        // keep the loads in flight); the other formats are fetched with
+        // plain loads kRawAhead - 1 stages ahead of use (a shared-memory
+        // ring for Q8_0 D and U, which leaves room for only three operand
+        // stages, measured slower).
         const int r = (threadIdx.x - 128) & 127;   // A row
         const int hh = (threadIdx.x - 128) >> 7;   // half of the 64 columns
         Cursor<KIND, NT, MA> cur, cf;
@@ -720,42 +708,6 @@ __global__ void __launch_bounds__(kGemmThreads, 1) k_umma_gemm(const __grid_cons
                     }
                     fence_proxy_async_smem();
                 }
-                __syncwarp();
-                if (lane == 0) mbar_arrive(&full[s]);
-                cur.next_stage(p);
-                ++it;
-            }
-            cp_async_wait_grp<0>();
-        } else if (RS > 0 && (KIND == G_GATEUP || KIND == G_DOWN) && p.efmt == LMOE_EXPERTS_NVFP4) {
-            constexpr int kRS = RS > 0 ? RS : 1;
-            uint8_t* ring = sRaw + (size_t)(threadIdx.x - 128) * 32;       // + stage * Plan::kRaw
-#pragma unroll 1
-            for (int k = 0; k < kRS - 1; ++k) {
-                if (!cf.done) {
-                    fetch_raw_async<KIND, NT>(p, cf, r, hh, ring + (size_t)k * Plan::kRaw);
-                    cf.next_stage(p);
-                }
-                cp_async_commit_grp();
-            }
-            uint32_t it = 0;
-            while (!cur.done) {
-                if (!cf.done) {
-                    fetch_raw_async<KIND, NT>(p, cf, r, hh, ring + (size_t)((it + kRS - 1) % kRS) * Plan::kRaw);
-                    cf.next_stage(p);
-                }
-                cp_async_commit_grp();
-                const int s = it % STAGES;
-                const uint32_t ph = (it / STAGES) & 1;
-                if (!mbar_wait(&empty[s], ph ^ 1, abort_flag, kWaitLimit)) break;
-                cp_async_wait_grp<kRS - 1>();
-                const uint8_t* slot = ring + (size_t)(it % kRS) * Plan::kRaw;
-                RawHalf raw;
-                raw.a = *reinterpret_cast<const uint4*>(slot);
-                raw.s = *reinterpret_cast<const uint32_t*>(slot + 16);
-                uint32_t o[16];
-                dequant_half<KIND>(p, raw, hh, o);
-                store_half_swizzled(sA + s * Plan::kA, r, hh, o);
-                fence_proxy_async_smem();
                 __syncwarp();
                 if (lane == 0) mbar_arrive(&full[s]);
                 cur.next_stage(p);
@@ -1270,9 +1222,9 @@ cudaError_t run_prefill_path(PrefillParams p, cudaStream_t st, void* memset_base
             if ((e = launch_gemm<G_DOWN, kNtExpert, 3, 4, 2>(m_down, p, st, (L / 256 + 1) * max_etiles)) != cudaSuccess)
                 return e;
         } else {
-            if ((e = launch_gemm<G_GATEUP, kNtExpert, 4, 8>(m_gu, p, st, (F / 64) * max_etiles)) != cudaSuccess) return e;
+            if ((e = launch_gemm<G_GATEUP, kNtExpert, 4, 0>(m_gu, p, st, (F / 64) * max_etiles)) != cudaSuccess) return e;
             mark(st);
-            if ((e = launch_gemm<G_DOWN, kNtExpert, 4, 8>(m_down, p, st, (L / 128) * max_etiles)) != cudaSuccess) return e;
+            if ((e = launch_gemm<G_DOWN, kNtExpert, 4, 0>(m_down, p, st, (L / 128) * max_etiles)) != cudaSuccess) return e;
         }
         mark(st);
     }
