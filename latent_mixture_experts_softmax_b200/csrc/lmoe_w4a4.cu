@@ -31,9 +31,10 @@
 //        slot of slack); once a stage has landed, each warp copies its
 //        weight and activation scale words to its 32-lane TMEM subpartition
 //        (scale columns 4k + b: rows / slots b*32 .. b*32+31)
-//   4-7  epilogue: accumulators (TMEM, two buffers) -> * G * ts -> SwiGLU
-//        (gate/up) or routing weight (down) -> fp16 zperm / operm
-//   8    MMA issue (one thread), TMEM allocation
+//   4-11 epilogue: accumulators (TMEM, two buffers) -> * G * ts -> SwiGLU
+//        (gate/up) or routing weight (down) -> fp16 zperm / operm; warps w
+//        and w + 4 read TMEM subpartition w & 3, alternate 16-column chunks
+//   12   MMA issue (one thread), TMEM allocation
 
 #include <cstring>
 
@@ -44,7 +45,8 @@ namespace {
 
 using namespace sm100;
 
-constexpr int kW4Threads = 288;
+constexpr int kW4Threads = 416;   // 4 loader warps, 8 epilogue warps, 1 MMA warp
+constexpr int kW4MmaWarp = 12;
 constexpr uint64_t kW4WaitLimit = 4000000000ull;   // SM cycles per barrier wait (about 2 s)
 constexpr uint32_t kW4TmemCols = 512;
 constexpr int kW4CodeBox = 128 * 128;    // bytes: 8 chunks x 128 rows x 16 B
@@ -212,13 +214,13 @@ __global__ void __launch_bounds__(kW4Threads, 1) k_w4a4(const __grid_constant__ 
         }
         for (int b = 0; b < 2; ++b) {
             mbar_init(&tfull[b], 1);
-            mbar_init(&tempty[b], 4);
+            mbar_init(&tempty[b], 8);
         }
         mbar_init(final_bar, 1);
         *abort_flag = 0;
         fence_barrier_init();
     }
-    if (warp == 8) {
+    if (warp == kW4MmaWarp) {
         __syncwarp();
         tmem_alloc(tmem_slot, kW4TmemCols);
         tmem_relinquish();
@@ -334,7 +336,7 @@ __global__ void __launch_bounds__(kW4Threads, 1) k_w4a4(const __grid_constant__ 
             }
         }
         cp_wait<0>();
-    } else if (warp == 8) {
+    } else if (warp == kW4MmaWarp) {
         // -------------------------------------------------------- MMA issue
         if (lane == 0) {
             uint32_t it = 0, pc = 0;
@@ -374,9 +376,11 @@ __global__ void __launch_bounds__(kW4Threads, 1) k_w4a4(const __grid_constant__ 
         }
         __syncwarp();
     } else {
-        // -------------------------------------------------------- epilogue (warps 4-7)
+        // -------------------------------------------------------- epilogue (warps 4-11)
+        // Warps w and w + 4 share TMEM subpartition w & 3 and take alternate
+        // 16-column chunks of the accumulator.
         const int et = threadIdx.x - 128;
-        const int sub = warp & 3;
+        const int sub = warp & 3, half = (warp - 4) >> 2;
         uint32_t pc = 0;
         bool dead = false, bad = false;
         // the next item's tile, per-slot scales (G; the routing weight for
@@ -397,15 +401,17 @@ __global__ void __launch_bounds__(kW4Threads, 1) k_w4a4(const __grid_constant__ 
             const int mat = cur.x, b0 = cur.y, nrow = cur.z, m0 = m0_of(i);
             (void)mat;
             const uint32_t acc = pc & 1;
-            float* mG = meta + acc * 256;
+            // per slot of the item, the factor of each accumulator column:
+            // G * gate (up) tensor scale, or G * down tensor scale * routing weight
+            float* mA = meta + acc * 256;
+            float* mB = mA + 128;
             if (et < nrow) {
-                mG[et] = nG;
-                if (KIND == G_DOWN) mG[128 + et] = nW;
+                mA[et] = KIND == G_DOWN ? nG * nts0 * nW : nG * nts0;
+                if (KIND == G_GATEUP) mB[et] = nG * nts1;
             }
-            const float ts0 = nts0, ts1 = nts1;
             const bool more = i + gridDim.x < n_items;
             if (more) fetch(nxt, nG, nW, nts0, nts1);
-            named_bar_sync(2, 128);
+            named_bar_sync(2, 256);
             if (!dead) dead = !mbar_wait(&tfull[acc], (pc >> 1) & 1, abort_flag, kW4WaitLimit);
             dead = __any_sync(0xffffffffu, dead);
             if (!dead) {
@@ -413,7 +419,7 @@ __global__ void __launch_bounds__(kW4Threads, 1) k_w4a4(const __grid_constant__ 
                 const uint32_t taddr = tmem_base + ((uint32_t)(32 * sub) << 16) + acc * 128;
                 const bool hi = lane >= 16;
                 const int row = KIND == G_GATEUP ? m0 + 16 * sub + (lane & 15) : m0 + 32 * sub + lane;
-                for (int c0 = 0; c0 < nrow; c0 += 16) {
+                for (int c0 = 16 * half; c0 < nrow; c0 += 32) {
                     uint32_t v[16];
                     __syncwarp();
                     tld_x16(taddr + c0, v);
@@ -427,8 +433,7 @@ __global__ void __launch_bounds__(kW4Threads, 1) k_w4a4(const __grid_constant__ 
                             const float other = __shfl_xor_sync(0xffffffffu, __uint_as_float(hi ? v[u] : v[u + 8]), 16);
                             const int s = c0 + u + (hi ? 8 : 0);
                             if (s < nrow) {
-                                const float g = mG[s];
-                                const float gv = (hi ? other : mine) * g * ts0, uv = (hi ? mine : other) * g * ts1;
+                                const float gv = (hi ? other : mine) * mA[s], uv = (hi ? mine : other) * mB[s];
                                 p.zperm[(size_t)(b0 + s) * p.F + row] = half_checked(silu(gv) * uv, bad);
                             }
                         }
@@ -436,10 +441,7 @@ __global__ void __launch_bounds__(kW4Threads, 1) k_w4a4(const __grid_constant__ 
 #pragma unroll
                         for (int u = 0; u < 16; ++u) {
                             const int s = c0 + u;
-                            if (s < nrow) {
-                                const float o = __uint_as_float(v[u]) * mG[s] * ts0 * mG[128 + s];
-                                p.operm[(size_t)(b0 + s) * p.L + row] = half_checked(o, bad);
-                            }
+                            if (s < nrow) p.operm[(size_t)(b0 + s) * p.L + row] = half_checked(__uint_as_float(v[u]) * mA[s], bad);
                         }
                     }
                 }
@@ -457,7 +459,7 @@ __global__ void __launch_bounds__(kW4Threads, 1) k_w4a4(const __grid_constant__ 
     __syncwarp();
     __syncthreads();
     if (*abort_flag && threadIdx.x == 0) set_status(p.ctrl, LMOE_ERR_TIMEOUT);
-    if (warp == 8) {
+    if (warp == kW4MmaWarp) {
         tc_fence_after();
         __syncwarp();
         tmem_dealloc(tmem_base, kW4TmemCols);
