@@ -536,7 +536,7 @@ __device__ __forceinline__ void epilogue_chunk(const PrefillParams& p, const Til
 // the GEMM kernel
 // ---------------------------------------------------------------------------
 
-template <int NT, int STAGES, int RS, int MA = 1>
+template <int NT, int STAGES, int RS, int MA = 1, bool TR = true>
 struct SmemPlan {
     static constexpr int kA = MA * 128 * 128;            // bytes per A stage (MA x 128 rows x 64 x 16-bit)
     static constexpr int kB = NT * 128;                  // bytes per B stage
@@ -547,7 +547,7 @@ struct SmemPlan {
     static constexpr int kRaw = 256 * 48;
     // gate/up exchange (32 x 64 fp32) or a tile's routing metadata (NT x (1 + 16) words)
     static constexpr int kXchg = (32 * 64 * 4 > NT * 4 * 17) ? 32 * 64 * 4 : NT * 4 * 17;
-    static constexpr int kTr = 4 * 32 * kTrPitch * 2;     // the epilogue warps' transpose buffers
+    static constexpr int kTr = TR ? 4 * 32 * kTrPitch * 2 : 0;   // the epilogue warps' transpose buffers (D, down)
     static constexpr int kBars = (2 * STAGES + 5) * 8;
     static constexpr int kTotal = 1024 /*alignment slack*/ + STAGES * (kA + kB) + RS * kRaw + kXchg + kTr + kBars + 16;
 };
@@ -559,7 +559,7 @@ constexpr int kGemmThreads = 448;  // 4 epilogue, 8 converter, 1 MMA, 1 loader w
 template <int KIND, int NT, int STAGES, int RS, int MA = 1>
 __global__ void __launch_bounds__(kGemmThreads, 1) k_umma_gemm(const __grid_constant__ TmaMaps maps, const PrefillParams p) {
     using S = Sched<KIND, NT, MA>;
-    using Plan = SmemPlan<NT, STAGES, RS, MA>;
+    using Plan = SmemPlan<NT, STAGES, RS, MA, KIND == G_DPROJ || KIND == G_DOWN>;
     extern __shared__ uint8_t smem_raw[];
     // aligned by pointer arithmetic on the shared array, so that the compiler
     // still knows every access through it is a shared-memory access
@@ -1141,7 +1141,7 @@ static int g_num_sms = 0;
 
 template <int KIND, int NT, int STAGES, int RS, int MA = 1>
 static cudaError_t launch_gemm(const TmaMaps& maps, const PrefillParams& p, cudaStream_t st, int max_tiles) {
-    const size_t smem = SmemPlan<NT, STAGES, RS, MA>::kTotal;
+    const size_t smem = SmemPlan<NT, STAGES, RS, MA, KIND == G_DPROJ || KIND == G_DOWN>::kTotal;
     auto kern = k_umma_gemm<KIND, NT, STAGES, RS, MA>;
     cudaError_t e = ensure_smem(reinterpret_cast<const void*>(kern), smem);
     if (e != cudaSuccess) return e;
