@@ -173,16 +173,19 @@ def step_cost(shape, idx: np.ndarray, groups: np.ndarray, T: int, prefill: bool)
 # When the sources have changed since the capture, or the kernel has no
 # capture, its traffic is reported as null.
 NCU_TRAFFIC = {
-    ("edge0_145b_decode", 4, "k_router_shared"): (9282560, "eb4da6755108"),
-    ("edge0_145b_decode", 4, "k_wstream_dproj"): (39070720, "eb4da6755108"),
-    ("edge0_145b_decode", 4, "k_wstream_gateup"): (42732544, "eb4da6755108"),
-    ("edge0_145b_decode", 4, "k_wstream_down"): (21392128, "eb4da6755108"),
-    ("edge0_145b_decode", 4, "k_wstream_uproj"): (43962112, "eb4da6755108"),
-    ("edge0_145b_prefill", 4096, "gateup"): (849587370, "eb4da6755108"),
-    ("edge0_145b_prefill", 4096, "uproj"): (447073280, "eb4da6755108"),
-    ("edge0_145b_prefill+w4a4", 4096, "uproj"): (446979754, "eb4da6755108"),
-    ("edge0_145b_prefill+w4a4", 4096, "gateup"): (745645568, "eb4da6755108"),
-    ("edge0_145b_prefill+w4a4", 4096, "down"): (464022442, "eb4da6755108"),
+    ("edge0_145b_decode", 4, "k_router_shared"): (9282560, "17e6b887e063"),
+    ("edge0_145b_decode", 4, "k_wstream_dproj"): (39070464, "17e6b887e063"),
+    ("edge0_145b_decode", 4, "k_wstream_gateup"): (42732288, "17e6b887e063"),
+    ("edge0_145b_decode", 4, "k_wstream_down"): (21392128, "17e6b887e063"),
+    ("edge0_145b_decode", 4, "k_wstream_uproj"): (43961344, "17e6b887e063"),
+    ("edge0_145b_prefill", 4096, "gateup"): (849031253, "17e6b887e063"),
+    ("edge0_145b_prefill", 4096, "down"): (502160469, "17e6b887e063"),
+    ("edge0_145b_prefill", 4096, "dproj"): (158619733, "17e6b887e063"),
+    ("edge0_145b_prefill", 4096, "uproj"): (265818368, "17e6b887e063"),
+    ("edge0_145b_prefill+w4a4", 4096, "uproj"): (265783978, "17e6b887e063"),
+    ("edge0_145b_prefill+w4a4", 4096, "dproj"): (158699264, "17e6b887e063"),
+    ("edge0_145b_prefill+w4a4", 4096, "gateup"): (742930005, "17e6b887e063"),
+    ("edge0_145b_prefill+w4a4", 4096, "down"): (463891200, "17e6b887e063"),
 }
 
 
