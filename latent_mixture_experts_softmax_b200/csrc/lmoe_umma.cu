@@ -2,18 +2,21 @@
 // the 5th-generation tensor cores (tcgen05.mma, fp32 accumulators in TMEM)
 // in one warp-specialised, persistent GEMM kernel template:
 //
-//   warps 0-3  epilogue: TMEM -> registers -> fused epilogue -> global
-//   warps 4-7  producers: TMA for the activation operand; the weight operand
-//              is read from its storage format (Q8_0, Q4_0, NVFP4, bf16),
-//              dequantised in registers and written to shared memory in the
-//              UMMA K-major 128-byte-swizzled layout
-//   warp 8     TMEM allocation and the single-thread UMMA issue
+//   warps 0-3   epilogue: TMEM -> registers -> fused epilogue -> global
+//   warps 4-11  converters: the weight operand is read from its storage
+//               format (Q8_0, Q4_0, NVFP4, Q3_K / IQ4_NL), dequantised in
+//               registers and written to shared memory in the UMMA K-major
+//               128-byte-swizzled layout
+//   warp 12     TMEM allocation and the single-thread UMMA issue
+//   warp 13     TMA of the activation operand (and of bf16 weights)
 //
 // Operands are swapped with respect to the usual "tokens x weights" view:
 // the weight rows are the MMA's M = 128 side and the tokens (or expert
 // slots) are its N side, so one dequantised weight tile feeds up to 256
-// tokens.  Every accumulator is fp32 in TMEM, double-buffered so the
-// epilogue of one tile overlaps the main loop of the next.
+// tokens; the NVFP4 expert GEMMs take two 128-row weight tiles per item
+// against each activation stage.  Every accumulator is fp32 in TMEM,
+// double-buffered so the epilogue of one tile overlaps the main loop of the
+// next.
 //
 // GEMMs of the block (teardown article "Edge0-145B: a Qwen MoE with its
 // experts squeezed", section "A latent in front of the experts"; Edge0
