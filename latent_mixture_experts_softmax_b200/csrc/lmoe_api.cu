@@ -60,7 +60,7 @@ struct WsLayout {
     // tensor-core path
     size_t p_zero_begin, p_tgmask, p_cnt, p_fill, p_dhit, p_n_etiles, p_zero_end;
     size_t p_n_unique, p_off, p_uexp, p_ucnt, p_uoff, p_etile, p_slot_pair, p_wslot, p_pair_slot, p_idx, p_w, p_logits;
-    size_t p_xh, p_xr, p_xr_lo, p_hperm, p_zperm, p_operm, p_s, p_zsh, p_aq, p_asf, p_aG;
+    size_t p_xh, p_xr, p_xr_lo, p_hperm, p_zperm, p_operm, p_s, p_zsh, p_aq, p_asf, p_aG, p_upart;
     size_t total;
 };
 
@@ -145,6 +145,7 @@ WsLayout ws_layout(const lmoe_cfg& c, int T) {
         L.p_operm = take(TK * c.latent * 2);
         L.p_s = take((size_t)T * c.n_groups * c.latent * 2);
         L.p_zsh = take((size_t)2 * T * c.shared_ffn * 2);
+        L.p_upart = take((size_t)kMaxUPieces * kNtDense * 128 * 4);   // U's split pieces
         if (c.act_fmt == LMOE_ACT_NVFP4) {
             const size_t Kmax = std::max(c.latent, c.ffn);
             L.p_aq = take(TK * Kmax / 2);
@@ -269,6 +270,7 @@ int run_prefill(const lmoe_cfg& c, const FwdParams& f, const WsLayout& L, void* 
     p.operm = reinterpret_cast<__half*>(b + L.p_operm);
     p.s = reinterpret_cast<__half*>(b + L.p_s);
     p.zsh = reinterpret_cast<uint16_t*>(b + L.p_zsh);
+    p.upart = reinterpret_cast<float*>(b + L.p_upart);
     if (f.act == LMOE_ACT_NVFP4) {
         p.aq = reinterpret_cast<uint8_t*>(b + L.p_aq);
         p.asf = reinterpret_cast<uint32_t*>(b + L.p_asf);

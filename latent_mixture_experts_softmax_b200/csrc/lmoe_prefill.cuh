@@ -12,6 +12,8 @@ enum GemmKind { G_ROUTER = 0, G_SHARED_GATEUP = 1, G_DPROJ = 2, G_GATEUP = 3, G_
 
 constexpr int kNtDense = 256;    // tokens per tile of the dense GEMMs (router, shared, D, U)
 constexpr int kNtExpert = 128;   // expert slots per tile of the expert GEMMs
+constexpr int kMaxUParts = 11;   // pieces of a split U tile (K segments: groups, then shared hi / lo)
+constexpr int kMaxUPieces = 160; // split U pieces per step (bounds the partial-sum workspace)
 
 struct __align__(64) TmaMaps {
     CUtensorMap a;    // weight operand (bf16 kinds)
@@ -62,6 +64,13 @@ struct PrefillParams {
     int32_t* uoff;
     int4* etile;         // expert token tiles {expert, first slot, slots (<= 128), distinct index}
     int32_t* slot_pair;  // [T*K]
+    // U's last, partial wave of tiles runs split by K segments so that every
+    // SM gets a share: tiles [u_whole, n) as u_parts pieces, piece p taking
+    // segments [u_segb[p], u_segb[p + 1]); their fp32 partial sums go to
+    // upart [piece][kNtDense tokens][128 rows] and k_u_reduce adds them up
+    int u_whole, u_parts;
+    int u_segb[kMaxUParts + 1];
+    float* upart;
     float* wslot;        // [T*K] routing weight of each expert slot
     int32_t* pair_slot;  // [T*K]
     __half* xh;          // [T][H]   fp16 block input

@@ -54,6 +54,8 @@ struct TileRef {
     int n;        // valid B rows
     int nq;       // token tile index (UPROJ / DPROJ hit flags)
     int na;       // 128-row A tiles of the item (2 in the two-tile expert GEMMs, else 1)
+    int piece;    // U: -1 for a whole tile, else the piece of a split tile (its segment range)
+    int part;     // U: the piece's segment range
 };
 
 // MA = 2 (expert GEMMs only): an item covers two 128-row A tiles that share
@@ -75,14 +77,24 @@ struct Sched {
     }
     __device__ static int num_tiles(const PrefillParams& p) {
         if (KIND == G_GATEUP || KIND == G_DOWN) return m_tiles(p) * __ldcg(p.n_etiles);
-        return m_tiles(p) * ((p.T + NT - 1) / NT);
+        const int n = m_tiles(p) * ((p.T + NT - 1) / NT);
+        if (KIND == G_UPROJ && p.u_parts > 1) return p.u_whole + (n - p.u_whole) * p.u_parts;
+        return n;
     }
-    __device__ static TileRef get(const PrefillParams& p, int i) {
+    __device__ static TileRef get(const PrefillParams& p, int i) {   // i: the work item
         TileRef t;
         const int mt = m_tiles(p);
         t.valid = 1;
         t.mat = 0;
         t.na = 1;
+        t.piece = -1;
+        t.part = -1;
+        if (KIND == G_UPROJ && p.u_parts > 1 && i >= p.u_whole) {
+            // a piece of a tile of the last wave
+            t.piece = i - p.u_whole;
+            t.part = t.piece % p.u_parts;
+            i = p.u_whole + t.piece / p.u_parts;
+        }
         if (KIND == G_GATEUP || KIND == G_DOWN) {
             // consecutive tiles share the expert's token rows
             const int et = i / mt, m = i % mt;
@@ -129,8 +141,9 @@ struct Sched {
         return 1;
     }
     __device__ static bool seg_active(const PrefillParams& p, const TileRef& t, int seg) {
-        if (KIND != G_UPROJ || seg >= p.G) return true;
-        return p.dhit[t.nq * p.G + seg] != 0;
+        if (KIND != G_UPROJ) return true;
+        if (t.part >= 0 && (seg < p.u_segb[t.part] || seg >= p.u_segb[t.part + 1])) return false;
+        return seg >= p.G || p.dhit[t.nq * p.G + seg] != 0;
     }
     __device__ static int seg_k(const PrefillParams& p, int seg) {
         switch (KIND) {
@@ -523,6 +536,12 @@ __device__ __forceinline__ void epilogue_chunk(const PrefillParams& p, const Til
         }
         __syncwarp();
         report_range(p.ctrl, bad);
+    } else if (t.piece >= 0) {
+        // UPROJ, a piece of a split tile: its fp32 partial sum, [piece][token][row]
+        float* dst = p.upart + ((size_t)t.piece * kNtDense + c0) * 128 + row;
+#pragma unroll
+        for (int j = 0; j < 32; ++j)
+            if (j < ncol) dst[(size_t)j * 128] = u2f(r[j]);
     } else {  // UPROJ
         const int hrow = t.m0 + row;
         float res[32];
@@ -1045,6 +1064,29 @@ __global__ void k_bucket_scatter(const PrefillParams p) {
     p.wslot[slot] = p.w[i];
 }
 
+// U's split tiles: y = bf16(sum of the pieces' partial sums, in piece order,
+// + residual).  A piece none of whose segments is active (no token of the
+// tile hits its groups) was skipped by the GEMM and adds nothing.  One CTA
+// per (split tile, token), a thread per row.
+__global__ void k_u_reduce(const PrefillParams p) {
+    const int tt = blockIdx.x, c = blockIdx.y, r = threadIdx.x;
+    const int mt = p.H / 128;
+    const int ti = p.u_whole + tt;                    // token-tile-major, as the GEMM's items
+    const int m = ti % mt, q = ti / mt;
+    const int tok = q * kNtDense + c;
+    if (tok >= p.T) return;
+    float acc = 0.f;
+    for (int part = 0; part < p.u_parts; ++part) {
+        bool active = false;
+        for (int seg = p.u_segb[part]; seg < p.u_segb[part + 1]; ++seg)
+            active |= seg >= p.G || p.dhit[q * p.G + seg] != 0;
+        if (active) acc += __ldcg(p.upart + ((size_t)(tt * p.u_parts + part) * kNtDense + c) * 128 + r);
+    }
+    const int h = m * 128 + r;
+    if (p.residual) acc += bf16_bits_to_f32(__ldg(p.residual + (size_t)tok * p.H + h));
+    p.y[(size_t)tok * p.H + h] = f32_to_bf16_bits(acc);
+}
+
 // s[t][g] = sum over the token's experts of group g of o (already weighted);
 // zero for groups the token does not hit.  One CTA per token, 16 bytes per thread.
 __global__ void k_combine(const PrefillParams p) {
@@ -1158,6 +1200,34 @@ static cudaError_t launch_gemm(const TmaMaps& maps, const PrefillParams& p, cuda
     return cudaGetLastError();
 }
 
+// U's split plan: the tiles of the last wave (n_u mod sms of them, if the
+// wave is partial) become u_parts pieces each, contiguous segment ranges of
+// about equal stage counts (a group segment is L / 64 stages, each shared
+// segment Fs / 64); at most kMaxUParts pieces a tile and kMaxUPieces in all.
+static void u_split_plan(PrefillParams& p, int n_u, int sms) {
+    p.u_whole = n_u;
+    p.u_parts = 1;
+    const int nseg = p.G + 2;
+    const int tail = n_u % sms;
+    if (tail == 0 || p.upart == nullptr) return;
+    const int parts = std::min(std::min(nseg, kMaxUParts), std::min(sms / tail, kMaxUPieces / tail));
+    if (parts < 2) return;
+    long total = 0;
+    for (int sg = 0; sg < nseg; ++sg) total += sg < p.G ? p.L / 64 : p.Fs / 64;
+    p.u_segb[0] = 0;
+    long acc = 0;
+    int b = 1;
+    for (int sg = 0; sg < nseg && b < parts; ++sg) {
+        acc += sg < p.G ? p.L / 64 : p.Fs / 64;
+        // close piece b - 1 once it holds its share, leaving a segment for each later piece
+        if (acc * parts >= total * b && nseg - (sg + 1) >= parts - b) p.u_segb[b++] = sg + 1;
+    }
+    if (b < parts) return;                            // fewer natural cuts than pieces: keep whole tiles
+    p.u_segb[parts] = nseg;
+    p.u_whole = n_u - tail;
+    p.u_parts = parts;
+}
+
 cudaError_t run_prefill_path(PrefillParams p, cudaStream_t st, void* memset_base, size_t memset_bytes,
                              void (*mark)(cudaStream_t)) {
     const int T = p.T, H = p.H, L = p.L, G = p.G, F = p.F, Fs = p.Fs, K = p.K, E = p.E;
@@ -1234,7 +1304,23 @@ cudaError_t run_prefill_path(PrefillParams p, cudaStream_t st, void* memset_base
     k_combine<<<T, 256, 0, st>>>(p);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
     mark(st);
-    if ((e = launch_gemm<G_UPROJ, kNtDense, 4, 0>(m_u, p, st, (H / 128) * ttiles)) != cudaSuccess) return e;
+    {
+        // the last, partial wave of U tiles runs split into pieces by K
+        // segment, so that every SM gets a share of it
+        if (g_num_sms == 0) {
+            int dev = 0;
+            cudaGetDevice(&dev);
+            cudaDeviceGetAttribute(&g_num_sms, cudaDevAttrMultiProcessorCount, dev);
+        }
+        const int n_u = (H / 128) * ttiles;
+        u_split_plan(p, n_u, g_num_sms);
+        const int items = p.u_whole + (n_u - p.u_whole) * p.u_parts;
+        if ((e = launch_gemm<G_UPROJ, kNtDense, 4, 0>(m_u, p, st, items)) != cudaSuccess) return e;
+        if (p.u_parts > 1) {
+            k_u_reduce<<<dim3(n_u - p.u_whole, kNtDense), 128, 0, st>>>(p);
+            if ((e = cudaGetLastError()) != cudaSuccess) return e;
+        }
+    }
     mark(st);
     return cudaSuccess;
 }
